@@ -1,0 +1,190 @@
+/*
+ * infllmv2.h -- C ABI of libinfllmv2.so: the InfLLM v2 sparse-attention path on NVIDIA B200 (sm_100a).
+ *
+ * The method (MiniCPM4 pages; cited by page title and section):
+ *   (1) semantic kernels: every KV head's key cache is summarised by "fine-grained semantic kernels",
+ *       here the mean of K over a 32-key window advanced by 16 keys;
+ *   (2) a query token's relevance to a 64-key context block is the max over the block's kernels of the
+ *       query-kernel score; the query heads of one GQA group share one block set; the top-k blocks are
+ *       taken, together with the initial block and the local blocks;
+ *   (3) attention runs over the selected blocks only, causally, for prefill and decode, with dense
+ *       attention for short contexts.
+ *   Sources: "Tsinghua & ModelBest: MiniCPM4 technical details" (QbitAI), section "Model architecture:
+ *   InfLLM v2", items 1) finer semantic kernels, 2) GQA-group query-head sharing, 3) operators and the
+ *   LogSumExp-based top-k; "MiniCPM 4.0 launch article" (senqingzn.com), section 1 "efficient
+ *   architecture" (dense/sparse switch); QbitAI article, section "speculative sampling, quantisation
+ *   and long text", long-context bullet (tree-draft verification with a bit-packed local mask).
+ *
+ * Conventions shared by every entry point
+ *   - All tensor pointers are DEVICE pointers owned by the caller; the library allocates nothing and
+ *     keeps no state between calls.  Every call is asynchronous on `stream` (0 = legacy default stream).
+ *   - bf16 = IEEE bfloat16 (2 bytes).  Layouts are dense row-major (innermost index last):
+ *       q        [B, T, Hq, d]       queries (T query tokens per sequence)
+ *       k, v     [B, Lcap, Hkv, d]   key / value cache, position-major
+ *       kern     [B, Hkv, nk_cap, d] semantic-kernel cache, bf16
+ *       idx      [B, T, Hkv, kmax]   int32 selected block ids, ascending, -1 padded; kmax = topk +
+ *                                    init_blocks + local_blocks
+ *       cnt      [B, T, Hkv]         int32 number of selected blocks
+ *       out      [B, T, Hq, d]       bf16; lse [B, T, Hq] fp32 natural-log softmax denominator (nullable)
+ *     GQA: query head h reads KV head h / (Hq / Hkv).
+ *   - Context of a query: n = the number of cache keys it may see.  q_ctx[b*T + t] gives it; when q_ctx
+ *     is NULL the T queries are the last T tokens of a causal sequence: n = ctx_lens[b] - T + t + 1.
+ *     Kernels visible to the query are the complete windows inside [0, n); its own block is c = (n-1)/64.
+ *   - Dense switch: a query with n <= params.dense_len attends to all keys [0, n).  Its selection row is
+ *     written as cnt = c + 1 with the first min(c + 1, kmax) block ids; attention ignores idx for it.
+ *   - Pointers must be 16-byte aligned; d must be 64 or 128; Hq / Hkv in {1, 2, 4, 8, 16}; the GPU path
+ *     supports block_size 64, kernel_size 32, kernel_stride 16 (other values -> INFLLMV2_ERR_UNSUPPORTED).
+ *   - Errors: every argument is checked on the host before any launch; on a bad argument the call
+ *     returns the status and launches nothing.  A failed launch returns INFLLMV2_ERR_CUDA.  Kernels
+ *     contain no waits on other kernels or devices.
+ *   - Workspace: entry points that take (ws, ws_bytes) need at least infllmv2_workspace_size(...) bytes
+ *     of device memory, 256-byte aligned, owned by the caller; calls that run concurrently need separate
+ *     workspaces.  Its contents need no initialisation and are scratch after the call.
+ */
+#ifndef INFLLMV2_H
+#define INFLLMV2_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st* infllmv2_stream_t; /* same type as cudaStream_t */
+
+typedef enum {
+    INFLLMV2_OK = 0,
+    INFLLMV2_ERR_INVALID_ARG = 1, /* null/misaligned pointer, negative or inconsistent size */
+    INFLLMV2_ERR_UNSUPPORTED = 2, /* valid but outside what the GPU kernels implement */
+    INFLLMV2_ERR_WORKSPACE = 3,   /* workspace missing, misaligned or too small */
+    INFLLMV2_ERR_CUDA = 4,        /* a CUDA launch failed (cudaGetLastError after the launch) */
+    INFLLMV2_ERR_TIMEOUT = 5      /* reserved: no kernel of this library waits */
+} infllmv2_status;
+
+/* Method constants (the pages give none; the workloads use 64 / 32 / 16, k = 8 or 64, 1 + 2 forced). */
+typedef struct {
+    int block_size;      /* keys per context block (GPU: 64) */
+    int kernel_size;     /* keys per semantic-kernel window (GPU: 32) */
+    int kernel_stride;   /* stride between windows (GPU: 16) */
+    int topk;            /* blocks chosen by score besides the forced ones, >= 0 */
+    int init_blocks;     /* blocks [0, init_blocks) always kept */
+    int local_blocks;    /* the query's own block and the local_blocks-1 before it always kept */
+    int dense_len;       /* queries with context n <= dense_len attend densely */
+    int membership;      /* 0 = OVERLAP: kernel j belongs to every block its window intersects;
+                            1 = CONTAINED: only to the block that contains its whole window */
+    float softmax_scale; /* <= 0 selects 1/sqrt(d); used for kernel scoring and attention */
+} infllmv2_params;
+
+/* Human-readable name of a status code (static storage). */
+const char* infllmv2_status_string(int status);
+
+/* Library version, as major*10000 + minor*100 + patch. */
+int infllmv2_version(void);
+
+/*
+ * Bytes of workspace the calls below need for problems up to the given sizes (host-only, no CUDA call).
+ *   max_q   : largest T (queries per sequence) of any call
+ *   max_ctx : largest context length n of any query
+ * Returns 0 when the arguments are invalid.
+ */
+size_t infllmv2_workspace_size(const infllmv2_params* params, int batch, int max_q, int max_ctx, int hq, int hkv,
+                               int head_dim);
+
+/*
+ * Step 1 -- semantic kernels (MiniCPM4 technical details, "Model architecture: InfLLM v2", item 1).
+ * For each sequence b, writes the kernels completed between old_lens[b] and new_lens[b] keys:
+ *   kern[b, g, j, :] = bf16_round_nearest_even( mean_{i in [16 j, 16 j + 32)} k[b, i, g, :] )
+ * for j in [nk(old), nk(new)), nk(n) = n >= 32 ? (n - 32) / 16 + 1 : 0.  Sums are fp32.
+ *   k            [B, Lcap, Hkv, d] bf16 (device)
+ *   old_lens,
+ *   new_lens     [B] int32 (device), 0 <= old <= new <= Lcap; device-side values are trusted
+ *   max_new_keys host upper bound of new_lens[b] - old_lens[b] over b (sizes the grid; 1 for a decode
+ *                step, the prompt length for a prefill)
+ *   kern         [B, Hkv, nk_cap, d] bf16 (device); requires nk(new_lens[b]) <= nk_cap
+ */
+int infllmv2_kernel_pool(const void* k, int batch, int lcap, int hkv, int head_dim, const int32_t* old_lens,
+                         const int32_t* new_lens, int max_new_keys, const infllmv2_params* params, void* kern,
+                         int nk_cap, infllmv2_stream_t stream);
+
+/*
+ * Step 2 -- block scoring and top-k selection (same section, items 1-3).
+ * For each query (b, t) and KV group g, with kernel scores z_h(j) = scale * q_h . kern_j over the visible
+ * kernels and LSE_h = log sum_j exp z_h(j) (exact), the group score of block blk is
+ *   S_g(blk) = sum_{h in g} max_{j in blk, visible} exp(z_h(j) - LSE_h)
+ * (kernel j is in blk per params.membership).  Forced blocks [0, init) and [c - local + 1, c] are kept;
+ * of the other blocks with a visible kernel, the topk with the largest S are taken (ties -> lower id).
+ * The union is written ascending to idx[b, t, g, :], padded with -1, its size to cnt[b, t, g].
+ *   q          [B, T, Hq, d] bf16 (device)
+ *   q_ctx      [B * T] int32 (device) or NULL (then the T queries end the sequence: see above)
+ *   ctx_lens   [B] int32 (device); required when q_ctx is NULL, else ignored (may be NULL)
+ *   max_ctx    host upper bound of every query's n (sizes the grid and the workspace)
+ *   kern       [B, Hkv, nk_cap, d] bf16 (device), valid for every kernel visible to the queries
+ *   idx, cnt   outputs as described; kmax = topk + init_blocks + local_blocks
+ *   ws         workspace of ws_bytes >= infllmv2_workspace_size(params, B, T, max_ctx, Hq, Hkv, d)
+ */
+int infllmv2_block_score_topk(const void* q, int batch, int num_q, int hq, int hkv, int head_dim,
+                              const int32_t* q_ctx, const int32_t* ctx_lens, int max_ctx, const void* kern,
+                              int nk_cap, const infllmv2_params* params, int32_t* idx, int32_t* cnt, void* ws,
+                              size_t ws_bytes, infllmv2_stream_t stream);
+
+/*
+ * Step 3a -- block-sparse attention of T query tokens per sequence (prefill / chunked prefill)
+ * (MiniCPM4 technical details, InfLLM v2 overview: only the selected blocks take part in attention).
+ * Query (b, t), head h, group g = h / (Hq/Hkv), context n:
+ *   keys = [0, n) if n <= dense_len, else the union over blk in idx[b, t, g, :cnt] of [64 blk, min(64 blk + 64, n))
+ *   out[b, t, h, :] = sum_{i in keys} softmax_i(scale * q . k_i) v_i ; lse = log sum_i exp(scale * q . k_i)
+ * Block ids must be ascending, unique, >= 0 and have 64 blk < n (checked on the device: an invalid id is
+ * skipped).  k, v: [B, Lcap, Hkv, d] bf16.  lse may be NULL.  ws as for block_score_topk.
+ */
+int infllmv2_sparse_attn_prefill(const void* q, int batch, int num_q, int hq, int hkv, int head_dim, const void* k,
+                                 const void* v, int lcap, const int32_t* q_ctx, const int32_t* ctx_lens,
+                                 int max_ctx, const int32_t* idx, const int32_t* cnt,
+                                 const infllmv2_params* params, void* out, float* lse, void* ws, size_t ws_bytes,
+                                 infllmv2_stream_t stream);
+
+/*
+ * Step 3b -- block-sparse attention of one new token per sequence (decode; MiniCPM4 technical details,
+ * efficiency evaluation: the number of blocks read stays constant as the context grows).  Same formula
+ * as 3a with T = 1 and n = ctx_lens[b] (the new token's key and value are already in the cache).
+ * Split over the selected blocks across CTAs, partial results merged by their LSE in the workspace.
+ *   q [B, 1, Hq, d]; out [B, 1, Hq, d]; lse [B, Hq] or NULL.
+ */
+int infllmv2_sparse_attn_decode(const void* q, int batch, int hq, int hkv, int head_dim, const void* k,
+                                const void* v, int lcap, const int32_t* ctx_lens, int max_ctx, const int32_t* idx,
+                                const int32_t* cnt, const infllmv2_params* params, void* out, float* lse, void* ws,
+                                size_t ws_bytes, infllmv2_stream_t stream);
+
+/*
+ * Step 3c -- tree-draft verification (QbitAI article, "speculative sampling, quantisation and long text",
+ * long-context bullet).  n_draft draft tokens per sequence, each a query that sees the whole prefix of
+ * prefix_lens[b] cache keys through its own selected blocks (its q_ctx is the prefix length), plus the
+ * draft tokens j whose bit j is set in tree_mask[b * n_draft + i] (its ancestors and itself):
+ *   keys(i) = prefix keys of idx[b, i, g, :cnt] (clipped to the prefix, or all of it when
+ *             prefix <= dense_len)  U  { draft j : bit j of tree_mask[b, i] }
+ *   q [B, n_draft, Hq, d]; k_draft, v_draft [B, n_draft, Hkv, d] bf16; tree_mask [B, n_draft] uint32;
+ *   n_draft <= 32; out [B, n_draft, Hq, d]; lse [B, n_draft, Hq] or NULL.
+ */
+int infllmv2_sparse_attn_tree_verify(const void* q, int batch, int n_draft, int hq, int hkv, int head_dim,
+                                     const void* k, const void* v, int lcap, const int32_t* prefix_lens, int max_ctx,
+                                     const void* k_draft, const void* v_draft, const uint32_t* tree_mask,
+                                     const int32_t* idx, const int32_t* cnt, const infllmv2_params* params,
+                                     void* out, float* lse, void* ws, size_t ws_bytes, infllmv2_stream_t stream);
+
+/*
+ * Dense path (MiniCPM 4.0 launch article, section 1: short texts keep dense attention).  Plain causal GQA
+ * attention over keys [0, n) for every query, whatever dense_len is; same layouts and n rules as 3a / 3b.
+ */
+int infllmv2_dense_attn_prefill(const void* q, int batch, int num_q, int hq, int hkv, int head_dim, const void* k,
+                                const void* v, int lcap, const int32_t* q_ctx, const int32_t* ctx_lens, int max_ctx,
+                                float softmax_scale, void* out, float* lse, void* ws, size_t ws_bytes,
+                                infllmv2_stream_t stream);
+int infllmv2_dense_attn_decode(const void* q, int batch, int hq, int hkv, int head_dim, const void* k, const void* v,
+                               int lcap, const int32_t* ctx_lens, int max_ctx, float softmax_scale, void* out,
+                               float* lse, void* ws, size_t ws_bytes, infllmv2_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* INFLLMV2_H */

@@ -1,0 +1,123 @@
+"""The C-ABI library: it loads, exports every symbol include/infllmv2.h declares, and rejects bad
+arguments on the host with the documented status before launching anything (no GPU needed: every call
+here fails validation, so no CUDA work is enqueued)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from trainable_block_sparse_v2_b200 import binding
+from trainable_block_sparse_v2_b200.build import build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "infllmv2.h")
+
+OK, INVALID, UNSUPPORTED, WORKSPACE = 0, 1, 2, 3
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build()
+    return binding.load()
+
+
+def declared_functions():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(infllmv2_[a-z_0-9]+)\s*\(", src)))
+
+
+def test_header_declares_the_entry_points():
+    names = declared_functions()
+    for n in ["infllmv2_kernel_pool", "infllmv2_block_score_topk", "infllmv2_sparse_attn_prefill",
+              "infllmv2_sparse_attn_decode", "infllmv2_sparse_attn_tree_verify", "infllmv2_dense_attn_prefill",
+              "infllmv2_dense_attn_decode", "infllmv2_workspace_size", "infllmv2_status_string"]:
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for name in declared_functions():
+        assert hasattr(lib, name), name
+    assert set(binding.EXPORTED) >= set(declared_functions())
+
+
+def test_status_strings_and_version(lib):
+    assert binding.infllmv2_status_string(0) == "ok"
+    assert "workspace" in binding.infllmv2_status_string(3)
+    assert binding.infllmv2_version() >= 100
+
+
+def test_workspace_size_host_only(lib):
+    p = binding.Params(topk=64, dense_len=8192)
+    n = binding.infllmv2_workspace_size(p, 4, 1, 131072 + 256, 32, 2, 128)
+    assert n > 0 and n % 256 == 0
+    assert binding.infllmv2_workspace_size(p, 4, 1, 131072, 32, 2, 128) <= n
+    assert binding.infllmv2_workspace_size(p, 4, 1, 131072, 32, 3, 128) == 0      # Hq % Hkv != 0
+    assert binding.infllmv2_workspace_size(p, 4, 1, 131072, 32, 2, 96) == 0       # unsupported d
+    assert binding.infllmv2_workspace_size(p, 4, 1, 0, 32, 2, 128) == 0           # empty context
+    bad = binding.Params(block_size=32)
+    assert binding.infllmv2_workspace_size(bad, 1, 1, 1000, 32, 2, 128) == 0
+
+
+# fake device pointers: aligned, never dereferenced because validation fails first
+A16 = 0x10000
+A16B = 0x20000
+A4 = 0x30000
+WS = 0x40000
+
+
+def _score(lib, p, **kw):
+    args = dict(q=A16, batch=1, num_q=1, hq=32, hkv=2, d=128, q_ctx=None, ctx_lens=A4, max_ctx=4096, kern=A16B,
+                nk_cap=255, idx=A4, cnt=A4, ws=WS, ws_bytes=1 << 30)
+    args.update(kw)
+    cp = p.c()
+    return lib.infllmv2_block_score_topk(args["q"], args["batch"], args["num_q"], args["hq"], args["hkv"], args["d"],
+                                         args["q_ctx"], args["ctx_lens"], args["max_ctx"], args["kern"],
+                                         args["nk_cap"], ctypes.byref(cp), args["idx"], args["cnt"], args["ws"],
+                                         args["ws_bytes"], None)
+
+
+def test_block_score_topk_rejects_bad_arguments(lib):
+    p = binding.Params(topk=8)
+    assert _score(lib, p, q=None) == INVALID
+    assert _score(lib, p, q=A16 + 2) == INVALID                  # misaligned
+    assert _score(lib, p, hkv=3) == INVALID                      # Hq % Hkv
+    assert _score(lib, p, hq=6, hkv=2) == UNSUPPORTED            # group of 3
+    assert _score(lib, p, d=96) == UNSUPPORTED
+    assert _score(lib, p, q_ctx=None, ctx_lens=None) == INVALID
+    assert _score(lib, p, max_ctx=0) == INVALID
+    assert _score(lib, p, nk_cap=10) == INVALID                  # kernel cache too small for max_ctx
+    assert _score(lib, p, max_ctx=300000, nk_cap=20000) == UNSUPPORTED
+    assert _score(lib, p, ws=None) == WORKSPACE                  # few-row path needs workspace
+    assert _score(lib, p, ws_bytes=16) == WORKSPACE
+    assert _score(lib, p, ws=WS + 16) == WORKSPACE               # workspace not 256-aligned
+    assert _score(lib, binding.Params(block_size=128)) == UNSUPPORTED
+    assert _score(lib, binding.Params(topk=-1)) == INVALID
+    assert _score(lib, binding.Params(membership=2)) == INVALID
+    assert _score(lib, binding.Params(topk=0, init_blocks=0, local_blocks=0)) == INVALID
+
+
+def test_attention_entry_points_reject_bad_arguments(lib):
+    p = binding.Params(topk=64, dense_len=8192)
+    cp = p.c()
+    # decode: lcap smaller than max_ctx
+    assert lib.infllmv2_sparse_attn_decode(A16, 1, 32, 2, 128, A16, A16, 1000, A4, 2000, A4, A4, ctypes.byref(cp),
+                                           A16, None, WS, 1 << 30, None) == INVALID
+    # decode: workspace too small
+    assert lib.infllmv2_sparse_attn_decode(A16, 1, 32, 2, 128, A16, A16, 4096, A4, 4096, A4, A4, ctypes.byref(cp),
+                                           A16, None, WS, 64, None) == WORKSPACE
+    # tree: more than 32 draft nodes
+    assert lib.infllmv2_sparse_attn_tree_verify(A16, 1, 33, 32, 2, 128, A16, A16, 4096, A4, 4096, A16, A16, A4, A4,
+                                                A4, ctypes.byref(cp), A16, None, WS, 1 << 30, None) == UNSUPPORTED
+    # prefill: null v
+    assert lib.infllmv2_sparse_attn_prefill(A16, 1, 16, 32, 2, 128, A16, None, 4096, None, A4, 4096, A4, A4,
+                                            ctypes.byref(cp), A16, None, None, 0, None) == INVALID
+    # dense: NaN scale
+    assert lib.infllmv2_dense_attn_prefill(A16, 1, 16, 32, 2, 128, A16, A16, 4096, None, A4, 4096,
+                                           ctypes.c_float(float("nan")), A16, None, None, 0, None) == INVALID
+    # kernel pool: unsupported window
+    bad = binding.Params(kernel_size=16).c()
+    assert lib.infllmv2_kernel_pool(A16, 1, 4096, 2, 128, A4, A4, 4096, ctypes.byref(bad), A16, 255, None) == \
+        UNSUPPORTED
+    assert lib.infllmv2_kernel_pool(A16, 1, 4096, 2, 128, A4, A4, 4096, ctypes.byref(cp), A16, 10, None) == INVALID

@@ -1,0 +1,248 @@
+"""GPU parity: every step of the CUDA path, called through the C ABI, against the fp64 CPU oracle on the
+same seeded inputs, at sizes that span several tiles and ragged tails, plus the edge cases (contexts
+shorter than one kernel window, lengths off the 16/64 grid, queries in the first blocks, the dense
+threshold and one past it, mixed lengths, head_dim 64/128, GQA groups 1/2/8/16)."""
+import numpy as np
+import pytest
+import torch
+
+from gpu_util import (bparams, check_attention, check_selection, dev, dev_i32, f64, host_u16, oparams)
+from trainable_block_sparse_v2_b200 import binding
+from trainable_block_sparse_v2_b200.workloads import (decode_case, f32_to_bf16_bits, prefill_case, tree_case)
+
+pytestmark = [pytest.mark.gpu,
+              pytest.mark.skipif(not torch.cuda.is_available(), reason="needs a CUDA GPU")]
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib():
+    from trainable_block_sparse_v2_b200.build import build
+    build()
+    binding.load()
+
+
+def gpu_pool(k_u16, old, new, max_new, nk_cap, kern=None):
+    K = dev(k_u16)
+    B, Lcap, Hkv, d = k_u16.shape
+    if kern is None:
+        kern = torch.zeros((B, Hkv, nk_cap, d), dtype=torch.bfloat16, device="cuda")
+    binding.infllmv2_kernel_pool(K, dev_i32(old), dev_i32(new), max_new, binding.Params(), kern)
+    return kern
+
+
+def gpu_select(w, kern, q_ctx=None, max_ctx=None, params=None):
+    p = bparams(params or w.params)
+    B, T, Hq, d = w.q.shape
+    Hkv = w.k.shape[2]
+    max_ctx = max_ctx or int(w.q_ctx.max())
+    idx = torch.full((B, T, Hkv, p.kmax), -7, dtype=torch.int32, device="cuda")
+    cnt = torch.full((B, T, Hkv), -7, dtype=torch.int32, device="cuda")
+    ws = binding.workspace(p, B, T, max_ctx, Hq, Hkv, d)
+    qc = dev_i32(w.q_ctx if q_ctx is None else q_ctx)
+    binding.infllmv2_block_score_topk(dev(w.q), qc, None, max_ctx, kern, p, idx, cnt, ws)
+    torch.cuda.synchronize()
+    return idx.cpu().numpy(), cnt.cpu().numpy()
+
+
+# ---------------------------------------------------------------------------------------------------
+# step 1: kernel pool
+# ---------------------------------------------------------------------------------------------------
+
+@pytest.mark.parametrize("d", [64, 128])
+def test_kernel_pool_bulk_and_incremental(oracle, d):
+    rng = np.random.default_rng(100 + d)
+    lens = np.array([1000, 777, 31, 32], np.int32)
+    Lcap = 1008
+    K = f32_to_bf16_bits(rng.standard_normal((4, Lcap, 2, d)).astype(np.float32))
+    nk_cap = oracle.num_kernels(1000)
+    want = oracle.kernel_pool(K, [0] * 4, lens, 32, 16, nk_cap=nk_cap)
+    got = host_u16(gpu_pool(K, np.zeros(4), lens, 1000, nk_cap))
+    assert np.array_equal(got, want)
+    # incremental: grow by 1, then by 13, then by 200 keys
+    kern = gpu_pool(K, np.zeros(4), np.array([500, 400, 0, 1]), 500, nk_cap)
+    cur = np.array([500, 400, 0, 1])
+    for step in (1, 13, 200, 1000):
+        new = np.minimum(cur + step, lens)
+        gpu_pool(K, cur, new, step, nk_cap, kern=kern)
+        cur = new
+    assert np.array_equal(host_u16(kern), want)
+
+
+# ---------------------------------------------------------------------------------------------------
+# step 2: scoring + selection
+# ---------------------------------------------------------------------------------------------------
+
+@pytest.mark.parametrize("membership", [0, 1])
+def test_selection_tiny_prefill_tile_path(oracle, membership):
+    """2048-token prefill, 4/2 heads, d 64, top-8 (token-tile path, many tiles, G = 2)."""
+    w = prefill_case(2048, 4, 2, 64, topk=8, dense_len=0, seed=1001, n_needles=3, membership=membership)
+    nk_cap = oracle.num_kernels(2048)
+    kern_o = oracle.kernel_pool(w.k, [0], [2048], 32, 16, nk_cap=nk_cap)
+    kern = gpu_pool(w.k, [0], [2048], 2048, nk_cap)
+    r = oracle.block_score_topk(w.q, kern_o, w.q_ctx, oparams(w.params))
+    gidx, gcnt = gpu_select(w, kern)
+    same = check_selection(gidx, gcnt, r)
+    assert same.mean() > 0.99
+
+
+@pytest.mark.parametrize("G,d", [(16, 128), (8, 64), (1, 128), (2, 64)])
+def test_selection_tile_path_groups(oracle, G, d):
+    """Ragged prefill length, dense rows at the start (dense_len 300), other group sizes."""
+    T = 1337
+    w = prefill_case(T, 2 * G, 2, d, topk=6, dense_len=300, seed=200 + G, n_needles=2)
+    nk_cap = oracle.num_kernels(T)
+    kern_o = oracle.kernel_pool(w.k, [0], [T], 32, 16, nk_cap=nk_cap)
+    kern = gpu_pool(w.k, [0], [T], T, nk_cap)
+    r = oracle.block_score_topk(w.q, kern_o, w.q_ctx, oparams(w.params))
+    gidx, gcnt = gpu_select(w, kern)
+    check_selection(gidx, gcnt, r)
+
+
+@pytest.mark.parametrize("G,d", [(16, 128), (2, 64), (8, 128)])
+def test_selection_decode_scan_path(oracle, G, d):
+    """Decode rows (scan path): ragged lengths, one at the dense threshold, one just past it, one
+    shorter than a kernel window, lengths off the 16/64 grid."""
+    lens = [20000, 8192, 8193, 30, 4500, 65]
+    w = decode_case(lens, 2 * G, 2, d, topk=16, dense_len=8192, seed=300 + G, n_needles=8)
+    nk_cap = oracle.num_kernels(max(lens))
+    kern_o = oracle.kernel_pool(w.k, [0] * 6, lens, 32, 16, nk_cap=nk_cap)
+    kern = gpu_pool(w.k, [0] * 6, lens, max(lens), nk_cap)
+    assert np.array_equal(host_u16(kern), kern_o)
+    r = oracle.block_score_topk(w.q, kern_o, w.q_ctx, oparams(w.params))
+    gidx, gcnt = gpu_select(w, kern)
+    check_selection(gidx, gcnt, r)
+    # needles are found (sanity; sequence 0 is the only sparse row long enough to hold 8 needles)
+    for b in (0,):
+        for g in range(2):
+            assert np.isin(w.extras["needles"][b], gidx[b, 0, g]).mean() >= 0.5
+
+
+def test_selection_explicit_q_ctx_and_early_blocks(oracle):
+    """Queries in block 0 and 1, contexts below one window, explicit per-query context lengths."""
+    rng = np.random.default_rng(400)
+    T = 100
+    w = prefill_case(T, 32, 2, 128, topk=2, dense_len=0, seed=400, n_needles=0)
+    q_ctx = np.sort(rng.integers(1, T + 1, size=(1, T))).astype(np.int32)
+    q_ctx[0, :5] = [1, 2, 31, 32, 33]
+    nk_cap = oracle.num_kernels(T)
+    kern_o = oracle.kernel_pool(w.k, [0], [T], 32, 16, nk_cap=nk_cap)
+    kern = gpu_pool(w.k, [0], [T], T, nk_cap)
+    r = oracle.block_score_topk(w.q, kern_o, q_ctx, oparams(w.params))
+    gidx, gcnt = gpu_select(w, kern, q_ctx=q_ctx, max_ctx=T)
+    check_selection(gidx, gcnt, r)
+
+
+# ---------------------------------------------------------------------------------------------------
+# step 3: attention (fed the oracle's selection, so it is compared on identical block sets)
+# ---------------------------------------------------------------------------------------------------
+
+@pytest.mark.parametrize("G,d,dense_len", [(2, 64, 0), (16, 128, 700), (1, 128, 0), (8, 64, 2000)])
+def test_sparse_prefill_attention(oracle, G, d, dense_len):
+    T = 1500
+    w = prefill_case(T, 2 * G, 2, d, topk=5, dense_len=dense_len, seed=500 + G, n_needles=2)
+    nk_cap = oracle.num_kernels(T)
+    kern_o = oracle.kernel_pool(w.k, [0], [T], 32, 16, nk_cap=nk_cap)
+    P = oparams(w.params)
+    r = oracle.block_score_topk(w.q, kern_o, w.q_ctx, P)
+    out_o, lse_o = oracle.sparse_attention(w.q, w.k, w.v, w.q_ctx, r["idx"], r["cnt"], P)
+    out = torch.empty((1, T, 2 * G, d), dtype=torch.bfloat16, device="cuda")
+    lse = torch.empty((1, T, 2 * G), dtype=torch.float32, device="cuda")
+    binding.infllmv2_sparse_attn_prefill(dev(w.q), dev(w.k), dev(w.v), None, dev_i32(w.ctx_lens), T,
+                                         dev_i32(r["idx"]), dev_i32(r["cnt"]), bparams(w.params), out, lse)
+    torch.cuda.synchronize()
+    check_attention(out, out_o, lse, lse_o, what="prefill")
+
+
+@pytest.mark.parametrize("G,d", [(16, 128), (2, 64)])
+def test_sparse_decode_attention(oracle, G, d):
+    lens = [20000, 8192, 8193, 30, 4500, 65]
+    w = decode_case(lens, 2 * G, 2, d, topk=16, dense_len=8192, seed=600 + G, n_needles=8)
+    nk_cap = oracle.num_kernels(max(lens))
+    kern_o = oracle.kernel_pool(w.k, [0] * 6, lens, 32, 16, nk_cap=nk_cap)
+    P = oparams(w.params)
+    r = oracle.block_score_topk(w.q, kern_o, w.q_ctx, P)
+    out_o, lse_o = oracle.sparse_attention(w.q, w.k, w.v, w.q_ctx, r["idx"], r["cnt"], P)
+    p = bparams(w.params)
+    B, _, Hq, _ = w.q.shape
+    out = torch.empty((B, 1, Hq, d), dtype=torch.bfloat16, device="cuda")
+    lse = torch.empty((B, 1, Hq), dtype=torch.float32, device="cuda")
+    ws = binding.workspace(p, B, 1, max(lens), Hq, 2, d)
+    binding.infllmv2_sparse_attn_decode(dev(w.q), dev(w.k), dev(w.v), dev_i32(w.ctx_lens), max(lens),
+                                        dev_i32(r["idx"]), dev_i32(r["cnt"]), p, out, lse, ws)
+    torch.cuda.synchronize()
+    check_attention(out, out_o, lse, lse_o, what="decode")
+
+
+@pytest.mark.parametrize("d", [64, 128])
+def test_dense_paths(oracle, d):
+    T = 700
+    w = prefill_case(T, 32, 2, d, topk=1, dense_len=0, seed=700 + d, n_needles=0)
+    out_o, lse_o = oracle.dense_attention(w.q, w.k, w.v, w.q_ctx)
+    out = torch.empty((1, T, 32, d), dtype=torch.bfloat16, device="cuda")
+    lse = torch.empty((1, T, 32), dtype=torch.float32, device="cuda")
+    binding.infllmv2_dense_attn_prefill(dev(w.q), dev(w.k), dev(w.v), None, dev_i32(w.ctx_lens), T, 0.0, out, lse)
+    torch.cuda.synchronize()
+    check_attention(out, out_o, lse, lse_o, what="dense prefill")
+    lens = [5000, 1, 64, 777]
+    wd = decode_case(lens, 32, 2, d, topk=1, dense_len=0, seed=710 + d, n_needles=0)
+    out_o, lse_o = oracle.dense_attention(wd.q, wd.k, wd.v, wd.q_ctx)
+    out = torch.empty((4, 1, 32, d), dtype=torch.bfloat16, device="cuda")
+    lse = torch.empty((4, 1, 32), dtype=torch.float32, device="cuda")
+    p = binding.Params()
+    ws = binding.workspace(p, 4, 1, max(lens), 32, 2, d)
+    binding.infllmv2_dense_attn_decode(dev(wd.q), dev(wd.k), dev(wd.v), dev_i32(wd.ctx_lens), max(lens), 0.0, out,
+                                       lse, ws)
+    torch.cuda.synchronize()
+    check_attention(out, out_o, lse, lse_o, what="dense decode")
+
+
+@pytest.mark.parametrize("parents", ["random", "chain", "star"])
+def test_tree_verify(oracle, parents):
+    P_, N = 3000, 16
+    par = None
+    if parents == "chain":
+        par = np.arange(-1, N - 1)
+    elif parents == "star":
+        par = np.array([-1] + [0] * (N - 1))
+    w = tree_case(P_, N, 32, 2, 128, topk=8, dense_len=1024, seed=800, B=2, parents=par)
+    nk_cap = oracle.num_kernels(P_)
+    kern_o = oracle.kernel_pool(w.k, [0, 0], [P_, P_], 32, 16, nk_cap=nk_cap)
+    Pm = oparams(w.params)
+    r = oracle.block_score_topk(w.q, kern_o, w.q_ctx, Pm)
+    gidx, gcnt = gpu_select(w, gpu_pool(w.k, [0, 0], [P_, P_], P_, nk_cap))
+    check_selection(gidx, gcnt, r)
+    out_o, lse_o = oracle.sparse_attention(w.q, w.k, w.v, w.q_ctx, r["idx"], r["cnt"], Pm, w.extras["k_draft"],
+                                           w.extras["v_draft"], w.extras["tree_mask"])
+    p = bparams(w.params)
+    out = torch.empty(w.q.shape, dtype=torch.bfloat16, device="cuda")
+    lse = torch.empty(w.q.shape[:3], dtype=torch.float32, device="cuda")
+    ws = binding.workspace(p, 2, N, P_, 32, 2, 128)
+    binding.infllmv2_sparse_attn_tree_verify(dev(w.q), dev(w.k), dev(w.v), dev_i32(w.ctx_lens), P_,
+                                             dev(w.extras["k_draft"]), dev(w.extras["v_draft"]),
+                                             dev_i32(w.extras["tree_mask"].view(np.int32)), dev_i32(r["idx"]),
+                                             dev_i32(r["cnt"]), p, out, lse, ws)
+    torch.cuda.synchronize()
+    check_attention(out, out_o, lse, lse_o, what="tree")
+
+
+# ---------------------------------------------------------------------------------------------------
+# the whole path on the GPU (its own kernels, its own selection) against the oracle
+# ---------------------------------------------------------------------------------------------------
+
+def test_end_to_end_tiny_prefill(oracle):
+    w = prefill_case(2048, 4, 2, 64, topk=8, dense_len=0, seed=1001, n_needles=3)
+    T = 2048
+    nk_cap = oracle.num_kernels(T)
+    P = oparams(w.params)
+    kern_o = oracle.kernel_pool(w.k, [0], [T], 32, 16, nk_cap=nk_cap)
+    r = oracle.block_score_topk(w.q, kern_o, w.q_ctx, P)
+    out_o, lse_o = oracle.sparse_attention(w.q, w.k, w.v, w.q_ctx, r["idx"], r["cnt"], P)
+    kern = gpu_pool(w.k, [0], [T], T, nk_cap)
+    gidx, gcnt = gpu_select(w, kern)
+    same = check_selection(gidx, gcnt, r)
+    out = torch.empty((1, T, 4, 64), dtype=torch.bfloat16, device="cuda")
+    binding.infllmv2_sparse_attn_prefill(dev(w.q), dev(w.k), dev(w.v), None, dev_i32(w.ctx_lens), T,
+                                         dev_i32(gidx), dev_i32(gcnt), bparams(w.params), out)
+    torch.cuda.synchronize()
+    row_same = same.all(axis=-1)  # [B, T]: both groups match
+    check_attention(out, out_o, mask=row_same, what="end-to-end")

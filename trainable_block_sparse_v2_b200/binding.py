@@ -1,0 +1,258 @@
+"""ctypes binding of libinfllmv2.so -- argument marshalling only.
+
+Every function has the name of the C entry point it calls (include/infllmv2.h), takes torch CUDA tensors
+(or plain ints), checks dtype / device / contiguity, passes raw device pointers and sizes, and raises
+``Infllmv2Error`` when the library returns a non-zero status.  All computation happens in the library's
+CUDA kernels; there is no CPU fallback: if the library is missing, ``load()`` raises.
+
+Layouts (bf16 unless stated): q [B, T, Hq, d]; k / v cache [B, Lcap, Hkv, d]; kern [B, Hkv, nk_cap, d];
+idx [B, T, Hkv, kmax] int32; cnt [B, T, Hkv] int32; out [B, T, Hq, d]; lse [B, T, Hq] float32.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+from dataclasses import dataclass
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libinfllmv2.so")
+_lib = None
+
+STATUS = {0: "ok", 1: "invalid argument", 2: "unsupported", 3: "workspace", 4: "cuda", 5: "timeout"}
+
+
+class Infllmv2Error(RuntimeError):
+    def __init__(self, fn, status, msg):
+        super().__init__(f"{fn}: status {status} ({msg})")
+        self.status = status
+
+
+class CParams(ctypes.Structure):
+    _fields_ = [("block_size", ctypes.c_int), ("kernel_size", ctypes.c_int), ("kernel_stride", ctypes.c_int),
+                ("topk", ctypes.c_int), ("init_blocks", ctypes.c_int), ("local_blocks", ctypes.c_int),
+                ("dense_len", ctypes.c_int), ("membership", ctypes.c_int), ("softmax_scale", ctypes.c_float)]
+
+
+@dataclass
+class Params:
+    """Method constants (infllmv2_params).  softmax_scale <= 0 selects 1/sqrt(d)."""
+    block_size: int = 64
+    kernel_size: int = 32
+    kernel_stride: int = 16
+    topk: int = 64
+    init_blocks: int = 1
+    local_blocks: int = 2
+    dense_len: int = 0
+    membership: int = 0
+    softmax_scale: float = 0.0
+
+    @property
+    def kmax(self) -> int:
+        return self.topk + self.init_blocks + self.local_blocks
+
+    def c(self) -> CParams:
+        return CParams(self.block_size, self.kernel_size, self.kernel_stride, self.topk, self.init_blocks,
+                       self.local_blocks, self.dense_len, self.membership, float(self.softmax_scale))
+
+
+_P = ctypes.c_void_p
+_I = ctypes.c_int
+_SZ = ctypes.c_size_t
+_PP = ctypes.POINTER(CParams)
+_F = ctypes.c_float
+
+_SIGS = {
+    "infllmv2_status_string": ([_I], ctypes.c_char_p),
+    "infllmv2_version": ([], _I),
+    "infllmv2_workspace_size": ([_PP, _I, _I, _I, _I, _I, _I], _SZ),
+    "infllmv2_kernel_pool": ([_P, _I, _I, _I, _I, _P, _P, _I, _PP, _P, _I, _P], _I),
+    "infllmv2_block_score_topk": ([_P, _I, _I, _I, _I, _I, _P, _P, _I, _P, _I, _PP, _P, _P, _P, _SZ, _P], _I),
+    "infllmv2_sparse_attn_prefill": ([_P, _I, _I, _I, _I, _I, _P, _P, _I, _P, _P, _I, _P, _P, _PP, _P, _P, _P,
+                                      _SZ, _P], _I),
+    "infllmv2_sparse_attn_decode": ([_P, _I, _I, _I, _I, _P, _P, _I, _P, _I, _P, _P, _PP, _P, _P, _P, _SZ, _P], _I),
+    "infllmv2_sparse_attn_tree_verify": ([_P, _I, _I, _I, _I, _I, _P, _P, _I, _P, _I, _P, _P, _P, _P, _P, _PP, _P,
+                                          _P, _P, _SZ, _P], _I),
+    "infllmv2_dense_attn_prefill": ([_P, _I, _I, _I, _I, _I, _P, _P, _I, _P, _P, _I, _F, _P, _P, _P, _SZ, _P], _I),
+    "infllmv2_dense_attn_decode": ([_P, _I, _I, _I, _I, _P, _P, _I, _P, _I, _F, _P, _P, _P, _SZ, _P], _I),
+}
+
+EXPORTED = tuple(_SIGS)
+
+
+def load(path: str = LIB_PATH):
+    """Load libinfllmv2.so (raises OSError when it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(path):
+            raise OSError(f"{path} not found: build it with `python -m trainable_block_sparse_v2_b200.build`")
+        lib = ctypes.CDLL(path)
+        for name, (args, res) in _SIGS.items():
+            fn = getattr(lib, name)
+            fn.argtypes = args
+            fn.restype = res
+        _lib = lib
+    return _lib
+
+
+def _ptr(t):
+    if t is None:
+        return None
+    if isinstance(t, int):
+        return t
+    return t.data_ptr()
+
+
+def _stream(stream):
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, int):
+        return stream
+    return stream.cuda_stream
+
+
+def _need(t, dtype, name, ndim=None):
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name}: expected a torch.Tensor")
+    if t.dtype != dtype:
+        raise TypeError(f"{name}: expected {dtype}, got {t.dtype}")
+    if not t.is_cuda:
+        raise ValueError(f"{name}: must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name}: must be contiguous")
+    if ndim is not None and t.dim() != ndim:
+        raise ValueError(f"{name}: expected {ndim} dims, got {tuple(t.shape)}")
+    return t
+
+
+def _check(fn, status):
+    if status != 0:
+        msg = load().infllmv2_status_string(status).decode()
+        raise Infllmv2Error(fn, status, msg)
+
+
+def infllmv2_version() -> int:
+    return load().infllmv2_version()
+
+
+def infllmv2_status_string(status: int) -> str:
+    return load().infllmv2_status_string(status).decode()
+
+
+def infllmv2_workspace_size(params: Params, batch, max_q, max_ctx, hq, hkv, head_dim) -> int:
+    cp = params.c()
+    return int(load().infllmv2_workspace_size(ctypes.byref(cp), batch, max_q, max_ctx, hq, hkv, head_dim))
+
+
+def infllmv2_kernel_pool(k, old_lens, new_lens, max_new_keys, params: Params, kern, stream=None):
+    _need(k, torch.bfloat16, "k", 4)
+    _need(kern, torch.bfloat16, "kern", 4)
+    _need(old_lens, torch.int32, "old_lens")
+    _need(new_lens, torch.int32, "new_lens")
+    B, Lcap, Hkv, d = k.shape
+    cp = params.c()
+    st = load().infllmv2_kernel_pool(_ptr(k), B, Lcap, Hkv, d, _ptr(old_lens), _ptr(new_lens), int(max_new_keys),
+                                     ctypes.byref(cp), _ptr(kern), kern.shape[2], _stream(stream))
+    _check("infllmv2_kernel_pool", st)
+
+
+def infllmv2_block_score_topk(q, q_ctx, ctx_lens, max_ctx, kern, params: Params, idx, cnt, ws, stream=None):
+    _need(q, torch.bfloat16, "q", 4)
+    _need(kern, torch.bfloat16, "kern", 4)
+    _need(idx, torch.int32, "idx", 4)
+    _need(cnt, torch.int32, "cnt", 3)
+    if q_ctx is not None:
+        _need(q_ctx, torch.int32, "q_ctx")
+    if ctx_lens is not None:
+        _need(ctx_lens, torch.int32, "ctx_lens")
+    B, T, Hq, d = q.shape
+    Hkv = kern.shape[1]
+    cp = params.c()
+    st = load().infllmv2_block_score_topk(_ptr(q), B, T, Hq, Hkv, d, _ptr(q_ctx), _ptr(ctx_lens), int(max_ctx),
+                                          _ptr(kern), kern.shape[2], ctypes.byref(cp), _ptr(idx), _ptr(cnt),
+                                          _ptr(ws), 0 if ws is None else ws.numel() * ws.element_size(),
+                                          _stream(stream))
+    _check("infllmv2_block_score_topk", st)
+
+
+def infllmv2_sparse_attn_prefill(q, k, v, q_ctx, ctx_lens, max_ctx, idx, cnt, params: Params, out, lse=None,
+                                 ws=None, stream=None):
+    for t, n in ((q, "q"), (k, "k"), (v, "v"), (out, "out")):
+        _need(t, torch.bfloat16, n, 4)
+    _need(idx, torch.int32, "idx", 4)
+    _need(cnt, torch.int32, "cnt", 3)
+    if lse is not None:
+        _need(lse, torch.float32, "lse")
+    B, T, Hq, d = q.shape
+    Lcap, Hkv = k.shape[1], k.shape[2]
+    cp = params.c()
+    st = load().infllmv2_sparse_attn_prefill(_ptr(q), B, T, Hq, Hkv, d, _ptr(k), _ptr(v), Lcap, _ptr(q_ctx),
+                                             _ptr(ctx_lens), int(max_ctx), _ptr(idx), _ptr(cnt), ctypes.byref(cp),
+                                             _ptr(out), _ptr(lse), _ptr(ws),
+                                             0 if ws is None else ws.numel() * ws.element_size(), _stream(stream))
+    _check("infllmv2_sparse_attn_prefill", st)
+
+
+def infllmv2_sparse_attn_decode(q, k, v, ctx_lens, max_ctx, idx, cnt, params: Params, out, lse, ws, stream=None):
+    for t, n in ((q, "q"), (k, "k"), (v, "v"), (out, "out")):
+        _need(t, torch.bfloat16, n)
+    B, Hq, d = q.shape[0], q.shape[-2], q.shape[-1]
+    Lcap, Hkv = k.shape[1], k.shape[2]
+    cp = params.c()
+    st = load().infllmv2_sparse_attn_decode(_ptr(q), B, Hq, Hkv, d, _ptr(k), _ptr(v), Lcap, _ptr(ctx_lens),
+                                            int(max_ctx), _ptr(idx), _ptr(cnt), ctypes.byref(cp), _ptr(out), _ptr(lse),
+                                            _ptr(ws), 0 if ws is None else ws.numel() * ws.element_size(),
+                                            _stream(stream))
+    _check("infllmv2_sparse_attn_decode", st)
+
+
+def infllmv2_sparse_attn_tree_verify(q, k, v, prefix_lens, max_ctx, k_draft, v_draft, tree_mask, idx, cnt,
+                                     params: Params, out, lse, ws, stream=None):
+    for t, n in ((q, "q"), (k, "k"), (v, "v"), (k_draft, "k_draft"), (v_draft, "v_draft"), (out, "out")):
+        _need(t, torch.bfloat16, n, 4)
+    B, N, Hq, d = q.shape
+    Lcap, Hkv = k.shape[1], k.shape[2]
+    cp = params.c()
+    st = load().infllmv2_sparse_attn_tree_verify(_ptr(q), B, N, Hq, Hkv, d, _ptr(k), _ptr(v), Lcap, _ptr(prefix_lens),
+                                                 int(max_ctx), _ptr(k_draft), _ptr(v_draft), _ptr(tree_mask), _ptr(idx),
+                                                 _ptr(cnt), ctypes.byref(cp), _ptr(out), _ptr(lse), _ptr(ws),
+                                                 0 if ws is None else ws.numel() * ws.element_size(), _stream(stream))
+    _check("infllmv2_sparse_attn_tree_verify", st)
+
+
+def infllmv2_dense_attn_prefill(q, k, v, q_ctx, ctx_lens, max_ctx, softmax_scale, out, lse=None, ws=None,
+                                stream=None):
+    for t, n in ((q, "q"), (k, "k"), (v, "v"), (out, "out")):
+        _need(t, torch.bfloat16, n, 4)
+    B, T, Hq, d = q.shape
+    Lcap, Hkv = k.shape[1], k.shape[2]
+    st = load().infllmv2_dense_attn_prefill(_ptr(q), B, T, Hq, Hkv, d, _ptr(k), _ptr(v), Lcap, _ptr(q_ctx),
+                                            _ptr(ctx_lens), int(max_ctx), float(softmax_scale), _ptr(out), _ptr(lse),
+                                            _ptr(ws), 0 if ws is None else ws.numel() * ws.element_size(),
+                                            _stream(stream))
+    _check("infllmv2_dense_attn_prefill", st)
+
+
+def infllmv2_dense_attn_decode(q, k, v, ctx_lens, max_ctx, softmax_scale, out, lse, ws, stream=None):
+    for t, n in ((q, "q"), (k, "k"), (v, "v"), (out, "out")):
+        _need(t, torch.bfloat16, n)
+    B, Hq, d = q.shape[0], q.shape[-2], q.shape[-1]
+    Lcap, Hkv = k.shape[1], k.shape[2]
+    st = load().infllmv2_dense_attn_decode(_ptr(q), B, Hq, Hkv, d, _ptr(k), _ptr(v), Lcap, _ptr(ctx_lens), int(max_ctx),
+                                           float(softmax_scale), _ptr(out), _ptr(lse), _ptr(ws),
+                                           0 if ws is None else ws.numel() * ws.element_size(), _stream(stream))
+    _check("infllmv2_dense_attn_decode", st)
+
+
+def num_kernels(n: int, kernel_size: int = 32, kernel_stride: int = 16) -> int:
+    return 0 if n < kernel_size else (n - kernel_size) // kernel_stride + 1
+
+
+def workspace(params: Params, batch, max_q, max_ctx, hq, hkv, head_dim, device="cuda"):
+    """Allocate (with torch) a workspace of infllmv2_workspace_size bytes, 256-byte aligned."""
+    n = infllmv2_workspace_size(params, batch, max_q, max_ctx, hq, hkv, head_dim)
+    if n == 0:
+        raise Infllmv2Error("infllmv2_workspace_size", 1, "invalid sizes")
+    return torch.empty(math.ceil(n / 256) * 256, dtype=torch.uint8, device=device)

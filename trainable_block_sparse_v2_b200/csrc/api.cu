@@ -1,0 +1,323 @@
+// api.cu -- the C ABI of libinfllmv2.so (declared in include/infllmv2.h).
+//
+// Every entry point validates its arguments on the host and returns a status before launching anything
+// when they are wrong; then it enqueues the kernels on the caller's stream.  The library allocates no
+// memory and keeps no state between calls.
+#include <cmath>
+#include <cstdint>
+
+#include "../../include/infllmv2.h"
+#include "common.cuh"
+#include "internal.h"
+
+using iv2::MethodConsts;
+using iv2::QueryRows;
+
+namespace {
+
+constexpr int kVersion = 100;  // 0.1.0
+
+bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+int nk_of(long n) { return n >= iv2::kKernelSize ? (int)((n - iv2::kKernelSize) / iv2::kKernelStride + 1) : 0; }
+
+constexpr int kMaxBlocks = 4096;  // contexts up to 256K keys
+
+int check_params(const infllmv2_params* p)
+{
+    if (!p) return INFLLMV2_ERR_INVALID_ARG;
+    if (p->topk < 0 || p->init_blocks < 0 || p->local_blocks < 0 || p->dense_len < 0) return INFLLMV2_ERR_INVALID_ARG;
+    if (p->membership != 0 && p->membership != 1) return INFLLMV2_ERR_INVALID_ARG;
+    if (p->topk + p->init_blocks + p->local_blocks < 1) return INFLLMV2_ERR_INVALID_ARG;
+    if (!(p->softmax_scale == p->softmax_scale) || std::isinf(p->softmax_scale)) return INFLLMV2_ERR_INVALID_ARG;
+    if (p->block_size != iv2::kBlock || p->kernel_size != iv2::kKernelSize || p->kernel_stride != iv2::kKernelStride)
+        return INFLLMV2_ERR_UNSUPPORTED;
+    return INFLLMV2_OK;
+}
+
+MethodConsts consts_of(const infllmv2_params* p, int d)
+{
+    MethodConsts mc;
+    mc.topk = p->topk;
+    mc.init_blocks = p->init_blocks;
+    mc.local_blocks = p->local_blocks;
+    mc.dense_len = p->dense_len;
+    mc.membership = p->membership;
+    mc.scale = p->softmax_scale > 0.f ? p->softmax_scale : 1.0f / std::sqrt((float)d);
+    mc.kmax = p->topk + p->init_blocks + p->local_blocks;
+    return mc;
+}
+
+MethodConsts dense_consts(float scale, int d)
+{
+    MethodConsts mc{};
+    mc.topk = 0;
+    mc.init_blocks = 0;
+    mc.local_blocks = 0;
+    mc.dense_len = 0;
+    mc.membership = 0;
+    mc.scale = scale > 0.f ? scale : 1.0f / std::sqrt((float)d);
+    mc.kmax = 1;
+    return mc;
+}
+
+int check_heads(int batch, int nq, int hq, int hkv, int d)
+{
+    if (batch < 1 || nq < 1 || hq < 1 || hkv < 1) return INFLLMV2_ERR_INVALID_ARG;
+    if (hq % hkv != 0) return INFLLMV2_ERR_INVALID_ARG;
+    const int G = hq / hkv;
+    if (G != 1 && G != 2 && G != 4 && G != 8 && G != 16) return INFLLMV2_ERR_UNSUPPORTED;
+    if (d != 64 && d != 128) return INFLLMV2_ERR_UNSUPPORTED;
+    if ((long)batch * nq * hkv > (1L << 30)) return INFLLMV2_ERR_UNSUPPORTED;
+    return INFLLMV2_OK;
+}
+
+int check_ptr16(const void* p) { return (p && aligned(p, 16)) ? INFLLMV2_OK : INFLLMV2_ERR_INVALID_ARG; }
+int check_ptr4(const void* p) { return (p && aligned(p, 4)) ? INFLLMV2_OK : INFLLMV2_ERR_INVALID_ARG; }
+int check_opt4(const void* p) { return (!p || aligned(p, 4)) ? INFLLMV2_OK : INFLLMV2_ERR_INVALID_ARG; }
+
+int check_ctx(int max_ctx, int lcap)
+{
+    if (max_ctx < 1) return INFLLMV2_ERR_INVALID_ARG;
+    if (lcap >= 0 && max_ctx > lcap) return INFLLMV2_ERR_INVALID_ARG;
+    if ((max_ctx - 1) / iv2::kBlock + 1 > kMaxBlocks) return INFLLMV2_ERR_UNSUPPORTED;
+    return INFLLMV2_OK;
+}
+
+int check_ws(void* ws, size_t ws_bytes, size_t need)
+{
+    if (need == 0) return INFLLMV2_OK;
+    if (!ws || !aligned(ws, 256) || ws_bytes < need) return INFLLMV2_ERR_WORKSPACE;
+    return INFLLMV2_OK;
+}
+
+int launched(cudaError_t e) { return e == cudaSuccess ? INFLLMV2_OK : INFLLMV2_ERR_CUDA; }
+
+#define IV2_TRY(expr)                        \
+    do {                                     \
+        const int _st = (expr);              \
+        if (_st != INFLLMV2_OK) return _st;  \
+    } while (0)
+
+size_t score_need(int batch, int nq, int hq, int hkv, int d, int max_ctx)
+{
+    if (!iv2::score_uses_scan_path(batch, nq, hq / hkv, d, max_ctx)) return 0;
+    return iv2::score_ws_bytes(batch * nq * hkv, max_ctx);
+}
+
+size_t split_need(int rows, int max_ctx, int kmax, int dense_len, bool dense_all, bool draft)
+{
+    const int nsplit = iv2::attn_split_count(iv2::attn_split_max_blocks(max_ctx, kmax, dense_len, dense_all)) +
+                       (draft ? 1 : 0);
+    return iv2::attn_ws_bytes(rows, nsplit);
+}
+
+QueryRows rows_of(const void* q, int B, int T, int hq, int hkv, int d, const int32_t* q_ctx, const int32_t* ctx_lens,
+                  int same_ctx, int max_ctx)
+{
+    QueryRows qr;
+    qr.q = q;
+    qr.B = B;
+    qr.T = T;
+    qr.Hq = hq;
+    qr.Hkv = hkv;
+    qr.D = d;
+    qr.q_ctx = q_ctx;
+    qr.ctx_lens = ctx_lens;
+    qr.same_ctx = same_ctx;
+    qr.max_ctx = max_ctx;
+    return qr;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* infllmv2_status_string(int status)
+{
+    switch (status) {
+    case INFLLMV2_OK: return "ok";
+    case INFLLMV2_ERR_INVALID_ARG: return "invalid argument";
+    case INFLLMV2_ERR_UNSUPPORTED: return "unsupported configuration";
+    case INFLLMV2_ERR_WORKSPACE: return "workspace missing, misaligned or too small";
+    case INFLLMV2_ERR_CUDA: return "CUDA launch failed";
+    case INFLLMV2_ERR_TIMEOUT: return "timeout";
+    default: return "unknown status";
+    }
+}
+
+int infllmv2_version(void) { return kVersion; }
+
+size_t infllmv2_workspace_size(const infllmv2_params* params, int batch, int max_q, int max_ctx, int hq, int hkv,
+                               int head_dim)
+{
+    if (check_params(params) != INFLLMV2_OK) return 0;
+    if (check_heads(batch, max_q, hq, hkv, head_dim) != INFLLMV2_OK) return 0;
+    if (check_ctx(max_ctx, -1) != INFLLMV2_OK) return 0;
+    const int kmax = params->topk + params->init_blocks + params->local_blocks;
+    size_t need = score_need(batch, max_q, hq, hkv, head_dim, max_ctx);
+    const int rows = batch * max_q * hkv;
+    const size_t attn = split_need(rows, max_ctx, kmax, params->dense_len, true, true);
+    if (attn > need) need = attn;
+    return need < 256 ? 256 : need;
+}
+
+int infllmv2_kernel_pool(const void* k, int batch, int lcap, int hkv, int head_dim, const int32_t* old_lens,
+                         const int32_t* new_lens, int max_new_keys, const infllmv2_params* params, void* kern,
+                         int nk_cap, infllmv2_stream_t stream)
+{
+    IV2_TRY(check_params(params));
+    IV2_TRY(check_heads(batch, 1, hkv, hkv, head_dim));
+    IV2_TRY(check_ptr16(k));
+    IV2_TRY(check_ptr16(kern));
+    IV2_TRY(check_ptr4(old_lens));
+    IV2_TRY(check_ptr4(new_lens));
+    if (lcap < 1 || max_new_keys < 0 || nk_cap < 1 || max_new_keys > lcap) return INFLLMV2_ERR_INVALID_ARG;
+    if (nk_cap < nk_of(max_new_keys)) return INFLLMV2_ERR_INVALID_ARG;
+    if (max_new_keys == 0) return INFLLMV2_OK;
+    return launched(iv2::launch_kernel_pool(k, batch, lcap, hkv, head_dim, old_lens, new_lens, max_new_keys, kern,
+                                            nk_cap, (cudaStream_t)stream));
+}
+
+int infllmv2_block_score_topk(const void* q, int batch, int num_q, int hq, int hkv, int head_dim,
+                              const int32_t* q_ctx, const int32_t* ctx_lens, int max_ctx, const void* kern,
+                              int nk_cap, const infllmv2_params* params, int32_t* idx, int32_t* cnt, void* ws,
+                              size_t ws_bytes, infllmv2_stream_t stream)
+{
+    IV2_TRY(check_params(params));
+    IV2_TRY(check_heads(batch, num_q, hq, hkv, head_dim));
+    IV2_TRY(check_ptr16(q));
+    IV2_TRY(check_ptr16(kern));
+    IV2_TRY(check_ptr4(idx));
+    IV2_TRY(check_ptr4(cnt));
+    IV2_TRY(check_opt4(q_ctx));
+    IV2_TRY(check_opt4(ctx_lens));
+    if (!q_ctx && !ctx_lens) return INFLLMV2_ERR_INVALID_ARG;
+    IV2_TRY(check_ctx(max_ctx, -1));
+    if (nk_cap < 1 || nk_cap < nk_of(max_ctx)) return INFLLMV2_ERR_INVALID_ARG;
+    IV2_TRY(check_ws(ws, ws_bytes, score_need(batch, num_q, hq, hkv, head_dim, max_ctx)));
+    const QueryRows qr = rows_of(q, batch, num_q, hq, hkv, head_dim, q_ctx, ctx_lens, 0, max_ctx);
+    return launched(iv2::launch_score_topk(qr, kern, nk_cap, consts_of(params, head_dim), idx, cnt, ws,
+                                           (cudaStream_t)stream));
+}
+
+int infllmv2_sparse_attn_prefill(const void* q, int batch, int num_q, int hq, int hkv, int head_dim, const void* k,
+                                 const void* v, int lcap, const int32_t* q_ctx, const int32_t* ctx_lens, int max_ctx,
+                                 const int32_t* idx, const int32_t* cnt, const infllmv2_params* params, void* out,
+                                 float* lse, void* ws, size_t ws_bytes, infllmv2_stream_t stream)
+{
+    (void)ws;
+    (void)ws_bytes;
+    IV2_TRY(check_params(params));
+    IV2_TRY(check_heads(batch, num_q, hq, hkv, head_dim));
+    IV2_TRY(check_ptr16(q));
+    IV2_TRY(check_ptr16(k));
+    IV2_TRY(check_ptr16(v));
+    IV2_TRY(check_ptr16(out));
+    IV2_TRY(check_ptr4(idx));
+    IV2_TRY(check_ptr4(cnt));
+    IV2_TRY(check_opt4(lse));
+    IV2_TRY(check_opt4(q_ctx));
+    IV2_TRY(check_opt4(ctx_lens));
+    if (!q_ctx && !ctx_lens) return INFLLMV2_ERR_INVALID_ARG;
+    IV2_TRY(check_ctx(max_ctx, lcap));
+    const QueryRows qr = rows_of(q, batch, num_q, hq, hkv, head_dim, q_ctx, ctx_lens, 0, max_ctx);
+    return launched(iv2::launch_attn_rows(qr, k, v, lcap, idx, cnt, consts_of(params, head_dim), false, out, lse,
+                                          (cudaStream_t)stream));
+}
+
+int infllmv2_sparse_attn_decode(const void* q, int batch, int hq, int hkv, int head_dim, const void* k, const void* v,
+                                int lcap, const int32_t* ctx_lens, int max_ctx, const int32_t* idx,
+                                const int32_t* cnt, const infllmv2_params* params, void* out, float* lse, void* ws,
+                                size_t ws_bytes, infllmv2_stream_t stream)
+{
+    IV2_TRY(check_params(params));
+    IV2_TRY(check_heads(batch, 1, hq, hkv, head_dim));
+    IV2_TRY(check_ptr16(q));
+    IV2_TRY(check_ptr16(k));
+    IV2_TRY(check_ptr16(v));
+    IV2_TRY(check_ptr16(out));
+    IV2_TRY(check_ptr4(idx));
+    IV2_TRY(check_ptr4(cnt));
+    IV2_TRY(check_ptr4(ctx_lens));
+    IV2_TRY(check_opt4(lse));
+    IV2_TRY(check_ctx(max_ctx, lcap));
+    const MethodConsts mc = consts_of(params, head_dim);
+    IV2_TRY(check_ws(ws, ws_bytes, split_need(batch * hkv, max_ctx, mc.kmax, mc.dense_len, false, false)));
+    const QueryRows qr = rows_of(q, batch, 1, hq, hkv, head_dim, nullptr, ctx_lens, 0, max_ctx);
+    return launched(iv2::launch_attn_split(qr, k, v, lcap, idx, cnt, mc, false, nullptr, nullptr, nullptr, out, lse,
+                                           ws, (cudaStream_t)stream));
+}
+
+int infllmv2_sparse_attn_tree_verify(const void* q, int batch, int n_draft, int hq, int hkv, int head_dim,
+                                     const void* k, const void* v, int lcap, const int32_t* prefix_lens, int max_ctx,
+                                     const void* k_draft, const void* v_draft, const uint32_t* tree_mask,
+                                     const int32_t* idx, const int32_t* cnt, const infllmv2_params* params, void* out,
+                                     float* lse, void* ws, size_t ws_bytes, infllmv2_stream_t stream)
+{
+    IV2_TRY(check_params(params));
+    IV2_TRY(check_heads(batch, n_draft, hq, hkv, head_dim));
+    if (n_draft > 32) return INFLLMV2_ERR_UNSUPPORTED;
+    IV2_TRY(check_ptr16(q));
+    IV2_TRY(check_ptr16(k));
+    IV2_TRY(check_ptr16(v));
+    IV2_TRY(check_ptr16(k_draft));
+    IV2_TRY(check_ptr16(v_draft));
+    IV2_TRY(check_ptr16(out));
+    IV2_TRY(check_ptr4(tree_mask));
+    IV2_TRY(check_ptr4(idx));
+    IV2_TRY(check_ptr4(cnt));
+    IV2_TRY(check_ptr4(prefix_lens));
+    IV2_TRY(check_opt4(lse));
+    IV2_TRY(check_ctx(max_ctx, lcap));
+    const MethodConsts mc = consts_of(params, head_dim);
+    IV2_TRY(check_ws(ws, ws_bytes, split_need(batch * n_draft * hkv, max_ctx, mc.kmax, mc.dense_len, false, true)));
+    const QueryRows qr = rows_of(q, batch, n_draft, hq, hkv, head_dim, nullptr, prefix_lens, 1, max_ctx);
+    return launched(iv2::launch_attn_split(qr, k, v, lcap, idx, cnt, mc, false, k_draft, v_draft, tree_mask, out, lse,
+                                           ws, (cudaStream_t)stream));
+}
+
+int infllmv2_dense_attn_prefill(const void* q, int batch, int num_q, int hq, int hkv, int head_dim, const void* k,
+                                const void* v, int lcap, const int32_t* q_ctx, const int32_t* ctx_lens, int max_ctx,
+                                float softmax_scale, void* out, float* lse, void* ws, size_t ws_bytes,
+                                infllmv2_stream_t stream)
+{
+    (void)ws;
+    (void)ws_bytes;
+    IV2_TRY(check_heads(batch, num_q, hq, hkv, head_dim));
+    if (!(softmax_scale == softmax_scale) || std::isinf(softmax_scale)) return INFLLMV2_ERR_INVALID_ARG;
+    IV2_TRY(check_ptr16(q));
+    IV2_TRY(check_ptr16(k));
+    IV2_TRY(check_ptr16(v));
+    IV2_TRY(check_ptr16(out));
+    IV2_TRY(check_opt4(lse));
+    IV2_TRY(check_opt4(q_ctx));
+    IV2_TRY(check_opt4(ctx_lens));
+    if (!q_ctx && !ctx_lens) return INFLLMV2_ERR_INVALID_ARG;
+    IV2_TRY(check_ctx(max_ctx, lcap));
+    const QueryRows qr = rows_of(q, batch, num_q, hq, hkv, head_dim, q_ctx, ctx_lens, 0, max_ctx);
+    return launched(iv2::launch_attn_rows(qr, k, v, lcap, nullptr, nullptr, dense_consts(softmax_scale, head_dim),
+                                          true, out, lse, (cudaStream_t)stream));
+}
+
+int infllmv2_dense_attn_decode(const void* q, int batch, int hq, int hkv, int head_dim, const void* k, const void* v,
+                               int lcap, const int32_t* ctx_lens, int max_ctx, float softmax_scale, void* out,
+                               float* lse, void* ws, size_t ws_bytes, infllmv2_stream_t stream)
+{
+    IV2_TRY(check_heads(batch, 1, hq, hkv, head_dim));
+    if (!(softmax_scale == softmax_scale) || std::isinf(softmax_scale)) return INFLLMV2_ERR_INVALID_ARG;
+    IV2_TRY(check_ptr16(q));
+    IV2_TRY(check_ptr16(k));
+    IV2_TRY(check_ptr16(v));
+    IV2_TRY(check_ptr16(out));
+    IV2_TRY(check_ptr4(ctx_lens));
+    IV2_TRY(check_opt4(lse));
+    IV2_TRY(check_ctx(max_ctx, lcap));
+    const MethodConsts mc = dense_consts(softmax_scale, head_dim);
+    IV2_TRY(check_ws(ws, ws_bytes, split_need(batch * hkv, max_ctx, mc.kmax, 0, true, false)));
+    const QueryRows qr = rows_of(q, batch, 1, hq, hkv, head_dim, nullptr, ctx_lens, 0, max_ctx);
+    return launched(iv2::launch_attn_split(qr, k, v, lcap, nullptr, nullptr, mc, true, nullptr, nullptr, nullptr, out,
+                                           lse, ws, (cudaStream_t)stream));
+}
+
+}  // extern "C"

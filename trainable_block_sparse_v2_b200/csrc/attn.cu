@@ -1,0 +1,504 @@
+// attn.cu -- block-sparse attention over the selected blocks (step 3 of InfLLM v2), mma.sync path.
+//
+// Query (b, t), head h of group g, context n (MiniCPM4 technical details, InfLLM v2 overview: only the
+// selected context blocks take part in attention; launch article section 1: short contexts dense):
+//   keys = [0, n) when dense, else U_{blk in idx} [64 blk, min(64 blk + 64, n))
+//   out  = sum_i softmax_i(scale q.k_i) v_i,   lse = log sum_i exp(scale q.k_i)
+// Tree verification adds the draft keys whose bit is set in the query's bit-packed ancestor mask
+// (QbitAI article, "speculative sampling, quantisation and long text", long-context bullet).
+//
+// One warp owns the 16 MMA rows of one query token: the G heads of its group (the heads share the block
+// set, so they share every K/V tile -- item 2 of "Model architecture: InfLLM v2" is what makes the tile
+// dense).  A 64-key block is staged in shared memory with cp.async (swizzled 16-byte chunks so ldmatrix
+// is conflict-free), S = Q K^T and O += P V run on m16n8k16, and the softmax is the online (running max
+// / running sum) form in log2 units.
+//  * prefill: one warp per (token, group) row walks the row's whole block list.
+//  * decode / tree: the block list of a row is split across CTAs (4 blocks per CTA, one per warp); each
+//    CTA merges its warps and writes (max, sum, unnormalised O) to the workspace; a merge kernel combines
+//    the splits by their LSE.  Tree rows get one extra split that attends to the draft tile.
+#include "common.cuh"
+#include "internal.h"
+
+namespace iv2 {
+
+template <int D>
+IV2_DEV uint32_t swz_kv(int r, int ch)
+{
+    return (uint32_t)(r * D * 2 + ((ch ^ (r & 7)) << 4));
+}
+
+template <int D>
+struct KvTile {
+    static constexpr int kBytes = kBlock * D * 2;  // one 64-key tile of K or V
+};
+
+// stage rows [0, 64) of a tile: row r comes from src + r * row_stride when r < nvalid, else zeros
+template <int D>
+IV2_DEV void warp_load_tile(unsigned char* dst, const __nv_bfloat16* src, size_t row_stride, int nvalid)
+{
+    constexpr int CH = D / 8;
+    const int lane = threadIdx.x & 31;
+#pragma unroll 4
+    for (int i = lane; i < kBlock * CH; i += 32) {
+        const int r = i / CH, ch = i % CH;
+        const bool ok = r < nvalid;
+        cp_async_16_zfill(dst + swz_kv<D>(r, ch), src + (ok ? (size_t)r * row_stride : 0) + ch * 8, ok ? 16 : 0);
+    }
+}
+
+template <int D>
+struct WarpAttnState {
+    float o[D / 8][4];
+    float m[2];  // running max, log2 units, rows gq and gq + 8
+    float l[2];  // running sum (this lane's columns only until finalised)
+
+    IV2_DEV void init()
+    {
+#pragma unroll
+        for (int i = 0; i < D / 8; ++i) o[i][0] = o[i][1] = o[i][2] = o[i][3] = 0.f;
+        m[0] = m[1] = neg_inf();
+        l[0] = l[1] = 0.f;
+    }
+};
+
+// q rows of one token: rows r < G are heads g*G + r; others zero.  Standard A-fragment layout.
+template <int D>
+IV2_DEV void load_q_rows(const __nv_bfloat16* q_row0, int G, uint32_t (&qf)[D / 16][4])
+{
+    const int lane = threadIdx.x & 31, gq = lane >> 2, tq = lane & 3;
+#pragma unroll
+    for (int ks = 0; ks < D / 16; ++ks)
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const int r = gq + 8 * (i & 1);
+            const int dcol = ks * 16 + 2 * tq + 8 * (i >> 1);
+            qf[ks][i] = r < G ? *reinterpret_cast<const uint32_t*>(q_row0 + (size_t)r * D + dcol) : 0u;
+        }
+}
+
+// S = Q K^T for the staged K tile; acc[nt][4] = rows (gq, gq+8) x keys nt*8 + 2tq + {0,1}
+template <int D>
+IV2_DEV void tile_qk(const uint32_t (&qf)[D / 16][4], const unsigned char* ks_tile, float (&acc)[8][4])
+{
+    const int lane = threadIdx.x & 31;
+#pragma unroll
+    for (int nt = 0; nt < 8; ++nt) acc[nt][0] = acc[nt][1] = acc[nt][2] = acc[nt][3] = 0.f;
+#pragma unroll
+    for (int nt = 0; nt < 8; ++nt) {
+#pragma unroll
+        for (int ks = 0; ks < D / 16; ks += 2) {
+            const int r = nt * 8 + (lane & 7);
+            const int ch = 2 * ks + (lane >> 3);
+            uint32_t b0, b1, b2, b3;
+            ldmatrix_x4(b0, b1, b2, b3, ks_tile + swz_kv<D>(r, ch));
+            mma_bf16_16816(acc[nt], qf[ks], b0, b1);
+            mma_bf16_16816(acc[nt], qf[ks + 1], b2, b3);
+        }
+    }
+}
+
+// online softmax update with the scores of one tile (already scaled to log2 units and masked),
+// then O += P V with the staged V tile
+template <int D>
+IV2_DEV void tile_softmax_pv(WarpAttnState<D>& st, float (&s)[8][4], const unsigned char* vs_tile)
+{
+    const int lane = threadIdx.x & 31;
+    float mnew[2];
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+        float mx = st.m[i];
+#pragma unroll
+        for (int nt = 0; nt < 8; ++nt) mx = fmaxf(mx, fmaxf(s[nt][2 * i], s[nt][2 * i + 1]));
+        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+        mnew[i] = mx;
+    }
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+        const float ref = mnew[i] == neg_inf() ? 0.f : mnew[i];
+        const float alpha = exp2_fast(st.m[i] - ref);  // 0 when the old max is -inf
+        st.l[i] *= alpha;
+#pragma unroll
+        for (int nd = 0; nd < D / 8; ++nd) {
+            st.o[nd][2 * i] *= alpha;
+            st.o[nd][2 * i + 1] *= alpha;
+        }
+#pragma unroll
+        for (int nt = 0; nt < 8; ++nt) {
+            s[nt][2 * i] = exp2_fast(s[nt][2 * i] - ref);
+            s[nt][2 * i + 1] = exp2_fast(s[nt][2 * i + 1] - ref);
+            st.l[i] += s[nt][2 * i] + s[nt][2 * i + 1];
+        }
+        st.m[i] = mnew[i];
+    }
+#pragma unroll
+    for (int kk = 0; kk < 4; ++kk) {  // 16 keys per k-step
+        uint32_t a[4];
+        a[0] = pack_bf16(s[2 * kk][0], s[2 * kk][1]);
+        a[1] = pack_bf16(s[2 * kk][2], s[2 * kk][3]);
+        a[2] = pack_bf16(s[2 * kk + 1][0], s[2 * kk + 1][1]);
+        a[3] = pack_bf16(s[2 * kk + 1][2], s[2 * kk + 1][3]);
+#pragma unroll
+        for (int nd = 0; nd < D / 8; nd += 2) {
+            const int mi = lane >> 3;
+            const int r = 16 * kk + (mi & 1) * 8 + (lane & 7);
+            const int ch = nd + (mi >> 1);
+            uint32_t b0, b1, b2, b3;
+            ldmatrix_x4_trans(b0, b1, b2, b3, vs_tile + swz_kv<D>(r, ch));
+            mma_bf16_16816(st.o[nd], a, b0, b1);
+            mma_bf16_16816(st.o[nd + 1], a, b2, b3);
+        }
+    }
+}
+
+// scale to log2 units and mask: key column c valid iff (valid_mask >> c) & 1 (64-bit mask)
+IV2_DEV void scale_mask(float (&acc)[8][4], float sl2, uint64_t valid)
+{
+    const int tq = threadIdx.x & 3;
+#pragma unroll
+    for (int nt = 0; nt < 8; ++nt)
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+            const int col = nt * 8 + 2 * tq + e;
+            const bool ok = (valid >> col) & 1ull;
+            acc[nt][e] = ok ? acc[nt][e] * sl2 : neg_inf();
+            acc[nt][2 + e] = ok ? acc[nt][2 + e] * sl2 : neg_inf();
+        }
+}
+
+IV2_DEV uint64_t prefix_mask64(int nvalid)
+{
+    return nvalid >= 64 ? ~0ull : (nvalid <= 0 ? 0ull : ((1ull << nvalid) - 1ull));
+}
+
+// the k-th block of a row's list; -1 when absent or invalid
+IV2_DEV int row_block(bool dense, int c, const int32_t* idx_row, int count, int k, int n)
+{
+    if (dense) return k <= c ? k : -1;
+    if (k >= count) return -1;
+    const int blk = idx_row[k];
+    return (blk >= 0 && blk * kBlock < n) ? blk : -1;
+}
+
+// finalise the row sums across the 4 lanes of a row
+template <int D>
+IV2_DEV void finalize_rows(WarpAttnState<D>& st)
+{
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+        st.l[i] += __shfl_xor_sync(0xffffffffu, st.l[i], 1);
+        st.l[i] += __shfl_xor_sync(0xffffffffu, st.l[i], 2);
+    }
+}
+
+// =====================================================================================================
+// prefill: one warp per (token, group) row
+// =====================================================================================================
+constexpr int kRowWarps = 4;
+
+template <int D>
+__global__ void __launch_bounds__(kRowWarps * 32) attn_rows_kernel(QueryRows qr, const __nv_bfloat16* __restrict__ k,
+                                                                   const __nv_bfloat16* __restrict__ v, int Lcap,
+                                                                   const int32_t* __restrict__ idx,
+                                                                   const int32_t* __restrict__ cnt, MethodConsts mc,
+                                                                   int dense_all, __nv_bfloat16* __restrict__ out,
+                                                                   float* __restrict__ lse)
+{
+    extern __shared__ __align__(128) unsigned char smem[];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, gq = lane >> 2, tq = lane & 3;
+    const long row = (long)blockIdx.x * kRowWarps + warp;
+    const int rows = qr.B * qr.T * qr.Hkv;
+    if (row >= rows) return;
+    unsigned char* ks_tile = smem + warp * 2 * KvTile<D>::kBytes;
+    unsigned char* vs_tile = ks_tile + KvTile<D>::kBytes;
+
+    const int g = (int)(row % qr.Hkv);
+    const long bt = row / qr.Hkv;
+    const int t = (int)(bt % qr.T), b = (int)(bt / qr.T);
+    const int G = qr.Hq / qr.Hkv;
+    const int n = query_ctx(qr, b, t);
+    const int c = (n - 1) / kBlock;
+    const bool dense = dense_all || n <= mc.dense_len;
+    const int count = dense ? c + 1 : min(cnt[row], mc.kmax);
+    const int32_t* idx_row = idx ? idx + row * mc.kmax : nullptr;
+
+    uint32_t qf[D / 16][4];
+    load_q_rows<D>(static_cast<const __nv_bfloat16*>(qr.q) + ((size_t)bt * qr.Hq + g * G) * D, G, qf);
+    const size_t rs = (size_t)qr.Hkv * D;
+    const __nv_bfloat16* kb = k + ((size_t)b * Lcap * qr.Hkv + g) * D;
+    const __nv_bfloat16* vb = v + ((size_t)b * Lcap * qr.Hkv + g) * D;
+    const float sl2 = mc.scale * kLog2e;
+
+    WarpAttnState<D> st;
+    st.init();
+    // first valid block
+    int kpos = 0, blk = -1;
+    while (kpos < count && (blk = row_block(dense, c, idx_row, count, kpos, n)) < 0) ++kpos;
+    if (blk >= 0) {
+        warp_load_tile<D>(ks_tile, kb + (size_t)blk * kBlock * rs, rs, min(kBlock, n - blk * kBlock));
+        cp_async_commit();
+        warp_load_tile<D>(vs_tile, vb + (size_t)blk * kBlock * rs, rs, min(kBlock, n - blk * kBlock));
+        cp_async_commit();
+    }
+    while (blk >= 0) {
+        int knext = kpos + 1, nblk = -1;
+        while (knext < count && (nblk = row_block(dense, c, idx_row, count, knext, n)) < 0) ++knext;
+        cp_async_wait<1>();  // K of blk
+        __syncwarp();
+        float acc[8][4];
+        tile_qk<D>(qf, ks_tile, acc);
+        scale_mask(acc, sl2, prefix_mask64(n - blk * kBlock));
+        __syncwarp();
+        if (nblk >= 0)
+            warp_load_tile<D>(ks_tile, kb + (size_t)nblk * kBlock * rs, rs, min(kBlock, n - nblk * kBlock));
+        cp_async_commit();
+        cp_async_wait<1>();  // V of blk
+        __syncwarp();
+        tile_softmax_pv<D>(st, acc, vs_tile);
+        __syncwarp();
+        if (nblk >= 0)
+            warp_load_tile<D>(vs_tile, vb + (size_t)nblk * kBlock * rs, rs, min(kBlock, n - nblk * kBlock));
+        cp_async_commit();
+        blk = nblk;
+        kpos = knext;
+    }
+    cp_async_wait<0>();
+    finalize_rows<D>(st);
+
+    // write rows gq, gq+8 (heads < G)
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+        const int r = gq + 8 * i;
+        if (r >= G) continue;
+        const float inv = st.l[i] > 0.f ? 1.f / st.l[i] : 0.f;
+        __nv_bfloat16* orow = out + ((size_t)bt * qr.Hq + g * G + r) * D;
+#pragma unroll
+        for (int nd = 0; nd < D / 8; ++nd)
+            *reinterpret_cast<uint32_t*>(orow + nd * 8 + 2 * tq) =
+                pack_bf16(st.o[nd][2 * i] * inv, st.o[nd][2 * i + 1] * inv);
+        if (lse && tq == 0)
+            lse[(size_t)bt * qr.Hq + g * G + r] = st.l[i] > 0.f ? (st.m[i] + __log2f(st.l[i])) * kLn2 : neg_inf();
+    }
+}
+
+// =====================================================================================================
+// decode / tree: split over the block list, merged by LSE
+// =====================================================================================================
+constexpr int kSplitWarps = 4;
+
+int attn_split_count(int max_blocks) { return (max_blocks + kSplitWarps - 1) / kSplitWarps; }
+
+int attn_split_max_blocks(int max_ctx, int kmax, int dense_len, bool dense_all)
+{
+    const int all_blocks = (max_ctx + kBlock - 1) / kBlock;
+    if (dense_all) return all_blocks;
+    const int dense_blocks = (min(max_ctx, dense_len) + kBlock - 1) / kBlock;
+    return min(all_blocks, max(kmax, dense_blocks));
+}
+
+template <int D>
+struct SplitWs {
+    static constexpr int kFloats = 16 * D + 32;  // O[16][D], m[16], l[16]
+};
+
+size_t attn_ws_bytes(int rows, int nsplit) { return ((size_t)rows * nsplit * SplitWs<128>::kFloats * 4 + 255) / 256 * 256; }
+
+template <int D>
+__global__ void __launch_bounds__(kSplitWarps * 32) attn_split_kernel(
+    QueryRows qr, const __nv_bfloat16* __restrict__ k, const __nv_bfloat16* __restrict__ v, int Lcap,
+    const int32_t* __restrict__ idx, const int32_t* __restrict__ cnt, MethodConsts mc, int dense_all, int nsplit_blocks,
+    const __nv_bfloat16* __restrict__ k_draft, const __nv_bfloat16* __restrict__ v_draft,
+    const uint32_t* __restrict__ tree_mask, float* __restrict__ ws)
+{
+    extern __shared__ __align__(128) unsigned char smem[];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, gq = lane >> 2, tq = lane & 3;
+    const int row = blockIdx.y;
+    const int split = blockIdx.x;
+    const int nsplit_total = gridDim.x;
+    unsigned char* ks_tile = smem + warp * 2 * KvTile<D>::kBytes;
+    unsigned char* vs_tile = ks_tile + KvTile<D>::kBytes;
+
+    const int g = row % qr.Hkv, bt = row / qr.Hkv, t = bt % qr.T, b = bt / qr.T;
+    const int G = qr.Hq / qr.Hkv;
+    const int n = query_ctx(qr, b, t);
+    const int c = (n - 1) / kBlock;
+    const bool dense = dense_all || n <= mc.dense_len;
+    const int count = dense ? c + 1 : min(cnt[row], mc.kmax);
+    const int32_t* idx_row = idx ? idx + (size_t)row * mc.kmax : nullptr;
+    const float sl2 = mc.scale * kLog2e;
+
+    WarpAttnState<D> st;
+    st.init();
+    const bool draft_split = tree_mask != nullptr && split == nsplit_blocks;
+    int blk = -1;
+    bool work = false;
+    uint64_t valid = 0;
+    if (draft_split) {
+        if (warp == 0) {
+            // draft keys j < T of this sequence, visible when bit j of the node's mask is set
+            const uint32_t msk = tree_mask[bt];
+            valid = (uint64_t)msk & prefix_mask64(qr.T);
+            const size_t rs = (size_t)qr.Hkv * D;
+            const size_t base = ((size_t)b * qr.T * qr.Hkv + g) * D;
+            warp_load_tile<D>(ks_tile, k_draft + base, rs, qr.T);
+            warp_load_tile<D>(vs_tile, v_draft + base, rs, qr.T);
+            cp_async_commit();
+            work = true;
+        }
+    } else {
+        blk = row_block(dense, c, idx_row, count, split * kSplitWarps + warp, n);
+        if (blk >= 0) {
+            const size_t rs = (size_t)qr.Hkv * D;
+            const size_t base = ((size_t)b * Lcap * qr.Hkv + g) * D + (size_t)blk * kBlock * rs;
+            const int nvalid = min(kBlock, n - blk * kBlock);
+            warp_load_tile<D>(ks_tile, k + base, rs, nvalid);
+            warp_load_tile<D>(vs_tile, v + base, rs, nvalid);
+            cp_async_commit();
+            valid = prefix_mask64(nvalid);
+            work = true;
+        }
+    }
+    if (work) {
+        uint32_t qf[D / 16][4];
+        load_q_rows<D>(static_cast<const __nv_bfloat16*>(qr.q) + ((size_t)bt * qr.Hq + g * G) * D, G, qf);
+        cp_async_wait<0>();
+        __syncwarp();
+        float acc[8][4];
+        tile_qk<D>(qf, ks_tile, acc);
+        scale_mask(acc, sl2, valid);
+        tile_softmax_pv<D>(st, acc, vs_tile);
+        finalize_rows<D>(st);
+    }
+    __syncthreads();  // tiles are dead: reuse shared memory for the CTA merge
+
+    // per-warp results to shared memory: O [warp][16][D], m/l [warp][16]
+    float* so = reinterpret_cast<float*>(smem);
+    float* sm = so + kSplitWarps * 16 * D;
+    float* sl = sm + kSplitWarps * 16;
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+        const int r = gq + 8 * i;
+#pragma unroll
+        for (int nd = 0; nd < D / 8; ++nd) {
+            so[(warp * 16 + r) * D + nd * 8 + 2 * tq] = st.o[nd][2 * i];
+            so[(warp * 16 + r) * D + nd * 8 + 2 * tq + 1] = st.o[nd][2 * i + 1];
+        }
+        if (tq == 0) {
+            sm[warp * 16 + r] = work ? st.m[i] : neg_inf();
+            sl[warp * 16 + r] = work ? st.l[i] : 0.f;
+        }
+    }
+    __syncthreads();
+    float* wsp = ws + ((size_t)row * nsplit_total + split) * SplitWs<D>::kFloats;
+    for (int item = threadIdx.x; item < G * D; item += kSplitWarps * 32) {
+        const int r = item / D, d = item % D;
+        float M = neg_inf();
+#pragma unroll
+        for (int w = 0; w < kSplitWarps; ++w) M = fmaxf(M, sm[w * 16 + r]);
+        float O = 0.f, L = 0.f;
+        if (M != neg_inf()) {
+#pragma unroll
+            for (int w = 0; w < kSplitWarps; ++w) {
+                const float f = exp2_fast(sm[w * 16 + r] - M);
+                O += so[(w * 16 + r) * D + d] * f;
+                L += sl[w * 16 + r] * f;
+            }
+        }
+        wsp[r * D + d] = O;
+        if (d == 0) {
+            wsp[16 * D + r] = M;
+            wsp[16 * D + 16 + r] = L;
+        }
+    }
+}
+
+template <int D>
+__global__ void __launch_bounds__(128) attn_merge_kernel(QueryRows qr, int nsplit_total, const float* __restrict__ ws,
+                                                         __nv_bfloat16* __restrict__ out, float* __restrict__ lse)
+{
+    const int row = blockIdx.x;
+    const int g = row % qr.Hkv, bt = row / qr.Hkv;
+    const int G = qr.Hq / qr.Hkv;
+    const float* base = ws + (size_t)row * nsplit_total * SplitWs<D>::kFloats;
+    for (int item = threadIdx.x; item < G * D; item += 128) {
+        const int r = item / D, d = item % D;
+        float M = neg_inf();
+        for (int s = 0; s < nsplit_total; ++s) M = fmaxf(M, base[(size_t)s * SplitWs<D>::kFloats + 16 * D + r]);
+        float O = 0.f, L = 0.f;
+        if (M != neg_inf()) {
+            for (int s = 0; s < nsplit_total; ++s) {
+                const float* p = base + (size_t)s * SplitWs<D>::kFloats;
+                const float f = exp2_fast(p[16 * D + r] - M);
+                O += p[r * D + d] * f;
+                L += p[16 * D + 16 + r] * f;
+            }
+        }
+        out[((size_t)bt * qr.Hq + g * G + r) * D + d] = __float2bfloat16_rn(L > 0.f ? O / L : 0.f);
+        if (lse && d == 0) lse[(size_t)bt * qr.Hq + g * G + r] = L > 0.f ? (M + __log2f(L)) * kLn2 : neg_inf();
+    }
+}
+
+// =====================================================================================================
+// host side
+// =====================================================================================================
+template <int D>
+static cudaError_t rows_impl(const QueryRows& qr, const void* k, const void* v, int Lcap, const int32_t* idx,
+                             const int32_t* cnt, const MethodConsts& mc, bool dense_all, void* out, float* lse,
+                             cudaStream_t s)
+{
+    const size_t smem = (size_t)kRowWarps * 2 * KvTile<D>::kBytes;
+    cudaError_t e = cudaFuncSetAttribute(attn_rows_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    const long rows = (long)qr.B * qr.T * qr.Hkv;
+    const unsigned grid = (unsigned)((rows + kRowWarps - 1) / kRowWarps);
+    attn_rows_kernel<D><<<grid, kRowWarps * 32, smem, s>>>(qr, static_cast<const __nv_bfloat16*>(k),
+                                                           static_cast<const __nv_bfloat16*>(v), Lcap, idx, cnt, mc,
+                                                           dense_all ? 1 : 0, static_cast<__nv_bfloat16*>(out), lse);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_attn_rows(const QueryRows& qr, const void* k, const void* v, int Lcap, const int32_t* idx,
+                             const int32_t* cnt, const MethodConsts& mc, bool dense_all, void* out, float* lse,
+                             cudaStream_t s)
+{
+    return qr.D == 128 ? rows_impl<128>(qr, k, v, Lcap, idx, cnt, mc, dense_all, out, lse, s)
+                       : rows_impl<64>(qr, k, v, Lcap, idx, cnt, mc, dense_all, out, lse, s);
+}
+
+template <int D>
+static cudaError_t split_impl(const QueryRows& qr, const void* k, const void* v, int Lcap, const int32_t* idx,
+                              const int32_t* cnt, const MethodConsts& mc, bool dense_all, const void* k_draft,
+                              const void* v_draft, const uint32_t* tree_mask, void* out, float* lse, void* ws,
+                              cudaStream_t s)
+{
+    const int max_blocks = attn_split_max_blocks(qr.max_ctx, mc.kmax, mc.dense_len, dense_all);
+    const int nsplit_blocks = attn_split_count(max_blocks);
+    const int nsplit_total = nsplit_blocks + (tree_mask ? 1 : 0);
+    const size_t smem = (size_t)kSplitWarps * 2 * KvTile<D>::kBytes;
+    cudaError_t e = cudaFuncSetAttribute(attn_split_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    const int rows = qr.B * qr.T * qr.Hkv;
+    dim3 grid(nsplit_total, rows);
+    attn_split_kernel<D><<<grid, kSplitWarps * 32, smem, s>>>(
+        qr, static_cast<const __nv_bfloat16*>(k), static_cast<const __nv_bfloat16*>(v), Lcap, idx, cnt, mc,
+        dense_all ? 1 : 0, nsplit_blocks, static_cast<const __nv_bfloat16*>(k_draft),
+        static_cast<const __nv_bfloat16*>(v_draft), tree_mask, static_cast<float*>(ws));
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    attn_merge_kernel<D><<<rows, 128, 0, s>>>(qr, nsplit_total, static_cast<const float*>(ws),
+                                              static_cast<__nv_bfloat16*>(out), lse);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_attn_split(const QueryRows& qr, const void* k, const void* v, int Lcap, const int32_t* idx,
+                              const int32_t* cnt, const MethodConsts& mc, bool dense_all, const void* k_draft,
+                              const void* v_draft, const uint32_t* tree_mask, void* out, float* lse, void* ws,
+                              cudaStream_t s)
+{
+    return qr.D == 128 ? split_impl<128>(qr, k, v, Lcap, idx, cnt, mc, dense_all, k_draft, v_draft, tree_mask, out,
+                                         lse, ws, s)
+                       : split_impl<64>(qr, k, v, Lcap, idx, cnt, mc, dense_all, k_draft, v_draft, tree_mask, out,
+                                        lse, ws, s);
+}
+
+}  // namespace iv2

@@ -1,0 +1,61 @@
+// internal.h -- launchers shared between the C-ABI layer (api.cu) and the kernel files.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+namespace iv2 {
+
+// Resolved per-call description of a set of query rows.
+struct QueryRows {
+    const void* q;            // [B, T, Hq, d] bf16
+    int B, T, Hq, Hkv, D;
+    const int32_t* q_ctx;     // [B*T] or null
+    const int32_t* ctx_lens;  // [B] (used when q_ctx is null)
+    int same_ctx;             // q_ctx null: 1 -> every query of b sees ctx_lens[b] keys (tree drafts),
+                              //             0 -> causal tail, n = ctx_lens[b] - T + t + 1
+    int max_ctx;
+};
+
+// context length n of query (b, t)
+__host__ __device__ inline int query_ctx(const QueryRows& qr, int b, int t)
+{
+    if (qr.q_ctx) return qr.q_ctx[b * qr.T + t];
+    return qr.same_ctx ? qr.ctx_lens[b] : qr.ctx_lens[b] - qr.T + t + 1;
+}
+
+struct MethodConsts {
+    int topk, init_blocks, local_blocks, dense_len, membership;
+    float scale;              // softmax scale (natural units)
+    int kmax;                 // topk + init + local
+};
+
+// scoring path: true -> split-kernel scan + per-row select (needs workspace), false -> token tiles
+bool score_uses_scan_path(int B, int T, int G, int D, int max_ctx);
+// workspace bytes of the scan path / of the split attention (256-byte multiples)
+size_t score_ws_bytes(int rows, int max_ctx);
+size_t attn_ws_bytes(int rows, int nsplit);
+// CTAs per row of the split attention for a block list of max_blocks entries
+int attn_split_count(int max_blocks);
+// largest block list the split attention handles for these sizes
+int attn_split_max_blocks(int max_ctx, int kmax, int dense_len, bool dense_all);
+
+cudaError_t launch_kernel_pool(const void* k, int B, int Lcap, int Hkv, int D, const int32_t* old_lens,
+                               const int32_t* new_lens, int max_new_keys, void* kern, int nk_cap, cudaStream_t s);
+
+cudaError_t launch_score_topk(const QueryRows& qr, const void* kern, int nk_cap, const MethodConsts& mc,
+                              int32_t* idx, int32_t* cnt, void* ws, cudaStream_t s);
+
+// attention over selected blocks (or all blocks when dense_all); prefill style: one warp per query row
+cudaError_t launch_attn_rows(const QueryRows& qr, const void* k, const void* v, int Lcap, const int32_t* idx,
+                             const int32_t* cnt, const MethodConsts& mc, bool dense_all, void* out, float* lse,
+                             cudaStream_t s);
+
+// attention split over the selected blocks across CTAs, merged by LSE (decode and tree verification)
+cudaError_t launch_attn_split(const QueryRows& qr, const void* k, const void* v, int Lcap, const int32_t* idx,
+                              const int32_t* cnt, const MethodConsts& mc, bool dense_all, const void* k_draft,
+                              const void* v_draft, const uint32_t* tree_mask, void* out, float* lse, void* ws,
+                              cudaStream_t s);
+
+}  // namespace iv2

@@ -1,0 +1,97 @@
+// pool.cu -- semantic-kernel pooling (step 1 of InfLLM v2).
+//
+// kern[b, g, j, :] = bf16_rne( mean of k[b, i, g, :] over the 32-key window i in [16 j, 16 j + 32) )
+// for the windows completed between old_lens[b] and new_lens[b] keys ("Tsinghua & ModelBest: MiniCPM4
+// technical details", "Model architecture: InfLLM v2", item 1: every block is made of several
+// fine-grained semantic kernels; the pages give no window size).
+//
+// HBM-bound: every key row is read once.  A window of 32 keys is the sum of two 16-key half windows
+// that it shares with its neighbours, so each CTA first sums 33 half windows (fp32) into shared memory
+// and then forms 32 kernels from adjacent pairs.  Rows are 16-byte coalesced loads (d = 128: 16 lanes
+// cover one 256-byte row), and all 16 rows of a half window are in flight per thread.
+#include "common.cuh"
+#include "internal.h"
+
+namespace iv2 {
+
+constexpr int kPoolKernelsPerCta = 32;
+constexpr int kPoolThreads = 256;
+
+template <int D>
+__global__ void __launch_bounds__(kPoolThreads) kernel_pool_kernel(const __nv_bfloat16* __restrict__ k, int Lcap,
+                                                                   int Hkv, const int32_t* __restrict__ old_lens,
+                                                                   const int32_t* __restrict__ new_lens,
+                                                                   __nv_bfloat16* __restrict__ kern, int nk_cap)
+{
+    constexpr int CH = D / 8;                  // 16-byte chunks per row
+    constexpr int HALVES = kPoolKernelsPerCta + 1;
+    __shared__ float hs[HALVES][D];
+
+    const int bg = blockIdx.y;
+    const int b = bg / Hkv, g = bg % Hkv;
+    const int n_old = old_lens[b], n_new = new_lens[b];
+    const int j_begin = num_kernels(n_old) + blockIdx.x * kPoolKernelsPerCta;
+    const int j_end = min(num_kernels(n_new), j_begin + kPoolKernelsPerCta);
+    if (j_begin >= j_end || j_end > nk_cap) return;
+
+    const size_t row_stride = (size_t)Hkv * D;
+    const __nv_bfloat16* kb = k + ((size_t)b * Lcap * Hkv + g) * D;
+    const int n_halves = j_end - j_begin + 1;  // half windows j_begin .. j_end
+
+    // half-window sums: item = (half h, chunk c)
+    for (int item = threadIdx.x; item < n_halves * CH; item += kPoolThreads) {
+        const int h = item / CH, c = item % CH;
+        const int row0 = (j_begin + h) * kKernelStride;
+        float acc[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) acc[e] = 0.f;
+        uint4 buf[kKernelStride];
+#pragma unroll
+        for (int r = 0; r < kKernelStride; ++r) buf[r] = ld_nc_v4(kb + (size_t)(row0 + r) * row_stride + c * 8);
+#pragma unroll
+        for (int r = 0; r < kKernelStride; ++r) {
+            const uint32_t w[4] = {buf[r].x, buf[r].y, buf[r].z, buf[r].w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                acc[2 * e] += bf16_lo(w[e]);
+                acc[2 * e + 1] += bf16_hi(w[e]);
+            }
+        }
+#pragma unroll
+        for (int e = 0; e < 8; ++e) hs[h][c * 8 + e] = acc[e];
+    }
+    __syncthreads();
+
+    constexpr float inv = 1.0f / kKernelSize;  // a power of two: the scaling is exact
+    for (int item = threadIdx.x; item < (j_end - j_begin) * CH; item += kPoolThreads) {
+        const int jj = item / CH, c = item % CH;
+        uint32_t w[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            const float lo = (hs[jj][c * 8 + 2 * e] + hs[jj + 1][c * 8 + 2 * e]) * inv;
+            const float hi = (hs[jj][c * 8 + 2 * e + 1] + hs[jj + 1][c * 8 + 2 * e + 1]) * inv;
+            w[e] = pack_bf16(lo, hi);
+        }
+        __nv_bfloat16* dst = kern + (((size_t)b * Hkv + g) * nk_cap + j_begin + jj) * D + c * 8;
+        *reinterpret_cast<uint4*>(dst) = make_uint4(w[0], w[1], w[2], w[3]);
+    }
+}
+
+cudaError_t launch_kernel_pool(const void* k, int B, int Lcap, int Hkv, int D, const int32_t* old_lens,
+                               const int32_t* new_lens, int max_new_keys, void* kern, int nk_cap, cudaStream_t s)
+{
+    // windows completed by appending max_new_keys keys: at most max_new_keys / 16 + 1
+    const int max_new_kernels = max_new_keys / kKernelStride + 1;
+    dim3 grid((max_new_kernels + kPoolKernelsPerCta - 1) / kPoolKernelsPerCta, B * Hkv);
+    if (D == 128)
+        kernel_pool_kernel<128><<<grid, kPoolThreads, 0, s>>>(static_cast<const __nv_bfloat16*>(k), Lcap, Hkv,
+                                                              old_lens, new_lens,
+                                                              static_cast<__nv_bfloat16*>(kern), nk_cap);
+    else
+        kernel_pool_kernel<64><<<grid, kPoolThreads, 0, s>>>(static_cast<const __nv_bfloat16*>(k), Lcap, Hkv,
+                                                             old_lens, new_lens, static_cast<__nv_bfloat16*>(kern),
+                                                             nk_cap);
+    return cudaGetLastError();
+}
+
+}  // namespace iv2
