@@ -246,3 +246,32 @@ def test_end_to_end_tiny_prefill(oracle):
     torch.cuda.synchronize()
     row_same = same.all(axis=-1)  # [B, T]: both groups match
     check_attention(out, out_o, mask=row_same, what="end-to-end")
+
+
+@pytest.mark.parametrize("path", ["scan_few_members", "scan_degenerate", "tile"])
+def test_selection_ties_go_to_lower_block(oracle, path):
+    """A zero query scores every block identically: the top-k must be the lowest candidate ids, exactly
+    (no near-tie excuse here)."""
+    if path == "tile":
+        w = prefill_case(2000, 32, 2, 128, topk=16, dense_len=0, seed=900, n_needles=0)
+    else:
+        L = 131000 if path == "scan_degenerate" else 3000
+        w = decode_case([L, 2000], 32, 2, 128, topk=64, dense_len=0, seed=901, n_needles=0)
+    w.q[:] = 0
+    n_all = w.q_ctx.reshape(-1)
+    nk_cap = oracle.num_kernels(int(n_all.max()))
+    B = w.k.shape[0]
+    kern = gpu_pool(w.k, [0] * B, list(w.ctx_lens), int(w.ctx_lens.max()), nk_cap)
+    gidx, gcnt = gpu_select(w, kern)
+    k = w.params["topk"]
+    for b in range(B):
+        for t in range(0, w.q.shape[1], 97):
+            n = int(w.q_ctx[b, t])
+            c = (n - 1) // 64
+            cand = [x for x in range(1, c - 1)]
+            want = sorted({0, c - 1, c} | set(cand[:k])) if c >= 1 else [0]
+            for g in range(2):
+                assert list(gidx[b, t, g, :gcnt[b, t, g]]) == want, (b, t, g)
+    kern_o = oracle.kernel_pool(w.k, [0] * B, list(w.ctx_lens), 32, 16, nk_cap=nk_cap)
+    r = oracle.block_score_topk(w.q, kern_o, w.q_ctx, oparams(w.params))
+    assert np.array_equal(r["idx"], gidx) and np.array_equal(r["cnt"], gcnt)

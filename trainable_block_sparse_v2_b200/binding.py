@@ -251,8 +251,8 @@ def num_kernels(n: int, kernel_size: int = 32, kernel_stride: int = 16) -> int:
 
 
 def workspace(params: Params, batch, max_q, max_ctx, hq, hkv, head_dim, device="cuda"):
-    """Allocate (with torch) a workspace of infllmv2_workspace_size bytes, 256-byte aligned."""
+    """Allocate (with torch) a zero-filled workspace of infllmv2_workspace_size bytes, 256-byte aligned."""
     n = infllmv2_workspace_size(params, batch, max_q, max_ctx, hq, hkv, head_dim)
     if n == 0:
         raise Infllmv2Error("infllmv2_workspace_size", 1, "invalid sizes")
-    return torch.empty(math.ceil(n / 256) * 256, dtype=torch.uint8, device=device)
+    return torch.zeros(math.ceil(n / 256) * 256, dtype=torch.uint8, device=device)

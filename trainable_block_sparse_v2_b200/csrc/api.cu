@@ -5,10 +5,36 @@
 // memory and keeps no state between calls.
 #include <cmath>
 #include <cstdint>
+#include <mutex>
 
 #include "../../include/infllmv2.h"
 #include "common.cuh"
 #include "internal.h"
+
+namespace iv2 {
+
+cudaError_t ensure_smem_impl(const void* func, size_t bytes)
+{
+    struct Entry {
+        const void* func;
+        int dev;
+        size_t bytes;
+    };
+    static Entry table[256];
+    static int n = 0;
+    static std::mutex mu;
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    std::lock_guard<std::mutex> lock(mu);
+    for (int i = 0; i < n; ++i)
+        if (table[i].func == func && table[i].dev == dev && table[i].bytes >= bytes) return cudaSuccess;
+    e = cudaFuncSetAttribute(func, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+    if (e == cudaSuccess && n < 256) table[n++] = Entry{func, dev, bytes};
+    return e;
+}
+
+}  // namespace iv2
 
 using iv2::MethodConsts;
 using iv2::QueryRows;
@@ -243,6 +269,7 @@ int infllmv2_sparse_attn_decode(const void* q, int batch, int hq, int hkv, int h
     IV2_TRY(check_opt4(lse));
     IV2_TRY(check_ctx(max_ctx, lcap));
     const MethodConsts mc = consts_of(params, head_dim);
+    if (batch * hkv > iv2::kMaxSplitRows) return INFLLMV2_ERR_UNSUPPORTED;
     IV2_TRY(check_ws(ws, ws_bytes, split_need(batch * hkv, max_ctx, mc.kmax, mc.dense_len, false, false)));
     const QueryRows qr = rows_of(q, batch, 1, hq, hkv, head_dim, nullptr, ctx_lens, 0, max_ctx);
     return launched(iv2::launch_attn_split(qr, k, v, lcap, idx, cnt, mc, false, nullptr, nullptr, nullptr, out, lse,
@@ -271,6 +298,7 @@ int infllmv2_sparse_attn_tree_verify(const void* q, int batch, int n_draft, int 
     IV2_TRY(check_opt4(lse));
     IV2_TRY(check_ctx(max_ctx, lcap));
     const MethodConsts mc = consts_of(params, head_dim);
+    if (batch * n_draft * hkv > iv2::kMaxSplitRows) return INFLLMV2_ERR_UNSUPPORTED;
     IV2_TRY(check_ws(ws, ws_bytes, split_need(batch * n_draft * hkv, max_ctx, mc.kmax, mc.dense_len, false, true)));
     const QueryRows qr = rows_of(q, batch, n_draft, hq, hkv, head_dim, nullptr, prefix_lens, 1, max_ctx);
     return launched(iv2::launch_attn_split(qr, k, v, lcap, idx, cnt, mc, false, k_draft, v_draft, tree_mask, out, lse,
@@ -314,6 +342,7 @@ int infllmv2_dense_attn_decode(const void* q, int batch, int hq, int hkv, int he
     IV2_TRY(check_opt4(lse));
     IV2_TRY(check_ctx(max_ctx, lcap));
     const MethodConsts mc = dense_consts(softmax_scale, head_dim);
+    if (batch * hkv > iv2::kMaxSplitRows) return INFLLMV2_ERR_UNSUPPORTED;
     IV2_TRY(check_ws(ws, ws_bytes, split_need(batch * hkv, max_ctx, mc.kmax, 0, true, false)));
     const QueryRows qr = rows_of(q, batch, 1, hq, hkv, head_dim, nullptr, ctx_lens, 0, max_ctx);
     return launched(iv2::launch_attn_split(qr, k, v, lcap, nullptr, nullptr, mc, true, nullptr, nullptr, nullptr, out,

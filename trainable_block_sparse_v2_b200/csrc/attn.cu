@@ -14,8 +14,9 @@
 // / running sum) form in log2 units.
 //  * prefill: one warp per (token, group) row walks the row's whole block list.
 //  * decode / tree: the block list of a row is split across CTAs (4 blocks per CTA, one per warp); each
-//    CTA merges its warps and writes (max, sum, unnormalised O) to the workspace; a merge kernel combines
-//    the splits by their LSE.  Tree rows get one extra split that attends to the draft tile.
+//    CTA merges its warps and writes (max, sum, unnormalised O) to the workspace; a merge kernel (one CTA
+//    per row and head) combines the splits by their LSE.  Tree rows get one extra split that attends to
+//    the draft tile.
 #include "common.cuh"
 #include "internal.h"
 
@@ -204,6 +205,8 @@ __global__ void __launch_bounds__(kRowWarps * 32) attn_rows_kernel(QueryRows qr,
                                                                    int dense_all, __nv_bfloat16* __restrict__ out,
                                                                    float* __restrict__ lse)
 {
+    pdl_launch_dependents();
+    pdl_wait();
     extern __shared__ __align__(128) unsigned char smem[];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, gq = lane >> 2, tq = lane & 3;
     const long row = (long)blockIdx.x * kRowWarps + warp;
@@ -301,7 +304,10 @@ struct SplitWs {
     static constexpr int kFloats = 16 * D + 32;  // O[16][D], m[16], l[16]
 };
 
-size_t attn_ws_bytes(int rows, int nsplit) { return ((size_t)rows * nsplit * SplitWs<128>::kFloats * 4 + 255) / 256 * 256; }
+size_t attn_ws_bytes(int rows, int nsplit)
+{
+    return ((size_t)rows * nsplit * SplitWs<128>::kFloats * 4 + 255) / 256 * 256;
+}
 
 template <int D>
 __global__ void __launch_bounds__(kSplitWarps * 32) attn_split_kernel(
@@ -310,6 +316,8 @@ __global__ void __launch_bounds__(kSplitWarps * 32) attn_split_kernel(
     const __nv_bfloat16* __restrict__ k_draft, const __nv_bfloat16* __restrict__ v_draft,
     const uint32_t* __restrict__ tree_mask, float* __restrict__ ws)
 {
+    pdl_launch_dependents();
+    pdl_wait();
     extern __shared__ __align__(128) unsigned char smem[];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, gq = lane >> 2, tq = lane & 3;
     const int row = blockIdx.y;
@@ -327,9 +335,10 @@ __global__ void __launch_bounds__(kSplitWarps * 32) attn_split_kernel(
     const int32_t* idx_row = idx ? idx + (size_t)row * mc.kmax : nullptr;
     const float sl2 = mc.scale * kLog2e;
 
+    const bool draft_split = tree_mask != nullptr && split == nsplit_blocks;
+    if (!draft_split && split * kSplitWarps >= count) return;  // no block for this CTA: the merge skips it
     WarpAttnState<D> st;
     st.init();
-    const bool draft_split = tree_mask != nullptr && split == nsplit_blocks;
     int blk = -1;
     bool work = false;
     uint64_t valid = 0;
@@ -412,30 +421,65 @@ __global__ void __launch_bounds__(kSplitWarps * 32) attn_split_kernel(
     }
 }
 
+// one CTA per (row, head); thread d owns output column d.  Only the splits that received blocks (and the
+// draft split of a tree row) are read.
 template <int D>
-__global__ void __launch_bounds__(128) attn_merge_kernel(QueryRows qr, int nsplit_total, const float* __restrict__ ws,
-                                                         __nv_bfloat16* __restrict__ out, float* __restrict__ lse)
+__global__ void __launch_bounds__(D) attn_merge_kernel(QueryRows qr, const int32_t* __restrict__ cnt, MethodConsts mc,
+                                                       int dense_all, int nsplit_blocks, int has_draft,
+                                                       const float* __restrict__ ws, __nv_bfloat16* __restrict__ out,
+                                                       float* __restrict__ lse)
 {
-    const int row = blockIdx.x;
-    const int g = row % qr.Hkv, bt = row / qr.Hkv;
+    pdl_launch_dependents();
+    pdl_wait();
+    constexpr int kMaxSplits = 1024;
+    __shared__ float fac[kMaxSplits];
+    __shared__ float red[D / 32];
+    const int row = blockIdx.x, r = blockIdx.y;
+    const int g = row % qr.Hkv, bt = row / qr.Hkv, t = bt % qr.T, b = bt / qr.T;
     const int G = qr.Hq / qr.Hkv;
+    const int n = query_ctx(qr, b, t);
+    const int c = (n - 1) / kBlock;
+    const bool dense = dense_all || n <= mc.dense_len;
+    const int count = dense ? c + 1 : min(cnt[row], mc.kmax);
+    const int nused = min((count + kSplitWarps - 1) / kSplitWarps, nsplit_blocks);
+    const int nsplit_total = nsplit_blocks + has_draft;
     const float* base = ws + (size_t)row * nsplit_total * SplitWs<D>::kFloats;
-    for (int item = threadIdx.x; item < G * D; item += 128) {
-        const int r = item / D, d = item % D;
-        float M = neg_inf();
-        for (int s = 0; s < nsplit_total; ++s) M = fmaxf(M, base[(size_t)s * SplitWs<D>::kFloats + 16 * D + r]);
-        float O = 0.f, L = 0.f;
-        if (M != neg_inf()) {
-            for (int s = 0; s < nsplit_total; ++s) {
-                const float* p = base + (size_t)s * SplitWs<D>::kFloats;
-                const float f = exp2_fast(p[16 * D + r] - M);
-                O += p[r * D + d] * f;
-                L += p[16 * D + 16 + r] * f;
-            }
-        }
-        out[((size_t)bt * qr.Hq + g * G + r) * D + d] = __float2bfloat16_rn(L > 0.f ? O / L : 0.f);
-        if (lse && d == 0) lse[(size_t)bt * qr.Hq + g * G + r] = L > 0.f ? (M + __log2f(L)) * kLn2 : neg_inf();
+    auto split_of = [&](int i) { return i < nused ? i : nsplit_blocks; };  // the draft split comes last
+    const int nread = min(nused + has_draft, kMaxSplits);
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+
+    float m_loc = neg_inf();
+    for (int i = threadIdx.x; i < nread; i += D) {
+        const float m = base[(size_t)split_of(i) * SplitWs<D>::kFloats + 16 * D + r];
+        fac[i] = m;
+        m_loc = fmaxf(m_loc, m);
     }
+    m_loc = warp_max(m_loc);
+    if (lane == 0) red[warp] = m_loc;
+    __syncthreads();
+    float M = neg_inf();
+#pragma unroll
+    for (int w = 0; w < D / 32; ++w) M = fmaxf(M, red[w]);
+    __syncthreads();
+    float l_loc = 0.f;
+    for (int i = threadIdx.x; i < nread; i += D) {
+        const float f = (M == neg_inf()) ? 0.f : exp2_fast(fac[i] - M);
+        fac[i] = f;
+        l_loc += f * base[(size_t)split_of(i) * SplitWs<D>::kFloats + 16 * D + 16 + r];
+    }
+    l_loc = warp_sum(l_loc);
+    __syncthreads();
+    if (lane == 0) red[warp] = l_loc;
+    __syncthreads();
+    float L = 0.f;
+#pragma unroll
+    for (int w = 0; w < D / 32; ++w) L += red[w];
+    const int d = threadIdx.x;
+    float O = 0.f;
+#pragma unroll 8
+    for (int i = 0; i < nread; ++i) O += fac[i] * base[(size_t)split_of(i) * SplitWs<D>::kFloats + r * D + d];
+    out[((size_t)bt * qr.Hq + g * G + r) * D + d] = __float2bfloat16_rn(L > 0.f ? O / L : 0.f);
+    if (lse && d == 0) lse[(size_t)bt * qr.Hq + g * G + r] = L > 0.f ? (M + __log2f(L)) * kLn2 : neg_inf();
 }
 
 // =====================================================================================================
@@ -447,14 +491,13 @@ static cudaError_t rows_impl(const QueryRows& qr, const void* k, const void* v, 
                              cudaStream_t s)
 {
     const size_t smem = (size_t)kRowWarps * 2 * KvTile<D>::kBytes;
-    cudaError_t e = cudaFuncSetAttribute(attn_rows_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    cudaError_t e = ensure_smem(attn_rows_kernel<D>, smem);
     if (e != cudaSuccess) return e;
     const long rows = (long)qr.B * qr.T * qr.Hkv;
     const unsigned grid = (unsigned)((rows + kRowWarps - 1) / kRowWarps);
-    attn_rows_kernel<D><<<grid, kRowWarps * 32, smem, s>>>(qr, static_cast<const __nv_bfloat16*>(k),
-                                                           static_cast<const __nv_bfloat16*>(v), Lcap, idx, cnt, mc,
-                                                           dense_all ? 1 : 0, static_cast<__nv_bfloat16*>(out), lse);
-    return cudaGetLastError();
+    return launch_pdl(attn_rows_kernel<D>, dim3(grid), dim3(kRowWarps * 32), smem, s, qr,
+                      static_cast<const __nv_bfloat16*>(k), static_cast<const __nv_bfloat16*>(v), Lcap, idx, cnt, mc,
+                      dense_all ? 1 : 0, static_cast<__nv_bfloat16*>(out), lse);
 }
 
 cudaError_t launch_attn_rows(const QueryRows& qr, const void* k, const void* v, int Lcap, const int32_t* idx,
@@ -475,19 +518,18 @@ static cudaError_t split_impl(const QueryRows& qr, const void* k, const void* v,
     const int nsplit_blocks = attn_split_count(max_blocks);
     const int nsplit_total = nsplit_blocks + (tree_mask ? 1 : 0);
     const size_t smem = (size_t)kSplitWarps * 2 * KvTile<D>::kBytes;
-    cudaError_t e = cudaFuncSetAttribute(attn_split_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    cudaError_t e = ensure_smem(attn_split_kernel<D>, smem);
     if (e != cudaSuccess) return e;
     const int rows = qr.B * qr.T * qr.Hkv;
     dim3 grid(nsplit_total, rows);
-    attn_split_kernel<D><<<grid, kSplitWarps * 32, smem, s>>>(
-        qr, static_cast<const __nv_bfloat16*>(k), static_cast<const __nv_bfloat16*>(v), Lcap, idx, cnt, mc,
-        dense_all ? 1 : 0, nsplit_blocks, static_cast<const __nv_bfloat16*>(k_draft),
-        static_cast<const __nv_bfloat16*>(v_draft), tree_mask, static_cast<float*>(ws));
-    e = cudaGetLastError();
+    e = launch_pdl(attn_split_kernel<D>, grid, dim3(kSplitWarps * 32), smem, s, qr,
+                   static_cast<const __nv_bfloat16*>(k), static_cast<const __nv_bfloat16*>(v), Lcap, idx, cnt, mc,
+                   dense_all ? 1 : 0, nsplit_blocks, static_cast<const __nv_bfloat16*>(k_draft),
+                   static_cast<const __nv_bfloat16*>(v_draft), tree_mask, static_cast<float*>(ws));
     if (e != cudaSuccess) return e;
-    attn_merge_kernel<D><<<rows, 128, 0, s>>>(qr, nsplit_total, static_cast<const float*>(ws),
-                                              static_cast<__nv_bfloat16*>(out), lse);
-    return cudaGetLastError();
+    return launch_pdl(attn_merge_kernel<D>, dim3(rows, qr.Hq / qr.Hkv), dim3(D), 0, s, qr, cnt, mc, dense_all ? 1 : 0,
+                      nsplit_blocks, tree_mask ? 1 : 0, static_cast<const float*>(ws),
+                      static_cast<__nv_bfloat16*>(out), lse);
 }
 
 cudaError_t launch_attn_split(const QueryRows& qr, const void* k, const void* v, int Lcap, const int32_t* idx,

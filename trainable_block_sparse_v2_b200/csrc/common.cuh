@@ -125,6 +125,13 @@ IV2_DEV float warp_sum(float v)
     return v;
 }
 
+// ---- programmatic dependent launch ---------------------------------------------------------------
+// Every kernel lets the next kernel of the stream start launching at once, and waits for the previous
+// kernel of the stream to finish (and its writes to be visible) before touching global memory.  The
+// wait is the hardware's grid dependency, not a spin loop.
+IV2_DEV void pdl_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+IV2_DEV void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
 // fast 2^x (MUFU) -- inputs are <= 0 or -inf on every use in this library
 IV2_DEV float exp2_fast(float x) { return exp2f(x); }
 

@@ -5,7 +5,59 @@
 #include <stddef.h>
 #include <stdint.h>
 
+#include <utility>
+
 namespace iv2 {
+
+// Raise a kernel's dynamic shared-memory limit once per (kernel, device), so that stream captures after
+// the first call see no attribute calls.  Returns the CUDA error of the attribute call.
+cudaError_t ensure_smem_impl(const void* func, size_t bytes);
+template <typename F>
+inline cudaError_t ensure_smem(F* func, size_t bytes)
+{
+    return ensure_smem_impl(reinterpret_cast<const void*>(func), bytes);
+}
+
+// Launch with programmatic stream serialization: the kernel may be scheduled while the previous kernel of
+// the stream is still running; it waits for it with griddepcontrol.wait (pdl_wait) before any global access.
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
+                              Args&&... args)
+{
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
+
+// The same with a thread-block cluster of `cluster_x` CTAs along x.
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_pdl_cluster(void (*kernel)(KArgs...), dim3 grid, dim3 block, int cluster_x, size_t smem,
+                                      cudaStream_t s, Args&&... args)
+{
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[2];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    attr[1].id = cudaLaunchAttributeClusterDimension;
+    attr[1].val.clusterDim.x = cluster_x;
+    attr[1].val.clusterDim.y = 1;
+    attr[1].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 2;
+    return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
 
 // Resolved per-call description of a set of query rows.
 struct QueryRows {
@@ -30,6 +82,9 @@ struct MethodConsts {
     float scale;              // softmax scale (natural units)
     int kmax;                 // topk + init + local
 };
+
+// rows (sequence x query x KV group) one split-attention launch handles
+constexpr int kMaxSplitRows = 1 << 16;
 
 // scoring path: true -> split-kernel scan + per-row select (needs workspace), false -> token tiles
 bool score_uses_scan_path(int B, int T, int G, int D, int max_ctx);

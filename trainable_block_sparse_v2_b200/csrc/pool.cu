@@ -23,6 +23,8 @@ __global__ void __launch_bounds__(kPoolThreads) kernel_pool_kernel(const __nv_bf
                                                                    const int32_t* __restrict__ new_lens,
                                                                    __nv_bfloat16* __restrict__ kern, int nk_cap)
 {
+    pdl_launch_dependents();
+    pdl_wait();
     constexpr int CH = D / 8;                  // 16-byte chunks per row
     constexpr int HALVES = kPoolKernelsPerCta + 1;
     __shared__ float hs[HALVES][D];
@@ -83,15 +85,13 @@ cudaError_t launch_kernel_pool(const void* k, int B, int Lcap, int Hkv, int D, c
     // windows completed by appending max_new_keys keys: at most max_new_keys / 16 + 1
     const int max_new_kernels = max_new_keys / kKernelStride + 1;
     dim3 grid((max_new_kernels + kPoolKernelsPerCta - 1) / kPoolKernelsPerCta, B * Hkv);
+    const auto* kp = static_cast<const __nv_bfloat16*>(k);
+    auto* kn = static_cast<__nv_bfloat16*>(kern);
     if (D == 128)
-        kernel_pool_kernel<128><<<grid, kPoolThreads, 0, s>>>(static_cast<const __nv_bfloat16*>(k), Lcap, Hkv,
-                                                              old_lens, new_lens,
-                                                              static_cast<__nv_bfloat16*>(kern), nk_cap);
-    else
-        kernel_pool_kernel<64><<<grid, kPoolThreads, 0, s>>>(static_cast<const __nv_bfloat16*>(k), Lcap, Hkv,
-                                                             old_lens, new_lens, static_cast<__nv_bfloat16*>(kern),
-                                                             nk_cap);
-    return cudaGetLastError();
+        return launch_pdl(kernel_pool_kernel<128>, grid, dim3(kPoolThreads), 0, s, kp, Lcap, Hkv, old_lens, new_lens,
+                          kn, nk_cap);
+    return launch_pdl(kernel_pool_kernel<64>, grid, dim3(kPoolThreads), 0, s, kp, Lcap, Hkv, old_lens, new_lens, kn,
+                      nk_cap);
 }
 
 }  // namespace iv2

@@ -10,7 +10,7 @@
 //
 // Two layouts of the same computation:
 //  * few query rows (decode, tree verification): the kernel cache is the HBM stream.  Each CTA scans a
-//    chunk of 64 blocks (256 kernels) of one row with mma.sync m16n8k16 (the G heads of the group are the
+//    chunk of 32 blocks (128 kernels) of one row with mma.sync m16n8k16 (the G heads of the group are the
 //    16 MMA rows), writing per-head partial (max, sum-exp) and raw block maxima; a second kernel merges
 //    the partials into LSE_h, forms S_g and selects, one CTA per row.  Kernel rows are loaded straight
 //    into MMA fragments with 16-byte loads: the head dimension is visited in a permuted order that is the
@@ -20,19 +20,23 @@
 //    for ldmatrix).  Pass 1 accumulates LSE_h online; pass 2 recomputes the scores, max-pools them into
 //    blocks, normalises, sums over the group and keeps S in shared memory; each warp then selects for
 //    its tokens.  No S or LSE ever goes to global memory.
+#include <cooperative_groups.h>
+
 #include "common.cuh"
 #include "internal.h"
 #include "select.cuh"
+
+namespace cg = cooperative_groups;
 
 namespace iv2 {
 
 // =====================================================================================================
 // few rows: split-kernel scan
 // =====================================================================================================
-constexpr int kChunkBlocks = 64;
-constexpr int kChunkKernels = kChunkBlocks * kKernelsPerBlock;   // 256 kernels owned per CTA
+constexpr int kChunkBlocks = 32;
+constexpr int kChunkKernels = kChunkBlocks * kKernelsPerBlock;   // 128 kernels owned per CTA
 constexpr int kChunkSlots = kChunkKernels + 8;                  // + halo kernel, rounded to n-tiles
-constexpr int kScanThreads = 256;
+constexpr int kScanThreads = 128;
 
 struct ScoreWs {
     float* pmax;   // [rows, nchunk, 16]
@@ -60,30 +64,12 @@ IV2_DEV void load_q_permuted(const __nv_bfloat16* q_row0, int nrows, uint32_t (&
     }
 }
 
-// z[16 rows x 8 kernels] for the 8 kernel rows starting at krow0 (row gq of this lane's load), permuted d
-template <int D>
-IV2_DEV void scores_8(const uint32_t (&qa)[D / 32][4], const uint32_t (&qb)[D / 32][4],
-                      const __nv_bfloat16* kern_row, bool row_ok, float (&c)[4])
-{
-    const int tq = threadIdx.x & 3;
-    uint4 kv[D / 32];
-#pragma unroll
-    for (int u = 0; u < D / 32; ++u)
-        kv[u] = row_ok ? ld_nc_v4(kern_row + (4 * u + tq) * 8) : make_uint4(0, 0, 0, 0);
-    c[0] = c[1] = c[2] = c[3] = 0.f;
-#pragma unroll
-    for (int u = 0; u < D / 32; ++u) {
-        const uint32_t a0[4] = {qa[u][0], qb[u][0], qa[u][1], qb[u][1]};
-        mma_bf16_16816(c, a0, kv[u].x, kv[u].y);
-        const uint32_t a1[4] = {qa[u][2], qb[u][2], qa[u][3], qb[u][3]};
-        mma_bf16_16816(c, a1, kv[u].z, kv[u].w);
-    }
-}
-
 template <int D>
 __global__ void __launch_bounds__(kScanThreads) score_scan_kernel(QueryRows qr, const __nv_bfloat16* __restrict__ kern,
                                                                   int nk_cap, MethodConsts mc, int nb_max, ScoreWs ws)
 {
+    pdl_launch_dependents();
+    pdl_wait();
     __shared__ float zs[16][kChunkSlots];
     const int row = blockIdx.y;  // (b, t, g)
     const int g = row % qr.Hkv, bt = row / qr.Hkv, t = bt % qr.T, b = bt / qr.T;
@@ -102,11 +88,31 @@ __global__ void __launch_bounds__(kScanThreads) score_scan_kernel(QueryRows qr, 
     const __nv_bfloat16* kbase = kern + ((size_t)b * qr.Hkv + g) * nk_cap * D;
     const float scale = mc.scale;
 
-    for (int tile = warp; tile < kChunkSlots / 8; tile += kScanThreads / 32) {
+    // tiles warp, warp + 4, ...: issue every kernel-row load of the warp first, then the MMAs
+    constexpr int kTiles = kChunkSlots / 8;                                            // 17
+    constexpr int kPerWarp = (kTiles + kScanThreads / 32 - 1) / (kScanThreads / 32);  // 5
+    uint4 kv[kPerWarp][D / 32];
+#pragma unroll
+    for (int i = 0; i < kPerWarp; ++i) {
+        const int tile = warp + i * (kScanThreads / 32);
         const int jr = j0 + tile * 8 + gq;  // the kernel row this lane loads
-        const bool ok = jr >= 0 && jr < nkv;
-        float acc[4];
-        scores_8<D>(qa, qb, kbase + (size_t)(ok ? jr : 0) * D, ok, acc);
+        const bool ok = tile < kTiles && jr >= 0 && jr < nkv;
+#pragma unroll
+        for (int u = 0; u < D / 32; ++u)
+            kv[i][u] = ok ? ld_nc_v4(kbase + (size_t)jr * D + (4 * u + tq) * 8) : make_uint4(0, 0, 0, 0);
+    }
+#pragma unroll
+    for (int i = 0; i < kPerWarp; ++i) {
+        const int tile = warp + i * (kScanThreads / 32);
+        if (tile >= kTiles) break;
+        float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int u = 0; u < D / 32; ++u) {
+            const uint32_t a0[4] = {qa[u][0], qb[u][0], qa[u][1], qb[u][1]};
+            mma_bf16_16816(acc, a0, kv[i][u].x, kv[i][u].y);
+            const uint32_t a1[4] = {qa[u][2], qb[u][2], qa[u][3], qb[u][3]};
+            mma_bf16_16816(acc, a1, kv[i][u].z, kv[i][u].w);
+        }
         const int col0 = tile * 8 + 2 * tq;
         const int ja = j0 + col0, jb = ja + 1;
         const bool va = ja >= 0 && ja < nkv, vb = jb >= 0 && jb < nkv;
@@ -118,7 +124,7 @@ __global__ void __launch_bounds__(kScanThreads) score_scan_kernel(QueryRows qr, 
     __syncthreads();
 
     const int nchunk = score_nchunk(nb_max);
-    // per-head partial LSE over the owned kernels (slots 1 .. 256)
+    // per-head partial LSE over the owned kernels (slots 1 .. kChunkKernels)
     for (int h = warp; h < G; h += kScanThreads / 32) {
         float m = neg_inf();
         for (int s = 1 + lane; s <= kChunkKernels; s += 32) m = fmaxf(m, zs[h][s]);
@@ -132,10 +138,11 @@ __global__ void __launch_bounds__(kScanThreads) score_scan_kernel(QueryRows qr, 
             ws.psum[((size_t)row * nchunk + blockIdx.x) * 16 + h] = sum;
         }
     }
-    // raw block maxima
+    // raw block maxima, head-major: bmax[row][h][blk] (consecutive threads write consecutive blocks)
     const int nblk = min(kChunkBlocks, c + 1 - cb0);
-    for (int item = threadIdx.x; item < G * nblk; item += kScanThreads) {
-        const int h = item / nblk, bl = item % nblk, blk = cb0 + bl;
+    for (int item = threadIdx.x; item < G * kChunkBlocks; item += kScanThreads) {
+        const int h = item / kChunkBlocks, bl = item % kChunkBlocks, blk = cb0 + bl;
+        if (bl >= nblk) continue;
         int lo, hi;
         block_kernel_range(blk, mc.membership, lo, hi);
         lo = max(lo, 0);
@@ -146,58 +153,85 @@ __global__ void __launch_bounds__(kScanThreads) score_scan_kernel(QueryRows qr, 
     }
 }
 
-constexpr int kSelThreads = 512;
-constexpr int kSelMaxE = 8;  // nb_max <= 512 * 8 = 4096 blocks (256K context)
+// The select of one row runs on a cluster of kSelCluster CTAs: every CTA merges the chunk partials into
+// LSE_h, forms S for 1/kSelCluster of the blocks (its block maxima are a contiguous head-major slice) and
+// stores them into the leader CTA's shared memory over distributed shared memory; after one cluster
+// barrier the leader (rank 0) selects.  Spreading the block maxima over 8 SMs is what makes this fast:
+// a single SM pulls the 128 KB of a 128K-context row far too slowly.
+constexpr int kSelCluster = 8;
+constexpr int kSelThreads = 512;  // the leader's top-k: up to 8 blocks per thread -> nb_max <= 4096
 
 template <int E>
 __global__ void __launch_bounds__(kSelThreads) score_select_kernel(QueryRows qr, MethodConsts mc, int nb_max,
                                                                    ScoreWs ws, int32_t* __restrict__ idx,
                                                                    int32_t* __restrict__ cnt)
 {
-    extern __shared__ float S[];  // nb_max
+    pdl_launch_dependents();
+    pdl_wait();
+    extern __shared__ float S[];  // nb_max; the leader's copy receives every CTA's scores
     __shared__ float lse[16];
-    __shared__ int red[2 * kSelThreads / 32 + kSelThreads / 32 + 1];
-    const int row = blockIdx.x;
-    const int g = row % qr.Hkv, bt = row / qr.Hkv, t = bt % qr.T, b = bt / qr.T;
+    __shared__ CtaSelectSmem sel_sm;
+    cg::cluster_group cluster = cg::this_cluster();
+    const int rank = (int)cluster.block_rank();
+    const int row = blockIdx.y;
+    const int bt = row / qr.Hkv, t = bt % qr.T, b = bt / qr.T;
     const int G = qr.Hq / qr.Hkv;
     const int n = query_ctx(qr, b, t);
     const int c = (n - 1) / kBlock;
     int32_t* idx_row = idx + (size_t)row * mc.kmax;
-    if (n <= mc.dense_len) {
-        if (threadIdx.x < 32) warp_write_dense_row(c, mc.kmax, idx_row, cnt + row);
+    if (n <= mc.dense_len) {  // uniform over the cluster: nobody touches distributed shared memory
+        if (rank == 0 && threadIdx.x < 32) warp_write_dense_row(c, mc.kmax, idx_row, cnt + row);
         return;
     }
     const int nchunk = score_nchunk(nb_max);
     const int nch_row = c / kChunkBlocks + 1;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    // this CTA's blocks and their raw maxima (loaded first: the load overlaps the LSE merge)
+    const int per = (c + kSelCluster) / kSelCluster;  // ceil((c + 1) / kSelCluster) <= kSelThreads
+    const int blk = rank * per + (int)threadIdx.x;
+    const bool mine = (int)threadIdx.x < per && blk <= c;
+    float mb[16];
+#pragma unroll
+    for (int h = 0; h < 16; ++h)
+        mb[h] = (mine && h < G) ? ws.bmax[((size_t)row * 16 + h) * nb_max + blk] : neg_inf();
     if (warp < G) {
+        // LSE_h from the chunk partials: both loads in flight together
         const int h = warp;
-        float m = neg_inf();
-        for (int i = lane; i < nch_row; i += 32) m = fmaxf(m, ws.pmax[((size_t)row * nchunk + i) * 16 + h]);
-        m = warp_max(m);
-        float s = 0.f;
-        if (m != neg_inf())
-            for (int i = lane; i < nch_row; i += 32)
-                s += ws.psum[((size_t)row * nchunk + i) * 16 + h] *
-                     exp2_fast((ws.pmax[((size_t)row * nchunk + i) * 16 + h] - m) * kLog2e);
-        s = warp_sum(s);
-        if (lane == 0) lse[h] = (m == neg_inf()) ? neg_inf() : m + logf(s);
-    }
-    __syncthreads();
-    for (int blk = threadIdx.x; blk <= c; blk += kSelThreads) {
-        float acc = 0.f;
-        bool member = false;
-        for (int h = 0; h < G; ++h) {
-            const float mb = ws.bmax[((size_t)row * 16 + h) * nb_max + blk];
-            if (mb != neg_inf()) {
-                member = true;
-                acc += exp2_fast((mb - lse[h]) * kLog2e);
-            }
+        constexpr int kMaxChunkPerLane = 4;  // nb_max <= 4096 blocks -> <= 128 chunks
+        float pm[kMaxChunkPerLane], ps[kMaxChunkPerLane];
+#pragma unroll
+        for (int u = 0; u < kMaxChunkPerLane; ++u) {
+            const int i = lane + 32 * u;
+            const bool ok = i < nch_row;
+            pm[u] = ok ? ws.pmax[((size_t)row * nchunk + i) * 16 + h] : neg_inf();
+            ps[u] = ok ? ws.psum[((size_t)row * nchunk + i) * 16 + h] : 0.f;
         }
-        S[blk] = member ? acc : neg_inf();
+        float m = neg_inf();
+#pragma unroll
+        for (int u = 0; u < kMaxChunkPerLane; ++u) m = fmaxf(m, pm[u]);
+        m = warp_max(m);
+        float ssum = 0.f;
+        if (m != neg_inf())
+#pragma unroll
+            for (int u = 0; u < kMaxChunkPerLane; ++u)
+                if (pm[u] != neg_inf()) ssum += ps[u] * exp2_fast((pm[u] - m) * kLog2e);
+        ssum = warp_sum(ssum);
+        if (lane == 0) lse[h] = (m == neg_inf()) ? neg_inf() : m + logf(ssum);
     }
     __syncthreads();
-    cta_select_topk<kSelThreads, E>(S, c, mc.init_blocks, mc.local_blocks, mc.topk, mc.kmax, idx_row, cnt + row, red);
+    if (mine) {
+        // every head of the group sees the same kernels: a block without a visible kernel is -inf for all
+        float acc = 0.f;
+#pragma unroll
+        for (int h = 0; h < 16; ++h)
+            if (h < G && mb[h] != neg_inf()) acc += exp2_fast((mb[h] - lse[h]) * kLog2e);
+        float* S_leader = cluster.map_shared_rank(S, 0);
+        S_leader[blk] = mb[0] != neg_inf() ? acc : neg_inf();
+    }
+    cluster.sync();  // release/acquire: the leader sees every score
+    if (rank != 0) return;
+    cta_select_topk<kSelThreads, E>(S, c, mc.init_blocks, mc.local_blocks, mc.topk, mc.kmax, idx_row, cnt + row,
+                                    sel_sm);
 }
 
 // =====================================================================================================
@@ -258,6 +292,8 @@ __global__ void __launch_bounds__(kPfThreads) score_prefill_kernel(QueryRows qr,
                                                                    int nk_cap, MethodConsts mc, int nb_max,
                                                                    int32_t* __restrict__ idx, int32_t* __restrict__ cnt)
 {
+    pdl_launch_dependents();
+    pdl_wait();
     constexpr int TW = 16 / G;               // tokens per warp
     constexpr int TPC = TW * kPfWarps;       // tokens per CTA
     constexpr int ZW = 72;                   // z row: column 7 = previous tile's last kernel, 8.. = this tile
@@ -473,12 +509,11 @@ static cudaError_t launch_prefill_score(const QueryRows& qr, const __nv_bfloat16
 {
     constexpr int TPC = (16 / G) * kPfWarps;
     const size_t smem = prefill_score_smem(G, D, nb_max);
-    cudaError_t e = cudaFuncSetAttribute(score_prefill_kernel<D, G>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)smem);
+    cudaError_t e = ensure_smem(score_prefill_kernel<D, G>, smem);
     if (e != cudaSuccess) return e;
     dim3 grid((qr.T + TPC - 1) / TPC, qr.B * qr.Hkv);
-    score_prefill_kernel<D, G><<<grid, kPfThreads, smem, s>>>(qr, kern, nk_cap, mc, nb_max, idx, cnt);
-    return cudaGetLastError();
+    return launch_pdl(score_prefill_kernel<D, G>, grid, dim3(kPfThreads), smem, s, qr, kern, nk_cap, mc, nb_max, idx,
+                      cnt);
 }
 
 template <int D>
@@ -512,19 +547,23 @@ cudaError_t launch_score_topk(const QueryRows& qr, const void* kern_v, int nk_ca
     sw.psum = reinterpret_cast<float*>(w + al((size_t)rows * nchunk * 16 * 4));
     sw.bmax = reinterpret_cast<float*>(w + 2 * al((size_t)rows * nchunk * 16 * 4));
     dim3 g1(nchunk, rows);
-    if (qr.D == 128)
-        score_scan_kernel<128><<<g1, kScanThreads, 0, s>>>(qr, kern, nk_cap, mc, nb_max, sw);
-    else
-        score_scan_kernel<64><<<g1, kScanThreads, 0, s>>>(qr, kern, nk_cap, mc, nb_max, sw);
-    cudaError_t e = cudaGetLastError();
+    cudaError_t e = qr.D == 128
+                        ? launch_pdl(score_scan_kernel<128>, g1, dim3(kScanThreads), 0, s, qr, kern, nk_cap, mc, nb_max, sw)
+                        : launch_pdl(score_scan_kernel<64>, g1, dim3(kScanThreads), 0, s, qr, kern, nk_cap, mc, nb_max, sw);
     if (e != cudaSuccess) return e;
     const size_t smem = (size_t)nb_max * 4;
     const int E = (nb_max + kSelThreads - 1) / kSelThreads;
-    if (E <= 1) score_select_kernel<1><<<rows, kSelThreads, smem, s>>>(qr, mc, nb_max, sw, idx, cnt);
-    else if (E <= 2) score_select_kernel<2><<<rows, kSelThreads, smem, s>>>(qr, mc, nb_max, sw, idx, cnt);
-    else if (E <= 4) score_select_kernel<4><<<rows, kSelThreads, smem, s>>>(qr, mc, nb_max, sw, idx, cnt);
-    else score_select_kernel<8><<<rows, kSelThreads, smem, s>>>(qr, mc, nb_max, sw, idx, cnt);
-    return cudaGetLastError();
+    const dim3 g2(kSelCluster, rows), b2(kSelThreads);
+    switch (E) {
+    case 1: return launch_pdl_cluster(score_select_kernel<1>, g2, b2, kSelCluster, smem, s, qr, mc, nb_max, sw, idx, cnt);
+    case 2: return launch_pdl_cluster(score_select_kernel<2>, g2, b2, kSelCluster, smem, s, qr, mc, nb_max, sw, idx, cnt);
+    case 3: return launch_pdl_cluster(score_select_kernel<3>, g2, b2, kSelCluster, smem, s, qr, mc, nb_max, sw, idx, cnt);
+    case 4: return launch_pdl_cluster(score_select_kernel<4>, g2, b2, kSelCluster, smem, s, qr, mc, nb_max, sw, idx, cnt);
+    case 5: return launch_pdl_cluster(score_select_kernel<5>, g2, b2, kSelCluster, smem, s, qr, mc, nb_max, sw, idx, cnt);
+    case 6: return launch_pdl_cluster(score_select_kernel<6>, g2, b2, kSelCluster, smem, s, qr, mc, nb_max, sw, idx, cnt);
+    case 7: return launch_pdl_cluster(score_select_kernel<7>, g2, b2, kSelCluster, smem, s, qr, mc, nb_max, sw, idx, cnt);
+    default: return launch_pdl_cluster(score_select_kernel<8>, g2, b2, kSelCluster, smem, s, qr, mc, nb_max, sw, idx, cnt);
+    }
 }
 
 }  // namespace iv2

@@ -6,9 +6,10 @@
 // the largest group score S are added, ties going to the lower block id.  The union is written in
 // ascending order, padded with -1 up to kmax; the count goes to *cnt.
 //
-// The k-th largest key is found by a 32-step bitwise search on the order-preserving uint32 image of S
-// (candidates only; non-candidates have key 0, below every float), counting keys >= the probe with
-// warp reductions.  Ties at the threshold are resolved by index with a prefix count.
+// Keys are the order-preserving uint32 image of S (non-candidates have key 0, below every float).  The
+// k-th largest key is found by a bitwise search (one warp: 32 probes counted with warp reductions) or
+// a radix select (whole CTA: 4 passes over 8-bit digits with shared-memory histograms).  Ties at the
+// threshold are resolved by block id with a prefix count.
 #pragma once
 
 #include "common.cuh"
@@ -127,15 +128,47 @@ IV2_DEV int cta_exclusive_scan(int v, int* scan_smem /* NT/32 + 1 ints */, int* 
     return wbase + incl - v;
 }
 
-// E = max elements per thread (nb <= NT * E); thread tid owns blocks [tid*E, tid*E + E)
+// E = max elements per thread (nb <= NT * E); thread tid owns blocks [tid*E, tid*E + E).
+//
+// Bucket select: the candidate keys are spread over kBuckets buckets by a monotone map of their value
+// range, a shared histogram finds the bucket B* that holds the k-th largest key, and one warp ranks the
+// few keys of B* exactly by (key descending, block ascending).  The rank-k element (T, I) of that total
+// order is the threshold: a candidate is chosen iff (key, -block) >= (T, -I).  Counting uses no warp
+// reductions in dependent loops (they are slow on sm_100): members are ranked by direct comparison.
+constexpr int kBuckets = 2048;
+constexpr int kMaxMembers = 1024;  // keys of the boundary bucket staged in shared memory
+constexpr int kRankMembers = 128;  // up to this many are ranked by one warp; more: CTA-wide search
+
+struct CtaSelectSmem {
+    int hist[kBuckets];
+    uint32_t mkey[kMaxMembers];
+    int midx[kMaxMembers];
+    int red[64];
+    int nmem;
+    uint32_t kmin, kmax;
+    int bstar, above;          // boundary bucket, candidates in buckets above it
+    uint32_t thr_key;
+    int thr_idx;
+};
+
+// monotone (non-decreasing) map of a key in [kmin, kmax] to [0, kBuckets): every key goes through the
+// same fp32 arithmetic, so equal keys share a bucket and a larger key never lands in a lower bucket
+IV2_DEV int bucket_of(uint32_t key, uint32_t kmin, float bucket_scale)
+{
+    return min((int)((float)(key - kmin) * bucket_scale), kBuckets - 1);
+}
+
 template <int NT, int E>
 IV2_DEV void cta_select_topk(const float* S, int c, int init, int local, int topk, int kmax, int32_t* idx_out,
-                             int32_t* cnt_out, int* red /* >= 2*NT/32 + NT/32 + 1 ints */)
+                             int32_t* cnt_out, CtaSelectSmem& sm)
 {
+    constexpr int NW = NT / 32;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int nb = c + 1;
     const int b0 = threadIdx.x * E;
     uint32_t key[E];
     int ncand_local = 0;
+    uint32_t lo = 0xffffffffu, hi = 0u;
 #pragma unroll
     for (int e = 0; e < E; ++e) {
         const int b = b0 + e;
@@ -144,42 +177,146 @@ IV2_DEV void cta_select_topk(const float* S, int c, int init, int local, int top
             const float s = S[b];
             if (s != neg_inf()) key[e] = float_key(s);
         }
-        ncand_local += key[e] != 0u;
-    }
-    int* scan_smem = red + 2 * (NT / 32);
-    int parity = 0;
-    const int ncand = cta_count<NT>(ncand_local, red, parity);
-    parity ^= 1;
-    const bool all = ncand <= topk;
-    uint32_t thr = 1u;
-    int need_eq = 0;
-    if (!all) {
-        uint32_t t = 0u;
-        for (int bit = 31; bit >= 0; --bit) {
-            const uint32_t probe = t | (1u << bit);
-            int ge = 0;
-#pragma unroll
-            for (int e = 0; e < E; ++e) ge += key[e] >= probe;
-            const int tot = cta_count<NT>(ge, red, parity);
-            parity ^= 1;
-            if (tot >= topk) t = probe;
+        if (key[e] != 0u) {
+            ++ncand_local;
+            lo = min(lo, key[e]);
+            hi = max(hi, key[e]);
         }
-        int gt = 0;
-#pragma unroll
-        for (int e = 0; e < E; ++e) gt += key[e] > t;
-        gt = cta_count<NT>(gt, red, parity);
-        parity ^= 1;
-        thr = t;
-        need_eq = topk - gt;
     }
-    // ties at the threshold: rank by block id
-    int eq_local = 0;
+    // candidate count and key range
+    ncand_local = __reduce_add_sync(0xffffffffu, ncand_local);
+    lo = __reduce_min_sync(0xffffffffu, lo);
+    hi = __reduce_max_sync(0xffffffffu, hi);
+    if (lane == 0) {
+        sm.red[warp] = ncand_local;
+        sm.red[NW + warp] = (int)lo;
+        sm.red[2 * NW + warp] = (int)hi;
+    }
+    for (int i = threadIdx.x; i < kBuckets; i += NT) sm.hist[i] = 0;
+    if (threadIdx.x == 0) sm.nmem = 0;
+    __syncthreads();
+    int ncand = 0;
+    uint32_t kmn = 0xffffffffu, kmx = 0u;
+#pragma unroll
+    for (int i = 0; i < NW; ++i) {
+        ncand += sm.red[i];
+        kmn = min(kmn, (uint32_t)sm.red[NW + i]);
+        kmx = max(kmx, (uint32_t)sm.red[2 * NW + i]);
+    }
+    const bool all = ncand <= topk;
+    const float bscale = kmx > kmn ? (float)(kBuckets - 1) / (float)(kmx - kmn) : 0.f;
+    int bstar = kBuckets;
+    uint32_t tkey = 0u;
+    int tidx = 0;
     if (!all) {
 #pragma unroll
-        for (int e = 0; e < E; ++e) eq_local += key[e] == thr;
+        for (int e = 0; e < E; ++e)
+            if (key[e] != 0u) atomicAdd(&sm.hist[bucket_of(key[e], kmn, bscale)], 1);
+        __syncthreads();
+        // descending suffix scan over buckets: thread t owns buckets [kBuckets - (t+1)*BPT, kBuckets - t*BPT)
+        constexpr int BPT = kBuckets / NT;
+        int cnt_b[BPT], sum = 0;
+#pragma unroll
+        for (int j = 0; j < BPT; ++j) {
+            cnt_b[j] = sm.hist[kBuckets - 1 - (threadIdx.x * BPT + j)];
+            sum += cnt_b[j];
+        }
+        int incl = sum;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int y = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += y;
+        }
+        __syncthreads();  // hist reads done before red is reused
+        if (lane == 31) sm.red[warp] = incl;
+        __syncthreads();
+        int wbase = 0;
+#pragma unroll
+        for (int i = 0; i < NW; ++i)
+            if (i < warp) wbase += sm.red[i];
+        const int excl = wbase + incl - sum;  // candidates in buckets above this thread's range
+        if (excl < topk && topk <= excl + sum) {
+            int acc = excl;
+#pragma unroll
+            for (int j = 0; j < BPT; ++j) {
+                if (acc + cnt_b[j] >= topk) {
+                    sm.bstar = kBuckets - 1 - (threadIdx.x * BPT + j);
+                    sm.above = acc;
+                    break;
+                }
+                acc += cnt_b[j];
+            }
+        }
+        __syncthreads();
+        bstar = sm.bstar;
+        const int rem = topk - sm.above;  // members of bucket B* still to take, >= 1
+        // stage the members of B*
+#pragma unroll
+        for (int e = 0; e < E; ++e) {
+            if (key[e] != 0u && bucket_of(key[e], kmn, bscale) == bstar) {
+                const int slot = atomicAdd(&sm.nmem, 1);
+                if (slot < kMaxMembers) {
+                    sm.mkey[slot] = key[e];
+                    sm.midx[slot] = b0 + e;
+                }
+            }
+        }
+        __syncthreads();
+        if (sm.nmem > kRankMembers) {
+            // degenerate spread (e.g. many equal scores): rank the bucket's members CTA-wide
+            int parity = 0;
+            uint32_t t = 0u;
+            for (int bit = 31; bit >= 0; --bit) {
+                const uint32_t probe = t | (1u << bit);
+                int ge = 0;
+#pragma unroll
+                for (int e = 0; e < E; ++e)
+                    ge += key[e] != 0u && bucket_of(key[e], kmn, bscale) == bstar && key[e] >= probe;
+                if (cta_count<NT>(ge, sm.red, parity) >= rem) t = probe;
+                parity ^= 1;
+            }
+            int gt = 0;
+#pragma unroll
+            for (int e = 0; e < E; ++e) gt += key[e] != 0u && bucket_of(key[e], kmn, bscale) == bstar && key[e] > t;
+            gt = cta_count<NT>(gt, sm.red, parity);
+            parity ^= 1;
+            const int need = rem - gt;
+            int ti = 0;
+            for (int bit = 12; bit >= 0; --bit) {
+                const int probe = ti | ((1 << bit) - 1);
+                int le = 0;
+#pragma unroll
+                for (int e = 0; e < E; ++e) le += key[e] == t && (b0 + e) <= probe;
+                if (cta_count<NT>(le, sm.red, parity) < need) ti |= 1 << bit;
+                parity ^= 1;
+            }
+            if (threadIdx.x == 0) {
+                sm.thr_key = t;
+                sm.thr_idx = ti;
+            }
+        } else if (warp == 0) {
+            // few members: the rank of member i in (key descending, block ascending) order is the number of
+            // members before it; the one of rank rem-1 is the threshold
+            const int nm = sm.nmem;
+            for (int i = lane; i < nm; i += 32) {
+                const uint32_t ki = sm.mkey[i];
+                const int ii = sm.midx[i];
+                int rank = 0;
+                for (int j = 0; j < nm; ++j) {
+                    const uint32_t kj = sm.mkey[j];
+                    rank += (kj > ki) || (kj == ki && sm.midx[j] < ii);
+                }
+                if (rank == rem - 1) {
+                    sm.thr_key = ki;
+                    sm.thr_idx = ii;
+                }
+            }
+        }
+        __syncthreads();
+        tkey = sm.thr_key;
+        tidx = sm.thr_idx;
     }
-    int eq_total;
-    int eq_rank = cta_exclusive_scan<NT>(eq_local, scan_smem, &eq_total);
+    // emit ascending
     bool chosen[E];
     int nchosen = 0;
 #pragma unroll
@@ -188,18 +325,19 @@ IV2_DEV void cta_select_topk(const float* S, int c, int init, int local, int top
         bool ch = false;
         if (b < nb) {
             if (is_forced(b, c, init, local)) ch = true;
-            else if (all) ch = key[e] != 0u;
-            else if (key[e] > thr) ch = true;
-            else if (key[e] == thr) {
-                ch = eq_rank < need_eq;
-                ++eq_rank;
+            else if (key[e] != 0u) {
+                if (all) ch = true;
+                else {
+                    const int bk = bucket_of(key[e], kmn, bscale);
+                    ch = bk > bstar || (bk == bstar && (key[e] > tkey || (key[e] == tkey && b <= tidx)));
+                }
             }
         }
         chosen[e] = ch;
         nchosen += ch;
     }
     int total;
-    int pos = cta_exclusive_scan<NT>(nchosen, scan_smem, &total);
+    int pos = cta_exclusive_scan<NT>(nchosen, sm.red, &total);
 #pragma unroll
     for (int e = 0; e < E; ++e) {
         if (chosen[e]) {
