@@ -172,6 +172,25 @@ int infllmv2_sparse_attn_tree_verify(const void* q, int batch, int n_draft, int 
                                      void* out, float* lse, void* ws, size_t ws_bytes, infllmv2_stream_t stream);
 
 /*
+ * Sparse decode attention without a workspace.  The pages have no counterpart: this is a convenience of
+ * the library.  It computes exactly what infllmv2_sparse_attn_decode computes, with the same arguments and
+ * layouts minus (ws, ws_bytes), for callers that cannot allocate device memory when they call: a process
+ * that hands out its GPU memory once at start-up, a plugin that may not use its host's allocator, a loop
+ * that must never allocate.  The split partials go to a 4 MiB array inside the library instead (one per
+ * GPU that loads the library, kept until the process exits).
+ *   Limit: B * Hkv * ceil(max(kmax, blocks of min(max_ctx, dense_len)) / 4) * (16 * d + 32) * 4 bytes must
+ *   fit in 4 MiB (for example B = 4, Hkv = 2, d = 128, kmax = 67, dense_len = 8192 needs 2.1 MiB); a larger
+ *   call returns INFLLMV2_ERR_WORKSPACE and launches nothing.
+ *   The first call on a device looks up the array's address (cudaGetSymbolAddress) with that device
+ *   current; make it before any stream capture.  All calls share the array, so calls whose kernels overlap
+ *   on the GPU (other streams or host threads) race on it.  Nothing in it needs clearing between calls.
+ */
+int infllmv2_sparse_attn_decode_noalloc(const void* q, int batch, int hq, int hkv, int head_dim, const void* k,
+                                        const void* v, int lcap, const int32_t* ctx_lens, int max_ctx,
+                                        const int32_t* idx, const int32_t* cnt, const infllmv2_params* params,
+                                        void* out, float* lse, infllmv2_stream_t stream);
+
+/*
  * Dense path (MiniCPM 4.0 launch article, section 1: short texts keep dense attention).  Plain causal GQA
  * attention over keys [0, n) for every query, whatever dense_len is; same layouts and n rules as 3a / 3b.
  */

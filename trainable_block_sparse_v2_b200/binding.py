@@ -73,6 +73,7 @@ _SIGS = {
     "infllmv2_sparse_attn_prefill": ([_P, _I, _I, _I, _I, _I, _P, _P, _I, _P, _P, _I, _P, _P, _PP, _P, _P, _P,
                                       _SZ, _P], _I),
     "infllmv2_sparse_attn_decode": ([_P, _I, _I, _I, _I, _P, _P, _I, _P, _I, _P, _P, _PP, _P, _P, _P, _SZ, _P], _I),
+    "infllmv2_sparse_attn_decode_noalloc": ([_P, _I, _I, _I, _I, _P, _P, _I, _P, _I, _P, _P, _PP, _P, _P, _P], _I),
     "infllmv2_sparse_attn_tree_verify": ([_P, _I, _I, _I, _I, _I, _P, _P, _I, _P, _I, _P, _P, _P, _P, _P, _PP, _P,
                                           _P, _P, _SZ, _P], _I),
     "infllmv2_dense_attn_prefill": ([_P, _I, _I, _I, _I, _I, _P, _P, _I, _P, _P, _I, _F, _P, _P, _P, _SZ, _P], _I),
@@ -206,6 +207,21 @@ def infllmv2_sparse_attn_decode(q, k, v, ctx_lens, max_ctx, idx, cnt, params: Pa
                                             _ptr(ws), 0 if ws is None else ws.numel() * ws.element_size(),
                                             _stream(stream))
     _check("infllmv2_sparse_attn_decode", st)
+
+
+def infllmv2_sparse_attn_decode_noalloc(q, k, v, ctx_lens, max_ctx, idx, cnt, params: Params, out, lse=None,
+                                        stream=None):
+    """infllmv2_sparse_attn_decode without a workspace: the library keeps the scratch in its own static
+    device array (4 MiB per GPU), for callers that cannot allocate device memory when they call."""
+    for t, n in ((q, "q"), (k, "k"), (v, "v"), (out, "out")):
+        _need(t, torch.bfloat16, n)
+    B, Hq, d = q.shape[0], q.shape[-2], q.shape[-1]
+    Lcap, Hkv = k.shape[1], k.shape[2]
+    cp = params.c()
+    st = load().infllmv2_sparse_attn_decode_noalloc(_ptr(q), B, Hq, Hkv, d, _ptr(k), _ptr(v), Lcap, _ptr(ctx_lens),
+                                                    int(max_ctx), _ptr(idx), _ptr(cnt), ctypes.byref(cp), _ptr(out),
+                                                    _ptr(lse), _stream(stream))
+    _check("infllmv2_sparse_attn_decode_noalloc", st)
 
 
 def infllmv2_sparse_attn_tree_verify(q, k, v, prefix_lens, max_ctx, k_draft, v_draft, tree_mask, idx, cnt,
