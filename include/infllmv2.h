@@ -36,7 +36,7 @@
  *     supports block_size 64, kernel_size 32, kernel_stride 16 (other values -> INFLLMV2_ERR_UNSUPPORTED).
  *   - Errors: every argument is checked on the host before any launch; on a bad argument the call
  *     returns the status and launches nothing.  A failed launch returns INFLLMV2_ERR_CUDA.  Kernels
- *     contain no waits on other kernels or devices.
+ *     never wait on other kernels or devices; waits inside one CTA are bounded (infllmv2_device_status).
  *   - Workspace: entry points that take (ws, ws_bytes) need at least infllmv2_workspace_size(...) bytes
  *     of device memory, 256-byte aligned, owned by the caller; calls that run concurrently need separate
  *     workspaces.  Its contents need no initialisation and are scratch after the call.
@@ -59,7 +59,7 @@ typedef enum {
     INFLLMV2_ERR_UNSUPPORTED = 2, /* valid but outside what the GPU kernels implement */
     INFLLMV2_ERR_WORKSPACE = 3,   /* workspace missing, misaligned or too small */
     INFLLMV2_ERR_CUDA = 4,        /* a CUDA launch failed (cudaGetLastError after the launch) */
-    INFLLMV2_ERR_TIMEOUT = 5      /* reserved: no kernel of this library waits */
+    INFLLMV2_ERR_TIMEOUT = 5      /* a bounded device-side wait ran out (see infllmv2_device_status) */
 } infllmv2_status;
 
 /* Method constants (the pages give none; the workloads use 64 / 32 / 16, k = 8 or 64, 1 + 2 forced). */
@@ -81,6 +81,15 @@ const char* infllmv2_status_string(int status);
 
 /* Library version, as major*10000 + minor*100 + patch. */
 int infllmv2_version(void);
+
+/*
+ * Device-side status of the kernels that wait on their own producer/consumer barriers (the tensor-core
+ * prefill attention): every such wait is bounded, and a wait that runs out records an error, makes its
+ * CTA skip the rest of its work and exit.  Returns INFLLMV2_ERR_TIMEOUT if that happened since the last
+ * call (and clears the record), INFLLMV2_OK otherwise, INFLLMV2_ERR_CUDA if the record cannot be read.
+ * Synchronous: it reads device memory on the current device.
+ */
+int infllmv2_device_status(void);
 
 /*
  * Bytes of workspace the calls below need for problems up to the given sizes (host-only, no CUDA call).

@@ -67,6 +67,7 @@ _F = ctypes.c_float
 _SIGS = {
     "infllmv2_status_string": ([_I], ctypes.c_char_p),
     "infllmv2_version": ([], _I),
+    "infllmv2_device_status": ([], _I),
     "infllmv2_workspace_size": ([_PP, _I, _I, _I, _I, _I, _I], _SZ),
     "infllmv2_kernel_pool": ([_P, _I, _I, _I, _I, _P, _P, _I, _PP, _P, _I, _P], _I),
     "infllmv2_block_score_topk": ([_P, _I, _I, _I, _I, _I, _P, _P, _I, _P, _I, _PP, _P, _P, _P, _SZ, _P], _I),
@@ -136,6 +137,11 @@ def _check(fn, status):
 
 def infllmv2_version() -> int:
     return load().infllmv2_version()
+
+
+def infllmv2_device_status() -> int:
+    """0 when no bounded device-side wait ran out since the last call (reading clears the record)."""
+    return int(load().infllmv2_device_status())
 
 
 def infllmv2_status_string(status: int) -> str:

@@ -174,6 +174,13 @@ const char* infllmv2_status_string(int status)
 
 int infllmv2_version(void) { return kVersion; }
 
+int infllmv2_device_status(void)
+{
+    const int f = iv2::tc_error_flag_read_and_clear();
+    if (f < 0) return INFLLMV2_ERR_CUDA;
+    return f ? INFLLMV2_ERR_TIMEOUT : INFLLMV2_OK;
+}
+
 size_t infllmv2_workspace_size(const infllmv2_params* params, int batch, int max_q, int max_ctx, int hq, int hkv,
                                int head_dim)
 {
@@ -248,8 +255,13 @@ int infllmv2_sparse_attn_prefill(const void* q, int batch, int num_q, int hq, in
     if (!q_ctx && !ctx_lens) return INFLLMV2_ERR_INVALID_ARG;
     IV2_TRY(check_ctx(max_ctx, lcap));
     const QueryRows qr = rows_of(q, batch, num_q, hq, hkv, head_dim, q_ctx, ctx_lens, 0, max_ctx);
-    return launched(iv2::launch_attn_rows(qr, k, v, lcap, idx, cnt, consts_of(params, head_dim), false, out, lse,
-                                          (cudaStream_t)stream));
+    const MethodConsts mc = consts_of(params, head_dim);
+    if (iv2::attn_tc_supported(qr)) {
+        const cudaError_t e = iv2::launch_attn_rows_tc(qr, k, v, lcap, idx, cnt, mc, false, out, lse,
+                                                       (cudaStream_t)stream);
+        if (e != cudaErrorNotSupported) return launched(e);
+    }
+    return launched(iv2::launch_attn_rows(qr, k, v, lcap, idx, cnt, mc, false, out, lse, (cudaStream_t)stream));
 }
 
 int infllmv2_sparse_attn_decode(const void* q, int batch, int hq, int hkv, int head_dim, const void* k, const void* v,
@@ -324,8 +336,13 @@ int infllmv2_dense_attn_prefill(const void* q, int batch, int num_q, int hq, int
     if (!q_ctx && !ctx_lens) return INFLLMV2_ERR_INVALID_ARG;
     IV2_TRY(check_ctx(max_ctx, lcap));
     const QueryRows qr = rows_of(q, batch, num_q, hq, hkv, head_dim, q_ctx, ctx_lens, 0, max_ctx);
-    return launched(iv2::launch_attn_rows(qr, k, v, lcap, nullptr, nullptr, dense_consts(softmax_scale, head_dim),
-                                          true, out, lse, (cudaStream_t)stream));
+    const MethodConsts mc = dense_consts(softmax_scale, head_dim);
+    if (iv2::attn_tc_supported(qr)) {
+        const cudaError_t e = iv2::launch_attn_rows_tc(qr, k, v, lcap, nullptr, nullptr, mc, true, out, lse,
+                                                       (cudaStream_t)stream);
+        if (e != cudaErrorNotSupported) return launched(e);
+    }
+    return launched(iv2::launch_attn_rows(qr, k, v, lcap, nullptr, nullptr, mc, true, out, lse, (cudaStream_t)stream));
 }
 
 int infllmv2_dense_attn_decode(const void* q, int batch, int hq, int hkv, int head_dim, const void* k, const void* v,

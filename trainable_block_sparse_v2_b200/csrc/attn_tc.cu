@@ -1,0 +1,461 @@
+// attn_tc.cu -- block-sparse prefill attention on the 5th-generation tensor cores (tcgen05 + TMEM + TMA).
+//
+// Same definition as attn.cu (MiniCPM4 technical details, InfLLM v2 overview: only the selected context
+// blocks take part in attention; "Model architecture: InfLLM v2" item 2: the query heads of one GQA group
+// share the block set).  Specialised for 16 query heads per KV group and head_dim 128.
+//
+// One CTA owns a 128-row tile = 8 consecutive query tokens x the 16 heads of one KV group, and walks the
+// ascending union of those tokens' selected blocks (a token attends to a block only when it selected it;
+// other rows of the tile are masked for that block).  Per 64-key block:
+//   S[128 x 64]  = Q[128 x 128] . K_blk^T   tcgen05.mma kind::f16 with A (Q) in TMEM and B (K) K-major in
+//                                            128B-swizzled smem, fp32 accumulator in TMEM (two S buffers)
+//   P            = online softmax of S       four warps, one TMEM lane (= one query row) per thread; P goes
+//                                            back to TMEM as bf16 pairs (two P buffers); the output is
+//                                            rescaled only when a row's max grows by more than 2^8 (exact:
+//                                            O and the row sum share the reference max)
+//   O[128 x 128] += P[128 x 64] . V_blk      A (P) in TMEM, B (V) MN-major in smem, O in TMEM
+// Keeping Q and P in TMEM leaves shared memory to the K/V stream: the operand reads of a block drop from
+// 80 KB to 32 KB.
+// Warp roles: warp 0 issues TMA loads (Q once, K/V per block into 4 stages), warp 1 (one thread) issues the
+// MMAs, warps 2-5 run the softmax and the epilogue.  Producer/consumer hand-offs use mbarriers; MMA
+// completion is signalled with tcgen05.commit.  Every wait is bounded: after the limit the CTA records an
+// error (g_tc_error), skips the rest of its work, frees its TMEM and exits.
+#include <mutex>
+
+#include "common.cuh"
+#include "internal.h"
+#include "tc.cuh"
+
+namespace iv2 {
+
+__device__ int g_tc_error = 0;
+
+namespace {
+
+constexpr int kTok = 8;           // tokens per tile
+constexpr int kG = 16;            // heads per KV group
+constexpr int kD = 128;           // head dim
+constexpr int kThreads = 192;     // 6 warps
+constexpr int kMaxBlk = 4096;     // context blocks (256K keys)
+constexpr int kWords = kMaxBlk / 32;
+constexpr uint32_t kTmemCols = 512;  // O [0,128), S0/S1 [128,256), P0/P1 [256,320), Q [320,384)
+constexpr uint32_t kColS = 128, kColP = 256, kColQ = 320;
+
+// dynamic shared memory layout (base aligned to 1024 B)
+constexpr int kQOff = 0;                     // 2 atoms x 128 rows x 128 B
+constexpr int kStages = 4;                   // K/V pipeline depth: hides the load latency of 3 blocks
+constexpr int kKvOff = 32768;                // kStages x (K0, K1, V0, V1) x 64 rows x 128 B
+constexpr int kKvStage = 32768;
+constexpr int kBitsOff = kKvOff + kStages * kKvStage;  // [kTok][kWords] uint32
+constexpr int kListOff = kBitsOff + kTok * kWords * 4;  // uint16 block ids
+constexpr int kSmemBytes = kListOff + kMaxBlk * 2 + 1024;  // + alignment slack
+
+struct Bars {
+    uint64_t q_full, q_tmem;
+    uint64_t kv_full[kStages], kv_empty[kStages];
+    uint64_t s_full[2], p_full[2], o_done[2];
+    uint32_t tmem_base;
+    int n_union;
+    int err;
+};
+
+__device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity, volatile int* err)
+{
+    for (uint32_t i = 0; i < (1u << 22); ++i) {
+        if (tc::mbar_try_wait(bar, parity)) return true;
+        if ((i & 255u) == 255u && *err) return false;
+    }
+    *err = 1;
+    atomicOr(&g_tc_error, 1);
+    return false;
+}
+
+}  // namespace
+
+__global__ void __launch_bounds__(kThreads, 1)
+attn_tc_kernel(QueryRows qr, const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+               const __grid_constant__ CUtensorMap tm_v, int Lcap, const int32_t* __restrict__ idx,
+               const int32_t* __restrict__ cnt, MethodConsts mc, int dense_all, __nv_bfloat16* __restrict__ out,
+               float* __restrict__ lse)
+{
+    pdl_launch_dependents();
+    pdl_wait();
+    extern __shared__ unsigned char smem_raw[];
+    unsigned char* smem = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    __shared__ Bars bars;
+    uint32_t* bits = reinterpret_cast<uint32_t*>(smem + kBitsOff);
+    uint16_t* list = reinterpret_cast<uint16_t*>(smem + kListOff);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int T = qr.T;
+    const int g = blockIdx.y % qr.Hkv, b = blockIdx.y / qr.Hkv;
+    const int t0 = blockIdx.x * kTok;
+
+    // ---- union of the tile's block sets, as one bitmap per token and an ascending list ----
+    int cmax = 0;
+#pragma unroll
+    for (int tt = 0; tt < kTok; ++tt)
+        if (t0 + tt < T) cmax = max(cmax, (query_ctx(qr, b, t0 + tt) - 1) / kBlock);
+    const int nwords = min(cmax / 32 + 1, kWords);
+    for (int i = threadIdx.x; i < kTok * kWords; i += kThreads) bits[i] = 0u;
+    if (threadIdx.x == 0) {
+        bars.err = 0;
+        bars.n_union = 0;
+    }
+    __syncthreads();
+    for (int item = threadIdx.x; item < kTok * max(mc.kmax, nwords); item += kThreads) {
+        const int tt = item % kTok, e = item / kTok;
+        const int t = t0 + tt;
+        if (t >= T) continue;
+        const int n = query_ctx(qr, b, t);
+        const int c = (n - 1) / kBlock;
+        if (dense_all || n <= mc.dense_len) {
+            if (e < nwords) {  // every block 0..c
+                const int lo = e * 32, hi = min(c + 1, lo + 32);
+                if (hi > lo) bits[tt * kWords + e] = (hi - lo == 32) ? 0xffffffffu : ((1u << (hi - lo)) - 1u);
+            }
+        } else if (e < mc.kmax) {
+            const size_t row = ((size_t)b * T + t) * qr.Hkv + g;
+            if (e < min(cnt[row], mc.kmax)) {
+                const int blk = idx[row * mc.kmax + e];
+                if (blk >= 0 && blk * kBlock < n) atomicOr(&bits[tt * kWords + (blk >> 5)], 1u << (blk & 31));
+            }
+        }
+    }
+    __syncthreads();
+    if (warp == 0) {
+        int base = 0;
+        for (int w0 = 0; w0 < nwords; w0 += 32) {
+            const int w = w0 + lane;
+            uint32_t u = 0u;
+            if (w < nwords)
+#pragma unroll
+                for (int tt = 0; tt < kTok; ++tt) u |= bits[tt * kWords + w];
+            const int cntw = __popc(u);
+            int incl = cntw;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int y = __shfl_up_sync(0xffffffffu, incl, o);
+                if (lane >= o) incl += y;
+            }
+            int pos = base + incl - cntw;
+            while (u) {
+                const int bit = __ffs(u) - 1;
+                list[pos++] = (uint16_t)(w * 32 + bit);
+                u &= u - 1u;
+            }
+            base += __shfl_sync(0xffffffffu, incl, 31);
+        }
+        if (lane == 0) bars.n_union = base;
+    }
+    if (threadIdx.x == 0) {
+        tc::mbar_init(&bars.q_full, 1);
+        tc::mbar_init(&bars.q_tmem, 128);
+        for (int i = 0; i < kStages; ++i) {
+            tc::mbar_init(&bars.kv_full[i], 1);
+            tc::mbar_init(&bars.kv_empty[i], 1);
+        }
+        for (int i = 0; i < 2; ++i) {
+            tc::mbar_init(&bars.s_full[i], 1);
+            tc::mbar_init(&bars.p_full[i], 128);
+            tc::mbar_init(&bars.o_done[i], 1);
+        }
+        tc::fence_barrier_init();
+    }
+    if (warp == 1) {
+        tc::tmem_alloc(&bars.tmem_base, kTmemCols);
+        tc::tmem_relinquish();
+    }
+    tc::tc_fence_before();
+    __syncthreads();
+    tc::tc_fence_after();
+    const int U = bars.n_union;
+    const uint32_t tmem = bars.tmem_base;
+    volatile int* err = &bars.err;
+
+    const uint32_t sKV = tc::smem_u32(smem + kKvOff);
+
+    if (warp == 0) {
+        // ---------------- TMA producer ----------------
+        if (lane == 0) {
+            tc::prefetch_tensormap(&tm_q);
+            tc::prefetch_tensormap(&tm_k);
+            tc::prefetch_tensormap(&tm_v);
+            tc::mbar_arrive_expect_tx(&bars.q_full, 2 * 128 * 128);
+            const int zq = b * T + t0;
+            tc::tma_load_3d(smem + kQOff, &tm_q, 0, g * kG, zq, &bars.q_full);
+            tc::tma_load_3d(smem + kQOff + 16384, &tm_q, 64, g * kG, zq, &bars.q_full);
+            for (int u = 0; u < U; ++u) {
+                const int s = u % kStages, k = u / kStages;
+                if (k >= 1 && !wait_bar(&bars.kv_empty[s], (k - 1) & 1, err)) break;
+                const int z = b * Lcap + (int)list[u] * kBlock;
+                unsigned char* st = smem + kKvOff + s * kKvStage;
+                tc::mbar_arrive_expect_tx(&bars.kv_full[s], kKvStage);
+                tc::tma_load_3d(st, &tm_k, 0, g, z, &bars.kv_full[s]);
+                tc::tma_load_3d(st + 8192, &tm_k, 64, g, z, &bars.kv_full[s]);
+                tc::tma_load_3d(st + 16384, &tm_v, 0, g, z, &bars.kv_full[s]);
+                tc::tma_load_3d(st + 24576, &tm_v, 64, g, z, &bars.kv_full[s]);
+            }
+        }
+    } else if (warp == 1) {
+        // ---------------- MMA issuer ----------------
+        if (lane == 0 && wait_bar(&bars.q_tmem, 0, err)) {
+            tc::tc_fence_after();
+            constexpr uint32_t idesc_s = tc::idesc_bf16(128, 64, false);
+            constexpr uint32_t idesc_o = tc::idesc_bf16(128, kD, true);
+            for (int u = 0; u <= U; ++u) {
+                if (u < U) {
+                    const int s = u % kStages, sb = u & 1;
+                    if (!wait_bar(&bars.kv_full[s], (u / kStages) & 1, err)) break;
+                    tc::tc_fence_after();
+                    const uint32_t d_s = tmem + kColS + 64 * sb;
+                    const uint32_t kbase = sKV + s * kKvStage;
+#pragma unroll
+                    for (int ks = 0; ks < kD / 16; ++ks) {
+                        const uint32_t koff = (ks >> 2) * 8192 + (ks & 3) * 32;
+                        tc::mma_bf16_ts(d_s, tmem + kColQ + 8 * ks, tc::desc_kmajor_sw128(kbase + koff), idesc_s,
+                                        ks > 0);
+                    }
+                    tc::mma_commit(&bars.s_full[sb]);
+                }
+                if (u >= 1) {
+                    const int v = u - 1, pv = v & 1;
+                    if (!wait_bar(&bars.p_full[pv], (v >> 1) & 1, err)) break;
+                    tc::tc_fence_after();
+                    const uint32_t vbase = sKV + (v % kStages) * kKvStage + 16384;
+#pragma unroll
+                    for (int ks = 0; ks < kBlock / 16; ++ks)
+                        tc::mma_bf16_ts(tmem, tmem + kColP + 32 * pv + 8 * ks,
+                                        tc::desc_mnmajor_sw128(vbase + ks * 2048, 8192), idesc_o, (v > 0 || ks > 0));
+                    tc::mma_commit(&bars.o_done[pv]);
+                    tc::mma_commit(&bars.kv_empty[v % kStages]);
+                }
+            }
+        }
+    } else {
+        // ---------------- softmax + epilogue: one TMEM lane (query row) per thread ----------------
+        const int q4 = warp & 3;
+        const int r = q4 * 32 + lane;  // row = token * 16 + head
+        const int tt = r >> 4, hh = r & 15;
+        const int t = t0 + tt;
+        const bool valid = t < T;
+        const int n = valid ? query_ctx(qr, b, t) : 0;
+        const uint32_t lane_addr = tmem + ((uint32_t)(q4 * 32) << 16);
+        const float sl2 = mc.scale * kLog2e;
+        float m_ref = neg_inf(), l = 0.f;
+        bool ok = wait_bar(&bars.q_full, 0, err);
+        {
+            // this row of Q (swizzled smem from TMA) -> TMEM columns [kColQ, kColQ + 64) as bf16 pairs
+#pragma unroll
+            for (int a = 0; a < 2; ++a) {
+                uint32_t w[32];
+                const unsigned char* qrow = smem + kQOff + a * 16384 + r * 128;
+#pragma unroll
+                for (int c = 0; c < 8; ++c) {
+                    const uint4 v4 = *reinterpret_cast<const uint4*>(qrow + ((c ^ (r & 7)) << 4));
+                    w[4 * c] = v4.x;
+                    w[4 * c + 1] = v4.y;
+                    w[4 * c + 2] = v4.z;
+                    w[4 * c + 3] = v4.w;
+                }
+                tc::tmem_st32(lane_addr + kColQ + 32 * a, w);
+            }
+            tc::tmem_wait_st();
+            tc::tc_fence_before();
+            tc::mbar_arrive(&bars.q_tmem);
+        }
+        ok = __all_sync(0xffffffffu, ok);
+        for (int u = 0; u < U && ok; ++u) {
+            const int sb = u & 1;
+            ok = wait_bar(&bars.s_full[sb], (u >> 1) & 1, err);
+            ok = __all_sync(0xffffffffu, ok);
+            if (!ok) break;
+            tc::tc_fence_after();
+            const int blk = list[u];
+            const bool sel = valid && ((bits[tt * kWords + (blk >> 5)] >> (blk & 31)) & 1u);
+            uint32_t sv[64];
+            {
+                uint32_t a[32], c2[32];
+                tc::tmem_ld32(lane_addr + kColS + 64 * sb, a);
+                tc::tmem_ld32(lane_addr + kColS + 64 * sb + 32, c2);
+                tc::tmem_wait_ld();
+#pragma unroll
+                for (int j = 0; j < 32; ++j) {
+                    sv[j] = a[j];
+                    sv[32 + j] = c2[j];
+                }
+            }
+            // the P buffer of this block was last read by PV(u-2)
+            if (u >= 2) ok = wait_bar(&bars.o_done[sb], ((u - 2) >> 1) & 1, err);
+            const int nvalid = sel ? min(kBlock, n - blk * kBlock) : 0;
+            const uint32_t prow = lane_addr + kColP + 32 * sb;
+            if (!__any_sync(0xffffffffu, sel)) {
+                // neither token of this warp selected the block: its P rows are zero
+                uint32_t z[32];
+#pragma unroll
+                for (int j = 0; j < 32; ++j) z[j] = 0u;
+                tc::tmem_st32(prow, z);
+            } else {
+                // scaled scores in log2 units; keys past the row's context (the diagonal block) are -inf
+                float x[64];
+#pragma unroll
+                for (int j = 0; j < 64; ++j) x[j] = __uint_as_float(sv[j]) * sl2;
+                if (nvalid < 64) {
+#pragma unroll
+                    for (int j = 0; j < 64; ++j)
+                        if (j >= nvalid) x[j] = neg_inf();
+                }
+                float m8[8];
+#pragma unroll
+                for (int i = 0; i < 8; ++i) m8[i] = fmaxf(fmaxf(fmaxf(x[i], x[i + 8]), fmaxf(x[i + 16], x[i + 24])),
+                                                          fmaxf(fmaxf(x[i + 32], x[i + 40]), fmaxf(x[i + 48], x[i + 56])));
+                const float mx = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])),
+                                       fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
+                const bool rescale = sel && mx > m_ref + 8.f;
+                const float new_ref = rescale ? mx : m_ref;
+                const float alpha = (rescale && l > 0.f) ? exp2_fast(m_ref - new_ref) : 1.f;
+                if (__any_sync(0xffffffffu, alpha != 1.f)) {
+                    // every PV so far must have landed before O is rewritten
+                    if (u >= 1) ok = wait_bar(&bars.o_done[(u - 1) & 1], ((u - 1) >> 1) & 1, err) && ok;
+                    ok = __all_sync(0xffffffffu, ok);
+                    if (!ok) break;
+#pragma unroll 1
+                    for (int c4 = 0; c4 < kD / 32; ++c4) {
+                        uint32_t o[32];
+                        tc::tmem_ld32(lane_addr + 32 * c4, o);
+                        tc::tmem_wait_ld();
+#pragma unroll
+                        for (int j = 0; j < 32; ++j) o[j] = __float_as_uint(__uint_as_float(o[j]) * alpha);
+                        tc::tmem_st32(lane_addr + 32 * c4, o);
+                    }
+                    tc::tmem_wait_st();
+                }
+                l *= alpha;
+                m_ref = new_ref;
+                // P = 2^(x - m_ref) (0 for unselected rows and masked keys), bf16 pairs along the keys
+                const float mneg = sel ? -m_ref : neg_inf();
+                float ps[4] = {0.f, 0.f, 0.f, 0.f};
+                uint32_t w[32];
+#pragma unroll
+                for (int j2 = 0; j2 < 32; ++j2) {
+                    const float p0 = ex2_approx(x[2 * j2] + mneg);
+                    const float p1 = ex2_approx(x[2 * j2 + 1] + mneg);
+                    ps[j2 & 3] += p0 + p1;
+                    w[j2] = pack_bf16(p0, p1);
+                }
+                tc::tmem_st32(prow, w);
+                l += (ps[0] + ps[1]) + (ps[2] + ps[3]);
+            }
+            tc::tmem_wait_st();
+            tc::tc_fence_before();
+            tc::mbar_arrive(&bars.p_full[sb]);
+        }
+        ok = __all_sync(0xffffffffu, ok);
+        if (ok && U > 0) ok = wait_bar(&bars.o_done[(U - 1) & 1], ((U - 1) >> 1) & 1, err);
+        ok = __all_sync(0xffffffffu, ok);
+        if (ok) {
+            tc::tc_fence_after();
+            const float inv = l > 0.f ? 1.f / l : 0.f;
+            __nv_bfloat16* orow = out + (((size_t)b * T + t) * qr.Hq + g * kG + hh) * kD;
+#pragma unroll 1
+            for (int c4 = 0; c4 < kD / 32; ++c4) {
+                uint32_t o[32];
+                tc::tmem_ld32(lane_addr + 32 * c4, o);
+                tc::tmem_wait_ld();
+                if (valid) {
+#pragma unroll
+                    for (int c = 0; c < 4; ++c) {
+                        uint32_t w[4];
+#pragma unroll
+                        for (int e = 0; e < 4; ++e)
+                            w[e] = pack_bf16(__uint_as_float(o[c * 8 + 2 * e]) * inv,
+                                             __uint_as_float(o[c * 8 + 2 * e + 1]) * inv);
+                        *reinterpret_cast<uint4*>(orow + c4 * 32 + c * 8) = make_uint4(w[0], w[1], w[2], w[3]);
+                    }
+                }
+            }
+            if (valid && lse)
+                lse[((size_t)b * T + t) * qr.Hq + g * kG + hh] = l > 0.f ? (m_ref + __log2f(l)) * kLn2 : neg_inf();
+        }
+    }
+    tc::tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc::tc_fence_after();
+        tc::tmem_dealloc(tmem, kTmemCols);
+    }
+}
+
+// ---------------------------------------------------------------- host
+namespace {
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn()
+{
+    static EncodeTiledFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+    });
+    return fn;
+}
+
+// 3-D bf16 map over rows of `inner` (=128) elements: dims {inner, mid, outer}, box {64, box_mid, box_outer}
+bool make_map(CUtensorMap* map, const void* base, uint64_t mid, uint64_t outer, uint64_t mid_stride_bytes,
+              uint64_t outer_stride_bytes, uint32_t box_mid, uint32_t box_outer)
+{
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    const cuuint64_t dims[3] = {(cuuint64_t)kD, mid, outer};
+    const cuuint64_t strides[2] = {mid_stride_bytes, outer_stride_bytes};
+    const cuuint32_t box[3] = {64, box_mid, box_outer};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+}  // namespace
+
+bool attn_tc_supported(const QueryRows& qr)
+{
+    return qr.D == kD && qr.Hq / qr.Hkv == kG && (qr.max_ctx - 1) / kBlock + 1 <= kMaxBlk;
+}
+
+cudaError_t launch_attn_rows_tc(const QueryRows& qr, const void* k, const void* v, int Lcap, const int32_t* idx,
+                                const int32_t* cnt, const MethodConsts& mc, bool dense_all, void* out, float* lse,
+                                cudaStream_t s)
+{
+    if (!attn_tc_supported(qr)) return cudaErrorNotSupported;
+    CUtensorMap tq, tk, tv;
+    const uint64_t row = (uint64_t)kD * 2;
+    if (!make_map(&tq, qr.q, qr.Hq, (uint64_t)qr.B * qr.T, row, row * qr.Hq, kG, kTok) ||
+        !make_map(&tk, k, qr.Hkv, (uint64_t)qr.B * Lcap, row, row * qr.Hkv, 1, kBlock) ||
+        !make_map(&tv, v, qr.Hkv, (uint64_t)qr.B * Lcap, row, row * qr.Hkv, 1, kBlock))
+        return cudaErrorNotSupported;
+    cudaError_t e = ensure_smem(attn_tc_kernel, kSmemBytes);
+    if (e != cudaSuccess) return e;
+    const dim3 grid((qr.T + kTok - 1) / kTok, qr.B * qr.Hkv);
+    return launch_pdl(attn_tc_kernel, grid, dim3(kThreads), (size_t)kSmemBytes, s, qr, tq, tk, tv, Lcap, idx, cnt,
+                      mc, dense_all ? 1 : 0, static_cast<__nv_bfloat16*>(out), lse);
+}
+
+int tc_error_flag_read_and_clear()
+{
+    int h = 0;
+    if (cudaMemcpyFromSymbol(&h, g_tc_error, sizeof(int)) != cudaSuccess) return -1;
+    if (h) {
+        const int zero = 0;
+        cudaMemcpyToSymbol(g_tc_error, &zero, sizeof(int));
+    }
+    return h;
+}
+
+}  // namespace iv2

@@ -135,4 +135,13 @@ IV2_DEV void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 // fast 2^x (MUFU) -- inputs are <= 0 or -inf on every use in this library
 IV2_DEV float exp2_fast(float x) { return exp2f(x); }
 
+// the hardware 2^x approximation (MUFU.EX2, flush-to-zero): 2^-inf = 0; used where the result is rounded
+// to bf16 right away
+IV2_DEV float ex2_approx(float x)
+{
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
 }  // namespace iv2

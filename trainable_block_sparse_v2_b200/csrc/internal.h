@@ -107,6 +107,14 @@ cudaError_t launch_attn_rows(const QueryRows& qr, const void* k, const void* v, 
                              const int32_t* cnt, const MethodConsts& mc, bool dense_all, void* out, float* lse,
                              cudaStream_t s);
 
+// the same on tcgen05/TMEM with TMA-staged K/V (16 heads per group, d = 128); cudaErrorNotSupported otherwise
+bool attn_tc_supported(const QueryRows& qr);
+cudaError_t launch_attn_rows_tc(const QueryRows& qr, const void* k, const void* v, int Lcap, const int32_t* idx,
+                                const int32_t* cnt, const MethodConsts& mc, bool dense_all, void* out, float* lse,
+                                cudaStream_t s);
+// device-side error flag of the bounded waits (1 = a wait ran out); reading clears it; -1 on a CUDA error
+int tc_error_flag_read_and_clear();
+
 // attention split over the selected blocks across CTAs, merged by LSE (decode and tree verification)
 cudaError_t launch_attn_split(const QueryRows& qr, const void* k, const void* v, int Lcap, const int32_t* idx,
                               const int32_t* cnt, const MethodConsts& mc, bool dense_all, const void* k_draft,
