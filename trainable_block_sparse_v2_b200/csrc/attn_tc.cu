@@ -5,18 +5,18 @@
 // share the block set).  Specialised for 16 query heads per KV group and head_dim 128.
 //
 // One CTA owns a 128-row tile = 8 consecutive query tokens x the 16 heads of one KV group, and walks the
-// ascending union of those tokens' selected blocks (a token attends to a block only when it selected it;
-// other rows of the tile are masked for that block).  Per 64-key block:
-//   S[128 x 64]  = Q[128 x 128] . K_blk^T   tcgen05.mma kind::f16 with A (Q) in TMEM and B (K) K-major in
+// ascending union of those tokens' selected blocks two blocks (128 keys) at a time (a token attends to a
+// block only when it selected it; other rows of the tile are masked for that block).  Per step:
+//   S[128 x 128] = Q[128 x 128] . K^T       tcgen05.mma kind::f16 with A (Q) in TMEM and B (K) K-major in
 //                                            128B-swizzled smem, fp32 accumulator in TMEM (two S buffers)
 //   P            = online softmax of S       four warps, one TMEM lane (= one query row) per thread; P goes
-//                                            back to TMEM as bf16 pairs (two P buffers); the output is
-//                                            rescaled only when a row's max grows by more than 2^8 (exact:
+//                                            back to TMEM as bf16 pairs over its own S buffer; the output
+//                                            is rescaled only when a row's max grows by more than 2^8 (exact:
 //                                            O and the row sum share the reference max)
-//   O[128 x 128] += P[128 x 64] . V_blk      A (P) in TMEM, B (V) MN-major in smem, O in TMEM
-// Keeping Q and P in TMEM leaves shared memory to the K/V stream: the operand reads of a block drop from
-// 80 KB to 32 KB.
-// Warp roles: warp 0 issues TMA loads (Q once, K/V per block into 4 stages), warp 1 (one thread) issues the
+//   O[128 x 128] += P[128 x 128] . V         A (P) in TMEM, B (V) MN-major in smem, O in TMEM
+// Keeping Q and P in TMEM leaves shared memory to the K/V stream, and 128-key steps halve the number of
+// MMA instructions and pipeline hand-offs per key.
+// Warp roles: warp 0 issues TMA loads (Q once; K and V per step into 3-deep rings, one lane each), warp 1 (one thread) issues the
 // MMAs, warps 2-5 run the softmax and the epilogue.  Producer/consumer hand-offs use mbarriers; MMA
 // completion is signalled with tcgen05.commit.  Every wait is bounded: after the limit the CTA records an
 // error (g_tc_error), skips the rest of its work, frees its TMEM and exits.
@@ -38,21 +38,26 @@ constexpr int kD = 128;           // head dim
 constexpr int kThreads = 192;     // 6 warps
 constexpr int kMaxBlk = 4096;     // context blocks (256K keys)
 constexpr int kWords = kMaxBlk / 32;
-constexpr uint32_t kTmemCols = 512;  // O [0,128), S0/S1 [128,256), P0/P1 [256,320), Q [320,384)
-constexpr uint32_t kColS = 128, kColP = 256, kColQ = 320;
+constexpr int kStepKeys = 128;       // two 64-key blocks per pipeline step
+constexpr uint32_t kTmemCols = 512;  // O [0,128), S0 [128,256), S1 [256,384), Q [384,448); P(step) overwrites
+                                     // the first 64 columns of its own S buffer
+constexpr uint32_t kColS = 128, kColQ = 384;
 
-// dynamic shared memory layout (base aligned to 1024 B)
-constexpr int kQOff = 0;                     // 2 atoms x 128 rows x 128 B
-constexpr int kStages = 4;                   // K/V pipeline depth: hides the load latency of 3 blocks
-constexpr int kKvOff = 32768;                // kStages x (K0, K1, V0, V1) x 64 rows x 128 B
-constexpr int kKvStage = 32768;
-constexpr int kBitsOff = kKvOff + kStages * kKvStage;  // [kTok][kWords] uint32
+// dynamic shared memory layout (base aligned to 1024 B).  K and V stream through separate rings so each
+// can be refilled as soon as its own MMA has consumed it; Q is staged once in the last V slot (it is
+// copied into TMEM before that slot is first filled).
+constexpr int kRing = 3;                     // ring depth, in steps of 128 keys
+constexpr int kSlot = 32768;                 // one step of K or V: two d-halves x 128 key rows x 128 B
+constexpr int kKOff = 0;
+constexpr int kVOff = kKOff + kRing * kSlot;
+constexpr int kQOff = kVOff + (kRing - 1) * kSlot;  // 2 atoms x 128 rows x 128 B, aliases V slot kRing-1
+constexpr int kBitsOff = kVOff + kRing * kSlot;     // [kTok][kWords] uint32
 constexpr int kListOff = kBitsOff + kTok * kWords * 4;  // uint16 block ids
 constexpr int kSmemBytes = kListOff + kMaxBlk * 2 + 1024;  // + alignment slack
 
 struct Bars {
     uint64_t q_full, q_tmem;
-    uint64_t kv_full[kStages], kv_empty[kStages];
+    uint64_t k_full[kRing], k_empty[kRing], v_full[kRing], v_empty[kRing];
     uint64_t s_full[2], p_full[2], o_done[2];
     uint32_t tmem_base;
     int n_union;
@@ -151,9 +156,11 @@ attn_tc_kernel(QueryRows qr, const __grid_constant__ CUtensorMap tm_q, const __g
     if (threadIdx.x == 0) {
         tc::mbar_init(&bars.q_full, 1);
         tc::mbar_init(&bars.q_tmem, 128);
-        for (int i = 0; i < kStages; ++i) {
-            tc::mbar_init(&bars.kv_full[i], 1);
-            tc::mbar_init(&bars.kv_empty[i], 1);
+        for (int i = 0; i < kRing; ++i) {
+            tc::mbar_init(&bars.k_full[i], 1);
+            tc::mbar_init(&bars.k_empty[i], 1);
+            tc::mbar_init(&bars.v_full[i], 1);
+            tc::mbar_init(&bars.v_empty[i], 1);
         }
         for (int i = 0; i < 2; ++i) {
             tc::mbar_init(&bars.s_full[i], 1);
@@ -173,62 +180,85 @@ attn_tc_kernel(QueryRows qr, const __grid_constant__ CUtensorMap tm_q, const __g
     const uint32_t tmem = bars.tmem_base;
     volatile int* err = &bars.err;
 
-    const uint32_t sKV = tc::smem_u32(smem + kKvOff);
+    const uint32_t sK = tc::smem_u32(smem + kKOff);
+    const uint32_t sV = tc::smem_u32(smem + kVOff);
 
+    const int NP = (U + 1) / 2;  // pipeline steps; an odd last block is paired with a masked copy of itself
     if (warp == 0) {
-        // ---------------- TMA producer ----------------
+        // ---------------- TMA producers: lane 0 streams K (and Q first), lane 1 streams V ----------------
         if (lane == 0) {
             tc::prefetch_tensormap(&tm_q);
             tc::prefetch_tensormap(&tm_k);
-            tc::prefetch_tensormap(&tm_v);
             tc::mbar_arrive_expect_tx(&bars.q_full, 2 * 128 * 128);
             const int zq = b * T + t0;
             tc::tma_load_3d(smem + kQOff, &tm_q, 0, g * kG, zq, &bars.q_full);
             tc::tma_load_3d(smem + kQOff + 16384, &tm_q, 64, g * kG, zq, &bars.q_full);
-            for (int u = 0; u < U; ++u) {
-                const int s = u % kStages, k = u / kStages;
-                if (k >= 1 && !wait_bar(&bars.kv_empty[s], (k - 1) & 1, err)) break;
-                const int z = b * Lcap + (int)list[u] * kBlock;
-                unsigned char* st = smem + kKvOff + s * kKvStage;
-                tc::mbar_arrive_expect_tx(&bars.kv_full[s], kKvStage);
-                tc::tma_load_3d(st, &tm_k, 0, g, z, &bars.kv_full[s]);
-                tc::tma_load_3d(st + 8192, &tm_k, 64, g, z, &bars.kv_full[s]);
-                tc::tma_load_3d(st + 16384, &tm_v, 0, g, z, &bars.kv_full[s]);
-                tc::tma_load_3d(st + 24576, &tm_v, 64, g, z, &bars.kv_full[s]);
+            for (int p = 0; p < NP; ++p) {
+                const int s = p % kRing, k = p / kRing;
+                if (k >= 1 && !wait_bar(&bars.k_empty[s], (k - 1) & 1, err)) break;
+                unsigned char* st = smem + kKOff + s * kSlot;
+                tc::mbar_arrive_expect_tx(&bars.k_full[s], kSlot);
+#pragma unroll
+                for (int i = 0; i < 2; ++i) {
+                    // key rows [64 i, 64 i + 64) of the step, d halves in two atoms of 128 rows
+                    const int z = b * Lcap + (int)list[min(2 * p + i, U - 1)] * kBlock;
+                    tc::tma_load_3d(st + i * 8192, &tm_k, 0, g, z, &bars.k_full[s]);
+                    tc::tma_load_3d(st + 16384 + i * 8192, &tm_k, 64, g, z, &bars.k_full[s]);
+                }
+            }
+        } else if (lane == 1) {
+            tc::prefetch_tensormap(&tm_v);
+            for (int p = 0; p < NP; ++p) {
+                const int s = p % kRing, k = p / kRing;
+                if (k >= 1 && !wait_bar(&bars.v_empty[s], (k - 1) & 1, err)) break;
+                // the last slot holds Q until the softmax warps have copied it into TMEM
+                if (p == kRing - 1 && !wait_bar(&bars.q_tmem, 0, err)) break;
+                unsigned char* st = smem + kVOff + s * kSlot;
+                tc::mbar_arrive_expect_tx(&bars.v_full[s], kSlot);
+#pragma unroll
+                for (int i = 0; i < 2; ++i) {
+                    const int z = b * Lcap + (int)list[min(2 * p + i, U - 1)] * kBlock;
+                    tc::tma_load_3d(st + i * 8192, &tm_v, 0, g, z, &bars.v_full[s]);
+                    tc::tma_load_3d(st + 16384 + i * 8192, &tm_v, 64, g, z, &bars.v_full[s]);
+                }
             }
         }
     } else if (warp == 1) {
         // ---------------- MMA issuer ----------------
         if (lane == 0 && wait_bar(&bars.q_tmem, 0, err)) {
             tc::tc_fence_after();
-            constexpr uint32_t idesc_s = tc::idesc_bf16(128, 64, false);
+            constexpr uint32_t idesc_s = tc::idesc_bf16(128, kStepKeys, false);
             constexpr uint32_t idesc_o = tc::idesc_bf16(128, kD, true);
-            for (int u = 0; u <= U; ++u) {
-                if (u < U) {
-                    const int s = u % kStages, sb = u & 1;
-                    if (!wait_bar(&bars.kv_full[s], (u / kStages) & 1, err)) break;
+            for (int p = 0; p <= NP; ++p) {
+                if (p < NP) {
+                    // S(p) = Q . [K_a ; K_b]^T into S buffer p&1 (in-order after PV(p-2), which read P(p-2) there)
+                    const int s = p % kRing, sb = p & 1;
+                    if (!wait_bar(&bars.k_full[s], (p / kRing) & 1, err)) break;
                     tc::tc_fence_after();
-                    const uint32_t d_s = tmem + kColS + 64 * sb;
-                    const uint32_t kbase = sKV + s * kKvStage;
+                    const uint32_t d_s = tmem + kColS + kStepKeys * sb;
+                    const uint32_t kbase = sK + s * kSlot;
 #pragma unroll
                     for (int ks = 0; ks < kD / 16; ++ks) {
-                        const uint32_t koff = (ks >> 2) * 8192 + (ks & 3) * 32;
+                        const uint32_t koff = (ks >> 2) * 16384 + (ks & 3) * 32;
                         tc::mma_bf16_ts(d_s, tmem + kColQ + 8 * ks, tc::desc_kmajor_sw128(kbase + koff), idesc_s,
                                         ks > 0);
                     }
                     tc::mma_commit(&bars.s_full[sb]);
+                    tc::mma_commit(&bars.k_empty[s]);
                 }
-                if (u >= 1) {
-                    const int v = u - 1, pv = v & 1;
+                if (p >= 1) {
+                    // O += P(v) . [V_a ; V_b], P(v) in the first 64 columns of S buffer v&1
+                    const int v = p - 1, pv = v & 1;
                     if (!wait_bar(&bars.p_full[pv], (v >> 1) & 1, err)) break;
+                    if (!wait_bar(&bars.v_full[v % kRing], (v / kRing) & 1, err)) break;
                     tc::tc_fence_after();
-                    const uint32_t vbase = sKV + (v % kStages) * kKvStage + 16384;
+                    const uint32_t vbase = sV + (v % kRing) * kSlot;
 #pragma unroll
-                    for (int ks = 0; ks < kBlock / 16; ++ks)
-                        tc::mma_bf16_ts(tmem, tmem + kColP + 32 * pv + 8 * ks,
-                                        tc::desc_mnmajor_sw128(vbase + ks * 2048, 8192), idesc_o, (v > 0 || ks > 0));
+                    for (int ks = 0; ks < kStepKeys / 16; ++ks)
+                        tc::mma_bf16_ts(tmem, tmem + kColS + kStepKeys * pv + 8 * ks,
+                                        tc::desc_mnmajor_sw128(vbase + ks * 2048, 16384), idesc_o, (v > 0 || ks > 0));
                     tc::mma_commit(&bars.o_done[pv]);
-                    tc::mma_commit(&bars.kv_empty[v % kStages]);
+                    tc::mma_commit(&bars.v_empty[v % kRing]);
                 }
             }
         }
@@ -265,58 +295,57 @@ attn_tc_kernel(QueryRows qr, const __grid_constant__ CUtensorMap tm_q, const __g
             tc::mbar_arrive(&bars.q_tmem);
         }
         ok = __all_sync(0xffffffffu, ok);
-        for (int u = 0; u < U && ok; ++u) {
-            const int sb = u & 1;
-            ok = wait_bar(&bars.s_full[sb], (u >> 1) & 1, err);
+        for (int p = 0; p < NP && ok; ++p) {
+            const int sb = p & 1;
+            ok = wait_bar(&bars.s_full[sb], (p >> 1) & 1, err);
             ok = __all_sync(0xffffffffu, ok);
             if (!ok) break;
             tc::tc_fence_after();
-            const int blk = list[u];
-            const bool sel = valid && ((bits[tt * kWords + (blk >> 5)] >> (blk & 31)) & 1u);
-            uint32_t sv[64];
-            {
-                uint32_t a[32], c2[32];
-                tc::tmem_ld32(lane_addr + kColS + 64 * sb, a);
-                tc::tmem_ld32(lane_addr + kColS + 64 * sb + 32, c2);
-                tc::tmem_wait_ld();
-#pragma unroll
-                for (int j = 0; j < 32; ++j) {
-                    sv[j] = a[j];
-                    sv[32 + j] = c2[j];
-                }
-            }
-            // the P buffer of this block was last read by PV(u-2)
-            if (u >= 2) ok = wait_bar(&bars.o_done[sb], ((u - 2) >> 1) & 1, err);
-            const int nvalid = sel ? min(kBlock, n - blk * kBlock) : 0;
-            const uint32_t prow = lane_addr + kColP + 32 * sb;
-            if (!__any_sync(0xffffffffu, sel)) {
-                // neither token of this warp selected the block: its P rows are zero
+            // the step's two blocks, whether this row's token selected each, and its keys in each
+            const int blk_a = list[2 * p];
+            const bool has_b = 2 * p + 1 < U;
+            const int blk_b = has_b ? list[2 * p + 1] : blk_a;
+            const bool sel_a = valid && ((bits[tt * kWords + (blk_a >> 5)] >> (blk_a & 31)) & 1u);
+            const bool sel_b = valid && has_b && ((bits[tt * kWords + (blk_b >> 5)] >> (blk_b & 31)) & 1u);
+            const int nv_a = sel_a ? min(kBlock, n - blk_a * kBlock) : 0;
+            const int nv_b = sel_b ? min(kBlock, n - blk_b * kBlock) : 0;
+            const uint32_t srow = lane_addr + kColS + kStepKeys * sb;
+            if (!__any_sync(0xffffffffu, sel_a || sel_b)) {
+                // neither token of this warp selected either block: its P rows are zero
                 uint32_t z[32];
 #pragma unroll
                 for (int j = 0; j < 32; ++j) z[j] = 0u;
-                tc::tmem_st32(prow, z);
+                tc::tmem_st32(srow, z);
+                tc::tmem_st32(srow + 32, z);
             } else {
-                // scaled scores in log2 units; keys past the row's context (the diagonal block) are -inf
-                float x[64];
+                // scaled scores in log2 units; unselected blocks and keys past the row's context are -inf
+                float x[kStepKeys];
 #pragma unroll
-                for (int j = 0; j < 64; ++j) x[j] = __uint_as_float(sv[j]) * sl2;
-                if (nvalid < 64) {
+                for (int h = 0; h < 4; ++h) {
+                    uint32_t sv[32];
+                    tc::tmem_ld32(srow + 32 * h, sv);
+                    tc::tmem_wait_ld();
+                    const int nv = h < 2 ? nv_a : nv_b;
 #pragma unroll
-                    for (int j = 0; j < 64; ++j)
-                        if (j >= nvalid) x[j] = neg_inf();
+                    for (int j = 0; j < 32; ++j)
+                        x[32 * h + j] = ((h & 1) * 32 + j) < nv ? __uint_as_float(sv[j]) * sl2 : neg_inf();
                 }
                 float m8[8];
 #pragma unroll
-                for (int i = 0; i < 8; ++i) m8[i] = fmaxf(fmaxf(fmaxf(x[i], x[i + 8]), fmaxf(x[i + 16], x[i + 24])),
-                                                          fmaxf(fmaxf(x[i + 32], x[i + 40]), fmaxf(x[i + 48], x[i + 56])));
+                for (int i = 0; i < 8; ++i) {
+                    float m = x[i];
+#pragma unroll
+                    for (int j = 1; j < 16; ++j) m = fmaxf(m, x[i + 8 * j]);
+                    m8[i] = m;
+                }
                 const float mx = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])),
                                        fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
-                const bool rescale = sel && mx > m_ref + 8.f;
+                const bool rescale = mx > m_ref + 8.f;  // mx is -inf for a row that selected neither block
                 const float new_ref = rescale ? mx : m_ref;
                 const float alpha = (rescale && l > 0.f) ? exp2_fast(m_ref - new_ref) : 1.f;
                 if (__any_sync(0xffffffffu, alpha != 1.f)) {
                     // every PV so far must have landed before O is rewritten
-                    if (u >= 1) ok = wait_bar(&bars.o_done[(u - 1) & 1], ((u - 1) >> 1) & 1, err) && ok;
+                    if (p >= 1) ok = wait_bar(&bars.o_done[(p - 1) & 1], ((p - 1) >> 1) & 1, err) && ok;
                     ok = __all_sync(0xffffffffu, ok);
                     if (!ok) break;
 #pragma unroll 1
@@ -332,18 +361,21 @@ attn_tc_kernel(QueryRows qr, const __grid_constant__ CUtensorMap tm_q, const __g
                 }
                 l *= alpha;
                 m_ref = new_ref;
-                // P = 2^(x - m_ref) (0 for unselected rows and masked keys), bf16 pairs along the keys
-                const float mneg = sel ? -m_ref : neg_inf();
+                // P = 2^(x - m_ref), bf16 pairs along the keys, over the first 64 columns of this S buffer
+                const float mneg = (sel_a || sel_b) ? -m_ref : neg_inf();
                 float ps[4] = {0.f, 0.f, 0.f, 0.f};
-                uint32_t w[32];
 #pragma unroll
-                for (int j2 = 0; j2 < 32; ++j2) {
-                    const float p0 = ex2_approx(x[2 * j2] + mneg);
-                    const float p1 = ex2_approx(x[2 * j2 + 1] + mneg);
-                    ps[j2 & 3] += p0 + p1;
-                    w[j2] = pack_bf16(p0, p1);
+                for (int h = 0; h < 2; ++h) {
+                    uint32_t w[32];
+#pragma unroll
+                    for (int j2 = 0; j2 < 32; ++j2) {
+                        const float p0 = ex2_approx(x[64 * h + 2 * j2] + mneg);
+                        const float p1 = ex2_approx(x[64 * h + 2 * j2 + 1] + mneg);
+                        ps[j2 & 3] += p0 + p1;
+                        w[j2] = pack_bf16(p0, p1);
+                    }
+                    tc::tmem_st32(srow + 32 * h, w);
                 }
-                tc::tmem_st32(prow, w);
                 l += (ps[0] + ps[1]) + (ps[2] + ps[3]);
             }
             tc::tmem_wait_st();
@@ -351,7 +383,7 @@ attn_tc_kernel(QueryRows qr, const __grid_constant__ CUtensorMap tm_q, const __g
             tc::mbar_arrive(&bars.p_full[sb]);
         }
         ok = __all_sync(0xffffffffu, ok);
-        if (ok && U > 0) ok = wait_bar(&bars.o_done[(U - 1) & 1], ((U - 1) >> 1) & 1, err);
+        if (ok && NP > 0) ok = wait_bar(&bars.o_done[(NP - 1) & 1], ((NP - 1) >> 1) & 1, err);
         ok = __all_sync(0xffffffffu, ok);
         if (ok) {
             tc::tc_fence_after();
