@@ -38,7 +38,8 @@ UNIT = "tokens/s"
 PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 LENS_128K = (131072, 98304, 65536, 131072)
 HQ, HKV, D = 32, 2, 128
-KERNELS_PER_STEP = 5  # kernel pool, score scan, select, split attention, merge
+KERNELS_PER_STEP = {"two_call": 5,  # kernel pool, score scan, select, split attention, merge
+                    "fused": 2}     # kernel pool, fused decode step (scoring + top-k + attention)
 
 
 def load_peaks():
@@ -123,13 +124,14 @@ def decode_step_bytes(lens, kmax=67):
 
 
 class DecodeBench:
-    def __init__(self, layers=8, steps_cycle=256):
+    def __init__(self, layers=8, steps_cycle=256, two_call=True):
         import torch
         from trainable_block_sparse_v2_b200 import binding
         from trainable_block_sparse_v2_b200.workloads import decode_128k_ragged
 
         self.torch, self.b = torch, binding
         self.NL, self.S = layers, steps_cycle
+        self.two_call = two_call
         w = decode_128k_ragged(steps=steps_cycle)
         self.w = w
         self.p = binding.Params(**w.params)
@@ -169,7 +171,8 @@ class DecodeBench:
     def q_of(self, layer, pos):
         return self.q_all[(pos + 37 * layer) % self.S]
 
-    # the three C-ABI calls of one decode step
+    # the C-ABI calls of one decode step: incremental kernel pooling, then scoring + top-k + sparse attention
+    # fused in one launch (infllmv2_sparse_decode_step; the two-call form is block_score_topk + sparse_attn_decode)
     def pool(self, layer, pos, stream=None):
         self.b.infllmv2_kernel_pool(self.k[layer], self.old[pos], self.lens[pos], 1, self.p, self.kern[layer], stream)
 
@@ -181,11 +184,19 @@ class DecodeBench:
         self.b.infllmv2_sparse_attn_decode(self.q_of(layer, pos), self.k[layer], self.v[layer], self.lens[pos],
                                            self.max_ctx, self.idx, self.cnt, self.p, self.out, None, self.ws, stream)
 
+    def fused(self, layer, pos, stream=None):
+        self.b.infllmv2_sparse_decode_step(self.q_of(layer, pos), self.kern[layer], self.k[layer], self.v[layer],
+                                           self.lens[pos], self.max_ctx, self.p, self.idx, self.cnt, self.out, None,
+                                           stream)
+
     def step_eager(self, s, stream=None):
         layer, pos = self._coords(s)
         self.pool(layer, pos, stream)
-        self.score(layer, pos, stream)
-        self.attend(layer, pos, stream)
+        if self.two_call:
+            self.score(layer, pos, stream)
+            self.attend(layer, pos, stream)
+        else:
+            self.fused(layer, pos, stream)
 
     def graph(self, s):
         torch = self.torch
@@ -222,8 +233,8 @@ class DecodeBench:
     def per_call_times(self, warmup, steps):
         """average device time of each C-ABI call, CUDA events around each launch on the current stream"""
         torch = self.torch
-        names = ["kernel_pool", "block_score_topk", "sparse_attn_decode"]
-        fns = [self.pool, self.score, self.attend]
+        names = ["kernel_pool", "block_score_topk", "sparse_attn_decode", "sparse_decode_step"]
+        fns = [self.pool, self.score, self.attend, self.fused]
         ev = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
               for _ in fns]
         for s in range(warmup):
@@ -265,10 +276,15 @@ class DecodeBench:
                 self.k[layer][b, row].copy_(kv_host[pos, 0, b], non_blocking=True)
                 self.v[layer][b, row].copy_(kv_host[pos, 1, b], non_blocking=True)
             self.b.infllmv2_kernel_pool(self.k[layer], self.old[pos], self.lens[pos], 1, self.p, self.kern[layer])
-            self.b.infllmv2_block_score_topk(q_dev, None, self.lens[pos], self.max_ctx, self.kern[layer], self.p,
-                                             self.idx, self.cnt, self.ws)
-            self.b.infllmv2_sparse_attn_decode(q_dev, self.k[layer], self.v[layer], self.lens[pos], self.max_ctx,
-                                               self.idx, self.cnt, self.p, self.out, None, self.ws)
+            if self.two_call:
+                self.b.infllmv2_block_score_topk(q_dev, None, self.lens[pos], self.max_ctx, self.kern[layer], self.p,
+                                                 self.idx, self.cnt, self.ws)
+                self.b.infllmv2_sparse_attn_decode(q_dev, self.k[layer], self.v[layer], self.lens[pos], self.max_ctx,
+                                                   self.idx, self.cnt, self.p, self.out, None, self.ws)
+            else:
+                self.b.infllmv2_sparse_decode_step(q_dev, self.kern[layer], self.k[layer], self.v[layer],
+                                                   self.lens[pos], self.max_ctx, self.p, self.idx, self.cnt, self.out,
+                                                   None)
             out_host.copy_(self.out, non_blocking=True)
 
         for s in range(warmup):
@@ -449,7 +465,8 @@ def run_ours(args):
     binding.load()
     peaks, peak_kind = load_peaks()
 
-    db = DecodeBench(layers=args.layers)
+    two_call = args.decode_path == "two_call"
+    db = DecodeBench(layers=args.layers, two_call=two_call)
     # timed region: exactly K decode steps (graph replays), barrier + synchronize on both sides
     for s in range(args.warmup + args.steps):
         db.graph(s)
@@ -462,12 +479,18 @@ def run_ours(args):
     value = tokens / t
 
     per = db.per_call_times(8, min(args.steps, 256)) if args.per_call else {
-        "kernel_pool": float("nan"), "block_score_topk": float("nan"), "sparse_attn_decode": float("nan")}
+        "kernel_pool": float("nan"), "block_score_topk": float("nan"), "sparse_attn_decode": float("nan"),
+        "sparse_decode_step": float("nan")}
     lens_mid = [n + 128 for n in LENS_128K]
     scan_b, kv_b, step_b = decode_step_bytes(lens_mid)
-    dom = max(per, key=lambda k: -1.0 if per[k] != per[k] else per[k])
-    dom_bytes = {"sparse_attn_decode": kv_b, "block_score_topk": scan_b,
-                 "kernel_pool": len(LENS_128K) * HKV * D * 2 * 33}[dom]
+    if two_call:
+        # dominant call of the two-call step: the larger of block scoring + top-k and sparse attention
+        dom = max(("block_score_topk", "sparse_attn_decode"), key=lambda k: per[k] if per[k] == per[k] else -1.0)
+        dom_bytes = {"block_score_topk": scan_b, "sparse_attn_decode": kv_b}[dom]
+    else:
+        # the fused scoring + top-k + attention launch carries the whole step's traffic
+        dom = "sparse_decode_step"
+        dom_bytes = scan_b + kv_b
     achieved = dom_bytes / per[dom] / 1e9
     e2e_steps = min(args.steps, 512)
     e2e_t, h2d, d2h = db.e2e(8, e2e_steps) if args.e2e else (float("nan"), 0, 0)
@@ -482,8 +505,10 @@ def run_ours(args):
                    "layers_rotating": args.layers, "parallelism": f"replicas{ws}",
                    "l2": "inputs larger than L2: 8 rotating layer caches, each step's 31 MB working set is evicted "
                          "before its layer returns",
-                   "step": "one decode step of one layer for 4 sequences: kernel_pool + block_score_topk + "
-                           "sparse_attn_decode (CUDA graph)"},
+                   "step": ("one decode step of one layer for 4 sequences: kernel_pool + block_score_topk + "
+                            "sparse_attn_decode, replayed as a CUDA graph" if two_call else
+                            "one decode step of one layer for 4 sequences: kernel_pool + sparse_decode_step "
+                            "(scoring, top-k and sparse attention in one cluster kernel), replayed as a CUDA graph")},
         "hbm": {"algorithmic_bytes_per_step": step_b, "achieved_gbs_per_gpu": step_b / (t / args.steps) / 1e9,
                 "frac_of_" + peak_kind: step_b / (t / args.steps) / 1e9 / peaks["hbm_gbs"]},
         "per_call_ms": {k: v * 1e3 for k, v in per.items()},
@@ -493,7 +518,7 @@ def run_ours(args):
         "clocks": clk.summary(),
         "e2e": {"value": len(LENS_128K) * e2e_steps / e2e_t, "unit": UNIT, "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "steps": e2e_steps},
-        "gpu_launches": KERNELS_PER_STEP * args.steps,
+        "gpu_launches": KERNELS_PER_STEP[args.decode_path] * args.steps,
     }
     del db
     torch.cuda.empty_cache()
@@ -582,6 +607,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=64)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--layers", type=int, default=8)
+    ap.add_argument("--decode-path", choices=["two_call", "fused"], default="two_call",
+                    help="decode step as block_score_topk + sparse_attn_decode, or the one-launch sparse_decode_step")
     ap.add_argument("--prefill-steps", type=int, default=3)
     ap.add_argument("--no-prefill", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")

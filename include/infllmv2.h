@@ -165,6 +165,22 @@ int infllmv2_sparse_attn_decode(const void* q, int batch, int hq, int hkv, int h
                                 size_t ws_bytes, infllmv2_stream_t stream);
 
 /*
+ * Steps 2 + 3b fused -- one decode step: block scoring, top-k selection and sparse attention of one new
+ * token per sequence in a single launch, with no workspace (efficiency evaluation of the QbitAI article:
+ * a decode step reads a constant number of blocks plus the kernel representations).  Writes exactly what
+ * infllmv2_block_score_topk followed by infllmv2_sparse_attn_decode write (idx, cnt, out, lse) for the
+ * same inputs: q [B, 1, Hq, d], n = ctx_lens[b], kernels visible up to n.  One thread-block cluster per
+ * (sequence, KV group) scans the kernel cache, merges the per-head LSE partials and the block scores
+ * over distributed shared memory, selects, and attends to the selected blocks.
+ *   kern [B, Hkv, nk_cap, d]: the kernel cache, already pooled up to ctx_lens (infllmv2_kernel_pool).
+ *   Limits: contexts up to 256K keys; B * Hkv <= 65535.
+ */
+int infllmv2_sparse_decode_step(const void* q, int batch, int hq, int hkv, int head_dim, const void* kern, int nk_cap,
+                                const void* k, const void* v, int lcap, const int32_t* ctx_lens, int max_ctx,
+                                const infllmv2_params* params, int32_t* idx, int32_t* cnt, void* out, float* lse,
+                                infllmv2_stream_t stream);
+
+/*
  * Step 3c -- tree-draft verification (QbitAI article, "speculative sampling, quantisation and long text",
  * long-context bullet).  n_draft draft tokens per sequence, each a query that sees the whole prefix of
  * prefix_lens[b] cache keys through its own selected blocks (its q_ctx is the prefix length), plus the

@@ -54,6 +54,30 @@ def test_decode_32k(oracle):
         assert np.isin(w.extras["needles"][0], idx[0, 0, g].cpu().numpy()).mean() >= 0.75
 
 
+def test_decode_32k_and_128k_fused_step(oracle):
+    """The fused decode step at full size: 32K (batch 1) and the 128K ragged batch at its first step."""
+    for w in (W.decode_32k(), W.decode_128k_ragged(steps=1)):
+        B = w.q.shape[0]
+        L = w.ctx_lens.astype(np.int64)
+        p, P = bparams(w.params), oparams(w.params)
+        K, V, q = dev(w.k), dev(w.v), dev(w.q)
+        max_ctx = int(L.max())
+        nk_cap = nk(max_ctx)
+        kern = torch.zeros((B, 2, nk_cap, 128), dtype=torch.bfloat16, device="cuda")
+        binding.infllmv2_kernel_pool(K, dev_i32(np.zeros(B)), dev_i32(L), max_ctx, p, kern)
+        idx = torch.empty((B, 1, 2, p.kmax), dtype=torch.int32, device="cuda")
+        cnt = torch.empty((B, 1, 2), dtype=torch.int32, device="cuda")
+        out = torch.empty((B, 1, 32, 128), dtype=torch.bfloat16, device="cuda")
+        lse = torch.empty((B, 1, 32), dtype=torch.float32, device="cuda")
+        binding.infllmv2_sparse_decode_step(q, kern, K, V, dev_i32(L), max_ctx, p, idx, cnt, out, lse)
+        torch.cuda.synchronize()
+        kern_o = oracle.kernel_pool(w.k, np.zeros(B), L, 32, 16, nk_cap=nk_cap)
+        r = oracle.block_score_topk(w.q, kern_o, w.q_ctx, P)
+        same = check_selection(idx.cpu().numpy(), cnt.cpu().numpy(), r)
+        out_o, lse_o = oracle.sparse_attention(w.q, w.k, w.v, w.q_ctx, r["idx"], r["cnt"], P)
+        check_attention(out, out_o, lse, lse_o, mask=same.all(axis=-1), what=f"fused decode {w.name}")
+
+
 def test_prefill_32k_sampled_rows(oracle):
     """32K prefill, dense below 8192; rows sampled across the dense part, the switch and the sparse part."""
     w = W.prefill_32k()

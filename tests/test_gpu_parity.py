@@ -275,3 +275,28 @@ def test_selection_ties_go_to_lower_block(oracle, path):
     kern_o = oracle.kernel_pool(w.k, [0] * B, list(w.ctx_lens), 32, 16, nk_cap=nk_cap)
     r = oracle.block_score_topk(w.q, kern_o, w.q_ctx, oparams(w.params))
     assert np.array_equal(r["idx"], gidx) and np.array_equal(r["cnt"], gcnt)
+
+
+@pytest.mark.parametrize("G,d", [(16, 128), (2, 64), (8, 128)])
+def test_fused_decode_step(oracle, G, d):
+    """infllmv2_sparse_decode_step (scoring + top-k + attention in one cluster kernel) against the oracle:
+    ragged lengths, a row at the dense threshold and one past it, rows shorter than one kernel window."""
+    lens = [20000, 8192, 8193, 30, 4500, 65, 70000]
+    w = decode_case(lens, 2 * G, 2, d, topk=16, dense_len=8192, seed=650 + G, n_needles=8)
+    B = len(lens)
+    nk_cap = oracle.num_kernels(max(lens))
+    P = oparams(w.params)
+    kern_o = oracle.kernel_pool(w.k, [0] * B, lens, 32, 16, nk_cap=nk_cap)
+    r = oracle.block_score_topk(w.q, kern_o, w.q_ctx, P)
+    out_o, lse_o = oracle.sparse_attention(w.q, w.k, w.v, w.q_ctx, r["idx"], r["cnt"], P)
+    p = bparams(w.params)
+    kern = gpu_pool(w.k, [0] * B, lens, max(lens), nk_cap)
+    idx = torch.full((B, 1, 2, p.kmax), -7, dtype=torch.int32, device="cuda")
+    cnt = torch.full((B, 1, 2), -7, dtype=torch.int32, device="cuda")
+    out = torch.empty((B, 1, 2 * G, d), dtype=torch.bfloat16, device="cuda")
+    lse = torch.empty((B, 1, 2 * G), dtype=torch.float32, device="cuda")
+    binding.infllmv2_sparse_decode_step(dev(w.q), kern, dev(w.k), dev(w.v), dev_i32(w.ctx_lens), max(lens), p, idx,
+                                        cnt, out, lse)
+    torch.cuda.synchronize()
+    same = check_selection(idx.cpu().numpy(), cnt.cpu().numpy(), r)
+    check_attention(out, out_o, lse, lse_o, mask=same.all(axis=-1), what="fused decode step")

@@ -75,6 +75,7 @@ _SIGS = {
                                       _SZ, _P], _I),
     "infllmv2_sparse_attn_decode": ([_P, _I, _I, _I, _I, _P, _P, _I, _P, _I, _P, _P, _PP, _P, _P, _P, _SZ, _P], _I),
     "infllmv2_sparse_attn_decode_noalloc": ([_P, _I, _I, _I, _I, _P, _P, _I, _P, _I, _P, _P, _PP, _P, _P, _P], _I),
+    "infllmv2_sparse_decode_step": ([_P, _I, _I, _I, _I, _P, _I, _P, _P, _I, _P, _I, _PP, _P, _P, _P, _P, _P], _I),
     "infllmv2_sparse_attn_tree_verify": ([_P, _I, _I, _I, _I, _I, _P, _P, _I, _P, _I, _P, _P, _P, _P, _P, _PP, _P,
                                           _P, _P, _SZ, _P], _I),
     "infllmv2_dense_attn_prefill": ([_P, _I, _I, _I, _I, _I, _P, _P, _I, _P, _P, _I, _F, _P, _P, _P, _SZ, _P], _I),
@@ -213,6 +214,22 @@ def infllmv2_sparse_attn_decode(q, k, v, ctx_lens, max_ctx, idx, cnt, params: Pa
                                             _ptr(ws), 0 if ws is None else ws.numel() * ws.element_size(),
                                             _stream(stream))
     _check("infllmv2_sparse_attn_decode", st)
+
+
+def infllmv2_sparse_decode_step(q, kern, k, v, ctx_lens, max_ctx, params: Params, idx, cnt, out, lse=None,
+                                stream=None):
+    """Scoring, top-k and sparse attention of one decode step in one launch (no workspace)."""
+    for t, n in ((q, "q"), (kern, "kern"), (k, "k"), (v, "v"), (out, "out")):
+        _need(t, torch.bfloat16, n)
+    _need(idx, torch.int32, "idx")
+    _need(cnt, torch.int32, "cnt")
+    B, Hq, d = q.shape[0], q.shape[-2], q.shape[-1]
+    Lcap, Hkv = k.shape[1], k.shape[2]
+    cp = params.c()
+    st = load().infllmv2_sparse_decode_step(_ptr(q), B, Hq, Hkv, d, _ptr(kern), kern.shape[2], _ptr(k), _ptr(v), Lcap,
+                                            _ptr(ctx_lens), int(max_ctx), ctypes.byref(cp), _ptr(idx), _ptr(cnt),
+                                            _ptr(out), _ptr(lse), _stream(stream))
+    _check("infllmv2_sparse_decode_step", st)
 
 
 def infllmv2_sparse_attn_decode_noalloc(q, k, v, ctx_lens, max_ctx, idx, cnt, params: Params, out, lse=None,

@@ -177,8 +177,9 @@ int infllmv2_version(void) { return kVersion; }
 int infllmv2_device_status(void)
 {
     const int f = iv2::tc_error_flag_read_and_clear();
-    if (f < 0) return INFLLMV2_ERR_CUDA;
-    return f ? INFLLMV2_ERR_TIMEOUT : INFLLMV2_OK;
+    const int h = iv2::fused_error_flag_read_and_clear();
+    if (f < 0 || h < 0) return INFLLMV2_ERR_CUDA;
+    return (f || h) ? INFLLMV2_ERR_TIMEOUT : INFLLMV2_OK;
 }
 
 size_t infllmv2_workspace_size(const infllmv2_params* params, int batch, int max_q, int max_ctx, int hq, int hkv,
@@ -286,6 +287,31 @@ int infllmv2_sparse_attn_decode(const void* q, int batch, int hq, int hkv, int h
     const QueryRows qr = rows_of(q, batch, 1, hq, hkv, head_dim, nullptr, ctx_lens, 0, max_ctx);
     return launched(iv2::launch_attn_split(qr, k, v, lcap, idx, cnt, mc, false, nullptr, nullptr, nullptr, out, lse,
                                            ws, (cudaStream_t)stream));
+}
+
+int infllmv2_sparse_decode_step(const void* q, int batch, int hq, int hkv, int head_dim, const void* kern, int nk_cap,
+                                const void* k, const void* v, int lcap, const int32_t* ctx_lens, int max_ctx,
+                                const infllmv2_params* params, int32_t* idx, int32_t* cnt, void* out, float* lse,
+                                infllmv2_stream_t stream)
+{
+    IV2_TRY(check_params(params));
+    IV2_TRY(check_heads(batch, 1, hq, hkv, head_dim));
+    IV2_TRY(check_ptr16(q));
+    IV2_TRY(check_ptr16(kern));
+    IV2_TRY(check_ptr16(k));
+    IV2_TRY(check_ptr16(v));
+    IV2_TRY(check_ptr16(out));
+    IV2_TRY(check_ptr4(ctx_lens));
+    IV2_TRY(check_ptr4(idx));
+    IV2_TRY(check_ptr4(cnt));
+    IV2_TRY(check_opt4(lse));
+    IV2_TRY(check_ctx(max_ctx, lcap));
+    if (nk_cap < 1 || nk_cap < nk_of(max_ctx)) return INFLLMV2_ERR_INVALID_ARG;
+    if (batch * hkv > 65535) return INFLLMV2_ERR_UNSUPPORTED;
+    const MethodConsts mc = consts_of(params, head_dim);
+    const QueryRows qr = rows_of(q, batch, 1, hq, hkv, head_dim, nullptr, ctx_lens, 0, max_ctx);
+    if (!iv2::decode_fused_supported(qr, mc)) return INFLLMV2_ERR_UNSUPPORTED;
+    return launched(iv2::launch_decode_fused(qr, kern, nk_cap, mc, k, v, lcap, idx, cnt, out, lse, (cudaStream_t)stream));
 }
 
 int infllmv2_sparse_attn_tree_verify(const void* q, int batch, int n_draft, int hq, int hkv, int head_dim,

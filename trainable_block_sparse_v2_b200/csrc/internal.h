@@ -115,6 +115,14 @@ cudaError_t launch_attn_rows_tc(const QueryRows& qr, const void* k, const void* 
 // device-side error flag of the bounded waits (1 = a wait ran out); reading clears it; -1 on a CUDA error
 int tc_error_flag_read_and_clear();
 
+// one decode step (scoring, top-k, sparse attention) in a single cluster kernel; cudaErrorNotSupported when
+// the shape is outside what it handles
+bool decode_fused_supported(const QueryRows& qr, const MethodConsts& mc);
+cudaError_t launch_decode_fused(const QueryRows& qr, const void* kern, int nk_cap, const MethodConsts& mc,
+                                const void* k, const void* v, int Lcap, int32_t* idx, int32_t* cnt, void* out,
+                                float* lse, cudaStream_t s);
+int fused_error_flag_read_and_clear();
+
 // attention split over the selected blocks across CTAs, merged by LSE (decode and tree verification)
 cudaError_t launch_attn_split(const QueryRows& qr, const void* k, const void* v, int Lcap, const int32_t* idx,
                               const int32_t* cnt, const MethodConsts& mc, bool dense_all, const void* k_draft,

@@ -68,6 +68,15 @@ IV2_DEV void tma_load_3d(void* dst, const CUtensorMap* map, int x, int y, int z,
         : "memory");
 }
 
+// contiguous global -> shared copy (size and both addresses multiples of 16 bytes), completion on `bar`
+IV2_DEV void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar)
+{
+    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+                     smem_u32(dst)),
+                 "l"(src), "r"(bytes), "r"(smem_u32(bar))
+                 : "memory");
+}
+
 IV2_DEV void prefetch_tensormap(const CUtensorMap* map)
 {
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
