@@ -277,12 +277,20 @@ def test_selection_ties_go_to_lower_block(oracle, path):
     assert np.array_equal(r["idx"], gidx) and np.array_equal(r["cnt"], gcnt)
 
 
-@pytest.mark.parametrize("G,d", [(16, 128), (2, 64), (8, 128)])
-def test_fused_decode_step(oracle, G, d):
+FUSED_LENS_14 = [20000, 8192, 8193, 30, 4500, 65, 70000]
+# 26 rows: more than one wave of 16-CTA clusters, so the launch takes 8-CTA clusters
+FUSED_LENS_26 = [20000, 8192, 8193, 30, 4500, 65, 70000, 9000, 12345, 64 * 130 + 1, 40000, 8300, 98304]
+
+
+@pytest.mark.parametrize("G,d,lens,membership", [(16, 128, FUSED_LENS_14, 0), (2, 64, FUSED_LENS_14, 0),
+                                                 (8, 128, FUSED_LENS_14, 1), (16, 128, FUSED_LENS_26, 0),
+                                                 (4, 64, FUSED_LENS_26, 1)])
+def test_fused_decode_step(oracle, G, d, lens, membership):
     """infllmv2_sparse_decode_step (scoring + top-k + attention in one cluster kernel) against the oracle:
-    ragged lengths, a row at the dense threshold and one past it, rows shorter than one kernel window."""
-    lens = [20000, 8192, 8193, 30, 4500, 65, 70000]
-    w = decode_case(lens, 2 * G, 2, d, topk=16, dense_len=8192, seed=650 + G, n_needles=8)
+    ragged lengths, a row at the dense threshold and one past it, rows shorter than one kernel window,
+    both block-membership rules, 16-CTA and 8-CTA clusters."""
+    w = decode_case(lens, 2 * G, 2, d, topk=16, dense_len=8192, seed=650 + G + len(lens), n_needles=8,
+                    membership=membership)
     B = len(lens)
     nk_cap = oracle.num_kernels(max(lens))
     P = oparams(w.params)
@@ -295,8 +303,12 @@ def test_fused_decode_step(oracle, G, d):
     cnt = torch.full((B, 1, 2), -7, dtype=torch.int32, device="cuda")
     out = torch.empty((B, 1, 2 * G, d), dtype=torch.bfloat16, device="cuda")
     lse = torch.empty((B, 1, 2 * G), dtype=torch.float32, device="cuda")
-    binding.infllmv2_sparse_decode_step(dev(w.q), kern, dev(w.k), dev(w.v), dev_i32(w.ctx_lens), max(lens), p, idx,
-                                        cnt, out, lse)
+    K, V = dev(w.k), dev(w.v)
+    for b, n in enumerate(lens):  # cache rows past a sequence's context must not leak in, even as NaN
+        K[b, n:] = float("nan")
+        V[b, n:] = float("nan")
+    binding.infllmv2_sparse_decode_step(dev(w.q), kern, K, V, dev_i32(w.ctx_lens), max(lens), p, idx, cnt, out, lse)
     torch.cuda.synchronize()
+    assert binding.infllmv2_device_status() == 0
     same = check_selection(idx.cpu().numpy(), cnt.cpu().numpy(), r)
     check_attention(out, out_o, lse, lse_o, mask=same.all(axis=-1), what="fused decode step")

@@ -86,7 +86,7 @@ attn_tc_kernel(QueryRows qr, const __grid_constant__ CUtensorMap tm_q, const __g
     pdl_launch_dependents();
     pdl_wait();
     extern __shared__ unsigned char smem_raw[];
-    unsigned char* smem = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    unsigned char* smem = tc::align_smem_1024(smem_raw);
     __shared__ Bars bars;
     uint32_t* bits = reinterpret_cast<uint32_t*>(smem + kBitsOff);
     uint16_t* list = reinterpret_cast<uint16_t*>(smem + kListOff);
@@ -419,43 +419,6 @@ attn_tc_kernel(QueryRows qr, const __grid_constant__ CUtensorMap tm_q, const __g
 }
 
 // ---------------------------------------------------------------- host
-namespace {
-
-typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
-                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
-                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-EncodeTiledFn encode_fn()
-{
-    static EncodeTiledFn fn = nullptr;
-    static std::once_flag once;
-    std::call_once(once, [] {
-        void* p = nullptr;
-        cudaDriverEntryPointQueryResult q;
-        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
-            q == cudaDriverEntryPointSuccess)
-            fn = reinterpret_cast<EncodeTiledFn>(p);
-    });
-    return fn;
-}
-
-// 3-D bf16 map over rows of `inner` (=128) elements: dims {inner, mid, outer}, box {64, box_mid, box_outer}
-bool make_map(CUtensorMap* map, const void* base, uint64_t mid, uint64_t outer, uint64_t mid_stride_bytes,
-              uint64_t outer_stride_bytes, uint32_t box_mid, uint32_t box_outer)
-{
-    EncodeTiledFn fn = encode_fn();
-    if (!fn) return false;
-    const cuuint64_t dims[3] = {(cuuint64_t)kD, mid, outer};
-    const cuuint64_t strides[2] = {mid_stride_bytes, outer_stride_bytes};
-    const cuuint32_t box[3] = {64, box_mid, box_outer};
-    const cuuint32_t estr[3] = {1, 1, 1};
-    return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
-              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
-}  // namespace
-
 bool attn_tc_supported(const QueryRows& qr)
 {
     return qr.D == kD && qr.Hq / qr.Hkv == kG && (qr.max_ctx - 1) / kBlock + 1 <= kMaxBlk;
@@ -468,9 +431,9 @@ cudaError_t launch_attn_rows_tc(const QueryRows& qr, const void* k, const void* 
     if (!attn_tc_supported(qr)) return cudaErrorNotSupported;
     CUtensorMap tq, tk, tv;
     const uint64_t row = (uint64_t)kD * 2;
-    if (!make_map(&tq, qr.q, qr.Hq, (uint64_t)qr.B * qr.T, row, row * qr.Hq, kG, kTok) ||
-        !make_map(&tk, k, qr.Hkv, (uint64_t)qr.B * Lcap, row, row * qr.Hkv, 1, kBlock) ||
-        !make_map(&tv, v, qr.Hkv, (uint64_t)qr.B * Lcap, row, row * qr.Hkv, 1, kBlock))
+    if (!make_tma_map_bf16(&tq, qr.q, kD, qr.Hq, (uint64_t)qr.B * qr.T, row, row * qr.Hq, kG, kTok) ||
+        !make_tma_map_bf16(&tk, k, kD, qr.Hkv, (uint64_t)qr.B * Lcap, row, row * qr.Hkv, 1, kBlock) ||
+        !make_tma_map_bf16(&tv, v, kD, qr.Hkv, (uint64_t)qr.B * Lcap, row, row * qr.Hkv, 1, kBlock))
         return cudaErrorNotSupported;
     cudaError_t e = ensure_smem(attn_tc_kernel, kSmemBytes);
     if (e != cudaSuccess) return e;

@@ -58,6 +58,15 @@ IV2_DEV void mma_bf16_16816(float (&c)[4], const uint32_t (&a)[4], uint32_t b0, 
         : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
 
+// D (+)= A * B, m16n8k8, bf16 in, f32 accumulate; a0 = (row g, cols 2t..2t+1), a1 = (row g+8, ...),
+// b0 = (k 2t..2t+1, n g)
+IV2_DEV void mma_bf16_1688(float (&c)[4], uint32_t a0, uint32_t a1, uint32_t b0)
+{
+    asm volatile("mma.sync.aligned.m16n8k8.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5}, {%6}, {%0,%1,%2,%3};\n"
+                 : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+                 : "r"(a0), "r"(a1), "r"(b0));
+}
+
 IV2_DEV void ldmatrix_x4(uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3, const void* smem_row_ptr)
 {
     uint32_t a = static_cast<uint32_t>(__cvta_generic_to_shared(smem_row_ptr));

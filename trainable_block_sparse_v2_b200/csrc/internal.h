@@ -1,6 +1,7 @@
 // internal.h -- launchers shared between the C-ABI layer (api.cu) and the kernel files.
 #pragma once
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <stddef.h>
 #include <stdint.h>
@@ -58,6 +59,11 @@ inline cudaError_t launch_pdl_cluster(void (*kernel)(KArgs...), dim3 grid, dim3 
     cfg.numAttrs = 2;
     return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
 }
+
+// 3-D bf16 TMA map with 128-byte swizzle over rows of `inner` elements: dims {inner, mid, outer}, box
+// {64, box_mid, box_outer}; false when the driver entry point is missing or the encoder rejects the shape
+bool make_tma_map_bf16(CUtensorMap* map, const void* base, uint64_t inner, uint64_t mid, uint64_t outer,
+                       uint64_t mid_stride_bytes, uint64_t outer_stride_bytes, uint32_t box_mid, uint32_t box_outer);
 
 // Resolved per-call description of a set of query rows.
 struct QueryRows {

@@ -158,9 +158,11 @@ IV2_DEV int bucket_of(uint32_t key, uint32_t kmin, float bucket_scale)
     return min((int)((float)(key - kmin) * bucket_scale), kBuckets - 1);
 }
 
+// Returns the number of chosen blocks (every thread); when idx_sm is given the list is also written there;
+// idx_out / cnt_out may be null (the list then only goes to idx_sm).
 template <int NT, int E>
-IV2_DEV void cta_select_topk(const float* S, int c, int init, int local, int topk, int kmax, int32_t* idx_out,
-                             int32_t* cnt_out, CtaSelectSmem& sm)
+IV2_DEV int cta_select_topk(const float* S, int c, int init, int local, int topk, int kmax, int32_t* idx_out,
+                            int32_t* cnt_out, CtaSelectSmem& sm, int32_t* idx_sm = nullptr)
 {
     constexpr int NW = NT / 32;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -341,12 +343,17 @@ IV2_DEV void cta_select_topk(const float* S, int c, int init, int local, int top
 #pragma unroll
     for (int e = 0; e < E; ++e) {
         if (chosen[e]) {
-            if (pos < kmax) idx_out[pos] = b0 + e;
+            if (pos < kmax) {
+                if (idx_out) idx_out[pos] = b0 + e;
+                if (idx_sm) idx_sm[pos] = b0 + e;
+            }
             ++pos;
         }
     }
-    for (int p = total + threadIdx.x; p < kmax; p += NT) idx_out[p] = -1;
-    if (threadIdx.x == 0) *cnt_out = total;
+    if (idx_out)
+        for (int p = total + threadIdx.x; p < kmax; p += NT) idx_out[p] = -1;
+    if (cnt_out && threadIdx.x == 0) *cnt_out = total;
+    return total;
 }
 
 }  // namespace iv2

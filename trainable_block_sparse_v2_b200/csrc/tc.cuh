@@ -18,6 +18,13 @@ namespace tc {
 
 IV2_DEV uint32_t smem_u32(const void* p) { return static_cast<uint32_t>(__cvta_generic_to_shared(p)); }
 
+// the first 1024-byte boundary at or after a dynamic shared-memory base; formed by pointer arithmetic on
+// the base so that the compiler keeps the shared state space (plain shared loads, stores and atomics)
+IV2_DEV unsigned char* align_smem_1024(unsigned char* base)
+{
+    return base + ((1024u - (smem_u32(base) & 1023u)) & 1023u);
+}
+
 // ---------------------------------------------------------------- mbarriers
 IV2_DEV void mbar_init(uint64_t* bar, uint32_t count)
 {
@@ -57,6 +64,11 @@ IV2_DEV bool mbar_wait(uint64_t* bar, uint32_t parity, uint32_t limit = (1u << 2
         if (mbar_try_wait(bar, parity)) return true;
     return false;
 }
+
+// split cluster barrier: arrive (releasing this thread's prior writes) now, wait (acquiring every CTA's)
+// later; each thread alternates arrive / wait, all threads of every CTA of the cluster take part
+IV2_DEV void cluster_arrive_release() { asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory"); }
+IV2_DEV void cluster_wait_acquire() { asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory"); }
 
 // ---------------------------------------------------------------- TMA
 IV2_DEV void tma_load_3d(void* dst, const CUtensorMap* map, int x, int y, int z, uint64_t* bar)
