@@ -108,6 +108,13 @@ cudaError_t launch_kernel_pool(const void* k, int B, int Lcap, int Hkv, int D, c
 cudaError_t launch_score_topk(const QueryRows& qr, const void* kern, int nk_cap, const MethodConsts& mc,
                               int32_t* idx, int32_t* cnt, void* ws, cudaStream_t s);
 
+// the token-tile scoring on tcgen05/TMEM (16 heads per group, d = 128, at most 2048 context blocks);
+// cudaErrorNotSupported otherwise
+bool score_tc_supported(const QueryRows& qr, int nb_max);
+cudaError_t launch_score_tc(const QueryRows& qr, const void* kern, int nk_cap, const MethodConsts& mc, int nb_max,
+                            int32_t* idx, int32_t* cnt, cudaStream_t s);
+int score_tc_error_flag_read_and_clear();
+
 // attention over selected blocks (or all blocks when dense_all); prefill style: one warp per query row
 cudaError_t launch_attn_rows(const QueryRows& qr, const void* k, const void* v, int Lcap, const int32_t* idx,
                              const int32_t* cnt, const MethodConsts& mc, bool dense_all, void* out, float* lse,

@@ -535,9 +535,11 @@ cudaError_t launch_score_topk(const QueryRows& qr, const void* kern_v, int nk_ca
 {
     const __nv_bfloat16* kern = static_cast<const __nv_bfloat16*>(kern_v);
     const int nb_max = nb_of(qr.max_ctx);
-    if (!score_uses_scan_path(qr.B, qr.T, qr.Hq / qr.Hkv, qr.D, qr.max_ctx))
+    if (!score_uses_scan_path(qr.B, qr.T, qr.Hq / qr.Hkv, qr.D, qr.max_ctx)) {
+        if (score_tc_supported(qr, nb_max)) return launch_score_tc(qr, kern, nk_cap, mc, nb_max, idx, cnt, s);
         return qr.D == 128 ? launch_prefill_score_g<128>(qr, kern, nk_cap, mc, nb_max, idx, cnt, s)
                            : launch_prefill_score_g<64>(qr, kern, nk_cap, mc, nb_max, idx, cnt, s);
+    }
     const int rows = qr.B * qr.T * qr.Hkv;
     const int nchunk = score_nchunk(nb_max);
     auto al = [](size_t x) { return (x + 255) / 256 * 256; };

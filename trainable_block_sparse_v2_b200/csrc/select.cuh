@@ -18,6 +18,15 @@ namespace iv2 {
 
 IV2_DEV bool is_forced(int b, int c, int init, int local) { return b < init || (b > c - local && b <= c); }
 
+// sum over the warp of a per-lane count in [0, 256): one ballot per bit, all independent
+IV2_DEV int warp_count(int v)
+{
+    int total = 0;
+#pragma unroll
+    for (int bit = 0; bit < 8; ++bit) total += __popc(__ballot_sync(0xffffffffu, (v >> bit) & 1)) << bit;
+    return total;
+}
+
 // ---------------------------------------------------------------------------------------------------
 // one warp selects for one row; S in shared memory (nb = c + 1 entries, -inf = no visible kernel)
 // ---------------------------------------------------------------------------------------------------
@@ -32,7 +41,7 @@ IV2_DEV void warp_select_topk(const float* S, int c, int init, int local, int to
     };
     int ncand = 0;
     for (int b = lane; b < nb; b += 32) ncand += key_of(b) != 0u;
-    ncand = __reduce_add_sync(0xffffffffu, ncand);
+    ncand = warp_count(ncand);
 
     uint32_t thr = 1u;  // keys >= thr are chosen (plus ties below)
     int need_eq = 0;    // how many keys == thr to take, lowest index first (only when thr is exact)
@@ -43,13 +52,13 @@ IV2_DEV void warp_select_topk(const float* S, int c, int init, int local, int to
             const uint32_t probe = t | (1u << bit);
             int cntge = 0;
             for (int b = lane; b < nb; b += 32) cntge += key_of(b) >= probe;
-            cntge = __reduce_add_sync(0xffffffffu, cntge);
+            cntge = warp_count(cntge);
             if (cntge >= topk) t = probe;
         }
         // t is the k-th largest key
         int gt = 0;
         for (int b = lane; b < nb; b += 32) gt += key_of(b) > t;
-        gt = __reduce_add_sync(0xffffffffu, gt);
+        gt = warp_count(gt);
         thr = t;
         need_eq = topk - gt;
     }
@@ -68,6 +77,179 @@ IV2_DEV void warp_select_topk(const float* S, int c, int init, int local, int to
             const int rank = eq_seen + __popc(eqmask & ((1u << lane) - 1u));
             if (eq && rank < need_eq) chosen = true;
             eq_seen += __popc(eqmask);
+        }
+        const unsigned cm = __ballot_sync(0xffffffffu, chosen);
+        const int pos = out_pos + __popc(cm & ((1u << lane) - 1u));
+        if (chosen && pos < kmax) idx_out[pos] = b;
+        out_pos += __popc(cm);
+    }
+    for (int p = out_pos + lane; p < kmax; p += 32) idx_out[p] = -1;
+    if (lane == 0) *cnt_out = out_pos;
+}
+
+// ---------------------------------------------------------------------------------------------------
+// one warp selects for one row with a 256-bucket histogram in its own shared scratch; S in shared memory
+// (nb = c + 1 <= 32 KW entries).  Lane l keeps blocks l, l + 32, ... in registers; the candidate keys are spread over
+// the buckets by the same monotone fp32 map as the CTA select, the bucket B* holding the k-th largest key
+// is found by a warp scan, and its members are ranked exactly by (key descending, block ascending).  The
+// chosen set is identical to warp_select_topk's.
+// ---------------------------------------------------------------------------------------------------
+constexpr int kWarpBuckets = 256;
+constexpr int kWarpMembers = 64;
+
+struct WarpSelectSmem {
+    int hist[kWarpBuckets];
+    uint32_t mkey[kWarpMembers];
+    int midx[kWarpMembers];
+};
+
+// KW = keys per lane kept in registers (nb <= 32 KW); lane l holds blocks l, l + 32, ...
+template <int KW>
+IV2_DEV void warp_select_topk_hist(const float* S, int c, int init, int local, int topk, int kmax, int32_t* idx_out,
+                                   int32_t* cnt_out, WarpSelectSmem& ws)
+{
+    const int lane = threadIdx.x & 31;
+    const int nb = c + 1;
+    uint32_t key[KW];
+    int ncand = 0;
+    uint32_t lo = 0xffffffffu, hi = 0u;
+#pragma unroll
+    for (int e = 0; e < KW; ++e) {
+        const int b = lane + 32 * e;
+        const float s = b < nb ? S[b] : neg_inf();
+        key[e] = (b < nb && !is_forced(b, c, init, local) && s != neg_inf()) ? float_key(s) : 0u;
+        if (key[e]) {
+            ++ncand;
+            lo = min(lo, key[e]);
+            hi = max(hi, key[e]);
+        }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+        ncand += __shfl_xor_sync(0xffffffffu, ncand, o);
+        lo = min(lo, __shfl_xor_sync(0xffffffffu, lo, o));
+        hi = max(hi, __shfl_xor_sync(0xffffffffu, hi, o));
+    }
+    const bool all = ncand <= topk;
+    const float bscale = hi > lo ? (float)(kWarpBuckets - 1) / (float)(hi - lo) : 0.f;
+    int bk[KW];
+    int bstar = kWarpBuckets;
+    uint32_t tkey = 0u;
+    int tidx = 0;
+    if (!all) {
+#pragma unroll
+        for (int i = 0; i < kWarpBuckets / 32; ++i) ws.hist[lane + 32 * i] = 0;
+        __syncwarp();
+#pragma unroll
+        for (int e = 0; e < KW; ++e) {
+            bk[e] = key[e] ? min((int)((float)(key[e] - lo) * bscale), kWarpBuckets - 1) : -1;
+            if (bk[e] >= 0) atomicAdd(&ws.hist[bk[e]], 1);
+        }
+        __syncwarp();
+        // descending scan: lane l owns buckets [256 - 8 (l + 1), 256 - 8 l)
+        constexpr int BPL = kWarpBuckets / 32;
+        const int base = kWarpBuckets - BPL * (lane + 1);
+        int cb[BPL], sum = 0;
+#pragma unroll
+        for (int j = 0; j < BPL; ++j) {
+            cb[j] = ws.hist[base + BPL - 1 - j];  // descending within the lane
+            sum += cb[j];
+        }
+        int incl = sum;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int y = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += y;
+        }
+        const int excl = incl - sum;
+        int my_b = -1, my_above = 0;
+        if (excl < topk && topk <= incl) {
+            int acc = excl;
+#pragma unroll
+            for (int j = 0; j < BPL; ++j) {
+                if (my_b < 0 && acc + cb[j] >= topk) {
+                    my_b = base + BPL - 1 - j;
+                    my_above = acc;
+                }
+                acc += cb[j];
+            }
+        }
+        const unsigned hitm = __ballot_sync(0xffffffffu, my_b >= 0);
+        const int src = __ffs(hitm) - 1;
+        bstar = __shfl_sync(0xffffffffu, my_b, src);
+        const int rem = topk - __shfl_sync(0xffffffffu, my_above, src);  // members of B* still to take, >= 1
+        // gather the members of B* (ascending block order) and count them
+        int nm = 0;
+#pragma unroll
+        for (int e = 0; e < KW; ++e) {
+            const bool mem = bk[e] == bstar;
+            const unsigned mm = __ballot_sync(0xffffffffu, mem);
+            const int pos = nm + __popc(mm & ((1u << lane) - 1u));
+            if (mem && pos < kWarpMembers) {
+                ws.mkey[pos] = key[e];
+                ws.midx[pos] = lane + 32 * e;
+            }
+            nm += __popc(mm);
+        }
+        __syncwarp();
+        if (nm <= kWarpMembers) {
+            // the member of rank rem - 1 in (key descending, block ascending) order is the threshold
+            int my_hit = -1;
+            for (int i = lane; i < nm; i += 32) {
+                const uint32_t ki = ws.mkey[i];
+                const int ii = ws.midx[i];
+                int rank = 0;
+                for (int j = 0; j < nm; ++j) {
+                    const uint32_t kj = ws.mkey[j];
+                    rank += (kj > ki) || (kj == ki && ws.midx[j] < ii);
+                }
+                if (rank == rem - 1) my_hit = i;
+            }
+            const unsigned th = __ballot_sync(0xffffffffu, my_hit >= 0);
+            const int ti = __shfl_sync(0xffffffffu, my_hit, __ffs(th) - 1);
+            tkey = ws.mkey[ti];
+            tidx = ws.midx[ti];
+        } else {
+            // many equal-bucket keys: bitwise search of the rem-th largest member key, then block ids
+            uint32_t t = 0u;
+            for (int bit = 31; bit >= 0; --bit) {
+                const uint32_t probe = t | (1u << bit);
+                int ge = 0;
+#pragma unroll
+                for (int e = 0; e < KW; ++e) ge += bk[e] == bstar && key[e] >= probe;
+                if (warp_count(ge) >= rem) t = probe;
+            }
+            int gt = 0;
+#pragma unroll
+            for (int e = 0; e < KW; ++e) gt += bk[e] == bstar && key[e] > t;
+            const int need = rem - warp_count(gt);
+            // the need-th lowest block id among the members with key t
+            int seen = 0;
+            tidx = -1;
+#pragma unroll
+            for (int e = 0; e < KW; ++e) {
+                const unsigned eq = __ballot_sync(0xffffffffu, bk[e] == bstar && key[e] == t);
+                if (tidx < 0 && seen + __popc(eq) >= need) {
+                    unsigned m2 = eq;
+                    for (int j = 0; j < need - seen - 1; ++j) m2 &= m2 - 1u;
+                    tidx = 32 * e + __ffs(m2) - 1;
+                }
+                seen += __popc(eq);
+            }
+            tkey = t;
+        }
+        __syncwarp();
+    }
+    // emit ascending
+    int out_pos = 0;
+#pragma unroll
+    for (int e = 0; e < KW; ++e) {
+        const int b = lane + 32 * e;
+        bool chosen = false;
+        if (b < nb) {
+            if (is_forced(b, c, init, local)) chosen = true;
+            else if (key[e])
+                chosen = all || bk[e] > bstar || (bk[e] == bstar && (key[e] > tkey || (key[e] == tkey && b <= tidx)));
         }
         const unsigned cm = __ballot_sync(0xffffffffu, chosen);
         const int pos = out_pos + __popc(cm & ((1u << lane) - 1u));

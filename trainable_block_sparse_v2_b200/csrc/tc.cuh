@@ -158,6 +158,14 @@ IV2_DEV void tmem_ld32(uint32_t taddr, uint32_t (&r)[32])
         : "r"(taddr));
 }
 
+// one 32-bit column of this thread's TMEM lane
+IV2_DEV uint32_t tmem_ld1(uint32_t taddr)
+{
+    uint32_t r;
+    asm volatile("tcgen05.ld.sync.aligned.32x32b.x1.b32 {%0}, [%1];" : "=r"(r) : "r"(taddr));
+    return r;
+}
+
 IV2_DEV void tmem_st32(uint32_t taddr, const uint32_t (&r)[32])
 {
     asm volatile(
@@ -172,6 +180,12 @@ IV2_DEV void tmem_st32(uint32_t taddr, const uint32_t (&r)[32])
 
 IV2_DEV void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 IV2_DEV void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+
+// named barrier `id` (1..15) over `nthreads` threads (a multiple of 32) of the CTA
+IV2_DEV void named_bar_sync(uint32_t id, uint32_t nthreads)
+{
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+}
 
 // ---------------------------------------------------------------- descriptors
 // K-major operand in 128-byte-swizzled atoms of rows x 64 bf16 (row pitch 128 B, 8-row groups 1024 B apart)
