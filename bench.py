@@ -38,6 +38,15 @@ UNIT = "tokens/s"
 PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 LENS_128K = (131072, 98304, 65536, 131072)
 HQ, HKV, D = 32, 2, 128
+# DRAM bytes (read + write) per call of the dominant C-ABI calls, each from one ncu capture of the kernels
+# as they stand (profiles/decode_128k_launches.md, profiles/decode_fused_128k.md); None where the kernel
+# changed after its capture
+NCU_TRAFFIC = {
+    "sparse_decode_step": 31_316_480,                   # decode_fused_kernel: 31.316 MB read, 512 B written
+    "sparse_attn_decode": 17_430_000 + 1_150_000,       # attn_split_kernel + attn_merge_kernel
+    "block_score_topk": 13_680_000 + 960_000,           # score_scan_kernel + score_select_kernel
+    "sparse_attn_prefill": None,
+}
 KERNELS_PER_STEP = {"two_call": 5,  # kernel pool, score scan, select, split attention, merge
                     "fused": 2}     # kernel pool, fused decode step (scoring + top-k + attention)
 
@@ -124,7 +133,7 @@ def decode_step_bytes(lens, kmax=67):
 
 
 class DecodeBench:
-    def __init__(self, layers=8, steps_cycle=256, two_call=True):
+    def __init__(self, layers=8, steps_cycle=256, two_call=False):
         import torch
         from trainable_block_sparse_v2_b200 import binding
         from trainable_block_sparse_v2_b200.workloads import decode_128k_ragged
@@ -198,55 +207,97 @@ class DecodeBench:
         else:
             self.fused(layer, pos, stream)
 
-    def graph(self, s):
+    def _capture(self, key, steps):
+        """one CUDA graph of the given consecutive steps (warmed outside capture first)"""
         torch = self.torch
-        key = self._coords(s)
         g = self.graphs.get(key)
         if g is None:
             g = torch.cuda.CUDAGraph()
             st = torch.cuda.Stream()
             st.wait_stream(torch.cuda.current_stream())
             with torch.cuda.stream(st):
-                self.step_eager(s)  # warm the launch path outside capture
+                for s in steps:
+                    self.step_eager(s)  # warm the launch path outside capture
             torch.cuda.current_stream().wait_stream(st)
             with torch.cuda.graph(g):
-                self.step_eager(s)
+                for s in steps:
+                    self.step_eager(s)
             self.graphs[key] = g
         return g
 
+    def graph(self, s):
+        """the single-step graph of step s"""
+        return self._capture(self._coords(s), [s])
+
+    def position_graph(self, s):
+        """steps s .. s + NL - 1 (s a multiple of NL): every layer at one decode position, as a model's decode
+        step runs them; one replay per position keeps PyTorch's per-replay generator prologue (two small fill
+        kernels) off all but one step in NL"""
+        return self._capture(("pos", self._coords(s)[1]), list(range(s, s + self.NL)))
+
+    def _plan(self, lo, hi):
+        """graphs covering steps [lo, hi): whole positions where they fit, single steps elsewhere"""
+        plan, s = [], lo
+        while s < hi:
+            if s % self.NL == 0 and s + self.NL <= hi:
+                plan.append(self.position_graph(s))
+                s += self.NL
+            else:
+                plan.append(self.graph(s))
+                s += 1
+        return plan
+
     def timed(self, warmup, steps):
         torch = self.torch
-        for s in range(warmup + steps):
-            self.graph(s)
+        warm = self._plan(0, warmup)
+        run = self._plan(warmup, warmup + steps)
         torch.cuda.synchronize()
-        for s in range(warmup):
-            self.graphs[self._coords(s)].replay()
+        for g in warm:
+            g.replay()
         torch.cuda.synchronize()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record()
-        for s in range(warmup, warmup + steps):
-            self.graphs[self._coords(s)].replay()
+        for g in run:
+            g.replay()
         e1.record()
         e1.synchronize()
         return e0.elapsed_time(e1) / 1e3
 
     def per_call_times(self, warmup, steps):
-        """average device time of each C-ABI call, CUDA events around each launch on the current stream"""
+        """average device time of each C-ABI call: `steps` consecutive calls of it (each on another layer cache
+        and position) captured in one CUDA graph, replayed between two CUDA events on the current stream, so
+        that neither host launch overhead nor the graph prologue is counted"""
         torch = self.torch
         names = ["kernel_pool", "block_score_topk", "sparse_attn_decode", "sparse_decode_step"]
         fns = [self.pool, self.score, self.attend, self.fused]
-        ev = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
-              for _ in fns]
         for s in range(warmup):
             self.step_eager(s)
-        for i, s in enumerate(range(warmup, warmup + steps)):
-            layer, pos = self._coords(s)
-            for j, fn in enumerate(fns):
-                ev[j][i][0].record()
-                fn(layer, pos)
-                ev[j][i][1].record()
         torch.cuda.synchronize()
-        return {n: float(np.mean([a.elapsed_time(b) for a, b in ev[j]])) / 1e3 for j, n in enumerate(names)}
+        out = {}
+        for name, fn in zip(names, fns):
+            calls = [self._coords(s) for s in range(warmup, warmup + steps)]
+            g = torch.cuda.CUDAGraph()
+            st = torch.cuda.Stream()
+            st.wait_stream(torch.cuda.current_stream())
+            with torch.cuda.stream(st):
+                for layer, pos in calls:
+                    fn(layer, pos)
+            torch.cuda.current_stream().wait_stream(st)
+            with torch.cuda.graph(g):
+                for layer, pos in calls:
+                    fn(layer, pos)
+            g.replay()
+            torch.cuda.synchronize()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            reps = 4
+            e0.record()
+            for _ in range(reps):
+                g.replay()
+            e1.record()
+            e1.synchronize()
+            out[name] = e0.elapsed_time(e1) / 1e3 / (reps * steps)
+            del g
+        return out
 
     def e2e(self, warmup, steps):
         """Same step through the C ABI with host buffers: every step copies that step's query and the new
@@ -465,63 +516,66 @@ def run_ours(args):
     binding.load()
     peaks, peak_kind = load_peaks()
 
-    two_call = args.decode_path == "two_call"
-    db = DecodeBench(layers=args.layers, two_call=two_call)
-    # timed region: exactly K decode steps (graph replays), barrier + synchronize on both sides
-    for s in range(args.warmup + args.steps):
-        db.graph(s)
-    barrier(ws)
-    with ClockSampler(torch.cuda.current_device()) as clk:
-        t = db.timed(args.warmup, args.steps)
-    barrier(ws)
-    t = barrier_max(t, ws)
-    tokens = len(LENS_128K) * args.steps * ws
-    value = tokens / t
+    if not args.no_decode:
+        two_call = args.decode_path == "two_call"
+        db = DecodeBench(layers=args.layers, two_call=two_call)
+        # timed region: exactly K decode steps (graph replays), barrier + synchronize on both sides
+        barrier(ws)
+        with ClockSampler(torch.cuda.current_device()) as clk:
+            t = db.timed(args.warmup, args.steps)
+        barrier(ws)
+        t = barrier_max(t, ws)
+        tokens = len(LENS_128K) * args.steps * ws
+        value = tokens / t
 
-    per = db.per_call_times(8, min(args.steps, 256)) if args.per_call else {
-        "kernel_pool": float("nan"), "block_score_topk": float("nan"), "sparse_attn_decode": float("nan"),
-        "sparse_decode_step": float("nan")}
-    lens_mid = [n + 128 for n in LENS_128K]
-    scan_b, kv_b, step_b = decode_step_bytes(lens_mid)
-    if two_call:
-        # dominant call of the two-call step: the larger of block scoring + top-k and sparse attention
-        dom = max(("block_score_topk", "sparse_attn_decode"), key=lambda k: per[k] if per[k] == per[k] else -1.0)
-        dom_bytes = {"block_score_topk": scan_b, "sparse_attn_decode": kv_b}[dom]
+        per = db.per_call_times(8, min(args.steps, 256)) if args.per_call else {
+            "kernel_pool": float("nan"), "block_score_topk": float("nan"), "sparse_attn_decode": float("nan"),
+            "sparse_decode_step": float("nan")}
+        lens_mid = [n + 128 for n in LENS_128K]
+        scan_b, kv_b, step_b = decode_step_bytes(lens_mid)
+        if two_call:
+            # dominant call of the two-call step: the larger of block scoring + top-k and sparse attention
+            dom = max(("block_score_topk", "sparse_attn_decode"), key=lambda k: per[k] if per[k] == per[k] else -1.0)
+            dom_bytes = {"block_score_topk": scan_b, "sparse_attn_decode": kv_b}[dom]
+        else:
+            # the fused scoring + top-k + attention launch carries the whole step's traffic
+            dom = "sparse_decode_step"
+            dom_bytes = scan_b + kv_b
+        achieved = dom_bytes / per[dom] / 1e9
+        e2e_steps = min(args.steps, 512)
+        e2e_t, h2d, d2h = db.e2e(8, e2e_steps) if args.e2e else (float("nan"), 0, 0)
+
+        line = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": ws, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": t / args.steps * 1e3, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": "decode_128k_ragged", "batch": 4, "ctx_lens_step0": list(LENS_128K),
+                       "heads_q_kv": [HQ, HKV], "head_dim": D, "block": 64, "kernel_window_stride": [32, 16],
+                       "topk": 64, "init_local": [1, 2], "dense_len": 8192, "decode_positions": 256,
+                       "layers_rotating": args.layers, "parallelism": f"replicas{ws}",
+                       "l2": "inputs larger than L2: 8 rotating layer caches, each step's 31 MB working set is evicted "
+                             "before its layer returns",
+                       "step": ("one decode step of one layer for 4 sequences: kernel_pool + block_score_topk + "
+                                "sparse_attn_decode, replayed as a CUDA graph" if two_call else
+                                "one decode step of one layer for 4 sequences: kernel_pool + sparse_decode_step "
+                                "(scoring, top-k and sparse attention in one cluster kernel), replayed as a CUDA graph")},
+            "hbm": {"algorithmic_bytes_per_step": step_b, "achieved_gbs_per_gpu": step_b / (t / args.steps) / 1e9,
+                    "frac_of_" + peak_kind: step_b / (t / args.steps) / 1e9 / peaks["hbm_gbs"]},
+            "per_call_ms": {k: v * 1e3 for k, v in per.items()},
+            "roofline": {"bound": "hbm", "kernel": dom, "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                         "frac": achieved / peaks["hbm_gbs"], "peak_kind": peak_kind + " (burst copy)",
+                         "algorithmic_bytes": dom_bytes, "traffic": NCU_TRAFFIC.get(dom)},
+            "clocks": clk.summary(),
+            "e2e": {"value": len(LENS_128K) * e2e_steps / e2e_t, "unit": UNIT, "h2d_bytes_per_step": h2d,
+                    "d2h_bytes_per_step": d2h, "steps": e2e_steps},
+            "gpu_launches": KERNELS_PER_STEP[args.decode_path] * args.steps,
+        }
+        del db
+        torch.cuda.empty_cache()
     else:
-        # the fused scoring + top-k + attention launch carries the whole step's traffic
-        dom = "sparse_decode_step"
-        dom_bytes = scan_b + kv_b
-    achieved = dom_bytes / per[dom] / 1e9
-    e2e_steps = min(args.steps, 512)
-    e2e_t, h2d, d2h = db.e2e(8, e2e_steps) if args.e2e else (float("nan"), 0, 0)
-
-    line = {
-        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": ws, "steps": args.steps, "warmup": args.warmup,
-        "ms_per_step": t / args.steps * 1e3, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-        "dtype": "bf16", "data": "synthetic",
-        "config": {"workload": "decode_128k_ragged", "batch": 4, "ctx_lens_step0": list(LENS_128K),
-                   "heads_q_kv": [HQ, HKV], "head_dim": D, "block": 64, "kernel_window_stride": [32, 16],
-                   "topk": 64, "init_local": [1, 2], "dense_len": 8192, "decode_positions": 256,
-                   "layers_rotating": args.layers, "parallelism": f"replicas{ws}",
-                   "l2": "inputs larger than L2: 8 rotating layer caches, each step's 31 MB working set is evicted "
-                         "before its layer returns",
-                   "step": ("one decode step of one layer for 4 sequences: kernel_pool + block_score_topk + "
-                            "sparse_attn_decode, replayed as a CUDA graph" if two_call else
-                            "one decode step of one layer for 4 sequences: kernel_pool + sparse_decode_step "
-                            "(scoring, top-k and sparse attention in one cluster kernel), replayed as a CUDA graph")},
-        "hbm": {"algorithmic_bytes_per_step": step_b, "achieved_gbs_per_gpu": step_b / (t / args.steps) / 1e9,
-                "frac_of_" + peak_kind: step_b / (t / args.steps) / 1e9 / peaks["hbm_gbs"]},
-        "per_call_ms": {k: v * 1e3 for k, v in per.items()},
-        "roofline": {"bound": "hbm", "kernel": dom, "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                     "frac": achieved / peaks["hbm_gbs"], "peak_kind": peak_kind + " (burst copy)",
-                     "algorithmic_bytes": dom_bytes, "traffic": None},
-        "clocks": clk.summary(),
-        "e2e": {"value": len(LENS_128K) * e2e_steps / e2e_t, "unit": UNIT, "h2d_bytes_per_step": h2d,
-                "d2h_bytes_per_step": d2h, "steps": e2e_steps},
-        "gpu_launches": KERNELS_PER_STEP[args.decode_path] * args.steps,
-    }
-    del db
-    torch.cuda.empty_cache()
+        # profiling runs of the prefill kernels alone: no decode line
+        line = {"metric": METRIC, "unit": UNIT, "n_gpus": ws, "note": "decode skipped (--no-decode)",
+                "gpu_launches": 0}
 
     if not args.no_prefill:
         pb = PrefillBench()
@@ -540,9 +594,9 @@ def run_ours(args):
             "per_call_ms": {k: v * 1e3 for k, v in pper.items()},
             "roofline": {"bound": "tensor", "kernel": pdom, "achieved": pach, "peak": peaks["bf16_tflops"],
                          "unit": "TFLOP/s", "frac": pach / peaks["bf16_tflops"], "peak_kind": peak_kind + " (burst)",
-                         "traffic": None},
+                         "traffic": NCU_TRAFFIC.get(pdom)},
         }
-        line["gpu_launches"] += args.prefill_steps * 5
+        line["gpu_launches"] += args.prefill_steps * 3  # kernel pool, scoring + top-k, attention
         del pb
         torch.cuda.empty_cache()
 
@@ -607,10 +661,11 @@ def main():
     ap.add_argument("--warmup", type=int, default=64)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--layers", type=int, default=8)
-    ap.add_argument("--decode-path", choices=["two_call", "fused"], default="two_call",
+    ap.add_argument("--decode-path", choices=["two_call", "fused"], default="fused",
                     help="decode step as block_score_topk + sparse_attn_decode, or the one-launch sparse_decode_step")
     ap.add_argument("--prefill-steps", type=int, default=3)
     ap.add_argument("--no-prefill", action="store_true")
+    ap.add_argument("--no-decode", action="store_true", help="prefill only (for profiling its kernels)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=15.0)
     ap.add_argument("--no-e2e", dest="e2e", action="store_false", help="skip the host-buffer end-to-end leg")

@@ -16,10 +16,11 @@
 //   O[128 x 128] += P[128 x 128] . V         A (P) in TMEM, B (V) MN-major in smem, O in TMEM
 // Keeping Q and P in TMEM leaves shared memory to the K/V stream, and 128-key steps halve the number of
 // MMA instructions and pipeline hand-offs per key.
-// Warp roles: warp 0 issues TMA loads (Q once; K and V per step into 3-deep rings, one lane each), warp 1 (one thread) issues the
-// MMAs, warps 2-5 run the softmax and the epilogue.  Producer/consumer hand-offs use mbarriers; MMA
-// completion is signalled with tcgen05.commit.  Every wait is bounded: after the limit the CTA records an
-// error (g_tc_error), skips the rest of its work, frees its TMEM and exits.
+// Warp roles: warps 0 and 6 issue TMA loads (Q once and K per step; V per step) into 3-deep rings, one
+// lane each, warp 1 (one thread) issues the MMAs, warps 2-5 run the softmax and the epilogue.
+// Producer/consumer hand-offs use mbarriers; MMA completion is signalled with tcgen05.commit.  Every wait
+// is bounded: after the limit the CTA records an error (g_tc_error), skips the rest of its work, frees its
+// TMEM and exits.
 #include <mutex>
 
 #include "common.cuh"
@@ -35,7 +36,7 @@ namespace {
 constexpr int kTok = 8;           // tokens per tile
 constexpr int kG = 16;            // heads per KV group
 constexpr int kD = 128;           // head dim
-constexpr int kThreads = 192;     // 6 warps
+constexpr int kThreads = 224;     // 7 warps
 constexpr int kMaxBlk = 4096;     // context blocks (256K keys)
 constexpr int kWords = kMaxBlk / 32;
 constexpr int kStepKeys = 128;       // two 64-key blocks per pipeline step
@@ -184,9 +185,10 @@ attn_tc_kernel(QueryRows qr, const __grid_constant__ CUtensorMap tm_q, const __g
     const uint32_t sV = tc::smem_u32(smem + kVOff);
 
     const int NP = (U + 1) / 2;  // pipeline steps; an odd last block is paired with a masked copy of itself
-    if (warp == 0) {
-        // ---------------- TMA producers: lane 0 streams K (and Q first), lane 1 streams V ----------------
-        if (lane == 0) {
+    if (warp == 0 || warp == 6) {
+        // ---------------- TMA producers: warp 0 streams K (and Q first), warp 6 streams V ----------------
+        // (one lane each, in separate warps: two spinning lanes of one warp would take turns)
+        if (warp == 0 && lane == 0) {
             tc::prefetch_tensormap(&tm_q);
             tc::prefetch_tensormap(&tm_k);
             tc::mbar_arrive_expect_tx(&bars.q_full, 2 * 128 * 128);
@@ -206,7 +208,7 @@ attn_tc_kernel(QueryRows qr, const __grid_constant__ CUtensorMap tm_q, const __g
                     tc::tma_load_3d(st + 16384 + i * 8192, &tm_k, 64, g, z, &bars.k_full[s]);
                 }
             }
-        } else if (lane == 1) {
+        } else if (warp == 6 && lane == 0) {
             tc::prefetch_tensormap(&tm_v);
             for (int p = 0; p < NP; ++p) {
                 const int s = p % kRing, k = p / kRing;
@@ -262,7 +264,7 @@ attn_tc_kernel(QueryRows qr, const __grid_constant__ CUtensorMap tm_q, const __g
                 }
             }
         }
-    } else {
+    } else if (warp >= 2 && warp <= 5) {
         // ---------------- softmax + epilogue: one TMEM lane (query row) per thread ----------------
         const int q4 = warp & 3;
         const int r = q4 * 32 + lane;  // row = token * 16 + head
