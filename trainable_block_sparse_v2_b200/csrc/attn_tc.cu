@@ -16,8 +16,9 @@
 //   O[128 x 128] += P[128 x 128] . V         A (P) in TMEM, B (V) MN-major in smem, O in TMEM
 // Keeping Q and P in TMEM leaves shared memory to the K/V stream, and 128-key steps halve the number of
 // MMA instructions and pipeline hand-offs per key.
-// Warp roles: warps 0 and 6 issue TMA loads (Q once and K per step; V per step) into 3-deep rings, one
-// lane each, warp 1 (one thread) issues the MMAs, warps 2-5 run the softmax and the epilogue.
+// Warp roles: warps 0 and 10 issue TMA loads (Q once and K per step; V per step) into 3-deep rings, one
+// lane each, warp 1 (one thread) issues the MMAs, warps 2-9 run the softmax and the epilogue, two warps per
+// TMEM lane quarter, each on one of the step's two blocks.
 // Producer/consumer hand-offs use mbarriers; MMA completion is signalled with tcgen05.commit.  Every wait
 // is bounded: after the limit the CTA records an error (g_tc_error), skips the rest of its work, frees its
 // TMEM and exits.
@@ -36,7 +37,7 @@ namespace {
 constexpr int kTok = 8;           // tokens per tile
 constexpr int kG = 16;            // heads per KV group
 constexpr int kD = 128;           // head dim
-constexpr int kThreads = 224;     // 7 warps
+constexpr int kThreads = 352;     // 11 warps
 constexpr int kMaxBlk = 4096;     // context blocks (256K keys)
 constexpr int kWords = kMaxBlk / 32;
 constexpr int kStepKeys = 128;       // two 64-key blocks per pipeline step
@@ -63,6 +64,7 @@ struct Bars {
     uint32_t tmem_base;
     int n_union;
     int err;
+    float xm[2][2][128];  // [step parity][half][row]: the two softmax halves' partial maxima, then sums
 };
 
 __device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity, volatile int* err)
@@ -165,7 +167,7 @@ attn_tc_kernel(QueryRows qr, const __grid_constant__ CUtensorMap tm_q, const __g
         }
         for (int i = 0; i < 2; ++i) {
             tc::mbar_init(&bars.s_full[i], 1);
-            tc::mbar_init(&bars.p_full[i], 128);
+            tc::mbar_init(&bars.p_full[i], 256);
             tc::mbar_init(&bars.o_done[i], 1);
         }
         tc::fence_barrier_init();
@@ -185,8 +187,8 @@ attn_tc_kernel(QueryRows qr, const __grid_constant__ CUtensorMap tm_q, const __g
     const uint32_t sV = tc::smem_u32(smem + kVOff);
 
     const int NP = (U + 1) / 2;  // pipeline steps; an odd last block is paired with a masked copy of itself
-    if (warp == 0 || warp == 6) {
-        // ---------------- TMA producers: warp 0 streams K (and Q first), warp 6 streams V ----------------
+    if (warp == 0 || warp == 10) {
+        // ---------------- TMA producers: warp 0 streams K (and Q first), warp 10 streams V ----------------
         // (one lane each, in separate warps: two spinning lanes of one warp would take turns)
         if (warp == 0 && lane == 0) {
             tc::prefetch_tensormap(&tm_q);
@@ -208,7 +210,7 @@ attn_tc_kernel(QueryRows qr, const __grid_constant__ CUtensorMap tm_q, const __g
                     tc::tma_load_3d(st + 16384 + i * 8192, &tm_k, 64, g, z, &bars.k_full[s]);
                 }
             }
-        } else if (warp == 6 && lane == 0) {
+        } else if (warp == 10 && lane == 0) {
             tc::prefetch_tensormap(&tm_v);
             for (int p = 0; p < NP; ++p) {
                 const int s = p % kRing, k = p / kRing;
@@ -264,19 +266,23 @@ attn_tc_kernel(QueryRows qr, const __grid_constant__ CUtensorMap tm_q, const __g
                 }
             }
         }
-    } else if (warp >= 2 && warp <= 5) {
-        // ---------------- softmax + epilogue: one TMEM lane (query row) per thread ----------------
-        const int q4 = warp & 3;
+    } else if (warp >= 2 && warp <= 9) {
+        // ---------------- softmax + epilogue: one TMEM lane (query row) per thread, one block of each step ----
+        // warps w and w + 4 (2 <= w <= 5) share the lane quarter w & 3: half 0 takes the step's first block
+        // (keys 0..63), half 1 its second (keys 64..127); they exchange row maxima and sums in shared memory
+        // under a named barrier of their own, and every barrier is reached by both on every step
+        const int q4 = warp & 3, half = (warp - 2) >> 2;
         const int r = q4 * 32 + lane;  // row = token * 16 + head
         const int tt = r >> 4, hh = r & 15;
         const int t = t0 + tt;
         const bool valid = t < T;
         const int n = valid ? query_ctx(qr, b, t) : 0;
         const uint32_t lane_addr = tmem + ((uint32_t)(q4 * 32) << 16);
+        const uint32_t pair_bar = 1 + q4;
         const float sl2 = mc.scale * kLog2e;
         float m_ref = neg_inf(), l = 0.f;
         bool ok = wait_bar(&bars.q_full, 0, err);
-        {
+        if (half == 0) {
             // this row of Q (swizzled smem from TMA) -> TMEM columns [kColQ, kColQ + 64) as bf16 pairs
 #pragma unroll
             for (int a = 0; a < 2; ++a) {
@@ -297,104 +303,109 @@ attn_tc_kernel(QueryRows qr, const __grid_constant__ CUtensorMap tm_q, const __g
             tc::mbar_arrive(&bars.q_tmem);
         }
         ok = __all_sync(0xffffffffu, ok);
-        for (int p = 0; p < NP && ok; ++p) {
+        for (int p = 0; p < NP; ++p) {
             const int sb = p & 1;
-            ok = wait_bar(&bars.s_full[sb], (p >> 1) & 1, err);
+            if (ok) ok = wait_bar(&bars.s_full[sb], (p >> 1) & 1, err);
             ok = __all_sync(0xffffffffu, ok);
-            if (!ok) break;
-            tc::tc_fence_after();
-            // the step's two blocks, whether this row's token selected each, and its keys in each
+            if (ok) tc::tc_fence_after();
+            // this half's block of the step, whether this row's token selected it, and its keys in it
             const int blk_a = list[2 * p];
             const bool has_b = 2 * p + 1 < U;
-            const int blk_b = has_b ? list[2 * p + 1] : blk_a;
-            const bool sel_a = valid && ((bits[tt * kWords + (blk_a >> 5)] >> (blk_a & 31)) & 1u);
-            const bool sel_b = valid && has_b && ((bits[tt * kWords + (blk_b >> 5)] >> (blk_b & 31)) & 1u);
-            const int nv_a = sel_a ? min(kBlock, n - blk_a * kBlock) : 0;
-            const int nv_b = sel_b ? min(kBlock, n - blk_b * kBlock) : 0;
+            const int blk = (half && has_b) ? list[2 * p + 1] : blk_a;
+            const bool sel = valid && (half == 0 || has_b) && ((bits[tt * kWords + (blk >> 5)] >> (blk & 31)) & 1u);
+            const int nv = sel ? min(kBlock, n - blk * kBlock) : 0;
             const uint32_t srow = lane_addr + kColS + kStepKeys * sb;
-            if (!__any_sync(0xffffffffu, sel_a || sel_b)) {
-                // neither token of this warp selected either block: its P rows are zero
-                uint32_t z[32];
+            const bool any_sel = __any_sync(0xffffffffu, sel);
+            // scaled scores in log2 units; keys this row does not attend to are -inf
+            float x[64];
+            float mx = neg_inf();
+            if (ok && any_sel) {
 #pragma unroll
-                for (int j = 0; j < 32; ++j) z[j] = 0u;
-                tc::tmem_st32(srow, z);
-                tc::tmem_st32(srow + 32, z);
-            } else {
-                // scaled scores in log2 units; unselected blocks and keys past the row's context are -inf
-                float x[kStepKeys];
-#pragma unroll
-                for (int h = 0; h < 4; ++h) {
+                for (int h2 = 0; h2 < 2; ++h2) {
                     uint32_t sv[32];
-                    tc::tmem_ld32(srow + 32 * h, sv);
+                    tc::tmem_ld32(srow + 64 * half + 32 * h2, sv);
                     tc::tmem_wait_ld();
-                    const int nv = h < 2 ? nv_a : nv_b;
 #pragma unroll
-                    for (int j = 0; j < 32; ++j)
-                        x[32 * h + j] = ((h & 1) * 32 + j) < nv ? __uint_as_float(sv[j]) * sl2 : neg_inf();
+                    for (int j = 0; j < 32; ++j) x[32 * h2 + j] = (32 * h2 + j) < nv ? __uint_as_float(sv[j]) * sl2 : neg_inf();
                 }
                 float m8[8];
 #pragma unroll
                 for (int i = 0; i < 8; ++i) {
                     float m = x[i];
 #pragma unroll
-                    for (int j = 1; j < 16; ++j) m = fmaxf(m, x[i + 8 * j]);
+                    for (int j = 1; j < 8; ++j) m = fmaxf(m, x[i + 8 * j]);
                     m8[i] = m;
                 }
-                const float mx = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])),
-                                       fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
-                const bool rescale = mx > m_ref + 8.f;  // mx is -inf for a row that selected neither block
-                const float new_ref = rescale ? mx : m_ref;
-                const float alpha = (rescale && l > 0.f) ? exp2_fast(m_ref - new_ref) : 1.f;
-                if (__any_sync(0xffffffffu, alpha != 1.f)) {
-                    // every PV so far must have landed before O is rewritten
-                    if (p >= 1) ok = wait_bar(&bars.o_done[(p - 1) & 1], ((p - 1) >> 1) & 1, err) && ok;
-                    ok = __all_sync(0xffffffffu, ok);
-                    if (!ok) break;
+                mx = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])), fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
+            }
+            // double-buffered by step parity: a half can be at most one step ahead of its partner here
+            bars.xm[p & 1][half][r] = mx;
+            // both halves' S loads are complete past this barrier, so P may overwrite S columns 0..63
+            tc::named_bar_sync(pair_bar, 64);
+            mx = fmaxf(mx, bars.xm[p & 1][half ^ 1][r]);
+            const bool rescale = mx > m_ref + 8.f;  // mx is -inf for a row that selected neither block
+            const float new_ref = rescale ? mx : m_ref;
+            // identical in both halves: O is zero until the row has a finite reference
+            const float alpha = (rescale && m_ref != neg_inf()) ? exp2_fast(m_ref - new_ref) : 1.f;
+            if (ok && __any_sync(0xffffffffu, alpha != 1.f)) {
+                // every PV so far must have landed before this half of O is rewritten
+                if (p >= 1) ok = wait_bar(&bars.o_done[(p - 1) & 1], ((p - 1) >> 1) & 1, err) && ok;
+                ok = __all_sync(0xffffffffu, ok);
+                if (ok) {
 #pragma unroll 1
-                    for (int c4 = 0; c4 < kD / 32; ++c4) {
+                    for (int c4 = 0; c4 < 2; ++c4) {
                         uint32_t o[32];
-                        tc::tmem_ld32(lane_addr + 32 * c4, o);
+                        tc::tmem_ld32(lane_addr + 64 * half + 32 * c4, o);
                         tc::tmem_wait_ld();
 #pragma unroll
                         for (int j = 0; j < 32; ++j) o[j] = __float_as_uint(__uint_as_float(o[j]) * alpha);
-                        tc::tmem_st32(lane_addr + 32 * c4, o);
+                        tc::tmem_st32(lane_addr + 64 * half + 32 * c4, o);
                     }
                     tc::tmem_wait_st();
                 }
-                l *= alpha;
-                m_ref = new_ref;
-                // P = 2^(x - m_ref), bf16 pairs along the keys, over the first 64 columns of this S buffer
-                const float mneg = (sel_a || sel_b) ? -m_ref : neg_inf();
-                float ps[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-                for (int h = 0; h < 2; ++h) {
-                    uint32_t w[32];
+            }
+            l *= alpha;
+            m_ref = new_ref;
+            if (ok) {
+                // P = 2^(x - m_ref) for this half's 64 keys, bf16 pairs into S columns [32 half, 32 half + 32)
+                uint32_t w[32];
+                if (any_sel) {
+                    const float mneg = (sel && m_ref != neg_inf()) ? -m_ref : neg_inf();
+                    float ps[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
                     for (int j2 = 0; j2 < 32; ++j2) {
-                        const float p0 = ex2_approx(x[64 * h + 2 * j2] + mneg);
-                        const float p1 = ex2_approx(x[64 * h + 2 * j2 + 1] + mneg);
+                        const float p0 = ex2_approx(x[2 * j2] + mneg);
+                        const float p1 = ex2_approx(x[2 * j2 + 1] + mneg);
                         ps[j2 & 3] += p0 + p1;
                         w[j2] = pack_bf16(p0, p1);
                     }
-                    tc::tmem_st32(srow + 32 * h, w);
+                    l += (ps[0] + ps[1]) + (ps[2] + ps[3]);
+                } else {
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) w[j] = 0u;
                 }
-                l += (ps[0] + ps[1]) + (ps[2] + ps[3]);
+                tc::tmem_st32(srow + 32 * half, w);
+                tc::tmem_wait_st();
+                tc::tc_fence_before();
+                tc::mbar_arrive(&bars.p_full[sb]);
             }
-            tc::tmem_wait_st();
-            tc::tc_fence_before();
-            tc::mbar_arrive(&bars.p_full[sb]);
         }
+        // the row sum over both halves
+        tc::named_bar_sync(pair_bar, 64);  // every read of xm for the maxima is done
+        bars.xm[0][half][r] = l;
+        tc::named_bar_sync(pair_bar, 64);
+        const float lt = l + bars.xm[0][half ^ 1][r];
         ok = __all_sync(0xffffffffu, ok);
         if (ok && NP > 0) ok = wait_bar(&bars.o_done[(NP - 1) & 1], ((NP - 1) >> 1) & 1, err);
         ok = __all_sync(0xffffffffu, ok);
         if (ok) {
             tc::tc_fence_after();
-            const float inv = l > 0.f ? 1.f / l : 0.f;
-            __nv_bfloat16* orow = out + (((size_t)b * T + t) * qr.Hq + g * kG + hh) * kD;
+            const float inv = lt > 0.f ? 1.f / lt : 0.f;
+            __nv_bfloat16* orow = out + (((size_t)b * T + t) * qr.Hq + g * kG + hh) * kD + 64 * half;
 #pragma unroll 1
-            for (int c4 = 0; c4 < kD / 32; ++c4) {
+            for (int c4 = 0; c4 < 2; ++c4) {
                 uint32_t o[32];
-                tc::tmem_ld32(lane_addr + 32 * c4, o);
+                tc::tmem_ld32(lane_addr + 64 * half + 32 * c4, o);
                 tc::tmem_wait_ld();
                 if (valid) {
 #pragma unroll
@@ -408,8 +419,8 @@ attn_tc_kernel(QueryRows qr, const __grid_constant__ CUtensorMap tm_q, const __g
                     }
                 }
             }
-            if (valid && lse)
-                lse[((size_t)b * T + t) * qr.Hq + g * kG + hh] = l > 0.f ? (m_ref + __log2f(l)) * kLn2 : neg_inf();
+            if (valid && lse && half == 0)
+                lse[((size_t)b * T + t) * qr.Hq + g * kG + hh] = lt > 0.f ? (m_ref + __log2f(lt)) * kLn2 : neg_inf();
         }
     }
     tc::tc_fence_before();
