@@ -469,7 +469,9 @@ def cpu_baseline(budget_s=15.0):
 
 
 # ------------------------------------------------------------------------------------------------
-def dist_setup(n):
+def dist_setup(n, backend="nccl"):
+    """one process per GPU: RANK / LOCAL_RANK / WORLD_SIZE / MASTER_* from the launcher's environment.
+    backend "gloo" (CPU, no device binding) serves the multi-process tests."""
     import torch
     ws = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -477,29 +479,41 @@ def dist_setup(n):
     if ws > 1:
         import datetime
         import torch.distributed as dist
-        torch.cuda.set_device(local)
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=torch.device("cuda", local))
-    else:
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+            dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                    device_id=torch.device("cuda", local))
+        else:
+            dist.init_process_group(backend, timeout=datetime.timedelta(seconds=60))
+    elif backend == "nccl":
         torch.cuda.set_device(0)
     return ws, rank, local
 
 
-def barrier_max(x, ws):
+def barrier_max(x, ws, device="cuda"):
+    """the max over ranks of a per-rank duration (every rank gets it)"""
     import torch
     if ws == 1:
         return x
     import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    t = torch.tensor([x], dtype=torch.float64, device=device)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
 
 
-def barrier(ws):
+def barrier(ws, cuda=True):
     import torch
-    torch.cuda.synchronize()
+    if cuda:
+        torch.cuda.synchronize()
     if ws > 1:
         import torch.distributed as dist
         dist.barrier()
+
+
+def whole_job_rate(units_per_rank, ws, t_max):
+    """whole-job throughput: the units every rank processed (weak scaling: the same count on each) over the
+    slowest rank's device time"""
+    return units_per_rank * ws / t_max
 
 
 def run_ours(args):
@@ -525,8 +539,7 @@ def run_ours(args):
             t = db.timed(args.warmup, args.steps)
         barrier(ws)
         t = barrier_max(t, ws)
-        tokens = len(LENS_128K) * args.steps * ws
-        value = tokens / t
+        value = whole_job_rate(len(LENS_128K) * args.steps, ws, t)
 
         per = db.per_call_times(8, min(args.steps, 256)) if args.per_call else {
             "kernel_pool": float("nan"), "block_score_topk": float("nan"), "sparse_attn_decode": float("nan"),
@@ -587,7 +600,7 @@ def run_ours(args):
         dom_flops = {"sparse_attn_prefill": af + df, "block_score_topk": 2 * sf, "kernel_pool": 0}[pdom]
         pach = dom_flops / pper[pdom] / 1e12
         line["prefill"] = {
-            "workload": "prefill_32k", "value": pb.T * args.prefill_steps * ws / pt, "unit": UNIT,
+            "workload": "prefill_32k", "value": whole_job_rate(pb.T * args.prefill_steps, ws, pt), "unit": UNIT,
             "ms_per_step": pt / args.prefill_steps * 1e3, "steps": args.prefill_steps,
             "algorithmic_tflop_per_step": flops / 1e12,
             "tc_frac_of_" + peak_kind: flops / (pt / args.prefill_steps) / 1e12 / peaks["bf16_tflops"],
