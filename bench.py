@@ -300,32 +300,35 @@ class DecodeBench:
         return out
 
     def e2e(self, warmup, steps):
-        """Same step through the C ABI with host buffers: every step copies that step's query and the new
-        key/value rows from pinned host memory to the device and reads the attention output back."""
+        """Same step through the C ABI with host buffers: every step copies that step's query and the new key
+        and value rows from pinned host memory to the device in one copy, appends the rows to the caches
+        (infllmv2_kv_append), pools, runs the step and reads the attention output back."""
         torch = self.torch
         B = self.B
-        q_host = torch.empty((self.S, B, 1, HQ, D), dtype=torch.bfloat16).pin_memory()
-        q_host.copy_(self.q_all.cpu())
-        kv_host = torch.empty((self.S, 2, B, HKV, D), dtype=torch.bfloat16).pin_memory()
+        nq, nkv = B * HQ * D, B * HKV * D
+        # per position: [query | new key rows | new value rows], bf16
+        host = torch.empty((self.S, nq + 2 * nkv), dtype=torch.bfloat16).pin_memory()
+        host[:, :nq].copy_(self.q_all.reshape(self.S, nq).cpu())
         lens_np = self.lens.cpu().numpy()
         k0c = self.k[0].cpu()
         v0c = self.v[0].cpu()
         for pos in range(self.S):
             for b in range(B):
-                kv_host[pos, 0, b] = k0c[b, lens_np[pos, b] - 1]
-                kv_host[pos, 1, b] = v0c[b, lens_np[pos, b] - 1]
+                row = lens_np[pos, b] - 1
+                host[pos, nq + b * HKV * D: nq + (b + 1) * HKV * D] = k0c[b, row].reshape(-1)
+                host[pos, nq + nkv + b * HKV * D: nq + nkv + (b + 1) * HKV * D] = v0c[b, row].reshape(-1)
         out_host = torch.empty((B, 1, HQ, D), dtype=torch.bfloat16).pin_memory()
-        q_dev = torch.empty((B, 1, HQ, D), dtype=torch.bfloat16, device="cuda")
-        h2d = q_dev.numel() * 2 + 2 * B * HKV * D * 2
+        stage = torch.empty(nq + 2 * nkv, dtype=torch.bfloat16, device="cuda")
+        q_dev = stage[:nq].view(B, 1, HQ, D)
+        k_new = stage[nq:nq + nkv].view(B, HKV, D)
+        v_new = stage[nq + nkv:].view(B, HKV, D)
+        h2d = stage.numel() * 2
         d2h = out_host.numel() * 2
 
         def one(s):
             layer, pos = self._coords(s)
-            q_dev.copy_(q_host[(pos + 37 * layer) % self.S], non_blocking=True)
-            for b in range(B):
-                row = int(lens_np[pos, b]) - 1
-                self.k[layer][b, row].copy_(kv_host[pos, 0, b], non_blocking=True)
-                self.v[layer][b, row].copy_(kv_host[pos, 1, b], non_blocking=True)
+            stage.copy_(host[pos], non_blocking=True)
+            self.b.infllmv2_kv_append(k_new, v_new, self.old[pos], self.k[layer], self.v[layer])
             self.b.infllmv2_kernel_pool(self.k[layer], self.old[pos], self.lens[pos], 1, self.p, self.kern[layer])
             if self.two_call:
                 self.b.infllmv2_block_score_topk(q_dev, None, self.lens[pos], self.max_ctx, self.kern[layer], self.p,

@@ -84,8 +84,8 @@ int infllmv2_version(void);
 
 /*
  * Device-side status of the kernels that wait on their own producer/consumer barriers (the tensor-core
- * prefill attention): every such wait is bounded, and a wait that runs out records an error, makes its
- * CTA skip the rest of its work and exit.  Returns INFLLMV2_ERR_TIMEOUT if that happened since the last
+ * prefill scoring and attention, the one-launch decode step): every such wait is bounded, and a wait that
+ * runs out records an error, makes its CTA skip the rest of its work and exit.  Returns INFLLMV2_ERR_TIMEOUT if that happened since the last
  * call (and clears the record), INFLLMV2_OK otherwise, INFLLMV2_ERR_CUDA if the record cannot be read.
  * Synchronous: it reads device memory on the current device.
  */
@@ -99,6 +99,18 @@ int infllmv2_device_status(void);
  */
 size_t infllmv2_workspace_size(const infllmv2_params* params, int batch, int max_q, int max_ctx, int hq, int hkv,
                                int head_dim);
+
+/*
+ * Cache maintenance of a decode step (the pages have no counterpart; it keeps a step's host traffic to one
+ * copy of the new rows): writes one new key and one new value row per sequence into the caches,
+ *   k_cache[b, pos[b], :, :] = k_new[b, :, :]   and   v_cache[b, pos[b], :, :] = v_new[b, :, :]
+ *   k_new, v_new      [B, Hkv, d] bf16 (device, 16-byte aligned)
+ *   pos               [B] int32 (device); a position outside [0, Lcap) writes nothing
+ *   k_cache, v_cache  [B, Lcap, Hkv, d] bf16 (device, 16-byte aligned); rows other than pos[b] untouched
+ * Ordered on `stream` like every call here; the new rows are visible to the calls enqueued after it.
+ */
+int infllmv2_kv_append(const void* k_new, const void* v_new, int batch, int hkv, int head_dim, const int32_t* pos,
+                       void* k_cache, void* v_cache, int lcap, infllmv2_stream_t stream);
 
 /*
  * Step 1 -- semantic kernels (MiniCPM4 technical details, "Model architecture: InfLLM v2", item 1).

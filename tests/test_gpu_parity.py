@@ -48,6 +48,28 @@ def gpu_select(w, kern, q_ctx=None, max_ctx=None, params=None):
 # step 1: kernel pool
 # ---------------------------------------------------------------------------------------------------
 
+@pytest.mark.gpu
+def test_kv_append_writes_exactly_the_new_rows():
+    """infllmv2_kv_append against plain PyTorch indexing: bit-exact, other rows untouched, a position outside
+    the cache writes nothing"""
+    torch.manual_seed(3)
+    B, L, H, d = 5, 300, 2, 128
+    K = torch.randn(B, L, H, d, device="cuda").to(torch.bfloat16)
+    V = torch.randn(B, L, H, d, device="cuda").to(torch.bfloat16)
+    kn = torch.randn(B, H, d, device="cuda").to(torch.bfloat16)
+    vn = torch.randn(B, H, d, device="cuda").to(torch.bfloat16)
+    pos = torch.tensor([0, 17, 299, -1, 300], dtype=torch.int32, device="cuda")
+    Kw, Vw = K.clone(), V.clone()
+    for b in range(B):
+        p = int(pos[b])
+        if 0 <= p < L:
+            Kw[b, p] = kn[b]
+            Vw[b, p] = vn[b]
+    binding.infllmv2_kv_append(kn, vn, pos, K, V)
+    torch.cuda.synchronize()
+    assert torch.equal(K, Kw) and torch.equal(V, Vw)
+
+
 @pytest.mark.parametrize("d", [64, 128])
 def test_kernel_pool_bulk_and_incremental(oracle, d):
     rng = np.random.default_rng(100 + d)

@@ -70,6 +70,7 @@ _SIGS = {
     "infllmv2_device_status": ([], _I),
     "infllmv2_workspace_size": ([_PP, _I, _I, _I, _I, _I, _I], _SZ),
     "infllmv2_kernel_pool": ([_P, _I, _I, _I, _I, _P, _P, _I, _PP, _P, _I, _P], _I),
+    "infllmv2_kv_append": ([_P, _P, _I, _I, _I, _P, _P, _P, _I, _P], _I),
     "infllmv2_block_score_topk": ([_P, _I, _I, _I, _I, _I, _P, _P, _I, _P, _I, _PP, _P, _P, _P, _SZ, _P], _I),
     "infllmv2_sparse_attn_prefill": ([_P, _I, _I, _I, _I, _I, _P, _P, _I, _P, _P, _I, _P, _P, _PP, _P, _P, _P,
                                       _SZ, _P], _I),
@@ -164,6 +165,22 @@ def infllmv2_kernel_pool(k, old_lens, new_lens, max_new_keys, params: Params, ke
     st = load().infllmv2_kernel_pool(_ptr(k), B, Lcap, Hkv, d, _ptr(old_lens), _ptr(new_lens), int(max_new_keys),
                                      ctypes.byref(cp), _ptr(kern), kern.shape[2], _stream(stream))
     _check("infllmv2_kernel_pool", st)
+
+
+def infllmv2_kv_append(k_new, v_new, pos, k_cache, v_cache, stream=None):
+    """k_cache[b, pos[b]] = k_new[b] and v_cache[b, pos[b]] = v_new[b] (cache maintenance of a decode step)"""
+    _need(k_new, torch.bfloat16, "k_new", 3)
+    _need(v_new, torch.bfloat16, "v_new", 3)
+    _need(k_cache, torch.bfloat16, "k_cache", 4)
+    _need(v_cache, torch.bfloat16, "v_cache", 4)
+    _need(pos, torch.int32, "pos")
+    B, Lcap, Hkv, d = k_cache.shape
+    if tuple(v_cache.shape) != (B, Lcap, Hkv, d) or tuple(k_new.shape) != (B, Hkv, d) or \
+            tuple(v_new.shape) != (B, Hkv, d):
+        raise ValueError("kv_append: shapes do not match the caches")
+    st = load().infllmv2_kv_append(_ptr(k_new), _ptr(v_new), B, Hkv, d, _ptr(pos), _ptr(k_cache), _ptr(v_cache), Lcap,
+                                   _stream(stream))
+    _check("infllmv2_kv_append", st)
 
 
 def infllmv2_block_score_topk(q, q_ctx, ctx_lens, max_ctx, kern, params: Params, idx, cnt, ws, stream=None):

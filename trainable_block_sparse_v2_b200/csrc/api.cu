@@ -251,6 +251,20 @@ int infllmv2_kernel_pool(const void* k, int batch, int lcap, int hkv, int head_d
                                             nk_cap, (cudaStream_t)stream));
 }
 
+int infllmv2_kv_append(const void* k_new, const void* v_new, int batch, int hkv, int head_dim, const int32_t* pos,
+                       void* k_cache, void* v_cache, int lcap, infllmv2_stream_t stream)
+{
+    IV2_TRY(check_heads(batch, 1, hkv, hkv, head_dim));
+    IV2_TRY(check_ptr16(k_new));
+    IV2_TRY(check_ptr16(v_new));
+    IV2_TRY(check_ptr16(k_cache));
+    IV2_TRY(check_ptr16(v_cache));
+    IV2_TRY(check_ptr4(pos));
+    if (lcap < 1) return INFLLMV2_ERR_INVALID_ARG;
+    return launched(iv2::launch_kv_append(k_new, v_new, batch, hkv, head_dim, pos, k_cache, v_cache, lcap,
+                                          (cudaStream_t)stream));
+}
+
 int infllmv2_block_score_topk(const void* q, int batch, int num_q, int hq, int hkv, int head_dim,
                               const int32_t* q_ctx, const int32_t* ctx_lens, int max_ctx, const void* kern,
                               int nk_cap, const infllmv2_params* params, int32_t* idx, int32_t* cnt, void* ws,

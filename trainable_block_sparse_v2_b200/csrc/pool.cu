@@ -94,4 +94,34 @@ cudaError_t launch_kernel_pool(const void* k, int B, int Lcap, int Hkv, int D, c
                       nk_cap);
 }
 
+// ---------------------------------------------------------------------------------------------------
+// Cache maintenance of a decode step (the pages have no counterpart): one new key and value row per
+// sequence into the caches, k_cache[b, pos[b], :, :] = k_new[b, :, :] (v likewise).  16-byte copies; a
+// position outside [0, Lcap) writes nothing.
+// ---------------------------------------------------------------------------------------------------
+__global__ void __launch_bounds__(256) kv_append_kernel(const uint4* __restrict__ k_new, const uint4* __restrict__ v_new,
+                                                       const int32_t* __restrict__ pos, int Lcap, int row16,
+                                                       uint4* __restrict__ k_cache, uint4* __restrict__ v_cache)
+{
+    pdl_launch_dependents();
+    pdl_wait();
+    const int b = blockIdx.x;
+    const int p = pos[b];
+    if (p < 0 || p >= Lcap) return;
+    const size_t dst = ((size_t)b * Lcap + p) * row16;
+    for (int i = threadIdx.x; i < 2 * row16; i += blockDim.x) {
+        if (i < row16) k_cache[dst + i] = k_new[(size_t)b * row16 + i];
+        else v_cache[dst + i - row16] = v_new[(size_t)b * row16 + i - row16];
+    }
+}
+
+cudaError_t launch_kv_append(const void* k_new, const void* v_new, int B, int Hkv, int D, const int32_t* pos,
+                             void* k_cache, void* v_cache, int Lcap, cudaStream_t s)
+{
+    const int row16 = Hkv * D / 8;  // 16-byte chunks of one position's keys (all KV heads)
+    return launch_pdl(kv_append_kernel, dim3(B), dim3(256), 0, s, static_cast<const uint4*>(k_new),
+                      static_cast<const uint4*>(v_new), pos, Lcap, row16, static_cast<uint4*>(k_cache),
+                      static_cast<uint4*>(v_cache));
+}
+
 }  // namespace iv2
