@@ -97,7 +97,8 @@ attn_tc_kernel(QueryRows qr, const __grid_constant__ CUtensorMap tm_q, const __g
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int T = qr.T;
     const int g = blockIdx.y % qr.Hkv, b = blockIdx.y / qr.Hkv;
-    const int t0 = blockIdx.x * kTok;
+    // longest tiles first (later tokens attend to more blocks): the short ones fill the last wave
+    const int t0 = (gridDim.x - 1 - blockIdx.x) * kTok;
 
     // ---- union of the tile's block sets, as one bitmap per token and an ascending list ----
     int cmax = 0;

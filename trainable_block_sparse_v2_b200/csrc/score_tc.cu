@@ -105,7 +105,8 @@ score_tc_kernel(QueryRows qr, const __grid_constant__ CUtensorMap tm_q, const __
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int T = qr.T;
     const int g = blockIdx.y % qr.Hkv, b = blockIdx.y / qr.Hkv;
-    const int t0 = blockIdx.x * kSTok;
+    // longest tiles first (later tokens see more kernels): the short ones fill the last wave
+    const int t0 = (gridDim.x - 1 - blockIdx.x) * kSTok;
 
     int n_max = 0;
     bool any_sparse = false;
