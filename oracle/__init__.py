@@ -101,6 +101,8 @@ def _load():
         lib.orc_sparse_attention.restype = i
         lib.orc_dense_attention.argtypes = [P, i, i, i, i, i, P, P, i, P, ctypes.c_double, P, P]
         lib.orc_dense_attention.restype = i
+        lib.orc_window_attention.argtypes = [P, i, i, i, i, i, P, P, i, P, i, ctypes.c_double, P, P]
+        lib.orc_window_attention.restype = i
         lib.orc_round_bf16.argtypes = [ctypes.c_double]
         lib.orc_round_bf16.restype = ctypes.c_uint16
         lib.orc_num_threads.restype = i
@@ -229,6 +231,26 @@ def dense_attention(q, K, V, q_ctx, scale=None):
                                  _ptr(out), _ptr(lse))
     if rc != 0:
         raise ValueError(f"orc_dense_attention: bad arguments (rc={rc})")
+    return out, lse
+
+
+def window_attention(q, K, V, q_ctx, window, scale=None):
+    """The draft model's sliding-window attention: keys [max(0, n - window), n) for every query.
+    Returns (out f64, lse f64)."""
+    lib = _load()
+    q = _c(q, np.uint16)
+    K = _c(K, np.uint16)
+    V = _c(V, np.uint16)
+    q_ctx = _c(q_ctx, np.int32)
+    B, T, Hq, d = q.shape
+    _, Lcap, Hkv, _ = K.shape
+    s = scale if scale is not None else 1.0 / math.sqrt(d)
+    out = np.empty((B, T, Hq, d), np.float64)
+    lse = np.empty((B, T, Hq), np.float64)
+    rc = lib.orc_window_attention(_ptr(q), B, T, Hq, Hkv, d, _ptr(K), _ptr(V), Lcap, _ptr(q_ctx), int(window),
+                                  float(s), _ptr(out), _ptr(lse))
+    if rc != 0:
+        raise ValueError(f"orc_window_attention: bad arguments (rc={rc})")
     return out, lse
 
 

@@ -27,6 +27,8 @@
  *      draft tokens whose bit is set in the node's bit-packed ancestor mask
  *        -- QbitAI article, section "speculative sampling, quantisation and long text", long-context
  *           bullet (local attention mask with bit packing for tree drafts).
+ *   6. the draft model's sliding-window attention: the last `window` keys of the context
+ *        -- the same bullet (sliding-window attention for the draft model; no window size given).
  *
  * Every floating-point step is fp64; inputs are bf16 bit patterns widened exactly.  Rows are
  * independent, so the only parallelism is an OpenMP loop over (sequence, token, group) rows; there is
@@ -459,12 +461,13 @@ int orc_sparse_attention(const uint16_t* q, int B, int T, int Hq, int Hkv, int d
 /* plain causal attention, written separately (used to pin the sparse routine and as the dense path) */
 /* ----------------------------------------------------------------------------------------------- */
 
-/* out[b,t,h,:] = sum_{i < n} softmax_i(scale q.k_i) v_i with n = q_ctx[b*T+t]; GQA head h -> group h/G. */
-int orc_dense_attention(const uint16_t* q, int B, int T, int Hq, int Hkv, int d, const uint16_t* K,
-                        const uint16_t* V, int Lcap, const int32_t* q_ctx, double scale, double* out,
-                        double* lse_out)
+/* out[b,t,h,:] = sum_{lo <= i < n} softmax_i(scale q.k_i) v_i with n = q_ctx[b*T+t] and lo = 0, or
+ * lo = max(0, n - window) when window > 0; GQA head h -> group h/G. */
+static int range_attention(const uint16_t* q, int B, int T, int Hq, int Hkv, int d, const uint16_t* K,
+                           const uint16_t* V, int Lcap, const int32_t* q_ctx, long window, double scale,
+                           double* out, double* lse_out)
 {
-    if (Hkv <= 0 || Hq % Hkv != 0) return -1;
+    if (Hkv <= 0 || Hq % Hkv != 0 || window < 0) return -1;
     const int G = Hq / Hkv;
     for (long r = 0; r < (long)B * T; ++r)
         if (q_ctx[r] < 1 || q_ctx[r] > Lcap) return -1;
@@ -474,10 +477,11 @@ int orc_dense_attention(const uint16_t* q, int B, int T, int Hq, int Hkv, int d,
         const long bt = r / Hq;
         const int b = (int)(bt / T);
         const long n = q_ctx[bt];
+        const long lo = (window > 0 && n > window) ? n - window : 0;
         const uint16_t* qh = q + (size_t)r * d;
         double* oh = out + (size_t)r * d;
         double mx = -INFINITY;
-        for (long i = 0; i < n; ++i) {
+        for (long i = lo; i < n; ++i) {
             const uint16_t* kr = K + (((size_t)b * Lcap + i) * Hkv + h / G) * d;
             double dot = 0.0;
             for (int c = 0; c < d; ++c) dot += bf16_bits_to_f64(qh[c]) * bf16_bits_to_f64(kr[c]);
@@ -485,7 +489,7 @@ int orc_dense_attention(const uint16_t* q, int B, int T, int Hq, int Hkv, int d,
         }
         double den = 0.0;
         for (int c = 0; c < d; ++c) oh[c] = 0.0;
-        for (long i = 0; i < n; ++i) {
+        for (long i = lo; i < n; ++i) {
             const uint16_t* kr = K + (((size_t)b * Lcap + i) * Hkv + h / G) * d;
             const uint16_t* vr = V + (((size_t)b * Lcap + i) * Hkv + h / G) * d;
             double dot = 0.0;
@@ -498,6 +502,25 @@ int orc_dense_attention(const uint16_t* q, int B, int T, int Hq, int Hkv, int d,
         if (lse_out) lse_out[r] = mx + log(den);
     }
     return 0;
+}
+
+/* plain causal attention over keys [0, n) */
+int orc_dense_attention(const uint16_t* q, int B, int T, int Hq, int Hkv, int d, const uint16_t* K,
+                        const uint16_t* V, int Lcap, const int32_t* q_ctx, double scale, double* out,
+                        double* lse_out)
+{
+    return range_attention(q, B, T, Hq, Hkv, d, K, V, Lcap, q_ctx, 0, scale, out, lse_out);
+}
+
+/* sliding-window attention of the draft model: keys [max(0, n - window), n), window >= 1
+ *   -- QbitAI article, section "speculative sampling, quantisation and long text", long-context bullet
+ *      (the draft model attends with a sliding window; the pages give no window size) */
+int orc_window_attention(const uint16_t* q, int B, int T, int Hq, int Hkv, int d, const uint16_t* K,
+                         const uint16_t* V, int Lcap, const int32_t* q_ctx, int window, double scale, double* out,
+                         double* lse_out)
+{
+    if (window < 1) return -1;
+    return range_attention(q, B, T, Hq, Hkv, d, K, V, Lcap, q_ctx, window, scale, out, lse_out);
 }
 
 int orc_num_threads(void)

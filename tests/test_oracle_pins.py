@@ -402,3 +402,48 @@ def test_tree_attention_special_shapes(oracle, shape):
             qq = f64(q[0, i, h])[None, None, None]
             want = sdpa_fp64(qq, kk, vv, np.ones((1, 1, 1, kk.shape[2]), bool), 1 / math.sqrt(d))[0, 0, 0]
             assert np.max(np.abs(out[0, i, h] - want)) < 1e-12
+
+
+# ------------------------------------------------------------------------------------------------
+# the draft model's sliding-window attention
+# ------------------------------------------------------------------------------------------------
+
+@pytest.mark.parametrize("window", [1, 37, 64, 150, 1000])
+def test_window_attention_is_banded_softmax_attention(oracle, window):
+    """Keys [max(0, n - W), n) per query = torch softmax attention under a banded causal mask (GQA expanded);
+    a window past the context is plain causal attention."""
+    rng = np.random.default_rng(40 + window)
+    T = L = 200
+    Hq, Hkv, d = 4, 2, 16
+    q, K, V = rand_case(rng, 1, T, L, Hq, Hkv, d)
+    qc = np.arange(1, T + 1, dtype=np.int32)[None]
+    out, lse = oracle.window_attention(q, K, V, qc, window)
+    G = Hq // Hkv
+    qq = f64(q[0]).transpose(1, 0, 2)
+    kk = np.repeat(f64(K[0]).transpose(1, 0, 2), G, axis=0)
+    vv = np.repeat(f64(V[0]).transpose(1, 0, 2), G, axis=0)
+    tq = np.arange(T)[:, None]
+    ik = np.arange(L)[None, :]
+    band = ((ik <= tq) & (ik > tq - window))[None]
+    want = sdpa_fp64(qq, kk, vv, band, 1 / math.sqrt(d)).transpose(1, 0, 2)
+    assert np.max(np.abs(out[0] - want)) < 1e-12
+    logits = np.einsum("htd,hsd->hts", qq, kk) / math.sqrt(d)
+    logits[~np.broadcast_to(band, logits.shape)] = -np.inf
+    want_lse = torch.logsumexp(torch.from_numpy(logits), -1).numpy().T
+    assert np.max(np.abs(lse[0] - want_lse)) < 1e-12
+    if window >= L:
+        dense, _ = oracle.dense_attention(q, K, V, qc)
+        assert np.max(np.abs(out - dense)) < 1e-12
+
+
+def test_window_of_one_key_returns_that_value(oracle):
+    """W = 1: the softmax has one term, so the output is the newest value row and lse its logit"""
+    rng = np.random.default_rng(41)
+    q, K, V = rand_case(rng, 2, 1, 90, 8, 2, 32)
+    qc = np.array([[90], [53]], np.int32)
+    out, lse = oracle.window_attention(q, K, V, qc, 1)
+    for b in range(2):
+        n = int(qc[b, 0])
+        for h in range(8):
+            assert np.array_equal(out[b, 0, h], f64(V[b, n - 1, h // 4]))
+            assert lse[b, 0, h] == pytest.approx(f64(q[b, 0, h]) @ f64(K[b, n - 1, h // 4]) / math.sqrt(32), abs=1e-12)
