@@ -239,6 +239,18 @@ int infllmv2_dense_attn_decode(const void* q, int batch, int hq, int hkv, int he
                                int lcap, const int32_t* ctx_lens, int max_ctx, float softmax_scale, void* out,
                                float* lse, void* ws, size_t ws_bytes, infllmv2_stream_t stream);
 
+/*
+ * The draft model's sliding-window attention (MiniCPM4 technical details, section "speculative sampling,
+ * quantisation and long text", long-context bullet: the draft model attends with a sliding window; the
+ * pages give no window size).  One query per sequence attends to its last `window` keys:
+ *   out[b, h, :] = sum_{i in [max(0, n - window), n)} softmax_i(scale * q . k_i) v_i,  n = ctx_lens[b]
+ * Same layouts, scale rule and workspace as infllmv2_dense_attn_decode (size it with the same call and
+ * max_ctx; the window needs at most that much).  window >= 1, else INFLLMV2_ERR_INVALID_ARG.
+ */
+int infllmv2_window_attn_decode(const void* q, int batch, int hq, int hkv, int head_dim, const void* k, const void* v,
+                                int lcap, const int32_t* ctx_lens, int max_ctx, int window, float softmax_scale,
+                                void* out, float* lse, void* ws, size_t ws_bytes, infllmv2_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

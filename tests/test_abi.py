@@ -121,6 +121,9 @@ def test_attention_entry_points_reject_bad_arguments(lib):
     assert lib.infllmv2_kernel_pool(A16, 1, 4096, 2, 128, A4, A4, 4096, ctypes.byref(bad), A16, 255, None) == \
         UNSUPPORTED
     assert lib.infllmv2_kernel_pool(A16, 1, 4096, 2, 128, A4, A4, 4096, ctypes.byref(cp), A16, 10, None) == INVALID
+    # window decode: window 0
+    assert lib.infllmv2_window_attn_decode(A16, 1, 32, 2, 128, A16, A16, 4096, A4, 4096, 0, ctypes.c_float(0.0),
+                                           A16, None, WS, 1 << 30, None) == INVALID
     # kv append: misaligned new rows, null cache, empty capacity
     assert lib.infllmv2_kv_append(A16 + 2, A16, 4, 2, 128, A4, A16, A16, 4096, None) == INVALID
     assert lib.infllmv2_kv_append(A16, A16, 4, 2, 128, A4, None, A16, 4096, None) == INVALID

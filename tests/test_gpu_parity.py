@@ -218,6 +218,24 @@ def test_dense_paths(oracle, d):
     check_attention(out, out_o, lse, lse_o, what="dense decode")
 
 
+@pytest.mark.parametrize("d,G", [(128, 16), (64, 2)])
+@pytest.mark.parametrize("window", [1, 37, 64, 100, 2048, 10000])
+def test_window_attention_decode(oracle, d, G, window):
+    """infllmv2_window_attn_decode (the draft model's sliding window) against the oracle: ragged contexts,
+    windows shorter than a block, block-aligned, longer than some contexts"""
+    lens = [5000, 1, 64, 777, 130]
+    w = decode_case(lens, 2 * G, 2, d, topk=1, dense_len=0, seed=760 + d + window, n_needles=0)
+    out_o, lse_o = oracle.window_attention(w.q, w.k, w.v, w.q_ctx, window)
+    B = len(lens)
+    out = torch.empty((B, 1, 2 * G, d), dtype=torch.bfloat16, device="cuda")
+    lse = torch.empty((B, 1, 2 * G), dtype=torch.float32, device="cuda")
+    ws = binding.workspace(binding.Params(), B, 1, max(lens), 2 * G, 2, d)
+    binding.infllmv2_window_attn_decode(dev(w.q), dev(w.k), dev(w.v), dev_i32(w.ctx_lens), max(lens), window, 0.0,
+                                        out, lse, ws)
+    torch.cuda.synchronize()
+    check_attention(out, out_o, lse, lse_o, what=f"window {window} decode")
+
+
 @pytest.mark.parametrize("parents", ["random", "chain", "star"])
 def test_tree_verify(oracle, parents):
     P_, N = 3000, 16

@@ -81,6 +81,7 @@ _SIGS = {
                                           _P, _P, _SZ, _P], _I),
     "infllmv2_dense_attn_prefill": ([_P, _I, _I, _I, _I, _I, _P, _P, _I, _P, _P, _I, _F, _P, _P, _P, _SZ, _P], _I),
     "infllmv2_dense_attn_decode": ([_P, _I, _I, _I, _I, _P, _P, _I, _P, _I, _F, _P, _P, _P, _SZ, _P], _I),
+    "infllmv2_window_attn_decode": ([_P, _I, _I, _I, _I, _P, _P, _I, _P, _I, _I, _F, _P, _P, _P, _SZ, _P], _I),
 }
 
 EXPORTED = tuple(_SIGS)
@@ -300,6 +301,18 @@ def infllmv2_dense_attn_decode(q, k, v, ctx_lens, max_ctx, softmax_scale, out, l
                                            float(softmax_scale), _ptr(out), _ptr(lse), _ptr(ws),
                                            0 if ws is None else ws.numel() * ws.element_size(), _stream(stream))
     _check("infllmv2_dense_attn_decode", st)
+
+
+def infllmv2_window_attn_decode(q, k, v, ctx_lens, max_ctx, window, softmax_scale, out, lse, ws, stream=None):
+    for t, n in ((q, "q"), (k, "k"), (v, "v"), (out, "out")):
+        _need(t, torch.bfloat16, n)
+    B, Hq, d = q.shape[0], q.shape[-2], q.shape[-1]
+    Lcap, Hkv = k.shape[1], k.shape[2]
+    st = load().infllmv2_window_attn_decode(_ptr(q), B, Hq, Hkv, d, _ptr(k), _ptr(v), Lcap, _ptr(ctx_lens),
+                                            int(max_ctx), int(window), float(softmax_scale), _ptr(out), _ptr(lse),
+                                            _ptr(ws), 0 if ws is None else ws.numel() * ws.element_size(),
+                                            _stream(stream))
+    _check("infllmv2_window_attn_decode", st)
 
 
 def num_kernels(n: int, kernel_size: int = 32, kernel_stride: int = 16) -> int:

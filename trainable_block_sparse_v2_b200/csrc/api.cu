@@ -100,7 +100,7 @@ int check_params(const infllmv2_params* p)
 
 MethodConsts consts_of(const infllmv2_params* p, int d)
 {
-    MethodConsts mc;
+    MethodConsts mc{};
     mc.topk = p->topk;
     mc.init_blocks = p->init_blocks;
     mc.local_blocks = p->local_blocks;
@@ -108,6 +108,7 @@ MethodConsts consts_of(const infllmv2_params* p, int d)
     mc.membership = p->membership;
     mc.scale = p->softmax_scale > 0.f ? p->softmax_scale : 1.0f / std::sqrt((float)d);
     mc.kmax = p->topk + p->init_blocks + p->local_blocks;
+    mc.window = 0;
     return mc;
 }
 
@@ -168,10 +169,11 @@ size_t score_need(int batch, int nq, int hq, int hkv, int d, int max_ctx)
     return iv2::score_ws_bytes(batch * nq * hkv, max_ctx);
 }
 
-size_t split_need(int rows, int max_ctx, int kmax, int dense_len, bool dense_all, bool draft)
+size_t split_need(int rows, int max_ctx, int kmax, int dense_len, bool dense_all, bool draft, int window = 0)
 {
-    const int nsplit = iv2::attn_split_count(iv2::attn_split_max_blocks(max_ctx, kmax, dense_len, dense_all)) +
-                       (draft ? 1 : 0);
+    const int nsplit =
+        iv2::attn_split_count(iv2::attn_split_max_blocks(max_ctx, kmax, dense_len, dense_all, window)) +
+        (draft ? 1 : 0);
     return iv2::attn_ws_bytes(rows, nsplit);
 }
 
@@ -439,6 +441,29 @@ int infllmv2_dense_attn_decode(const void* q, int batch, int hq, int hkv, int he
     const MethodConsts mc = dense_consts(softmax_scale, head_dim);
     if (batch * hkv > iv2::kMaxSplitRows) return INFLLMV2_ERR_UNSUPPORTED;
     IV2_TRY(check_ws(ws, ws_bytes, split_need(batch * hkv, max_ctx, mc.kmax, 0, true, false)));
+    const QueryRows qr = rows_of(q, batch, 1, hq, hkv, head_dim, nullptr, ctx_lens, 0, max_ctx);
+    return launched(iv2::launch_attn_split(qr, k, v, lcap, nullptr, nullptr, mc, true, nullptr, nullptr, nullptr, out,
+                                           lse, ws, (cudaStream_t)stream));
+}
+
+int infllmv2_window_attn_decode(const void* q, int batch, int hq, int hkv, int head_dim, const void* k, const void* v,
+                                int lcap, const int32_t* ctx_lens, int max_ctx, int window, float softmax_scale,
+                                void* out, float* lse, void* ws, size_t ws_bytes, infllmv2_stream_t stream)
+{
+    IV2_TRY(check_heads(batch, 1, hq, hkv, head_dim));
+    if (!(softmax_scale == softmax_scale) || std::isinf(softmax_scale)) return INFLLMV2_ERR_INVALID_ARG;
+    if (window < 1) return INFLLMV2_ERR_INVALID_ARG;
+    IV2_TRY(check_ptr16(q));
+    IV2_TRY(check_ptr16(k));
+    IV2_TRY(check_ptr16(v));
+    IV2_TRY(check_ptr16(out));
+    IV2_TRY(check_ptr4(ctx_lens));
+    IV2_TRY(check_opt4(lse));
+    IV2_TRY(check_ctx(max_ctx, lcap));
+    MethodConsts mc = dense_consts(softmax_scale, head_dim);
+    mc.window = window;
+    if (batch * hkv > iv2::kMaxSplitRows) return INFLLMV2_ERR_UNSUPPORTED;
+    IV2_TRY(check_ws(ws, ws_bytes, split_need(batch * hkv, max_ctx, mc.kmax, 0, true, false, window)));
     const QueryRows qr = rows_of(q, batch, 1, hq, hkv, head_dim, nullptr, ctx_lens, 0, max_ctx);
     return launched(iv2::launch_attn_split(qr, k, v, lcap, nullptr, nullptr, mc, true, nullptr, nullptr, nullptr, out,
                                            lse, ws, (cudaStream_t)stream));

@@ -122,9 +122,11 @@ constexpr int kSplitWarps = 4;
 
 int attn_split_count(int max_blocks) { return (max_blocks + kSplitWarps - 1) / kSplitWarps; }
 
-int attn_split_max_blocks(int max_ctx, int kmax, int dense_len, bool dense_all)
+int attn_split_max_blocks(int max_ctx, int kmax, int dense_len, bool dense_all, int window)
 {
     const int all_blocks = (max_ctx + kBlock - 1) / kBlock;
+    // a window of W keys starting anywhere touches at most ceil(W / 64) + 1 blocks
+    if (window > 0) return min(all_blocks, (window + kBlock - 1) / kBlock + 1);
     if (dense_all) return all_blocks;
     const int dense_blocks = (min(max_ctx, dense_len) + kBlock - 1) / kBlock;
     return min(all_blocks, max(kmax, dense_blocks));
@@ -162,7 +164,10 @@ __global__ void __launch_bounds__(kSplitWarps * 32) attn_split_kernel(
     const int n = query_ctx(qr, b, t);
     const int c = (n - 1) / kBlock;
     const bool dense = dense_all || n <= mc.dense_len;
-    const int count = dense ? c + 1 : min(cnt[row], mc.kmax);
+    // sliding window: the blocks of keys [w0, n), walked like a dense row from block w0 / 64
+    const int w0 = mc.window > 0 ? max(0, n - mc.window) : 0;
+    const int bw = w0 / kBlock;
+    const int count = mc.window > 0 ? c + 1 - bw : (dense ? c + 1 : min(cnt[row], mc.kmax));
     const int32_t* idx_row = idx ? idx + (size_t)row * mc.kmax : nullptr;
     const float sl2 = mc.scale * kLog2e;
 
@@ -186,7 +191,8 @@ __global__ void __launch_bounds__(kSplitWarps * 32) attn_split_kernel(
             work = true;
         }
     } else {
-        blk = row_block(dense, c, idx_row, count, split * kSplitWarps + warp, n);
+        const int e = split * kSplitWarps + warp;
+        blk = mc.window > 0 ? (e < count ? bw + e : -1) : row_block(dense, c, idx_row, count, e, n);
         if (blk >= 0) {
             const size_t rs = (size_t)qr.Hkv * D;
             const size_t base = ((size_t)b * Lcap * qr.Hkv + g) * D + (size_t)blk * kBlock * rs;
@@ -194,7 +200,8 @@ __global__ void __launch_bounds__(kSplitWarps * 32) attn_split_kernel(
             warp_load_tile<D>(ks_tile, k + base, rs, nvalid);
             warp_load_tile<D>(vs_tile, v + base, rs, nvalid);
             cp_async_commit();
-            valid = prefix_mask64(nvalid);
+            // keys [blk 64, blk 64 + nvalid), less those before the window's first key
+            valid = prefix_mask64(nvalid) & ~prefix_mask64(max(0, w0 - blk * kBlock));
             work = true;
         }
     }
@@ -271,7 +278,8 @@ __global__ void __launch_bounds__(D) attn_merge_kernel(QueryRows qr, const int32
     const int n = query_ctx(qr, b, t);
     const int c = (n - 1) / kBlock;
     const bool dense = dense_all || n <= mc.dense_len;
-    const int count = dense ? c + 1 : min(cnt[row], mc.kmax);
+    const int count = mc.window > 0 ? c + 1 - max(0, n - mc.window) / kBlock
+                                    : (dense ? c + 1 : min(cnt[row], mc.kmax));
     const int nused = min((count + kSplitWarps - 1) / kSplitWarps, nsplit_blocks);
     const int nsplit_total = nsplit_blocks + has_draft;
     const float* base = ws + (size_t)row * nsplit_total * SplitWs<D>::kFloats;
@@ -345,7 +353,7 @@ static cudaError_t split_impl(const QueryRows& qr, const void* k, const void* v,
                               const void* v_draft, const uint32_t* tree_mask, void* out, float* lse, void* ws,
                               cudaStream_t s)
 {
-    const int max_blocks = attn_split_max_blocks(qr.max_ctx, mc.kmax, mc.dense_len, dense_all);
+    const int max_blocks = attn_split_max_blocks(qr.max_ctx, mc.kmax, mc.dense_len, dense_all, mc.window);
     const int nsplit_blocks = attn_split_count(max_blocks);
     const int nsplit_total = nsplit_blocks + (tree_mask ? 1 : 0);
     const size_t smem = (size_t)kSplitWarps * 2 * KvTile<D>::kBytes;

@@ -73,7 +73,7 @@ extern "C" int infllmv2_sparse_attn_decode_noalloc(const void* q, int batch, int
     if (max_ctx < 1 || max_ctx > lcap) return INFLLMV2_ERR_INVALID_ARG;
     if ((max_ctx - 1) / iv2::kBlock + 1 > 4096) return INFLLMV2_ERR_UNSUPPORTED;
 
-    iv2::MethodConsts mc;
+    iv2::MethodConsts mc{};
     mc.topk = params->topk;
     mc.init_blocks = params->init_blocks;
     mc.local_blocks = params->local_blocks;

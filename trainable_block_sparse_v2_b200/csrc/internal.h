@@ -87,6 +87,7 @@ struct MethodConsts {
     int topk, init_blocks, local_blocks, dense_len, membership;
     float scale;              // softmax scale (natural units)
     int kmax;                 // topk + init + local
+    int window;               // > 0: attend to the last `window` keys only (sliding window); 0: off
 };
 
 // rows (sequence x query x KV group) one split-attention launch handles
@@ -100,7 +101,7 @@ size_t attn_ws_bytes(int rows, int nsplit);
 // CTAs per row of the split attention for a block list of max_blocks entries
 int attn_split_count(int max_blocks);
 // largest block list the split attention handles for these sizes
-int attn_split_max_blocks(int max_ctx, int kmax, int dense_len, bool dense_all);
+int attn_split_max_blocks(int max_ctx, int kmax, int dense_len, bool dense_all, int window = 0);
 
 cudaError_t launch_kernel_pool(const void* k, int B, int Lcap, int Hkv, int D, const int32_t* old_lens,
                                const int32_t* new_lens, int max_new_keys, void* kern, int nk_cap, cudaStream_t s);
