@@ -299,6 +299,38 @@ class DecodeBench:
             del g
         return out
 
+    def window_time(self, window, steps):
+        """device time of one sliding-window decode call (the draft model's attention: the last `window` keys of
+        each sequence), from `steps` consecutive calls over the rotating layer caches captured in one graph"""
+        torch = self.torch
+        p = self.b.Params(**self.w.params)
+        ws = self.b.workspace(p, self.B, 1, self.max_ctx, HQ, HKV, D)
+        out = torch.empty((self.B, 1, HQ, D), dtype=torch.bfloat16, device="cuda")
+        calls = [self._coords(s) for s in range(steps)]
+
+        def run():
+            for layer, pos in calls:
+                self.b.infllmv2_window_attn_decode(self.q_of(layer, pos), self.k[layer], self.v[layer], self.lens[pos],
+                                                   self.max_ctx, window, 0.0, out, None, ws)
+        st = torch.cuda.Stream()
+        st.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(st):
+            run()
+        torch.cuda.current_stream().wait_stream(st)
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            run()
+        g.replay()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        reps = 4
+        e0.record()
+        for _ in range(reps):
+            g.replay()
+        e1.record()
+        e1.synchronize()
+        return e0.elapsed_time(e1) / 1e3 / (reps * steps)
+
     def e2e(self, warmup, steps):
         """Same step through the C ABI with host buffers: every step copies that step's query and the new key
         and value rows from pinned host memory to the device in one copy, appends the rows to the caches
@@ -558,6 +590,10 @@ def run_ours(args):
             dom = "sparse_decode_step"
             dom_bytes = scan_b + kv_b
         achieved = dom_bytes / per[dom] / 1e9
+        # the draft model's sliding-window attention on the same caches (next-row measurement)
+        win = 2048
+        t_win = db.window_time(win, min(args.steps, 256))
+        win_bytes = len(LENS_128K) * HKV * win * D * 2 * 2
         e2e_steps = min(args.steps, 512)
         e2e_t, h2d, d2h = db.e2e(8, e2e_steps) if args.e2e else (float("nan"), 0, 0)
 
@@ -585,6 +621,11 @@ def run_ours(args):
             "e2e": {"value": len(LENS_128K) * e2e_steps / e2e_t, "unit": UNIT, "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h, "steps": e2e_steps},
             "gpu_launches": KERNELS_PER_STEP[args.decode_path] * args.steps,
+            "window_decode": {"window": win, "value": len(LENS_128K) / t_win, "unit": UNIT, "us_per_call": t_win * 1e6,
+                              "algorithmic_bytes": win_bytes, "achieved_gbs": win_bytes / t_win / 1e9,
+                              "frac_of_" + peak_kind: win_bytes / t_win / 1e9 / peaks["hbm_gbs"],
+                              "note": "the draft model's sliding-window decode attention (last 2048 keys), "
+                                      "4 sequences per call, split + merge kernels"},
         }
         del db
         torch.cuda.empty_cache()
