@@ -23,7 +23,8 @@
 //   5. combine: each CTA pushes its (O, m, l) of head h to CTA h % CL; after a third barrier that CTA
 //      merges the CL partials and writes the output row.
 // The footprint (about 112 KB of shared memory) lets two CTAs share an SM, so eight 16-CTA clusters are
-// resident at once.
+// resident at once.  Every 2^x here has x <= 0 (a difference from a running or final maximum) or -inf,
+// so the hardware ex2.approx (one MUFU op, tiny results flushed to zero) serves throughout.
 #include <cooperative_groups.h>
 
 #include "attn_warp.cuh"
@@ -112,7 +113,7 @@ IV2_DEV void online_merge(float& m, float& s, float m2, float s2)
         return;
     }
     const float M = fmaxf(m, m2);
-    s = s * exp2_fast(m - M) + s2 * exp2_fast(m2 - M);
+    s = s * ex2_approx(m - M) + s2 * ex2_approx(m2 - M);
     m = M;
 }
 
@@ -251,8 +252,8 @@ decode_fused_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_con
             for (int r = 0; r < 2; ++r) {
                 const float m4 = fmaxf(fmaxf(z[0][2 * r], z[0][2 * r + 1]), fmaxf(z[1][2 * r], z[1][2 * r + 1]));
                 const float mn = fmaxf(lm[r], m4);
-                ls[r] = ls[r] * exp2_fast(lm[r] - mn) + (exp2_fast(z[0][2 * r] - mn) + exp2_fast(z[0][2 * r + 1] - mn)) +
-                        (exp2_fast(z[1][2 * r] - mn) + exp2_fast(z[1][2 * r + 1] - mn));
+                ls[r] = ls[r] * ex2_approx(lm[r] - mn) + (ex2_approx(z[0][2 * r] - mn) + ex2_approx(z[0][2 * r + 1] - mn)) +
+                        (ex2_approx(z[1][2 * r] - mn) + ex2_approx(z[1][2 * r + 1] - mn));
                 lm[r] = mn;
             }
             // block maxima: tile j holds the stage's blocks 2 tt and 2 tt + 1 (tt = warp + 8 j) as cols 0..3 and
@@ -307,7 +308,7 @@ decode_fused_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_con
             }
 #pragma unroll
             for (int w = 0; w < kFWarps; ++w)
-                s += (mw[w] == neg_inf()) ? 0.f : wred[kFWarps * 16 + w * 16 + tid] * exp2_fast(mw[w] - m);
+                s += (mw[w] == neg_inf()) ? 0.f : wred[kFWarps * 16 + w * 16 + tid] * ex2_approx(mw[w] - m);
             part_m[tid] = m;
             part_s[tid] = s;
         }
@@ -337,7 +338,7 @@ decode_fused_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_con
                 m = fmaxf(m, mr[r]);
             }
 #pragma unroll
-            for (int r = 0; r < CL; ++r) s += (mr[r] == neg_inf()) ? 0.f : lse_slot[r][tid][1] * exp2_fast(mr[r] - m);
+            for (int r = 0; r < CL; ++r) s += (mr[r] == neg_inf()) ? 0.f : lse_slot[r][tid][1] * ex2_approx(mr[r] - m);
             lse2[tid] = m == neg_inf() ? neg_inf() : m + __log2f(s);
         }
         __syncthreads();
@@ -347,7 +348,7 @@ decode_fused_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_con
 #pragma unroll
             for (int h = 0; h < 16; ++h) {
                 const uint32_t key = bmax[h * kFBmaxPitch + k];
-                if (h < G && key != 0u) acc += exp2_fast(key_float(key) - lse2[h]);
+                if (h < G && key != 0u) acc += ex2_approx(key_float(key) - lse2[h]);
             }
             S[b0 + k] = member ? acc : neg_inf();
         }
@@ -456,7 +457,7 @@ decode_fused_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_con
                     mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
                     mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
                     const float mnew = fmaxf(st.m[r], mx);
-                    const float alpha = st.m[r] == neg_inf() ? 0.f : exp2_fast(st.m[r] - mnew);
+                    const float alpha = st.m[r] == neg_inf() ? 0.f : ex2_approx(st.m[r] - mnew);
                     st.m[r] = mnew;
                     st.l[r] *= alpha;
 #pragma unroll
@@ -464,8 +465,8 @@ decode_fused_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_con
                         st.o[nt][2 * r] *= alpha;
                         st.o[nt][2 * r + 1] *= alpha;
                     }
-                    p[2 * r] = exp2_fast(sc[2 * r] - mnew);
-                    p[2 * r + 1] = exp2_fast(sc[2 * r + 1] - mnew);
+                    p[2 * r] = ex2_approx(sc[2 * r] - mnew);
+                    p[2 * r + 1] = ex2_approx(sc[2 * r + 1] - mnew);
                     st.l[r] += p[2 * r] + p[2 * r + 1];
                 }
                 const uint32_t pa0 = pack_bf16(p[0], p[1]), pa1 = pack_bf16(p[2], p[3]);
@@ -511,7 +512,7 @@ decode_fused_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_con
 #pragma unroll
         for (int w = 0; w < kFWarps; ++w) {
             const float mw = wm[w * 16 + tid];
-            const float f = (mw == neg_inf()) ? 0.f : exp2_fast(mw - M);
+            const float f = (mw == neg_inf()) ? 0.f : ex2_approx(mw - M);
             wf[w * 16 + tid] = f;
             Ls += f * wl[w * 16 + tid];
         }
@@ -560,7 +561,7 @@ decode_fused_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_con
 #pragma unroll
                 for (int r = 0; r < CL; ++r) {
                     const float mr = hs[r * L::kSlotPitch + D];
-                    const float f = (mr == neg_inf()) ? 0.f : exp2_fast(mr - M);
+                    const float f = (mr == neg_inf()) ? 0.f : ex2_approx(mr - M);
                     O += hs[r * L::kSlotPitch + d] * f;
                     Lsum += hs[r * L::kSlotPitch + D + 1] * f;
                 }
