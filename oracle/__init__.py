@@ -15,7 +15,11 @@ Functions and the steps they follow (sources: the MiniCPM4 pages):
                               group, top-k plus initial and local blocks (same section, items 1-3)
   * ``sparse_attention``   -- attention over the selected blocks, optional bit-packed tree-draft mask
                               (same article, "speculative sampling ... long text", long-context bullet)
+  * ``sparse_attention_backward`` -- gradients of that attention for a fixed selection (training; same
+                              section, item 3: operators for training and inference; the derivative of
+                              the forward's definition)
   * ``dense_attention``    -- plain causal GQA attention, written separately
+  * ``window_attention``   -- the draft model's sliding-window attention (same bullet as the tree drafts)
 The pages' "efficient LogSumExp estimation" is not implemented: parity unpinned (not defined there).
 """
 from __future__ import annotations
@@ -99,6 +103,9 @@ def _load():
         lib.orc_sparse_attention.argtypes = [P, i, i, i, i, i, P, P, i, P, P, P, i, ctypes.POINTER(_Params),
                                              P, P, P, P, P]
         lib.orc_sparse_attention.restype = i
+        lib.orc_sparse_attention_backward.argtypes = [P, i, i, i, i, i, P, P, i, P, P, P, i,
+                                                      ctypes.POINTER(_Params), P, P, P, P]
+        lib.orc_sparse_attention_backward.restype = i
         lib.orc_dense_attention.argtypes = [P, i, i, i, i, i, P, P, i, P, ctypes.c_double, P, P]
         lib.orc_dense_attention.restype = i
         lib.orc_window_attention.argtypes = [P, i, i, i, i, i, P, P, i, P, i, ctypes.c_double, P, P]
@@ -213,6 +220,35 @@ def sparse_attention(q, K, V, q_ctx, idx, cnt, params: Params, k_draft=None, v_d
     if rc != 0:
         raise ValueError(f"orc_sparse_attention: bad arguments (rc={rc})")
     return out, lse
+
+
+def sparse_attention_backward(q, K, V, q_ctx, idx, cnt, params: Params, dout):
+    """Gradients of sum(dout * out) for the sparse attention with a fixed selection (no tree drafts).
+
+    Same inputs as sparse_attention plus dout [B,T,Hq,d] (bf16 bits).  Returns (dq [B,T,Hq,d],
+    dk [B,Lcap,Hkv,d], dv [B,Lcap,Hkv,d]), all f64.
+    """
+    lib = _load()
+    q = _c(q, np.uint16)
+    K = _c(K, np.uint16)
+    V = _c(V, np.uint16)
+    dout = _c(dout, np.uint16)
+    q_ctx = _c(q_ctx, np.int32)
+    idx = _c(idx, np.int32)
+    cnt = _c(cnt, np.int32)
+    B, T, Hq, d = q.shape
+    _, Lcap, Hkv, _ = K.shape
+    kmax = idx.shape[-1]
+    dq = np.empty((B, T, Hq, d), np.float64)
+    dk = np.empty((B, Lcap, Hkv, d), np.float64)
+    dv = np.empty((B, Lcap, Hkv, d), np.float64)
+    cp = params.c_struct(d)
+    rc = lib.orc_sparse_attention_backward(_ptr(q), B, T, Hq, Hkv, d, _ptr(K), _ptr(V), Lcap, _ptr(q_ctx),
+                                           _ptr(idx), _ptr(cnt), kmax, ctypes.byref(cp), _ptr(dout), _ptr(dq),
+                                           _ptr(dk), _ptr(dv))
+    if rc != 0:
+        raise ValueError(f"orc_sparse_attention_backward: bad arguments (rc={rc})")
+    return dq, dk, dv
 
 
 def dense_attention(q, K, V, q_ctx, scale=None):

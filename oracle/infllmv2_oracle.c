@@ -29,6 +29,9 @@
  *           bullet (local attention mask with bit packing for tree drafts).
  *   6. the draft model's sliding-window attention: the last `window` keys of the context
  *        -- the same bullet (sliding-window attention for the draft model; no window size given).
+ *   7. the gradients of step 5's attention with respect to q, K and V for a fixed selection (training)
+ *        -- "Model architecture: InfLLM v2", item 3 (operators for training as well as inference); the
+ *           derivative of step 5's definition, the pages give no formula.
  *
  * Every floating-point step is fp64; inputs are bf16 bit patterns widened exactly.  Rows are
  * independent, so the only parallelism is an OpenMP loop over (sequence, token, group) rows; there is
@@ -43,7 +46,9 @@
  *     counted against k; the output set is sorted ascending and padded with -1.
  *
  * Parity pins (tests/test_oracle_pins.py): hand-worked two-block example, closed forms of the window
- * mean, special cases that reduce to library softmax attention / average pooling, and invariants.
+ * mean, special cases that reduce to library softmax attention / average pooling, and invariants; the
+ * backward (item 7) against central differences of the forward, library autograd on the dense case,
+ * the one-key closed form and the sum rules of the softmax Jacobian.
  * The pages' "efficient LogSumExp estimation" is not implemented here (parity unpinned: the pages do
  * not define it).
  */
@@ -453,6 +458,129 @@ int orc_sparse_attention(const uint16_t* q, int B, int T, int Hq, int Hkv, int d
         }
         free(keys);
         free(logit);
+    }
+    return status;
+}
+
+/* ----------------------------------------------------------------------------------------------- */
+/* backward of the sparse attention for a fixed selection (training)                                */
+/* ----------------------------------------------------------------------------------------------- */
+
+/*
+ * Gradients of L = sum over (b, t, h, c) of dout * out with respect to q, K and V, where out is the
+ * sparse attention above (no tree drafts).  The pages train InfLLM v2 with the same sparse attention
+ * ("Tsinghua & ModelBest: MiniCPM4 technical details", "Model architecture: InfLLM v2", item 3: efficient
+ * operators for training and inference) but give no formula; this is the derivative of the forward's own
+ * definition.  The selection is a piecewise-constant function of q and K, so for a fixed selection no
+ * gradient flows through the block scores or the semantic kernels.
+ *
+ * For a row (b, t, h) with key set K(t) (the forward's), logits s_e = scale q.k_e, probabilities
+ * p_e = exp(s_e) / sum exp(s), and out = sum_e p_e v_e:
+ *   dp_e  = dout . v_e                       (dL/dp_e)
+ *   Dsum  = sum_e p_e dp_e                   (= dout . out)
+ *   ds_e  = p_e (dp_e - Dsum)                (dL/ds_e, the softmax Jacobian)
+ *   dq   += scale sum_e ds_e k_e
+ *   dk_e += scale ds_e q,   dv_e += p_e dout (summed over the rows that read key e)
+ * dout: [B, T, Hq, d] bf16 bits.  dq: [B, T, Hq, d] fp64; dk, dv: [B, Lcap, Hkv, d] fp64, overwritten
+ * (keys no row reads get 0).  Returns 0, or -1 on a bad argument (as orc_sparse_attention).
+ */
+int orc_sparse_attention_backward(const uint16_t* q, int B, int T, int Hq, int Hkv, int d, const uint16_t* K,
+                                  const uint16_t* V, int Lcap, const int32_t* q_ctx, const int32_t* idx,
+                                  const int32_t* cnt, int kmax, const orc_params* p, const uint16_t* dout,
+                                  double* dq, double* dk, double* dv)
+{
+    if (Hkv <= 0 || Hq % Hkv != 0) return -1;
+    const int G = Hq / Hkv;
+    const long rows = (long)B * T * Hkv;
+    for (long r = 0; r < rows; ++r) {
+        const long bt = r / Hkv;
+        const long n = q_ctx[bt];
+        if (n < 1 || n > Lcap) return -1;
+        if (n <= p->dense_len) continue;
+        if (cnt[r] < 0 || cnt[r] > kmax) return -1;
+        for (int i = 0; i < cnt[r]; ++i) {
+            long blk = idx[r * kmax + i];
+            if (blk < 0 || blk * p->block_size >= n) return -1;
+        }
+    }
+    memset(dk, 0, sizeof(double) * (size_t)B * Lcap * Hkv * d);
+    memset(dv, 0, sizeof(double) * (size_t)B * Lcap * Hkv * d);
+    int status = 0;
+    /* one (sequence, KV group) per task: the rows of a task are the only writers of its dk / dv slice */
+#pragma omp parallel
+    {
+        long* keys = (long*)malloc(sizeof(long) * (size_t)(Lcap + 1));
+        double* prob = (double*)malloc(sizeof(double) * (size_t)(Lcap + 1));
+        double* dprob = (double*)malloc(sizeof(double) * (size_t)(Lcap + 1));
+        if (!keys || !prob || !dprob) {
+#pragma omp atomic write
+            status = -2;
+        } else {
+#pragma omp for schedule(dynamic, 1)
+            for (long bg = 0; bg < (long)B * Hkv; ++bg) {
+                const int b = (int)(bg / Hkv), g = (int)(bg % Hkv);
+                for (int t = 0; t < T; ++t) {
+                    const long bt = (long)b * T + t;
+                    const long r = bt * Hkv + g;
+                    const long n = q_ctx[bt];
+                    long nkeys = 0;
+                    if (n <= p->dense_len) {
+                        for (long i = 0; i < n; ++i) keys[nkeys++] = i;
+                    } else {
+                        for (int s = 0; s < cnt[r]; ++s) {
+                            long blk = idx[r * kmax + s];
+                            long k0 = blk * p->block_size, k1 = k0 + p->block_size;
+                            if (k1 > n) k1 = n;
+                            for (long i = k0; i < k1; ++i) keys[nkeys++] = i;
+                        }
+                    }
+                    for (int hh = 0; hh < G; ++hh) {
+                        const int h = g * G + hh;
+                        const uint16_t* qh = q + ((size_t)bt * Hq + h) * d;
+                        const uint16_t* doh = dout + ((size_t)bt * Hq + h) * d;
+                        double* dqh = dq + ((size_t)bt * Hq + h) * d;
+                        for (int c2 = 0; c2 < d; ++c2) dqh[c2] = 0.0;
+                        if (nkeys == 0) continue;
+                        /* probabilities of the forward */
+                        double mx = -INFINITY;
+                        for (long e = 0; e < nkeys; ++e) {
+                            const uint16_t* kr = K + (((size_t)b * Lcap + keys[e]) * Hkv + g) * d;
+                            double dot = 0.0;
+                            for (int c2 = 0; c2 < d; ++c2) dot += bf16_bits_to_f64(qh[c2]) * bf16_bits_to_f64(kr[c2]);
+                            prob[e] = p->scale * dot;
+                            if (prob[e] > mx) mx = prob[e];
+                        }
+                        double den = 0.0;
+                        for (long e = 0; e < nkeys; ++e) {
+                            prob[e] = exp(prob[e] - mx);
+                            den += prob[e];
+                        }
+                        for (long e = 0; e < nkeys; ++e) prob[e] /= den;
+                        /* dL/dp and the softmax Jacobian */
+                        double dsum = 0.0;
+                        for (long e = 0; e < nkeys; ++e) {
+                            const uint16_t* vr = V + (((size_t)b * Lcap + keys[e]) * Hkv + g) * d;
+                            double dot = 0.0;
+                            for (int c2 = 0; c2 < d; ++c2) dot += bf16_bits_to_f64(doh[c2]) * bf16_bits_to_f64(vr[c2]);
+                            dprob[e] = dot;
+                            dsum += prob[e] * dot;
+                        }
+                        for (long e = 0; e < nkeys; ++e) {
+                            const double ds = prob[e] * (dprob[e] - dsum);
+                            const size_t kv = (((size_t)b * Lcap + keys[e]) * Hkv + g) * d;
+                            for (int c2 = 0; c2 < d; ++c2) {
+                                dqh[c2] += p->scale * ds * bf16_bits_to_f64(K[kv + c2]);
+                                dk[kv + c2] += p->scale * ds * bf16_bits_to_f64(qh[c2]);
+                                dv[kv + c2] += prob[e] * bf16_bits_to_f64(doh[c2]);
+                            }
+                        }
+                    }
+                }
+            }
+        }
+        free(keys);
+        free(prob);
+        free(dprob);
     }
     return status;
 }

@@ -447,3 +447,129 @@ def test_window_of_one_key_returns_that_value(oracle):
         for h in range(8):
             assert np.array_equal(out[b, 0, h], f64(V[b, n - 1, h // 4]))
             assert lse[b, 0, h] == pytest.approx(f64(q[b, 0, h]) @ f64(K[b, n - 1, h // 4]) / math.sqrt(32), abs=1e-12)
+
+
+# ------------------------------------------------------------------------------------------------
+# backward of the sparse attention (fixed selection)
+# ------------------------------------------------------------------------------------------------
+
+def _grid_case(rng, B, T, L, Hq, Hkv, d):
+    """inputs on the grid k/8, |k| <= 8, so that x +- 1/64 and x +- 1/32 are exact bf16 values"""
+    def g(shape):
+        return bits(rng.integers(-8, 9, size=shape).astype(np.float32) / 8.0)
+    return g((B, T, Hq, d)), g((B, L, Hkv, d)), g((B, L, Hkv, d))
+
+
+def test_backward_matches_central_differences(oracle):
+    """Each gradient entry = Richardson-extrapolated central difference of the oracle's own forward loss
+    sum(dout * out), stepping the bf16 input by exactly 1/64 and 1/32 (error O(h^4) ~ 1e-8)."""
+    rng = np.random.default_rng(50)
+    B, T, L, Hq, Hkv, d = 1, 5, 10, 4, 2, 4
+    q, K, V = _grid_case(rng, B, T, L, Hq, Hkv, d)
+    dout = bits(rng.integers(-8, 9, size=(B, T, Hq, d)).astype(np.float32) / 8.0)
+    # block size 2: explicit sets with gaps, a partial last block, and one dense row (n <= dense_len)
+    P = oracle.Params(block_size=2, topk=2, init_blocks=0, local_blocks=0, dense_len=3)
+    qc = np.array([[10, 7, 3, 9, 5]], np.int32)
+    sets = [[[0, 3], [4]], [[1, 3], [0, 2]], [[0], [0]], [[4], [1, 3]], [[2], [0, 1]]]
+    idx = np.full((B, T, Hkv, 2), -1, np.int32)
+    cnt = np.zeros((B, T, Hkv), np.int32)
+    for t in range(T):
+        for g in range(Hkv):
+            idx[0, t, g, :len(sets[t][g])] = sets[t][g]
+            cnt[0, t, g] = len(sets[t][g])
+    dq, dk, dv = oracle.sparse_attention_backward(q, K, V, qc, idx, cnt, P, dout)
+    w = f64(dout)
+
+    def loss(qb, Kb, Vb):
+        out, _ = oracle.sparse_attention(qb, Kb, Vb, qc, idx, cnt, P)
+        return float(np.sum(w * out))
+
+    def fd(arr, which, pos):
+        vals = []
+        for h in (1 / 64, 1 / 32):
+            plus, minus = arr.copy(), arr.copy()
+            x = f64(arr[pos])
+            plus[pos] = bits(np.array([x + h], np.float32))[0]
+            minus[pos] = bits(np.array([x - h], np.float32))[0]
+            args_p = [q, K, V]
+            args_m = [q, K, V]
+            args_p[which] = plus
+            args_m[which] = minus
+            vals.append((loss(*args_p) - loss(*args_m)) / (2 * h))
+        return (4 * vals[0] - vals[1]) / 3
+
+    for which, arr, grad in ((0, q, dq), (1, K, dk), (2, V, dv)):
+        for pos in np.ndindex(arr.shape):
+            assert grad[pos] == pytest.approx(fd(arr, which, pos), abs=2e-6), (which, pos)
+    # keys 8, 9 lie past every sparse row's blocks except row 0 (block 4) and row 3: nonzero there
+    assert np.any(dv[0, 8:] != 0)
+
+
+def test_backward_dense_matches_torch_autograd(oracle):
+    """Every block selected: the gradients are those of torch causal softmax attention (fp64 autograd,
+    GQA by repeating K/V over the group, whose backward sums the group's heads)."""
+    rng = np.random.default_rng(51)
+    T = L = 150
+    Hq, Hkv, d = 4, 2, 16
+    q, K, V = rand_case(rng, 1, T, L, Hq, Hkv, d)
+    dout = f32_to_bf16_bits(rng.standard_normal((1, T, Hq, d)).astype(np.float32))
+    qc = np.arange(1, T + 1, dtype=np.int32)[None]
+    P = oracle.Params(topk=100)
+    kern = oracle.kernel_pool(K, [0], [L], 32, 16)
+    r = oracle.block_score_topk(q, kern, qc, P)
+    dq, dk, dv = oracle.sparse_attention_backward(q, K, V, qc, r["idx"], r["cnt"], P, dout)
+    G = Hq // Hkv
+    qt = torch.from_numpy(f64(q[0]).transpose(1, 0, 2).copy()).requires_grad_()
+    kt = torch.from_numpy(f64(K[0]).transpose(1, 0, 2).copy()).requires_grad_()
+    vt = torch.from_numpy(f64(V[0]).transpose(1, 0, 2).copy()).requires_grad_()
+    causal = torch.from_numpy(np.tril(np.ones((T, L), bool)))[None]
+    out = torch.nn.functional.scaled_dot_product_attention(
+        qt, kt.repeat_interleave(G, 0), vt.repeat_interleave(G, 0), attn_mask=causal, scale=1 / math.sqrt(d))
+    out.backward(torch.from_numpy(f64(dout[0]).transpose(1, 0, 2).copy()))
+    assert np.max(np.abs(dq[0] - qt.grad.numpy().transpose(1, 0, 2))) < 1e-11
+    assert np.max(np.abs(dk[0] - kt.grad.numpy().transpose(1, 0, 2))) < 1e-11
+    assert np.max(np.abs(dv[0] - vt.grad.numpy().transpose(1, 0, 2))) < 1e-11
+
+
+def test_backward_one_key_closed_form(oracle):
+    """A query that sees one key has p = 1: its dq and that key's dk are exactly 0, and dv of the key is
+    the sum of dout over the rows that read it."""
+    rng = np.random.default_rng(52)
+    q, K, V = rand_case(rng, 1, 3, 70, 4, 2, 8)
+    dout = f32_to_bf16_bits(rng.standard_normal((1, 3, 4, 8)).astype(np.float32))
+    qc = np.array([[1, 1, 1]], np.int32)
+    P = oracle.Params(topk=1)
+    idx = np.zeros((1, 3, 2, 4), np.int32)
+    idx[..., 1:] = -1
+    cnt = np.ones((1, 3, 2), np.int32)
+    dq, dk, dv = oracle.sparse_attention_backward(q, K, V, qc, idx, cnt, P, dout)
+    assert np.array_equal(dq, np.zeros_like(dq)) and np.array_equal(dk, np.zeros_like(dk))
+    for g in range(2):
+        assert np.max(np.abs(dv[0, 0, g] - f64(dout[0, :, 2 * g:2 * g + 2]).sum(axis=(0, 1)))) < 1e-13
+    assert np.array_equal(dv[0, 1:], np.zeros_like(dv[0, 1:]))
+
+
+def test_backward_sum_rules(oracle):
+    """Identities of any softmax attention, on a sparse case with dense rows:
+    sum_j dk_j = 0 (a common shift of the keys leaves every softmax unchanged);
+    sum_j dv_j = sum over rows of dout (each row's probabilities sum to 1);
+    sum dv . V = sum dout . out (out is linear in V);  sum dq . q = sum dk . K (logits are bilinear)."""
+    rng = np.random.default_rng(53)
+    B, T, L, Hq, Hkv, d = 2, 40, 400, 8, 2, 16
+    q, K, V = rand_case(rng, B, T, L, Hq, Hkv, d)
+    dout = f32_to_bf16_bits(rng.standard_normal((B, T, Hq, d)).astype(np.float32))
+    qc = np.stack([np.linspace(20, 400, T).astype(np.int32), np.linspace(5, 300, T).astype(np.int32)])
+    P = oracle.Params(topk=2, dense_len=100)
+    kern = oracle.kernel_pool(K, [0, 0], [L, L], 32, 16)
+    r = oracle.block_score_topk(q, kern, qc, P)
+    dq, dk, dv = oracle.sparse_attention_backward(q, K, V, qc, r["idx"], r["cnt"], P, dout)
+    out, _ = oracle.sparse_attention(q, K, V, qc, r["idx"], r["cnt"], P)
+    G = Hq // Hkv
+    for b in range(B):
+        for g in range(Hkv):
+            assert np.max(np.abs(dk[b, :, g].sum(axis=0))) < 1e-10
+            want = f64(dout[b, :, g * G:(g + 1) * G]).sum(axis=(0, 1))
+            assert np.max(np.abs(dv[b, :, g].sum(axis=0) - want)) < 1e-10
+    assert np.sum(dv * f64(V)) == pytest.approx(np.sum(f64(dout) * out), rel=1e-12)
+    assert np.sum(dq * f64(q)) == pytest.approx(np.sum(dk * f64(K)), rel=1e-10, abs=1e-10)
+    assert np.max(np.abs(dq)) > 0.01 and np.max(np.abs(dk)) > 0.01
