@@ -10,7 +10,8 @@ left the 126 MB L2 before the layer comes back; each layer walks the 256 decode 
 
 Second workload (``prefill`` object): a 32K-token prefill of one layer (kernel pooling, scoring + top-k,
 sparse attention with the first 8192 rows dense), 32 / 2 heads, d 128, Q/K/V ~ N(0,1) plus per-block
-offsets N(0, 0.3^2).
+offsets N(0, 0.3^2).  Third (``backward`` object): the gradients dq, dk, dv of that prefill's sparse
+attention for its selection, with a seeded N(0,1) dout.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
@@ -429,6 +430,40 @@ class PrefillBench:
         self.b.infllmv2_sparse_attn_prefill(self.q, self.k, self.v, None, self.lens, self.T, self.idx, self.cnt,
                                             self.p, self.out)
 
+    def backward_setup(self):
+        """The forward's out / lse for the current selection and a seeded dout, for the gradient pass."""
+        torch, b = self.torch, self.b
+        dev = torch.device("cuda")
+        self.lse = torch.empty((1, self.T, HQ), dtype=torch.float32, device=dev)
+        self.pool()
+        self.score()
+        b.infllmv2_sparse_attn_prefill(self.q, self.k, self.v, None, self.lens, self.T, self.idx, self.cnt, self.p,
+                                       self.out, self.lse)
+        gen = torch.Generator(device=dev).manual_seed(1103)
+        self.dout = torch.randn((1, self.T, HQ, D), generator=gen, device=dev).to(torch.bfloat16)
+        self.dq = torch.empty((1, self.T, HQ, D), dtype=torch.float32, device=dev)
+        self.dk = torch.empty((1, self.T, HKV, D), dtype=torch.float32, device=dev)
+        self.dv = torch.empty((1, self.T, HKV, D), dtype=torch.float32, device=dev)
+        self.bws = b.backward_workspace(self.p, 1, self.T, self.T, HQ, HKV, D)
+
+    def backward(self):
+        self.b.infllmv2_sparse_attn_backward(self.q, self.k, self.v, None, self.lens, self.T, self.idx, self.cnt,
+                                             self.p, self.out, self.lse, self.dout, self.dq, self.dk, self.dv,
+                                             self.bws)
+
+    def run_backward(self, warmup, steps):
+        torch = self.torch
+        for _ in range(warmup):
+            self.backward()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(steps):
+            self.backward()
+        e1.record()
+        e1.synchronize()
+        return e0.elapsed_time(e1) / 1e3
+
     def run(self, warmup, steps):
         torch = self.torch
         fns = {"kernel_pool": self.pool, "block_score_topk": self.score, "sparse_attn_prefill": self.attend}
@@ -654,6 +689,20 @@ def run_ours(args):
                          "traffic": NCU_TRAFFIC.get(pdom)},
         }
         line["gpu_launches"] += args.prefill_steps * 3  # kernel pool, scoring + top-k, attention
+        if not args.no_backward:
+            pb.backward_setup()
+            bt = barrier_max(pb.run_backward(3, args.prefill_steps), ws)
+            bflops = 2.5 * (af + df)  # 10 d flops per attended (row, key): S, dP, dV, dQ, dK
+            bach = bflops / (bt / args.prefill_steps) / 1e12
+            line["backward"] = {
+                "workload": "prefill_32k gradients (dq, dk, dv) for the forward's selection",
+                "value": whole_job_rate(pb.T * args.prefill_steps, ws, bt), "unit": UNIT,
+                "ms_per_step": bt / args.prefill_steps * 1e3, "steps": args.prefill_steps,
+                "algorithmic_tflop_per_step": bflops / 1e12, "achieved_tflops": bach,
+                "tc_frac_of_" + peak_kind: bach / peaks["bf16_tflops"],
+                "kernels": "zero, prep, scan, fill (block lists), dq (mma.sync), dkdv (mma.sync, fp32 atomics)",
+            }
+            line["gpu_launches"] += args.prefill_steps * 6
         del pb
         torch.cuda.empty_cache()
 
@@ -722,6 +771,7 @@ def main():
                     help="decode step as block_score_topk + sparse_attn_decode, or the one-launch sparse_decode_step")
     ap.add_argument("--prefill-steps", type=int, default=3)
     ap.add_argument("--no-prefill", action="store_true")
+    ap.add_argument("--no-backward", action="store_true", help="skip the prefill gradient pass")
     ap.add_argument("--no-decode", action="store_true", help="prefill only (for profiling its kernels)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=15.0)

@@ -240,6 +240,31 @@ int infllmv2_dense_attn_decode(const void* q, int batch, int hq, int hkv, int he
                                float* lse, void* ws, size_t ws_bytes, infllmv2_stream_t stream);
 
 /*
+ * Backward of step 3a for a fixed selection (training: MiniCPM4 technical details, "Model architecture:
+ * InfLLM v2", item 3 -- the operators serve training as well as inference; the pages give no formula, so
+ * this is the derivative of 3a's definition).  The selection is piecewise constant in q and K, so no
+ * gradient flows through the block scores or the semantic kernels.  With the forward's key sets (3a) and
+ * p_i = exp(scale q.k_i - lse), for a loss L with dout = dL/dout:
+ *   dv_i += p_i dout;   ds_i = p_i (dout . v_i - dout . out);   dq = scale sum_i ds_i k_i;   dk_i += scale ds_i q
+ * summed over every (query, head) that reads key i (GQA: the heads of a group add into one KV head).
+ *   q, k, v, q_ctx, ctx_lens, max_ctx, idx, cnt, params: exactly as given to infllmv2_sparse_attn_prefill.
+ *               idx and cnt both NULL: every query attends to all of [0, n) (the dense attention's backward).
+ *   out        [B, T, Hq, d] bf16: the forward's output;  lse [B, T, Hq] fp32: the forward's lse (required)
+ *   dout       [B, T, Hq, d] bf16
+ *   dq         [B, T, Hq, d] fp32, overwritten
+ *   dk, dv     [B, Lcap, Hkv, d] fp32, overwritten: keys no query reads get 0
+ *   ws         >= infllmv2_backward_workspace_size(params, B, T, max_ctx, Hq, Hkv, d) bytes, 256-byte aligned
+ * dk / dv are sums of fp32 atomics: equal up to rounding order between runs.
+ */
+size_t infllmv2_backward_workspace_size(const infllmv2_params* params, int batch, int max_q, int max_ctx, int hq,
+                                        int hkv, int head_dim);
+int infllmv2_sparse_attn_backward(const void* q, int batch, int num_q, int hq, int hkv, int head_dim, const void* k,
+                                  const void* v, int lcap, const int32_t* q_ctx, const int32_t* ctx_lens, int max_ctx,
+                                  const int32_t* idx, const int32_t* cnt, const infllmv2_params* params,
+                                  const void* out, const float* lse, const void* dout, float* dq, float* dk,
+                                  float* dv, void* ws, size_t ws_bytes, infllmv2_stream_t stream);
+
+/*
  * The draft model's sliding-window attention (MiniCPM4 technical details, section "speculative sampling,
  * quantisation and long text", long-context bullet: the draft model attends with a sliding window; the
  * pages give no window size).  One query per sequence attends to its last `window` keys:

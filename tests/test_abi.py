@@ -128,3 +128,29 @@ def test_attention_entry_points_reject_bad_arguments(lib):
     assert lib.infllmv2_kv_append(A16 + 2, A16, 4, 2, 128, A4, A16, A16, 4096, None) == INVALID
     assert lib.infllmv2_kv_append(A16, A16, 4, 2, 128, A4, None, A16, 4096, None) == INVALID
     assert lib.infllmv2_kv_append(A16, A16, 4, 2, 128, A4, A16, A16, 0, None) == INVALID
+
+
+def test_backward_rejects_bad_arguments(lib):
+    p = binding.Params(topk=64, dense_len=8192)
+    cp = p.c()
+    need = binding.infllmv2_backward_workspace_size(p, 1, 4096, 4096, 32, 2, 128)
+    assert need > 0 and need % 256 == 0
+    assert binding.infllmv2_backward_workspace_size(p, 1, 4096, 4096, 32, 2, 96) == 0
+
+    def call(**kw):
+        a = dict(q=A16, k=A16, v=A16, lcap=4096, q_ctx=None, ctx=A4, max_ctx=4096, idx=A4, cnt=A4, out=A16,
+                 lse=A4, dout=A16, dq=A16, dk=A16, dv=A16, ws=WS, wsb=need)
+        a.update(kw)
+        return lib.infllmv2_sparse_attn_backward(a["q"], 1, 4096, 32, 2, 128, a["k"], a["v"], a["lcap"], a["q_ctx"],
+                                                 a["ctx"], a["max_ctx"], a["idx"], a["cnt"], ctypes.byref(cp),
+                                                 a["out"], a["lse"], a["dout"], a["dq"], a["dk"], a["dv"], a["ws"],
+                                                 a["wsb"], None)
+
+    assert call(lse=None) == INVALID                 # the forward's lse is required
+    assert call(dout=A16 + 2) == INVALID             # misaligned gradient input
+    assert call(dk=None) == INVALID
+    assert call(idx=None) == INVALID                 # idx without cnt (or the reverse)
+    assert call(ctx=None) == INVALID                 # neither q_ctx nor ctx_lens
+    assert call(max_ctx=5000) == INVALID             # max_ctx past the cache
+    assert call(wsb=need - 256) == WORKSPACE
+    assert call(ws=WS + 16) == WORKSPACE

@@ -81,6 +81,9 @@ _SIGS = {
                                           _P, _P, _SZ, _P], _I),
     "infllmv2_dense_attn_prefill": ([_P, _I, _I, _I, _I, _I, _P, _P, _I, _P, _P, _I, _F, _P, _P, _P, _SZ, _P], _I),
     "infllmv2_dense_attn_decode": ([_P, _I, _I, _I, _I, _P, _P, _I, _P, _I, _F, _P, _P, _P, _SZ, _P], _I),
+    "infllmv2_backward_workspace_size": ([_PP, _I, _I, _I, _I, _I, _I], _SZ),
+    "infllmv2_sparse_attn_backward": ([_P, _I, _I, _I, _I, _I, _P, _P, _I, _P, _P, _I, _P, _P, _PP, _P, _P, _P,
+                                       _P, _P, _P, _P, _SZ, _P], _I),
     "infllmv2_window_attn_decode": ([_P, _I, _I, _I, _I, _P, _P, _I, _P, _I, _I, _F, _P, _P, _P, _SZ, _P], _I),
 }
 
@@ -313,6 +316,42 @@ def infllmv2_window_attn_decode(q, k, v, ctx_lens, max_ctx, window, softmax_scal
                                             _ptr(ws), 0 if ws is None else ws.numel() * ws.element_size(),
                                             _stream(stream))
     _check("infllmv2_window_attn_decode", st)
+
+
+def infllmv2_backward_workspace_size(params: Params, batch, max_q, max_ctx, hq, hkv, head_dim) -> int:
+    cp = params.c()
+    return int(load().infllmv2_backward_workspace_size(ctypes.byref(cp), batch, max_q, max_ctx, hq, hkv, head_dim))
+
+
+def infllmv2_sparse_attn_backward(q, k, v, q_ctx, ctx_lens, max_ctx, idx, cnt, params: Params, out, lse, dout,
+                                  dq, dk, dv, ws, stream=None):
+    """Gradients (dq, dk, dv; fp32, overwritten) of the sparse attention for a fixed selection; idx and cnt
+    both None means dense attention over [0, n)."""
+    for t, n in ((q, "q"), (k, "k"), (v, "v"), (out, "out"), (dout, "dout")):
+        _need(t, torch.bfloat16, n, 4)
+    for t, n in ((dq, "dq"), (dk, "dk"), (dv, "dv")):
+        _need(t, torch.float32, n, 4)
+    _need(lse, torch.float32, "lse")
+    if idx is not None:
+        _need(idx, torch.int32, "idx", 4)
+        _need(cnt, torch.int32, "cnt", 3)
+    B, T, Hq, d = q.shape
+    Lcap, Hkv = k.shape[1], k.shape[2]
+    cp = params.c()
+    st = load().infllmv2_sparse_attn_backward(_ptr(q), B, T, Hq, Hkv, d, _ptr(k), _ptr(v), Lcap, _ptr(q_ctx),
+                                              _ptr(ctx_lens), int(max_ctx), _ptr(idx), _ptr(cnt), ctypes.byref(cp),
+                                              _ptr(out), _ptr(lse), _ptr(dout), _ptr(dq), _ptr(dk), _ptr(dv),
+                                              _ptr(ws), 0 if ws is None else ws.numel() * ws.element_size(),
+                                              _stream(stream))
+    _check("infllmv2_sparse_attn_backward", st)
+
+
+def backward_workspace(params: Params, batch, max_q, max_ctx, hq, hkv, head_dim, device="cuda"):
+    """Allocate (with torch) a workspace of infllmv2_backward_workspace_size bytes, 256-byte aligned."""
+    n = infllmv2_backward_workspace_size(params, batch, max_q, max_ctx, hq, hkv, head_dim)
+    if n == 0:
+        raise Infllmv2Error("infllmv2_backward_workspace_size", 1, "invalid sizes")
+    return torch.empty(math.ceil(n / 256) * 256, dtype=torch.uint8, device=device)
 
 
 def num_kernels(n: int, kernel_size: int = 32, kernel_stride: int = 16) -> int:

@@ -425,6 +425,52 @@ int infllmv2_dense_attn_prefill(const void* q, int batch, int num_q, int hq, int
     return launched(iv2::launch_attn_rows(qr, k, v, lcap, nullptr, nullptr, mc, true, out, lse, (cudaStream_t)stream));
 }
 
+size_t infllmv2_backward_workspace_size(const infllmv2_params* params, int batch, int max_q, int max_ctx, int hq,
+                                        int hkv, int head_dim)
+{
+    if (check_params(params) != INFLLMV2_OK) return 0;
+    if (check_heads(batch, max_q, hq, hkv, head_dim) != INFLLMV2_OK) return 0;
+    if (check_ctx(max_ctx, -1) != INFLLMV2_OK) return 0;
+    const int kmax = params->topk + params->init_blocks + params->local_blocks;
+    // sized for the dense case too (idx == NULL), which bounds every sparse one
+    const size_t sparse = iv2::attn_bwd_ws_bytes(batch, max_q, hq, hkv, max_ctx, kmax, params->dense_len, false);
+    const size_t dense = iv2::attn_bwd_ws_bytes(batch, max_q, hq, hkv, max_ctx, kmax, params->dense_len, true);
+    return sparse > dense ? sparse : dense;
+}
+
+int infllmv2_sparse_attn_backward(const void* q, int batch, int num_q, int hq, int hkv, int head_dim, const void* k,
+                                  const void* v, int lcap, const int32_t* q_ctx, const int32_t* ctx_lens, int max_ctx,
+                                  const int32_t* idx, const int32_t* cnt, const infllmv2_params* params,
+                                  const void* out, const float* lse, const void* dout, float* dq, float* dk,
+                                  float* dv, void* ws, size_t ws_bytes, infllmv2_stream_t stream)
+{
+    IV2_TRY(check_params(params));
+    IV2_TRY(check_heads(batch, num_q, hq, hkv, head_dim));
+    IV2_TRY(check_ptr16(q));
+    IV2_TRY(check_ptr16(k));
+    IV2_TRY(check_ptr16(v));
+    IV2_TRY(check_ptr16(out));
+    IV2_TRY(check_ptr16(dout));
+    IV2_TRY(check_ptr16(dq));
+    IV2_TRY(check_ptr16(dk));
+    IV2_TRY(check_ptr16(dv));
+    IV2_TRY(check_ptr4(lse));
+    if ((idx == nullptr) != (cnt == nullptr)) return INFLLMV2_ERR_INVALID_ARG;
+    IV2_TRY(check_opt4(idx));
+    IV2_TRY(check_opt4(cnt));
+    IV2_TRY(check_opt4(q_ctx));
+    IV2_TRY(check_opt4(ctx_lens));
+    if (!q_ctx && !ctx_lens) return INFLLMV2_ERR_INVALID_ARG;
+    IV2_TRY(check_ctx(max_ctx, lcap));
+    const bool dense_all = idx == nullptr;
+    const MethodConsts mc = consts_of(params, head_dim);
+    IV2_TRY(check_ws(ws, ws_bytes,
+                     iv2::attn_bwd_ws_bytes(batch, num_q, hq, hkv, max_ctx, mc.kmax, mc.dense_len, dense_all)));
+    const QueryRows qr = rows_of(q, batch, num_q, hq, hkv, head_dim, q_ctx, ctx_lens, 0, max_ctx);
+    return launched(iv2::launch_attn_backward(qr, k, v, lcap, idx, cnt, mc, dense_all, out, lse, dout, dq, dk, dv, ws,
+                                              (cudaStream_t)stream));
+}
+
 int infllmv2_dense_attn_decode(const void* q, int batch, int hq, int hkv, int head_dim, const void* k, const void* v,
                                int lcap, const int32_t* ctx_lens, int max_ctx, float softmax_scale, void* out,
                                float* lse, void* ws, size_t ws_bytes, infllmv2_stream_t stream)

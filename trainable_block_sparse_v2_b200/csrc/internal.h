@@ -146,4 +146,11 @@ cudaError_t launch_attn_split(const QueryRows& qr, const void* k, const void* v,
                               const void* v_draft, const uint32_t* tree_mask, void* out, float* lse, void* ws,
                               cudaStream_t s);
 
+// gradients of the attention for a fixed selection (prefill layout): workspace bytes, and the launches
+size_t attn_bwd_ws_bytes(int B, int T, int Hq, int Hkv, int max_ctx, int kmax, int dense_len, bool dense_all);
+cudaError_t launch_attn_backward(const QueryRows& qr, const void* k, const void* v, int Lcap, const int32_t* idx,
+                                 const int32_t* cnt, const MethodConsts& mc, bool dense_all, const void* out,
+                                 const float* lse, const void* dout, float* dq, float* dk, float* dv, void* ws,
+                                 cudaStream_t s);
+
 }  // namespace iv2
