@@ -322,14 +322,15 @@ FUSED_LENS_14 = [20000, 8192, 8193, 30, 4500, 65, 70000]
 FUSED_LENS_26 = [20000, 8192, 8193, 30, 4500, 65, 70000, 9000, 12345, 64 * 130 + 1, 40000, 8300, 98304]
 
 
-@pytest.mark.parametrize("G,d,lens,membership", [(16, 128, FUSED_LENS_14, 0), (2, 64, FUSED_LENS_14, 0),
-                                                 (8, 128, FUSED_LENS_14, 1), (16, 128, FUSED_LENS_26, 0),
-                                                 (4, 64, FUSED_LENS_26, 1)])
-def test_fused_decode_step(oracle, G, d, lens, membership):
+@pytest.mark.parametrize("G,d,lens,membership,topk", [(16, 128, FUSED_LENS_14, 0, 16), (2, 64, FUSED_LENS_14, 0, 16),
+                                                      (8, 128, FUSED_LENS_14, 1, 16), (16, 128, FUSED_LENS_26, 0, 16),
+                                                      (4, 64, FUSED_LENS_26, 1, 16), (16, 128, FUSED_LENS_14, 0, 1200)])
+def test_fused_decode_step(oracle, G, d, lens, membership, topk):
     """infllmv2_sparse_decode_step (scoring + top-k + attention in one cluster kernel) against the oracle:
     ragged lengths, a row at the dense threshold and one past it, rows shorter than one kernel window,
-    both block-membership rules, 16-CTA and 8-CTA clusters."""
-    w = decode_case(lens, 2 * G, 2, d, topk=16, dense_len=8192, seed=650 + G + len(lens), n_needles=8,
+    both block-membership rules, 16-CTA and 8-CTA clusters; k = 1200 gives block lists of over a thousand
+    entries (about 70 per CTA) next to rows that select every block."""
+    w = decode_case(lens, 2 * G, 2, d, topk=topk, dense_len=8192, seed=650 + G + len(lens), n_needles=8,
                     membership=membership)
     B = len(lens)
     nk_cap = oracle.num_kernels(max(lens))

@@ -389,13 +389,16 @@ IV2_DEV int cta_select_topk(const float* S, int c, int init, int local, int topk
     }
     const bool all = ncand <= topk;
     const float bscale = kmx > kmn ? (float)(kBuckets - 1) / (float)(kmx - kmn) : 0.f;
+    int bk[E];  // bucket of each key (unused for keys that are 0)
+#pragma unroll
+    for (int e = 0; e < E; ++e) bk[e] = bucket_of(key[e], kmn, bscale);
     int bstar = kBuckets;
     uint32_t tkey = 0u;
     int tidx = 0;
     if (!all) {
 #pragma unroll
         for (int e = 0; e < E; ++e)
-            if (key[e] != 0u) atomicAdd(&sm.hist[bucket_of(key[e], kmn, bscale)], 1);
+            if (key[e] != 0u) atomicAdd(&sm.hist[bk[e]], 1);
         __syncthreads();
         // descending suffix scan over buckets: thread t owns buckets [kBuckets - (t+1)*BPT, kBuckets - t*BPT)
         constexpr int BPT = kBuckets / NT;
@@ -437,7 +440,7 @@ IV2_DEV int cta_select_topk(const float* S, int c, int init, int local, int topk
         // stage the members of B*
 #pragma unroll
         for (int e = 0; e < E; ++e) {
-            if (key[e] != 0u && bucket_of(key[e], kmn, bscale) == bstar) {
+            if (key[e] != 0u && bk[e] == bstar) {
                 const int slot = atomicAdd(&sm.nmem, 1);
                 if (slot < kMaxMembers) {
                     sm.mkey[slot] = key[e];
@@ -455,13 +458,13 @@ IV2_DEV int cta_select_topk(const float* S, int c, int init, int local, int topk
                 int ge = 0;
 #pragma unroll
                 for (int e = 0; e < E; ++e)
-                    ge += key[e] != 0u && bucket_of(key[e], kmn, bscale) == bstar && key[e] >= probe;
+                    ge += key[e] != 0u && bk[e] == bstar && key[e] >= probe;
                 if (cta_count<NT>(ge, sm.red, parity) >= rem) t = probe;
                 parity ^= 1;
             }
             int gt = 0;
 #pragma unroll
-            for (int e = 0; e < E; ++e) gt += key[e] != 0u && bucket_of(key[e], kmn, bscale) == bstar && key[e] > t;
+            for (int e = 0; e < E; ++e) gt += key[e] != 0u && bk[e] == bstar && key[e] > t;
             gt = cta_count<NT>(gt, sm.red, parity);
             parity ^= 1;
             const int need = rem - gt;
@@ -500,25 +503,17 @@ IV2_DEV int cta_select_topk(const float* S, int c, int init, int local, int topk
         tkey = sm.thr_key;
         tidx = sm.thr_idx;
     }
-    // emit ascending
+    // emit ascending (branch-free: a key is 0 for blocks past nb, forced blocks and blocks with no kernel)
     bool chosen[E];
     int nchosen = 0;
 #pragma unroll
     for (int e = 0; e < E; ++e) {
         const int b = b0 + e;
-        bool ch = false;
-        if (b < nb) {
-            if (is_forced(b, c, init, local)) ch = true;
-            else if (key[e] != 0u) {
-                if (all) ch = true;
-                else {
-                    const int bk = bucket_of(key[e], kmn, bscale);
-                    ch = bk > bstar || (bk == bstar && (key[e] > tkey || (key[e] == tkey && b <= tidx)));
-                }
-            }
-        }
-        chosen[e] = ch;
-        nchosen += ch;
+        const bool forced = b < nb && is_forced(b, c, init, local);
+        const bool above =
+            all || bk[e] > bstar || (bk[e] == bstar && (key[e] > tkey || (key[e] == tkey && b <= tidx)));
+        chosen[e] = forced || (key[e] != 0u && above);
+        nchosen += chosen[e];
     }
     int total;
     int pos = cta_exclusive_scan<NT>(nchosen, sm.red, &total);
