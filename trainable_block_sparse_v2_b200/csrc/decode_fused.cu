@@ -66,8 +66,10 @@ struct FLayout {
     static constexpr int kSelWs = kFMaxCL * kFMaxBpc * 4 + 16;  // bucket-select scratch (S may overhang 3)
     static constexpr int kSelList = round_up(kSelWs + (int)sizeof(CtaSelectSmem), 16);  // the whole list
     static constexpr int kSelEnd = kSelList + kFMaxKmax * 4;
-    static constexpr int kWo = 0;                              // [warp][16][D] scaled warp outputs
-    static constexpr int kWml = kFWarps * 16 * D * 4;          // [warp][16] m, then [warp][16] l
+    static constexpr int kWo = 0;                              // [warp][16][kWoPitch] scaled warp outputs
+    static constexpr int kWoPitch = D + 8;                     // floats; the 8 head rows a warp stores at once
+                                                               // start 8 banks apart (conflict-free float2)
+    static constexpr int kWml = kFWarps * 16 * kWoPitch * 4;   // [warp][16] m, then [warp][16] l
     static constexpr int kWf = kWml + 2 * kFWarps * 16 * 4;    // [warp][16] factors, [16] M, [16] L
     static constexpr int kMergeEnd = kWf + (kFWarps + 2) * 16 * 4;
     static constexpr int kRegionA = round_up(cmax(cmax(kScanRing, kAttnRing), cmax(kSelEnd, kMergeEnd)), 1024);
@@ -490,7 +492,7 @@ decode_fused_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_con
     }
     finalize_rows<D>(st);
     // the eight warp states -> this CTA's partial: factors 2^(m_w - M) once per (warp, head), then sums
-    float* wo = reinterpret_cast<float*>(smem + L::kWo);  // [warp][16][D]
+    float* wo = reinterpret_cast<float*>(smem + L::kWo);  // [warp][16][kWoPitch]
     float* wm = reinterpret_cast<float*>(smem + L::kWml);  // [warp][16]
     float* wl = wm + kFWarps * 16;                         // [warp][16]
     float* wf = reinterpret_cast<float*>(smem + L::kWf);   // [warp][16]
@@ -526,7 +528,7 @@ decode_fused_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_con
         const float f = wf[warp * 16 + h];
 #pragma unroll
         for (int nt = 0; nt < D / 8; ++nt)
-            *reinterpret_cast<float2*>(&wo[(warp * 16 + h) * D + nt * 8 + 2 * tq]) =
+            *reinterpret_cast<float2*>(&wo[(warp * 16 + h) * L::kWoPitch + nt * 8 + 2 * tq]) =
                 make_float2(st.o[nt][2 * r] * f, st.o[nt][2 * r + 1] * f);
     }
     __syncthreads();
@@ -535,7 +537,7 @@ decode_fused_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_con
         float4 o = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
         for (int w = 0; w < kFWarps; ++w) {
-            const float4 v = *reinterpret_cast<const float4*>(&wo[(w * 16 + h) * D + d4]);
+            const float4 v = *reinterpret_cast<const float4*>(&wo[(w * 16 + h) * L::kWoPitch + d4]);
             o.x += v.x;
             o.y += v.y;
             o.z += v.z;
