@@ -43,7 +43,7 @@ HQ, HKV, D = 32, 2, 128
 # as they stand (profiles/decode_128k_launches.md, profiles/decode_fused_128k.md); None where the kernel
 # changed after its capture
 NCU_TRAFFIC = {
-    "sparse_decode_step": None,                         # decode_fused_kernel changed after its capture
+    "sparse_decode_step": 31_304_192,                   # decode_fused_kernel: 31.30 MB read, ~0 written
     "sparse_attn_decode": 17_430_000 + 1_150_000,       # attn_split_kernel + attn_merge_kernel
     "block_score_topk": 13_680_000 + 960_000,           # score_scan_kernel + score_select_kernel
     "sparse_attn_prefill": 322_021_888 + 222_341_376,   # attn_tc_kernel (profiles/prefill_32k.md)
