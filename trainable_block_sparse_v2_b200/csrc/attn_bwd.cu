@@ -33,7 +33,8 @@ namespace iv2 {
 
 namespace {
 
-constexpr int kBwdRowWarps = 4;   // rows per CTA of the prep, fill and dq kernels
+constexpr int kBwdRowWarps = 4;   // rows per CTA of the prep and fill kernels
+constexpr int kDqWarps = 2;       // rows per CTA of the dq kernel: 64 KB of staging, three CTAs per SM
 constexpr int kDkvThreads = 128;  // 4 warps x 16 keys of one 64-key block
 constexpr int kItemTokens = 256;  // tokens per dkdv work item
 constexpr int kScanThreads = 1024;
@@ -257,7 +258,7 @@ template <int D>
 struct DqSmem {
     static constexpr int kHalf = 32 * D * 2;            // K or V rows of one 32-key half block
     static constexpr int kWarpBytes = 4 * kHalf;        // [2 buffers] x (K | V)
-    static constexpr int kBytes = kBwdRowWarps * kWarpBytes;
+    static constexpr int kBytes = kDqWarps * kWarpBytes;
 };
 
 // stage rows [0, 32) of a half block: row r from src + r * row_stride when r < nvalid, else zeros
@@ -291,7 +292,7 @@ IV2_DEV int next_half(const RowCtx& r, int& kpos, int& half)
 }
 
 template <int D>
-__global__ void __launch_bounds__(kBwdRowWarps * 32) bwd_dq_kernel(QueryRows qr, const __nv_bfloat16* __restrict__ k,
+__global__ void __launch_bounds__(kDqWarps * 32) bwd_dq_kernel(QueryRows qr, const __nv_bfloat16* __restrict__ k,
                                                                    const __nv_bfloat16* __restrict__ v, int Lcap,
                                                                    const int32_t* __restrict__ idx,
                                                                    const int32_t* __restrict__ cnt, MethodConsts mc,
@@ -305,7 +306,7 @@ __global__ void __launch_bounds__(kBwdRowWarps * 32) bwd_dq_kernel(QueryRows qr,
     pdl_wait();
     extern __shared__ __align__(128) unsigned char smem[];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, gq = lane >> 2, tq = lane & 3;
-    const long row = (long)blockIdx.x * kBwdRowWarps + warp;
+    const long row = (long)blockIdx.x * kDqWarps + warp;
     if (row >= (long)qr.B * qr.T * qr.Hkv) return;
     unsigned char* wsm = smem + warp * L::kWarpBytes;  // buffer u: K at u * 2 * kHalf, V right after
     const RowCtx r = row_ctx(qr, row, idx, cnt, mc, dense_all);
@@ -636,7 +637,8 @@ cudaError_t bwd_impl(const QueryRows& qr, const void* k, const void* v, int Lcap
     const size_t dq_smem = (size_t)DqSmem<D>::kBytes;
     e = ensure_smem(bwd_dq_kernel<D>, dq_smem);
     if (e != cudaSuccess) return e;
-    e = launch_pdl(bwd_dq_kernel<D>, dim3(row_grid), dim3(kBwdRowWarps * 32), dq_smem, s, qr,
+    const unsigned dq_grid = (unsigned)((rows + kDqWarps - 1) / kDqWarps);
+    e = launch_pdl(bwd_dq_kernel<D>, dim3(dq_grid), dim3(kDqWarps * 32), dq_smem, s, qr,
                    static_cast<const __nv_bfloat16*>(k), static_cast<const __nv_bfloat16*>(v), Lcap, idx, cnt, mc,
                    dense_flag, lse, static_cast<const float*>(dsum), static_cast<const __nv_bfloat16*>(dout), dq);
     if (e != cudaSuccess) return e;
