@@ -332,10 +332,13 @@ class DecodeBench:
         e1.synchronize()
         return e0.elapsed_time(e1) / 1e3 / (reps * steps)
 
-    def e2e(self, warmup, steps):
+    def e2e(self, warmup, steps, graphs=True):
         """Same step through the C ABI with host buffers: every step copies that step's query and the new key
         and value rows from pinned host memory to the device in one copy, appends the rows to the caches
-        (infllmv2_kv_append), pools, runs the step and reads the attention output back."""
+        (infllmv2_kv_append), pools, runs the step and reads the attention output back.  graphs: the calls of
+        every layer at one decode position (copies included) are captured once as a CUDA graph and replayed
+        per position, the way a serving loop issues a decode step; otherwise each call is issued eagerly from
+        Python."""
         torch = self.torch
         B = self.B
         nq, nkv = B * HQ * D, B * HKV * D
@@ -377,13 +380,31 @@ class DecodeBench:
         for s in range(warmup):
             one(s)
         torch.cuda.synchronize()
+        if graphs:
+            # whole positions only: warm-up and timed steps start on a position boundary
+            lo = (warmup + self.NL - 1) // self.NL * self.NL
+            steps = steps // self.NL * self.NL
+            plan = []
+            for s0 in range(lo, lo + steps, self.NL):
+                g = torch.cuda.CUDAGraph()
+                with torch.cuda.graph(g):
+                    for s in range(s0, s0 + self.NL):
+                        one(s)
+                plan.append(g)
+            for g in plan[:2]:
+                g.replay()
+            torch.cuda.synchronize()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record()
-        for s in range(warmup, warmup + steps):
-            one(s)
+        if graphs:
+            for g in plan:
+                g.replay()
+        else:
+            for s in range(warmup, warmup + steps):
+                one(s)
         e1.record()
         e1.synchronize()
-        return e0.elapsed_time(e1) / 1e3, h2d, d2h
+        return e0.elapsed_time(e1) / 1e3, h2d, d2h, steps
 
 
 # ------------------------------------------------------------------------------------------------
@@ -630,7 +651,9 @@ def run_ours(args):
         t_win = db.window_time(win, min(args.steps, 256))
         win_bytes = len(LENS_128K) * HKV * win * D * 2 * 2
         e2e_steps = min(args.steps, 512)
-        e2e_t, h2d, d2h = db.e2e(8, e2e_steps) if args.e2e else (float("nan"), 0, 0)
+        e2e_t, h2d, d2h, e2e_steps = db.e2e(8, e2e_steps) if args.e2e else (float("nan"), 0, 0, e2e_steps)
+        e2e_eager_t, _, _, e2e_eager_steps = db.e2e(8, e2e_steps, graphs=False) if args.e2e else \
+            (float("nan"), 0, 0, e2e_steps)
 
         line = {
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": ws, "steps": args.steps, "warmup": args.warmup,
@@ -654,7 +677,9 @@ def run_ours(args):
                          "algorithmic_bytes": dom_bytes, "traffic": NCU_TRAFFIC.get(dom)},
             "clocks": clk.summary(),
             "e2e": {"value": len(LENS_128K) * e2e_steps / e2e_t, "unit": UNIT, "h2d_bytes_per_step": h2d,
-                    "d2h_bytes_per_step": d2h, "steps": e2e_steps},
+                    "d2h_bytes_per_step": d2h, "steps": e2e_steps,
+                    "mode": "per decode position, one CUDA graph of the 8 layers' C-ABI calls with their copies",
+                    "eager_value": len(LENS_128K) * e2e_eager_steps / e2e_eager_t},
             "gpu_launches": KERNELS_PER_STEP[args.decode_path] * args.steps,
             "window_decode": {"window": win, "value": len(LENS_128K) / t_win, "unit": UNIT, "us_per_call": t_win * 1e6,
                               "algorithmic_bytes": win_bytes, "achieved_gbs": win_bytes / t_win / 1e9,
