@@ -505,12 +505,12 @@ def test_backward_matches_central_differences(oracle):
     assert np.any(dv[0, 8:] != 0)
 
 
-def test_backward_dense_matches_torch_autograd(oracle):
+@pytest.mark.parametrize("Hq,Hkv,d", [(4, 2, 16), (16, 1, 8)])
+def test_backward_dense_matches_torch_autograd(oracle, Hq, Hkv, d):
     """Every block selected: the gradients are those of torch causal softmax attention (fp64 autograd,
     GQA by repeating K/V over the group, whose backward sums the group's heads)."""
-    rng = np.random.default_rng(51)
+    rng = np.random.default_rng(51 + Hq)
     T = L = 150
-    Hq, Hkv, d = 4, 2, 16
     q, K, V = rand_case(rng, 1, T, L, Hq, Hkv, d)
     dout = f32_to_bf16_bits(rng.standard_normal((1, T, Hq, d)).astype(np.float32))
     qc = np.arange(1, T + 1, dtype=np.int32)[None]
