@@ -135,6 +135,20 @@ def _need(t, dtype, name, ndim=None):
     return t
 
 
+def _checking() -> bool:
+    """INFLLMV2_CHECK=1: check the device-side inputs (contexts, block lists) on the host before each call
+    (checks.py); off by default, since it copies them to the host and synchronises."""
+    return os.environ.get("INFLLMV2_CHECK", "") == "1"
+
+
+def _check_rows(what, B, T, q_ctx, ctx_lens, same_ctx, lcap, max_ctx, idx=None, cnt=None, params=None):
+    from . import checks
+    ctx = checks.query_contexts(B, T, q_ctx, ctx_lens, same_ctx)
+    checks.check_contexts(ctx, lcap, int(max_ctx), what)
+    if idx is not None:
+        checks.check_block_lists(idx, cnt, ctx, params.kmax, params.dense_len, params.block_size, what)
+
+
 def _check(fn, status):
     if status != 0:
         msg = load().infllmv2_status_string(status).decode()
@@ -165,6 +179,10 @@ def infllmv2_kernel_pool(k, old_lens, new_lens, max_new_keys, params: Params, ke
     _need(old_lens, torch.int32, "old_lens")
     _need(new_lens, torch.int32, "new_lens")
     B, Lcap, Hkv, d = k.shape
+    if _checking():
+        from . import checks
+        checks.check_pool_lengths(old_lens, new_lens, Lcap, int(max_new_keys), kern.shape[2], params.kernel_size,
+                                  params.kernel_stride, "infllmv2_kernel_pool")
     cp = params.c()
     st = load().infllmv2_kernel_pool(_ptr(k), B, Lcap, Hkv, d, _ptr(old_lens), _ptr(new_lens), int(max_new_keys),
                                      ctypes.byref(cp), _ptr(kern), kern.shape[2], _stream(stream))
@@ -198,6 +216,8 @@ def infllmv2_block_score_topk(q, q_ctx, ctx_lens, max_ctx, kern, params: Params,
         _need(ctx_lens, torch.int32, "ctx_lens")
     B, T, Hq, d = q.shape
     Hkv = kern.shape[1]
+    if _checking():
+        _check_rows("infllmv2_block_score_topk", B, T, q_ctx, ctx_lens, False, int(max_ctx), max_ctx)
     cp = params.c()
     st = load().infllmv2_block_score_topk(_ptr(q), B, T, Hq, Hkv, d, _ptr(q_ctx), _ptr(ctx_lens), int(max_ctx),
                                           _ptr(kern), kern.shape[2], ctypes.byref(cp), _ptr(idx), _ptr(cnt),
@@ -216,6 +236,8 @@ def infllmv2_sparse_attn_prefill(q, k, v, q_ctx, ctx_lens, max_ctx, idx, cnt, pa
         _need(lse, torch.float32, "lse")
     B, T, Hq, d = q.shape
     Lcap, Hkv = k.shape[1], k.shape[2]
+    if _checking():
+        _check_rows("infllmv2_sparse_attn_prefill", B, T, q_ctx, ctx_lens, False, Lcap, max_ctx, idx, cnt, params)
     cp = params.c()
     st = load().infllmv2_sparse_attn_prefill(_ptr(q), B, T, Hq, Hkv, d, _ptr(k), _ptr(v), Lcap, _ptr(q_ctx),
                                              _ptr(ctx_lens), int(max_ctx), _ptr(idx), _ptr(cnt), ctypes.byref(cp),
@@ -229,6 +251,9 @@ def infllmv2_sparse_attn_decode(q, k, v, ctx_lens, max_ctx, idx, cnt, params: Pa
         _need(t, torch.bfloat16, n)
     B, Hq, d = q.shape[0], q.shape[-2], q.shape[-1]
     Lcap, Hkv = k.shape[1], k.shape[2]
+    if _checking():
+        _check_rows("infllmv2_sparse_attn_decode", B, 1, None, ctx_lens, True, Lcap, max_ctx,
+                    idx.reshape(B, 1, Hkv, -1), cnt.reshape(B, 1, Hkv), params)
     cp = params.c()
     st = load().infllmv2_sparse_attn_decode(_ptr(q), B, Hq, Hkv, d, _ptr(k), _ptr(v), Lcap, _ptr(ctx_lens),
                                             int(max_ctx), _ptr(idx), _ptr(cnt), ctypes.byref(cp), _ptr(out), _ptr(lse),
@@ -246,6 +271,8 @@ def infllmv2_sparse_decode_step(q, kern, k, v, ctx_lens, max_ctx, params: Params
     _need(cnt, torch.int32, "cnt")
     B, Hq, d = q.shape[0], q.shape[-2], q.shape[-1]
     Lcap, Hkv = k.shape[1], k.shape[2]
+    if _checking():
+        _check_rows("infllmv2_sparse_decode_step", B, 1, None, ctx_lens, True, Lcap, max_ctx)
     cp = params.c()
     st = load().infllmv2_sparse_decode_step(_ptr(q), B, Hq, Hkv, d, _ptr(kern), kern.shape[2], _ptr(k), _ptr(v), Lcap,
                                             _ptr(ctx_lens), int(max_ctx), ctypes.byref(cp), _ptr(idx), _ptr(cnt),
@@ -274,6 +301,9 @@ def infllmv2_sparse_attn_tree_verify(q, k, v, prefix_lens, max_ctx, k_draft, v_d
         _need(t, torch.bfloat16, n, 4)
     B, N, Hq, d = q.shape
     Lcap, Hkv = k.shape[1], k.shape[2]
+    if _checking():
+        _check_rows("infllmv2_sparse_attn_tree_verify", B, N, None, prefix_lens, True, Lcap, max_ctx, idx, cnt,
+                    params)
     cp = params.c()
     st = load().infllmv2_sparse_attn_tree_verify(_ptr(q), B, N, Hq, Hkv, d, _ptr(k), _ptr(v), Lcap, _ptr(prefix_lens),
                                                  int(max_ctx), _ptr(k_draft), _ptr(v_draft), _ptr(tree_mask), _ptr(idx),
@@ -288,6 +318,8 @@ def infllmv2_dense_attn_prefill(q, k, v, q_ctx, ctx_lens, max_ctx, softmax_scale
         _need(t, torch.bfloat16, n, 4)
     B, T, Hq, d = q.shape
     Lcap, Hkv = k.shape[1], k.shape[2]
+    if _checking():
+        _check_rows("infllmv2_dense_attn_prefill", B, T, q_ctx, ctx_lens, False, Lcap, max_ctx)
     st = load().infllmv2_dense_attn_prefill(_ptr(q), B, T, Hq, Hkv, d, _ptr(k), _ptr(v), Lcap, _ptr(q_ctx),
                                             _ptr(ctx_lens), int(max_ctx), float(softmax_scale), _ptr(out), _ptr(lse),
                                             _ptr(ws), 0 if ws is None else ws.numel() * ws.element_size(),
@@ -300,6 +332,8 @@ def infllmv2_dense_attn_decode(q, k, v, ctx_lens, max_ctx, softmax_scale, out, l
         _need(t, torch.bfloat16, n)
     B, Hq, d = q.shape[0], q.shape[-2], q.shape[-1]
     Lcap, Hkv = k.shape[1], k.shape[2]
+    if _checking():
+        _check_rows("infllmv2_dense_attn_decode", B, 1, None, ctx_lens, True, Lcap, max_ctx)
     st = load().infllmv2_dense_attn_decode(_ptr(q), B, Hq, Hkv, d, _ptr(k), _ptr(v), Lcap, _ptr(ctx_lens), int(max_ctx),
                                            float(softmax_scale), _ptr(out), _ptr(lse), _ptr(ws),
                                            0 if ws is None else ws.numel() * ws.element_size(), _stream(stream))
@@ -311,6 +345,8 @@ def infllmv2_window_attn_decode(q, k, v, ctx_lens, max_ctx, window, softmax_scal
         _need(t, torch.bfloat16, n)
     B, Hq, d = q.shape[0], q.shape[-2], q.shape[-1]
     Lcap, Hkv = k.shape[1], k.shape[2]
+    if _checking():
+        _check_rows("infllmv2_window_attn_decode", B, 1, None, ctx_lens, True, Lcap, max_ctx)
     st = load().infllmv2_window_attn_decode(_ptr(q), B, Hq, Hkv, d, _ptr(k), _ptr(v), Lcap, _ptr(ctx_lens),
                                             int(max_ctx), int(window), float(softmax_scale), _ptr(out), _ptr(lse),
                                             _ptr(ws), 0 if ws is None else ws.numel() * ws.element_size(),
@@ -337,6 +373,8 @@ def infllmv2_sparse_attn_backward(q, k, v, q_ctx, ctx_lens, max_ctx, idx, cnt, p
         _need(cnt, torch.int32, "cnt", 3)
     B, T, Hq, d = q.shape
     Lcap, Hkv = k.shape[1], k.shape[2]
+    if _checking():
+        _check_rows("infllmv2_sparse_attn_backward", B, T, q_ctx, ctx_lens, False, Lcap, max_ctx, idx, cnt, params)
     cp = params.c()
     st = load().infllmv2_sparse_attn_backward(_ptr(q), B, T, Hq, Hkv, d, _ptr(k), _ptr(v), Lcap, _ptr(q_ctx),
                                               _ptr(ctx_lens), int(max_ctx), _ptr(idx), _ptr(cnt), ctypes.byref(cp),

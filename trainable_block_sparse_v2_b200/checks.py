@@ -1,0 +1,93 @@
+"""Host-side checks of the device-side inputs of the C-ABI calls, for debugging.
+
+The library validates every size and pointer on the host before it launches anything, but it trusts the
+values that live in device memory: the per-query contexts (``q_ctx`` or ``ctx_lens``) and the block lists
+(``idx`` / ``cnt``).  The kernels skip a block id that is negative or lies past the query's context, but a
+context past ``max_ctx`` or the cache, or a list that repeats a block, gives results that are not the
+method's (a repeated block counts its keys twice).  With ``INFLLMV2_CHECK=1`` in the environment the binding
+copies those inputs to the host before every call and checks them here; a violation raises
+``InputCheckError`` naming the first offending row.  The checks synchronise with the device, so they are a
+debugging aid, not part of the timed path.
+"""
+from __future__ import annotations
+
+import numpy as np
+
+
+class InputCheckError(ValueError):
+    pass
+
+
+def _np(a):
+    if a is None:
+        return None
+    if hasattr(a, "detach"):  # torch tensor (any device)
+        return a.detach().cpu().numpy()
+    return np.asarray(a)
+
+
+def query_contexts(B: int, T: int, q_ctx=None, ctx_lens=None, same_ctx: bool = False) -> np.ndarray:
+    """Context length n of every query [B, T]: q_ctx when given; otherwise ctx_lens[b] for every query
+    (tree drafts, decode) when same_ctx, else the causal tail n = ctx_lens[b] - T + t + 1."""
+    if q_ctx is not None:
+        return _np(q_ctx).reshape(B, T).astype(np.int64)
+    if ctx_lens is None:
+        raise InputCheckError("neither q_ctx nor ctx_lens given")
+    lens = _np(ctx_lens).reshape(B).astype(np.int64)
+    if same_ctx:
+        return np.repeat(lens[:, None], T, axis=1)
+    return lens[:, None] - T + np.arange(T)[None, :] + 1
+
+
+def check_contexts(ctx: np.ndarray, lcap: int, max_ctx: int, what: str = "") -> None:
+    """1 <= n <= max_ctx <= lcap for every query."""
+    if max_ctx > lcap:
+        raise InputCheckError(f"{what}: max_ctx {max_ctx} > cache length {lcap}")
+    bad = np.argwhere((ctx < 1) | (ctx > max_ctx))
+    if bad.size:
+        pos = tuple(int(i) for i in bad[0])
+        raise InputCheckError(f"{what}: query {pos} has context {int(ctx[pos])}, outside [1, {max_ctx}]")
+
+
+def check_block_lists(idx, cnt, ctx: np.ndarray, kmax: int, dense_len: int, block: int = 64,
+                      what: str = "") -> None:
+    """Every sparse query's list (n > dense_len): 0 <= cnt <= kmax, and its first cnt ids ascending,
+    unique, >= 0 and starting before the context (block * id < n).  Dense queries' lists are not read."""
+    idx = _np(idx)
+    cnt = _np(cnt)
+    B, T, Hkv, km = idx.shape
+    if km != kmax:
+        raise InputCheckError(f"{what}: idx rows hold {km} entries, kmax is {kmax}")
+    if cnt.shape != (B, T, Hkv):
+        raise InputCheckError(f"{what}: cnt has shape {cnt.shape}, expected {(B, T, Hkv)}")
+    for b in range(B):
+        for t in range(T):
+            n = int(ctx[b, t])
+            if n <= dense_len:
+                continue
+            for g in range(Hkv):
+                c = int(cnt[b, t, g])
+                if c < 0 or c > kmax:
+                    raise InputCheckError(f"{what}: row {(b, t, g)} has cnt {c}, outside [0, {kmax}]")
+                ids = idx[b, t, g, :c].astype(np.int64)
+                if c and (ids[0] < 0 or ids[-1] * block >= n):
+                    raise InputCheckError(f"{what}: row {(b, t, g)} has a block id outside [0, {(n - 1) // block}]: "
+                                          f"{ids.tolist()}")
+                if c > 1 and np.any(np.diff(ids) <= 0):
+                    raise InputCheckError(f"{what}: row {(b, t, g)} block ids are not ascending and unique: "
+                                          f"{ids.tolist()}")
+
+
+def check_pool_lengths(old_lens, new_lens, lcap: int, max_new_keys: int, nk_cap: int, kernel_size: int = 32,
+                       kernel_stride: int = 16, what: str = "") -> None:
+    """0 <= old <= new <= lcap, new - old <= max_new_keys, and the kernels of new keys fit in nk_cap."""
+    old = _np(old_lens).astype(np.int64).ravel()
+    new = _np(new_lens).astype(np.int64).ravel()
+    for b, (o, n) in enumerate(zip(old, new)):
+        if not (0 <= o <= n <= lcap):
+            raise InputCheckError(f"{what}: sequence {b} has old {o}, new {n} (cache {lcap})")
+        if n - o > max_new_keys:
+            raise InputCheckError(f"{what}: sequence {b} adds {n - o} keys, max_new_keys is {max_new_keys}")
+        nk = (n - kernel_size) // kernel_stride + 1 if n >= kernel_size else 0
+        if nk > nk_cap:
+            raise InputCheckError(f"{what}: sequence {b} needs {nk} kernels, nk_cap is {nk_cap}")
