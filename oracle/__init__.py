@@ -20,7 +20,8 @@ Functions and the steps they follow (sources: the MiniCPM4 pages):
                               the forward's definition)
   * ``dense_attention``    -- plain causal GQA attention, written separately
   * ``window_attention``   -- the draft model's sliding-window attention (same bullet as the tree drafts)
-The pages' "efficient LogSumExp estimation" is not implemented: parity unpinned (not defined there).
+The pages' "efficient LogSumExp estimation" is not defined there (parity unpinned); ``Params.lse_stride`` selects
+one reading of it (the LSE from every s-th visible kernel, times s), pinned only to its special cases.
 """
 from __future__ import annotations
 
@@ -63,6 +64,7 @@ class _Params(ctypes.Structure):
         ("dense_len", ctypes.c_int),
         ("membership", ctypes.c_int),
         ("scale", ctypes.c_double),
+        ("lse_stride", ctypes.c_int),
     ]
 
 
@@ -78,6 +80,7 @@ class Params:
     dense_len: int = 0
     membership: int = 0
     scale: float | None = None
+    lse_stride: int = 0  # 0 / 1: exact LSE; s > 1: estimated from every s-th visible kernel (times s)
 
     @property
     def kmax(self) -> int:
@@ -86,7 +89,7 @@ class Params:
     def c_struct(self, head_dim: int) -> _Params:
         s = self.scale if self.scale is not None else 1.0 / math.sqrt(head_dim)
         return _Params(self.block_size, self.kernel_size, self.kernel_stride, self.topk, self.init_blocks,
-                       self.local_blocks, self.dense_len, self.membership, float(s))
+                       self.local_blocks, self.dense_len, self.membership, float(s), int(self.lse_stride))
 
 
 def _load():

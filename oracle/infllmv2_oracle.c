@@ -49,8 +49,9 @@
  * mean, special cases that reduce to library softmax attention / average pooling, and invariants; the
  * backward (item 7) against central differences of the forward, library autograd on the dense case,
  * the one-key closed form and the sum rules of the softmax Jacobian.
- * The pages' "efficient LogSumExp estimation" is not implemented here (parity unpinned: the pages do
- * not define it).
+ * The pages' "efficient LogSumExp estimation" is not defined there (parity unpinned): params.lse_stride > 1
+ * selects one reading of it, the LSE from every s-th visible kernel times s, pinned only to its special cases
+ * (s = 1 is exact; the closed form on equal scores).
  */
 #include <math.h>
 #include <stdint.h>
@@ -114,6 +115,7 @@ typedef struct {
     int dense_len;      /* a query whose context n <= dense_len attends densely */
     int membership;     /* 0 = OVERLAP (window intersects block), 1 = CONTAINED (window inside block) */
     double scale;       /* softmax scale for both kernel scoring and attention */
+    int lse_stride;     /* 0 or 1: exact LSE; s > 1: the estimate log(s * sum over every s-th visible kernel) */
 } orc_params;
 
 /* number of complete kernel windows over the first n keys */
@@ -205,12 +207,15 @@ static void group_scores_row(const uint16_t* q, int T, int Hq, int Hkv, int d, c
             zbuf[j] = p->scale * dot;
             if (zbuf[j] > zmax) zmax = zbuf[j];
         }
-        /* LSE_h = log sum_j exp z_h(j), evaluated exactly (max-shifted) */
+        /* LSE_h = log sum_j exp z_h(j), evaluated exactly (max-shifted); with lse_stride s > 1, the estimate
+         * log(s * sum_{j = 0, s, 2s, ...} exp z_h(j)) from every s-th visible kernel (a reading of the pages'
+         * "LogSumExp estimation", which they do not define) */
         double lse = -INFINITY;
         if (nkv > 0) {
+            const long st = p->lse_stride > 1 ? p->lse_stride : 1;
             double s = 0.0;
-            for (long j = 0; j < nkv; ++j) s += exp(zbuf[j] - zmax);
-            lse = zmax + log(s);
+            for (long j = 0; j < nkv; j += st) s += exp(zbuf[j] - zmax);
+            lse = zmax + log(s * (double)st);
         }
         lse_heads[hh] = lse;
         /* block score of head h: max over the block's visible kernels of exp(z - LSE) */

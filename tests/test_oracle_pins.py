@@ -573,3 +573,31 @@ def test_backward_sum_rules(oracle):
     assert np.sum(dv * f64(V)) == pytest.approx(np.sum(f64(dout) * out), rel=1e-12)
     assert np.sum(dq * f64(q)) == pytest.approx(np.sum(dk * f64(K)), rel=1e-10, abs=1e-10)
     assert np.max(np.abs(dq)) > 0.01 and np.max(np.abs(dk)) > 0.01
+
+
+# ------------------------------------------------------------------------------------------------
+# LSE estimate from every s-th kernel (a reading of the pages' undefined "LogSumExp estimation")
+# ------------------------------------------------------------------------------------------------
+
+def test_lse_estimate_stride_one_is_exact(oracle):
+    rng = np.random.default_rng(60)
+    q, K, V = rand_case(rng, 1, 20, 900, 4, 2, 16)
+    qc = np.linspace(100, 900, 20).astype(np.int32)[None]
+    kern = oracle.kernel_pool(K, [0], [900], 32, 16)
+    a = oracle.block_score_topk(q, kern, qc, oracle.Params(topk=3))
+    b = oracle.block_score_topk(q, kern, qc, oracle.Params(topk=3, lse_stride=1))
+    assert np.array_equal(a["lse"], b["lse"]) and np.array_equal(a["idx"], b["idx"])
+
+
+@pytest.mark.parametrize("stride", [2, 3, 4])
+def test_lse_estimate_closed_form_on_equal_scores(oracle, stride):
+    """q = 0: every kernel scores 0, so the exact LSE is log(nk) and the estimate log(s * ceil(nk / s))."""
+    rng = np.random.default_rng(61)
+    _, K, _ = rand_case(rng, 1, 1, 700, 4, 2, 16)
+    q = np.zeros((1, 3, 4, 16), np.uint16)
+    qc = np.array([[700, 333, 130]], np.int32)
+    kern = oracle.kernel_pool(K, [0], [700], 32, 16)
+    r = oracle.block_score_topk(q, kern, qc, oracle.Params(topk=2, lse_stride=stride))
+    for t in range(3):
+        nk = oracle.num_kernels(int(qc[0, t]))
+        assert np.allclose(r["lse"][0, t], math.log(stride * math.ceil(nk / stride)), rtol=0, atol=1e-12)
