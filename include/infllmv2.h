@@ -67,9 +67,9 @@ typedef struct {
     int block_size;      /* keys per context block (GPU: 64) */
     int kernel_size;     /* keys per semantic-kernel window (GPU: 32) */
     int kernel_stride;   /* stride between windows (GPU: 16) */
-    int topk;            /* blocks chosen by score besides the forced ones, >= 0 */
-    int init_blocks;     /* blocks [0, init_blocks) always kept */
-    int local_blocks;    /* the query's own block and the local_blocks-1 before it always kept */
+    int topk;            /* blocks chosen by score besides the forced ones, 0 <= topk <= 2^24 */
+    int init_blocks;     /* blocks [0, init_blocks) always kept, 0 <= init_blocks <= 2^24 */
+    int local_blocks;    /* the query's own block and the local_blocks-1 before it always kept, 0 .. 2^24 */
     int dense_len;       /* queries with context n <= dense_len attend densely */
     int membership;      /* 0 = OVERLAP: kernel j belongs to every block its window intersects;
                             1 = CONTAINED: only to the block that contains its whole window */

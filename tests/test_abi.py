@@ -96,6 +96,10 @@ def test_block_score_topk_rejects_bad_arguments(lib):
     assert _score(lib, binding.Params(topk=-1)) == INVALID
     assert _score(lib, binding.Params(membership=2)) == INVALID
     assert _score(lib, binding.Params(topk=0, init_blocks=0, local_blocks=0)) == INVALID
+    # counts whose sum would overflow an int are refused before any use
+    assert _score(lib, binding.Params(topk=2**31 - 1)) == INVALID
+    assert _score(lib, binding.Params(topk=1, init_blocks=2**30, local_blocks=2**30)) == INVALID
+    assert binding.infllmv2_workspace_size(binding.Params(topk=2**31 - 1), 1, 1, 4096, 32, 2, 128) == 0
 
 
 def test_attention_entry_points_reject_bad_arguments(lib):

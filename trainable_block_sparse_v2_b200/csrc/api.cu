@@ -90,6 +90,10 @@ int check_params(const infllmv2_params* p)
 {
     if (!p) return INFLLMV2_ERR_INVALID_ARG;
     if (p->topk < 0 || p->init_blocks < 0 || p->local_blocks < 0 || p->dense_len < 0) return INFLLMV2_ERR_INVALID_ARG;
+    // far past any supported context (kMaxBlocks), and small enough that their sum stays an int
+    constexpr int kMaxCount = 1 << 24;
+    if (p->topk > kMaxCount || p->init_blocks > kMaxCount || p->local_blocks > kMaxCount)
+        return INFLLMV2_ERR_INVALID_ARG;
     if (p->membership != 0 && p->membership != 1) return INFLLMV2_ERR_INVALID_ARG;
     if (p->topk + p->init_blocks + p->local_blocks < 1) return INFLLMV2_ERR_INVALID_ARG;
     if (!(p->softmax_scale == p->softmax_scale) || std::isinf(p->softmax_scale)) return INFLLMV2_ERR_INVALID_ARG;
