@@ -121,18 +121,61 @@ def _stream(stream):
     return stream.cuda_stream
 
 
-def _need(t, dtype, name, ndim=None):
+def _need(t, dtype, name, ndim=None, numel=None, shape=None):
+    """Type, dtype, contiguity and size of one argument.  The library reads and writes every buffer by the
+    sizes it is given, so a buffer smaller than its layout needs would be accessed out of bounds on the
+    device: each wrapper checks every tensor's element count (or exact shape) against the sizes it passes.
+    The device is checked last, for all arguments at once (_devices)."""
     if not isinstance(t, torch.Tensor):
         raise TypeError(f"{name}: expected a torch.Tensor")
-    if t.dtype != dtype:
+    if dtype is not None and t.dtype != dtype:
         raise TypeError(f"{name}: expected {dtype}, got {t.dtype}")
-    if not t.is_cuda:
-        raise ValueError(f"{name}: must be a CUDA tensor")
     if not t.is_contiguous():
         raise ValueError(f"{name}: must be contiguous")
     if ndim is not None and t.dim() != ndim:
         raise ValueError(f"{name}: expected {ndim} dims, got {tuple(t.shape)}")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name}: expected shape {tuple(shape)}, got {tuple(t.shape)}")
+    if numel is not None and t.numel() != numel:
+        raise ValueError(f"{name}: expected {numel} elements, got {t.numel()} (shape {tuple(t.shape)})")
     return t
+
+
+def _opt(t, dtype, name, numel):
+    """An optional argument (None, or as _need)."""
+    return None if t is None else _need(t, dtype, name, numel=numel)
+
+
+def _devices(fn, *ts):
+    """Every tensor argument on one CUDA device."""
+    ts = [t for t in ts if isinstance(t, torch.Tensor)]  # None, or a raw device address given as an int
+    if not all(t.is_cuda for t in ts):
+        raise ValueError(f"{fn}: every tensor argument must be a CUDA tensor")
+    if len({t.device for t in ts}) > 1:
+        raise ValueError(f"{fn}: tensor arguments are on different devices")
+
+
+def _int32(t, name, numel):
+    """An int32 device array of numel entries (lengths, contexts, positions)."""
+    return _need(t, torch.int32, name, numel=numel)
+
+
+def _qkv(q, k, v, q_ndim=None):
+    """q [B, T, Hq, d] (or, for decode, [B, Hq, d] / [B, 1, Hq, d]); k and v [B, Lcap, Hkv, d] of one shape.
+    Returns (B, T, Hq, d, Lcap, Hkv)."""
+    _need(q, torch.bfloat16, "q", q_ndim)
+    if q_ndim is None:  # decode: one query per sequence
+        if q.dim() < 3:
+            raise ValueError(f"q: expected [B, Hq, d] or [B, 1, Hq, d], got {tuple(q.shape)}")
+        B, T, Hq, d = q.shape[0], 1, q.shape[-2], q.shape[-1]
+        _need(q, torch.bfloat16, "q", numel=B * Hq * d)
+    else:
+        B, T, Hq, d = q.shape
+    _need(k, torch.bfloat16, "k", 4)
+    if k.shape[0] != B or k.shape[3] != d:
+        raise ValueError(f"k: expected shape ({B}, Lcap, Hkv, {d}), got {tuple(k.shape)}")
+    _need(v, torch.bfloat16, "v", shape=tuple(k.shape))
+    return B, T, Hq, d, k.shape[1], k.shape[2]
 
 
 def _checking() -> bool:
@@ -175,10 +218,13 @@ def infllmv2_workspace_size(params: Params, batch, max_q, max_ctx, hq, hkv, head
 
 def infllmv2_kernel_pool(k, old_lens, new_lens, max_new_keys, params: Params, kern, stream=None):
     _need(k, torch.bfloat16, "k", 4)
-    _need(kern, torch.bfloat16, "kern", 4)
-    _need(old_lens, torch.int32, "old_lens")
-    _need(new_lens, torch.int32, "new_lens")
     B, Lcap, Hkv, d = k.shape
+    _need(kern, torch.bfloat16, "kern", 4)
+    if (kern.shape[0], kern.shape[1], kern.shape[3]) != (B, Hkv, d):
+        raise ValueError(f"kern: expected shape ({B}, {Hkv}, nk_cap, {d}), got {tuple(kern.shape)}")
+    _int32(old_lens, "old_lens", B)
+    _int32(new_lens, "new_lens", B)
+    _devices("infllmv2_kernel_pool", k, kern, old_lens, new_lens)
     if _checking():
         from . import checks
         checks.check_pool_lengths(old_lens, new_lens, Lcap, int(max_new_keys), kern.shape[2], params.kernel_size,
@@ -191,15 +237,13 @@ def infllmv2_kernel_pool(k, old_lens, new_lens, max_new_keys, params: Params, ke
 
 def infllmv2_kv_append(k_new, v_new, pos, k_cache, v_cache, stream=None):
     """k_cache[b, pos[b]] = k_new[b] and v_cache[b, pos[b]] = v_new[b] (cache maintenance of a decode step)"""
-    _need(k_new, torch.bfloat16, "k_new", 3)
-    _need(v_new, torch.bfloat16, "v_new", 3)
     _need(k_cache, torch.bfloat16, "k_cache", 4)
-    _need(v_cache, torch.bfloat16, "v_cache", 4)
-    _need(pos, torch.int32, "pos")
     B, Lcap, Hkv, d = k_cache.shape
-    if tuple(v_cache.shape) != (B, Lcap, Hkv, d) or tuple(k_new.shape) != (B, Hkv, d) or \
-            tuple(v_new.shape) != (B, Hkv, d):
-        raise ValueError("kv_append: shapes do not match the caches")
+    _need(v_cache, torch.bfloat16, "v_cache", shape=(B, Lcap, Hkv, d))
+    _need(k_new, torch.bfloat16, "k_new", shape=(B, Hkv, d))
+    _need(v_new, torch.bfloat16, "v_new", shape=(B, Hkv, d))
+    _int32(pos, "pos", B)
+    _devices("infllmv2_kv_append", k_new, v_new, pos, k_cache, v_cache)
     st = load().infllmv2_kv_append(_ptr(k_new), _ptr(v_new), B, Hkv, d, _ptr(pos), _ptr(k_cache), _ptr(v_cache), Lcap,
                                    _stream(stream))
     _check("infllmv2_kv_append", st)
@@ -207,15 +251,16 @@ def infllmv2_kv_append(k_new, v_new, pos, k_cache, v_cache, stream=None):
 
 def infllmv2_block_score_topk(q, q_ctx, ctx_lens, max_ctx, kern, params: Params, idx, cnt, ws, stream=None):
     _need(q, torch.bfloat16, "q", 4)
-    _need(kern, torch.bfloat16, "kern", 4)
-    _need(idx, torch.int32, "idx", 4)
-    _need(cnt, torch.int32, "cnt", 3)
-    if q_ctx is not None:
-        _need(q_ctx, torch.int32, "q_ctx")
-    if ctx_lens is not None:
-        _need(ctx_lens, torch.int32, "ctx_lens")
     B, T, Hq, d = q.shape
+    _need(kern, torch.bfloat16, "kern", 4)
     Hkv = kern.shape[1]
+    if (kern.shape[0], kern.shape[3]) != (B, d):
+        raise ValueError(f"kern: expected shape ({B}, Hkv, nk_cap, {d}), got {tuple(kern.shape)}")
+    _need(idx, torch.int32, "idx", numel=B * T * Hkv * params.kmax)
+    _need(cnt, torch.int32, "cnt", numel=B * T * Hkv)
+    _opt(q_ctx, torch.int32, "q_ctx", B * T)
+    _opt(ctx_lens, torch.int32, "ctx_lens", B)
+    _devices("infllmv2_block_score_topk", q, kern, idx, cnt, q_ctx, ctx_lens, ws)
     if _checking():
         _check_rows("infllmv2_block_score_topk", B, T, q_ctx, ctx_lens, False, int(max_ctx), max_ctx)
     cp = params.c()
@@ -228,14 +273,14 @@ def infllmv2_block_score_topk(q, q_ctx, ctx_lens, max_ctx, kern, params: Params,
 
 def infllmv2_sparse_attn_prefill(q, k, v, q_ctx, ctx_lens, max_ctx, idx, cnt, params: Params, out, lse=None,
                                  ws=None, stream=None):
-    for t, n in ((q, "q"), (k, "k"), (v, "v"), (out, "out")):
-        _need(t, torch.bfloat16, n, 4)
-    _need(idx, torch.int32, "idx", 4)
-    _need(cnt, torch.int32, "cnt", 3)
-    if lse is not None:
-        _need(lse, torch.float32, "lse")
-    B, T, Hq, d = q.shape
-    Lcap, Hkv = k.shape[1], k.shape[2]
+    B, T, Hq, d, Lcap, Hkv = _qkv(q, k, v, 4)
+    _need(out, torch.bfloat16, "out", numel=B * T * Hq * d)
+    _need(idx, torch.int32, "idx", numel=B * T * Hkv * params.kmax)
+    _need(cnt, torch.int32, "cnt", numel=B * T * Hkv)
+    _opt(lse, torch.float32, "lse", B * T * Hq)
+    _opt(q_ctx, torch.int32, "q_ctx", B * T)
+    _opt(ctx_lens, torch.int32, "ctx_lens", B)
+    _devices("infllmv2_sparse_attn_prefill", q, k, v, out, idx, cnt, lse, q_ctx, ctx_lens, ws)
     if _checking():
         _check_rows("infllmv2_sparse_attn_prefill", B, T, q_ctx, ctx_lens, False, Lcap, max_ctx, idx, cnt, params)
     cp = params.c()
@@ -246,11 +291,27 @@ def infllmv2_sparse_attn_prefill(q, k, v, q_ctx, ctx_lens, max_ctx, idx, cnt, pa
     _check("infllmv2_sparse_attn_prefill", st)
 
 
+def _decode_args(fn, q, k, v, ctx_lens, out, lse, idx=None, cnt=None, params=None, kern=None, ws=None):
+    """The arguments of the decode entry points: q [B, (1,) Hq, d], k / v [B, Lcap, Hkv, d], ctx_lens [B],
+    out like q, lse [B, (1,) Hq], idx [B, (1,) Hkv, kmax], cnt [B, (1,) Hkv], kern [B, Hkv, nk_cap, d]."""
+    B, _, Hq, d, Lcap, Hkv = _qkv(q, k, v)
+    _need(out, torch.bfloat16, "out", numel=B * Hq * d)
+    _int32(ctx_lens, "ctx_lens", B)
+    _opt(lse, torch.float32, "lse", B * Hq)
+    if idx is not None or cnt is not None:
+        _need(idx, torch.int32, "idx", numel=B * Hkv * params.kmax)
+        _need(cnt, torch.int32, "cnt", numel=B * Hkv)
+    if kern is not None:
+        _need(kern, torch.bfloat16, "kern", 4)
+        if (kern.shape[0], kern.shape[1], kern.shape[3]) != (B, Hkv, d):
+            raise ValueError(f"kern: expected shape ({B}, {Hkv}, nk_cap, {d}), got {tuple(kern.shape)}")
+    _devices(fn, q, k, v, ctx_lens, out, lse, idx, cnt, kern, ws)
+    return B, Hq, d, Lcap, Hkv
+
+
 def infllmv2_sparse_attn_decode(q, k, v, ctx_lens, max_ctx, idx, cnt, params: Params, out, lse, ws, stream=None):
-    for t, n in ((q, "q"), (k, "k"), (v, "v"), (out, "out")):
-        _need(t, torch.bfloat16, n)
-    B, Hq, d = q.shape[0], q.shape[-2], q.shape[-1]
-    Lcap, Hkv = k.shape[1], k.shape[2]
+    B, Hq, d, Lcap, Hkv = _decode_args("infllmv2_sparse_attn_decode", q, k, v, ctx_lens, out, lse, idx, cnt, params,
+                                       ws=ws)
     if _checking():
         _check_rows("infllmv2_sparse_attn_decode", B, 1, None, ctx_lens, True, Lcap, max_ctx,
                     idx.reshape(B, 1, Hkv, -1), cnt.reshape(B, 1, Hkv), params)
@@ -265,12 +326,8 @@ def infllmv2_sparse_attn_decode(q, k, v, ctx_lens, max_ctx, idx, cnt, params: Pa
 def infllmv2_sparse_decode_step(q, kern, k, v, ctx_lens, max_ctx, params: Params, idx, cnt, out, lse=None,
                                 stream=None):
     """Scoring, top-k and sparse attention of one decode step in one launch (no workspace)."""
-    for t, n in ((q, "q"), (kern, "kern"), (k, "k"), (v, "v"), (out, "out")):
-        _need(t, torch.bfloat16, n)
-    _need(idx, torch.int32, "idx")
-    _need(cnt, torch.int32, "cnt")
-    B, Hq, d = q.shape[0], q.shape[-2], q.shape[-1]
-    Lcap, Hkv = k.shape[1], k.shape[2]
+    B, Hq, d, Lcap, Hkv = _decode_args("infllmv2_sparse_decode_step", q, k, v, ctx_lens, out, lse, idx, cnt, params,
+                                       kern=kern)
     if _checking():
         _check_rows("infllmv2_sparse_decode_step", B, 1, None, ctx_lens, True, Lcap, max_ctx)
     cp = params.c()
@@ -284,10 +341,8 @@ def infllmv2_sparse_attn_decode_noalloc(q, k, v, ctx_lens, max_ctx, idx, cnt, pa
                                         stream=None):
     """infllmv2_sparse_attn_decode without a workspace: the library keeps the scratch in its own static
     device array (4 MiB per GPU), for callers that cannot allocate device memory when they call."""
-    for t, n in ((q, "q"), (k, "k"), (v, "v"), (out, "out")):
-        _need(t, torch.bfloat16, n)
-    B, Hq, d = q.shape[0], q.shape[-2], q.shape[-1]
-    Lcap, Hkv = k.shape[1], k.shape[2]
+    B, Hq, d, Lcap, Hkv = _decode_args("infllmv2_sparse_attn_decode_noalloc", q, k, v, ctx_lens, out, lse, idx, cnt,
+                                       params)
     cp = params.c()
     st = load().infllmv2_sparse_attn_decode_noalloc(_ptr(q), B, Hq, Hkv, d, _ptr(k), _ptr(v), Lcap, _ptr(ctx_lens),
                                                     int(max_ctx), _ptr(idx), _ptr(cnt), ctypes.byref(cp), _ptr(out),
@@ -297,10 +352,19 @@ def infllmv2_sparse_attn_decode_noalloc(q, k, v, ctx_lens, max_ctx, idx, cnt, pa
 
 def infllmv2_sparse_attn_tree_verify(q, k, v, prefix_lens, max_ctx, k_draft, v_draft, tree_mask, idx, cnt,
                                      params: Params, out, lse, ws, stream=None):
-    for t, n in ((q, "q"), (k, "k"), (v, "v"), (k_draft, "k_draft"), (v_draft, "v_draft"), (out, "out")):
-        _need(t, torch.bfloat16, n, 4)
-    B, N, Hq, d = q.shape
-    Lcap, Hkv = k.shape[1], k.shape[2]
+    B, N, Hq, d, Lcap, Hkv = _qkv(q, k, v, 4)
+    _need(k_draft, torch.bfloat16, "k_draft", numel=B * N * Hkv * d)
+    _need(v_draft, torch.bfloat16, "v_draft", numel=B * N * Hkv * d)
+    _need(tree_mask, None, "tree_mask", numel=B * N)
+    if tree_mask.element_size() != 4:
+        raise TypeError(f"tree_mask: expected 32-bit words, got {tree_mask.dtype}")
+    _need(out, torch.bfloat16, "out", numel=B * N * Hq * d)
+    _int32(prefix_lens, "prefix_lens", B)
+    _need(idx, torch.int32, "idx", numel=B * N * Hkv * params.kmax)
+    _need(cnt, torch.int32, "cnt", numel=B * N * Hkv)
+    _opt(lse, torch.float32, "lse", B * N * Hq)
+    _devices("infllmv2_sparse_attn_tree_verify", q, k, v, prefix_lens, k_draft, v_draft, tree_mask, idx, cnt, out, lse,
+             ws)
     if _checking():
         _check_rows("infllmv2_sparse_attn_tree_verify", B, N, None, prefix_lens, True, Lcap, max_ctx, idx, cnt,
                     params)
@@ -314,10 +378,12 @@ def infllmv2_sparse_attn_tree_verify(q, k, v, prefix_lens, max_ctx, k_draft, v_d
 
 def infllmv2_dense_attn_prefill(q, k, v, q_ctx, ctx_lens, max_ctx, softmax_scale, out, lse=None, ws=None,
                                 stream=None):
-    for t, n in ((q, "q"), (k, "k"), (v, "v"), (out, "out")):
-        _need(t, torch.bfloat16, n, 4)
-    B, T, Hq, d = q.shape
-    Lcap, Hkv = k.shape[1], k.shape[2]
+    B, T, Hq, d, Lcap, Hkv = _qkv(q, k, v, 4)
+    _need(out, torch.bfloat16, "out", numel=B * T * Hq * d)
+    _opt(lse, torch.float32, "lse", B * T * Hq)
+    _opt(q_ctx, torch.int32, "q_ctx", B * T)
+    _opt(ctx_lens, torch.int32, "ctx_lens", B)
+    _devices("infllmv2_dense_attn_prefill", q, k, v, out, lse, q_ctx, ctx_lens, ws)
     if _checking():
         _check_rows("infllmv2_dense_attn_prefill", B, T, q_ctx, ctx_lens, False, Lcap, max_ctx)
     st = load().infllmv2_dense_attn_prefill(_ptr(q), B, T, Hq, Hkv, d, _ptr(k), _ptr(v), Lcap, _ptr(q_ctx),
@@ -328,10 +394,7 @@ def infllmv2_dense_attn_prefill(q, k, v, q_ctx, ctx_lens, max_ctx, softmax_scale
 
 
 def infllmv2_dense_attn_decode(q, k, v, ctx_lens, max_ctx, softmax_scale, out, lse, ws, stream=None):
-    for t, n in ((q, "q"), (k, "k"), (v, "v"), (out, "out")):
-        _need(t, torch.bfloat16, n)
-    B, Hq, d = q.shape[0], q.shape[-2], q.shape[-1]
-    Lcap, Hkv = k.shape[1], k.shape[2]
+    B, Hq, d, Lcap, Hkv = _decode_args("infllmv2_dense_attn_decode", q, k, v, ctx_lens, out, lse, ws=ws)
     if _checking():
         _check_rows("infllmv2_dense_attn_decode", B, 1, None, ctx_lens, True, Lcap, max_ctx)
     st = load().infllmv2_dense_attn_decode(_ptr(q), B, Hq, Hkv, d, _ptr(k), _ptr(v), Lcap, _ptr(ctx_lens), int(max_ctx),
@@ -341,10 +404,7 @@ def infllmv2_dense_attn_decode(q, k, v, ctx_lens, max_ctx, softmax_scale, out, l
 
 
 def infllmv2_window_attn_decode(q, k, v, ctx_lens, max_ctx, window, softmax_scale, out, lse, ws, stream=None):
-    for t, n in ((q, "q"), (k, "k"), (v, "v"), (out, "out")):
-        _need(t, torch.bfloat16, n)
-    B, Hq, d = q.shape[0], q.shape[-2], q.shape[-1]
-    Lcap, Hkv = k.shape[1], k.shape[2]
+    B, Hq, d, Lcap, Hkv = _decode_args("infllmv2_window_attn_decode", q, k, v, ctx_lens, out, lse, ws=ws)
     if _checking():
         _check_rows("infllmv2_window_attn_decode", B, 1, None, ctx_lens, True, Lcap, max_ctx)
     st = load().infllmv2_window_attn_decode(_ptr(q), B, Hq, Hkv, d, _ptr(k), _ptr(v), Lcap, _ptr(ctx_lens),
@@ -363,16 +423,21 @@ def infllmv2_sparse_attn_backward(q, k, v, q_ctx, ctx_lens, max_ctx, idx, cnt, p
                                   dq, dk, dv, ws, stream=None):
     """Gradients (dq, dk, dv; fp32, overwritten) of the sparse attention for a fixed selection; idx and cnt
     both None means dense attention over [0, n)."""
-    for t, n in ((q, "q"), (k, "k"), (v, "v"), (out, "out"), (dout, "dout")):
-        _need(t, torch.bfloat16, n, 4)
-    for t, n in ((dq, "dq"), (dk, "dk"), (dv, "dv")):
-        _need(t, torch.float32, n, 4)
-    _need(lse, torch.float32, "lse")
+    B, T, Hq, d, Lcap, Hkv = _qkv(q, k, v, 4)
+    _need(out, torch.bfloat16, "out", shape=tuple(q.shape))
+    _need(dout, torch.bfloat16, "dout", shape=tuple(q.shape))
+    _need(dq, torch.float32, "dq", shape=tuple(q.shape))
+    _need(dk, torch.float32, "dk", shape=tuple(k.shape))
+    _need(dv, torch.float32, "dv", shape=tuple(k.shape))
+    _need(lse, torch.float32, "lse", numel=B * T * Hq)
+    if (idx is None) != (cnt is None):
+        raise ValueError("idx and cnt: give both (sparse) or neither (dense)")
     if idx is not None:
-        _need(idx, torch.int32, "idx", 4)
-        _need(cnt, torch.int32, "cnt", 3)
-    B, T, Hq, d = q.shape
-    Lcap, Hkv = k.shape[1], k.shape[2]
+        _need(idx, torch.int32, "idx", numel=B * T * Hkv * params.kmax)
+        _need(cnt, torch.int32, "cnt", numel=B * T * Hkv)
+    _opt(q_ctx, torch.int32, "q_ctx", B * T)
+    _opt(ctx_lens, torch.int32, "ctx_lens", B)
+    _devices("infllmv2_sparse_attn_backward", q, k, v, out, dout, dq, dk, dv, lse, idx, cnt, q_ctx, ctx_lens, ws)
     if _checking():
         _check_rows("infllmv2_sparse_attn_backward", B, T, q_ctx, ctx_lens, False, Lcap, max_ctx, idx, cnt, params)
     cp = params.c()
