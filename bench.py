@@ -573,6 +573,74 @@ class PrefillBench:
         return total, per
 
 
+class TreeBench:
+    """Tree-draft verification at a 64K prefix (one sequence, 16 draft nodes of depth <= 6, 32 / 2 heads,
+    d 128, top-k 64).  One pass: the draft queries' block scoring + top-k over the whole prefix, then the tree
+    attention over each draft's selected prefix blocks and its ancestor drafts.  The prefix's kernel cache is
+    pooled once, untimed; L2 is flushed before every timed pass."""
+
+    def __init__(self):
+        import torch
+        from trainable_block_sparse_v2_b200 import binding
+        from trainable_block_sparse_v2_b200.workloads import tree_verify_64k
+
+        self.torch, self.b = torch, binding
+        w = tree_verify_64k()
+        dev = torch.device("cuda")
+        to = lambda a: torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).to(dev).view(torch.bfloat16)  # noqa: E731
+        i32 = lambda a: torch.from_numpy(np.ascontiguousarray(a, dtype=np.int32)).to(dev)  # noqa: E731
+        self.P = int(w.ctx_lens[0])
+        self.N = w.q.shape[1]
+        self.q, self.k, self.v = to(w.q), to(w.k), to(w.v)
+        self.k_draft, self.v_draft = to(w.extras["k_draft"]), to(w.extras["v_draft"])
+        self.mask = i32(w.extras["tree_mask"].view(np.int32))
+        self.p = binding.Params(**w.params)
+        self.lens = i32(w.ctx_lens)
+        self.q_ctx = i32(w.q_ctx)
+        self.kern = torch.zeros((1, HKV, nk(self.P), D), dtype=torch.bfloat16, device=dev)
+        binding.infllmv2_kernel_pool(self.k, i32([0]), self.lens, self.P, self.p, self.kern)
+        self.idx = torch.empty((1, self.N, HKV, self.p.kmax), dtype=torch.int32, device=dev)
+        self.cnt = torch.empty((1, self.N, HKV), dtype=torch.int32, device=dev)
+        self.out = torch.empty((1, self.N, HQ, D), dtype=torch.bfloat16, device=dev)
+        self.ws = binding.workspace(self.p, 1, self.N, self.P, HQ, HKV, D)
+        self.l2_flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+
+    def verify(self):
+        self.b.infllmv2_block_score_topk(self.q, self.q_ctx, None, self.P, self.kern, self.p, self.idx, self.cnt,
+                                         self.ws)
+        self.b.infllmv2_sparse_attn_tree_verify(self.q, self.k, self.v, self.lens, self.P, self.k_draft, self.v_draft,
+                                                self.mask, self.idx, self.cnt, self.p, self.out, None, self.ws)
+
+    def run(self, warmup, passes):
+        """median seconds per pass, each pass timed alone after an L2 flush"""
+        torch = self.torch
+        for _ in range(warmup):
+            self.verify()
+        torch.cuda.synchronize()
+        evs = []
+        for _ in range(passes):
+            self.l2_flush.fill_(1)
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record()
+            self.verify()
+            b.record()
+            evs.append((a, b))
+        torch.cuda.synchronize()
+        return float(np.median([a.elapsed_time(b) for a, b in evs])) / 1e3
+
+    def bytes_per_pass(self):
+        """Algorithmic bytes: the kernel cache once, each group's union of selected prefix blocks once (keys
+        and values; a partial last block counts its keys), the draft keys / values, queries and outputs."""
+        idx, cnt = self.idx.cpu().numpy(), self.cnt.cpu().numpy()
+        keys = 0
+        for g in range(HKV):
+            blocks = {int(x) for i in range(self.N) for x in idx[0, i, g, :max(0, min(int(cnt[0, i, g]), self.p.kmax))]
+                      if 0 <= x and 64 * int(x) < self.P}
+            keys += sum(min(64, self.P - 64 * b) for b in blocks)
+        return (nk(self.P) * HKV * D * 2 + keys * D * 2 * 2 + self.N * HKV * D * 2 * 2 + self.N * HQ * D * 2 * 2,
+                keys)
+
+
 # ------------------------------------------------------------------------------------------------
 # oracle (CPU) timing on a bounded sample of the decode workload
 # ------------------------------------------------------------------------------------------------
@@ -800,6 +868,30 @@ def run_ours(args):
         del pb
         torch.cuda.empty_cache()
 
+    if not args.no_tree:
+        # tree-draft verification at a 64K prefix; a failure here is reported in the line, not raised, and every
+        # rank takes the same collective step either way
+        tree, t_tree, err = None, float("nan"), None
+        try:
+            tree = TreeBench()
+            t_tree = tree.run(10, 1000)
+        except Exception as e:  # noqa: BLE001
+            err = f"{type(e).__name__}: {e}"[:300]
+        t_tree = barrier_max(t_tree, ws)
+        if err is None and t_tree == t_tree:
+            tb, tkeys = tree.bytes_per_pass()
+            line["tree_verify"] = {
+                "workload": "tree_verify_64k", "value": whole_job_rate(tree.N, ws, t_tree), "unit": UNIT,
+                "us_per_pass": t_tree * 1e6, "passes": 1000, "timing": "median of 1000 passes, L2 flushed before each",
+                "algorithmic_bytes": tb, "attended_prefix_keys": tkeys, "achieved_gbs": tb / t_tree / 1e9,
+                "frac_of_" + peak_kind: tb / t_tree / 1e9 / peaks["hbm_gbs"],
+                "note": "one pass = block_score_topk of the 16 draft queries + sparse_attn_tree_verify",
+            }
+        else:
+            line["tree_verify"] = {"workload": "tree_verify_64k", "error": err or "no time"}
+        del tree
+        torch.cuda.empty_cache()
+
     if rank == 0 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(args.cpu_budget)
     if rank == 0:
@@ -866,6 +958,7 @@ def main():
     ap.add_argument("--prefill-steps", type=int, default=3)
     ap.add_argument("--no-prefill", action="store_true")
     ap.add_argument("--no-backward", action="store_true", help="skip the prefill gradient pass")
+    ap.add_argument("--no-tree", action="store_true", help="skip the tree-verification leg")
     ap.add_argument("--no-decode", action="store_true", help="prefill only (for profiling its kernels)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=15.0)
