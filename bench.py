@@ -573,6 +573,56 @@ class PrefillBench:
         return total, per
 
 
+class Decode32kBench:
+    """Decode at a 32K context, batch 1 (32 / 2 heads, d 128, top-k 64): one step = the kernel pool of the new
+    key + the fused decode step (scoring, top-k, attention), on a cache restored every step (the pool of the
+    step's window rewrites the same kernel).  Its working set (~5.4 MB) fits in L2, so L2 is flushed before
+    every timed step; the time is the median of the steps."""
+
+    def __init__(self):
+        import torch
+        from trainable_block_sparse_v2_b200 import binding
+        from trainable_block_sparse_v2_b200.workloads import decode_32k
+
+        self.torch, self.b = torch, binding
+        w = decode_32k()
+        dev = torch.device("cuda")
+        to = lambda a: torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).to(dev).view(torch.bfloat16)  # noqa: E731
+        i32 = lambda a: torch.from_numpy(np.ascontiguousarray(a, dtype=np.int32)).to(dev)  # noqa: E731
+        self.L = int(w.ctx_lens[0])
+        self.q, self.k, self.v = to(w.q), to(w.k), to(w.v)
+        self.p = binding.Params(**w.params)
+        self.lens, self.old = i32([self.L]), i32([self.L - 1])
+        self.kern = torch.zeros((1, HKV, nk(self.L), D), dtype=torch.bfloat16, device=dev)
+        binding.infllmv2_kernel_pool(self.k, i32([0]), self.old, self.L - 1, self.p, self.kern)
+        self.idx = torch.empty((1, 1, HKV, self.p.kmax), dtype=torch.int32, device=dev)
+        self.cnt = torch.empty((1, 1, HKV), dtype=torch.int32, device=dev)
+        self.out = torch.empty((1, 1, HQ, D), dtype=torch.bfloat16, device=dev)
+        self.l2_flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+
+    def step(self):
+        self.b.infllmv2_kernel_pool(self.k, self.old, self.lens, 1, self.p, self.kern)
+        self.b.infllmv2_sparse_decode_step(self.q, self.kern, self.k, self.v, self.lens, self.L, self.p, self.idx,
+                                           self.cnt, self.out, None)
+
+    def run(self, warmup, steps):
+        """median seconds per step, each step timed alone after an L2 flush"""
+        torch = self.torch
+        for _ in range(warmup):
+            self.step()
+        torch.cuda.synchronize()
+        evs = []
+        for _ in range(steps):
+            self.l2_flush.fill_(1)
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record()
+            self.step()
+            b.record()
+            evs.append((a, b))
+        torch.cuda.synchronize()
+        return float(np.median([a.elapsed_time(b) for a, b in evs])) / 1e3
+
+
 class TreeBench:
     """Tree-draft verification at a 64K prefix (one sequence, 16 draft nodes of depth <= 6, 32 / 2 heads,
     d 128, top-k 64).  One pass: the draft queries' block scoring + top-k over the whole prefix, then the tree
@@ -868,6 +918,30 @@ def run_ours(args):
         del pb
         torch.cuda.empty_cache()
 
+    if not args.no_decode32k:
+        # batch-1 decode at 32K: launch-latency bound by nature (5.4 MB per step); reported, like the tree leg,
+        # without raising, and with the same collective steps on every rank
+        d32, t32, err = None, float("nan"), None
+        try:
+            d32 = Decode32kBench()
+            t32 = d32.run(10, 1000)
+        except Exception as e:  # noqa: BLE001
+            err = f"{type(e).__name__}: {e}"[:300]
+        t32 = barrier_max(t32, ws)
+        if err is None and t32 == t32:
+            _, _, b32 = decode_step_bytes([d32.L])
+            line["decode_32k"] = {
+                "workload": "decode_32k", "value": whole_job_rate(1, ws, t32), "unit": UNIT, "us_per_step": t32 * 1e6,
+                "steps": 1000, "timing": "median of 1000 steps, L2 flushed before each",
+                "algorithmic_bytes": b32, "achieved_gbs": b32 / t32 / 1e9,
+                "frac_of_" + peak_kind: b32 / t32 / 1e9 / peaks["hbm_gbs"],
+                "note": "one step = kernel_pool of the new key + sparse_decode_step, batch 1",
+            }
+        else:
+            line["decode_32k"] = {"workload": "decode_32k", "error": err or "no time"}
+        del d32
+        torch.cuda.empty_cache()
+
     if not args.no_tree:
         # tree-draft verification at a 64K prefix; a failure here is reported in the line, not raised, and every
         # rank takes the same collective step either way
@@ -959,6 +1033,7 @@ def main():
     ap.add_argument("--no-prefill", action="store_true")
     ap.add_argument("--no-backward", action="store_true", help="skip the prefill gradient pass")
     ap.add_argument("--no-tree", action="store_true", help="skip the tree-verification leg")
+    ap.add_argument("--no-decode32k", action="store_true", help="skip the batch-1 32K decode leg")
     ap.add_argument("--no-decode", action="store_true", help="prefill only (for profiling its kernels)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=15.0)
