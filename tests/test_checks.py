@@ -85,3 +85,19 @@ def test_binding_hook_reads_the_environment_and_checks_tensors(oracle, monkeypat
     with pytest.raises(checks.InputCheckError, match=r"\(0, 650, 1\)"):
         binding._check_rows("prefill", 1, 700, None, lens, False, 700, 700, torch.from_numpy(bad),
                             torch.from_numpy(cnt), p)
+
+
+def test_tree_mask():
+    from trainable_block_sparse_v2_b200.workloads import tree_mask_from_parents
+    rng = np.random.default_rng(5)
+    for _ in range(20):  # masks built from random trees pass
+        n = int(rng.integers(1, 33))
+        parent = np.array([-1] + [int(rng.integers(0, i)) for i in range(1, n)])
+        checks.check_tree_mask(tree_mask_from_parents(parent)[None], 1, n)
+    good = tree_mask_from_parents(np.array([-1, 0, 1, 1]))  # 0 <- 1 <- {2, 3}
+    for i, bad, msg in ((2, int(good[2]) & ~(1 << 2), "own bit"), (1, int(good[1]) | (1 << 4), "past n_draft"),
+                        (3, (1 << 3) | (1 << 1), "ancestors")):
+        m = good.astype(np.int64).copy()
+        m[i] = bad
+        with pytest.raises(checks.InputCheckError, match=msg):
+            checks.check_tree_mask(m.astype(np.uint32)[None], 1, 4)

@@ -368,6 +368,8 @@ def infllmv2_sparse_attn_tree_verify(q, k, v, prefix_lens, max_ctx, k_draft, v_d
     if _checking():
         _check_rows("infllmv2_sparse_attn_tree_verify", B, N, None, prefix_lens, True, Lcap, max_ctx, idx, cnt,
                     params)
+        from . import checks
+        checks.check_tree_mask(tree_mask, B, N, "infllmv2_sparse_attn_tree_verify")
     cp = params.c()
     st = load().infllmv2_sparse_attn_tree_verify(_ptr(q), B, N, Hq, Hkv, d, _ptr(k), _ptr(v), Lcap, _ptr(prefix_lens),
                                                  int(max_ctx), _ptr(k_draft), _ptr(v_draft), _ptr(tree_mask), _ptr(idx),

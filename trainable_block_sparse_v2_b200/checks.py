@@ -91,3 +91,20 @@ def check_pool_lengths(old_lens, new_lens, lcap: int, max_new_keys: int, nk_cap:
         nk = (n - kernel_size) // kernel_stride + 1 if n >= kernel_size else 0
         if nk > nk_cap:
             raise InputCheckError(f"{what}: sequence {b} needs {nk} kernels, nk_cap is {nk_cap}")
+
+
+def check_tree_mask(tree_mask, B: int, n_draft: int, what: str = "") -> None:
+    """Every draft node's mask is an ancestor mask: it has its own bit, no bit at or past n_draft, and it holds
+    every node its nodes see (node i seeing node j sees all of j's ancestors)."""
+    m = _np(tree_mask).astype(np.int64).reshape(B, n_draft) & 0xFFFFFFFF
+    for b in range(B):
+        for i in range(n_draft):
+            mi = int(m[b, i])
+            if not (mi >> i) & 1:
+                raise InputCheckError(f"{what}: tree_mask[{b}, {i}] lacks the node's own bit")
+            if mi >> n_draft:
+                raise InputCheckError(f"{what}: tree_mask[{b}, {i}] has bits at or past n_draft = {n_draft}")
+            for j in range(n_draft):
+                if (mi >> j) & 1 and int(m[b, j]) & ~mi:
+                    raise InputCheckError(f"{what}: node {i} of sequence {b} sees node {j} but not all of node "
+                                          f"{j}'s ancestors")
