@@ -25,6 +25,8 @@
 // The footprint (about 112 KB of shared memory) lets two CTAs share an SM, so eight 16-CTA clusters are
 // resident at once.  Every 2^x here has x <= 0 (a difference from a running or final maximum) or -inf,
 // so the hardware ex2.approx (one MUFU op, tiny results flushed to zero) serves throughout.
+#include <atomic>
+
 #include <cooperative_groups.h>
 
 #include "attn_warp.cuh"
@@ -602,15 +604,17 @@ cudaError_t fused_launch(const CUtensorMap& tk, const CUtensorMap& tv, const Que
                               static_cast<__nv_bfloat16*>(out), lse);
 }
 
-// 16-CTA clusters of this kernel the device keeps resident at once (0 when 16 is not schedulable)
+// 16-CTA clusters of this kernel the device keeps resident at once (0 when 16 is not schedulable).  Cached per
+// device in an atomic (0: not yet known, else the count + 1), so that host threads calling at once are safe;
+// two of them may both query the device, and store the same value.
 template <int D, int E>
 int resident_clusters16()
 {
-    static int cached[64];
-    static bool done[64];
+    static std::atomic<int> cached[64];
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 0;
-    if (done[dev]) return cached[dev];
+    const int known = cached[dev].load(std::memory_order_relaxed);
+    if (known > 0) return known - 1;
     int n = 0;
     auto kfn = decode_fused_kernel<D, 16, E>;
     if (ensure_smem(kfn, FLayout<D>::kBytes) == cudaSuccess &&
@@ -629,8 +633,7 @@ int resident_clusters16()
         if (cudaOccupancyMaxActiveClusters(&n, kfn, &cfg) != cudaSuccess) n = 0;
     }
     (void)cudaGetLastError();
-    cached[dev] = n;
-    done[dev] = true;
+    cached[dev].store(n + 1, std::memory_order_relaxed);
     return n;
 }
 
