@@ -116,7 +116,9 @@ int infllmv2_kv_append(const void* k_new, const void* v_new, int batch, int hkv,
  * Step 1 -- semantic kernels (MiniCPM4 technical details, "Model architecture: InfLLM v2", item 1).
  * For each sequence b, writes the kernels completed between old_lens[b] and new_lens[b] keys:
  *   kern[b, g, j, :] = bf16_round_nearest_even( mean_{i in [16 j, 16 j + 32)} k[b, i, g, :] )
- * for j in [nk(old), nk(new)), nk(n) = n >= 32 ? (n - 32) / 16 + 1 : 0.  Sums are fp32.
+ * for j in [nk(old), nk(new)), nk(n) = n >= 32 ? (n - 32) / 16 + 1 : 0.  The window sum is formed in fp64
+ * (exact unless the 32 keys' exponents spread over more than ~40 binary orders) and the mean is rounded once
+ * to bf16, so the result is the correctly rounded mean.
  *   k            [B, Lcap, Hkv, d] bf16 (device)
  *   old_lens,
  *   new_lens     [B] int32 (device), 0 <= old <= new <= Lcap; device-side values are trusted

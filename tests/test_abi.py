@@ -158,3 +158,27 @@ def test_backward_rejects_bad_arguments(lib):
     assert call(max_ctx=5000) == INVALID             # max_ctx past the cache
     assert call(wsb=need - 256) == WORKSPACE
     assert call(ws=WS + 16) == WORKSPACE
+
+
+def test_noalloc_decode_refuses_what_the_workspace_decode_refuses(lib):
+    """The allocation-free decode shares the workspace entry point's argument checks: oversized block counts
+    (whose sum would overflow an int), an infinite scale, a context past the cache or past 4096 blocks, and
+    too many rows are refused with the same status, before any launch."""
+
+    def both(params, batch=1, hkv=2, lcap=4096, max_ctx=4096, lse=None):
+        cp = params.c()
+        a = lib.infllmv2_sparse_attn_decode(A16, batch, 16 * hkv, hkv, 128, A16, A16, lcap, A4, max_ctx, A4, A4,
+                                            ctypes.byref(cp), A16, lse, WS, 1 << 40, None)
+        b = lib.infllmv2_sparse_attn_decode_noalloc(A16, batch, 16 * hkv, hkv, 128, A16, A16, lcap, A4, max_ctx, A4,
+                                                    A4, ctypes.byref(cp), A16, lse, None)
+        return a, b
+
+    assert both(binding.Params(topk=2**31 - 1)) == (INVALID, INVALID)
+    assert both(binding.Params(topk=1, init_blocks=2**30, local_blocks=2**30)) == (INVALID, INVALID)
+    assert both(binding.Params(topk=64, softmax_scale=float("inf"))) == (INVALID, INVALID)
+    assert both(binding.Params(topk=64, membership=2)) == (INVALID, INVALID)
+    assert both(binding.Params(topk=64), lcap=1000, max_ctx=2000) == (INVALID, INVALID)
+    assert both(binding.Params(topk=64), lcap=1 << 20, max_ctx=4096 * 64 + 1) == (UNSUPPORTED, UNSUPPORTED)
+    assert both(binding.Params(topk=64), lse=A4 + 2) == (INVALID, INVALID)
+    assert both(binding.Params(topk=64), batch=1 << 15, hkv=4) == (UNSUPPORTED, UNSUPPORTED)
+    assert both(binding.Params(block_size=32)) == (UNSUPPORTED, UNSUPPORTED)

@@ -90,6 +90,23 @@ def test_kernel_pool_bulk_and_incremental(oracle, d):
     assert np.array_equal(host_u16(kern), want)
 
 
+@pytest.mark.parametrize("d", [64, 128])
+def test_kernel_pool_rounds_the_exact_mean_once(oracle, d):
+    """Windows whose exact sum sits a hair beside a bf16 midpoint, or exactly on one: the kernel must be the
+    exact mean rounded once (bits worked out by hand in tests/pool_midpoints.py), in bulk and one key at a
+    time."""
+    from pool_midpoints import midpoint_case
+    K, want = midpoint_case(d)
+    L = K.shape[1]
+    assert np.array_equal(oracle.kernel_pool(K, [0], [L], 32, 16), want)
+    got = host_u16(gpu_pool(K, np.zeros(1), np.array([L]), L, want.shape[2]))
+    assert np.array_equal(got, want)
+    kern = gpu_pool(K, np.zeros(1), np.zeros(1), 1, want.shape[2])
+    for n in range(1, L + 1):
+        gpu_pool(K, np.array([n - 1]), np.array([n]), 1, want.shape[2], kern=kern)
+    assert np.array_equal(host_u16(kern), want)
+
+
 # ---------------------------------------------------------------------------------------------------
 # step 2: scoring + selection
 # ---------------------------------------------------------------------------------------------------
@@ -286,6 +303,10 @@ def test_end_to_end_tiny_prefill(oracle):
     torch.cuda.synchronize()
     row_same = same.all(axis=-1)  # [B, T]: both groups match
     check_attention(out, out_o, mask=row_same, what="end-to-end")
+    # rows whose selection differs at a near tie: the oracle's attention on the GPU's own selection
+    if not row_same.all():
+        out_g, _ = oracle.sparse_attention(w.q, w.k, w.v, w.q_ctx, gidx, gcnt, P)
+        check_attention(out, out_g, what="end-to-end (own selection)")
 
 
 @pytest.mark.parametrize("path", ["scan_few_members", "scan_degenerate", "tile"])
@@ -351,5 +372,9 @@ def test_fused_decode_step(oracle, G, d, lens, membership, topk):
     binding.infllmv2_sparse_decode_step(dev(w.q), kern, K, V, dev_i32(w.ctx_lens), max(lens), p, idx, cnt, out, lse)
     torch.cuda.synchronize()
     assert binding.infllmv2_device_status() == 0
-    same = check_selection(idx.cpu().numpy(), cnt.cpu().numpy(), r)
+    gi, gc = idx.cpu().numpy(), cnt.cpu().numpy()
+    same = check_selection(gi, gc, r)
     check_attention(out, out_o, lse, lse_o, mask=same.all(axis=-1), what="fused decode step")
+    if not same.all():  # near-tie rows: the oracle's attention on the GPU's own selection
+        out_g, lse_g = oracle.sparse_attention(w.q, w.k, w.v, w.q_ctx, gi, gc, P)
+        check_attention(out, out_g, lse, lse_g, what="fused decode step (own selection)")

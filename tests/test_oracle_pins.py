@@ -134,6 +134,17 @@ def test_kernel_pool_incremental_equals_bulk(oracle):
     assert np.array_equal(inc, bulk)
 
 
+def test_kernel_pool_rounds_the_exact_mean_once(oracle):
+    """Hand-worked windows whose exact sum sits a hair beside a bf16 midpoint (an fp32 sum would drop the
+    2^-30 key and tie the other way) or exactly on one (ties to even): the expected bits are worked out by
+    hand in tests/pool_midpoints.py."""
+    from pool_midpoints import midpoint_case
+    for d in (16, 64):
+        K, want = midpoint_case(d)
+        got = oracle.kernel_pool(K, [0], [K.shape[1]], 32, 16)
+        assert np.array_equal(got, want)
+
+
 def test_round_bf16_single_rounding(oracle):
     rng = np.random.default_rng(9)
     x = (rng.standard_normal(2000) * np.exp(rng.uniform(-20, 20, 2000))).astype(np.float32)

@@ -200,6 +200,30 @@ QueryRows rows_of(const void* q, int B, int T, int hq, int hkv, int d, const int
 
 }  // namespace
 
+// Argument checks and method constants of the two-call decode attention, shared by
+// infllmv2_sparse_attn_decode and infllmv2_sparse_attn_decode_noalloc so that both refuse the same calls.
+int iv2::check_decode_attn(const void* q, int batch, int hq, int hkv, int head_dim, const void* k, const void* v,
+                           int lcap, const int32_t* ctx_lens, int max_ctx, const int32_t* idx, const int32_t* cnt,
+                           const infllmv2_params* params, const void* out, const float* lse, MethodConsts* mc,
+                           int* nsplit)
+{
+    IV2_TRY(check_params(params));
+    IV2_TRY(check_heads(batch, 1, hq, hkv, head_dim));
+    IV2_TRY(check_ptr16(q));
+    IV2_TRY(check_ptr16(k));
+    IV2_TRY(check_ptr16(v));
+    IV2_TRY(check_ptr16(out));
+    IV2_TRY(check_ptr4(idx));
+    IV2_TRY(check_ptr4(cnt));
+    IV2_TRY(check_ptr4(ctx_lens));
+    IV2_TRY(check_opt4(lse));
+    IV2_TRY(check_ctx(max_ctx, lcap));
+    *mc = consts_of(params, head_dim);
+    if (batch * hkv > iv2::kMaxSplitRows) return INFLLMV2_ERR_UNSUPPORTED;
+    *nsplit = iv2::attn_split_count(iv2::attn_split_max_blocks(max_ctx, mc->kmax, mc->dense_len, false));
+    return INFLLMV2_OK;
+}
+
 extern "C" {
 
 const char* infllmv2_status_string(int status)
@@ -328,20 +352,11 @@ int infllmv2_sparse_attn_decode(const void* q, int batch, int hq, int hkv, int h
                                 const int32_t* cnt, const infllmv2_params* params, void* out, float* lse, void* ws,
                                 size_t ws_bytes, infllmv2_stream_t stream)
 {
-    IV2_TRY(check_params(params));
-    IV2_TRY(check_heads(batch, 1, hq, hkv, head_dim));
-    IV2_TRY(check_ptr16(q));
-    IV2_TRY(check_ptr16(k));
-    IV2_TRY(check_ptr16(v));
-    IV2_TRY(check_ptr16(out));
-    IV2_TRY(check_ptr4(idx));
-    IV2_TRY(check_ptr4(cnt));
-    IV2_TRY(check_ptr4(ctx_lens));
-    IV2_TRY(check_opt4(lse));
-    IV2_TRY(check_ctx(max_ctx, lcap));
-    const MethodConsts mc = consts_of(params, head_dim);
-    if (batch * hkv > iv2::kMaxSplitRows) return INFLLMV2_ERR_UNSUPPORTED;
-    IV2_TRY(check_ws(ws, ws_bytes, split_need(batch * hkv, max_ctx, mc.kmax, mc.dense_len, false, false)));
+    MethodConsts mc;
+    int nsplit = 0;
+    IV2_TRY(iv2::check_decode_attn(q, batch, hq, hkv, head_dim, k, v, lcap, ctx_lens, max_ctx, idx, cnt, params, out,
+                                   lse, &mc, &nsplit));
+    IV2_TRY(check_ws(ws, ws_bytes, iv2::attn_ws_bytes(batch * hkv, nsplit)));
     const QueryRows qr = rows_of(q, batch, 1, hq, hkv, head_dim, nullptr, ctx_lens, 0, max_ctx);
     return launched(iv2::launch_attn_split(qr, k, v, lcap, idx, cnt, mc, false, nullptr, nullptr, nullptr, out, lse,
                                            ws, (cudaStream_t)stream));

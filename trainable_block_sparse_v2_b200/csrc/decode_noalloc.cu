@@ -45,8 +45,6 @@ cudaError_t scratch_address(void** out)
     return cudaSuccess;
 }
 
-bool aligned_to(const void* p, uintptr_t a) { return p && (reinterpret_cast<uintptr_t>(p) % a) == 0; }
-
 }  // namespace
 
 extern "C" int infllmv2_sparse_attn_decode_noalloc(const void* q, int batch, int hq, int hkv, int head_dim,
@@ -55,34 +53,13 @@ extern "C" int infllmv2_sparse_attn_decode_noalloc(const void* q, int batch, int
                                                    const infllmv2_params* params, void* out, float* lse,
                                                    infllmv2_stream_t stream)
 {
-    if (!params) return INFLLMV2_ERR_INVALID_ARG;
-    if (params->block_size != iv2::kBlock || params->kernel_size != iv2::kKernelSize ||
-        params->kernel_stride != iv2::kKernelStride)
-        return INFLLMV2_ERR_UNSUPPORTED;
-    if (params->topk < 0 || params->init_blocks < 0 || params->local_blocks < 0 || params->dense_len < 0 ||
-        params->topk + params->init_blocks + params->local_blocks < 1 ||
-        (params->membership != 0 && params->membership != 1) || !(params->softmax_scale == params->softmax_scale))
-        return INFLLMV2_ERR_INVALID_ARG;
-    if (batch < 1 || hq < 1 || hkv < 1 || hq % hkv != 0) return INFLLMV2_ERR_INVALID_ARG;
-    const int G = hq / hkv;
-    if ((G != 1 && G != 2 && G != 4 && G != 8 && G != 16) || (head_dim != 64 && head_dim != 128))
-        return INFLLMV2_ERR_UNSUPPORTED;
-    if (!aligned_to(q, 16) || !aligned_to(k, 16) || !aligned_to(v, 16) || !aligned_to(out, 16) ||
-        !aligned_to(ctx_lens, 4) || !aligned_to(idx, 4) || !aligned_to(cnt, 4) || (lse && !aligned_to(lse, 4)))
-        return INFLLMV2_ERR_INVALID_ARG;
-    if (max_ctx < 1 || max_ctx > lcap) return INFLLMV2_ERR_INVALID_ARG;
-    if ((max_ctx - 1) / iv2::kBlock + 1 > 4096) return INFLLMV2_ERR_UNSUPPORTED;
-
-    iv2::MethodConsts mc{};
-    mc.topk = params->topk;
-    mc.init_blocks = params->init_blocks;
-    mc.local_blocks = params->local_blocks;
-    mc.dense_len = params->dense_len;
-    mc.membership = params->membership;
-    mc.scale = params->softmax_scale > 0.f ? params->softmax_scale : 1.0f / sqrtf((float)head_dim);
-    mc.kmax = params->topk + params->init_blocks + params->local_blocks;
+    // the same argument checks as infllmv2_sparse_attn_decode
+    iv2::MethodConsts mc;
+    int nsplit = 0;
+    const int st = iv2::check_decode_attn(q, batch, hq, hkv, head_dim, k, v, lcap, ctx_lens, max_ctx, idx, cnt, params,
+                                          out, lse, &mc, &nsplit);
+    if (st != INFLLMV2_OK) return st;
     // the partials of this call must fit the static array
-    const int nsplit = iv2::attn_split_count(iv2::attn_split_max_blocks(max_ctx, mc.kmax, mc.dense_len, false));
     if (iv2::attn_ws_bytes(batch * hkv, nsplit) > kNoAllocScratchBytes) return INFLLMV2_ERR_WORKSPACE;
 
     void* scratch = nullptr;

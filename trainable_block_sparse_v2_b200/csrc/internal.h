@@ -8,6 +8,8 @@
 
 #include <utility>
 
+#include "../../include/infllmv2.h"
+
 namespace iv2 {
 
 // Raise a kernel's dynamic shared-memory limit once per (kernel, device), so that stream captures after
@@ -92,6 +94,14 @@ struct MethodConsts {
 
 // rows (sequence x query x KV group) one split-attention launch handles
 constexpr int kMaxSplitRows = 1 << 16;
+
+// Argument checks of the two-call decode attention (api.cu): the status the workspace entry point would
+// return before its workspace check, the method constants, and the number of KV splits per row.  Shared with
+// the allocation-free entry point, so that both refuse exactly the same calls.
+int check_decode_attn(const void* q, int batch, int hq, int hkv, int head_dim, const void* k, const void* v, int lcap,
+                      const int32_t* ctx_lens, int max_ctx, const int32_t* idx, const int32_t* cnt,
+                      const infllmv2_params* params, const void* out, const float* lse, MethodConsts* mc,
+                      int* nsplit);
 
 // scoring path: true -> split-kernel scan + per-row select (needs workspace), false -> token tiles
 bool score_uses_scan_path(int B, int T, int G, int D, int max_ctx);

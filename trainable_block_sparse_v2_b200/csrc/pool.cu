@@ -6,9 +6,19 @@
 // fine-grained semantic kernels; the pages give no window size).
 //
 // HBM-bound: every key row is read once.  A window of 32 keys is the sum of two 16-key half windows
-// that it shares with its neighbours, so each CTA first sums 33 half windows (fp32) into shared memory
-// and then forms 32 kernels from adjacent pairs.  Rows are 16-byte coalesced loads (d = 128: 16 lanes
-// cover one 256-byte row), and all 16 rows of a half window are in flight per thread.
+// that it shares with its neighbours, so each CTA first sums 33 half windows into shared memory and then
+// forms 32 kernels from adjacent pairs.  Rows are 16-byte coalesced loads (d = 128: 16 lanes cover one
+// 256-byte row), and all 16 rows of a half window are in flight per thread.
+//
+// Exactness.  The kernel is the window mean rounded ONCE to bf16.  The sums are formed in fp64: a bf16
+// value has an 8-bit significand, so a sum of 32 of them is exact in fp64 unless their exponents spread
+// over more than ~40 binary orders (never for activations of a model; an fp32 sum of N(0,1) keys is
+// inexact about once in a few million kernels and then double-rounds).  The scaling by 1/32 is exact, and
+// the fp64 mean reaches bf16 through one correctly rounded step: round-to-odd into fp32, then
+// round-to-nearest-even into bf16.  Rounding to odd into a format with at least two more significand bits
+// than the target makes the second rounding equal to a direct one (S. Boldo and G. Melquiond, "Emulation
+// of FMA and correctly rounded sums: proved algorithms using rounding to odd", IEEE Trans. Computers 57(4),
+// 2008); fp32 has 24 bits against bf16's 8.
 #include "common.cuh"
 #include "internal.h"
 
@@ -16,6 +26,15 @@ namespace iv2 {
 
 constexpr int kPoolKernelsPerCta = 32;
 constexpr int kPoolThreads = 256;
+
+// fp64 -> bf16, round to nearest even, in one correctly rounded step (round-to-odd into fp32 first).
+IV2_DEV uint16_t f64_to_bf16_rne(double x)
+{
+    float f = __double2float_rz(x);                 // truncate toward zero into fp32
+    if ((double)f != x) f = __uint_as_float(__float_as_uint(f) | 1u);  // inexact: make the last bit odd
+    __nv_bfloat16 h = __float2bfloat16_rn(f);
+    return *reinterpret_cast<uint16_t*>(&h);
+}
 
 template <int D>
 __global__ void __launch_bounds__(kPoolThreads) kernel_pool_kernel(const __nv_bfloat16* __restrict__ k, int Lcap,
@@ -27,7 +46,7 @@ __global__ void __launch_bounds__(kPoolThreads) kernel_pool_kernel(const __nv_bf
     pdl_wait();
     constexpr int CH = D / 8;                  // 16-byte chunks per row
     constexpr int HALVES = kPoolKernelsPerCta + 1;
-    __shared__ float hs[HALVES][D];
+    __shared__ double hs[HALVES][D];  // exact half-window sums (33.8 KB at d = 128)
 
     const int bg = blockIdx.y;
     const int b = bg / Hkv, g = bg % Hkv;
@@ -44,9 +63,9 @@ __global__ void __launch_bounds__(kPoolThreads) kernel_pool_kernel(const __nv_bf
     for (int item = threadIdx.x; item < n_halves * CH; item += kPoolThreads) {
         const int h = item / CH, c = item % CH;
         const int row0 = (j_begin + h) * kKernelStride;
-        float acc[8];
+        double acc[8];
 #pragma unroll
-        for (int e = 0; e < 8; ++e) acc[e] = 0.f;
+        for (int e = 0; e < 8; ++e) acc[e] = 0.0;
         uint4 buf[kKernelStride];
 #pragma unroll
         for (int r = 0; r < kKernelStride; ++r) buf[r] = ld_nc_v4(kb + (size_t)(row0 + r) * row_stride + c * 8);
@@ -55,8 +74,8 @@ __global__ void __launch_bounds__(kPoolThreads) kernel_pool_kernel(const __nv_bf
             const uint32_t w[4] = {buf[r].x, buf[r].y, buf[r].z, buf[r].w};
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
-                acc[2 * e] += bf16_lo(w[e]);
-                acc[2 * e + 1] += bf16_hi(w[e]);
+                acc[2 * e] += (double)bf16_lo(w[e]);
+                acc[2 * e + 1] += (double)bf16_hi(w[e]);
             }
         }
 #pragma unroll
@@ -64,15 +83,15 @@ __global__ void __launch_bounds__(kPoolThreads) kernel_pool_kernel(const __nv_bf
     }
     __syncthreads();
 
-    constexpr float inv = 1.0f / kKernelSize;  // a power of two: the scaling is exact
+    constexpr double inv = 1.0 / kKernelSize;  // a power of two: the scaling is exact
     for (int item = threadIdx.x; item < (j_end - j_begin) * CH; item += kPoolThreads) {
         const int jj = item / CH, c = item % CH;
         uint32_t w[4];
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
-            const float lo = (hs[jj][c * 8 + 2 * e] + hs[jj + 1][c * 8 + 2 * e]) * inv;
-            const float hi = (hs[jj][c * 8 + 2 * e + 1] + hs[jj + 1][c * 8 + 2 * e + 1]) * inv;
-            w[e] = pack_bf16(lo, hi);
+            const double lo = (hs[jj][c * 8 + 2 * e] + hs[jj + 1][c * 8 + 2 * e]) * inv;
+            const double hi = (hs[jj][c * 8 + 2 * e + 1] + hs[jj + 1][c * 8 + 2 * e + 1]) * inv;
+            w[e] = (uint32_t)f64_to_bf16_rne(lo) | ((uint32_t)f64_to_bf16_rne(hi) << 16);
         }
         __nv_bfloat16* dst = kern + (((size_t)b * Hkv + g) * nk_cap + j_begin + jj) * D + c * 8;
         *reinterpret_cast<uint4*>(dst) = make_uint4(w[0], w[1], w[2], w[3]);
