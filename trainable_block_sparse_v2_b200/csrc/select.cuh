@@ -162,7 +162,7 @@ IV2_DEV void warp_select_topk_hist(const float* S, int c, int init, int local, i
             if (lane >= o) incl += y;
         }
         const int excl = incl - sum;
-        int my_b = -1, my_above = 0;
+        int my_b = -1, my_above = 0, my_cnt = 0;
         if (excl < topk && topk <= incl) {
             int acc = excl;
 #pragma unroll
@@ -170,6 +170,7 @@ IV2_DEV void warp_select_topk_hist(const float* S, int c, int init, int local, i
                 if (my_b < 0 && acc + cb[j] >= topk) {
                     my_b = base + BPL - 1 - j;
                     my_above = acc;
+                    my_cnt = cb[j];
                 }
                 acc += cb[j];
             }
@@ -178,65 +179,72 @@ IV2_DEV void warp_select_topk_hist(const float* S, int c, int init, int local, i
         const int src = __ffs(hitm) - 1;
         bstar = __shfl_sync(0xffffffffu, my_b, src);
         const int rem = topk - __shfl_sync(0xffffffffu, my_above, src);  // members of B* still to take, >= 1
-        // gather the members of B* (ascending block order) and count them
-        int nm = 0;
-#pragma unroll
-        for (int e = 0; e < KW; ++e) {
-            const bool mem = bk[e] == bstar;
-            const unsigned mm = __ballot_sync(0xffffffffu, mem);
-            const int pos = nm + __popc(mm & ((1u << lane) - 1u));
-            if (mem && pos < kWarpMembers) {
-                ws.mkey[pos] = key[e];
-                ws.midx[pos] = lane + 32 * e;
-            }
-            nm += __popc(mm);
-        }
-        __syncwarp();
-        if (nm <= kWarpMembers) {
-            // the member of rank rem - 1 in (key descending, block ascending) order is the threshold
-            int my_hit = -1;
-            for (int i = lane; i < nm; i += 32) {
-                const uint32_t ki = ws.mkey[i];
-                const int ii = ws.midx[i];
-                int rank = 0;
-                for (int j = 0; j < nm; ++j) {
-                    const uint32_t kj = ws.mkey[j];
-                    rank += (kj > ki) || (kj == ki && ws.midx[j] < ii);
-                }
-                if (rank == rem - 1) my_hit = i;
-            }
-            const unsigned th = __ballot_sync(0xffffffffu, my_hit >= 0);
-            const int ti = __shfl_sync(0xffffffffu, my_hit, __ffs(th) - 1);
-            tkey = ws.mkey[ti];
-            tidx = ws.midx[ti];
+        const int bcnt = __shfl_sync(0xffffffffu, my_cnt, src);           // members of B*
+        if (bcnt == rem) {
+            // the boundary bucket is taken whole: every candidate in a bucket >= B* is chosen, no ranking
+            tkey = 0u;
+            tidx = 0x7fffffff;
         } else {
-            // many equal-bucket keys: bitwise search of the rem-th largest member key, then block ids
-            uint32_t t = 0u;
-            for (int bit = 31; bit >= 0; --bit) {
-                const uint32_t probe = t | (1u << bit);
-                int ge = 0;
-#pragma unroll
-                for (int e = 0; e < KW; ++e) ge += bk[e] == bstar && key[e] >= probe;
-                if (warp_count(ge) >= rem) t = probe;
-            }
-            int gt = 0;
-#pragma unroll
-            for (int e = 0; e < KW; ++e) gt += bk[e] == bstar && key[e] > t;
-            const int need = rem - warp_count(gt);
-            // the need-th lowest block id among the members with key t
-            int seen = 0;
-            tidx = -1;
+            // gather the members of B* (ascending block order) and count them
+            int nm = 0;
 #pragma unroll
             for (int e = 0; e < KW; ++e) {
-                const unsigned eq = __ballot_sync(0xffffffffu, bk[e] == bstar && key[e] == t);
-                if (tidx < 0 && seen + __popc(eq) >= need) {
-                    unsigned m2 = eq;
-                    for (int j = 0; j < need - seen - 1; ++j) m2 &= m2 - 1u;
-                    tidx = 32 * e + __ffs(m2) - 1;
+                const bool mem = bk[e] == bstar;
+                const unsigned mm = __ballot_sync(0xffffffffu, mem);
+                const int pos = nm + __popc(mm & ((1u << lane) - 1u));
+                if (mem && pos < kWarpMembers) {
+                    ws.mkey[pos] = key[e];
+                    ws.midx[pos] = lane + 32 * e;
                 }
-                seen += __popc(eq);
+                nm += __popc(mm);
             }
-            tkey = t;
+            __syncwarp();
+            if (nm <= kWarpMembers) {
+                // the member of rank rem - 1 in (key descending, block ascending) order is the threshold
+                int my_hit = -1;
+                for (int i = lane; i < nm; i += 32) {
+                    const uint32_t ki = ws.mkey[i];
+                    const int ii = ws.midx[i];
+                    int rank = 0;
+                    for (int j = 0; j < nm; ++j) {
+                        const uint32_t kj = ws.mkey[j];
+                        rank += (kj > ki) || (kj == ki && ws.midx[j] < ii);
+                    }
+                    if (rank == rem - 1) my_hit = i;
+                }
+                const unsigned th = __ballot_sync(0xffffffffu, my_hit >= 0);
+                const int ti = __shfl_sync(0xffffffffu, my_hit, __ffs(th) - 1);
+                tkey = ws.mkey[ti];
+                tidx = ws.midx[ti];
+            } else {
+                // many equal-bucket keys: bitwise search of the rem-th largest member key, then block ids
+                uint32_t t = 0u;
+                for (int bit = 31; bit >= 0; --bit) {
+                    const uint32_t probe = t | (1u << bit);
+                    int ge = 0;
+#pragma unroll
+                    for (int e = 0; e < KW; ++e) ge += bk[e] == bstar && key[e] >= probe;
+                    if (warp_count(ge) >= rem) t = probe;
+                }
+                int gt = 0;
+#pragma unroll
+                for (int e = 0; e < KW; ++e) gt += bk[e] == bstar && key[e] > t;
+                const int need = rem - warp_count(gt);
+                // the need-th lowest block id among the members with key t
+                int seen = 0;
+                tidx = -1;
+#pragma unroll
+                for (int e = 0; e < KW; ++e) {
+                    const unsigned eq = __ballot_sync(0xffffffffu, bk[e] == bstar && key[e] == t);
+                    if (tidx < 0 && seen + __popc(eq) >= need) {
+                        unsigned m2 = eq;
+                        for (int j = 0; j < need - seen - 1; ++j) m2 &= m2 - 1u;
+                        tidx = 32 * e + __ffs(m2) - 1;
+                    }
+                    seen += __popc(eq);
+                }
+                tkey = t;
+            }
         }
         __syncwarp();
     }
@@ -328,7 +336,7 @@ struct CtaSelectSmem {
     int red[64];
     int nmem;
     uint32_t kmin, kmax;
-    int bstar, above;          // boundary bucket, candidates in buckets above it
+    int bstar, above, bcount;  // boundary bucket, candidates in buckets above it, candidates in it
     uint32_t thr_key;
     int thr_idx;
 };
@@ -429,6 +437,7 @@ IV2_DEV int cta_select_topk(const float* S, int c, int init, int local, int topk
                 if (acc + cnt_b[j] >= topk) {
                     sm.bstar = kBuckets - 1 - (threadIdx.x * BPT + j);
                     sm.above = acc;
+                    sm.bcount = cnt_b[j];
                     break;
                 }
                 acc += cnt_b[j];
@@ -437,71 +446,78 @@ IV2_DEV int cta_select_topk(const float* S, int c, int init, int local, int topk
         __syncthreads();
         bstar = sm.bstar;
         const int rem = topk - sm.above;  // members of bucket B* still to take, >= 1
-        // stage the members of B*
+        if (sm.bcount == rem) {
+            // the boundary bucket is taken whole (the usual case: its members are few): every candidate in a
+            // bucket >= B* is chosen, with no ranking inside B* (the same for every thread: a uniform branch)
+            tkey = 0u;
+            tidx = 0x7fffffff;
+        } else {
+            // stage the members of B*
 #pragma unroll
-        for (int e = 0; e < E; ++e) {
-            if (key[e] != 0u && bk[e] == bstar) {
-                const int slot = atomicAdd(&sm.nmem, 1);
-                if (slot < kMaxMembers) {
-                    sm.mkey[slot] = key[e];
-                    sm.midx[slot] = b0 + e;
+            for (int e = 0; e < E; ++e) {
+                if (key[e] != 0u && bk[e] == bstar) {
+                    const int slot = atomicAdd(&sm.nmem, 1);
+                    if (slot < kMaxMembers) {
+                        sm.mkey[slot] = key[e];
+                        sm.midx[slot] = b0 + e;
+                    }
                 }
             }
-        }
-        __syncthreads();
-        if (sm.nmem > kRankMembers) {
-            // degenerate spread (e.g. many equal scores): rank the bucket's members CTA-wide
-            int parity = 0;
-            uint32_t t = 0u;
-            for (int bit = 31; bit >= 0; --bit) {
-                const uint32_t probe = t | (1u << bit);
-                int ge = 0;
+            __syncthreads();
+            if (sm.nmem > kRankMembers) {
+                // degenerate spread (e.g. many equal scores): rank the bucket's members CTA-wide
+                int parity = 0;
+                uint32_t t = 0u;
+                for (int bit = 31; bit >= 0; --bit) {
+                    const uint32_t probe = t | (1u << bit);
+                    int ge = 0;
 #pragma unroll
-                for (int e = 0; e < E; ++e)
-                    ge += key[e] != 0u && bk[e] == bstar && key[e] >= probe;
-                if (cta_count<NT>(ge, sm.red, parity) >= rem) t = probe;
+                    for (int e = 0; e < E; ++e)
+                        ge += key[e] != 0u && bk[e] == bstar && key[e] >= probe;
+                    if (cta_count<NT>(ge, sm.red, parity) >= rem) t = probe;
+                    parity ^= 1;
+                }
+                int gt = 0;
+#pragma unroll
+                for (int e = 0; e < E; ++e) gt += key[e] != 0u && bk[e] == bstar && key[e] > t;
+                gt = cta_count<NT>(gt, sm.red, parity);
                 parity ^= 1;
-            }
-            int gt = 0;
+                const int need = rem - gt;
+                int ti = 0;
+                for (int bit = 12; bit >= 0; --bit) {
+                    const int probe = ti | ((1 << bit) - 1);
+                    int le = 0;
 #pragma unroll
-            for (int e = 0; e < E; ++e) gt += key[e] != 0u && bk[e] == bstar && key[e] > t;
-            gt = cta_count<NT>(gt, sm.red, parity);
-            parity ^= 1;
-            const int need = rem - gt;
-            int ti = 0;
-            for (int bit = 12; bit >= 0; --bit) {
-                const int probe = ti | ((1 << bit) - 1);
-                int le = 0;
-#pragma unroll
-                for (int e = 0; e < E; ++e) le += key[e] == t && (b0 + e) <= probe;
-                if (cta_count<NT>(le, sm.red, parity) < need) ti |= 1 << bit;
-                parity ^= 1;
-            }
-            if (threadIdx.x == 0) {
-                sm.thr_key = t;
-                sm.thr_idx = ti;
-            }
-        } else if (warp == 0) {
-            // few members: the rank of member i in (key descending, block ascending) order is the number of
-            // members before it; the one of rank rem-1 is the threshold
-            const int nm = sm.nmem;
-            for (int i = lane; i < nm; i += 32) {
-                const uint32_t ki = sm.mkey[i];
-                const int ii = sm.midx[i];
-                int rank = 0;
-                for (int j = 0; j < nm; ++j) {
-                    const uint32_t kj = sm.mkey[j];
-                    rank += (kj > ki) || (kj == ki && sm.midx[j] < ii);
+                    for (int e = 0; e < E; ++e) le += key[e] == t && (b0 + e) <= probe;
+                    if (cta_count<NT>(le, sm.red, parity) < need) ti |= 1 << bit;
+                    parity ^= 1;
                 }
-                if (rank == rem - 1) {
-                    sm.thr_key = ki;
-                    sm.thr_idx = ii;
+                if (threadIdx.x == 0) {
+                    sm.thr_key = t;
+                    sm.thr_idx = ti;
+                }
+            } else if (warp == 0) {
+                // few members: the rank of member i in (key descending, block ascending) order is the number of
+                // members before it; the one of rank rem-1 is the threshold
+                const int nm = sm.nmem;
+                for (int i = lane; i < nm; i += 32) {
+                    const uint32_t ki = sm.mkey[i];
+                    const int ii = sm.midx[i];
+                    int rank = 0;
+                    for (int j = 0; j < nm; ++j) {
+                        const uint32_t kj = sm.mkey[j];
+                        rank += (kj > ki) || (kj == ki && sm.midx[j] < ii);
+                    }
+                    if (rank == rem - 1) {
+                        sm.thr_key = ki;
+                        sm.thr_idx = ii;
+                    }
                 }
             }
+            __syncthreads();
+            tkey = sm.thr_key;
+            tidx = sm.thr_idx;
         }
-        __syncthreads();
-        tkey = sm.thr_key;
-        tidx = sm.thr_idx;
     }
     // emit ascending (branch-free: a key is 0 for blocks past nb, forced blocks and blocks with no kernel)
     bool chosen[E];
