@@ -124,12 +124,14 @@ def attn_tc_model(m: PipelineModel, U: int, rescale_steps=(), parts: int = 2, mi
 # --------------------------------------------------------------------------------------------------------------
 # score_tc_kernel (csrc/score_tc.cu): two 128-row Q tiles against 128-kernel stages, stages 0..ntiles-1 for the
 # LSE pass and ntiles..2 ntiles-1 for the block maxima.  Warp 0: both Q tiles, then the kernel stages (3-slot
-# ring); warp 1: S(tile) = Q(tile) kern^T per stage; warps 2-9: TMEM readers, two per lane quarter, 64 columns
-# each; the LSE halves meet in shared memory; pass 2 writes the group scores over the Q staging area; then
-# reader warp w selects tokens w - 2 and w + 6.
+# ring); warp 1: S(tile) = Q(tile) kern^T per stage; warps 2-17: TMEM readers, four per lane quarter, 32
+# columns each (pass 2 also reads the column before its first: the previous part's last, or for part 0 the
+# stage's last); the four LSE parts meet in shared memory; pass 2 writes the group scores over the Q staging
+# area; then reader warp w selects token w - 2.
 # --------------------------------------------------------------------------------------------------------------
-def score_tc_model(m: PipelineModel, ntiles: int, mistake: str = ""):
+def score_tc_model(m: PipelineModel, ntiles: int, mistake: str = "", parts: int = 4):
     nq = 2 * ntiles
+    nreaders = 4 * parts
     m.bar("q_full", 1)
     m.bar("q_tmem", 128)
     for i in range(RING):
@@ -137,7 +139,7 @@ def score_tc_model(m: PipelineModel, ntiles: int, mistake: str = ""):
         m.bar(f"k_empty{i}", 1)
     for t in range(2):
         m.bar(f"s_full{t}", 1)
-        m.bar(f"s_empty{t}", 256)
+        m.bar(f"s_empty{t}", 32 * nreaders)
 
     def producer():
         yield ("arrive_tx", "q_full", 1, 2)
@@ -159,14 +161,14 @@ def score_tc_model(m: PipelineModel, ntiles: int, mistake: str = ""):
                 if q >= 1 and mistake != "issuer skips s_empty":
                     yield ("wait", f"s_empty{tile}", q - 1)
                 yield ("mma", [(f"QT{tile}.q{x}", "Q") for x in range(4)] + [(f"kern{s}", ("kern", q))],
-                       [(f"S{tile}.q{x}.h{h}", ("S", q)) for x in range(4) for h in range(2)], f"S{tile}.{q}")
+                       [(f"S{tile}.q{x}.p{h}", ("S", q)) for x in range(4) for h in range(parts)], f"S{tile}.{q}")
                 yield ("commit", f"s_full{tile}")
             yield ("commit", f"k_empty{s}")
 
     def reader(w):
-        q4, half = w & 3, (w - 2) >> 2
+        q4, part = w & 3, (w - 2) >> 2
         yield ("wait", "q_full", 0)
-        if half == 0:
+        if part == 0:
             yield ("read", "area", "Q")
             yield ("read", "area2", "Q")
             yield ("write", f"QT0.q{q4}", "Q")
@@ -175,34 +177,30 @@ def score_tc_model(m: PipelineModel, ntiles: int, mistake: str = ""):
         for q in range(nq):
             for tile in range(2):
                 yield ("wait", f"s_full{tile}", q)
-                yield ("read", f"S{tile}.q{q4}.h{half}", ("S", q))
-                if q >= ntiles and half == 1:
-                    yield ("read", f"S{tile}.q{q4}.h0", ("S", q))  # the column before this half's first
+                yield ("read", f"S{tile}.q{q4}.p{part}", ("S", q))
+                if q >= ntiles:
+                    yield ("read", f"S{tile}.q{q4}.p{(part - 1) % parts}", ("S", q))
                 yield ("arrive", f"s_empty{tile}", 32)
                 if q >= ntiles:  # group scores over the Q staging area
                     yield ("write", "area", "S")
-                    yield ("write", f"Ssm.t{8 * tile + 2 * q4}.s{q}.h{half}", "S")  # this stage's blocks
+                    for tok in (8 * tile + 2 * q4, 8 * tile + 2 * q4 + 1):
+                        yield ("write", f"Ssm.t{tok}.s{q}.p{part}", "S")  # this stage's blocks of the part
             if q == ntiles - 1:
-                if half == 1:
-                    yield ("write", f"hm.q{q4}", "m")
+                yield ("write", f"hm.q{q4}.p{part}", "m")
                 if mistake != "no barrier in the LSE exchange":
-                    yield ("nbar", 1, 8)
-                if half == 0:
-                    yield ("read", f"hm.q{q4}", "m")
-                    yield ("write", f"lse.q{q4}", "lse")
-                yield ("nbar", 1, 8)
-                yield ("read", f"lse.q{q4}", "lse")
+                    yield ("nbar", 1, nreaders)
+                for k in range(parts):
+                    yield ("read", f"hm.q{q4}.p{k}", "m")
         if mistake != "no barrier before the select":
-            yield ("nbar", 1, 8)
-        for k2 in range(2):
-            ts = w - 2 + 8 * k2  # Ssm rows are written per lane-quarter pair of tokens
-            for q in range(ntiles, nq):
-                for h in range(2):
-                    yield ("read", f"Ssm.t{ts - ts % 2}.s{q}.h{h}", "S")
+            yield ("nbar", 1, nreaders)
+        ts = w - 2
+        for q in range(ntiles, nq):
+            for h in range(parts):
+                yield ("read", f"Ssm.t{ts}.s{q}.p{h}", "S")
 
     m.role("producer", producer())
     m.role("issuer", issuer())
-    for w in range(2, 10):
+    for w in range(2, 2 + nreaders):
         m.role(f"reader{w}", reader(w))
 
 

@@ -15,9 +15,9 @@
 //   pass 1: LSE of every row (online max / sum of 2^z, scores in log2 units);
 //   pass 2: block maxima from the same scores, 2^(max - LSE), summed over the 16 heads of a token by
 //           warp shuffles (a token's rows are 16 consecutive lanes) into S in shared memory.
-// Then each reader warp selects the blocks of two tokens (warp_select_topk_hist).
-// Warp roles: warp 0 issues the TMA loads, warp 1 (one thread) issues the MMAs, warps 2-9 read TMEM: one
-// lane of each tile per thread, each of a warp pair taking one 64-column half of the 128 kernels.  The
+// Then each reader warp selects the blocks of one token (warp_select_topk_hist).
+// Warp roles: warp 0 issues the TMA loads, warp 1 (one thread) issues the MMAs, warps 2-17 read TMEM: one
+// lane of each tile per thread, the four warps of a lane quarter each taking 32 of the 128 kernels.  The
 // readers hand a stage's accumulators back right after loading them, so the next stage's MMAs overlap
 // their arithmetic.  Every wait is bounded: after the limit the CTA records an error (g_score_tc_error)
 // and skips its work.
@@ -36,8 +36,9 @@ constexpr int kSTile = 8;            // tokens per 128-row tile
 constexpr int kSTok = 2 * kSTile;    // tokens per CTA
 constexpr int kSG = 16;              // heads per KV group
 constexpr int kSD = 128;             // head dim
-constexpr int kSThreads = 320;       // 10 warps
-constexpr int kSEpiThreads = 256;    // warps 2..9
+constexpr int kSThreads = 576;       // 18 warps
+constexpr int kSParts = 4;           // reader warps per TMEM lane quarter
+constexpr int kSEpiThreads = 128 * kSParts;  // warps 2..17
 constexpr int kSRing = 3;
 constexpr int kSSlot = 32768;        // 128 kernel rows x 128 dims: two 64-dim atoms of 16 KB
 constexpr int kSMaxNb = 1024;        // context blocks (64K keys)
@@ -52,9 +53,9 @@ struct SLayout {
     __host__ __device__ explicit SLayout(int nb_max)
     {
         s_bytes = kSTok * nb_max * 4;
-        lse_off = kSQOff + (s_bytes > kSQBytes ? s_bytes : kSQBytes);  // [256] LSE, [256] max, [256] sum
-        ws_off = lse_off + 3 * 256 * 4;                                  // per reader warp: WarpSelectSmem
-        bytes = ws_off + 8 * (int)sizeof(WarpSelectSmem) + 1024;          // + alignment slack
+        lse_off = kSQOff + (s_bytes > kSQBytes ? s_bytes : kSQBytes);  // [parts][256] max, [parts][256] sum
+        ws_off = lse_off + 2 * kSParts * 256 * 4;                        // per reader warp: WarpSelectSmem
+        bytes = ws_off + 4 * kSParts * (int)sizeof(WarpSelectSmem) + 1024;  // + alignment slack
     }
 };
 
@@ -77,11 +78,11 @@ __device__ __forceinline__ bool swait(uint64_t* bar, uint32_t parity, volatile i
     return false;
 }
 
-// 64 scores of this thread's half of one row, scaled to log2 units; kernels at or past nkv are -inf
-IV2_DEV void scaled_row(const uint32_t (&v)[64], int j0, int nkv, float sl2, float (&z)[64])
+// 32 scores of this thread's part of one row, scaled to log2 units; kernels at or past nkv are -inf
+IV2_DEV void scaled_row(const uint32_t (&v)[32], int j0, int nkv, float sl2, float (&z)[32])
 {
 #pragma unroll
-    for (int c = 0; c < 64; ++c) z[c] = j0 + c < nkv ? __uint_as_float(v[c]) * sl2 : neg_inf();
+    for (int c = 0; c < 32; ++c) z[c] = j0 + c < nkv ? __uint_as_float(v[c]) * sl2 : neg_inf();
 }
 
 }  // namespace
@@ -98,9 +99,8 @@ score_tc_kernel(QueryRows qr, const __grid_constant__ CUtensorMap tm_q, const __
     __shared__ SBars bars;
     const SLayout lay(nb_max);
     float* Ssm = reinterpret_cast<float*>(smem + kSQOff);  // after Q has gone to TMEM
-    float* lse_sm = reinterpret_cast<float*>(smem + lay.lse_off);
-    float* hm_sm = lse_sm + 256;
-    float* hs_sm = hm_sm + 256;
+    float* hm_sm = reinterpret_cast<float*>(smem + lay.lse_off);  // [part][tile * 128 + row]
+    float* hs_sm = hm_sm + kSParts * 256;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int T = qr.T;
@@ -208,8 +208,8 @@ score_tc_kernel(QueryRows qr, const __grid_constant__ CUtensorMap tm_q, const __
             }
         }
     } else {
-        // ---------------- TMEM readers: lane r of both tiles per thread, one 64-column half per warp ----------------
-        const int q4 = warp & 3, half = (warp - 2) >> 2;
+        // ---------------- TMEM readers: lane r of both tiles per thread, 32 columns per warp ----------------
+        const int q4 = warp & 3, part = (warp - 2) >> 2;
         const int r = q4 * 32 + lane;  // row = token * 16 + head within a tile
         const uint32_t lane_addr = tmem + ((uint32_t)(q4 * 32) << 16);
         const float sl2 = mc.scale * kLog2e;
@@ -225,7 +225,7 @@ score_tc_kernel(QueryRows qr, const __grid_constant__ CUtensorMap tm_q, const __
             c_t[tile] = n > 0 ? (n - 1) / kBlock : -1;
         }
         bool ok = swait(&bars.q_full, 0, err);
-        if (half == 0) {
+        if (part == 0) {
             // row r of both Q tiles (swizzled smem from TMA) -> TMEM columns [kSColQ + 64 tile, +64) as bf16 pairs
 #pragma unroll
             for (int tile = 0; tile < 2; ++tile)
@@ -253,80 +253,78 @@ score_tc_kernel(QueryRows qr, const __grid_constant__ CUtensorMap tm_q, const __
         constexpr float kFloor = -1e30f;
         float m[2] = {kFloor, kFloor}, s[2] = {0.f, 0.f};
         for (int q = 0; q < ntiles && ok; ++q) {
-            const int j0 = 128 * q + 64 * half;
+            const int j0 = 128 * q + 32 * part;
 #pragma unroll
             for (int tile = 0; tile < 2; ++tile) {
                 ok = __all_sync(0xffffffffu, swait(&bars.s_full[tile], q & 1, err));
                 if (!ok) break;
                 tc::tc_fence_after();
-                uint32_t v[64];
-                tc::tmem_ld32(lane_addr + 128 * tile + 64 * half, *reinterpret_cast<uint32_t(*)[32]>(&v[0]));
-                tc::tmem_ld32(lane_addr + 128 * tile + 64 * half + 32, *reinterpret_cast<uint32_t(*)[32]>(&v[32]));
+                uint32_t v[32];
+                tc::tmem_ld32(lane_addr + 128 * tile + 32 * part, v);
                 tc::tmem_wait_ld();
                 tc::tc_fence_before();
                 tc::mbar_arrive(&bars.s_empty[tile]);
-                float z[64], mx = kFloor;
+                float z[32], mx = kFloor;
                 scaled_row(v, j0, nkv[tile], sl2, z);
 #pragma unroll
-                for (int c = 0; c < 64; ++c) mx = fmaxf(mx, z[c]);
+                for (int c = 0; c < 32; ++c) mx = fmaxf(mx, z[c]);
                 const float mn = fmaxf(m[tile], mx);
                 float acc[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-                for (int c = 0; c < 64; ++c) acc[c & 3] += ex2_approx(z[c] - mn);  // one MUFU op, 2^-inf = 0
+                for (int c = 0; c < 32; ++c) acc[c & 3] += ex2_approx(z[c] - mn);  // one MUFU op, 2^-inf = 0
                 s[tile] = s[tile] * ex2_approx(m[tile] - mn) + ((acc[0] + acc[1]) + (acc[2] + acc[3]));
                 m[tile] = mn;
             }
         }
-        // the two halves of each row -> LSE (named barrier over the 256 reader threads)
-        if (half == 1) {
+        // the four parts of each row -> LSE (every part forms the same value; named barrier over the readers)
 #pragma unroll
-            for (int tile = 0; tile < 2; ++tile) {
-                hm_sm[128 * tile + r] = m[tile];
-                hs_sm[128 * tile + r] = s[tile];
-            }
+        for (int tile = 0; tile < 2; ++tile) {
+            hm_sm[part * 256 + 128 * tile + r] = m[tile];
+            hs_sm[part * 256 + 128 * tile + r] = s[tile];
         }
         tc::named_bar_sync(1, kSEpiThreads);
-        if (half == 0) {
+        float lse_r[2];
 #pragma unroll
-            for (int tile = 0; tile < 2; ++tile) {
-                const float m2 = hm_sm[128 * tile + r], s2 = hs_sm[128 * tile + r];
-                const float M = fmaxf(m[tile], m2);
-                const float sum = s[tile] * exp2_fast(m[tile] - M) + s2 * exp2_fast(m2 - M);
-                lse_sm[128 * tile + r] = (M == kFloor) ? neg_inf() : M + __log2f(sum);
-            }
+        for (int tile = 0; tile < 2; ++tile) {
+            float M = kFloor;
+#pragma unroll
+            for (int k2 = 0; k2 < kSParts; ++k2) M = fmaxf(M, hm_sm[k2 * 256 + 128 * tile + r]);
+            float sum = 0.f;
+#pragma unroll
+            for (int k2 = 0; k2 < kSParts; ++k2)
+                sum += hs_sm[k2 * 256 + 128 * tile + r] * exp2_fast(hm_sm[k2 * 256 + 128 * tile + r] - M);
+            lse_r[tile] = (M == kFloor) ? neg_inf() : M + __log2f(sum);
         }
-        tc::named_bar_sync(1, kSEpiThreads);
-        const float lse_r[2] = {lse_sm[r], lse_sm[128 + r]};
         const bool overlap = mc.membership == 0;
 
         // ---- pass 2: block maxima -> 2^(max - LSE) -> summed over the token's 16 heads -> S ----
-        float prev_last[2] = {neg_inf(), neg_inf()};  // the kernel before this half's first column (half 0)
+        float prev_last[2] = {neg_inf(), neg_inf()};  // part 0: the kernel before its first column
         for (int q = ntiles; q < nq && ok; ++q) {
             const int i = q - ntiles;
-            const int j0 = 128 * i + 64 * half;
+            const int j0 = 128 * i + 32 * part;
 #pragma unroll
             for (int tile = 0; tile < 2; ++tile) {
                 ok = __all_sync(0xffffffffu, swait(&bars.s_full[tile], q & 1, err));
                 if (!ok) break;
                 tc::tc_fence_after();
-                uint32_t v[64];
-                tc::tmem_ld32(lane_addr + 128 * tile + 64 * half, *reinterpret_cast<uint32_t(*)[32]>(&v[0]));
-                tc::tmem_ld32(lane_addr + 128 * tile + 64 * half + 32, *reinterpret_cast<uint32_t(*)[32]>(&v[32]));
-                // half 1: col 63 precedes its first column; half 0: col 127 precedes the next stage's
-                const uint32_t extra = tc::tmem_ld1(lane_addr + 128 * tile + (half ? 63 : 127));
+                uint32_t v[32];
+                tc::tmem_ld32(lane_addr + 128 * tile + 32 * part, v);
+                // parts 1-3: column 32 part - 1 precedes their first column; part 0: column 127 precedes the
+                // next stage's first
+                const uint32_t extra = tc::tmem_ld1(lane_addr + 128 * tile + (part ? 32 * part - 1 : 127));
                 tc::tmem_wait_ld();
                 tc::tc_fence_before();
                 tc::mbar_arrive(&bars.s_empty[tile]);
-                const float halo = half ? (j0 - 1 < nkv[tile] ? __uint_as_float(extra) * sl2 : neg_inf())
+                const float halo = part ? (j0 - 1 < nkv[tile] ? __uint_as_float(extra) * sl2 : neg_inf())
                                         : prev_last[tile];
-                if (half == 0) prev_last[tile] = j0 + 127 < nkv[tile] ? __uint_as_float(extra) * sl2 : neg_inf();
-                float z[64];
+                if (part == 0) prev_last[tile] = j0 + 127 < nkv[tile] ? __uint_as_float(extra) * sl2 : neg_inf();
+                float z[32];
                 scaled_row(v, j0, nkv[tile], sl2, z);
-                // the 16 blocks of this half: 2^(max - LSE) of each, then the sums over the token's 16 heads
-                // (16 independent shuffle chains, interleaved)
-                float e[16];
+                // the 8 blocks of this part: 2^(max - LSE) of each, then the sums over the token's 16 heads
+                // (8 independent shuffle chains, interleaved)
+                float e[8];
 #pragma unroll
-                for (int k = 0; k < 16; ++k) {
+                for (int k = 0; k < 8; ++k) {
                     float bm = overlap ? fmaxf(fmaxf(z[4 * k], z[4 * k + 1]), fmaxf(z[4 * k + 2], z[4 * k + 3]))
                                        : fmaxf(fmaxf(z[4 * k], z[4 * k + 1]), z[4 * k + 2]);
                     if (overlap) bm = fmaxf(bm, k == 0 ? halo : z[4 * k - 1]);
@@ -335,11 +333,11 @@ score_tc_kernel(QueryRows qr, const __grid_constant__ CUtensorMap tm_q, const __
 #pragma unroll
                 for (int o = 1; o < 16; o <<= 1)
 #pragma unroll
-                    for (int k = 0; k < 16; ++k) e[k] += __shfl_xor_sync(0xffffffffu, e[k], o);
+                    for (int k = 0; k < 8; ++k) e[k] += __shfl_xor_sync(0xffffffffu, e[k], o);
                 if ((lane & 15) == 0 && valid[tile]) {
 #pragma unroll
-                    for (int k = 0; k < 16; ++k) {
-                        const int blk = 32 * i + 16 * half + k;
+                    for (int k = 0; k < 8; ++k) {
+                        const int blk = 32 * i + 8 * part + k;
                         // a block scores only when one of its kernels is visible (same rule for every head)
                         int lo, hi;
                         block_kernel_range(blk, mc.membership, lo, hi);
@@ -349,13 +347,11 @@ score_tc_kernel(QueryRows qr, const __grid_constant__ CUtensorMap tm_q, const __
                 }
             }
         }
-        // ---- selection: reader warp w takes tokens w and w + 8 ----
+        // ---- selection: reader warp w takes token w - 2 ----
         tc::named_bar_sync(1, kSEpiThreads);
         ok = __all_sync(0xffffffffu, ok && !*err);
-#pragma unroll 1
-        for (int k2 = 0; k2 < 2 && ok; ++k2) {
-            const int ts = warp - 2 + 8 * k2;
-            if (t0 + ts >= T) break;
+        const int ts = warp - 2;
+        if (ok && t0 + ts < T) {
             const int tsel = t0 + ts;
             const int ns = query_ctx(qr, b, tsel);
             const int cs = (ns - 1) / kBlock;
