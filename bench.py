@@ -536,6 +536,40 @@ class PrefillBench:
                                              self.p, self.out, self.lse, self.dout, self.dq, self.dk, self.dv,
                                              self.bws)
 
+    def lse_estimate_leg(self, strides=(2, 4), reps=5):
+        """Scoring + top-k with the LSE estimated from every s-th visible kernel (lse_stride = s) against the
+        exact scoring of the same kernel cache: the time of one call (mean of `reps`, after two untimed) and the
+        share of sparse (token, group) rows whose selection is unchanged.  The pages name a LogSumExp estimation
+        for fast top-k but do not define it, so this reading's parity with the pages is unpinned."""
+        import dataclasses
+        torch, b = self.torch, self.b
+        self.pool()
+
+        def timed(p, idx, cnt):
+            for _ in range(2):
+                b.infllmv2_block_score_topk(self.q, None, self.lens, self.T, self.kern, p, idx, cnt, self.ws)
+            torch.cuda.synchronize()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            for _ in range(reps):
+                b.infllmv2_block_score_topk(self.q, None, self.lens, self.T, self.kern, p, idx, cnt, self.ws)
+            e1.record()
+            e1.synchronize()
+            return e0.elapsed_time(e1) / reps
+
+        exact_ms = timed(self.p, self.idx, self.cnt)
+        ref_idx, ref_cnt = self.idx.clone(), self.cnt.clone()
+        idx2, cnt2 = torch.empty_like(self.idx), torch.empty_like(self.cnt)
+        t0 = self.p.dense_len  # rows below the dense switch take no selection
+        res = {"exact_ms": exact_ms, "rows": f"tokens {t0}..{self.T - 1} x {HKV} groups",
+               "parity": "unpinned by the pages (the estimate is this library's reading)"}
+        for s in strides:
+            ms = timed(dataclasses.replace(self.p, lse_stride=s), idx2, cnt2)
+            same = ((cnt2 == ref_cnt) & (idx2 == ref_idx).all(-1))[0, t0:]
+            res[f"s{s}"] = {"ms": ms, "time_saved_frac": 1.0 - ms / exact_ms,
+                            "rows_unchanged": float(same.float().mean().item())}
+        return res
+
     def run_backward(self, warmup, steps):
         torch = self.torch
         for _ in range(warmup):
@@ -901,6 +935,9 @@ def run_ours(args):
                          "traffic": NCU_TRAFFIC.get(pdom)},
         }
         line["gpu_launches"] += args.prefill_steps * 3  # kernel pool, scoring + top-k, attention
+        if not args.no_lse_estimate:
+            # untimed for the headline: the scoring call alone at lse_stride 2 and 4, against the exact call
+            line["lse_estimate"] = pb.lse_estimate_leg()
         if not args.no_backward:
             pb.backward_setup()
             bt = barrier_max(pb.run_backward(3, args.prefill_steps), ws)
@@ -1032,6 +1069,7 @@ def main():
     ap.add_argument("--prefill-steps", type=int, default=3)
     ap.add_argument("--no-prefill", action="store_true")
     ap.add_argument("--no-backward", action="store_true", help="skip the prefill gradient pass")
+    ap.add_argument("--no-lse-estimate", action="store_true", help="skip the LSE-estimate scoring leg")
     ap.add_argument("--no-tree", action="store_true", help="skip the tree-verification leg")
     ap.add_argument("--no-decode32k", action="store_true", help="skip the batch-1 32K decode leg")
     ap.add_argument("--no-decode", action="store_true", help="prefill only (for profiling its kernels)")

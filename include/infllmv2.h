@@ -74,6 +74,11 @@ typedef struct {
     int membership;      /* 0 = OVERLAP: kernel j belongs to every block its window intersects;
                             1 = CONTAINED: only to the block that contains its whole window */
     float softmax_scale; /* <= 0 selects 1/sqrt(d); used for kernel scoring and attention */
+    int lse_stride;      /* 0 or 1: exact LSE_h.  2, 4 or 8: the estimate LSE_h ~ log(s * sum of exp z_h(j) over the
+                            visible kernels j = 0, s, 2s, ...), one reading of the LogSumExp estimation the pages
+                            name for fast top-k (QbitAI, "Model architecture: InfLLM v2", item 3; the pages do
+                            not define it).  Only the prefill scoring on the tensor cores (16 heads per group,
+                            d 128) takes it; other scoring paths return INFLLMV2_ERR_UNSUPPORTED */
 } infllmv2_params;
 
 /* Human-readable name of a status code (static storage). */

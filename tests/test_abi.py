@@ -100,6 +100,9 @@ def test_block_score_topk_rejects_bad_arguments(lib):
     assert _score(lib, binding.Params(topk=2**31 - 1)) == INVALID
     assert _score(lib, binding.Params(topk=1, init_blocks=2**30, local_blocks=2**30)) == INVALID
     assert binding.infllmv2_workspace_size(binding.Params(topk=2**31 - 1), 1, 1, 4096, 32, 2, 128) == 0
+    assert _score(lib, binding.Params(lse_stride=-1)) == INVALID
+    assert _score(lib, binding.Params(lse_stride=3)) == UNSUPPORTED
+    assert _score(lib, binding.Params(lse_stride=4)) == UNSUPPORTED  # one query per sequence: the scan path
 
 
 def test_attention_entry_points_reject_bad_arguments(lib):

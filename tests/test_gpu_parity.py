@@ -137,6 +137,28 @@ def test_selection_tile_path_groups(oracle, G, d):
     check_selection(gidx, gcnt, r)
 
 
+@pytest.mark.parametrize("stride", [2, 4, 8])
+def test_selection_lse_estimate_tile_path(oracle, stride):
+    """lse_stride = s on the tensor-core prefill scoring against the oracle's same reading of the pages'
+    LogSumExp estimation (the LSE from every s-th visible kernel, times s; the pages do not define it, so this
+    pins the implementation to the reading, not to the pages): bit-exact selection except at the oracle's near
+    ties.  1,500 tokens (ragged last tile, 24 blocks) and 8,500 (133 blocks: three pass-1 stages at s = 2, one
+    at s = 8)"""
+    for T, seed in ((1500, 980 + stride), (8500, 990 + stride)):
+        w = prefill_case(T, 32, 2, 128, topk=6, dense_len=300, seed=seed, n_needles=3)
+        nk_cap = oracle.num_kernels(T)
+        kern_o = oracle.kernel_pool(w.k, [0], [T], 32, 16, nk_cap=nk_cap)
+        rows = slice(T - 256, T)  # the longest rows: the most pass-1 stages
+        q_ctx = w.q_ctx[:, rows]
+        r = oracle.block_score_topk(w.q[:, rows], kern_o, q_ctx, oparams(dict(w.params, lse_stride=stride)))
+        kern = gpu_pool(w.k, [0], [T], T, nk_cap)
+        gidx, gcnt = gpu_select(w, kern, params=dict(w.params, lse_stride=stride))
+        check_selection(gidx[:, rows], gcnt[:, rows], r)
+        # the exact path on the same inputs differs from the estimate somewhere (the estimate is not a no-op)
+        e_idx, _ = gpu_select(w, kern)
+        assert not np.array_equal(e_idx, gidx)
+
+
 @pytest.mark.parametrize("G,d", [(16, 128), (2, 64), (8, 128)])
 def test_selection_decode_scan_path(oracle, G, d):
     """Decode rows (scan path): ragged lengths, one at the dense threshold, one just past it, one

@@ -33,7 +33,8 @@ class Infllmv2Error(RuntimeError):
 class CParams(ctypes.Structure):
     _fields_ = [("block_size", ctypes.c_int), ("kernel_size", ctypes.c_int), ("kernel_stride", ctypes.c_int),
                 ("topk", ctypes.c_int), ("init_blocks", ctypes.c_int), ("local_blocks", ctypes.c_int),
-                ("dense_len", ctypes.c_int), ("membership", ctypes.c_int), ("softmax_scale", ctypes.c_float)]
+                ("dense_len", ctypes.c_int), ("membership", ctypes.c_int), ("softmax_scale", ctypes.c_float),
+                ("lse_stride", ctypes.c_int)]
 
 
 @dataclass
@@ -48,6 +49,7 @@ class Params:
     dense_len: int = 0
     membership: int = 0
     softmax_scale: float = 0.0
+    lse_stride: int = 0  # 0 / 1: exact LSE; 2, 4, 8: estimated from every s-th kernel (prefill scoring, tensor cores)
 
     @property
     def kmax(self) -> int:
@@ -55,7 +57,8 @@ class Params:
 
     def c(self) -> CParams:
         return CParams(self.block_size, self.kernel_size, self.kernel_stride, self.topk, self.init_blocks,
-                       self.local_blocks, self.dense_len, self.membership, float(self.softmax_scale))
+                       self.local_blocks, self.dense_len, self.membership, float(self.softmax_scale),
+                       int(self.lse_stride))
 
 
 _P = ctypes.c_void_p

@@ -99,6 +99,9 @@ int check_params(const infllmv2_params* p)
     if (!(p->softmax_scale == p->softmax_scale) || std::isinf(p->softmax_scale)) return INFLLMV2_ERR_INVALID_ARG;
     if (p->block_size != iv2::kBlock || p->kernel_size != iv2::kKernelSize || p->kernel_stride != iv2::kKernelStride)
         return INFLLMV2_ERR_UNSUPPORTED;
+    if (p->lse_stride < 0) return INFLLMV2_ERR_INVALID_ARG;
+    if (p->lse_stride > 1 && p->lse_stride != 2 && p->lse_stride != 4 && p->lse_stride != 8)
+        return INFLLMV2_ERR_UNSUPPORTED;
     return INFLLMV2_OK;
 }
 
@@ -113,6 +116,7 @@ MethodConsts consts_of(const infllmv2_params* p, int d)
     mc.scale = p->softmax_scale > 0.f ? p->softmax_scale : 1.0f / std::sqrt((float)d);
     mc.kmax = p->topk + p->init_blocks + p->local_blocks;
     mc.window = 0;
+    mc.lse_stride = p->lse_stride > 1 ? p->lse_stride : 1;
     return mc;
 }
 
@@ -313,6 +317,10 @@ int infllmv2_block_score_topk(const void* q, int batch, int num_q, int hq, int h
     if (nk_cap < 1 || nk_cap < nk_of(max_ctx)) return INFLLMV2_ERR_INVALID_ARG;
     IV2_TRY(check_ws(ws, ws_bytes, score_need(batch, num_q, hq, hkv, head_dim, max_ctx)));
     const QueryRows qr = rows_of(q, batch, num_q, hq, hkv, head_dim, q_ctx, ctx_lens, 0, max_ctx);
+    // the LSE estimate exists on the tensor-core prefill scoring only
+    if (params->lse_stride > 1 && (iv2::score_uses_scan_path(batch, num_q, hq / hkv, head_dim, max_ctx) ||
+                                   !iv2::score_tc_supported(qr, (max_ctx - 1) / iv2::kBlock + 1)))
+        return INFLLMV2_ERR_UNSUPPORTED;
     return launched(iv2::launch_score_topk(qr, kern, nk_cap, consts_of(params, head_dim), idx, cnt, ws,
                                            (cudaStream_t)stream));
 }
@@ -368,6 +376,7 @@ int infllmv2_sparse_decode_step(const void* q, int batch, int hq, int hkv, int h
                                 infllmv2_stream_t stream)
 {
     IV2_TRY(check_params(params));
+    if (params->lse_stride > 1) return INFLLMV2_ERR_UNSUPPORTED;  // the estimate is built for prefill scoring only
     IV2_TRY(check_heads(batch, 1, hq, hkv, head_dim));
     IV2_TRY(check_ptr16(q));
     IV2_TRY(check_ptr16(kern));

@@ -90,6 +90,7 @@ struct MethodConsts {
     float scale;              // softmax scale (natural units)
     int kmax;                 // topk + init + local
     int window;               // > 0: attend to the last `window` keys only (sliding window); 0: off
+    int lse_stride;           // <= 1: exact LSE; s > 1: LSE estimated from every s-th visible kernel
 };
 
 // rows (sequence x query x KV group) one split-attention launch handles

@@ -90,7 +90,8 @@ IV2_DEV void scaled_row(const uint32_t (&v)[32], int j0, int nkv, float sl2, flo
 template <int KW>
 __global__ void __launch_bounds__(kSThreads, 1)
 score_tc_kernel(QueryRows qr, const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_kern,
-                int nk_cap, MethodConsts mc, int nb_max, int32_t* __restrict__ idx, int32_t* __restrict__ cnt)
+                const __grid_constant__ CUtensorMap tm_kern_s, int nk_cap, MethodConsts mc, int nb_max,
+                int32_t* __restrict__ idx, int32_t* __restrict__ cnt)
 {
     pdl_launch_dependents();
     pdl_wait();
@@ -127,7 +128,10 @@ score_tc_kernel(QueryRows qr, const __grid_constant__ CUtensorMap tm_q, const __
     }
     const int nb = min((n_max - 1) / kBlock + 1, nb_max);
     const int ntiles = (nb + 31) / 32;  // 32 blocks (128 kernels) per stage
-    const int nq = 2 * ntiles;           // stages over both passes
+    // pass 1 reads every ls-th kernel (ls = 1: all of them) through tm_kern_s, 128 per stage
+    const int ls = mc.lse_stride > 1 ? mc.lse_stride : 1;
+    const int n1 = (nb + 32 * ls - 1) / (32 * ls);
+    const int nq = n1 + ntiles;          // stages over both passes
 
     if (threadIdx.x == 0) {
         bars.err = 0;
@@ -158,6 +162,7 @@ score_tc_kernel(QueryRows qr, const __grid_constant__ CUtensorMap tm_q, const __
         if (lane == 0) {
             tc::prefetch_tensormap(&tm_q);
             tc::prefetch_tensormap(&tm_kern);
+            if (ls > 1) tc::prefetch_tensormap(&tm_kern_s);
             tc::mbar_arrive_expect_tx(&bars.q_full, kSQBytes);
 #pragma unroll
             for (int tile = 0; tile < 2; ++tile) {
@@ -170,10 +175,12 @@ score_tc_kernel(QueryRows qr, const __grid_constant__ CUtensorMap tm_q, const __
                 const int s = q % kSRing, k = q / kSRing;
                 if (k >= 1 && !swait(&bars.k_empty[s], (k - 1) & 1, err)) break;
                 unsigned char* st = smem + s * kSSlot;
-                const int row0 = (q % ntiles) * 128;
+                // pass 1: rows 128 q .. of the strided view (kernels ls * row); pass 2: kernels 128 (q - n1) ..
+                const CUtensorMap* map = q < n1 ? &tm_kern_s : &tm_kern;
+                const int row0 = (q < n1 ? q : q - n1) * 128;
                 tc::mbar_arrive_expect_tx(&bars.k_full[s], kSSlot);
-                tc::tma_load_3d(st, &tm_kern, 0, row0, zk, &bars.k_full[s]);
-                tc::tma_load_3d(st + 16384, &tm_kern, 64, row0, zk, &bars.k_full[s]);
+                tc::tma_load_3d(st, map, 0, row0, zk, &bars.k_full[s]);
+                tc::tma_load_3d(st + 16384, map, 64, row0, zk, &bars.k_full[s]);
             }
         }
     } else if (warp == 1) {
@@ -252,8 +259,8 @@ score_tc_kernel(QueryRows qr, const __grid_constant__ CUtensorMap tm_q, const __
         // ---- pass 1: LSE of both rows over their visible kernels (finite floor: no inf - inf) ----
         constexpr float kFloor = -1e30f;
         float m[2] = {kFloor, kFloor}, s[2] = {0.f, 0.f};
-        for (int q = 0; q < ntiles && ok; ++q) {
-            const int j0 = 128 * q + 32 * part;
+        for (int q = 0; q < n1 && ok; ++q) {
+            const int i0 = 128 * q + 32 * part;  // strided rows: column c is kernel ls * (i0 + c)
 #pragma unroll
             for (int tile = 0; tile < 2; ++tile) {
                 ok = __all_sync(0xffffffffu, swait(&bars.s_full[tile], q & 1, err));
@@ -265,7 +272,8 @@ score_tc_kernel(QueryRows qr, const __grid_constant__ CUtensorMap tm_q, const __
                 tc::tc_fence_before();
                 tc::mbar_arrive(&bars.s_empty[tile]);
                 float z[32], mx = kFloor;
-                scaled_row(v, j0, nkv[tile], sl2, z);
+                // visible: ls * (i0 + c) < nkv, i.e. i0 + c < ceil(nkv / ls)
+                scaled_row(v, i0, (nkv[tile] + ls - 1) / ls, sl2, z);
 #pragma unroll
                 for (int c = 0; c < 32; ++c) mx = fmaxf(mx, z[c]);
                 const float mn = fmaxf(m[tile], mx);
@@ -293,14 +301,15 @@ score_tc_kernel(QueryRows qr, const __grid_constant__ CUtensorMap tm_q, const __
 #pragma unroll
             for (int k2 = 0; k2 < kSParts; ++k2)
                 sum += hs_sm[k2 * 256 + 128 * tile + r] * exp2_fast(hm_sm[k2 * 256 + 128 * tile + r] - M);
-            lse_r[tile] = (M == kFloor) ? neg_inf() : M + __log2f(sum);
+            // the estimate scales the strided sum by ls (ls = 1: exact)
+            lse_r[tile] = (M == kFloor) ? neg_inf() : M + __log2f(sum * (float)ls);
         }
         const bool overlap = mc.membership == 0;
 
         // ---- pass 2: block maxima -> 2^(max - LSE) -> summed over the token's 16 heads -> S ----
         float prev_last[2] = {neg_inf(), neg_inf()};  // part 0: the kernel before its first column
-        for (int q = ntiles; q < nq && ok; ++q) {
-            const int i = q - ntiles;
+        for (int q = n1; q < nq && ok; ++q) {
+            const int i = q - n1;
             const int j0 = 128 * i + 32 * part;
 #pragma unroll
             for (int tile = 0; tile < 2; ++tile) {
@@ -384,30 +393,37 @@ bool score_tc_supported(const QueryRows& qr, int nb_max)
 }
 
 template <int KW>
-static cudaError_t score_tc_launch(const CUtensorMap& tq, const CUtensorMap& tk, const QueryRows& qr, int nk_cap,
-                                   const MethodConsts& mc, int nb_max, int32_t* idx, int32_t* cnt, cudaStream_t s)
+static cudaError_t score_tc_launch(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tks,
+                                   const QueryRows& qr, int nk_cap, const MethodConsts& mc, int nb_max, int32_t* idx,
+                                   int32_t* cnt, cudaStream_t s)
 {
     const SLayout lay(nb_max);
     cudaError_t e = ensure_smem(score_tc_kernel<KW>, lay.bytes);
     if (e != cudaSuccess) return e;
     const dim3 grid((qr.T + kSTok - 1) / kSTok, qr.B * qr.Hkv);
-    return launch_pdl(score_tc_kernel<KW>, grid, dim3(kSThreads), (size_t)lay.bytes, s, qr, tq, tk, nk_cap, mc, nb_max,
-                      idx, cnt);
+    return launch_pdl(score_tc_kernel<KW>, grid, dim3(kSThreads), (size_t)lay.bytes, s, qr, tq, tk, tks, nk_cap, mc,
+                      nb_max, idx, cnt);
 }
 
 cudaError_t launch_score_tc(const QueryRows& qr, const void* kern, int nk_cap, const MethodConsts& mc, int nb_max,
                             int32_t* idx, int32_t* cnt, cudaStream_t s)
 {
     if (!score_tc_supported(qr, nb_max)) return cudaErrorNotSupported;
-    CUtensorMap tq, tk;
+    CUtensorMap tq, tk, tks;
     const uint64_t row = (uint64_t)kSD * 2;
     if (!make_tma_map_bf16(&tq, qr.q, kSD, qr.Hq, (uint64_t)qr.B * qr.T, row, row * qr.Hq, kSG, kSTile) ||
         !make_tma_map_bf16(&tk, kern, kSD, (uint64_t)nk_cap, (uint64_t)qr.B * qr.Hkv, row, row * nk_cap, 128, 1))
         return cudaErrorNotSupported;
+    // the LSE estimate's view: every ls-th kernel row (row stride ls rows; rows past nk_cap are outside the map)
+    const int ls = mc.lse_stride > 1 ? mc.lse_stride : 1;
+    if (ls == 1) tks = tk;
+    else if (!make_tma_map_bf16(&tks, kern, kSD, (uint64_t)(nk_cap + ls - 1) / ls, (uint64_t)qr.B * qr.Hkv, row * ls,
+                                row * nk_cap, 128, 1))
+        return cudaErrorNotSupported;
     // keys per lane of the warp select: nb_max <= 32 KW
-    if (nb_max <= 256) return score_tc_launch<8>(tq, tk, qr, nk_cap, mc, nb_max, idx, cnt, s);
-    if (nb_max <= 512) return score_tc_launch<16>(tq, tk, qr, nk_cap, mc, nb_max, idx, cnt, s);
-    return score_tc_launch<32>(tq, tk, qr, nk_cap, mc, nb_max, idx, cnt, s);
+    if (nb_max <= 256) return score_tc_launch<8>(tq, tk, tks, qr, nk_cap, mc, nb_max, idx, cnt, s);
+    if (nb_max <= 512) return score_tc_launch<16>(tq, tk, tks, qr, nk_cap, mc, nb_max, idx, cnt, s);
+    return score_tc_launch<32>(tq, tk, tks, qr, nk_cap, mc, nb_max, idx, cnt, s);
 }
 
 int score_tc_error_flag_read_and_clear()
