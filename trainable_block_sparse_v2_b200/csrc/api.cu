@@ -250,8 +250,9 @@ int infllmv2_device_status(void)
     const int f = iv2::tc_error_flag_read_and_clear();
     const int h = iv2::fused_error_flag_read_and_clear();
     const int sc = iv2::score_tc_error_flag_read_and_clear();
-    if (f < 0 || h < 0 || sc < 0) return INFLLMV2_ERR_CUDA;
-    return (f || h || sc) ? INFLLMV2_ERR_TIMEOUT : INFLLMV2_OK;
+    const int bw = iv2::bwd_tc_error_flag_read_and_clear();
+    if (f < 0 || h < 0 || sc < 0 || bw < 0) return INFLLMV2_ERR_CUDA;
+    return (f || h || sc || bw) ? INFLLMV2_ERR_TIMEOUT : INFLLMV2_OK;
 }
 
 size_t infllmv2_workspace_size(const infllmv2_params* params, int batch, int max_q, int max_ctx, int hq, int hkv,

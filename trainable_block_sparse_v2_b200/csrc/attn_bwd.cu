@@ -634,13 +634,18 @@ cudaError_t bwd_impl(const QueryRows& qr, const void* k, const void* v, int Lcap
     e = launch_pdl(bwd_fill_kernel, dim3(row_grid), dim3(kBwdRowWarps * 32), 0, s, qr, idx, cnt, mc, dense_flag, w.nb,
                    cursor, tokens, w.cap);
     if (e != cudaSuccess) return e;
-    const size_t dq_smem = (size_t)DqSmem<D>::kBytes;
-    e = ensure_smem(bwd_dq_kernel<D>, dq_smem);
-    if (e != cudaSuccess) return e;
-    const unsigned dq_grid = (unsigned)((rows + kDqWarps - 1) / kDqWarps);
-    e = launch_pdl(bwd_dq_kernel<D>, dim3(dq_grid), dim3(kDqWarps * 32), dq_smem, s, qr,
-                   static_cast<const __nv_bfloat16*>(k), static_cast<const __nv_bfloat16*>(v), Lcap, idx, cnt, mc,
-                   dense_flag, lse, static_cast<const float*>(dsum), static_cast<const __nv_bfloat16*>(dout), dq);
+    e = cudaErrorNotSupported;
+    if (D == 128 && bwd_dq_tc_supported(qr))
+        e = launch_bwd_dq_tc(qr, k, v, Lcap, idx, cnt, mc, dense_all, lse, dsum, dout, dq, s);
+    if (e == cudaErrorNotSupported) {  // other shapes: the mma.sync kernel
+        const size_t dq_smem = (size_t)DqSmem<D>::kBytes;
+        e = ensure_smem(bwd_dq_kernel<D>, dq_smem);
+        if (e != cudaSuccess) return e;
+        const unsigned dq_grid = (unsigned)((rows + kDqWarps - 1) / kDqWarps);
+        e = launch_pdl(bwd_dq_kernel<D>, dim3(dq_grid), dim3(kDqWarps * 32), dq_smem, s, qr,
+                       static_cast<const __nv_bfloat16*>(k), static_cast<const __nv_bfloat16*>(v), Lcap, idx, cnt, mc,
+                       dense_flag, lse, static_cast<const float*>(dsum), static_cast<const __nv_bfloat16*>(dout), dq);
+    }
     if (e != cudaSuccess) return e;
     e = ensure_smem(bwd_dkdv_kernel<D>, DkvSmem<D>::kBytes);
     if (e != cudaSuccess) return e;

@@ -1,0 +1,400 @@
+// attn_bwd_tc.cu -- dq of the block-sparse attention backward on the 5th-generation tensor cores.
+//
+// Same definition as attn_bwd.cu (the derivative of the forward's definition for a fixed selection; "Tsinghua
+// & ModelBest: MiniCPM4 technical details", "Model architecture: InfLLM v2", item 3: the operators serve
+// training as well as inference).  For a row (token t, head h) with key set K(t):
+//   p_e = 2^(scale log2e q.k_e - lse log2e),  ds_e = p_e (dout . v_e - Dsum),  dq = scale sum_e ds_e k_e.
+// Specialised for 16 query heads per KV group and head_dim 128.
+//
+// One CTA owns a 128-row tile (8 consecutive tokens x the 16 heads of one KV group) and walks the ascending
+// union of its tokens' block sets, one 64-key block per step (a token reads a block only when it selected
+// it; the other rows are masked for that block).  Per step:
+//   S  [128 x 64]  = Q  . K^T      tcgen05.mma, A (Q) in TMEM, B (K) K-major in 128B-swizzled smem
+//   dP [128 x 64]  = dO . V^T      the same with dO and V
+//   dS             = P (dP - Dsum) eight warps, one TMEM lane (row) per thread, 32 keys each; dS goes back
+//                                  to TMEM as bf16 pairs over its own S buffer
+//   dQ [128 x 128] += dS . K       A (dS) in TMEM, B (K) MN-major in smem, dQ in TMEM
+// S and dP are double-buffered, so the products of step p + 1 run while the warps form dS of step p.  No
+// online softmax is needed: the forward's lse normalises every step directly.
+// Warp roles: warp 0 loads Q and dO once and K per step, warp 10 loads V per step (TMA, one lane each, 3-deep
+// rings), warp 1 (one thread) issues the MMAs, warps 2-9 form dS and write dq.  Every wait is bounded: after
+// the limit the CTA records an error (g_bwd_tc_error), skips the rest of its work, frees its TMEM and exits.
+#include "common.cuh"
+#include "internal.h"
+#include "tc.cuh"
+
+namespace iv2 {
+
+__device__ int g_bwd_tc_error = 0;
+
+namespace {
+
+constexpr int kTok = 8;         // tokens per tile
+constexpr int kG = 16;          // heads per KV group
+constexpr int kD = 128;         // head dim
+constexpr int kThreads = 352;   // 11 warps
+constexpr int kMaxBlk = 4096;   // context blocks (256K keys)
+constexpr int kWords = kMaxBlk / 32;
+constexpr int kRing = 3;
+constexpr int kSlot = 16384;    // one 64-key block of K or V: two d-halves x 64 rows x 128 B
+constexpr int kKOff = 0;
+constexpr int kVOff = kKOff + kRing * kSlot;
+constexpr int kQOff = kVOff + kRing * kSlot;   // Q tile: two d-halves x 128 rows x 128 B
+constexpr int kDoOff = kQOff + 32768;          // dO tile, same layout
+constexpr int kBitsOff = kDoOff + 32768;       // [kTok][kWords] uint32
+constexpr int kListOff = kBitsOff + kTok * kWords * 4;  // uint16 block ids
+constexpr int kSmemBytes = kListOff + kMaxBlk * 2 + 1024;  // + alignment slack
+// TMEM: dQ [0,128), S [128,256) (two 64-column buffers), dP [256,384) (two), Q [384,448), dO [448,512)
+constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kColS = 128, kColDP = 256, kColQ = 384, kColDO = 448;
+
+struct Bars {
+    uint64_t qd_full, qd_tmem;
+    uint64_t k_full[kRing], k_empty[kRing], v_full[kRing], v_empty[kRing];
+    uint64_t s_full[2], ds_full[2], dq_done[2];
+    uint32_t tmem_base;
+    int n_union;
+    int err;
+};
+
+__device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity, volatile int* err)
+{
+    for (uint32_t i = 0; i < (1u << 22); ++i) {
+        if (tc::mbar_try_wait(bar, parity)) return true;
+        if ((i & 255u) == 255u && *err) return false;
+    }
+    *err = 1;
+    atomicOr(&g_bwd_tc_error, 1);
+    return false;
+}
+
+}  // namespace
+
+__global__ void __launch_bounds__(kThreads, 1)
+bwd_dq_tc_kernel(QueryRows qr, const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_do,
+                 const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v, int Lcap,
+                 const int32_t* __restrict__ idx, const int32_t* __restrict__ cnt, MethodConsts mc, int dense_all,
+                 const float* __restrict__ lse, const float* __restrict__ dsum, float* __restrict__ dq)
+{
+    pdl_launch_dependents();
+    pdl_wait();
+    extern __shared__ unsigned char smem_raw[];
+    unsigned char* smem = tc::align_smem_1024(smem_raw);
+    __shared__ Bars bars;
+    uint32_t* bits = reinterpret_cast<uint32_t*>(smem + kBitsOff);
+    uint16_t* list = reinterpret_cast<uint16_t*>(smem + kListOff);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int T = qr.T;
+    const int g = blockIdx.y % qr.Hkv, b = blockIdx.y / qr.Hkv;
+    const int t0 = (gridDim.x - 1 - blockIdx.x) * kTok;  // longest tiles first
+
+    // ---- union of the tile's block sets, as one bitmap per token and an ascending list ----
+    int cmax = 0;
+#pragma unroll
+    for (int tt = 0; tt < kTok; ++tt)
+        if (t0 + tt < T) cmax = max(cmax, (query_ctx(qr, b, t0 + tt) - 1) / kBlock);
+    const int nwords = min(cmax / 32 + 1, kWords);
+    for (int i = threadIdx.x; i < kTok * kWords; i += kThreads) bits[i] = 0u;
+    if (threadIdx.x == 0) {
+        bars.err = 0;
+        bars.n_union = 0;
+    }
+    __syncthreads();
+    for (int item = threadIdx.x; item < kTok * max(mc.kmax, nwords); item += kThreads) {
+        const int tt = item % kTok, e = item / kTok;
+        const int t = t0 + tt;
+        if (t >= T) continue;
+        const int n = query_ctx(qr, b, t);
+        const int c = (n - 1) / kBlock;
+        if (dense_all || n <= mc.dense_len) {
+            if (e < nwords) {  // every block 0..c
+                const int lo = e * 32, hi = min(c + 1, lo + 32);
+                if (hi > lo) bits[tt * kWords + e] = (hi - lo == 32) ? 0xffffffffu : ((1u << (hi - lo)) - 1u);
+            }
+        } else if (e < mc.kmax) {
+            const size_t row = ((size_t)b * T + t) * qr.Hkv + g;
+            if (e < min(cnt[row], mc.kmax)) {
+                const int blk = idx[row * mc.kmax + e];
+                if (blk >= 0 && blk * kBlock < n) atomicOr(&bits[tt * kWords + (blk >> 5)], 1u << (blk & 31));
+            }
+        }
+    }
+    __syncthreads();
+    if (warp == 0) {
+        int base = 0;
+        for (int w0 = 0; w0 < nwords; w0 += 32) {
+            const int w = w0 + lane;
+            uint32_t u = 0u;
+            if (w < nwords)
+#pragma unroll
+                for (int tt = 0; tt < kTok; ++tt) u |= bits[tt * kWords + w];
+            const int cntw = __popc(u);
+            int incl = cntw;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int y = __shfl_up_sync(0xffffffffu, incl, o);
+                if (lane >= o) incl += y;
+            }
+            int pos = base + incl - cntw;
+            while (u) {
+                const int bit = __ffs(u) - 1;
+                list[pos++] = (uint16_t)(w * 32 + bit);
+                u &= u - 1u;
+            }
+            base += __shfl_sync(0xffffffffu, incl, 31);
+        }
+        if (lane == 0) bars.n_union = base;
+    }
+    if (threadIdx.x == 0) {
+        tc::mbar_init(&bars.qd_full, 1);
+        tc::mbar_init(&bars.qd_tmem, 128);
+        for (int i = 0; i < kRing; ++i) {
+            tc::mbar_init(&bars.k_full[i], 1);
+            tc::mbar_init(&bars.k_empty[i], 1);
+            tc::mbar_init(&bars.v_full[i], 1);
+            tc::mbar_init(&bars.v_empty[i], 1);
+        }
+        for (int i = 0; i < 2; ++i) {
+            tc::mbar_init(&bars.s_full[i], 1);
+            tc::mbar_init(&bars.ds_full[i], 256);
+            tc::mbar_init(&bars.dq_done[i], 1);
+        }
+        tc::fence_barrier_init();
+    }
+    if (warp == 1) {
+        tc::tmem_alloc(&bars.tmem_base, kTmemCols);
+        tc::tmem_relinquish();
+    }
+    tc::tc_fence_before();
+    __syncthreads();
+    tc::tc_fence_after();
+    const int U = bars.n_union;
+    const uint32_t tmem = bars.tmem_base;
+    volatile int* err = &bars.err;
+    const uint32_t sK = tc::smem_u32(smem + kKOff);
+    const uint32_t sV = tc::smem_u32(smem + kVOff);
+
+    if (warp == 0 || warp == 10) {
+        // ---------------- TMA producers: warp 0 Q, dO once and K per step; warp 10 V per step ----------------
+        if (warp == 0 && lane == 0) {
+            tc::prefetch_tensormap(&tm_q);
+            tc::prefetch_tensormap(&tm_do);
+            tc::prefetch_tensormap(&tm_k);
+            tc::mbar_arrive_expect_tx(&bars.qd_full, 4 * 16384);
+            const int zq = b * T + t0;
+#pragma unroll
+            for (int a = 0; a < 2; ++a) {
+                tc::tma_load_3d(smem + kQOff + a * 16384, &tm_q, 64 * a, g * kG, zq, &bars.qd_full);
+                tc::tma_load_3d(smem + kDoOff + a * 16384, &tm_do, 64 * a, g * kG, zq, &bars.qd_full);
+            }
+            for (int p = 0; p < U; ++p) {
+                const int s = p % kRing, k = p / kRing;
+                if (k >= 1 && !wait_bar(&bars.k_empty[s], (k - 1) & 1, err)) break;
+                unsigned char* st = smem + kKOff + s * kSlot;
+                const int z = b * Lcap + (int)list[p] * kBlock;
+                tc::mbar_arrive_expect_tx(&bars.k_full[s], kSlot);
+                tc::tma_load_3d(st, &tm_k, 0, g, z, &bars.k_full[s]);
+                tc::tma_load_3d(st + 8192, &tm_k, 64, g, z, &bars.k_full[s]);
+            }
+        } else if (warp == 10 && lane == 0) {
+            tc::prefetch_tensormap(&tm_v);
+            for (int p = 0; p < U; ++p) {
+                const int s = p % kRing, k = p / kRing;
+                if (k >= 1 && !wait_bar(&bars.v_empty[s], (k - 1) & 1, err)) break;
+                unsigned char* st = smem + kVOff + s * kSlot;
+                const int z = b * Lcap + (int)list[p] * kBlock;
+                tc::mbar_arrive_expect_tx(&bars.v_full[s], kSlot);
+                tc::tma_load_3d(st, &tm_v, 0, g, z, &bars.v_full[s]);
+                tc::tma_load_3d(st + 8192, &tm_v, 64, g, z, &bars.v_full[s]);
+            }
+        }
+    } else if (warp == 1) {
+        // ---------------- MMA issuer ----------------
+        if (lane == 0 && wait_bar(&bars.qd_tmem, 0, err)) {
+            tc::tc_fence_after();
+            constexpr uint32_t idesc_s = tc::idesc_bf16(128, kBlock, false);
+            constexpr uint32_t idesc_q = tc::idesc_bf16(128, kD, true);
+            for (int p = 0; p <= U; ++p) {
+                if (p < U) {
+                    // S(p) = Q . K^T and dP(p) = dO . V^T into buffers p & 1 (in order after dQ(p - 2), which
+                    // read dS(p - 2) from S buffer p & 1; the warps loaded dP(p - 2) before dS(p - 2) was ready)
+                    const int s = p % kRing, sb = p & 1;
+                    if (!wait_bar(&bars.k_full[s], (p / kRing) & 1, err)) break;
+                    if (!wait_bar(&bars.v_full[s], (p / kRing) & 1, err)) break;
+                    tc::tc_fence_after();
+                    const uint32_t kb = sK + s * kSlot, vb = sV + s * kSlot;
+#pragma unroll
+                    for (int ks = 0; ks < kD / 16; ++ks) {
+                        const uint32_t off = (ks >> 2) * 8192 + (ks & 3) * 32;
+                        tc::mma_bf16_ts(tmem + kColS + kBlock * sb, tmem + kColQ + 8 * ks,
+                                        tc::desc_kmajor_sw128(kb + off), idesc_s, ks > 0);
+                        tc::mma_bf16_ts(tmem + kColDP + kBlock * sb, tmem + kColDO + 8 * ks,
+                                        tc::desc_kmajor_sw128(vb + off), idesc_s, ks > 0);
+                    }
+                    tc::mma_commit(&bars.s_full[sb]);
+                    tc::mma_commit(&bars.v_empty[s]);
+                }
+                if (p >= 1) {
+                    // dQ += dS(v) . K(v), dS(v) in the first 32 columns of S buffer v & 1
+                    const int v = p - 1, db = v & 1, s = v % kRing;
+                    if (!wait_bar(&bars.ds_full[db], (v >> 1) & 1, err)) break;
+                    tc::tc_fence_after();
+                    const uint32_t kb = sK + s * kSlot;
+#pragma unroll
+                    for (int ks = 0; ks < kBlock / 16; ++ks)
+                        tc::mma_bf16_ts(tmem, tmem + kColS + kBlock * db + 8 * ks,
+                                        tc::desc_mnmajor_sw128(kb + ks * 2048, 8192), idesc_q, (v > 0 || ks > 0));
+                    tc::mma_commit(&bars.dq_done[db]);
+                    tc::mma_commit(&bars.k_empty[s]);
+                }
+            }
+        }
+    } else {
+        // ---------------- dS and dq: one TMEM lane (query row) per thread, 32 keys of each step ----------------
+        // warps w and w + 4 (2 <= w <= 5) share the lane quarter w & 3: half 0 takes keys 0..31 of the block,
+        // half 1 keys 32..63; they meet at a named barrier of their own on every step before dS overwrites S
+        const int q4 = warp & 3, half = (warp - 2) >> 2;
+        const int r = q4 * 32 + lane;  // row = token * 16 + head
+        const int tt = r >> 4, hh = r & 15;
+        const int t = t0 + tt;
+        const bool valid = t < T;
+        const int n = valid ? query_ctx(qr, b, t) : 0;
+        const uint32_t lane_addr = tmem + ((uint32_t)(q4 * 32) << 16);
+        const uint32_t pair_bar = 1 + q4;
+        const float sl2 = mc.scale * kLog2e;
+        const size_t head = ((size_t)b * T + (valid ? t : 0)) * qr.Hq + g * kG + hh;
+        float lse2 = __int_as_float(0x7f800000), dd = 0.f;  // +inf: this row's p is 0
+        if (valid) {
+            const float lv = lse[head];
+            if (lv > neg_inf() && lv < __int_as_float(0x7f800000)) lse2 = lv * kLog2e;
+            dd = dsum[head];
+        }
+        bool ok = wait_bar(&bars.qd_full, 0, err);
+        if (half == 0) {
+            // this row of Q and of dO (swizzled smem from TMA) -> TMEM as bf16 pairs
+#pragma unroll
+            for (int m2 = 0; m2 < 2; ++m2)
+#pragma unroll
+                for (int a = 0; a < 2; ++a) {
+                    uint32_t w[32];
+                    const unsigned char* src = smem + (m2 ? kDoOff : kQOff) + a * 16384 + r * 128;
+#pragma unroll
+                    for (int c = 0; c < 8; ++c) {
+                        const uint4 v4 = *reinterpret_cast<const uint4*>(src + ((c ^ (r & 7)) << 4));
+                        w[4 * c] = v4.x;
+                        w[4 * c + 1] = v4.y;
+                        w[4 * c + 2] = v4.z;
+                        w[4 * c + 3] = v4.w;
+                    }
+                    tc::tmem_st32(lane_addr + (m2 ? kColDO : kColQ) + 32 * a, w);
+                }
+            tc::tmem_wait_st();
+            tc::tc_fence_before();
+            tc::mbar_arrive(&bars.qd_tmem);
+        }
+        ok = __all_sync(0xffffffffu, ok);
+        for (int p = 0; p < U; ++p) {
+            const int sb = p & 1;
+            if (ok) ok = wait_bar(&bars.s_full[sb], (p >> 1) & 1, err);
+            ok = __all_sync(0xffffffffu, ok);
+            if (ok) tc::tc_fence_after();
+            const int blk = list[p];
+            const bool sel = valid && ((bits[tt * kWords + (blk >> 5)] >> (blk & 31)) & 1u);
+            const int nv = sel ? min(32, n - blk * kBlock - 32 * half) : 0;  // may be <= 0
+            const bool any_sel = __any_sync(0xffffffffu, sel);
+            uint32_t sv[32], pv[32];
+            if (ok && any_sel) {
+                tc::tmem_ld32(lane_addr + kColS + kBlock * sb + 32 * half, sv);
+                tc::tmem_ld32(lane_addr + kColDP + kBlock * sb + 32 * half, pv);
+                tc::tmem_wait_ld();
+            }
+            // both halves' S loads are complete past this barrier, so dS may overwrite S columns 0..31
+            tc::named_bar_sync(pair_bar, 64);
+            if (ok) {
+                uint32_t w[16];
+                if (any_sel) {
+#pragma unroll
+                    for (int j2 = 0; j2 < 16; ++j2) {
+                        const int j = 2 * j2;
+                        const float p0 = j < nv ? ex2_approx(__uint_as_float(sv[j]) * sl2 - lse2) : 0.f;
+                        const float p1 = j + 1 < nv ? ex2_approx(__uint_as_float(sv[j + 1]) * sl2 - lse2) : 0.f;
+                        w[j2] = pack_bf16(p0 * (__uint_as_float(pv[j]) - dd), p1 * (__uint_as_float(pv[j + 1]) - dd));
+                    }
+                } else {
+#pragma unroll
+                    for (int j = 0; j < 16; ++j) w[j] = 0u;
+                }
+                tc::tmem_st16(lane_addr + kColS + kBlock * sb + 16 * half, w);
+                tc::tmem_wait_st();
+                tc::tc_fence_before();
+                tc::mbar_arrive(&bars.ds_full[sb]);
+            }
+        }
+        ok = __all_sync(0xffffffffu, ok);
+        if (ok && U > 0) ok = wait_bar(&bars.dq_done[(U - 1) & 1], ((U - 1) >> 1) & 1, err);
+        ok = __all_sync(0xffffffffu, ok);
+        if (ok) {
+            tc::tc_fence_after();
+            float* drow = dq + head * kD + 64 * half;
+#pragma unroll 1
+            for (int c4 = 0; c4 < 2; ++c4) {
+                uint32_t o[32];
+                tc::tmem_ld32(lane_addr + 64 * half + 32 * c4, o);
+                tc::tmem_wait_ld();
+                if (valid) {
+#pragma unroll
+                    for (int c = 0; c < 8; ++c)
+                        *reinterpret_cast<float4*>(drow + 32 * c4 + 4 * c) =
+                            make_float4(__uint_as_float(o[4 * c]) * mc.scale, __uint_as_float(o[4 * c + 1]) * mc.scale,
+                                        __uint_as_float(o[4 * c + 2]) * mc.scale,
+                                        __uint_as_float(o[4 * c + 3]) * mc.scale);
+                }
+            }
+        }
+    }
+    tc::tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc::tc_fence_after();
+        tc::tmem_dealloc(tmem, kTmemCols);
+    }
+}
+
+// ---------------------------------------------------------------- host
+bool bwd_dq_tc_supported(const QueryRows& qr)
+{
+    return qr.D == kD && qr.Hq / qr.Hkv == kG && (qr.max_ctx - 1) / kBlock + 1 <= kMaxBlk;
+}
+
+cudaError_t launch_bwd_dq_tc(const QueryRows& qr, const void* k, const void* v, int Lcap, const int32_t* idx,
+                             const int32_t* cnt, const MethodConsts& mc, bool dense_all, const float* lse,
+                             const float* dsum, const void* dout, float* dq, cudaStream_t s)
+{
+    if (!bwd_dq_tc_supported(qr)) return cudaErrorNotSupported;
+    CUtensorMap tq, tdo, tk, tv;
+    const uint64_t row = (uint64_t)kD * 2;
+    if (!make_tma_map_bf16(&tq, qr.q, kD, qr.Hq, (uint64_t)qr.B * qr.T, row, row * qr.Hq, kG, kTok) ||
+        !make_tma_map_bf16(&tdo, dout, kD, qr.Hq, (uint64_t)qr.B * qr.T, row, row * qr.Hq, kG, kTok) ||
+        !make_tma_map_bf16(&tk, k, kD, qr.Hkv, (uint64_t)qr.B * Lcap, row, row * qr.Hkv, 1, kBlock) ||
+        !make_tma_map_bf16(&tv, v, kD, qr.Hkv, (uint64_t)qr.B * Lcap, row, row * qr.Hkv, 1, kBlock))
+        return cudaErrorNotSupported;
+    cudaError_t e = ensure_smem(bwd_dq_tc_kernel, kSmemBytes);
+    if (e != cudaSuccess) return e;
+    const dim3 grid((qr.T + kTok - 1) / kTok, qr.B * qr.Hkv);
+    return launch_pdl(bwd_dq_tc_kernel, grid, dim3(kThreads), (size_t)kSmemBytes, s, qr, tq, tdo, tk, tv, Lcap, idx,
+                      cnt, mc, dense_all ? 1 : 0, lse, dsum, dq);
+}
+
+int bwd_tc_error_flag_read_and_clear()
+{
+    int h = 0;
+    if (cudaMemcpyFromSymbol(&h, g_bwd_tc_error, sizeof(int)) != cudaSuccess) return -1;
+    if (h) {
+        const int zero = 0;
+        cudaMemcpyToSymbol(g_bwd_tc_error, &zero, sizeof(int));
+    }
+    return h;
+}
+
+}  // namespace iv2

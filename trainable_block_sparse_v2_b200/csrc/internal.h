@@ -164,4 +164,11 @@ cudaError_t launch_attn_backward(const QueryRows& qr, const void* k, const void*
                                  const float* lse, const void* dout, float* dq, float* dk, float* dv, void* ws,
                                  cudaStream_t s);
 
+// dq of the backward on tcgen05/TMEM (16 heads per group, d = 128); cudaErrorNotSupported otherwise
+bool bwd_dq_tc_supported(const QueryRows& qr);
+cudaError_t launch_bwd_dq_tc(const QueryRows& qr, const void* k, const void* v, int Lcap, const int32_t* idx,
+                             const int32_t* cnt, const MethodConsts& mc, bool dense_all, const float* lse,
+                             const float* dsum, const void* dout, float* dq, cudaStream_t s);
+int bwd_tc_error_flag_read_and_clear();
+
 }  // namespace iv2
