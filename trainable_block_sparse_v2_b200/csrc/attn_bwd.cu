@@ -647,6 +647,11 @@ cudaError_t bwd_impl(const QueryRows& qr, const void* k, const void* v, int Lcap
                        dense_flag, lse, static_cast<const float*>(dsum), static_cast<const __nv_bfloat16*>(dout), dq);
     }
     if (e != cudaSuccess) return e;
+    if (D == 128 && bwd_dkdv_tc_supported(qr)) {
+        e = launch_bwd_dkdv_tc(qr, k, v, Lcap, mc, w.nb, lse, dsum, dout, counts, offsets, tokens, nitems, item_list,
+                               item_start, w.cap, w.max_items, dk, dv, s);
+        if (e != cudaErrorNotSupported) return e;
+    }
     e = ensure_smem(bwd_dkdv_kernel<D>, DkvSmem<D>::kBytes);
     if (e != cudaSuccess) return e;
     int per_sm = 1;

@@ -386,6 +386,328 @@ cudaError_t launch_bwd_dq_tc(const QueryRows& qr, const void* k, const void* v, 
                       cnt, mc, dense_all ? 1 : 0, lse, dsum, dq);
 }
 
+// =====================================================================================================
+// dk, dv: one 64-key block against 8-token tiles of its token list
+// =====================================================================================================
+//   S   [128 rows x 64 keys]   = Q . K^T            A (Q) and B (K) K-major in smem
+//   dP  [128 x 64]             = dO . V^T
+//   P, dS                      rows in TMEM -> bf16 tiles in smem (four warps, one row per thread)
+//   dV^T [128 dims x 64 keys] += dO^T . P           A (dO) MN-major, B (P) MN-major, in TMEM
+//   dK^T [128 dims x 64 keys] += Q^T . dS           the same with Q and dS
+// S and dP are double-buffered, so tile i + 1's products run while the warps form tile i's P and dS.  A
+// work item's sums go to dk / dv by fp32 atomics (one TMEM lane = one head dimension per thread).
+namespace {
+
+constexpr int kKvThreads = 192;   // warp 0 TMA, warp 1 MMA, warps 2-5 P / dS and the flush
+constexpr int kKvItemTokens = 256;  // tokens per work item (the list builder's chunk)
+constexpr int kKvTile = 16384;    // one 64-key block of K or V
+constexpr int kKvQd = 32768;      // one 8-token tile of Q or dO: two d-halves x 128 rows x 128 B
+constexpr int kKvKOff = 0;
+constexpr int kKvVOff = kKvKOff + kKvTile;
+constexpr int kKvQOff = kKvVOff + kKvTile;       // [2] x (Q | dO)
+constexpr int kKvPOff = kKvQOff + 4 * kKvQd;     // P tile: 128 rows x 64 keys bf16 (128 B rows, swizzled)
+constexpr int kKvSOff = kKvPOff + 16384;         // dS tile
+constexpr int kKvTokOff = kKvSOff + 16384;       // [2][8] token ids of the Q / dO buffers
+constexpr int kKvSmemBytes = kKvTokOff + 64 + 1024;
+// TMEM: S [0,128) (two 64-column buffers), dP [128,256) (two), dV^T [256,320), dK^T [320,384)
+constexpr uint32_t kKvCols = 512, kKvColS = 0, kKvColDP = 128, kKvColDV = 256, kKvColDK = 320;
+
+struct KvBars {
+    uint64_t kv_full, kv_free, qd_full[2], qd_free[2], s_full[2], pd_full, pd_free, acc_done, acc_free;
+    uint32_t tmem_base;
+    int err;
+};
+
+}  // namespace
+
+__global__ void __launch_bounds__(kKvThreads, 1)
+bwd_dkdv_tc_kernel(QueryRows qr, const __grid_constant__ CUtensorMap tm_q1, const __grid_constant__ CUtensorMap tm_do1,
+                   const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v, int Lcap,
+                   MethodConsts mc, int nb, const float* __restrict__ lse, const float* __restrict__ dsum,
+                   const int* __restrict__ counts, const int* __restrict__ offsets, const int* __restrict__ tokens,
+                   const int* __restrict__ nitems, const int* __restrict__ item_list,
+                   const int* __restrict__ item_start, int cap, float* __restrict__ dk, float* __restrict__ dv)
+{
+    pdl_launch_dependents();
+    pdl_wait();
+    extern __shared__ unsigned char smem_raw[];
+    unsigned char* smem = tc::align_smem_1024(smem_raw);
+    __shared__ KvBars bars;
+    int* tok_sm = reinterpret_cast<int*>(smem + kKvTokOff);  // [2][8]
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int T = qr.T;
+    const int n_items = *nitems;
+
+    if (threadIdx.x == 0) {
+        bars.err = 0;
+        tc::mbar_init(&bars.kv_full, 1);
+        tc::mbar_init(&bars.kv_free, 1);
+        for (int i = 0; i < 2; ++i) {
+            tc::mbar_init(&bars.qd_full[i], 1);
+            tc::mbar_init(&bars.qd_free[i], 1);
+            tc::mbar_init(&bars.s_full[i], 1);
+        }
+        tc::mbar_init(&bars.pd_full, 128);
+        tc::mbar_init(&bars.pd_free, 1);
+        tc::mbar_init(&bars.acc_done, 1);
+        tc::mbar_init(&bars.acc_free, 128);
+        tc::fence_barrier_init();
+    }
+    if (warp == 1) {
+        tc::tmem_alloc(&bars.tmem_base, kKvCols);
+        tc::tmem_relinquish();
+    }
+    tc::tc_fence_before();
+    __syncthreads();
+    tc::tc_fence_after();
+    const uint32_t tmem = bars.tmem_base;
+    volatile int* err = &bars.err;
+    const uint32_t sbase = tc::smem_u32(smem);
+
+    // every role walks the same items and tiles; the counters give each barrier's phase
+    if (warp == 0) {
+        // ---------------- TMA: the block's K and V per item, Q and dO rows of 8 tokens per tile ----------------
+        if (lane == 0) {
+            tc::prefetch_tensormap(&tm_q1);
+            tc::prefetch_tensormap(&tm_do1);
+            tc::prefetch_tensormap(&tm_k);
+            tc::prefetch_tensormap(&tm_v);
+            int n_item = 0, n_tile = 0;
+            bool ok = true;
+            for (int item = blockIdx.x; item < n_items && ok; item += gridDim.x, ++n_item) {
+                const int l = item_list[item], start = item_start[item];
+                const int b = l / (qr.Hkv * nb), g = (l / nb) % qr.Hkv, kb = l % nb;
+                const int ntok = min(min(kKvItemTokens, counts[l] - start), cap - offsets[l] - start);
+                const int* toks = tokens + offsets[l] + start;
+                if (n_item >= 1 && !(ok = wait_bar(&bars.kv_free, (n_item - 1) & 1, err))) break;
+                tc::mbar_arrive_expect_tx(&bars.kv_full, 2 * kKvTile);
+                const int z = b * Lcap + kb * kBlock;
+#pragma unroll
+                for (int a = 0; a < 2; ++a) {
+                    tc::tma_load_3d(smem + kKvKOff + a * 8192, &tm_k, 64 * a, g, z, &bars.kv_full);
+                    tc::tma_load_3d(smem + kKvVOff + a * 8192, &tm_v, 64 * a, g, z, &bars.kv_full);
+                }
+                const int ntiles = ntok > 0 ? (ntok + kTok - 1) / kTok : 0;
+                for (int i = 0; i < ntiles; ++i, ++n_tile) {
+                    const int qb = n_tile & 1, use = n_tile >> 1;
+                    if (use >= 1 && !(ok = wait_bar(&bars.qd_free[qb], (use - 1) & 1, err))) break;
+                    // token slots past the list repeat its first token (finite rows; their p is masked to 0); the
+                    // ids are stored before the arrive, whose release orders them for the readers
+                    unsigned char* qt = smem + kKvQOff + qb * 2 * kKvQd;
+                    int tsl[kTok];
+#pragma unroll
+                    for (int s = 0; s < kTok; ++s) {
+                        const int j = i * kTok + s;
+                        tsl[s] = toks[j < ntok ? j : i * kTok];
+                        tok_sm[qb * kTok + s] = j < ntok ? tsl[s] : -1;
+                    }
+                    tc::mbar_arrive_expect_tx(&bars.qd_full[qb], 2 * kKvQd);
+#pragma unroll
+                    for (int s = 0; s < kTok; ++s) {
+                        const int t = tsl[s];
+#pragma unroll
+                        for (int a = 0; a < 2; ++a) {
+                            tc::tma_load_3d(qt + a * 16384 + s * 2048, &tm_q1, 64 * a, g * kG, b * T + t, &bars.qd_full[qb]);
+                            tc::tma_load_3d(qt + kKvQd + a * 16384 + s * 2048, &tm_do1, 64 * a, g * kG, b * T + t,
+                                            &bars.qd_full[qb]);
+                        }
+                    }
+                }
+            }
+        }
+    } else if (warp == 1) {
+        // ---------------- MMA issuer ----------------
+        if (lane == 0) {
+            constexpr uint32_t idesc_s = tc::idesc_bf16_ab(128, kBlock, false, false);
+            constexpr uint32_t idesc_t = tc::idesc_bf16_ab(128, kBlock, true, true);
+            int n_item = 0, n_tile = 0;
+            bool ok = true;
+            auto issue_s = [&](int tile_ctr) {  // S, dP of the tile with global counter tile_ctr
+                const int qb = tile_ctr & 1, sb = tile_ctr & 1;
+                const uint32_t qa = sbase + kKvQOff + qb * 2 * kKvQd, da = qa + kKvQd;
+#pragma unroll
+                for (int ks = 0; ks < kD / 16; ++ks) {
+                    const uint32_t off = (ks >> 2) * 16384 + (ks & 3) * 32;
+                    const uint32_t boff = (ks >> 2) * 8192 + (ks & 3) * 32;
+                    tc::mma_bf16_ss(tmem + kKvColS + kBlock * sb, tc::desc_kmajor_sw128(qa + off),
+                                    tc::desc_kmajor_sw128(sbase + kKvKOff + boff), idesc_s, ks > 0);
+                    tc::mma_bf16_ss(tmem + kKvColDP + kBlock * sb, tc::desc_kmajor_sw128(da + off),
+                                    tc::desc_kmajor_sw128(sbase + kKvVOff + boff), idesc_s, ks > 0);
+                }
+                tc::mma_commit(&bars.s_full[sb]);
+            };
+            for (int item = blockIdx.x; item < n_items && ok; item += gridDim.x, ++n_item) {
+                const int l = item_list[item], start = item_start[item];
+                const int ntok = min(min(kKvItemTokens, counts[l] - start), cap - offsets[l] - start);
+                const int ntiles = ntok > 0 ? (ntok + kTok - 1) / kTok : 0;
+                if (!(ok = wait_bar(&bars.kv_full, n_item & 1, err))) break;
+                // the flush of the previous item's sums must be done before this item's first accumulation
+                if (n_item >= 1 && !(ok = wait_bar(&bars.acc_free, (n_item - 1) & 1, err))) break;
+                tc::tc_fence_after();
+                const int tile0 = n_tile;
+                if (ntiles > 0) {
+                    if (!(ok = wait_bar(&bars.qd_full[tile0 & 1], (tile0 >> 1) & 1, err))) break;
+                    tc::tc_fence_after();
+                    issue_s(tile0);
+                }
+                for (int i = 0; i < ntiles; ++i) {
+                    const int ctr = tile0 + i;
+                    if (i + 1 < ntiles) {
+                        // tile i + 1's products into the other S / dP buffers, read back by the warps for tile i - 1
+                        if (!(ok = wait_bar(&bars.qd_full[(ctr + 1) & 1], ((ctr + 1) >> 1) & 1, err))) break;
+                        tc::tc_fence_after();
+                        issue_s(ctr + 1);
+                    }
+                    if (!(ok = wait_bar(&bars.pd_full, ctr & 1, err))) break;
+                    tc::tc_fence_after();
+                    const uint32_t qa = sbase + kKvQOff + (ctr & 1) * 2 * kKvQd, da = qa + kKvQd;
+#pragma unroll
+                    for (int ks = 0; ks < 128 / 16; ++ks) {  // over the tile's 128 rows
+                        tc::mma_bf16_ss(tmem + kKvColDV, tc::desc_mnmajor_sw128(da + ks * 2048, 16384),
+                                        tc::desc_mnmajor_sw128(sbase + kKvPOff + ks * 2048, 16384), idesc_t,
+                                        (i > 0 || ks > 0));
+                        tc::mma_bf16_ss(tmem + kKvColDK, tc::desc_mnmajor_sw128(qa + ks * 2048, 16384),
+                                        tc::desc_mnmajor_sw128(sbase + kKvSOff + ks * 2048, 16384), idesc_t,
+                                        (i > 0 || ks > 0));
+                    }
+                    tc::mma_commit(&bars.pd_free);
+                    tc::mma_commit(&bars.qd_free[ctr & 1]);
+                }
+                if (!ok) break;
+                n_tile += ntiles;
+                tc::mma_commit(&bars.kv_free);
+                tc::mma_commit(&bars.acc_done);
+            }
+        }
+    } else {
+        // ---------------- P, dS (one query row per thread) and the flush (one head dimension per thread) ----------
+        const int q4 = warp & 3;
+        const int r = q4 * 32 + lane;  // tile row = token slot * 16 + head; in the flush: head dimension
+        const uint32_t lane_addr = tmem + ((uint32_t)(q4 * 32) << 16);
+        const float sl2 = mc.scale * kLog2e;
+        int n_item = 0, n_tile = 0;
+        bool ok = true;
+        for (int item = blockIdx.x; item < n_items; item += gridDim.x, ++n_item) {
+            const int l = item_list[item], start = item_start[item];
+            const int b = l / (qr.Hkv * nb), g = (l / nb) % qr.Hkv, kb = l % nb;
+            const int ntok = min(min(kKvItemTokens, counts[l] - start), cap - offsets[l] - start);
+            const int ntiles = ntok > 0 ? (ntok + kTok - 1) / kTok : 0;
+            for (int i = 0; i < ntiles; ++i, ++n_tile) {
+                const int sb = n_tile & 1;
+                if (ok) ok = wait_bar(&bars.s_full[sb], (n_tile >> 1) & 1, err);
+                ok = __all_sync(0xffffffffu, ok);
+                if (ok) tc::tc_fence_after();
+                const int t = tok_sm[sb * kTok + (r >> 4)];  // the Q / dO buffer of this tile is n_tile & 1 too
+                const bool valid = t >= 0;
+                const size_t head = ((size_t)b * T + (valid ? t : 0)) * qr.Hq + g * kG + (r & 15);
+                const int n = valid ? query_ctx(qr, b, t) : 0;
+                float lse2 = __int_as_float(0x7f800000), dd = 0.f;
+                if (valid) {
+                    const float lv = lse[head];
+                    if (lv > neg_inf() && lv < __int_as_float(0x7f800000)) lse2 = lv * kLog2e;
+                    dd = dsum[head];
+                }
+                const int nv = valid ? min(kBlock, n - kb * kBlock) : 0;  // keys of the block this row sees
+                uint32_t sv[64], pv[64];
+                if (ok) {
+                    tc::tmem_ld32(lane_addr + kKvColS + kBlock * sb, *reinterpret_cast<uint32_t(*)[32]>(&sv[0]));
+                    tc::tmem_ld32(lane_addr + kKvColS + kBlock * sb + 32, *reinterpret_cast<uint32_t(*)[32]>(&sv[32]));
+                    tc::tmem_ld32(lane_addr + kKvColDP + kBlock * sb, *reinterpret_cast<uint32_t(*)[32]>(&pv[0]));
+                    tc::tmem_ld32(lane_addr + kKvColDP + kBlock * sb + 32, *reinterpret_cast<uint32_t(*)[32]>(&pv[32]));
+                    tc::tmem_wait_ld();
+                }
+                // the P / dS tiles of the previous tile must have been read by its products
+                if (ok && n_tile >= 1) ok = wait_bar(&bars.pd_free, (n_tile - 1) & 1, err);
+                ok = __all_sync(0xffffffffu, ok);
+                if (ok) {
+                    unsigned char* prow = smem + kKvPOff + r * 128;
+                    unsigned char* drow = smem + kKvSOff + r * 128;
+#pragma unroll
+                    for (int c = 0; c < 8; ++c) {
+                        uint32_t pw[4], dw[4];
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            const int j = 8 * c + 2 * e;
+                            const float p0 = j < nv ? ex2_approx(__uint_as_float(sv[j]) * sl2 - lse2) : 0.f;
+                            const float p1 = j + 1 < nv ? ex2_approx(__uint_as_float(sv[j + 1]) * sl2 - lse2) : 0.f;
+                            pw[e] = pack_bf16(p0, p1);
+                            dw[e] = pack_bf16(p0 * (__uint_as_float(pv[j]) - dd), p1 * (__uint_as_float(pv[j + 1]) - dd));
+                        }
+                        const int sw = (c ^ (r & 7)) << 4;
+                        *reinterpret_cast<uint4*>(prow + sw) = make_uint4(pw[0], pw[1], pw[2], pw[3]);
+                        *reinterpret_cast<uint4*>(drow + sw) = make_uint4(dw[0], dw[1], dw[2], dw[3]);
+                    }
+                    tc::fence_proxy_async_smem();  // generic-proxy tile writes -> visible to the tensor core
+                    tc::tc_fence_before();
+                    tc::mbar_arrive(&bars.pd_full);
+                }
+            }
+            // this item's dV^T, dK^T: lane r is head dimension r; 64 columns are the block's keys
+            if (ok) ok = wait_bar(&bars.acc_done, n_item & 1, err);
+            ok = __all_sync(0xffffffffu, ok);
+            if (ok && ntiles > 0) {
+                tc::tc_fence_after();
+#pragma unroll 1
+                for (int m2 = 0; m2 < 2; ++m2) {
+                    float* dst = m2 ? dk : dv;
+                    const float mul = m2 ? mc.scale : 1.f;
+#pragma unroll 1
+                    for (int h2 = 0; h2 < 2; ++h2) {
+                        uint32_t a[32];
+                        tc::tmem_ld32(lane_addr + (m2 ? kKvColDK : kKvColDV) + 32 * h2, a);
+                        tc::tmem_wait_ld();
+#pragma unroll 4
+                        for (int j = 0; j < 32; ++j) {
+                            const int key = kb * kBlock + 32 * h2 + j;
+                            if (key < Lcap)
+                                atomicAdd(dst + (((size_t)b * Lcap + key) * qr.Hkv + g) * kD + r,
+                                          __uint_as_float(a[j]) * mul);
+                        }
+                    }
+                }
+            }
+            if (ok) {
+                tc::tc_fence_before();
+                tc::mbar_arrive(&bars.acc_free);
+            }
+        }
+    }
+    tc::tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc::tc_fence_after();
+        tc::tmem_dealloc(tmem, kKvCols);
+    }
+}
+
+bool bwd_dkdv_tc_supported(const QueryRows& qr)
+{
+    return qr.D == kD && qr.Hq / qr.Hkv == kG;
+}
+
+cudaError_t launch_bwd_dkdv_tc(const QueryRows& qr, const void* k, const void* v, int Lcap, const MethodConsts& mc,
+                               int nb, const float* lse, const float* dsum, const void* dout, const int* counts,
+                               const int* offsets, const int* tokens, const int* nitems, const int* item_list,
+                               const int* item_start, int cap, int max_items, float* dk, float* dv, cudaStream_t s)
+{
+    if (!bwd_dkdv_tc_supported(qr)) return cudaErrorNotSupported;
+    CUtensorMap tq, tdo, tk, tv;
+    const uint64_t row = (uint64_t)kD * 2;
+    if (!make_tma_map_bf16(&tq, qr.q, kD, qr.Hq, (uint64_t)qr.B * qr.T, row, row * qr.Hq, kG, 1) ||
+        !make_tma_map_bf16(&tdo, dout, kD, qr.Hq, (uint64_t)qr.B * qr.T, row, row * qr.Hq, kG, 1) ||
+        !make_tma_map_bf16(&tk, k, kD, qr.Hkv, (uint64_t)qr.B * Lcap, row, row * qr.Hkv, 1, kBlock) ||
+        !make_tma_map_bf16(&tv, v, kD, qr.Hkv, (uint64_t)qr.B * Lcap, row, row * qr.Hkv, 1, kBlock))
+        return cudaErrorNotSupported;
+    cudaError_t e = ensure_smem(bwd_dkdv_tc_kernel, kKvSmemBytes);
+    if (e != cudaSuccess) return e;
+    int dev = 0, nsm = 148;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
+    const int grid = max(1, min(nsm, max_items));
+    return launch_pdl(bwd_dkdv_tc_kernel, dim3(grid), dim3(kKvThreads), (size_t)kKvSmemBytes, s, qr, tq, tdo, tk, tv,
+                      Lcap, mc, nb, lse, dsum, counts, offsets, tokens, nitems, item_list, item_start, cap, dk, dv);
+}
+
 int bwd_tc_error_flag_read_and_clear()
 {
     int h = 0;

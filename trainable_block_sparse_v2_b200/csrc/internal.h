@@ -169,6 +169,11 @@ bool bwd_dq_tc_supported(const QueryRows& qr);
 cudaError_t launch_bwd_dq_tc(const QueryRows& qr, const void* k, const void* v, int Lcap, const int32_t* idx,
                              const int32_t* cnt, const MethodConsts& mc, bool dense_all, const float* lse,
                              const float* dsum, const void* dout, float* dq, cudaStream_t s);
+bool bwd_dkdv_tc_supported(const QueryRows& qr);
+cudaError_t launch_bwd_dkdv_tc(const QueryRows& qr, const void* k, const void* v, int Lcap, const MethodConsts& mc,
+                               int nb, const float* lse, const float* dsum, const void* dout, const int* counts,
+                               const int* offsets, const int* tokens, const int* nitems, const int* item_list,
+                               const int* item_start, int cap, int max_items, float* dk, float* dv, cudaStream_t s);
 int bwd_tc_error_flag_read_and_clear();
 
 }  // namespace iv2

@@ -228,5 +228,11 @@ __host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, bool b_mn_major)
            ((uint32_t)(M >> 4) << 24);
 }
 
+// the same with the major-ness of A and B given separately (A MN-major: bit 15; B MN-major: bit 16)
+__host__ __device__ constexpr uint32_t idesc_bf16_ab(int M, int N, bool a_mn_major, bool b_mn_major)
+{
+    return idesc_bf16(M, N, b_mn_major) | ((a_mn_major ? 1u : 0u) << 15);
+}
+
 }  // namespace tc
 }  // namespace iv2
