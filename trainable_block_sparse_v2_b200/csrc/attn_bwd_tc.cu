@@ -342,6 +342,10 @@ bwd_dq_tc_kernel(QueryRows qr, const __grid_constant__ CUtensorMap tm_q, const _
                 uint32_t o[32];
                 tc::tmem_ld32(lane_addr + 64 * half + 32 * c4, o);
                 tc::tmem_wait_ld();
+                if (U == 0) {  // no token of the tile selected a block: dQ was never written, dq is 0
+#pragma unroll
+                    for (int c = 0; c < 32; ++c) o[c] = 0u;
+                }
                 if (valid) {
 #pragma unroll
                     for (int c = 0; c < 8; ++c)
@@ -594,10 +598,14 @@ bwd_dkdv_tc_kernel(QueryRows qr, const __grid_constant__ CUtensorMap tm_q1, cons
             const int ntiles = ntok > 0 ? (ntok + kTok - 1) / kTok : 0;
             for (int i = 0; i < ntiles; ++i, ++n_tile) {
                 const int sb = n_tile & 1;
+                // the token ids of this tile's Q / dO buffer (n_tile & 1, as S) were stored before the TMA warp's
+                // arrive on qd_full: waiting on it orders those stores before the reads below.  It completed
+                // before s_full and cannot run ahead (its next phase needs this tile's products done).
+                if (ok) ok = wait_bar(&bars.qd_full[sb], (n_tile >> 1) & 1, err);
                 if (ok) ok = wait_bar(&bars.s_full[sb], (n_tile >> 1) & 1, err);
                 ok = __all_sync(0xffffffffu, ok);
                 if (ok) tc::tc_fence_after();
-                const int t = tok_sm[sb * kTok + (r >> 4)];  // the Q / dO buffer of this tile is n_tile & 1 too
+                const int t = ok ? tok_sm[sb * kTok + (r >> 4)] : -1;
                 const bool valid = t >= 0;
                 const size_t head = ((size_t)b * T + (valid ? t : 0)) * qr.Hq + g * kG + (r & 15);
                 const int n = valid ? query_ctx(qr, b, t) : 0;
