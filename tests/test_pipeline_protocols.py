@@ -262,3 +262,217 @@ def test_checker_reports_a_deadlock_and_a_wrong_phase():
     m.role("a", [("arrive", "b", 1), ("arrive", "b", 1), ("arrive", "b", 1), ("wait", "b", 0)])
     with pytest.raises(ProtocolError, match="phase 0 returned with 3"):
         m.run()
+
+
+# --------------------------------------------------------------------------------------------------------------
+# bwd_dq_tc_kernel (csrc/attn_bwd_tc.cu): one 128-row tile over U union blocks.  Warp 0: Q and dO once, K per
+# step (3-slot ring); warp 10: V per step; warp 1: S(p) = Q K^T and dP(p) = dO V^T into buffers p & 1, then
+# dQ += dS(p - 1) K; warps 2-9: dS, two per lane quarter (half 0: keys 0-31, half 1: keys 32-63); dS goes
+# back over the first 32 columns of its S buffer after both halves' loads (named barrier per quarter).
+# --------------------------------------------------------------------------------------------------------------
+def bwd_dq_model(m: PipelineModel, U: int, mistake: str = ""):
+    m.bar("qd_full", 1)
+    m.bar("qd_tmem", 128)
+    for i in range(RING):
+        for n in ("k_full", "k_empty", "v_full", "v_empty"):
+            m.bar(f"{n}{i}", 1)
+    for i in range(2):
+        m.bar(f"s_full{i}", 1)
+        m.bar(f"ds_full{i}", 256)
+        m.bar(f"dq_done{i}", 1)
+
+    def warp0():
+        yield ("arrive_tx", "qd_full", 1, 2)
+        yield ("tma", "qd_full", 1, [("Qs", "Q")])
+        yield ("tma", "qd_full", 1, [("dOs", "dO")])
+        for p in range(U):
+            s, k = p % RING, p // RING
+            if k >= 1 and mistake != "K producer skips k_empty":
+                yield ("wait", f"k_empty{s}", k - 1)
+            yield ("arrive_tx", f"k_full{s}", 1, 1)
+            yield ("tma", f"k_full{s}", 1, [(f"K{s}", ("K", p))])
+
+    def warp10():
+        for p in range(U):
+            s, k = p % RING, p // RING
+            if k >= 1:
+                yield ("wait", f"v_empty{s}", k - 1)
+            yield ("arrive_tx", f"v_full{s}", 1, 1)
+            yield ("tma", f"v_full{s}", 1, [(f"V{s}", ("V", p))])
+
+    def issuer():
+        yield ("wait", "qd_tmem", 0)
+        for p in range(U + 1):
+            if p < U:
+                s, sb = p % RING, p & 1
+                yield ("wait", f"k_full{s}", p // RING)
+                yield ("wait", f"v_full{s}", p // RING)
+                yield ("mma", [(f"QT.q{q}", "Q") for q in range(4)] + [(f"K{s}", ("K", p))],
+                       [(f"S{sb}.q{q}.{c}", ("S", p)) for q in range(4) for c in ("a", "b", "hi")], f"S{p}")
+                yield ("mma", [(f"dOT.q{q}", "dO") for q in range(4)] + [(f"V{s}", ("V", p))],
+                       [(f"DP{sb}.q{q}.{c}", ("DP", p)) for q in range(4) for c in ("lo", "hi")], f"DP{p}")
+                yield ("commit", f"s_full{sb}")
+                yield ("commit", f"v_empty{s}")
+            if p >= 1:
+                v = p - 1
+                db, s = v & 1, v % RING
+                if mistake != "issuer skips ds_full":
+                    yield ("wait", f"ds_full{db}", v >> 1)
+                reads = [(f"S{db}.q{q}.{c}", ("dS", v)) for q in range(4) for c in ("a", "b")]
+                reads += [(f"K{s}", ("K", v))] + ([("dQ", ("dQ", v - 1))] if v > 0 else [])
+                yield ("mma", reads, [("dQ", ("dQ", v))], f"dQ{v}")
+                yield ("commit", f"dq_done{db}")
+                yield ("commit", f"k_empty{s}")
+
+    def ds_warp(w):
+        q4, half = w & 3, (w - 2) >> 2
+        yield ("wait", "qd_full", 0)
+        if half == 0:
+            yield ("read", "Qs", "Q")
+            yield ("read", "dOs", "dO")
+            yield ("write", f"QT.q{q4}", "Q")
+            yield ("write", f"dOT.q{q4}", "dO")
+            yield ("arrive", "qd_tmem", 32)
+        for p in range(U):
+            sb = p & 1
+            yield ("wait", f"s_full{sb}", p >> 1)
+            if half == 0:
+                yield ("read", f"S{sb}.q{q4}.a", ("S", p))
+                yield ("read", f"S{sb}.q{q4}.b", ("S", p))
+                yield ("read", f"DP{sb}.q{q4}.lo", ("DP", p))
+            else:
+                yield ("read", f"S{sb}.q{q4}.hi", ("S", p))
+                yield ("read", f"DP{sb}.q{q4}.hi", ("DP", p))
+            if mistake != "no pair barrier":
+                yield ("nbar", 1 + q4, 2)
+            yield ("write", f"S{sb}.q{q4}.{'a' if half == 0 else 'b'}", ("dS", p))
+            yield ("arrive", f"ds_full{sb}", 32)
+        if U > 0:
+            if mistake != "no final dq_done wait":
+                yield ("wait", f"dq_done{(U - 1) & 1}", (U - 1) >> 1)
+            yield ("read", "dQ", ("dQ", U - 1))
+
+    m.role("warp0", warp0())
+    m.role("warp10", warp10())
+    m.role("issuer", issuer())
+    for w in range(2, 10):
+        m.role(f"ds{w}", ds_warp(w))
+
+
+# --------------------------------------------------------------------------------------------------------------
+# bwd_dkdv_tc_kernel (csrc/attn_bwd_tc.cu): work items (one 64-key block and up to 256 of its listed tokens),
+# each in 8-token tiles.  Warp 0: the item's K and V, then per tile the token ids (shared memory) and the Q / dO
+# rows (TMA, 2 buffers); warp 1: S, dP per tile into buffers tile & 1 (one tile ahead), then dV^T += dO^T P and
+# dK^T += Q^T dS; warps 2-5: P and dS into shared-memory tiles (one row per thread), and after each item the
+# flush of dV^T / dK^T from TMEM.
+# --------------------------------------------------------------------------------------------------------------
+def bwd_dkdv_model(m: PipelineModel, items, mistake: str = ""):
+    m.bar("kv_full", 1)
+    m.bar("kv_free", 1)
+    for i in range(2):
+        m.bar(f"qd_full{i}", 1)
+        m.bar(f"qd_free{i}", 1)
+        m.bar(f"s_full{i}", 1)
+    m.bar("pd_full", 128)
+    m.bar("pd_free", 1)
+    m.bar("acc_done", 1)
+    m.bar("acc_free", 128)
+    Q4 = range(4)
+
+    def producer():
+        n_tile = 0
+        for n_item, ntiles in enumerate(items):
+            if n_item >= 1 and mistake != "producer skips kv_free":
+                yield ("wait", "kv_free", n_item - 1)
+            yield ("arrive_tx", "kv_full", 1, 1)
+            yield ("tma", "kv_full", 1, [("KV", ("KV", n_item))])
+            for _ in range(ntiles):
+                qb, use = n_tile & 1, n_tile >> 1
+                if use >= 1 and mistake != "producer skips qd_free":
+                    yield ("wait", f"qd_free{qb}", use - 1)
+                yield ("write", f"tok{qb}", ("tok", n_tile))
+                yield ("arrive_tx", f"qd_full{qb}", 1, 1)
+                yield ("tma", f"qd_full{qb}", 1, [(f"QdO{qb}", ("QdO", n_tile))])
+                n_tile += 1
+
+    def issuer():
+        n_tile = 0
+
+        def issue_s(ctr, n_item):
+            b = ctr & 1
+            yield ("mma", [(f"QdO{b}", ("QdO", ctr)), ("KV", ("KV", n_item))],
+                   [(f"S{b}.q{q}", ("S", ctr)) for q in Q4] + [(f"DP{b}.q{q}", ("DP", ctr)) for q in Q4], f"S{ctr}")
+            yield ("commit", f"s_full{b}")
+
+        for n_item, ntiles in enumerate(items):
+            yield ("wait", "kv_full", n_item)
+            if n_item >= 1 and mistake != "issuer skips acc_free":
+                yield ("wait", "acc_free", n_item - 1)
+            tile0 = n_tile
+            if ntiles > 0:
+                yield ("wait", f"qd_full{tile0 & 1}", tile0 >> 1)
+                yield from issue_s(tile0, n_item)
+            for i in range(ntiles):
+                ctr = tile0 + i
+                if i + 1 < ntiles:
+                    yield ("wait", f"qd_full{(ctr + 1) & 1}", (ctr + 1) >> 1)
+                    yield from issue_s(ctr + 1, n_item)
+                yield ("wait", "pd_full", ctr)
+                reads = [(f"QdO{ctr & 1}", ("QdO", ctr))] + [(f"P.q{q}", ("P", ctr)) for q in Q4]
+                if i > 0:
+                    reads += [(f"acc.q{q}", ("acc", n_item, i - 1)) for q in Q4]
+                yield ("mma", reads, [(f"acc.q{q}", ("acc", n_item, i)) for q in Q4], f"dVdK{ctr}")
+                yield ("commit", "pd_free")
+                yield ("commit", f"qd_free{ctr & 1}")
+            n_tile += ntiles
+            yield ("commit", "kv_free")
+            yield ("commit", "acc_done")
+
+    def warps(q4):
+        n_tile = 0
+        for n_item, ntiles in enumerate(items):
+            for _ in range(ntiles):
+                b = n_tile & 1
+                yield ("wait", f"qd_full{b}", n_tile >> 1)
+                yield ("wait", f"s_full{b}", n_tile >> 1)
+                yield ("read", f"tok{b}", ("tok", n_tile))
+                yield ("read", f"S{b}.q{q4}", ("S", n_tile))
+                yield ("read", f"DP{b}.q{q4}", ("DP", n_tile))
+                if n_tile >= 1 and mistake != "warps skip pd_free":
+                    yield ("wait", "pd_free", n_tile - 1)
+                yield ("write", f"P.q{q4}", ("P", n_tile))
+                yield ("arrive", "pd_full", 32)
+                n_tile += 1
+            if mistake != "warps skip acc_done":
+                yield ("wait", "acc_done", n_item)
+            if ntiles > 0:
+                yield ("read", f"acc.q{q4}", ("acc", n_item, ntiles - 1))
+            yield ("arrive", "acc_free", 32)
+
+    m.role("producer", producer())
+    m.role("issuer", issuer())
+    for q4 in Q4:
+        m.role(f"warp{2 + q4}", warps(q4))
+
+
+@pytest.mark.parametrize("U", [0, 1, 2, 3, 4, 7, 12])
+def test_bwd_dq_protocol(U):
+    _run(bwd_dq_model, range(60), U)
+
+
+@pytest.mark.parametrize("items", [[1], [0], [3, 0, 2], [5, 1, 0, 4], [2, 2, 2, 2, 2], [0, 0, 1]])
+def test_bwd_dkdv_protocol(items):
+    _run(bwd_dkdv_model, range(60), items)
+
+
+@pytest.mark.parametrize("mistake", ["K producer skips k_empty", "issuer skips ds_full", "no pair barrier",
+                                     "no final dq_done wait"])
+def test_bwd_dq_planted_mistakes_are_caught(mistake):
+    assert _caught(bwd_dq_model, range(300), 7, mistake=mistake), mistake
+
+
+@pytest.mark.parametrize("mistake", ["producer skips kv_free", "producer skips qd_free", "issuer skips acc_free",
+                                     "warps skip pd_free", "warps skip acc_done"])
+def test_bwd_dkdv_planted_mistakes_are_caught(mistake):
+    # acc_free matters only where empty items let the issuer commit acc_done twice without a P tile between
+    assert _caught(bwd_dkdv_model, range(300), [3, 0, 0, 2, 4], mistake=mistake), mistake
