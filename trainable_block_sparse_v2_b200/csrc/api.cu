@@ -540,6 +540,13 @@ int infllmv2_window_attn_decode(const void* q, int batch, int hq, int hkv, int h
     if (batch * hkv > iv2::kMaxSplitRows) return INFLLMV2_ERR_UNSUPPORTED;
     IV2_TRY(check_ws(ws, ws_bytes, split_need(batch * hkv, max_ctx, mc.kmax, 0, true, false, window)));
     const QueryRows qr = rows_of(q, batch, 1, hq, hkv, head_dim, nullptr, ctx_lens, 0, max_ctx);
+    // one cluster launch (the decode step's kernel walking the window's blocks, partials merged on chip) when
+    // the shape allows it; else the split attention and its merge
+    if (batch * hkv <= 65535 && iv2::decode_fused_supported(qr, mc)) {
+        const cudaError_t e = iv2::launch_decode_fused(qr, nullptr, 1, mc, k, v, lcap, nullptr, nullptr, out, lse,
+                                                       (cudaStream_t)stream);
+        if (e != cudaErrorNotSupported) return launched(e);
+    }
     return launched(iv2::launch_attn_split(qr, k, v, lcap, nullptr, nullptr, mc, true, nullptr, nullptr, nullptr, out,
                                            lse, ws, (cudaStream_t)stream));
 }

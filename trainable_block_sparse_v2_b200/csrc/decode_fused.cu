@@ -196,7 +196,10 @@ decode_fused_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_con
     const int n = query_ctx(qr, b, t);
     const int c = (n - 1) / kBlock;
     const int nb = c + 1;
-    const bool dense = n <= mc.dense_len;
+    // the draft model's sliding window (mc.window > 0): attend densely to the keys [w0, n), blocks bw .. c
+    const int w0 = mc.window > 0 ? max(0, n - mc.window) : 0;
+    const int bw = w0 / kBlock;
+    const bool dense = mc.window > 0 || n <= mc.dense_len;
     const int nkv = min(num_kernels(n), nk_cap);
     const int bpc = ((nb + CL - 1) / CL + 3) & ~3;  // blocks per CTA, a multiple of 4
     const int b0 = rank * bpc, b1 = min(b0 + bpc, nb);
@@ -205,7 +208,7 @@ decode_fused_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_con
     const bool bad = !dense && (bpc > kFMaxBpc || nb > kFThreads * E);
     const bool sparse = !dense && !bad;
     const __nv_bfloat16* qrow = static_cast<const __nv_bfloat16*>(qr.q) + ((size_t)bt * qr.Hq + g * G) * D;
-    int32_t* idx_row = idx + (size_t)row * mc.kmax;
+    int32_t* idx_row = idx ? idx + (size_t)row * mc.kmax : nullptr;  // null: no block list is written
     const float sl2 = mc.scale * kLog2e;
     uint32_t phase_bits = 0;  // parity of each ring stage
     bool failed = bad;
@@ -370,9 +373,9 @@ decode_fused_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_con
 
     // ---------------- 3. selection (every CTA, identical result; the leader writes it out) ----------------
     int32_t* my_list = reinterpret_cast<int32_t*>(smem + L::kMyList);
-    int count = nb;
+    int count = nb - bw;
     if (dense) {
-        if (rank == 0 && tid < 32) warp_write_dense_row(c, mc.kmax, idx_row, cnt + row);
+        if (rank == 0 && tid < 32 && idx_row) warp_write_dense_row(c, mc.kmax, idx_row, cnt + row);
     } else if (bad) {
         count = 0;
         if (rank == 0 && tid == 0) cnt[row] = 0;
@@ -398,7 +401,7 @@ decode_fused_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_con
     {
         const int z_base = b * Lcap;
         auto issue_block = [&](int i) {
-            const int blk = dense ? rank + CL * i : my_list[i];
+            const int blk = dense ? bw + rank + CL * i : my_list[i];
             const int sidx = i % kFStages;
             unsigned char* stg = smem + (size_t)sidx * L::kStageBytes;
             tc::mbar_arrive_expect_tx(&full[sidx], (uint32_t)L::kStageBytes);
@@ -420,10 +423,13 @@ decode_fused_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_con
             const int sidx = i % kFStages;
             if (!tc::mbar_wait(&full[sidx], (phase_bits >> sidx) & 1u, 1u << 24)) failed = true;
             phase_bits ^= 1u << sidx;
-            const int blk = dense ? rank + CL * i : my_list[i];
+            const int blk = dense ? bw + rank + CL * i : my_list[i];
             const int nvalid = min(kBlock, n - blk * kBlock);
+            const int nskip = max(0, w0 - blk * kBlock);  // keys of the block before the window (0 without one)
             unsigned char* stg = smem + (size_t)sidx * L::kStageBytes;
-            if (key0 < nvalid) {
+            // a warp works when one of its 8 keys is in [nskip, nvalid) (nskip < nvalid for every walked block),
+            // so every row's running max is finite after its first block
+            if (key0 < nvalid && key0 + 8 > nskip) {
                 unsigned char* vt = stg + L::kTileBytes;
                 if (key0 + 8 > nvalid) {
                     // rows past the context may hold anything: zero them so that 0 * V stays 0
@@ -448,7 +454,7 @@ decode_fused_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_con
                     mma_bf16_16816(s4, qf[2 * kk + 1], b2r, b3r);
                 }
                 const int ka = key0 + 2 * tq;
-                const bool va = ka < nvalid, vb = ka + 1 < nvalid;
+                const bool va = ka < nvalid && ka >= nskip, vb = ka + 1 < nvalid && ka + 1 >= nskip;
                 float sc[4];
                 sc[0] = va ? s4[0] * sl2 : neg_inf();
                 sc[1] = vb ? s4[1] * sl2 : neg_inf();
