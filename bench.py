@@ -657,6 +657,154 @@ class Decode32kBench:
         return float(np.median([a.elapsed_time(b) for a, b in evs])) / 1e3
 
 
+class PagedDecodeBench:
+    """The 128K ragged decode batch (step 0) on a paged cache: the keys and values of the 4 sequences scattered
+    over a shuffled pool of 64-position pages.  One step = the paged kernel pool of the new key + the paged fused
+    decode step; the same step on the contiguous cache is timed the same way beside it.  L2 is flushed before
+    every timed step; the time is the median of the steps."""
+
+    def __init__(self):
+        import torch
+        from trainable_block_sparse_v2_b200 import binding
+        from trainable_block_sparse_v2_b200.workloads import decode_128k_ragged
+
+        self.torch, self.b = torch, binding
+        w = decode_128k_ragged(steps=1)
+        dev = torch.device("cuda")
+        to = lambda a: torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).to(dev).view(torch.bfloat16)  # noqa: E731
+        i32 = lambda a: torch.from_numpy(np.ascontiguousarray(a, dtype=np.int32)).to(dev)  # noqa: E731
+        self.lens_h = w.ctx_lens.astype(np.int64)
+        B = len(self.lens_h)
+        self.L = int(self.lens_h.max())
+        self.q, self.k, self.v = to(w.q), to(w.k), to(w.v)
+        self.p = binding.Params(**w.params)
+        # pages: every sequence's blocks on a shuffled set of pages
+        need = [int((n + 63) // 64) for n in self.lens_h]
+        max_pages = max(need)
+        rng = np.random.default_rng(77)
+        perm = rng.permutation(sum(need)).astype(np.int32)
+        table = np.full((B, max_pages), -1, np.int32)
+        off = 0
+        for b, m in enumerate(need):
+            table[b, :m] = perm[off:off + m]
+            off += m
+        self.table = i32(table)
+        num_pages = sum(need)
+        Hkv, Dd = self.k.shape[2], self.k.shape[3]
+        self.kp = torch.empty((num_pages * 64, Hkv, Dd), dtype=torch.bfloat16, device=dev)
+        self.vp = torch.empty_like(self.kp)
+        for b, m in enumerate(need):
+            rows = (torch.from_numpy(table[b, :m].astype(np.int64)).to(dev)[:, None] * 64 +
+                    torch.arange(64, device=dev)[None]).reshape(-1)
+            n = min(m * 64, self.k.shape[1])
+            self.kp[rows[:n]] = self.k[b, :n]
+            self.vp[rows[:n]] = self.v[b, :n]
+        self.lens, self.old = i32(self.lens_h), i32(self.lens_h - 1)
+        self.kern_p = torch.zeros((B, HKV, nk(self.L), D), dtype=torch.bfloat16, device=dev)
+        self.kern_c = torch.zeros_like(self.kern_p)
+        binding.infllmv2_kernel_pool_paged(self.kp, self.table, i32(np.zeros(B)), self.old, self.L, self.p,
+                                           self.kern_p)
+        binding.infllmv2_kernel_pool(self.k, i32(np.zeros(B)), self.old, self.L, self.p, self.kern_c)
+        self.idx = torch.empty((B, 1, HKV, self.p.kmax), dtype=torch.int32, device=dev)
+        self.cnt = torch.empty((B, 1, HKV), dtype=torch.int32, device=dev)
+        self.out = torch.empty((B, 1, HQ, D), dtype=torch.bfloat16, device=dev)
+        self.l2_flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+
+    def step_paged(self):
+        self.b.infllmv2_kernel_pool_paged(self.kp, self.table, self.old, self.lens, 1, self.p, self.kern_p)
+        self.b.infllmv2_sparse_decode_step_paged(self.q, self.kern_p, self.kp, self.vp, self.table, self.lens, self.L,
+                                                 self.p, self.idx, self.cnt, self.out, None)
+
+    def step_contiguous(self):
+        self.b.infllmv2_kernel_pool(self.k, self.old, self.lens, 1, self.p, self.kern_c)
+        self.b.infllmv2_sparse_decode_step(self.q, self.kern_c, self.k, self.v, self.lens, self.L, self.p, self.idx,
+                                           self.cnt, self.out, None)
+
+    def run(self, fn, warmup, steps):
+        """median seconds per step, each step timed alone after an L2 flush"""
+        torch = self.torch
+        for _ in range(warmup):
+            fn()
+        torch.cuda.synchronize()
+        evs = []
+        for _ in range(steps):
+            self.l2_flush.fill_(1)
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record()
+            fn()
+            b.record()
+            evs.append((a, b))
+        torch.cuda.synchronize()
+        return float(np.median([a.elapsed_time(b) for a, b in evs])) / 1e3
+
+
+class VarlenPrefillBench:
+    """A packed batch of 4 prefill sequences (T = L = 32768, 16384, 8192, 4096 tokens; 32 / 2 heads, d 128,
+    top-k 64, dense below 8192, N(0,1) with per-block offsets like the 32K prefill): one call of the packed
+    prefill (kernel pool, scoring + top-k, attention: three launches for the batch) against the same sequences
+    one at a time through the per-sequence calls (three launches each).  Mean of `steps` passes."""
+
+    LENS = (32768, 16384, 8192, 4096)
+
+    def __init__(self):
+        import torch
+        from trainable_block_sparse_v2_b200 import binding
+        from trainable_block_sparse_v2_b200.workloads import prefill_case
+
+        self.torch, self.b = torch, binding
+        dev = torch.device("cuda")
+        to = lambda a: torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).to(dev).view(torch.bfloat16)  # noqa: E731
+        self.seqs = []
+        for i, T in enumerate(self.LENS):
+            w = prefill_case(T, HQ, HKV, D, topk=64, dense_len=8192, seed=1300 + i, n_needles=0,
+                             block_offset_std=0.3)
+            self.seqs.append((to(w.q[0]), to(w.k[0]), to(w.v[0])))
+        self.p = binding.Params(**w.params)
+        B = len(self.LENS)
+        cu = np.concatenate([[0], np.cumsum(self.LENS)]).astype(np.int32)
+        self.cu = torch.from_numpy(cu).to(dev)
+        self.q = torch.cat([s[0] for s in self.seqs])
+        self.k = torch.cat([s[1] for s in self.seqs])
+        self.v = torch.cat([s[2] for s in self.seqs])
+        self.T = int(cu[-1])
+        self.Lmax = max(self.LENS)
+        self.kern = torch.zeros((B, HKV, nk(self.Lmax), D), dtype=torch.bfloat16, device=dev)
+        self.idx = torch.empty((self.T, HKV, self.p.kmax), dtype=torch.int32, device=dev)
+        self.cnt = torch.empty((self.T, HKV), dtype=torch.int32, device=dev)
+        self.out = torch.empty((self.T, HQ, D), dtype=torch.bfloat16, device=dev)
+        self.ws = binding.workspace(self.p, B, self.Lmax, self.Lmax, HQ, HKV, D)
+        self.lens = [torch.tensor([T], dtype=torch.int32, device=dev) for T in self.LENS]
+        self.kerns = [torch.zeros((1, HKV, nk(T), D), dtype=torch.bfloat16, device=dev) for T in self.LENS]
+        self.zero = torch.zeros(1, dtype=torch.int32, device=dev)
+
+    def packed(self):
+        self.b.infllmv2_sparse_prefill_varlen(self.q, self.k, self.v, self.cu, self.cu, self.Lmax, self.Lmax, self.p,
+                                              self.kern, self.idx, self.cnt, self.out, None, self.ws)
+
+    def one_by_one(self):
+        b, off = self.b, 0
+        for i, T in enumerate(self.LENS):
+            q, k, v = self.seqs[i]
+            idx, cnt, out = self.idx[off:off + T][None], self.cnt[off:off + T][None], self.out[off:off + T][None]
+            b.infllmv2_kernel_pool(k[None], self.zero, self.lens[i], T, self.p, self.kerns[i])
+            b.infllmv2_block_score_topk(q[None], None, self.lens[i], T, self.kerns[i], self.p, idx, cnt, self.ws)
+            b.infllmv2_sparse_attn_prefill(q[None], k[None], v[None], None, self.lens[i], T, idx, cnt, self.p, out)
+            off += T
+
+    def run(self, fn, warmup, steps):
+        torch = self.torch
+        for _ in range(warmup):
+            fn()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(steps):
+            fn()
+        e1.record()
+        e1.synchronize()
+        return e0.elapsed_time(e1) / 1e3 / steps
+
+
 class TreeBench:
     """Tree-draft verification at a 64K prefix (one sequence, 16 draft nodes of depth <= 6, 32 / 2 heads,
     d 128, top-k 64).  One pass: the draft queries' block scoring + top-k over the whole prefix, then the tree
@@ -1003,6 +1151,49 @@ def run_ours(args):
         del tree
         torch.cuda.empty_cache()
 
+    if not args.no_paged:
+        # the 128K decode step on a paged cache (reported, not raised; same collective steps on every rank)
+        pg, tp, tc, err = None, float("nan"), float("nan"), None
+        try:
+            pg = PagedDecodeBench()
+            tp = pg.run(pg.step_paged, 10, 300)
+            tc = pg.run(pg.step_contiguous, 10, 300)
+        except Exception as e:  # noqa: BLE001
+            err = f"{type(e).__name__}: {e}"[:300]
+        tp, tc = barrier_max(tp, ws), barrier_max(tc, ws)
+        if err is None and tp == tp:
+            _, _, bp = decode_step_bytes(list(pg.lens_h))
+            line["paged_decode"] = {
+                "workload": "decode_128k_ragged step 0 on 64-position pages (shuffled page table)",
+                "value": whole_job_rate(len(pg.lens_h), ws, tp), "unit": UNIT, "us_per_step": tp * 1e6,
+                "contiguous_us_per_step": tc * 1e6, "timing": "median of 300 steps, L2 flushed before each",
+                "algorithmic_bytes": bp, "frac_of_" + peak_kind: bp / tp / 1e9 / peaks["hbm_gbs"],
+                "note": "one step = kernel_pool_paged of the new key + sparse_decode_step_paged",
+            }
+        else:
+            line["paged_decode"] = {"workload": "decode_128k_ragged paged", "error": err or "no time"}
+        del pg
+        torch.cuda.empty_cache()
+        vb, tv, t1, err = None, float("nan"), float("nan"), None
+        try:
+            vb = VarlenPrefillBench()
+            tv = vb.run(vb.packed, 1, 3)
+            t1 = vb.run(vb.one_by_one, 1, 3)
+        except Exception as e:  # noqa: BLE001
+            err = f"{type(e).__name__}: {e}"[:300]
+        tv, t1 = barrier_max(tv, ws), barrier_max(t1, ws)
+        if err is None and tv == tv:
+            line["varlen_prefill"] = {
+                "workload": "packed prefill of 4 sequences, T = L = 32768 + 16384 + 8192 + 4096",
+                "value": whole_job_rate(vb.T, ws, tv), "unit": UNIT, "ms_per_pass": tv * 1e3,
+                "one_sequence_at_a_time_ms": t1 * 1e3, "timing": "mean of 3 passes",
+                "note": "one pass = infllmv2_sparse_prefill_varlen (3 launches for the batch)",
+            }
+        else:
+            line["varlen_prefill"] = {"workload": "packed prefill", "error": err or "no time"}
+        del vb
+        torch.cuda.empty_cache()
+
     if rank == 0 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(args.cpu_budget)
     if rank == 0:
@@ -1070,6 +1261,7 @@ def main():
     ap.add_argument("--no-prefill", action="store_true")
     ap.add_argument("--no-backward", action="store_true", help="skip the prefill gradient pass")
     ap.add_argument("--no-lse-estimate", action="store_true", help="skip the LSE-estimate scoring leg")
+    ap.add_argument("--no-paged", action="store_true", help="skip the paged-decode and packed-prefill legs")
     ap.add_argument("--no-tree", action="store_true", help="skip the tree-verification leg")
     ap.add_argument("--no-decode32k", action="store_true", help="skip the batch-1 32K decode leg")
     ap.add_argument("--no-decode", action="store_true", help="prefill only (for profiling its kernels)")

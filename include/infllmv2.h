@@ -16,8 +16,11 @@
  *   and long text", long-context bullet (tree-draft verification with a bit-packed local mask).
  *
  * Conventions shared by every entry point
- *   - All tensor pointers are DEVICE pointers owned by the caller; the library allocates nothing and
- *     keeps no state between calls.  Every call is asynchronous on `stream` (0 = legacy default stream).
+ *   - All tensor pointers are DEVICE pointers owned by the caller; the library allocates no device memory.
+ *     Between calls it keeps only: per-device caches of kernel attributes and cluster occupancy, the
+ *     device-side flags that bounded waits raise (read and cleared by infllmv2_device_status), and the
+ *     fixed scratch array of infllmv2_sparse_attn_decode_noalloc.  Every call is asynchronous on `stream`
+ *     (0 = legacy default stream).
  *   - bf16 = IEEE bfloat16 (2 bytes).  Layouts are dense row-major (innermost index last):
  *       q        [B, T, Hq, d]       queries (T query tokens per sequence)
  *       k, v     [B, Lcap, Hkv, d]   key / value cache, position-major
@@ -198,6 +201,70 @@ int infllmv2_sparse_decode_step(const void* q, int batch, int hq, int hkv, int h
                                 const void* k, const void* v, int lcap, const int32_t* ctx_lens, int max_ctx,
                                 const infllmv2_params* params, int32_t* idx, int32_t* cnt, void* out, float* lse,
                                 infllmv2_stream_t stream);
+
+/*
+ * Paged key/value cache (serving; the pages give no cache layout -- the CPM.cu runtime of the QbitAI
+ * article, section "CPM.cu", manages static device memory, and a pool of fixed-size pages is that idea for
+ * many sequences of unknown length).  One page holds one context block, 64 positions, so a selected block
+ * is one page.  Position i of sequence b lives in row
+ *     page_table[b * max_pages + i / 64] * 64 + i % 64
+ * of the page pools k_pages / v_pages [num_pages * 64, Hkv, d] bf16 (device, 16-byte aligned).
+ *   page_table   [B, max_pages] int32 (device, 4-byte aligned), owned by the caller; entries past a
+ *                sequence's length are not read.  An entry outside [0, num_pages) is never dereferenced:
+ *                its positions read as zeros and are not written (such a row's results are then not the
+ *                method's; the Python binding's INFLLMV2_CHECK=1 mode checks the table on the host).
+ *   1 <= num_pages <= 2^24 and 1 <= max_pages <= 4096 (contexts up to 256K positions), else
+ *   INFLLMV2_ERR_UNSUPPORTED / INFLLMV2_ERR_INVALID_ARG.
+ * Each call computes exactly its contiguous counterpart on the cache gathered through the page table:
+ *   infllmv2_kv_append_paged          = infllmv2_kv_append        (writes through the table)
+ *   infllmv2_kernel_pool_paged        = infllmv2_kernel_pool
+ *   infllmv2_sparse_decode_step_paged = infllmv2_sparse_decode_step
+ *   infllmv2_sparse_attn_prefill_paged = infllmv2_sparse_attn_prefill (chunked prefill: q holds the last T
+ *                                      positions of each context; score them with infllmv2_block_score_topk,
+ *                                      which reads only the kernel cache)
+ * The kernel cache kern [B, Hkv, nk_cap, d] stays contiguous per sequence (1/16 of the keys).
+ */
+int infllmv2_kv_append_paged(const void* k_new, const void* v_new, int batch, int hkv, int head_dim, const int32_t* pos,
+                             void* k_pages, void* v_pages, int num_pages, const int32_t* page_table, int max_pages,
+                             infllmv2_stream_t stream);
+int infllmv2_kernel_pool_paged(const void* k_pages, int num_pages, const int32_t* page_table, int max_pages,
+                               int batch, int hkv, int head_dim, const int32_t* old_lens, const int32_t* new_lens,
+                               int max_new_keys, const infllmv2_params* params, void* kern, int nk_cap,
+                               infllmv2_stream_t stream);
+int infllmv2_sparse_decode_step_paged(const void* q, int batch, int hq, int hkv, int head_dim, const void* kern,
+                                      int nk_cap, const void* k_pages, const void* v_pages, int num_pages,
+                                      const int32_t* page_table, int max_pages, const int32_t* ctx_lens, int max_ctx,
+                                      const infllmv2_params* params, int32_t* idx, int32_t* cnt, void* out,
+                                      float* lse, infllmv2_stream_t stream);
+int infllmv2_sparse_attn_prefill_paged(const void* q, int batch, int num_q, int hq, int hkv, int head_dim,
+                                       const void* k_pages, const void* v_pages, int num_pages,
+                                       const int32_t* page_table, int max_pages, const int32_t* q_ctx,
+                                       const int32_t* ctx_lens, int max_ctx, const int32_t* idx, const int32_t* cnt,
+                                       const infllmv2_params* params, void* out, float* lse,
+                                       infllmv2_stream_t stream);
+
+/*
+ * Steps 1 + 2 + 3a for a packed batch of variable-length sequences (serving prefill without padding; the
+ * pages define no batching, this is the usual cu_seqlens packing).  Sequence b owns query rows
+ * [cu_seqlens_q[b], cu_seqlens_q[b+1]) and key / value rows [cu_seqlens_k[b], cu_seqlens_k[b+1]); its
+ * T_b queries are the last T_b of its L_b keys (query t sees n = L_b - T_b + t + 1 keys).  Three launches
+ * for the whole batch: the kernel pool of every sequence's keys into kern[b], block scoring + top-k of
+ * every query, and sparse attention -- per sequence exactly infllmv2_kernel_pool, infllmv2_block_score_topk
+ * and infllmv2_sparse_attn_prefill on that sequence alone.
+ *   q, out        [total_q, Hq, d] bf16;   k, v [total_k, Hkv, d] bf16
+ *   cu_seqlens_q,
+ *   cu_seqlens_k  [B + 1] int32 (device): 0 = cu[0] <= cu[1] <= ... , cu[B] = total; T_b <= L_b (trusted:
+ *                 the Python binding checks them on the host under INFLLMV2_CHECK=1)
+ *   max_seqlen_q, max_seqlen_k: host upper bounds of T_b and L_b (they size the grids)
+ *   kern          [B, Hkv, nk_cap, d] bf16 (device), nk_cap >= the kernel count of max_seqlen_k; written
+ *   idx, cnt      [total_q, Hkv, kmax] / [total_q, Hkv] int32;   lse [total_q, Hq] fp32 or NULL
+ *   ws            >= infllmv2_workspace_size(params, B, max_seqlen_q, max_seqlen_k, Hq, Hkv, d) bytes
+ */
+int infllmv2_sparse_prefill_varlen(const void* q, const void* k, const void* v, int batch, int hq, int hkv, int head_dim,
+                                   const int32_t* cu_seqlens_q, const int32_t* cu_seqlens_k, int total_q, int total_k,
+                                   int max_seqlen_q, int max_seqlen_k, const infllmv2_params* params, void* kern,
+                                   int nk_cap, int32_t* idx, int32_t* cnt, void* out, float* lse, void* ws,
+                                   size_t ws_bytes, infllmv2_stream_t stream);
 
 /*
  * Step 3c -- tree-draft verification (QbitAI article, "speculative sampling, quantisation and long text",

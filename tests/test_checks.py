@@ -101,3 +101,29 @@ def test_tree_mask():
         m[i] = bad
         with pytest.raises(checks.InputCheckError, match=msg):
             checks.check_tree_mask(m.astype(np.uint32)[None], 1, 4)
+
+
+def test_page_table_check():
+    table = np.array([[3, 0, -1], [1, 2, -1]], np.int32)
+    checks.check_page_table(table, [128, 70], num_pages=4)              # 2 pages each, all in range
+    with pytest.raises(checks.InputCheckError, match="outside"):
+        checks.check_page_table(table, [129, 70], num_pages=4)          # a third page, mapped to -1
+    with pytest.raises(checks.InputCheckError, match="outside"):
+        checks.check_page_table(table, [128, 70], num_pages=3)          # page 3 past the pool
+    with pytest.raises(checks.InputCheckError, match="serves both"):
+        checks.check_page_table(np.array([[0, 1], [1, 2]], np.int32), [128, 64], num_pages=4)
+    with pytest.raises(checks.InputCheckError, match="needs"):
+        checks.check_page_table(table, [64 * 3 + 1, 1], num_pages=4)    # more pages than the table holds
+
+
+def test_cu_seqlens_check():
+    cq, ck = np.array([0, 5, 5, 9], np.int32), np.array([0, 7, 20, 29], np.int32)
+    checks.check_cu_seqlens(cq, ck, 9, 29, 5, 13)
+    with pytest.raises(checks.InputCheckError, match="never decrease"):
+        checks.check_cu_seqlens(np.array([0, 5, 4, 9]), ck, 9, 29, 5, 13)
+    with pytest.raises(checks.InputCheckError, match="queries but"):
+        checks.check_cu_seqlens(np.array([0, 8, 8, 9]), ck, 9, 29, 8, 13)
+    with pytest.raises(checks.InputCheckError, match="max_seqlen"):
+        checks.check_cu_seqlens(cq, ck, 9, 29, 4, 13)
+    with pytest.raises(checks.InputCheckError, match="end at"):
+        checks.check_cu_seqlens(cq, ck, 10, 29, 5, 13)

@@ -88,6 +88,14 @@ _SIGS = {
     "infllmv2_sparse_attn_backward": ([_P, _I, _I, _I, _I, _I, _P, _P, _I, _P, _P, _I, _P, _P, _PP, _P, _P, _P,
                                        _P, _P, _P, _P, _SZ, _P], _I),
     "infllmv2_window_attn_decode": ([_P, _I, _I, _I, _I, _P, _P, _I, _P, _I, _I, _F, _P, _P, _P, _SZ, _P], _I),
+    "infllmv2_kv_append_paged": ([_P, _P, _I, _I, _I, _P, _P, _P, _I, _P, _I, _P], _I),
+    "infllmv2_kernel_pool_paged": ([_P, _I, _P, _I, _I, _I, _I, _P, _P, _I, _PP, _P, _I, _P], _I),
+    "infllmv2_sparse_decode_step_paged": ([_P, _I, _I, _I, _I, _P, _I, _P, _P, _I, _P, _I, _P, _I, _PP, _P, _P, _P,
+                                           _P, _P], _I),
+    "infllmv2_sparse_attn_prefill_paged": ([_P, _I, _I, _I, _I, _I, _P, _P, _I, _P, _I, _P, _P, _I, _P, _P, _PP,
+                                            _P, _P, _P], _I),
+    "infllmv2_sparse_prefill_varlen": ([_P, _P, _P, _I, _I, _I, _I, _P, _P, _I, _I, _I, _I, _PP, _P, _I, _P, _P,
+                                        _P, _P, _P, _SZ, _P], _I),
 }
 
 EXPORTED = tuple(_SIGS)
@@ -417,6 +425,160 @@ def infllmv2_window_attn_decode(q, k, v, ctx_lens, max_ctx, window, softmax_scal
                                             _ptr(ws), 0 if ws is None else ws.numel() * ws.element_size(),
                                             _stream(stream))
     _check("infllmv2_window_attn_decode", st)
+
+
+# ---- paged key/value cache: pools [num_pages * 64, Hkv, d], page_table [B, max_pages] int32 ----
+def _pages(fn, k_pages, v_pages, page_table, B):
+    """The page pools (one shape, [num_pages * 64, Hkv, d]) and the page table ([B, max_pages]).
+    Returns (num_pages, max_pages, Hkv, d)."""
+    _need(k_pages, torch.bfloat16, "k_pages", 3)
+    if k_pages.shape[0] % 64 != 0 or k_pages.shape[0] == 0:
+        raise ValueError(f"{fn}: k_pages: expected [num_pages * 64, Hkv, d], got {tuple(k_pages.shape)}")
+    if v_pages is not None:
+        _need(v_pages, torch.bfloat16, "v_pages", shape=tuple(k_pages.shape))
+    _need(page_table, torch.int32, "page_table", 2)
+    if page_table.shape[0] != B:
+        raise ValueError(f"{fn}: page_table: expected [{B}, max_pages], got {tuple(page_table.shape)}")
+    return k_pages.shape[0] // 64, page_table.shape[1], k_pages.shape[1], k_pages.shape[2]
+
+
+def _check_pages(what, page_table, lens, num_pages):
+    from . import checks
+    checks.check_page_table(page_table, lens, num_pages, what)
+
+
+def infllmv2_kv_append_paged(k_new, v_new, pos, k_pages, v_pages, page_table, stream=None):
+    """The row of position pos[b] through the page table: k_pages[page * 64 + pos % 64] = k_new[b] (v likewise)"""
+    _need(k_new, torch.bfloat16, "k_new", 3)
+    B = k_new.shape[0]
+    num_pages, max_pages, Hkv, d = _pages("infllmv2_kv_append_paged", k_pages, v_pages, page_table, B)
+    _need(k_new, torch.bfloat16, "k_new", shape=(B, Hkv, d))
+    _need(v_new, torch.bfloat16, "v_new", shape=(B, Hkv, d))
+    _int32(pos, "pos", B)
+    _devices("infllmv2_kv_append_paged", k_new, v_new, pos, k_pages, v_pages, page_table)
+    if _checking():
+        _check_pages("infllmv2_kv_append_paged", page_table, pos.detach().cpu().numpy().astype("int64") + 1,
+                     num_pages)
+    st = load().infllmv2_kv_append_paged(_ptr(k_new), _ptr(v_new), B, Hkv, d, _ptr(pos), _ptr(k_pages), _ptr(v_pages),
+                                         num_pages, _ptr(page_table), max_pages, _stream(stream))
+    _check("infllmv2_kv_append_paged", st)
+
+
+def infllmv2_kernel_pool_paged(k_pages, page_table, old_lens, new_lens, max_new_keys, params: Params, kern,
+                               stream=None):
+    """infllmv2_kernel_pool over a paged key cache"""
+    B = page_table.shape[0] if isinstance(page_table, torch.Tensor) and page_table.dim() == 2 else -1
+    num_pages, max_pages, Hkv, d = _pages("infllmv2_kernel_pool_paged", k_pages, None, page_table, B)
+    _need(kern, torch.bfloat16, "kern", 4)
+    if (kern.shape[0], kern.shape[1], kern.shape[3]) != (B, Hkv, d):
+        raise ValueError(f"kern: expected shape ({B}, {Hkv}, nk_cap, {d}), got {tuple(kern.shape)}")
+    _int32(old_lens, "old_lens", B)
+    _int32(new_lens, "new_lens", B)
+    _devices("infllmv2_kernel_pool_paged", k_pages, page_table, kern, old_lens, new_lens)
+    if _checking():
+        from . import checks
+        checks.check_pool_lengths(old_lens, new_lens, max_pages * 64, int(max_new_keys), kern.shape[2],
+                                  params.kernel_size, params.kernel_stride, "infllmv2_kernel_pool_paged")
+        _check_pages("infllmv2_kernel_pool_paged", page_table, new_lens, num_pages)
+    cp = params.c()
+    st = load().infllmv2_kernel_pool_paged(_ptr(k_pages), num_pages, _ptr(page_table), max_pages, B, Hkv, d,
+                                           _ptr(old_lens), _ptr(new_lens), int(max_new_keys), ctypes.byref(cp),
+                                           _ptr(kern), kern.shape[2], _stream(stream))
+    _check("infllmv2_kernel_pool_paged", st)
+
+
+def infllmv2_sparse_decode_step_paged(q, kern, k_pages, v_pages, page_table, ctx_lens, max_ctx, params: Params, idx,
+                                      cnt, out, lse=None, stream=None):
+    """infllmv2_sparse_decode_step over a paged key/value cache"""
+    _need(q, torch.bfloat16, "q")
+    if q.dim() < 3:
+        raise ValueError(f"q: expected [B, Hq, d] or [B, 1, Hq, d], got {tuple(q.shape)}")
+    B, Hq = q.shape[0], q.shape[-2]
+    num_pages, max_pages, Hkv, d = _pages("infllmv2_sparse_decode_step_paged", k_pages, v_pages, page_table, B)
+    _need(q, torch.bfloat16, "q", numel=B * Hq * d)
+    _need(out, torch.bfloat16, "out", numel=B * Hq * d)
+    _int32(ctx_lens, "ctx_lens", B)
+    _opt(lse, torch.float32, "lse", B * Hq)
+    _need(idx, torch.int32, "idx", numel=B * Hkv * params.kmax)
+    _need(cnt, torch.int32, "cnt", numel=B * Hkv)
+    _need(kern, torch.bfloat16, "kern", 4)
+    if (kern.shape[0], kern.shape[1], kern.shape[3]) != (B, Hkv, d):
+        raise ValueError(f"kern: expected shape ({B}, {Hkv}, nk_cap, {d}), got {tuple(kern.shape)}")
+    _devices("infllmv2_sparse_decode_step_paged", q, kern, k_pages, v_pages, page_table, ctx_lens, idx, cnt, out, lse)
+    if _checking():
+        _check_rows("infllmv2_sparse_decode_step_paged", B, 1, None, ctx_lens, True, max_pages * 64, max_ctx)
+        _check_pages("infllmv2_sparse_decode_step_paged", page_table, ctx_lens, num_pages)
+    cp = params.c()
+    st = load().infllmv2_sparse_decode_step_paged(_ptr(q), B, Hq, Hkv, d, _ptr(kern), kern.shape[2], _ptr(k_pages),
+                                                  _ptr(v_pages), num_pages, _ptr(page_table), max_pages,
+                                                  _ptr(ctx_lens), int(max_ctx), ctypes.byref(cp), _ptr(idx),
+                                                  _ptr(cnt), _ptr(out), _ptr(lse), _stream(stream))
+    _check("infllmv2_sparse_decode_step_paged", st)
+
+
+def infllmv2_sparse_attn_prefill_paged(q, k_pages, v_pages, page_table, q_ctx, ctx_lens, max_ctx, idx, cnt,
+                                       params: Params, out, lse=None, stream=None):
+    """infllmv2_sparse_attn_prefill over a paged key/value cache (q [B, T, Hq, d]: the last T positions of each
+    context unless q_ctx gives every query's context)"""
+    _need(q, torch.bfloat16, "q", 4)
+    B, T, Hq = q.shape[0], q.shape[1], q.shape[2]
+    num_pages, max_pages, Hkv, d = _pages("infllmv2_sparse_attn_prefill_paged", k_pages, v_pages, page_table, B)
+    _need(q, torch.bfloat16, "q", shape=(B, T, Hq, d))
+    _need(out, torch.bfloat16, "out", numel=B * T * Hq * d)
+    _need(idx, torch.int32, "idx", numel=B * T * Hkv * params.kmax)
+    _need(cnt, torch.int32, "cnt", numel=B * T * Hkv)
+    _opt(lse, torch.float32, "lse", B * T * Hq)
+    _opt(q_ctx, torch.int32, "q_ctx", B * T)
+    _opt(ctx_lens, torch.int32, "ctx_lens", B)
+    _devices("infllmv2_sparse_attn_prefill_paged", q, k_pages, v_pages, page_table, out, idx, cnt, lse, q_ctx,
+             ctx_lens)
+    if _checking():
+        from . import checks
+        _check_rows("infllmv2_sparse_attn_prefill_paged", B, T, q_ctx, ctx_lens, False, max_pages * 64, max_ctx, idx,
+                    cnt, params)
+        ctx = checks.query_contexts(B, T, q_ctx, ctx_lens, False)
+        _check_pages("infllmv2_sparse_attn_prefill_paged", page_table, ctx.max(axis=1), num_pages)
+    cp = params.c()
+    st = load().infllmv2_sparse_attn_prefill_paged(_ptr(q), B, T, Hq, Hkv, d, _ptr(k_pages), _ptr(v_pages),
+                                                   num_pages, _ptr(page_table), max_pages, _ptr(q_ctx),
+                                                   _ptr(ctx_lens), int(max_ctx), _ptr(idx), _ptr(cnt),
+                                                   ctypes.byref(cp), _ptr(out), _ptr(lse), _stream(stream))
+    _check("infllmv2_sparse_attn_prefill_paged", st)
+
+
+# ---- packed variable-length prefill: q [total_q, Hq, d], k / v [total_k, Hkv, d], cu_seqlens [B + 1] ----
+def infllmv2_sparse_prefill_varlen(q, k, v, cu_seqlens_q, cu_seqlens_k, max_seqlen_q, max_seqlen_k, params: Params,
+                                   kern, idx, cnt, out, lse=None, ws=None, stream=None):
+    """Kernel pool, scoring + top-k and sparse attention of a packed batch (three launches for the batch)"""
+    _need(q, torch.bfloat16, "q", 3)
+    _need(k, torch.bfloat16, "k", 3)
+    _need(v, torch.bfloat16, "v", shape=tuple(k.shape))
+    total_q, Hq, d = q.shape
+    total_k, Hkv = k.shape[0], k.shape[1]
+    if k.shape[2] != d:
+        raise ValueError(f"k: head_dim {k.shape[2]} differs from q's {d}")
+    _need(cu_seqlens_q, torch.int32, "cu_seqlens_q", 1)
+    B = cu_seqlens_q.numel() - 1
+    _int32(cu_seqlens_k, "cu_seqlens_k", B + 1)
+    _need(out, torch.bfloat16, "out", shape=(total_q, Hq, d))
+    _need(idx, torch.int32, "idx", numel=total_q * Hkv * params.kmax)
+    _need(cnt, torch.int32, "cnt", numel=total_q * Hkv)
+    _opt(lse, torch.float32, "lse", total_q * Hq)
+    _need(kern, torch.bfloat16, "kern", 4)
+    if (kern.shape[0], kern.shape[1], kern.shape[3]) != (B, Hkv, d):
+        raise ValueError(f"kern: expected shape ({B}, {Hkv}, nk_cap, {d}), got {tuple(kern.shape)}")
+    _devices("infllmv2_sparse_prefill_varlen", q, k, v, cu_seqlens_q, cu_seqlens_k, kern, idx, cnt, out, lse, ws)
+    if _checking():
+        from . import checks
+        checks.check_cu_seqlens(cu_seqlens_q, cu_seqlens_k, total_q, total_k, int(max_seqlen_q), int(max_seqlen_k),
+                                "infllmv2_sparse_prefill_varlen")
+    cp = params.c()
+    st = load().infllmv2_sparse_prefill_varlen(_ptr(q), _ptr(k), _ptr(v), B, Hq, Hkv, d, _ptr(cu_seqlens_q),
+                                               _ptr(cu_seqlens_k), total_q, total_k, int(max_seqlen_q),
+                                               int(max_seqlen_k), ctypes.byref(cp), _ptr(kern), kern.shape[2],
+                                               _ptr(idx), _ptr(cnt), _ptr(out), _ptr(lse), _ptr(ws),
+                                               0 if ws is None else ws.numel() * ws.element_size(), _stream(stream))
+    _check("infllmv2_sparse_prefill_varlen", st)
 
 
 def infllmv2_backward_workspace_size(params: Params, batch, max_q, max_ctx, hq, hkv, head_dim) -> int:

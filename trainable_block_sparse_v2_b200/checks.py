@@ -108,3 +108,42 @@ def check_tree_mask(tree_mask, B: int, n_draft: int, what: str = "") -> None:
                 if (mi >> j) & 1 and int(m[b, j]) & ~mi:
                     raise InputCheckError(f"{what}: node {i} of sequence {b} sees node {j} but not all of node "
                                           f"{j}'s ancestors")
+
+
+def check_page_table(page_table, lens, num_pages: int, what: str = "") -> None:
+    """Every page a sequence's first lens[b] positions use (entries [0, ceil(lens[b] / 64))) is in
+    [0, num_pages), the table has room for them, and no page serves two (sequence, block) slots."""
+    table = _np(page_table).astype(np.int64)
+    lens = _np(lens).astype(np.int64).ravel()
+    B, max_pages = table.shape
+    seen = {}
+    for b in range(B):
+        used = (int(lens[b]) + 63) // 64
+        if used > max_pages:
+            raise InputCheckError(f"{what}: sequence {b} needs {used} pages, the table has {max_pages}")
+        for i in range(used):
+            p = int(table[b, i])
+            if p < 0 or p >= num_pages:
+                raise InputCheckError(f"{what}: page_table[{b}, {i}] = {p}, outside [0, {num_pages})")
+            if p in seen:
+                raise InputCheckError(f"{what}: page {p} serves both {seen[p]} and {(b, i)}")
+            seen[p] = (b, i)
+
+
+def check_cu_seqlens(cu_q, cu_k, total_q: int, total_k: int, max_q: int, max_k: int, what: str = "") -> None:
+    """Packed batch offsets: both start at 0, never decrease and end at the totals; every sequence has at most
+    as many queries as keys, and the maxima bound the lengths."""
+    cq = _np(cu_q).astype(np.int64).ravel()
+    ck = _np(cu_k).astype(np.int64).ravel()
+    if len(cq) != len(ck) or len(cq) < 2:
+        raise InputCheckError(f"{what}: cu_seqlens_q / cu_seqlens_k must both hold B + 1 >= 2 offsets")
+    for name, cu, total in (("cu_seqlens_q", cq, total_q), ("cu_seqlens_k", ck, total_k)):
+        if cu[0] != 0 or cu[-1] != total or np.any(np.diff(cu) < 0):
+            raise InputCheckError(f"{what}: {name} must start at 0, never decrease and end at {total}")
+    tq, tk = np.diff(cq), np.diff(ck)
+    bad = np.nonzero(tq > tk)[0]
+    if len(bad):
+        raise InputCheckError(f"{what}: sequence {int(bad[0])} has {int(tq[bad[0]])} queries but {int(tk[bad[0]])} keys")
+    if tq.max() > max_q or tk.max() > max_k:
+        raise InputCheckError(f"{what}: max_seqlen_q / max_seqlen_k below the longest sequence "
+                              f"({int(tq.max())} / {int(tk.max())})")

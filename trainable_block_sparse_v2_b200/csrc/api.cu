@@ -199,6 +199,8 @@ QueryRows rows_of(const void* q, int B, int T, int hq, int hkv, int d, const int
     qr.ctx_lens = ctx_lens;
     qr.same_ctx = same_ctx;
     qr.max_ctx = max_ctx;
+    qr.cu_q = nullptr;
+    qr.q_rows = (long)B * T;
     return qr;
 }
 
@@ -227,6 +229,42 @@ int iv2::check_decode_attn(const void* q, int batch, int hq, int hkv, int head_d
     *nsplit = iv2::attn_split_count(iv2::attn_split_max_blocks(max_ctx, mc->kmax, mc->dense_len, false));
     return INFLLMV2_OK;
 }
+
+// ---- packed variable-length batches and paged caches ----
+namespace {
+
+constexpr int kMaxPagesInPool = 1 << 24;  // page * 64 rows stays an int
+
+int check_pages(const void* pool0, const void* pool1, int num_pages, const int32_t* table, int max_pages)
+{
+    IV2_TRY(check_ptr16(pool0));
+    if (pool1) IV2_TRY(check_ptr16(pool1));
+    IV2_TRY(check_ptr4(table));
+    if (num_pages < 1 || max_pages < 1) return INFLLMV2_ERR_INVALID_ARG;
+    if (num_pages > kMaxPagesInPool || max_pages > kMaxBlocks) return INFLLMV2_ERR_UNSUPPORTED;
+    return INFLLMV2_OK;
+}
+
+iv2::KvRows kv_paged(const int32_t* table, int max_pages, int num_pages)
+{
+    iv2::KvRows kr;
+    kr.Lcap = max_pages * iv2::kBlock;  // positions the table can address
+    kr.table = table;
+    kr.max_pages = max_pages;
+    kr.num_pages = num_pages;
+    kr.rows = (long)num_pages * iv2::kBlock;
+    return kr;
+}
+
+iv2::KvRows kv_packed(const int32_t* cu, long total)
+{
+    iv2::KvRows kr;
+    kr.cu = cu;
+    kr.rows = total;
+    return kr;
+}
+
+}  // namespace
 
 extern "C" {
 
@@ -282,8 +320,8 @@ int infllmv2_kernel_pool(const void* k, int batch, int lcap, int hkv, int head_d
     if (lcap < 1 || max_new_keys < 0 || nk_cap < 1 || max_new_keys > lcap) return INFLLMV2_ERR_INVALID_ARG;
     if (nk_cap < nk_of(max_new_keys)) return INFLLMV2_ERR_INVALID_ARG;
     if (max_new_keys == 0) return INFLLMV2_OK;
-    return launched(iv2::launch_kernel_pool(k, batch, lcap, hkv, head_dim, old_lens, new_lens, max_new_keys, kern,
-                                            nk_cap, (cudaStream_t)stream));
+    return launched(iv2::launch_kernel_pool(k, batch, iv2::kv_contiguous(batch, lcap), hkv, head_dim, old_lens, new_lens,
+                                            max_new_keys, kern, nk_cap, (cudaStream_t)stream));
 }
 
 int infllmv2_kv_append(const void* k_new, const void* v_new, int batch, int hkv, int head_dim, const int32_t* pos,
@@ -296,8 +334,8 @@ int infllmv2_kv_append(const void* k_new, const void* v_new, int batch, int hkv,
     IV2_TRY(check_ptr16(v_cache));
     IV2_TRY(check_ptr4(pos));
     if (lcap < 1) return INFLLMV2_ERR_INVALID_ARG;
-    return launched(iv2::launch_kv_append(k_new, v_new, batch, hkv, head_dim, pos, k_cache, v_cache, lcap,
-                                          (cudaStream_t)stream));
+    return launched(iv2::launch_kv_append(k_new, v_new, batch, hkv, head_dim, pos, k_cache, v_cache,
+                                          iv2::kv_contiguous(batch, lcap), (cudaStream_t)stream));
 }
 
 int infllmv2_block_score_topk(const void* q, int batch, int num_q, int hq, int hkv, int head_dim,
@@ -349,11 +387,11 @@ int infllmv2_sparse_attn_prefill(const void* q, int batch, int num_q, int hq, in
     const QueryRows qr = rows_of(q, batch, num_q, hq, hkv, head_dim, q_ctx, ctx_lens, 0, max_ctx);
     const MethodConsts mc = consts_of(params, head_dim);
     if (iv2::attn_tc_supported(qr)) {
-        const cudaError_t e = iv2::launch_attn_rows_tc(qr, k, v, lcap, idx, cnt, mc, false, out, lse,
+        const cudaError_t e = iv2::launch_attn_rows_tc(qr, k, v, iv2::kv_contiguous(batch, lcap), idx, cnt, mc, false, out, lse,
                                                        (cudaStream_t)stream);
         if (e != cudaErrorNotSupported) return launched(e);
     }
-    return launched(iv2::launch_attn_rows(qr, k, v, lcap, idx, cnt, mc, false, out, lse, (cudaStream_t)stream));
+    return launched(iv2::launch_attn_rows(qr, k, v, iv2::kv_contiguous(batch, lcap), idx, cnt, mc, false, out, lse, (cudaStream_t)stream));
 }
 
 int infllmv2_sparse_attn_decode(const void* q, int batch, int hq, int hkv, int head_dim, const void* k, const void* v,
@@ -367,7 +405,7 @@ int infllmv2_sparse_attn_decode(const void* q, int batch, int hq, int hkv, int h
                                    lse, &mc, &nsplit));
     IV2_TRY(check_ws(ws, ws_bytes, iv2::attn_ws_bytes(batch * hkv, nsplit)));
     const QueryRows qr = rows_of(q, batch, 1, hq, hkv, head_dim, nullptr, ctx_lens, 0, max_ctx);
-    return launched(iv2::launch_attn_split(qr, k, v, lcap, idx, cnt, mc, false, nullptr, nullptr, nullptr, out, lse,
+    return launched(iv2::launch_attn_split(qr, k, v, iv2::kv_contiguous(batch, lcap), idx, cnt, mc, false, nullptr, nullptr, nullptr, out, lse,
                                            ws, (cudaStream_t)stream));
 }
 
@@ -394,7 +432,8 @@ int infllmv2_sparse_decode_step(const void* q, int batch, int hq, int hkv, int h
     const MethodConsts mc = consts_of(params, head_dim);
     const QueryRows qr = rows_of(q, batch, 1, hq, hkv, head_dim, nullptr, ctx_lens, 0, max_ctx);
     if (!iv2::decode_fused_supported(qr, mc)) return INFLLMV2_ERR_UNSUPPORTED;
-    return launched(iv2::launch_decode_fused(qr, kern, nk_cap, mc, k, v, lcap, idx, cnt, out, lse, (cudaStream_t)stream));
+    return launched(iv2::launch_decode_fused(qr, kern, nk_cap, mc, k, v, iv2::kv_contiguous(batch, lcap), idx, cnt, out, lse,
+                                             (cudaStream_t)stream));
 }
 
 int infllmv2_sparse_attn_tree_verify(const void* q, int batch, int n_draft, int hq, int hkv, int head_dim,
@@ -422,7 +461,7 @@ int infllmv2_sparse_attn_tree_verify(const void* q, int batch, int n_draft, int 
     if (batch * n_draft * hkv > iv2::kMaxSplitRows) return INFLLMV2_ERR_UNSUPPORTED;
     IV2_TRY(check_ws(ws, ws_bytes, split_need(batch * n_draft * hkv, max_ctx, mc.kmax, mc.dense_len, false, true)));
     const QueryRows qr = rows_of(q, batch, n_draft, hq, hkv, head_dim, nullptr, prefix_lens, 1, max_ctx);
-    return launched(iv2::launch_attn_split(qr, k, v, lcap, idx, cnt, mc, false, k_draft, v_draft, tree_mask, out, lse,
+    return launched(iv2::launch_attn_split(qr, k, v, iv2::kv_contiguous(batch, lcap), idx, cnt, mc, false, k_draft, v_draft, tree_mask, out, lse,
                                            ws, (cudaStream_t)stream));
 }
 
@@ -447,11 +486,11 @@ int infllmv2_dense_attn_prefill(const void* q, int batch, int num_q, int hq, int
     const QueryRows qr = rows_of(q, batch, num_q, hq, hkv, head_dim, q_ctx, ctx_lens, 0, max_ctx);
     const MethodConsts mc = dense_consts(softmax_scale, head_dim);
     if (iv2::attn_tc_supported(qr)) {
-        const cudaError_t e = iv2::launch_attn_rows_tc(qr, k, v, lcap, nullptr, nullptr, mc, true, out, lse,
+        const cudaError_t e = iv2::launch_attn_rows_tc(qr, k, v, iv2::kv_contiguous(batch, lcap), nullptr, nullptr, mc, true, out, lse,
                                                        (cudaStream_t)stream);
         if (e != cudaErrorNotSupported) return launched(e);
     }
-    return launched(iv2::launch_attn_rows(qr, k, v, lcap, nullptr, nullptr, mc, true, out, lse, (cudaStream_t)stream));
+    return launched(iv2::launch_attn_rows(qr, k, v, iv2::kv_contiguous(batch, lcap), nullptr, nullptr, mc, true, out, lse, (cudaStream_t)stream));
 }
 
 size_t infllmv2_backward_workspace_size(const infllmv2_params* params, int batch, int max_q, int max_ctx, int hq,
@@ -517,7 +556,7 @@ int infllmv2_dense_attn_decode(const void* q, int batch, int hq, int hkv, int he
     if (batch * hkv > iv2::kMaxSplitRows) return INFLLMV2_ERR_UNSUPPORTED;
     IV2_TRY(check_ws(ws, ws_bytes, split_need(batch * hkv, max_ctx, mc.kmax, 0, true, false)));
     const QueryRows qr = rows_of(q, batch, 1, hq, hkv, head_dim, nullptr, ctx_lens, 0, max_ctx);
-    return launched(iv2::launch_attn_split(qr, k, v, lcap, nullptr, nullptr, mc, true, nullptr, nullptr, nullptr, out,
+    return launched(iv2::launch_attn_split(qr, k, v, iv2::kv_contiguous(batch, lcap), nullptr, nullptr, mc, true, nullptr, nullptr, nullptr, out,
                                            lse, ws, (cudaStream_t)stream));
 }
 
@@ -543,12 +582,154 @@ int infllmv2_window_attn_decode(const void* q, int batch, int hq, int hkv, int h
     // one cluster launch (the decode step's kernel walking the window's blocks, partials merged on chip) when
     // the shape allows it; else the split attention and its merge
     if (batch * hkv <= 65535 && iv2::decode_fused_supported(qr, mc)) {
-        const cudaError_t e = iv2::launch_decode_fused(qr, nullptr, 1, mc, k, v, lcap, nullptr, nullptr, out, lse,
+        const cudaError_t e = iv2::launch_decode_fused(qr, nullptr, 1, mc, k, v, iv2::kv_contiguous(batch, lcap), nullptr, nullptr, out, lse,
                                                        (cudaStream_t)stream);
         if (e != cudaErrorNotSupported) return launched(e);
     }
-    return launched(iv2::launch_attn_split(qr, k, v, lcap, nullptr, nullptr, mc, true, nullptr, nullptr, nullptr, out,
+    return launched(iv2::launch_attn_split(qr, k, v, iv2::kv_contiguous(batch, lcap), nullptr, nullptr, mc, true, nullptr, nullptr, nullptr, out,
                                            lse, ws, (cudaStream_t)stream));
+}
+
+
+// ---- paged key/value cache ----
+int infllmv2_kv_append_paged(const void* k_new, const void* v_new, int batch, int hkv, int head_dim, const int32_t* pos,
+                             void* k_pages, void* v_pages, int num_pages, const int32_t* page_table, int max_pages,
+                             infllmv2_stream_t stream)
+{
+    IV2_TRY(check_heads(batch, 1, hkv, hkv, head_dim));
+    IV2_TRY(check_ptr16(k_new));
+    IV2_TRY(check_ptr16(v_new));
+    IV2_TRY(check_ptr4(pos));
+    IV2_TRY(check_ptr16(v_pages));
+    IV2_TRY(check_pages(k_pages, v_pages, num_pages, page_table, max_pages));
+    return launched(iv2::launch_kv_append(k_new, v_new, batch, hkv, head_dim, pos, k_pages, v_pages,
+                                          kv_paged(page_table, max_pages, num_pages), (cudaStream_t)stream));
+}
+
+int infllmv2_kernel_pool_paged(const void* k_pages, int num_pages, const int32_t* page_table, int max_pages,
+                               int batch, int hkv, int head_dim, const int32_t* old_lens, const int32_t* new_lens,
+                               int max_new_keys, const infllmv2_params* params, void* kern, int nk_cap,
+                               infllmv2_stream_t stream)
+{
+    IV2_TRY(check_params(params));
+    IV2_TRY(check_heads(batch, 1, hkv, hkv, head_dim));
+    IV2_TRY(check_pages(k_pages, nullptr, num_pages, page_table, max_pages));
+    IV2_TRY(check_ptr16(kern));
+    IV2_TRY(check_ptr4(old_lens));
+    IV2_TRY(check_ptr4(new_lens));
+    const int lcap = max_pages * iv2::kBlock;
+    if (max_new_keys < 0 || nk_cap < 1 || max_new_keys > lcap) return INFLLMV2_ERR_INVALID_ARG;
+    if (nk_cap < nk_of(max_new_keys)) return INFLLMV2_ERR_INVALID_ARG;
+    if (max_new_keys == 0) return INFLLMV2_OK;
+    return launched(iv2::launch_kernel_pool(k_pages, batch, kv_paged(page_table, max_pages, num_pages), hkv, head_dim,
+                                            old_lens, new_lens, max_new_keys, kern, nk_cap, (cudaStream_t)stream));
+}
+
+int infllmv2_sparse_decode_step_paged(const void* q, int batch, int hq, int hkv, int head_dim, const void* kern,
+                                      int nk_cap, const void* k_pages, const void* v_pages, int num_pages,
+                                      const int32_t* page_table, int max_pages, const int32_t* ctx_lens, int max_ctx,
+                                      const infllmv2_params* params, int32_t* idx, int32_t* cnt, void* out,
+                                      float* lse, infllmv2_stream_t stream)
+{
+    IV2_TRY(check_params(params));
+    if (params->lse_stride > 1) return INFLLMV2_ERR_UNSUPPORTED;
+    IV2_TRY(check_heads(batch, 1, hq, hkv, head_dim));
+    IV2_TRY(check_ptr16(q));
+    IV2_TRY(check_ptr16(kern));
+    IV2_TRY(check_pages(k_pages, v_pages, num_pages, page_table, max_pages));
+    IV2_TRY(check_ptr16(out));
+    IV2_TRY(check_ptr4(ctx_lens));
+    IV2_TRY(check_ptr4(idx));
+    IV2_TRY(check_ptr4(cnt));
+    IV2_TRY(check_opt4(lse));
+    IV2_TRY(check_ctx(max_ctx, max_pages * iv2::kBlock));
+    if (nk_cap < 1 || nk_cap < nk_of(max_ctx)) return INFLLMV2_ERR_INVALID_ARG;
+    if (batch * hkv > 65535) return INFLLMV2_ERR_UNSUPPORTED;
+    const MethodConsts mc = consts_of(params, head_dim);
+    const QueryRows qr = rows_of(q, batch, 1, hq, hkv, head_dim, nullptr, ctx_lens, 0, max_ctx);
+    if (!iv2::decode_fused_supported(qr, mc)) return INFLLMV2_ERR_UNSUPPORTED;
+    return launched(iv2::launch_decode_fused(qr, kern, nk_cap, mc, k_pages, v_pages,
+                                             kv_paged(page_table, max_pages, num_pages), idx, cnt, out, lse,
+                                             (cudaStream_t)stream));
+}
+
+int infllmv2_sparse_attn_prefill_paged(const void* q, int batch, int num_q, int hq, int hkv, int head_dim,
+                                       const void* k_pages, const void* v_pages, int num_pages,
+                                       const int32_t* page_table, int max_pages, const int32_t* q_ctx,
+                                       const int32_t* ctx_lens, int max_ctx, const int32_t* idx, const int32_t* cnt,
+                                       const infllmv2_params* params, void* out, float* lse,
+                                       infllmv2_stream_t stream)
+{
+    IV2_TRY(check_params(params));
+    IV2_TRY(check_heads(batch, num_q, hq, hkv, head_dim));
+    IV2_TRY(check_ptr16(q));
+    IV2_TRY(check_pages(k_pages, v_pages, num_pages, page_table, max_pages));
+    IV2_TRY(check_ptr16(out));
+    IV2_TRY(check_ptr4(idx));
+    IV2_TRY(check_ptr4(cnt));
+    IV2_TRY(check_opt4(lse));
+    IV2_TRY(check_opt4(q_ctx));
+    IV2_TRY(check_opt4(ctx_lens));
+    if (!q_ctx && !ctx_lens) return INFLLMV2_ERR_INVALID_ARG;
+    IV2_TRY(check_ctx(max_ctx, max_pages * iv2::kBlock));
+    const QueryRows qr = rows_of(q, batch, num_q, hq, hkv, head_dim, q_ctx, ctx_lens, 0, max_ctx);
+    const MethodConsts mc = consts_of(params, head_dim);
+    const iv2::KvRows kr = kv_paged(page_table, max_pages, num_pages);
+    if (iv2::attn_tc_supported(qr)) {
+        const cudaError_t e = iv2::launch_attn_rows_tc(qr, k_pages, v_pages, kr, idx, cnt, mc, false, out, lse,
+                                                       (cudaStream_t)stream);
+        if (e != cudaErrorNotSupported) return launched(e);
+    }
+    return launched(iv2::launch_attn_rows(qr, k_pages, v_pages, kr, idx, cnt, mc, false, out, lse, (cudaStream_t)stream));
+}
+
+// ---- packed variable-length prefill ----
+int infllmv2_sparse_prefill_varlen(const void* q, const void* k, const void* v, int batch, int hq, int hkv, int head_dim,
+                                   const int32_t* cu_seqlens_q, const int32_t* cu_seqlens_k, int total_q, int total_k,
+                                   int max_seqlen_q, int max_seqlen_k, const infllmv2_params* params, void* kern,
+                                   int nk_cap, int32_t* idx, int32_t* cnt, void* out, float* lse, void* ws,
+                                   size_t ws_bytes, infllmv2_stream_t stream)
+{
+    IV2_TRY(check_params(params));
+    IV2_TRY(check_heads(batch, max_seqlen_q < 1 ? 1 : max_seqlen_q, hq, hkv, head_dim));
+    IV2_TRY(check_ptr16(q));
+    IV2_TRY(check_ptr16(k));
+    IV2_TRY(check_ptr16(v));
+    IV2_TRY(check_ptr16(kern));
+    IV2_TRY(check_ptr16(out));
+    IV2_TRY(check_ptr4(idx));
+    IV2_TRY(check_ptr4(cnt));
+    IV2_TRY(check_ptr4(cu_seqlens_q));
+    IV2_TRY(check_ptr4(cu_seqlens_k));
+    IV2_TRY(check_opt4(lse));
+    if (total_q < 0 || total_k < 0 || max_seqlen_q < 0 || max_seqlen_k < 0 || nk_cap < 1)
+        return INFLLMV2_ERR_INVALID_ARG;
+    if (max_seqlen_q > max_seqlen_k || max_seqlen_q > total_q || max_seqlen_k > total_k) return INFLLMV2_ERR_INVALID_ARG;
+    if (max_seqlen_q == 0) return INFLLMV2_OK;  // no query anywhere
+    IV2_TRY(check_ctx(max_seqlen_k, -1));
+    if (nk_cap < nk_of(max_seqlen_k)) return INFLLMV2_ERR_INVALID_ARG;
+    IV2_TRY(check_ws(ws, ws_bytes, score_need(batch, max_seqlen_q, hq, hkv, head_dim, max_seqlen_k)));
+    if (params->lse_stride > 1 && (iv2::score_uses_scan_path(batch, max_seqlen_q, hq / hkv, head_dim, max_seqlen_k) ||
+                                   head_dim != 128 || hq / hkv != 16))
+        return INFLLMV2_ERR_UNSUPPORTED;
+    QueryRows qr = rows_of(q, batch, max_seqlen_q, hq, hkv, head_dim, nullptr, nullptr, 0, max_seqlen_k);
+    qr.cu_q = cu_seqlens_q;
+    qr.cu_k = cu_seqlens_k;
+    qr.q_rows = total_q;
+    const MethodConsts mc = consts_of(params, head_dim);
+    const iv2::KvRows kr = kv_packed(cu_seqlens_k, total_k);
+    const cudaStream_t s = (cudaStream_t)stream;
+    // 1. every complete kernel window of every sequence (old length 0, new length L_b)
+    IV2_TRY(launched(iv2::launch_kernel_pool(k, batch, kr, hkv, head_dim, nullptr, nullptr, max_seqlen_k, kern, nk_cap,
+                                             s)));
+    // 2. scoring and top-k of every query
+    IV2_TRY(launched(iv2::launch_score_topk(qr, kern, nk_cap, mc, idx, cnt, ws, s)));
+    // 3. attention over the selected blocks
+    if (iv2::attn_tc_supported(qr)) {
+        const cudaError_t e = iv2::launch_attn_rows_tc(qr, k, v, kr, idx, cnt, mc, false, out, lse, s);
+        if (e != cudaErrorNotSupported) return launched(e);
+    }
+    return launched(iv2::launch_attn_rows(qr, k, v, kr, idx, cnt, mc, false, out, lse, s));
 }
 
 }  // extern "C"

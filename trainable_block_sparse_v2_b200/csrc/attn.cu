@@ -30,7 +30,7 @@ constexpr int kRowWarps = 4;
 
 template <int D>
 __global__ void __launch_bounds__(kRowWarps * 32) attn_rows_kernel(QueryRows qr, const __nv_bfloat16* __restrict__ k,
-                                                                   const __nv_bfloat16* __restrict__ v, int Lcap,
+                                                                   const __nv_bfloat16* __restrict__ v, KvRows kr,
                                                                    const int32_t* __restrict__ idx,
                                                                    const int32_t* __restrict__ cnt, MethodConsts mc,
                                                                    int dense_all, __nv_bfloat16* __restrict__ out,
@@ -47,21 +47,27 @@ __global__ void __launch_bounds__(kRowWarps * 32) attn_rows_kernel(QueryRows qr,
     unsigned char* vs_tile = ks_tile + KvTile<D>::kBytes;
 
     const int g = (int)(row % qr.Hkv);
-    const long bt = row / qr.Hkv;
-    const int t = (int)(bt % qr.T), b = (int)(bt / qr.T);
+    const int t = (int)((row / qr.Hkv) % qr.T), b = (int)(row / qr.Hkv / qr.T);
+    if (t >= q_len(qr, b)) return;           // past this sequence's queries (packed batch)
+    const long bt = q_row(qr, b, t);         // row of q / out / lse
+    const long orow_i = bt * qr.Hkv + g;     // row of idx / cnt
     const int G = qr.Hq / qr.Hkv;
     const int n = query_ctx(qr, b, t);
     const int c = (n - 1) / kBlock;
     const bool dense = dense_all || n <= mc.dense_len;
-    const int count = dense ? c + 1 : min(cnt[row], mc.kmax);
-    const int32_t* idx_row = idx ? idx + row * mc.kmax : nullptr;
+    const int count = dense ? c + 1 : min(cnt[orow_i], mc.kmax);
+    const int32_t* idx_row = idx ? idx + orow_i * mc.kmax : nullptr;
 
     uint32_t qf[D / 16][4];
     load_q_rows<D>(static_cast<const __nv_bfloat16*>(qr.q) + ((size_t)bt * qr.Hq + g * G) * D, G, qf);
     const size_t rs = (size_t)qr.Hkv * D;
-    const __nv_bfloat16* kb = k + ((size_t)b * Lcap * qr.Hkv + g) * D;
-    const __nv_bfloat16* vb = v + ((size_t)b * Lcap * qr.Hkv + g) * D;
     const float sl2 = mc.scale * kLog2e;
+    // first key (value) row of block blk and the keys to stage from it (0 for a page the table does not map)
+    auto block_src = [&](const __nv_bfloat16* base, int blk, int& nv) {
+        const long r0 = kv_block_row(kr, b, blk);
+        nv = r0 < 0 ? 0 : min(kBlock, n - blk * kBlock);
+        return base + ((size_t)(r0 < 0 ? 0 : r0) * qr.Hkv + g) * D;
+    };
 
     WarpAttnState<D> st;
     st.init();
@@ -69,9 +75,11 @@ __global__ void __launch_bounds__(kRowWarps * 32) attn_rows_kernel(QueryRows qr,
     int kpos = 0, blk = -1;
     while (kpos < count && (blk = row_block(dense, c, idx_row, count, kpos, n)) < 0) ++kpos;
     if (blk >= 0) {
-        warp_load_tile<D>(ks_tile, kb + (size_t)blk * kBlock * rs, rs, min(kBlock, n - blk * kBlock));
+        int nv;
+        const __nv_bfloat16* ksrc = block_src(k, blk, nv);
+        warp_load_tile<D>(ks_tile, ksrc, rs, nv);
         cp_async_commit();
-        warp_load_tile<D>(vs_tile, vb + (size_t)blk * kBlock * rs, rs, min(kBlock, n - blk * kBlock));
+        warp_load_tile<D>(vs_tile, block_src(v, blk, nv), rs, nv);
         cp_async_commit();
     }
     while (blk >= 0) {
@@ -83,15 +91,21 @@ __global__ void __launch_bounds__(kRowWarps * 32) attn_rows_kernel(QueryRows qr,
         tile_qk<D>(qf, ks_tile, acc);
         scale_mask(acc, sl2, prefix_mask64(n - blk * kBlock));
         __syncwarp();
-        if (nblk >= 0)
-            warp_load_tile<D>(ks_tile, kb + (size_t)nblk * kBlock * rs, rs, min(kBlock, n - nblk * kBlock));
+        if (nblk >= 0) {
+            int nv;
+            const __nv_bfloat16* ksrc = block_src(k, nblk, nv);
+            warp_load_tile<D>(ks_tile, ksrc, rs, nv);
+        }
         cp_async_commit();
         cp_async_wait<1>();  // V of blk
         __syncwarp();
         tile_softmax_pv<D>(st, acc, vs_tile);
         __syncwarp();
-        if (nblk >= 0)
-            warp_load_tile<D>(vs_tile, vb + (size_t)nblk * kBlock * rs, rs, min(kBlock, n - nblk * kBlock));
+        if (nblk >= 0) {
+            int nv;
+            const __nv_bfloat16* vsrc = block_src(v, nblk, nv);
+            warp_load_tile<D>(vs_tile, vsrc, rs, nv);
+        }
         cp_async_commit();
         blk = nblk;
         kpos = knext;
@@ -144,7 +158,7 @@ size_t attn_ws_bytes(int rows, int nsplit)
 
 template <int D>
 __global__ void __launch_bounds__(kSplitWarps * 32) attn_split_kernel(
-    QueryRows qr, const __nv_bfloat16* __restrict__ k, const __nv_bfloat16* __restrict__ v, int Lcap,
+    QueryRows qr, const __nv_bfloat16* __restrict__ k, const __nv_bfloat16* __restrict__ v, KvRows kr,
     const int32_t* __restrict__ idx, const int32_t* __restrict__ cnt, MethodConsts mc, int dense_all, int nsplit_blocks,
     const __nv_bfloat16* __restrict__ k_draft, const __nv_bfloat16* __restrict__ v_draft,
     const uint32_t* __restrict__ tree_mask, float* __restrict__ ws)
@@ -195,8 +209,9 @@ __global__ void __launch_bounds__(kSplitWarps * 32) attn_split_kernel(
         blk = mc.window > 0 ? (e < count ? bw + e : -1) : row_block(dense, c, idx_row, count, e, n);
         if (blk >= 0) {
             const size_t rs = (size_t)qr.Hkv * D;
-            const size_t base = ((size_t)b * Lcap * qr.Hkv + g) * D + (size_t)blk * kBlock * rs;
-            const int nvalid = min(kBlock, n - blk * kBlock);
+            const long r0 = kv_block_row(kr, b, blk);  // -1: a page the table does not map (read as zeros)
+            const size_t base = ((size_t)(r0 < 0 ? 0 : r0) * qr.Hkv + g) * D;
+            const int nvalid = r0 < 0 ? 0 : min(kBlock, n - blk * kBlock);
             warp_load_tile<D>(ks_tile, k + base, rs, nvalid);
             warp_load_tile<D>(vs_tile, v + base, rs, nvalid);
             cp_async_commit();
@@ -325,7 +340,7 @@ __global__ void __launch_bounds__(D) attn_merge_kernel(QueryRows qr, const int32
 // host side
 // =====================================================================================================
 template <int D>
-static cudaError_t rows_impl(const QueryRows& qr, const void* k, const void* v, int Lcap, const int32_t* idx,
+static cudaError_t rows_impl(const QueryRows& qr, const void* k, const void* v, const KvRows& kr, const int32_t* idx,
                              const int32_t* cnt, const MethodConsts& mc, bool dense_all, void* out, float* lse,
                              cudaStream_t s)
 {
@@ -335,20 +350,20 @@ static cudaError_t rows_impl(const QueryRows& qr, const void* k, const void* v, 
     const long rows = (long)qr.B * qr.T * qr.Hkv;
     const unsigned grid = (unsigned)((rows + kRowWarps - 1) / kRowWarps);
     return launch_pdl(attn_rows_kernel<D>, dim3(grid), dim3(kRowWarps * 32), smem, s, qr,
-                      static_cast<const __nv_bfloat16*>(k), static_cast<const __nv_bfloat16*>(v), Lcap, idx, cnt, mc,
+                      static_cast<const __nv_bfloat16*>(k), static_cast<const __nv_bfloat16*>(v), kr, idx, cnt, mc,
                       dense_all ? 1 : 0, static_cast<__nv_bfloat16*>(out), lse);
 }
 
-cudaError_t launch_attn_rows(const QueryRows& qr, const void* k, const void* v, int Lcap, const int32_t* idx,
+cudaError_t launch_attn_rows(const QueryRows& qr, const void* k, const void* v, const KvRows& kr, const int32_t* idx,
                              const int32_t* cnt, const MethodConsts& mc, bool dense_all, void* out, float* lse,
                              cudaStream_t s)
 {
-    return qr.D == 128 ? rows_impl<128>(qr, k, v, Lcap, idx, cnt, mc, dense_all, out, lse, s)
-                       : rows_impl<64>(qr, k, v, Lcap, idx, cnt, mc, dense_all, out, lse, s);
+    return qr.D == 128 ? rows_impl<128>(qr, k, v, kr, idx, cnt, mc, dense_all, out, lse, s)
+                       : rows_impl<64>(qr, k, v, kr, idx, cnt, mc, dense_all, out, lse, s);
 }
 
 template <int D>
-static cudaError_t split_impl(const QueryRows& qr, const void* k, const void* v, int Lcap, const int32_t* idx,
+static cudaError_t split_impl(const QueryRows& qr, const void* k, const void* v, const KvRows& kr, const int32_t* idx,
                               const int32_t* cnt, const MethodConsts& mc, bool dense_all, const void* k_draft,
                               const void* v_draft, const uint32_t* tree_mask, void* out, float* lse, void* ws,
                               cudaStream_t s)
@@ -362,7 +377,7 @@ static cudaError_t split_impl(const QueryRows& qr, const void* k, const void* v,
     const int rows = qr.B * qr.T * qr.Hkv;
     dim3 grid(nsplit_total, rows);
     e = launch_pdl(attn_split_kernel<D>, grid, dim3(kSplitWarps * 32), smem, s, qr,
-                   static_cast<const __nv_bfloat16*>(k), static_cast<const __nv_bfloat16*>(v), Lcap, idx, cnt, mc,
+                   static_cast<const __nv_bfloat16*>(k), static_cast<const __nv_bfloat16*>(v), kr, idx, cnt, mc,
                    dense_all ? 1 : 0, nsplit_blocks, static_cast<const __nv_bfloat16*>(k_draft),
                    static_cast<const __nv_bfloat16*>(v_draft), tree_mask, static_cast<float*>(ws));
     if (e != cudaSuccess) return e;
@@ -371,14 +386,14 @@ static cudaError_t split_impl(const QueryRows& qr, const void* k, const void* v,
                       static_cast<__nv_bfloat16*>(out), lse);
 }
 
-cudaError_t launch_attn_split(const QueryRows& qr, const void* k, const void* v, int Lcap, const int32_t* idx,
+cudaError_t launch_attn_split(const QueryRows& qr, const void* k, const void* v, const KvRows& kr, const int32_t* idx,
                               const int32_t* cnt, const MethodConsts& mc, bool dense_all, const void* k_draft,
                               const void* v_draft, const uint32_t* tree_mask, void* out, float* lse, void* ws,
                               cudaStream_t s)
 {
-    return qr.D == 128 ? split_impl<128>(qr, k, v, Lcap, idx, cnt, mc, dense_all, k_draft, v_draft, tree_mask, out,
+    return qr.D == 128 ? split_impl<128>(qr, k, v, kr, idx, cnt, mc, dense_all, k_draft, v_draft, tree_mask, out,
                                          lse, ws, s)
-                       : split_impl<64>(qr, k, v, Lcap, idx, cnt, mc, dense_all, k_draft, v_draft, tree_mask, out,
+                       : split_impl<64>(qr, k, v, kr, idx, cnt, mc, dense_all, k_draft, v_draft, tree_mask, out,
                                         lse, ws, s);
 }
 

@@ -82,7 +82,7 @@ __device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity, volatil
 
 __global__ void __launch_bounds__(kThreads, 1)
 attn_tc_kernel(QueryRows qr, const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-               const __grid_constant__ CUtensorMap tm_v, int Lcap, const int32_t* __restrict__ idx,
+               const __grid_constant__ CUtensorMap tm_v, KvRows kr, const int32_t* __restrict__ idx,
                const int32_t* __restrict__ cnt, MethodConsts mc, int dense_all, __nv_bfloat16* __restrict__ out,
                float* __restrict__ lse)
 {
@@ -95,16 +95,17 @@ attn_tc_kernel(QueryRows qr, const __grid_constant__ CUtensorMap tm_q, const __g
     uint16_t* list = reinterpret_cast<uint16_t*>(smem + kListOff);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int T = qr.T;
     const int g = blockIdx.y % qr.Hkv, b = blockIdx.y / qr.Hkv;
     // longest tiles first (later tokens attend to more blocks): the short ones fill the last wave
     const int t0 = (gridDim.x - 1 - blockIdx.x) * kTok;
+    const int Tb = q_len(qr, b);  // this sequence's queries (T unless the batch is packed)
+    if (t0 >= Tb) return;         // uniform over the CTA, before any barrier
 
     // ---- union of the tile's block sets, as one bitmap per token and an ascending list ----
     int cmax = 0;
 #pragma unroll
     for (int tt = 0; tt < kTok; ++tt)
-        if (t0 + tt < T) cmax = max(cmax, (query_ctx(qr, b, t0 + tt) - 1) / kBlock);
+        if (t0 + tt < Tb) cmax = max(cmax, (query_ctx(qr, b, t0 + tt) - 1) / kBlock);
     const int nwords = min(cmax / 32 + 1, kWords);
     for (int i = threadIdx.x; i < kTok * kWords; i += kThreads) bits[i] = 0u;
     if (threadIdx.x == 0) {
@@ -115,7 +116,7 @@ attn_tc_kernel(QueryRows qr, const __grid_constant__ CUtensorMap tm_q, const __g
     for (int item = threadIdx.x; item < kTok * max(mc.kmax, nwords); item += kThreads) {
         const int tt = item % kTok, e = item / kTok;
         const int t = t0 + tt;
-        if (t >= T) continue;
+        if (t >= Tb) continue;
         const int n = query_ctx(qr, b, t);
         const int c = (n - 1) / kBlock;
         if (dense_all || n <= mc.dense_len) {
@@ -124,7 +125,7 @@ attn_tc_kernel(QueryRows qr, const __grid_constant__ CUtensorMap tm_q, const __g
                 if (hi > lo) bits[tt * kWords + e] = (hi - lo == 32) ? 0xffffffffu : ((1u << (hi - lo)) - 1u);
             }
         } else if (e < mc.kmax) {
-            const size_t row = ((size_t)b * T + t) * qr.Hkv + g;
+            const size_t row = (size_t)q_row(qr, b, t) * qr.Hkv + g;
             if (e < min(cnt[row], mc.kmax)) {
                 const int blk = idx[row * mc.kmax + e];
                 if (blk >= 0 && blk * kBlock < n) atomicOr(&bits[tt * kWords + (blk >> 5)], 1u << (blk & 31));
@@ -195,7 +196,7 @@ attn_tc_kernel(QueryRows qr, const __grid_constant__ CUtensorMap tm_q, const __g
             tc::prefetch_tensormap(&tm_q);
             tc::prefetch_tensormap(&tm_k);
             tc::mbar_arrive_expect_tx(&bars.q_full, 2 * 128 * 128);
-            const int zq = b * T + t0;
+            const int zq = (int)q_row(qr, b, t0);  // rows past this sequence are masked (or zero-filled)
             tc::tma_load_3d(smem + kQOff, &tm_q, 0, g * kG, zq, &bars.q_full);
             tc::tma_load_3d(smem + kQOff + 16384, &tm_q, 64, g * kG, zq, &bars.q_full);
             for (int p = 0; p < NP; ++p) {
@@ -205,8 +206,10 @@ attn_tc_kernel(QueryRows qr, const __grid_constant__ CUtensorMap tm_q, const __g
                 tc::mbar_arrive_expect_tx(&bars.k_full[s], kSlot);
 #pragma unroll
                 for (int i = 0; i < 2; ++i) {
-                    // key rows [64 i, 64 i + 64) of the step, d halves in two atoms of 128 rows
-                    const int z = b * Lcap + (int)list[min(2 * p + i, U - 1)] * kBlock;
+                    // key rows [64 i, 64 i + 64) of the step, d halves in two atoms of 128 rows; an unmapped
+                    // page starts a block before row 0, which the tensor map fills with zeros
+                    const long zr = kv_block_row(kr, b, (int)list[min(2 * p + i, U - 1)]);
+                    const int z = zr >= 0 ? (int)zr : -kBlock;
                     tc::tma_load_3d(st + i * 8192, &tm_k, 0, g, z, &bars.k_full[s]);
                     tc::tma_load_3d(st + 16384 + i * 8192, &tm_k, 64, g, z, &bars.k_full[s]);
                 }
@@ -222,7 +225,8 @@ attn_tc_kernel(QueryRows qr, const __grid_constant__ CUtensorMap tm_q, const __g
                 tc::mbar_arrive_expect_tx(&bars.v_full[s], kSlot);
 #pragma unroll
                 for (int i = 0; i < 2; ++i) {
-                    const int z = b * Lcap + (int)list[min(2 * p + i, U - 1)] * kBlock;
+                    const long zr = kv_block_row(kr, b, (int)list[min(2 * p + i, U - 1)]);
+                    const int z = zr >= 0 ? (int)zr : -kBlock;
                     tc::tma_load_3d(st + i * 8192, &tm_v, 0, g, z, &bars.v_full[s]);
                     tc::tma_load_3d(st + 16384 + i * 8192, &tm_v, 64, g, z, &bars.v_full[s]);
                 }
@@ -276,7 +280,7 @@ attn_tc_kernel(QueryRows qr, const __grid_constant__ CUtensorMap tm_q, const __g
         const int r = q4 * 32 + lane;  // row = token * 16 + head
         const int tt = r >> 4, hh = r & 15;
         const int t = t0 + tt;
-        const bool valid = t < T;
+        const bool valid = t < Tb;
         const int n = valid ? query_ctx(qr, b, t) : 0;
         const uint32_t lane_addr = tmem + ((uint32_t)(q4 * 32) << 16);
         const uint32_t pair_bar = 1 + q4;
@@ -402,7 +406,7 @@ attn_tc_kernel(QueryRows qr, const __grid_constant__ CUtensorMap tm_q, const __g
         if (ok) {
             tc::tc_fence_after();
             const float inv = lt > 0.f ? 1.f / lt : 0.f;
-            __nv_bfloat16* orow = out + (((size_t)b * T + t) * qr.Hq + g * kG + hh) * kD + 64 * half;
+            __nv_bfloat16* orow = out + ((size_t)q_row(qr, b, valid ? t : 0) * qr.Hq + g * kG + hh) * kD + 64 * half;
 #pragma unroll 1
             for (int c4 = 0; c4 < 2; ++c4) {
                 uint32_t o[32];
@@ -421,7 +425,7 @@ attn_tc_kernel(QueryRows qr, const __grid_constant__ CUtensorMap tm_q, const __g
                 }
             }
             if (valid && lse && half == 0)
-                lse[((size_t)b * T + t) * qr.Hq + g * kG + hh] = lt > 0.f ? (m_ref + __log2f(lt)) * kLn2 : neg_inf();
+                lse[(size_t)q_row(qr, b, t) * qr.Hq + g * kG + hh] = lt > 0.f ? (m_ref + __log2f(lt)) * kLn2 : neg_inf();
         }
     }
     tc::tc_fence_before();
@@ -438,21 +442,21 @@ bool attn_tc_supported(const QueryRows& qr)
     return qr.D == kD && qr.Hq / qr.Hkv == kG && (qr.max_ctx - 1) / kBlock + 1 <= kMaxBlk;
 }
 
-cudaError_t launch_attn_rows_tc(const QueryRows& qr, const void* k, const void* v, int Lcap, const int32_t* idx,
-                                const int32_t* cnt, const MethodConsts& mc, bool dense_all, void* out, float* lse,
-                                cudaStream_t s)
+cudaError_t launch_attn_rows_tc(const QueryRows& qr, const void* k, const void* v, const KvRows& kr,
+                                const int32_t* idx, const int32_t* cnt, const MethodConsts& mc, bool dense_all,
+                                void* out, float* lse, cudaStream_t s)
 {
     if (!attn_tc_supported(qr)) return cudaErrorNotSupported;
     CUtensorMap tq, tk, tv;
     const uint64_t row = (uint64_t)kD * 2;
-    if (!make_tma_map_bf16(&tq, qr.q, kD, qr.Hq, (uint64_t)qr.B * qr.T, row, row * qr.Hq, kG, kTok) ||
-        !make_tma_map_bf16(&tk, k, kD, qr.Hkv, (uint64_t)qr.B * Lcap, row, row * qr.Hkv, 1, kBlock) ||
-        !make_tma_map_bf16(&tv, v, kD, qr.Hkv, (uint64_t)qr.B * Lcap, row, row * qr.Hkv, 1, kBlock))
+    if (!make_tma_map_bf16(&tq, qr.q, kD, qr.Hq, (uint64_t)qr.q_rows, row, row * qr.Hq, kG, kTok) ||
+        !make_tma_map_bf16(&tk, k, kD, qr.Hkv, (uint64_t)kr.rows, row, row * qr.Hkv, 1, kBlock) ||
+        !make_tma_map_bf16(&tv, v, kD, qr.Hkv, (uint64_t)kr.rows, row, row * qr.Hkv, 1, kBlock))
         return cudaErrorNotSupported;
     cudaError_t e = ensure_smem(attn_tc_kernel, kSmemBytes);
     if (e != cudaSuccess) return e;
     const dim3 grid((qr.T + kTok - 1) / kTok, qr.B * qr.Hkv);
-    return launch_pdl(attn_tc_kernel, grid, dim3(kThreads), (size_t)kSmemBytes, s, qr, tq, tk, tv, Lcap, idx, cnt,
+    return launch_pdl(attn_tc_kernel, grid, dim3(kThreads), (size_t)kSmemBytes, s, qr, tq, tk, tv, kr, idx, cnt,
                       mc, dense_all ? 1 : 0, static_cast<__nv_bfloat16*>(out), lse);
 }
 

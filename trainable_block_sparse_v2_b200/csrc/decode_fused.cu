@@ -156,7 +156,7 @@ IV2_DEV void scan_tile(const unsigned char* rows, int row0, int nvalid, const ui
 template <int D, int CL, int E>
 __global__ void __launch_bounds__(kFThreads, 2)
 decode_fused_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_constant__ CUtensorMap tmap_v,
-                    QueryRows qr, const __nv_bfloat16* __restrict__ kern, int nk_cap, MethodConsts mc, int Lcap,
+                    QueryRows qr, const __nv_bfloat16* __restrict__ kern, int nk_cap, MethodConsts mc, KvRows kr,
                     int32_t* __restrict__ idx, int32_t* __restrict__ cnt, __nv_bfloat16* __restrict__ out,
                     float* __restrict__ lse_out)
 {
@@ -399,17 +399,19 @@ decode_fused_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_con
     st.init();
     bool worked = false;
     {
-        const int z_base = b * Lcap;
         auto issue_block = [&](int i) {
             const int blk = dense ? bw + rank + CL * i : my_list[i];
+            // first cache row of the block; a page the table does not map starts the copy a block before row 0,
+            // which the tensor map fills with zeros
+            const long zr = kv_block_row(kr, b, blk);
+            const int zrow = zr >= 0 ? (int)zr : -kBlock;
             const int sidx = i % kFStages;
             unsigned char* stg = smem + (size_t)sidx * L::kStageBytes;
             tc::mbar_arrive_expect_tx(&full[sidx], (uint32_t)L::kStageBytes);
 #pragma unroll
             for (int dh = 0; dh < D / 64; ++dh) {
-                tc::tma_load_3d(stg + dh * L::kBoxBytes, &tmap_k, dh * 64, g, z_base + blk * kBlock, &full[sidx]);
-                tc::tma_load_3d(stg + L::kTileBytes + dh * L::kBoxBytes, &tmap_v, dh * 64, g, z_base + blk * kBlock,
-                                &full[sidx]);
+                tc::tma_load_3d(stg + dh * L::kBoxBytes, &tmap_k, dh * 64, g, zrow, &full[sidx]);
+                tc::tma_load_3d(stg + L::kTileBytes + dh * L::kBoxBytes, &tmap_v, dh * 64, g, zrow, &full[sidx]);
             }
         };
         if (tid == 0)
@@ -594,7 +596,7 @@ namespace {
 
 template <int D, int CL, int E>
 cudaError_t fused_launch(const CUtensorMap& tk, const CUtensorMap& tv, const QueryRows& qr, const void* kern,
-                         int nk_cap, const MethodConsts& mc, int Lcap, int32_t* idx, int32_t* cnt, void* out,
+                         int nk_cap, const MethodConsts& mc, const KvRows& kr, int32_t* idx, int32_t* cnt, void* out,
                          float* lse, cudaStream_t s)
 {
     auto kfn = decode_fused_kernel<D, CL, E>;
@@ -606,7 +608,7 @@ cudaError_t fused_launch(const CUtensorMap& tk, const CUtensorMap& tv, const Que
     }
     const int rows = qr.B * qr.T * qr.Hkv;
     return launch_pdl_cluster(kfn, dim3(CL, rows), dim3(kFThreads), CL, FLayout<D>::kBytes, s, tk, tv, qr,
-                              static_cast<const __nv_bfloat16*>(kern), nk_cap, mc, Lcap, idx, cnt,
+                              static_cast<const __nv_bfloat16*>(kern), nk_cap, mc, kr, idx, cnt,
                               static_cast<__nv_bfloat16*>(out), lse);
 }
 
@@ -646,7 +648,7 @@ int resident_clusters16()
 // 16-CTA clusters when every row fits in one wave of them (or the rows need 16), else 8-CTA clusters
 template <int D, int E>
 cudaError_t fused_dispatch_cl(const CUtensorMap& tk, const CUtensorMap& tv, const QueryRows& qr, const void* kern,
-                              int nk_cap, const MethodConsts& mc, int nb_max, int Lcap, int32_t* idx, int32_t* cnt,
+                              int nk_cap, const MethodConsts& mc, int nb_max, const KvRows& kr, int32_t* idx, int32_t* cnt,
                               void* out, float* lse, cudaStream_t s)
 {
     const int rows = qr.B * qr.T * qr.Hkv;
@@ -654,9 +656,9 @@ cudaError_t fused_dispatch_cl(const CUtensorMap& tk, const CUtensorMap& tv, cons
     const int r16 = resident_clusters16<D, E>();
     if (need16 || (r16 > 0 && rows <= r16)) {
         if (r16 <= 0) return cudaErrorNotSupported;
-        return fused_launch<D, 16, E>(tk, tv, qr, kern, nk_cap, mc, Lcap, idx, cnt, out, lse, s);
+        return fused_launch<D, 16, E>(tk, tv, qr, kern, nk_cap, mc, kr, idx, cnt, out, lse, s);
     }
-    return fused_launch<D, 8, E>(tk, tv, qr, kern, nk_cap, mc, Lcap, idx, cnt, out, lse, s);
+    return fused_launch<D, 8, E>(tk, tv, qr, kern, nk_cap, mc, kr, idx, cnt, out, lse, s);
 }
 
 }  // namespace
@@ -669,19 +671,20 @@ bool decode_fused_supported(const QueryRows& qr, const MethodConsts& mc)
 }
 
 cudaError_t launch_decode_fused(const QueryRows& qr, const void* kern, int nk_cap, const MethodConsts& mc,
-                                const void* k, const void* v, int Lcap, int32_t* idx, int32_t* cnt, void* out,
+                                const void* k, const void* v, const KvRows& kr, int32_t* idx, int32_t* cnt, void* out,
                                 float* lse, cudaStream_t s)
 {
     const int nb_max = (qr.max_ctx - 1) / kBlock + 1;
     if (!decode_fused_supported(qr, mc)) return cudaErrorNotSupported;
     CUtensorMap tk, tv;
     const uint64_t rowb = (uint64_t)qr.D * 2;
-    if (!make_tma_map_bf16(&tk, k, qr.D, qr.Hkv, (uint64_t)qr.B * Lcap, rowb, rowb * qr.Hkv, 1, kBlock) ||
-        !make_tma_map_bf16(&tv, v, qr.D, qr.Hkv, (uint64_t)qr.B * Lcap, rowb, rowb * qr.Hkv, 1, kBlock))
+    // the rows the caches hold: every sequence's [0, Lcap), the packed rows, or the page pool
+    if (!make_tma_map_bf16(&tk, k, qr.D, qr.Hkv, (uint64_t)kr.rows, rowb, rowb * qr.Hkv, 1, kBlock) ||
+        !make_tma_map_bf16(&tv, v, qr.D, qr.Hkv, (uint64_t)kr.rows, rowb, rowb * qr.Hkv, 1, kBlock))
         return cudaErrorNotSupported;
     // the leader's top-k keeps E = ceil(nb_max / 256) blocks per thread
 #define IV2_FUSED(DD, EE) \
-    fused_dispatch_cl<DD, EE>(tk, tv, qr, kern, nk_cap, mc, nb_max, Lcap, idx, cnt, out, lse, s)
+    fused_dispatch_cl<DD, EE>(tk, tv, qr, kern, nk_cap, mc, nb_max, kr, idx, cnt, out, lse, s)
     if (qr.D == 128) {
         if (nb_max <= 1024) return IV2_FUSED(128, 4);
         if (nb_max <= 2048) return IV2_FUSED(128, 8);

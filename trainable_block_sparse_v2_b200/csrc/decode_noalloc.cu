@@ -76,7 +76,9 @@ extern "C" int infllmv2_sparse_attn_decode_noalloc(const void* q, int batch, int
     qr.ctx_lens = ctx_lens;
     qr.same_ctx = 0;
     qr.max_ctx = max_ctx;
-    const cudaError_t e = iv2::launch_attn_split(qr, k, v, lcap, idx, cnt, mc, false, nullptr, nullptr, nullptr, out,
+    qr.cu_q = nullptr;
+    qr.q_rows = batch;
+    const cudaError_t e = iv2::launch_attn_split(qr, k, v, iv2::kv_contiguous(batch, lcap), idx, cnt, mc, false, nullptr, nullptr, nullptr, out,
                                                  lse, scratch, (cudaStream_t)stream);
     return e == cudaSuccess ? INFLLMV2_OK : INFLLMV2_ERR_CUDA;
 }

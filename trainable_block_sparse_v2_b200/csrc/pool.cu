@@ -37,7 +37,7 @@ IV2_DEV uint16_t f64_to_bf16_rne(double x)
 }
 
 template <int D>
-__global__ void __launch_bounds__(kPoolThreads) kernel_pool_kernel(const __nv_bfloat16* __restrict__ k, int Lcap,
+__global__ void __launch_bounds__(kPoolThreads) kernel_pool_kernel(const __nv_bfloat16* __restrict__ k, KvRows kr,
                                                                    int Hkv, const int32_t* __restrict__ old_lens,
                                                                    const int32_t* __restrict__ new_lens,
                                                                    __nv_bfloat16* __restrict__ kern, int nk_cap)
@@ -50,13 +50,13 @@ __global__ void __launch_bounds__(kPoolThreads) kernel_pool_kernel(const __nv_bf
 
     const int bg = blockIdx.y;
     const int b = bg / Hkv, g = bg % Hkv;
-    const int n_old = old_lens[b], n_new = new_lens[b];
+    const int n_old = old_lens ? old_lens[b] : 0;
+    const int n_new = new_lens ? new_lens[b] : kr.cu[b + 1] - kr.cu[b];
     const int j_begin = num_kernels(n_old) + blockIdx.x * kPoolKernelsPerCta;
     const int j_end = min(num_kernels(n_new), j_begin + kPoolKernelsPerCta);
     if (j_begin >= j_end || j_end > nk_cap) return;
 
     const size_t row_stride = (size_t)Hkv * D;
-    const __nv_bfloat16* kb = k + ((size_t)b * Lcap * Hkv + g) * D;
     const int n_halves = j_end - j_begin + 1;  // half windows j_begin .. j_end
 
     // half-window sums: item = (half h, chunk c)
@@ -67,8 +67,13 @@ __global__ void __launch_bounds__(kPoolThreads) kernel_pool_kernel(const __nv_bf
 #pragma unroll
         for (int e = 0; e < 8; ++e) acc[e] = 0.0;
         uint4 buf[kKernelStride];
+        // the 16 rows of a half window are consecutive in every layout (16 divides a 64-position page); a
+        // page the table does not map reads as zeros
+        const long r0 = kv_pos_row(kr, b, row0);
+        const __nv_bfloat16* hr = k + (r0 * Hkv + g) * D + c * 8;
 #pragma unroll
-        for (int r = 0; r < kKernelStride; ++r) buf[r] = ld_nc_v4(kb + (size_t)(row0 + r) * row_stride + c * 8);
+        for (int r = 0; r < kKernelStride; ++r)
+            buf[r] = r0 >= 0 ? ld_nc_v4(hr + (size_t)r * row_stride) : make_uint4(0u, 0u, 0u, 0u);
 #pragma unroll
         for (int r = 0; r < kKernelStride; ++r) {
             const uint32_t w[4] = {buf[r].x, buf[r].y, buf[r].z, buf[r].w};
@@ -98,7 +103,7 @@ __global__ void __launch_bounds__(kPoolThreads) kernel_pool_kernel(const __nv_bf
     }
 }
 
-cudaError_t launch_kernel_pool(const void* k, int B, int Lcap, int Hkv, int D, const int32_t* old_lens,
+cudaError_t launch_kernel_pool(const void* k, int B, const KvRows& kr, int Hkv, int D, const int32_t* old_lens,
                                const int32_t* new_lens, int max_new_keys, void* kern, int nk_cap, cudaStream_t s)
 {
     // windows completed by appending max_new_keys keys: at most max_new_keys / 16 + 1
@@ -107,27 +112,30 @@ cudaError_t launch_kernel_pool(const void* k, int B, int Lcap, int Hkv, int D, c
     const auto* kp = static_cast<const __nv_bfloat16*>(k);
     auto* kn = static_cast<__nv_bfloat16*>(kern);
     if (D == 128)
-        return launch_pdl(kernel_pool_kernel<128>, grid, dim3(kPoolThreads), 0, s, kp, Lcap, Hkv, old_lens, new_lens,
+        return launch_pdl(kernel_pool_kernel<128>, grid, dim3(kPoolThreads), 0, s, kp, kr, Hkv, old_lens, new_lens,
                           kn, nk_cap);
-    return launch_pdl(kernel_pool_kernel<64>, grid, dim3(kPoolThreads), 0, s, kp, Lcap, Hkv, old_lens, new_lens, kn,
+    return launch_pdl(kernel_pool_kernel<64>, grid, dim3(kPoolThreads), 0, s, kp, kr, Hkv, old_lens, new_lens, kn,
                       nk_cap);
 }
 
 // ---------------------------------------------------------------------------------------------------
 // Cache maintenance of a decode step (the pages have no counterpart): one new key and value row per
 // sequence into the caches, k_cache[b, pos[b], :, :] = k_new[b, :, :] (v likewise).  16-byte copies; a
-// position outside [0, Lcap) writes nothing.
+// position outside [0, Lcap) writes nothing.  With a paged cache the row is that of position pos[b] through
+// the page table, and a position past the table or on a page id outside [0, num_pages) writes nothing.
 // ---------------------------------------------------------------------------------------------------
 __global__ void __launch_bounds__(256) kv_append_kernel(const uint4* __restrict__ k_new, const uint4* __restrict__ v_new,
-                                                       const int32_t* __restrict__ pos, int Lcap, int row16,
+                                                       const int32_t* __restrict__ pos, KvRows kr, int row16,
                                                        uint4* __restrict__ k_cache, uint4* __restrict__ v_cache)
 {
     pdl_launch_dependents();
     pdl_wait();
     const int b = blockIdx.x;
     const int p = pos[b];
-    if (p < 0 || p >= Lcap) return;
-    const size_t dst = ((size_t)b * Lcap + p) * row16;
+    if (p < 0 || (!kr.table && p >= kr.Lcap)) return;
+    const long r = kv_pos_row(kr, b, p);
+    if (r < 0) return;
+    const size_t dst = (size_t)r * row16;
     for (int i = threadIdx.x; i < 2 * row16; i += blockDim.x) {
         if (i < row16) k_cache[dst + i] = k_new[(size_t)b * row16 + i];
         else v_cache[dst + i - row16] = v_new[(size_t)b * row16 + i - row16];
@@ -135,11 +143,11 @@ __global__ void __launch_bounds__(256) kv_append_kernel(const uint4* __restrict_
 }
 
 cudaError_t launch_kv_append(const void* k_new, const void* v_new, int B, int Hkv, int D, const int32_t* pos,
-                             void* k_cache, void* v_cache, int Lcap, cudaStream_t s)
+                             void* k_cache, void* v_cache, const KvRows& kr, cudaStream_t s)
 {
     const int row16 = Hkv * D / 8;  // 16-byte chunks of one position's keys (all KV heads)
     return launch_pdl(kv_append_kernel, dim3(B), dim3(256), 0, s, static_cast<const uint4*>(k_new),
-                      static_cast<const uint4*>(v_new), pos, Lcap, row16, static_cast<uint4*>(k_cache),
+                      static_cast<const uint4*>(v_new), pos, kr, row16, static_cast<uint4*>(k_cache),
                       static_cast<uint4*>(v_cache));
 }
 

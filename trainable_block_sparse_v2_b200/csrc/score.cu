@@ -71,8 +71,10 @@ __global__ void __launch_bounds__(kScanThreads) score_scan_kernel(QueryRows qr, 
     pdl_launch_dependents();
     pdl_wait();
     __shared__ float zs[16][kChunkSlots];
-    const int row = blockIdx.y;  // (b, t, g)
-    const int g = row % qr.Hkv, bt = row / qr.Hkv, t = bt % qr.T, b = bt / qr.T;
+    const int row = blockIdx.y;  // (b, t, g); the workspace is indexed by it
+    const int g = row % qr.Hkv, t = (row / qr.Hkv) % qr.T, b = row / qr.Hkv / qr.T;
+    if (t >= q_len(qr, b)) return;  // past this sequence's queries (packed batch)
+    const long bt = q_row(qr, b, t);
     const int G = qr.Hq / qr.Hkv;
     const int n = query_ctx(qr, b, t);
     if (n <= mc.dense_len) return;
@@ -173,14 +175,16 @@ __global__ void __launch_bounds__(kSelThreads) score_select_kernel(QueryRows qr,
     __shared__ CtaSelectSmem sel_sm;
     cg::cluster_group cluster = cg::this_cluster();
     const int rank = (int)cluster.block_rank();
-    const int row = blockIdx.y;
-    const int bt = row / qr.Hkv, t = bt % qr.T, b = bt / qr.T;
+    const int row = blockIdx.y;  // (b, t, g): the workspace row
+    const int t = (row / qr.Hkv) % qr.T, b = row / qr.Hkv / qr.T;
+    if (t >= q_len(qr, b)) return;  // past this sequence's queries: uniform over the cluster
+    const long orow = q_row(qr, b, t) * qr.Hkv + row % qr.Hkv;  // row of idx / cnt
     const int G = qr.Hq / qr.Hkv;
     const int n = query_ctx(qr, b, t);
     const int c = (n - 1) / kBlock;
-    int32_t* idx_row = idx + (size_t)row * mc.kmax;
+    int32_t* idx_row = idx + (size_t)orow * mc.kmax;
     if (n <= mc.dense_len) {  // uniform over the cluster: nobody touches distributed shared memory
-        if (rank == 0 && threadIdx.x < 32) warp_write_dense_row(c, mc.kmax, idx_row, cnt + row);
+        if (rank == 0 && threadIdx.x < 32) warp_write_dense_row(c, mc.kmax, idx_row, cnt + orow);
         return;
     }
     const int nchunk = score_nchunk(nb_max);
@@ -230,7 +234,7 @@ __global__ void __launch_bounds__(kSelThreads) score_select_kernel(QueryRows qr,
     }
     cluster.sync();  // release/acquire: the leader sees every score
     if (rank != 0) return;
-    cta_select_topk<kSelThreads, E>(S, c, mc.init_blocks, mc.local_blocks, mc.topk, mc.kmax, idx_row, cnt + row,
+    cta_select_topk<kSelThreads, E>(S, c, mc.init_blocks, mc.local_blocks, mc.topk, mc.kmax, idx_row, cnt + orow,
                                     sel_sm);
 }
 
@@ -307,7 +311,8 @@ __global__ void __launch_bounds__(kPfThreads) score_prefill_kernel(QueryRows qr,
     const int g = blockIdx.y % qr.Hkv, b = blockIdx.y / qr.Hkv;
     const int t0 = blockIdx.x * TPC;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, gq = lane >> 2, tq = lane & 3;
-    const int T = qr.T;
+    const int T = q_len(qr, b);  // this sequence's queries (qr.T unless the batch is packed)
+    if (t0 >= T) return;         // uniform over the CTA, before any barrier
 
     if (threadIdx.x == 0) n_max_sh = 0;
     __syncthreads();
@@ -339,7 +344,7 @@ __global__ void __launch_bounds__(kPfThreads) score_prefill_kernel(QueryRows qr,
             qf[ks][i] = 0u;
             if (any_sparse && tk < T)
                 qf[ks][i] = *reinterpret_cast<const uint32_t*>(
-                    qbase + (((size_t)b * T + tk) * qr.Hq + g * G + hh) * D + dcol);
+                    qbase + ((size_t)q_row(qr, b, tk) * qr.Hq + g * G + hh) * D + dcol);
         }
     }
 
@@ -467,7 +472,7 @@ __global__ void __launch_bounds__(kPfThreads) score_prefill_kernel(QueryRows qr,
         if (tk >= T) break;
         const int n = query_ctx(qr, b, tk);
         const int c = (n - 1) / kBlock;
-        const size_t row = ((size_t)b * T + tk) * qr.Hkv + g;
+        const size_t row = (size_t)q_row(qr, b, tk) * qr.Hkv + g;
         if (n <= mc.dense_len)
             warp_write_dense_row(c, mc.kmax, idx + row * mc.kmax, cnt + row);
         else

@@ -104,10 +104,11 @@ score_tc_kernel(QueryRows qr, const __grid_constant__ CUtensorMap tm_q, const __
     float* hs_sm = hm_sm + kSParts * 256;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int T = qr.T;
     const int g = blockIdx.y % qr.Hkv, b = blockIdx.y / qr.Hkv;
     // longest tiles first (later tokens see more kernels): the short ones fill the last wave
     const int t0 = (gridDim.x - 1 - blockIdx.x) * kSTok;
+    const int T = q_len(qr, b);  // this sequence's queries (qr.T unless the batch is packed)
+    if (t0 >= T) return;         // uniform over the CTA, before any barrier
 
     int n_max = 0;
     bool any_sparse = false;
@@ -121,7 +122,7 @@ score_tc_kernel(QueryRows qr, const __grid_constant__ CUtensorMap tm_q, const __
     if (!any_sparse) {  // uniform over the CTA: dense rows only
         for (int tt = warp; tt < kSTok && t0 + tt < T; tt += kSThreads / 32) {
             const int n = query_ctx(qr, b, t0 + tt);
-            const size_t row = ((size_t)b * T + t0 + tt) * qr.Hkv + g;
+            const size_t row = (size_t)q_row(qr, b, t0 + tt) * qr.Hkv + g;
             warp_write_dense_row((n - 1) / kBlock, mc.kmax, idx + row * mc.kmax, cnt + row);
         }
         return;
@@ -166,7 +167,7 @@ score_tc_kernel(QueryRows qr, const __grid_constant__ CUtensorMap tm_q, const __
             tc::mbar_arrive_expect_tx(&bars.q_full, kSQBytes);
 #pragma unroll
             for (int tile = 0; tile < 2; ++tile) {
-                const int zq = b * T + t0 + kSTile * tile;
+                const int zq = (int)q_row(qr, b, t0 + kSTile * tile);  // rows past the sequence are masked
                 tc::tma_load_3d(smem + kSQOff + 32768 * tile, &tm_q, 0, g * kSG, zq, &bars.q_full);
                 tc::tma_load_3d(smem + kSQOff + 32768 * tile + 16384, &tm_q, 64, g * kSG, zq, &bars.q_full);
             }
@@ -364,7 +365,7 @@ score_tc_kernel(QueryRows qr, const __grid_constant__ CUtensorMap tm_q, const __
             const int tsel = t0 + ts;
             const int ns = query_ctx(qr, b, tsel);
             const int cs = (ns - 1) / kBlock;
-            const size_t row = ((size_t)b * T + tsel) * qr.Hkv + g;
+            const size_t row = (size_t)q_row(qr, b, tsel) * qr.Hkv + g;
             if (ns <= mc.dense_len)
                 warp_write_dense_row(cs, mc.kmax, idx + row * mc.kmax, cnt + row);
             else if (cs >= nb_max) {  // a context past the launch's max_ctx: no scores for it
@@ -411,7 +412,7 @@ cudaError_t launch_score_tc(const QueryRows& qr, const void* kern, int nk_cap, c
     if (!score_tc_supported(qr, nb_max)) return cudaErrorNotSupported;
     CUtensorMap tq, tk, tks;
     const uint64_t row = (uint64_t)kSD * 2;
-    if (!make_tma_map_bf16(&tq, qr.q, kSD, qr.Hq, (uint64_t)qr.B * qr.T, row, row * qr.Hq, kSG, kSTile) ||
+    if (!make_tma_map_bf16(&tq, qr.q, kSD, qr.Hq, (uint64_t)qr.q_rows, row, row * qr.Hq, kSG, kSTile) ||
         !make_tma_map_bf16(&tk, kern, kSD, (uint64_t)nk_cap, (uint64_t)qr.B * qr.Hkv, row, row * nk_cap, 128, 1))
         return cudaErrorNotSupported;
     // the LSE estimate's view: every ls-th kernel row (row stride ls rows; rows past nk_cap are outside the map)
