@@ -1162,10 +1162,11 @@ def run_ours(args):
             err = f"{type(e).__name__}: {e}"[:300]
         tp, tc = barrier_max(tp, ws), barrier_max(tc, ws)
         if err is None and tp == tp:
-            _, _, bp = decode_step_bytes(list(pg.lens_h))
+            _, _, bp = decode_step_bytes([int(n) for n in pg.lens_h])
             line["paged_decode"] = {
                 "workload": "decode_128k_ragged step 0 on 64-position pages (shuffled page table)",
                 "value": whole_job_rate(len(pg.lens_h), ws, tp), "unit": UNIT, "us_per_step": tp * 1e6,
+                "seq_lens": [int(n) for n in pg.lens_h],
                 "contiguous_us_per_step": tc * 1e6, "timing": "median of 300 steps, L2 flushed before each",
                 "algorithmic_bytes": bp, "frac_of_" + peak_kind: bp / tp / 1e9 / peaks["hbm_gbs"],
                 "note": "one step = kernel_pool_paged of the new key + sparse_decode_step_paged",

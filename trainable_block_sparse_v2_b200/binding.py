@@ -71,6 +71,7 @@ _SIGS = {
     "infllmv2_status_string": ([_I], ctypes.c_char_p),
     "infllmv2_version": ([], _I),
     "infllmv2_device_status": ([], _I),
+    "infllmv2_test_set_first_wait_limit": ([ctypes.c_uint], _I),
     "infllmv2_workspace_size": ([_PP, _I, _I, _I, _I, _I, _I], _SZ),
     "infllmv2_kernel_pool": ([_P, _I, _I, _I, _I, _P, _P, _I, _PP, _P, _I, _P], _I),
     "infllmv2_kv_append": ([_P, _P, _I, _I, _I, _P, _P, _P, _I, _P], _I),

@@ -732,4 +732,9 @@ int infllmv2_sparse_prefill_varlen(const void* q, const void* k, const void* v, 
     return launched(iv2::launch_attn_rows(qr, k, v, kr, idx, cnt, mc, false, out, lse, s));
 }
 
+int infllmv2_test_set_first_wait_limit(unsigned polls)
+{
+    return iv2::fused_set_first_wait_limit(polls) == 0 ? INFLLMV2_OK : INFLLMV2_ERR_CUDA;
+}
+
 }  // extern "C"

@@ -86,6 +86,8 @@ struct FLayout {
 };
 
 __device__ int g_fused_error = 0;
+// testing only: when nonzero, the first kernel-cache wait of every CTA gives up after this many polls
+__device__ unsigned g_fused_first_wait_limit = 0u;
 
 // order-preserving key -> float (inverse of float_key)
 IV2_DEV float key_float(uint32_t k) { return __uint_as_float((k & 0x80000000u) ? (k & 0x7fffffffu) : ~k); }
@@ -164,6 +166,8 @@ decode_fused_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_con
     extern __shared__ unsigned char smem_raw[];
     unsigned char* smem = tc::align_smem_1024(smem_raw);
     __shared__ uint64_t full[kFStages];
+    __shared__ uint64_t never;  // testing only: a barrier no thread or copy arrives on
+    __shared__ uint32_t n_issued, n_done;  // thread 0: copies issued / seen complete per ring stage (8 bits each)
     __shared__ float part_m[16], part_s[16], lse2[16], halo_out[16];
     __shared__ __align__(16) float lse_slot[kFMaxCL][16][2];  // (max, sum) partials pushed by every CTA
 
@@ -183,6 +187,8 @@ decode_fused_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_con
     for (int i = tid; i < 16 * kFBmaxPitch; i += kFThreads) bmax[i] = 0u;
     if (tid == 0) {
         for (int s = 0; s < kFStages; ++s) tc::mbar_init(&full[s], 1);
+        tc::mbar_init(&never, 1);
+        n_issued = n_done = 0u;
         tc::fence_barrier_init();
         tc::prefetch_tensormap(&tmap_k);
         tc::prefetch_tensormap(&tmap_v);
@@ -212,6 +218,20 @@ decode_fused_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_con
     const float sl2 = mc.scale * kLog2e;
     uint32_t phase_bits = 0;  // parity of each ring stage
     bool failed = bad;
+    // A wait that runs out (bounded polls) makes the whole CTA stop: it learns of it at the stage's barrier
+    // (__syncthreads_or), issues no further copy, skips the rest of its loads and attention, still takes part
+    // in every cluster barrier (with neutral partials), and before its shared memory is reused waits, bounded,
+    // for the copies still in flight.  Thread 0 counts the copies issued and seen complete per ring stage
+    // (n_issued, n_done); the k-th completion of a stage has parity k & 1.
+    bool cta_failed = false;
+    auto drain = [&]() {
+        if (tid == 0)
+            for (int s = 0; s < kFStages; ++s) {
+                const uint32_t is = (n_issued >> (8 * s)) & 255u, dn = (n_done >> (8 * s)) & 255u;
+                if (is != dn) (void)tc::mbar_wait(&full[s], dn & 1u, 1u << 20);
+            }
+        __syncthreads();
+    };
 
     // ---------------- 1. scan this CTA's blocks of the kernel cache ----------------
     const int nch = (sparse && nown > 0) ? (nown + kFChunkBlocks - 1) / kFChunkBlocks : 0;
@@ -221,6 +241,7 @@ decode_fused_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_con
             const int sc = b0 + i * kFChunkBlocks, se = min(sc + kFChunkBlocks, b1);
             const int lo = sc * kKernelsPerBlock, hi = min(se * kKernelsPerBlock, nkv);
             uint64_t* bar = &full[i % kFStages];
+            n_issued += 1u << (8 * (i % kFStages));
             if (hi > lo) {
                 tc::mbar_arrive_expect_tx(bar, (uint32_t)(hi - lo) * D * 2);
                 tc::bulk_load(smem + (size_t)(i % kFStages) * L::kChunkBytes, kbase + (size_t)lo * D,
@@ -244,49 +265,70 @@ decode_fused_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_con
 
         for (int i = 0; i < nch; ++i) {
             const int st = i % kFStages;
-            if (!tc::mbar_wait(&full[st], (phase_bits >> st) & 1u, 1u << 24)) failed = true;
+            // testing only (a limit set from the host): the first wait polls a barrier nothing arrives on, so it
+            // runs out after that many polls while the stage's copy is still in flight
+            const uint32_t tlim = i == 0 ? g_fused_first_wait_limit : 0u;
+            const bool landed = tlim ? tc::mbar_wait(&never, 0u, tlim)
+                                     : tc::mbar_wait(&full[st], (phase_bits >> st) & 1u, 1u << 24);
+            failed |= !landed;
+            if (landed && tid == 0) n_done += 1u << (8 * st);
             phase_bits ^= 1u << st;
-            const int sc = b0 + i * kFChunkBlocks, se = min(sc + kFChunkBlocks, b1);
-            const int nblk = se - sc;
-            const int nvalid = max(min(se * kKernelsPerBlock, nkv) - sc * kKernelsPerBlock, 0);  // rows staged
-            const unsigned char* rows = smem + (size_t)st * L::kChunkBytes;
-            // this warp's tiles: warp and warp + 8 of the stage's 16 (4 kernel rows per block, 8 per tile)
-            float z[2][4];
+            // a warp with a lane that did not see the stage land skips it (its bytes may not be there)
+            if (!__any_sync(0xffffffffu, !landed)) {
+                const int sc = b0 + i * kFChunkBlocks, se = min(sc + kFChunkBlocks, b1);
+                const int nblk = se - sc;
+                const int nvalid = max(min(se * kKernelsPerBlock, nkv) - sc * kKernelsPerBlock, 0);  // rows staged
+                const unsigned char* rows = smem + (size_t)st * L::kChunkBytes;
+                // this warp's tiles: warp and warp + 8 of the stage's 16 (4 kernel rows per block, 8 per tile)
+                float z[2][4];
 #pragma unroll
-            for (int j = 0; j < 2; ++j) scan_tile<D>(rows, 8 * (warp + 8 * j), nvalid, qa, qb, sl2, z[j]);
-            // LSE partials, branch-free (every row of the stage is owned by this CTA; invalid scores are -inf)
-#pragma unroll
-            for (int r = 0; r < 2; ++r) {
-                const float m4 = fmaxf(fmaxf(z[0][2 * r], z[0][2 * r + 1]), fmaxf(z[1][2 * r], z[1][2 * r + 1]));
-                const float mn = fmaxf(lm[r], m4);
-                ls[r] = ls[r] * ex2_approx(lm[r] - mn) + (ex2_approx(z[0][2 * r] - mn) + ex2_approx(z[0][2 * r + 1] - mn)) +
-                        (ex2_approx(z[1][2 * r] - mn) + ex2_approx(z[1][2 * r + 1] - mn));
-                lm[r] = mn;
-            }
-            // block maxima: tile j holds the stage's blocks 2 tt and 2 tt + 1 (tt = warp + 8 j) as cols 0..3 and
-            // 4..7, so lane tq's two cols belong to block 2 tt + (tq >> 1).  Shuffle-free, one atomicMax per
-            // lane for its own block; under the overlapping-window rule an odd lane's second col is the last
-            // kernel of that block and also goes to the block after it (in this CTA, or the next CTA's first).
-#pragma unroll
-            for (int j = 0; j < 2; ++j) {
-                const int tt = warp + 8 * j;
-                const int own = sc - b0 + 2 * tt + (tq >> 1);  // CTA-local block of this lane's cols
-                const bool own_ok = 2 * tt + (tq >> 1) < nblk;
+                for (int j = 0; j < 2; ++j) scan_tile<D>(rows, 8 * (warp + 8 * j), nvalid, qa, qb, sl2, z[j]);
+                // LSE partials, branch-free (every row of the stage is owned by this CTA; invalid scores are -inf)
 #pragma unroll
                 for (int r = 0; r < 2; ++r) {
-                    const float v0 = z[j][2 * r], v1 = z[j][2 * r + 1];
-                    // contained windows: a block's kernels are cols 0..2 of its four
-                    const float vo = (!overlap && (tq & 1)) ? v0 : fmaxf(v0, v1);
-                    uint32_t* bm = bmax + (gq + 8 * r) * kFBmaxPitch;
-                    if (hv[r] && own_ok && vo != neg_inf()) atomicMax(&bm[own], float_key(vo));
-                    if (overlap && (tq & 1) && hv[r] && own_ok && v1 != neg_inf()) {
-                        if (own + 1 < nown) atomicMax(&bm[own + 1], float_key(v1));
-                        else halo_out[gq + 8 * r] = v1;  // the CTA's last kernel: next CTA's block 0
+                    const float m4 = fmaxf(fmaxf(z[0][2 * r], z[0][2 * r + 1]), fmaxf(z[1][2 * r], z[1][2 * r + 1]));
+                    const float mn = fmaxf(lm[r], m4);
+                    ls[r] = ls[r] * ex2_approx(lm[r] - mn) + (ex2_approx(z[0][2 * r] - mn) + ex2_approx(z[0][2 * r + 1] - mn)) +
+                            (ex2_approx(z[1][2 * r] - mn) + ex2_approx(z[1][2 * r + 1] - mn));
+                    lm[r] = mn;
+                }
+                // block maxima: tile j holds the stage's blocks 2 tt and 2 tt + 1 (tt = warp + 8 j) as cols 0..3 and
+                // 4..7, so lane tq's two cols belong to block 2 tt + (tq >> 1).  Shuffle-free, one atomicMax per
+                // lane for its own block; under the overlapping-window rule an odd lane's second col is the last
+                // kernel of that block and also goes to the block after it (in this CTA, or the next CTA's first).
+#pragma unroll
+                for (int j = 0; j < 2; ++j) {
+                    const int tt = warp + 8 * j;
+                    const int own = sc - b0 + 2 * tt + (tq >> 1);  // CTA-local block of this lane's cols
+                    const bool own_ok = 2 * tt + (tq >> 1) < nblk;
+#pragma unroll
+                    for (int r = 0; r < 2; ++r) {
+                        const float v0 = z[j][2 * r], v1 = z[j][2 * r + 1];
+                        // contained windows: a block's kernels are cols 0..2 of its four
+                        const float vo = (!overlap && (tq & 1)) ? v0 : fmaxf(v0, v1);
+                        uint32_t* bm = bmax + (gq + 8 * r) * kFBmaxPitch;
+                        if (hv[r] && own_ok && vo != neg_inf()) atomicMax(&bm[own], float_key(vo));
+                        if (overlap && (tq & 1) && hv[r] && own_ok && v1 != neg_inf()) {
+                            if (own + 1 < nown) atomicMax(&bm[own + 1], float_key(v1));
+                            else halo_out[gq + 8 * r] = v1;  // the CTA's last kernel: next CTA's block 0
+                        }
                     }
                 }
+            }  // the stage's scores
+            // stage consumed by every warp; a wait that ran out anywhere in the CTA stops the scan
+            if (__syncthreads_or(!landed)) {
+                cta_failed = true;
+                break;
             }
-            __syncthreads();  // stage consumed by every warp
             if (tid == 0 && i + kFStages < nch) issue_chunk(i + kFStages);
+        }
+        if (cta_failed) {
+            // this CTA contributes no kernel to the LSE and no block maximum to the scores
+            lm[0] = lm[1] = kFloor;
+            ls[0] = ls[1] = 0.f;
+            for (int k2 = tid; k2 < 16 * kFBmaxPitch; k2 += kFThreads) bmax[k2] = 0u;
+            if (tid < 16) halo_out[tid] = neg_inf();
+            drain();
         }
         for (int r = 0; r < 2; ++r)
             if (lm[r] == kFloor) lm[r] = neg_inf();
@@ -394,7 +436,7 @@ decode_fused_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_con
     tc::fence_proxy_async_smem();
 
     // ---------------- 4. attention over this CTA's entries rank, rank + CL, ... ----------------
-    const int my_n = count > rank ? (count - rank + CL - 1) / CL : 0;
+    const int my_n = (count > rank && !cta_failed) ? (count - rank + CL - 1) / CL : 0;
     WarpAttnState<D> st;
     st.init();
     bool worked = false;
@@ -407,6 +449,7 @@ decode_fused_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_con
             const int zrow = zr >= 0 ? (int)zr : -kBlock;
             const int sidx = i % kFStages;
             unsigned char* stg = smem + (size_t)sidx * L::kStageBytes;
+            n_issued += 1u << (8 * sidx);
             tc::mbar_arrive_expect_tx(&full[sidx], (uint32_t)L::kStageBytes);
 #pragma unroll
             for (int dh = 0; dh < D / 64; ++dh) {
@@ -423,7 +466,9 @@ decode_fused_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_con
         const int krow = key0 + (lane & 7);  // the key row this lane addresses in ldmatrix
         for (int i = 0; i < my_n; ++i) {
             const int sidx = i % kFStages;
-            if (!tc::mbar_wait(&full[sidx], (phase_bits >> sidx) & 1u, 1u << 24)) failed = true;
+            const bool landed = tc::mbar_wait(&full[sidx], (phase_bits >> sidx) & 1u, 1u << 24);
+            failed |= !landed;
+            if (landed && tid == 0) n_done += 1u << (8 * sidx);
             phase_bits ^= 1u << sidx;
             const int blk = dense ? bw + rank + CL * i : my_list[i];
             const int nvalid = min(kBlock, n - blk * kBlock);
@@ -431,7 +476,8 @@ decode_fused_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_con
             unsigned char* stg = smem + (size_t)sidx * L::kStageBytes;
             // a warp works when one of its 8 keys is in [nskip, nvalid) (nskip < nvalid for every walked block),
             // so every row's running max is finite after its first block
-            if (key0 < nvalid && key0 + 8 > nskip) {
+            // a warp with a lane that did not see the stage land skips it (its bytes may not be there)
+            if (key0 < nvalid && key0 + 8 > nskip && !__any_sync(0xffffffffu, !landed)) {
                 unsigned char* vt = stg + L::kTileBytes;
                 if (key0 + 8 > nvalid) {
                     // rows past the context may hold anything: zero them so that 0 * V stays 0
@@ -496,9 +542,14 @@ decode_fused_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_con
                 }
                 worked = true;
             }
-            __syncthreads();  // stage consumed by every warp
+            // stage consumed by every warp; a wait that ran out anywhere in the CTA stops the walk
+            if (__syncthreads_or(!landed)) {
+                cta_failed = true;
+                break;
+            }
             if (tid == 0 && i + kFStages < my_n) issue_block(i + kFStages);
         }
+        if (cta_failed) drain();
     }
     finalize_rows<D>(st);
     // the eight warp states -> this CTA's partial: factors 2^(m_w - M) once per (warp, head), then sums
@@ -583,12 +634,9 @@ decode_fused_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_con
                 lse_out[(size_t)bt * qr.Hq + g * G + h] = Lsum > 0.f ? (M + __log2f(Lsum)) * kLn2 : neg_inf();
         }
     }
-    if (failed) {
-        atomicOr(&g_fused_error, 1);
-        // a wait ran out: give every copy still in flight a bounded chance to land before the CTA exits
-        if (tid == 0)
-            for (int s = 0; s < kFStages; ++s) (void)tc::mbar_wait(&full[s], (phase_bits >> s) & 1u, 1u << 20);
-    }
+    // a wait that ran out (or a context past the launch's tables): the results of this row are not the method's;
+    // the copies still in flight were waited for where the loop stopped
+    if (failed) atomicOr(&g_fused_error, 1);
 }
 
 // ---------------------------------------------------------------- host
@@ -694,6 +742,12 @@ cudaError_t launch_decode_fused(const QueryRows& qr, const void* kern, int nk_ca
     if (nb_max <= 2048) return IV2_FUSED(64, 8);
     return IV2_FUSED(64, 12);
 #undef IV2_FUSED
+}
+
+// testing only: the poll limit of the first kernel-cache wait of every CTA (0: the normal wait)
+int fused_set_first_wait_limit(unsigned polls)
+{
+    return cudaMemcpyToSymbol(g_fused_first_wait_limit, &polls, sizeof(unsigned)) == cudaSuccess ? 0 : -1;
 }
 
 int fused_error_flag_read_and_clear()

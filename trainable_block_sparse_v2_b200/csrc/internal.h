@@ -206,6 +206,7 @@ cudaError_t launch_decode_fused(const QueryRows& qr, const void* kern, int nk_ca
                                 const void* k, const void* v, const KvRows& kr, int32_t* idx, int32_t* cnt, void* out,
                                 float* lse, cudaStream_t s);
 int fused_error_flag_read_and_clear();
+int fused_set_first_wait_limit(unsigned polls);  // testing only
 
 // attention split over the selected blocks across CTAs, merged by LSE (decode and tree verification)
 cudaError_t launch_attn_split(const QueryRows& qr, const void* k, const void* v, const KvRows& kr, const int32_t* idx,
