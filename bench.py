@@ -483,6 +483,31 @@ def prefill_flops(T=32768, dense_len=8192, kmax=67):
     return score, attn, dense
 
 
+def attn_tc_executed_flops(idx, cnt, T, dense_len, tok=8, step_keys=128):
+    """MMA flops the tensor-core prefill attention issues for this selection: each 8-token tile walks the union of
+    its tokens' block sets (every block 0..c for a dense row), two 64-key blocks per step (an odd last block is
+    paired with a masked copy), and every step runs S = Q K^T and O += P V on 128 rows x 128 keys x d."""
+    idx = np.asarray(idx)[0]  # [T, Hkv, kmax]
+    cnt = np.asarray(cnt)[0]  # [T, Hkv]
+    nb = (T - 1) // 64 + 1
+    total = 0
+    for g in range(idx.shape[1]):
+        sel = np.zeros((T, nb), bool)
+        k = idx[:, g, :]
+        valid = (np.arange(k.shape[1])[None, :] < cnt[:, g][:, None]) & (k >= 0)
+        rows = np.nonzero(valid)
+        sel[rows[0], k[valid]] = True
+        t = np.arange(T)
+        dense = (t + 1) <= dense_len
+        c = t // 64
+        sel[dense] = np.arange(nb)[None, :] <= c[dense][:, None]
+        ntile = (T + tok - 1) // tok
+        pad = ntile * tok - T
+        un = np.concatenate([sel, np.zeros((pad, nb), bool)]).reshape(ntile, tok, nb).any(axis=1).sum(axis=1)
+        total += int(((un + 1) // 2).sum())
+    return total * 2 * (2 * 128 * step_keys * D)
+
+
 class PrefillBench:
     def __init__(self):
         import torch
@@ -1076,6 +1101,10 @@ def run_ours(args):
             "workload": "prefill_32k", "value": whole_job_rate(pb.T * args.prefill_steps, ws, pt), "unit": UNIT,
             "ms_per_step": pt / args.prefill_steps * 1e3, "steps": args.prefill_steps,
             "algorithmic_tflop_per_step": flops / 1e12,
+            "executed_tflop": {"sparse_attn_prefill": attn_tc_executed_flops(pb.idx.cpu().numpy(), pb.cnt.cpu().numpy(),
+                                                                             pb.T, pb.p.dense_len) / 1e12,
+                               "note": "MMA flops issued by the tensor-core attention (8-token tiles over the union "
+                                       "of their block sets), against af + df algorithmic"},
             "tc_frac_of_" + peak_kind: flops / (pt / args.prefill_steps) / 1e12 / peaks["bf16_tflops"],
             "per_call_ms": {k: v * 1e3 for k, v in pper.items()},
             "roofline": {"bound": "tensor", "kernel": pdom, "achieved": pach, "peak": peaks["bf16_tflops"],
