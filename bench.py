@@ -797,7 +797,9 @@ class VarlenPrefillBench:
         self.idx = torch.empty((self.T, HKV, self.p.kmax), dtype=torch.int32, device=dev)
         self.cnt = torch.empty((self.T, HKV), dtype=torch.int32, device=dev)
         self.out = torch.empty((self.T, HQ, D), dtype=torch.bfloat16, device=dev)
-        self.ws = binding.workspace(self.p, B, self.Lmax, self.Lmax, HQ, HKV, D)
+        # the packed scoring of long prompts runs on the token tiles, which need no workspace (a workspace sized
+        # for every entry point at B x 32K rows would be the split attention's, hundreds of GB)
+        self.ws = None
         self.lens = [torch.tensor([T], dtype=torch.int32, device=dev) for T in self.LENS]
         self.kerns = [torch.zeros((1, HKV, nk(T), D), dtype=torch.bfloat16, device=dev) for T in self.LENS]
         self.zero = torch.zeros(1, dtype=torch.int32, device=dev)

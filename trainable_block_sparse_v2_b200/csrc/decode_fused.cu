@@ -80,8 +80,9 @@ struct FLayout {
     static constexpr int kBmaxBytes = 16 * kFBmaxPitch * 4;
     static constexpr int kSlotPitch = D + 4;                   // floats: O[D], m, l (16-byte rows)
     static constexpr int kSlotBytes = 16 * kSlotPitch * 4;     // [heads / CL][CL][kSlotPitch]
-    static constexpr int kMyList = kBmax + kSlotBytes;         // int32 [kFListCap]
-    static constexpr int kEnd = kBmax + cmax(kBmaxBytes, kSlotBytes + kFListCap * 4);
+    static constexpr int kMyList = kBmax + kSlotBytes;         // int32 [kFListCap] block ids
+    static constexpr int kMyRows = kMyList + kFListCap * 4;    // int32 [kFListCap] first cache row of each
+    static constexpr int kEnd = kBmax + cmax(kBmaxBytes, kSlotBytes + 2 * kFListCap * 4);
     static constexpr int kBytes = kEnd + 1024;                 // + slack to align the base to 1024 B
 };
 
@@ -273,48 +274,47 @@ decode_fused_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_con
             failed |= !landed;
             if (landed && tid == 0) n_done += 1u << (8 * st);
             phase_bits ^= 1u << st;
-            // a warp with a lane that did not see the stage land skips it (its bytes may not be there)
-            if (!__any_sync(0xffffffffu, !landed)) {
-                const int sc = b0 + i * kFChunkBlocks, se = min(sc + kFChunkBlocks, b1);
-                const int nblk = se - sc;
-                const int nvalid = max(min(se * kKernelsPerBlock, nkv) - sc * kKernelsPerBlock, 0);  // rows staged
-                const unsigned char* rows = smem + (size_t)st * L::kChunkBytes;
-                // this warp's tiles: warp and warp + 8 of the stage's 16 (4 kernel rows per block, 8 per tile)
-                float z[2][4];
+            // a stage that did not land in some thread is computed all the same: the CTA then stops below, and
+            // resets everything the stage wrote (block maxima, halo, LSE partials) before anything reads it
+            const int sc = b0 + i * kFChunkBlocks, se = min(sc + kFChunkBlocks, b1);
+            const int nblk = se - sc;
+            const int nvalid = max(min(se * kKernelsPerBlock, nkv) - sc * kKernelsPerBlock, 0);  // rows staged
+            const unsigned char* rows = smem + (size_t)st * L::kChunkBytes;
+            // this warp's tiles: warp and warp + 8 of the stage's 16 (4 kernel rows per block, 8 per tile)
+            float z[2][4];
 #pragma unroll
-                for (int j = 0; j < 2; ++j) scan_tile<D>(rows, 8 * (warp + 8 * j), nvalid, qa, qb, sl2, z[j]);
-                // LSE partials, branch-free (every row of the stage is owned by this CTA; invalid scores are -inf)
+            for (int j = 0; j < 2; ++j) scan_tile<D>(rows, 8 * (warp + 8 * j), nvalid, qa, qb, sl2, z[j]);
+            // LSE partials, branch-free (every row of the stage is owned by this CTA; invalid scores are -inf)
+#pragma unroll
+            for (int r = 0; r < 2; ++r) {
+                const float m4 = fmaxf(fmaxf(z[0][2 * r], z[0][2 * r + 1]), fmaxf(z[1][2 * r], z[1][2 * r + 1]));
+                const float mn = fmaxf(lm[r], m4);
+                ls[r] = ls[r] * ex2_approx(lm[r] - mn) + (ex2_approx(z[0][2 * r] - mn) + ex2_approx(z[0][2 * r + 1] - mn)) +
+                        (ex2_approx(z[1][2 * r] - mn) + ex2_approx(z[1][2 * r + 1] - mn));
+                lm[r] = mn;
+            }
+            // block maxima: tile j holds the stage's blocks 2 tt and 2 tt + 1 (tt = warp + 8 j) as cols 0..3 and
+            // 4..7, so lane tq's two cols belong to block 2 tt + (tq >> 1).  Shuffle-free, one atomicMax per
+            // lane for its own block; under the overlapping-window rule an odd lane's second col is the last
+            // kernel of that block and also goes to the block after it (in this CTA, or the next CTA's first).
+#pragma unroll
+            for (int j = 0; j < 2; ++j) {
+                const int tt = warp + 8 * j;
+                const int own = sc - b0 + 2 * tt + (tq >> 1);  // CTA-local block of this lane's cols
+                const bool own_ok = 2 * tt + (tq >> 1) < nblk;
 #pragma unroll
                 for (int r = 0; r < 2; ++r) {
-                    const float m4 = fmaxf(fmaxf(z[0][2 * r], z[0][2 * r + 1]), fmaxf(z[1][2 * r], z[1][2 * r + 1]));
-                    const float mn = fmaxf(lm[r], m4);
-                    ls[r] = ls[r] * ex2_approx(lm[r] - mn) + (ex2_approx(z[0][2 * r] - mn) + ex2_approx(z[0][2 * r + 1] - mn)) +
-                            (ex2_approx(z[1][2 * r] - mn) + ex2_approx(z[1][2 * r + 1] - mn));
-                    lm[r] = mn;
-                }
-                // block maxima: tile j holds the stage's blocks 2 tt and 2 tt + 1 (tt = warp + 8 j) as cols 0..3 and
-                // 4..7, so lane tq's two cols belong to block 2 tt + (tq >> 1).  Shuffle-free, one atomicMax per
-                // lane for its own block; under the overlapping-window rule an odd lane's second col is the last
-                // kernel of that block and also goes to the block after it (in this CTA, or the next CTA's first).
-#pragma unroll
-                for (int j = 0; j < 2; ++j) {
-                    const int tt = warp + 8 * j;
-                    const int own = sc - b0 + 2 * tt + (tq >> 1);  // CTA-local block of this lane's cols
-                    const bool own_ok = 2 * tt + (tq >> 1) < nblk;
-#pragma unroll
-                    for (int r = 0; r < 2; ++r) {
-                        const float v0 = z[j][2 * r], v1 = z[j][2 * r + 1];
-                        // contained windows: a block's kernels are cols 0..2 of its four
-                        const float vo = (!overlap && (tq & 1)) ? v0 : fmaxf(v0, v1);
-                        uint32_t* bm = bmax + (gq + 8 * r) * kFBmaxPitch;
-                        if (hv[r] && own_ok && vo != neg_inf()) atomicMax(&bm[own], float_key(vo));
-                        if (overlap && (tq & 1) && hv[r] && own_ok && v1 != neg_inf()) {
-                            if (own + 1 < nown) atomicMax(&bm[own + 1], float_key(v1));
-                            else halo_out[gq + 8 * r] = v1;  // the CTA's last kernel: next CTA's block 0
-                        }
+                    const float v0 = z[j][2 * r], v1 = z[j][2 * r + 1];
+                    // contained windows: a block's kernels are cols 0..2 of its four
+                    const float vo = (!overlap && (tq & 1)) ? v0 : fmaxf(v0, v1);
+                    uint32_t* bm = bmax + (gq + 8 * r) * kFBmaxPitch;
+                    if (hv[r] && own_ok && vo != neg_inf()) atomicMax(&bm[own], float_key(vo));
+                    if (overlap && (tq & 1) && hv[r] && own_ok && v1 != neg_inf()) {
+                        if (own + 1 < nown) atomicMax(&bm[own + 1], float_key(v1));
+                        else halo_out[gq + 8 * r] = v1;  // the CTA's last kernel: next CTA's block 0
                     }
                 }
-            }  // the stage's scores
+            }
             // stage consumed by every warp; a wait that ran out anywhere in the CTA stops the scan
             if (__syncthreads_or(!landed)) {
                 cta_failed = true;
@@ -415,9 +415,18 @@ decode_fused_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_con
 
     // ---------------- 3. selection (every CTA, identical result; the leader writes it out) ----------------
     int32_t* my_list = reinterpret_cast<int32_t*>(smem + L::kMyList);
+    // the first cache row of each of this CTA's blocks, found here by all threads (contiguous, packed or through
+    // the page table) so that the thread issuing the copies only reads it; an unmapped page starts a block
+    // before row 0, which the tensor map fills with zeros
+    int32_t* my_row = reinterpret_cast<int32_t*>(smem + L::kMyRows);
+    auto first_row = [&](int blk) {
+        const long zr = kv_block_row(kr, b, blk);
+        return zr >= 0 ? (int)zr : -kBlock;
+    };
     int count = nb - bw;
     if (dense) {
         if (rank == 0 && tid < 32 && idx_row) warp_write_dense_row(c, mc.kmax, idx_row, cnt + row);
+        for (int i = tid; rank + CL * i < count; i += kFThreads) my_row[i] = first_row(bw + rank + CL * i);
     } else if (bad) {
         count = 0;
         if (rank == 0 && tid == 0) cnt[row] = 0;
@@ -429,7 +438,11 @@ decode_fused_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_con
                                                         sel, list_all);
         count = min(total, mc.kmax);
         __syncthreads();
-        for (int i = tid; rank + CL * i < count; i += kFThreads) my_list[i] = list_all[rank + CL * i];
+        for (int i = tid; rank + CL * i < count; i += kFThreads) {
+            const int blk = list_all[rank + CL * i];
+            my_list[i] = blk;
+            my_row[i] = first_row(blk);
+        }
     }
     __syncthreads();
     // region A held generic-proxy data (scores, select scratch): order it before the TMA writes
@@ -442,11 +455,7 @@ decode_fused_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_con
     bool worked = false;
     {
         auto issue_block = [&](int i) {
-            const int blk = dense ? bw + rank + CL * i : my_list[i];
-            // first cache row of the block; a page the table does not map starts the copy a block before row 0,
-            // which the tensor map fills with zeros
-            const long zr = kv_block_row(kr, b, blk);
-            const int zrow = zr >= 0 ? (int)zr : -kBlock;
+            const int zrow = my_row[i];
             const int sidx = i % kFStages;
             unsigned char* stg = smem + (size_t)sidx * L::kStageBytes;
             n_issued += 1u << (8 * sidx);
