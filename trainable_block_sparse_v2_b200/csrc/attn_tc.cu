@@ -321,17 +321,22 @@ attn_tc_kernel(QueryRows qr, const __grid_constant__ CUtensorMap tm_q, const __g
             const int nv = sel ? min(kBlock, n - blk * kBlock) : 0;
             const uint32_t srow = lane_addr + kColS + kStepKeys * sb;
             const bool any_sel = __any_sync(0xffffffffu, sel);
-            // scaled scores in log2 units; keys this row does not attend to are -inf
+            // raw scores of this half's 64 keys (both TMEM loads in flight together); keys this row does not
+            // attend to are -inf.  The scale is applied later, inside the exponent's FFMA: with sl2 > 0 the
+            // maximum of the scaled scores is sl2 times the maximum of the raw ones
             float x[64];
             float mx = neg_inf();
             if (ok && any_sel) {
+                uint32_t sv[64];
+                tc::tmem_ld32(srow + 64 * half, *reinterpret_cast<uint32_t(*)[32]>(&sv[0]));
+                tc::tmem_ld32(srow + 64 * half + 32, *reinterpret_cast<uint32_t(*)[32]>(&sv[32]));
+                tc::tmem_wait_ld();
+                if (__all_sync(0xffffffffu, nv == kBlock)) {  // every row of the warp sees the whole block
 #pragma unroll
-                for (int h2 = 0; h2 < 2; ++h2) {
-                    uint32_t sv[32];
-                    tc::tmem_ld32(srow + 64 * half + 32 * h2, sv);
-                    tc::tmem_wait_ld();
+                    for (int j = 0; j < 64; ++j) x[j] = __uint_as_float(sv[j]);
+                } else {
 #pragma unroll
-                    for (int j = 0; j < 32; ++j) x[32 * h2 + j] = (32 * h2 + j) < nv ? __uint_as_float(sv[j]) * sl2 : neg_inf();
+                    for (int j = 0; j < 64; ++j) x[j] = j < nv ? __uint_as_float(sv[j]) : neg_inf();
                 }
                 float m8[8];
 #pragma unroll
@@ -342,6 +347,7 @@ attn_tc_kernel(QueryRows qr, const __grid_constant__ CUtensorMap tm_q, const __g
                     m8[i] = m;
                 }
                 mx = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])), fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
+                mx *= sl2;  // log2 units (-inf stays -inf)
             }
             // double-buffered by step parity: a half can be at most one step ahead of its partner here
             bars.xm[p & 1][half][r] = mx;
@@ -375,12 +381,14 @@ attn_tc_kernel(QueryRows qr, const __grid_constant__ CUtensorMap tm_q, const __g
                 // P = 2^(x - m_ref) for this half's 64 keys, bf16 pairs into S columns [32 half, 32 half + 32)
                 uint32_t w[32];
                 if (any_sel) {
+                    // 2^(sl2 s - m_ref) in one FFMA per key; a row that did not select the block (or has no
+                    // finite reference yet) gets 2^-inf = 0
                     const float mneg = (sel && m_ref != neg_inf()) ? -m_ref : neg_inf();
                     float ps[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
                     for (int j2 = 0; j2 < 32; ++j2) {
-                        const float p0 = ex2_approx(x[2 * j2] + mneg);
-                        const float p1 = ex2_approx(x[2 * j2 + 1] + mneg);
+                        const float p0 = ex2_approx(fmaf(x[2 * j2], sl2, mneg));
+                        const float p1 = ex2_approx(fmaf(x[2 * j2 + 1], sl2, mneg));
                         ps[j2 & 3] += p0 + p1;
                         w[j2] = pack_bf16(p0, p1);
                     }
