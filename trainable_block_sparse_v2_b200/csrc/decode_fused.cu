@@ -169,6 +169,9 @@ decode_fused_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_con
     __shared__ uint64_t full[kFStages];
     __shared__ uint64_t never;  // testing only: a barrier no thread or copy arrives on
     __shared__ uint32_t n_issued, n_done;  // thread 0: copies issued / seen complete per ring stage (8 bits each)
+    // a wait of some thread ran out in the ring iteration of that parity: written before the iteration's barrier,
+    // read after it; the next iteration writes the other slot, so no thread can change a slot still being read
+    __shared__ int ring_fail[2];
     __shared__ float part_m[16], part_s[16], lse2[16], halo_out[16];
     __shared__ __align__(16) float lse_slot[kFMaxCL][16][2];  // (max, sum) partials pushed by every CTA
 
@@ -190,6 +193,7 @@ decode_fused_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_con
         for (int s = 0; s < kFStages; ++s) tc::mbar_init(&full[s], 1);
         tc::mbar_init(&never, 1);
         n_issued = n_done = 0u;
+        ring_fail[0] = ring_fail[1] = 0;
         tc::fence_barrier_init();
         tc::prefetch_tensormap(&tmap_k);
         tc::prefetch_tensormap(&tmap_v);
@@ -272,6 +276,7 @@ decode_fused_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_con
             const bool landed = tlim ? tc::mbar_wait(&never, 0u, tlim)
                                      : tc::mbar_wait(&full[st], (phase_bits >> st) & 1u, 1u << 24);
             failed |= !landed;
+            if (!landed) ring_fail[i & 1] = 1;
             if (landed && tid == 0) n_done += 1u << (8 * st);
             phase_bits ^= 1u << st;
             // a stage that did not land in some thread is computed all the same: the CTA then stops below, and
@@ -316,7 +321,8 @@ decode_fused_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_con
                 }
             }
             // stage consumed by every warp; a wait that ran out anywhere in the CTA stops the scan
-            if (__syncthreads_or(!landed)) {
+            __syncthreads();
+            if (ring_fail[i & 1]) {
                 cta_failed = true;
                 break;
             }
@@ -477,6 +483,7 @@ decode_fused_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_con
             const int sidx = i % kFStages;
             const bool landed = tc::mbar_wait(&full[sidx], (phase_bits >> sidx) & 1u, 1u << 24);
             failed |= !landed;
+            if (!landed) ring_fail[(nch + i) & 1] = 1;
             if (landed && tid == 0) n_done += 1u << (8 * sidx);
             phase_bits ^= 1u << sidx;
             const int blk = dense ? bw + rank + CL * i : my_list[i];
@@ -552,7 +559,8 @@ decode_fused_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_con
                 worked = true;
             }
             // stage consumed by every warp; a wait that ran out anywhere in the CTA stops the walk
-            if (__syncthreads_or(!landed)) {
+            __syncthreads();
+            if (ring_fail[(nch + i) & 1]) {
                 cta_failed = true;
                 break;
             }
