@@ -168,7 +168,6 @@ decode_fused_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_con
     unsigned char* smem = tc::align_smem_1024(smem_raw);
     __shared__ uint64_t full[kFStages];
     __shared__ uint64_t never;  // testing only: a barrier no thread or copy arrives on
-    __shared__ uint32_t n_issued, n_done;  // thread 0: copies issued / seen complete per ring stage (8 bits each)
     // a wait of some thread ran out in the ring iteration of that parity: written before the iteration's barrier,
     // read after it; the next iteration writes the other slot, so no thread can change a slot still being read
     __shared__ int ring_fail[2];
@@ -192,7 +191,6 @@ decode_fused_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_con
     if (tid == 0) {
         for (int s = 0; s < kFStages; ++s) tc::mbar_init(&full[s], 1);
         tc::mbar_init(&never, 1);
-        n_issued = n_done = 0u;
         ring_fail[0] = ring_fail[1] = 0;
         tc::fence_barrier_init();
         tc::prefetch_tensormap(&tmap_k);
@@ -226,14 +224,17 @@ decode_fused_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_con
     // A wait that runs out (bounded polls) makes the whole CTA stop: it learns of it at the stage's barrier
     // (__syncthreads_or), issues no further copy, skips the rest of its loads and attention, still takes part
     // in every cluster barrier (with neutral partials), and before its shared memory is reused waits, bounded,
-    // for the copies still in flight.  Thread 0 counts the copies issued and seen complete per ring stage
-    // (n_issued, n_done); the k-th completion of a stage has parity k & 1.
+    // for the copies still in flight.  The ring holds one copy per stage: when the loop stops in iteration i of n,
+    // copies i .. min(n, i + kFStages) - 1 are in flight, each on stage j % kFStages, with the parity that stage
+    // expects next (phase_bits), except the failed stage i % kFStages, whose bit the loop has already flipped.
     bool cta_failed = false;
-    auto drain = [&]() {
+    int stop_at = 0;  // the ring iteration in which the CTA stopped
+    auto drain = [&](int i, int n) {
         if (tid == 0)
-            for (int s = 0; s < kFStages; ++s) {
-                const uint32_t is = (n_issued >> (8 * s)) & 255u, dn = (n_done >> (8 * s)) & 255u;
-                if (is != dn) (void)tc::mbar_wait(&full[s], dn & 1u, 1u << 20);
+            for (int j = i; j < n && j < i + kFStages; ++j) {
+                const int s = j % kFStages;
+                const uint32_t par = ((phase_bits >> s) & 1u) ^ (s == i % kFStages ? 1u : 0u);
+                (void)tc::mbar_wait(&full[s], par, 1u << 20);
             }
         __syncthreads();
     };
@@ -246,7 +247,6 @@ decode_fused_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_con
             const int sc = b0 + i * kFChunkBlocks, se = min(sc + kFChunkBlocks, b1);
             const int lo = sc * kKernelsPerBlock, hi = min(se * kKernelsPerBlock, nkv);
             uint64_t* bar = &full[i % kFStages];
-            n_issued += 1u << (8 * (i % kFStages));
             if (hi > lo) {
                 tc::mbar_arrive_expect_tx(bar, (uint32_t)(hi - lo) * D * 2);
                 tc::bulk_load(smem + (size_t)(i % kFStages) * L::kChunkBytes, kbase + (size_t)lo * D,
@@ -277,7 +277,6 @@ decode_fused_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_con
                                      : tc::mbar_wait(&full[st], (phase_bits >> st) & 1u, 1u << 24);
             failed |= !landed;
             if (!landed) ring_fail[i & 1] = 1;
-            if (landed && tid == 0) n_done += 1u << (8 * st);
             phase_bits ^= 1u << st;
             // a stage that did not land in some thread is computed all the same: the CTA then stops below, and
             // resets everything the stage wrote (block maxima, halo, LSE partials) before anything reads it
@@ -324,6 +323,7 @@ decode_fused_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_con
             __syncthreads();
             if (ring_fail[i & 1]) {
                 cta_failed = true;
+                stop_at = i;
                 break;
             }
             if (tid == 0 && i + kFStages < nch) issue_chunk(i + kFStages);
@@ -334,7 +334,7 @@ decode_fused_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_con
             ls[0] = ls[1] = 0.f;
             for (int k2 = tid; k2 < 16 * kFBmaxPitch; k2 += kFThreads) bmax[k2] = 0u;
             if (tid < 16) halo_out[tid] = neg_inf();
-            drain();
+            drain(stop_at, nch);
         }
         for (int r = 0; r < 2; ++r)
             if (lm[r] == kFloor) lm[r] = neg_inf();
@@ -464,7 +464,6 @@ decode_fused_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_con
             const int zrow = my_row[i];
             const int sidx = i % kFStages;
             unsigned char* stg = smem + (size_t)sidx * L::kStageBytes;
-            n_issued += 1u << (8 * sidx);
             tc::mbar_arrive_expect_tx(&full[sidx], (uint32_t)L::kStageBytes);
 #pragma unroll
             for (int dh = 0; dh < D / 64; ++dh) {
@@ -484,7 +483,6 @@ decode_fused_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_con
             const bool landed = tc::mbar_wait(&full[sidx], (phase_bits >> sidx) & 1u, 1u << 24);
             failed |= !landed;
             if (!landed) ring_fail[(nch + i) & 1] = 1;
-            if (landed && tid == 0) n_done += 1u << (8 * sidx);
             phase_bits ^= 1u << sidx;
             const int blk = dense ? bw + rank + CL * i : my_list[i];
             const int nvalid = min(kBlock, n - blk * kBlock);
@@ -562,11 +560,12 @@ decode_fused_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_con
             __syncthreads();
             if (ring_fail[(nch + i) & 1]) {
                 cta_failed = true;
+                stop_at = i;
                 break;
             }
             if (tid == 0 && i + kFStages < my_n) issue_block(i + kFStages);
         }
-        if (cta_failed) drain();
+        if (cta_failed) drain(stop_at, my_n);
     }
     finalize_rows<D>(st);
     // the eight warp states -> this CTA's partial: factors 2^(m_w - M) once per (warp, head), then sums
