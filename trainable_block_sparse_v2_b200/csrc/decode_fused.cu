@@ -221,26 +221,29 @@ decode_fused_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_con
     const float sl2 = mc.scale * kLog2e;
     uint32_t phase_bits = 0;  // parity of each ring stage
     bool failed = bad;
-    // A wait that runs out (bounded polls) makes the whole CTA stop: it learns of it at the stage's barrier
-    // (__syncthreads_or), issues no further copy, skips the rest of its loads and attention, still takes part
-    // in every cluster barrier (with neutral partials), and before its shared memory is reused waits, bounded,
-    // for the copies still in flight.  The ring holds one copy per stage: when the loop stops in iteration i of n,
-    // copies i .. min(n, i + kFStages) - 1 are in flight, each on stage j % kFStages, with the parity that stage
-    // expects next (phase_bits), except the failed stage i % kFStages, whose bit the loop has already flipped.
+    // A wait that runs out (bounded polls) makes the whole CTA stop.  The thread sets the ring flag of that
+    // iteration (ring_fail, by parity), which every thread reads after the stage barrier; the CTA then issues no
+    // further copy, skips the rest of its loads and attention, still takes part in every cluster barrier (with
+    // neutral partials), and before its shared memory is reused waits, bounded, for the copies still in flight.
+    // Thread 0 issues every copy, and issues the copy for ring position i + kFStages only after its own wait saw
+    // position i land (then that buffer is free, whatever other threads saw).  So when a loop stops at position
+    // i, the copies in flight are positions [first, end): first = i + 1 if thread 0 saw i land, else i, and
+    // end = min(n, i + kFStages + (saw ? 1 : 0)).  Position j uses stage j % kFStages, whose phase parity is
+    // (j / kFStages) & 1 in the scan, flipped in the attention walk by the scan's uses of that stage.
     bool cta_failed = false;
-    int stop_at = 0;  // the ring iteration in which the CTA stopped
-    auto drain = [&](int i, int n) {
+
+    // ---------------- 1. scan this CTA's blocks of the kernel cache ----------------
+    const int nch = (sparse && nown > 0) ? (nown + kFChunkBlocks - 1) / kFChunkBlocks : 0;
+    auto drain = [&](int i, int n, bool saw, bool attn) {
         if (tid == 0)
-            for (int j = i; j < n && j < i + kFStages; ++j) {
+            for (int j = saw ? i + 1 : i; j < n && j < i + kFStages + (saw ? 1 : 0); ++j) {
                 const int s = j % kFStages;
-                const uint32_t par = ((phase_bits >> s) & 1u) ^ (s == i % kFStages ? 1u : 0u);
+                uint32_t par = (j / kFStages) & 1u;
+                if (attn) par ^= ((nch - s + kFStages - 1) / kFStages) & 1u;
                 (void)tc::mbar_wait(&full[s], par, 1u << 20);
             }
         __syncthreads();
     };
-
-    // ---------------- 1. scan this CTA's blocks of the kernel cache ----------------
-    const int nch = (sparse && nown > 0) ? (nown + kFChunkBlocks - 1) / kFChunkBlocks : 0;
     if (nch > 0) {
         const __nv_bfloat16* kbase = kern + ((size_t)b * qr.Hkv + g) * nk_cap * D;
         auto issue_chunk = [&](int i) {
@@ -321,12 +324,12 @@ decode_fused_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_con
             }
             // stage consumed by every warp; a wait that ran out anywhere in the CTA stops the scan
             __syncthreads();
+            if (tid == 0 && landed && i + kFStages < nch) issue_chunk(i + kFStages);
             if (ring_fail[i & 1]) {
                 cta_failed = true;
-                stop_at = i;
+                drain(i, nch, landed, false);
                 break;
             }
-            if (tid == 0 && i + kFStages < nch) issue_chunk(i + kFStages);
         }
         if (cta_failed) {
             // this CTA contributes no kernel to the LSE and no block maximum to the scores
@@ -334,7 +337,6 @@ decode_fused_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_con
             ls[0] = ls[1] = 0.f;
             for (int k2 = tid; k2 < 16 * kFBmaxPitch; k2 += kFThreads) bmax[k2] = 0u;
             if (tid < 16) halo_out[tid] = neg_inf();
-            drain(stop_at, nch);
         }
         for (int r = 0; r < 2; ++r)
             if (lm[r] == kFloor) lm[r] = neg_inf();
@@ -558,14 +560,13 @@ decode_fused_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_con
             }
             // stage consumed by every warp; a wait that ran out anywhere in the CTA stops the walk
             __syncthreads();
+            if (tid == 0 && landed && i + kFStages < my_n) issue_block(i + kFStages);
             if (ring_fail[(nch + i) & 1]) {
                 cta_failed = true;
-                stop_at = i;
+                drain(i, my_n, landed, true);
                 break;
             }
-            if (tid == 0 && i + kFStages < my_n) issue_block(i + kFStages);
         }
-        if (cta_failed) drain(stop_at, my_n);
     }
     finalize_rows<D>(st);
     // the eight warp states -> this CTA's partial: factors 2^(m_w - M) once per (warp, head), then sums
