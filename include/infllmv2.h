@@ -103,11 +103,11 @@ int infllmv2_device_status(void);
  * Testing only (the pages have no counterpart): with polls > 0, the first kernel-cache wait of every CTA of
  * the fused decode step (infllmv2_sparse_decode_step and its paged form) polls a barrier that nothing
  * arrives on and gives up after `polls` polls, as a wait whose copy never lands would after its normal
- * limit.  That drives the bounded-wait error path without a fault: the step's CTAs stop loading, still
- * reach every cluster barrier, wait (bounded) for the copies in flight, and infllmv2_device_status then
+ * limit.  That drives the bounded-wait error path without a fault: the step's CTAs issue no further copy,
+ * wait (bounded) for the copies in flight, still reach every cluster barrier, and infllmv2_device_status then
  * returns INFLLMV2_ERR_TIMEOUT; the step's outputs are not the method's.  polls = 0 restores the normal
- * wait.  The limit is a device variable of the current device, written synchronously (it applies to calls
- * enqueued after this returns).  Returns INFLLMV2_OK or INFLLMV2_ERR_CUDA.
+ * wait.  The limit is process-wide and becomes a launch argument of every fused step launched after this
+ * returns (a CUDA graph captured before keeps the value it captured).  Returns INFLLMV2_OK.
  */
 int infllmv2_test_set_first_wait_limit(unsigned polls);
 

@@ -87,8 +87,21 @@ struct FLayout {
 };
 
 __device__ int g_fused_error = 0;
-// testing only: when nonzero, the first kernel-cache wait of every CTA gives up after this many polls
-__device__ unsigned g_fused_first_wait_limit = 0u;
+// testing only: when nonzero, the first kernel-cache wait of every CTA launched from now on gives up after this
+// many polls (passed to the kernel as an argument, so the normal path reads nothing extra)
+std::atomic<unsigned> g_first_wait_limit{0u};
+
+// Bounded wait on a ring barrier: false after `limit` polls, or early once another thread of the CTA has marked a
+// wait that ran out (checked every 256 polls, so a wait that succeeds within a few polls never reads it).
+IV2_DEV bool fused_wait(uint64_t* bar, uint32_t parity, uint32_t limit, volatile int* cta_err)
+{
+    for (uint32_t i = 0; i < limit; ++i) {
+        if (tc::mbar_try_wait(bar, parity)) return true;
+        if ((i & 255u) == 255u && *cta_err) return false;
+    }
+    *cta_err = 1;
+    return false;
+}
 
 // order-preserving key -> float (inverse of float_key)
 IV2_DEV float key_float(uint32_t k) { return __uint_as_float((k & 0x80000000u) ? (k & 0x7fffffffu) : ~k); }
@@ -161,16 +174,14 @@ __global__ void __launch_bounds__(kFThreads, 2)
 decode_fused_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_constant__ CUtensorMap tmap_v,
                     QueryRows qr, const __nv_bfloat16* __restrict__ kern, int nk_cap, MethodConsts mc, KvRows kr,
                     int32_t* __restrict__ idx, int32_t* __restrict__ cnt, __nv_bfloat16* __restrict__ out,
-                    float* __restrict__ lse_out)
+                    float* __restrict__ lse_out, unsigned first_wait_limit)
 {
     using L = FLayout<D>;
     extern __shared__ unsigned char smem_raw[];
     unsigned char* smem = tc::align_smem_1024(smem_raw);
     __shared__ uint64_t full[kFStages];
     __shared__ uint64_t never;  // testing only: a barrier no thread or copy arrives on
-    // a wait of some thread ran out in the ring iteration of that parity: written before the iteration's barrier,
-    // read after it; the next iteration writes the other slot, so no thread can change a slot still being read
-    __shared__ int ring_fail[2];
+    __shared__ int cta_err;  // set by a wait that ran out: the CTA's other waits then give up early
     __shared__ float part_m[16], part_s[16], lse2[16], halo_out[16];
     __shared__ __align__(16) float lse_slot[kFMaxCL][16][2];  // (max, sum) partials pushed by every CTA
 
@@ -191,7 +202,7 @@ decode_fused_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_con
     if (tid == 0) {
         for (int s = 0; s < kFStages; ++s) tc::mbar_init(&full[s], 1);
         tc::mbar_init(&never, 1);
-        ring_fail[0] = ring_fail[1] = 0;
+        cta_err = 0;
         tc::fence_barrier_init();
         tc::prefetch_tensormap(&tmap_k);
         tc::prefetch_tensormap(&tmap_v);
@@ -221,29 +232,18 @@ decode_fused_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_con
     const float sl2 = mc.scale * kLog2e;
     uint32_t phase_bits = 0;  // parity of each ring stage
     bool failed = bad;
-    // A wait that runs out (bounded polls) makes the whole CTA stop.  The thread sets the ring flag of that
-    // iteration (ring_fail, by parity), which every thread reads after the stage barrier; the CTA then issues no
-    // further copy, skips the rest of its loads and attention, still takes part in every cluster barrier (with
-    // neutral partials), and before its shared memory is reused waits, bounded, for the copies still in flight.
-    // Thread 0 issues every copy, and issues the copy for ring position i + kFStages only after its own wait saw
-    // position i land (then that buffer is free, whatever other threads saw).  So when a loop stops at position
-    // i, the copies in flight are positions [first, end): first = i + 1 if thread 0 saw i land, else i, and
-    // end = min(n, i + kFStages + (saw ? 1 : 0)).  Position j uses stage j % kFStages, whose phase parity is
-    // (j / kFStages) & 1 in the scan, flipped in the attention walk by the scan's uses of that stage.
-    bool cta_failed = false;
+    // A wait that runs out (bounded polls) marks the thread failed; the thread's later waits then give up after a
+    // few polls, and every wait also gives up once another thread has marked the CTA (cta_err, checked every 256
+    // polls, so a wait that succeeds on time never reads it).  Thread 0 issues every copy, and issues the copy
+    // for ring position i + kFStages only while none of its own waits has run out: its own wait for position i
+    // saw that buffer's copy land.  So after a failure the CTA issues no further copy; at its first wait that ran
+    // out, thread 0 waits (bounded) for the copies of that ring it issued and did not see land, before the
+    // stage barrier, so that no copy lands in region A once the loop is over.  The CTA still runs every loop (on
+    // whatever the buffers hold: no address depends on the data) and takes part in every cluster barrier.  The
+    // results of such a row are not the method's, and infllmv2_device_status reports the timeout.
 
     // ---------------- 1. scan this CTA's blocks of the kernel cache ----------------
     const int nch = (sparse && nown > 0) ? (nown + kFChunkBlocks - 1) / kFChunkBlocks : 0;
-    auto drain = [&](int i, int n, bool saw, bool attn) {
-        if (tid == 0)
-            for (int j = saw ? i + 1 : i; j < n && j < i + kFStages + (saw ? 1 : 0); ++j) {
-                const int s = j % kFStages;
-                uint32_t par = (j / kFStages) & 1u;
-                if (attn) par ^= ((nch - s + kFStages - 1) / kFStages) & 1u;
-                (void)tc::mbar_wait(&full[s], par, 1u << 20);
-            }
-        __syncthreads();
-    };
     if (nch > 0) {
         const __nv_bfloat16* kbase = kern + ((size_t)b * qr.Hkv + g) * nk_cap * D;
         auto issue_chunk = [&](int i) {
@@ -275,14 +275,16 @@ decode_fused_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_con
             const int st = i % kFStages;
             // testing only (a limit set from the host): the first wait polls a barrier nothing arrives on, so it
             // runs out after that many polls while the stage's copy is still in flight
-            const uint32_t tlim = i == 0 ? g_fused_first_wait_limit : 0u;
-            const bool landed = tlim ? tc::mbar_wait(&never, 0u, tlim)
-                                     : tc::mbar_wait(&full[st], (phase_bits >> st) & 1u, 1u << 24);
-            failed |= !landed;
-            if (!landed) ring_fail[i & 1] = 1;
+            const bool test_wait = i == 0 && first_wait_limit != 0u;
+            const bool landed = fused_wait(test_wait ? &never : &full[st], test_wait ? 0u : (phase_bits >> st) & 1u,
+                                           test_wait ? first_wait_limit : failed ? 64u : (1u << 24), &cta_err);
+            if (!landed) {
+                if (tid == 0 && !failed)  // in flight: positions i .. i + kFStages - 1, each on its own stage
+                    for (int j = i; j < nch && j < i + kFStages; ++j)
+                        (void)tc::mbar_wait(&full[j % kFStages], (j / kFStages) & 1u, 1u << 20);
+                failed = true;
+            }
             phase_bits ^= 1u << st;
-            // a stage that did not land in some thread is computed all the same: the CTA then stops below, and
-            // resets everything the stage wrote (block maxima, halo, LSE partials) before anything reads it
             const int sc = b0 + i * kFChunkBlocks, se = min(sc + kFChunkBlocks, b1);
             const int nblk = se - sc;
             const int nvalid = max(min(se * kKernelsPerBlock, nkv) - sc * kKernelsPerBlock, 0);  // rows staged
@@ -322,21 +324,8 @@ decode_fused_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_con
                     }
                 }
             }
-            // stage consumed by every warp; a wait that ran out anywhere in the CTA stops the scan
-            __syncthreads();
-            if (tid == 0 && landed && i + kFStages < nch) issue_chunk(i + kFStages);
-            if (ring_fail[i & 1]) {
-                cta_failed = true;
-                drain(i, nch, landed, false);
-                break;
-            }
-        }
-        if (cta_failed) {
-            // this CTA contributes no kernel to the LSE and no block maximum to the scores
-            lm[0] = lm[1] = kFloor;
-            ls[0] = ls[1] = 0.f;
-            for (int k2 = tid; k2 < 16 * kFBmaxPitch; k2 += kFThreads) bmax[k2] = 0u;
-            if (tid < 16) halo_out[tid] = neg_inf();
+            __syncthreads();  // stage consumed by every warp
+            if (tid == 0 && !failed && i + kFStages < nch) issue_chunk(i + kFStages);
         }
         for (int r = 0; r < 2; ++r)
             if (lm[r] == kFloor) lm[r] = neg_inf();
@@ -457,7 +446,7 @@ decode_fused_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_con
     tc::fence_proxy_async_smem();
 
     // ---------------- 4. attention over this CTA's entries rank, rank + CL, ... ----------------
-    const int my_n = (count > rank && !cta_failed) ? (count - rank + CL - 1) / CL : 0;
+    const int my_n = count > rank ? (count - rank + CL - 1) / CL : 0;
     WarpAttnState<D> st;
     st.init();
     bool worked = false;
@@ -473,7 +462,7 @@ decode_fused_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_con
                 tc::tma_load_3d(stg + L::kTileBytes + dh * L::kBoxBytes, &tmap_v, dh * 64, g, zrow, &full[sidx]);
             }
         };
-        if (tid == 0)
+        if (tid == 0 && !failed)
             for (int i = 0; i < kFStages && i < my_n; ++i) issue_block(i);
 
         uint32_t qf[D / 16][4];
@@ -482,9 +471,15 @@ decode_fused_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_con
         const int krow = key0 + (lane & 7);  // the key row this lane addresses in ldmatrix
         for (int i = 0; i < my_n; ++i) {
             const int sidx = i % kFStages;
-            const bool landed = tc::mbar_wait(&full[sidx], (phase_bits >> sidx) & 1u, 1u << 24);
-            failed |= !landed;
-            if (!landed) ring_fail[(nch + i) & 1] = 1;
+            if (!fused_wait(&full[sidx], (phase_bits >> sidx) & 1u, failed ? 64u : (1u << 24), &cta_err)) {
+                if (tid == 0 && !failed)  // as in the scan; a stage's parity also counts its uses by the scan
+                    for (int j = i; j < my_n && j < i + kFStages; ++j) {
+                        const int s = j % kFStages;
+                        (void)tc::mbar_wait(&full[s], ((nch - s + kFStages - 1) / kFStages + j / kFStages) & 1u,
+                                            1u << 20);
+                    }
+                failed = true;
+            }
             phase_bits ^= 1u << sidx;
             const int blk = dense ? bw + rank + CL * i : my_list[i];
             const int nvalid = min(kBlock, n - blk * kBlock);
@@ -492,8 +487,7 @@ decode_fused_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_con
             unsigned char* stg = smem + (size_t)sidx * L::kStageBytes;
             // a warp works when one of its 8 keys is in [nskip, nvalid) (nskip < nvalid for every walked block),
             // so every row's running max is finite after its first block
-            // a warp with a lane that did not see the stage land skips it (its bytes may not be there)
-            if (key0 < nvalid && key0 + 8 > nskip && !__any_sync(0xffffffffu, !landed)) {
+            if (key0 < nvalid && key0 + 8 > nskip) {
                 unsigned char* vt = stg + L::kTileBytes;
                 if (key0 + 8 > nvalid) {
                     // rows past the context may hold anything: zero them so that 0 * V stays 0
@@ -558,14 +552,8 @@ decode_fused_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_con
                 }
                 worked = true;
             }
-            // stage consumed by every warp; a wait that ran out anywhere in the CTA stops the walk
-            __syncthreads();
-            if (tid == 0 && landed && i + kFStages < my_n) issue_block(i + kFStages);
-            if (ring_fail[(nch + i) & 1]) {
-                cta_failed = true;
-                drain(i, my_n, landed, true);
-                break;
-            }
+            __syncthreads();  // stage consumed by every warp
+            if (tid == 0 && !failed && i + kFStages < my_n) issue_block(i + kFStages);
         }
     }
     finalize_rows<D>(st);
@@ -651,8 +639,7 @@ decode_fused_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_con
                 lse_out[(size_t)bt * qr.Hq + g * G + h] = Lsum > 0.f ? (M + __log2f(Lsum)) * kLn2 : neg_inf();
         }
     }
-    // a wait that ran out (or a context past the launch's tables): the results of this row are not the method's;
-    // the copies still in flight were waited for where the loop stopped
+    // a wait that ran out (or a context past the launch's tables): the results of this row are not the method's
     if (failed) atomicOr(&g_fused_error, 1);
 }
 
@@ -674,7 +661,7 @@ cudaError_t fused_launch(const CUtensorMap& tk, const CUtensorMap& tv, const Que
     const int rows = qr.B * qr.T * qr.Hkv;
     return launch_pdl_cluster(kfn, dim3(CL, rows), dim3(kFThreads), CL, FLayout<D>::kBytes, s, tk, tv, qr,
                               static_cast<const __nv_bfloat16*>(kern), nk_cap, mc, kr, idx, cnt,
-                              static_cast<__nv_bfloat16*>(out), lse);
+                              static_cast<__nv_bfloat16*>(out), lse, g_first_wait_limit.load(std::memory_order_relaxed));
 }
 
 // 16-CTA clusters of this kernel the device keeps resident at once (0 when 16 is not schedulable).  Cached per
@@ -764,7 +751,8 @@ cudaError_t launch_decode_fused(const QueryRows& qr, const void* kern, int nk_ca
 // testing only: the poll limit of the first kernel-cache wait of every CTA (0: the normal wait)
 int fused_set_first_wait_limit(unsigned polls)
 {
-    return cudaMemcpyToSymbol(g_fused_first_wait_limit, &polls, sizeof(unsigned)) == cudaSuccess ? 0 : -1;
+    g_first_wait_limit.store(polls, std::memory_order_relaxed);
+    return 0;
 }
 
 int fused_error_flag_read_and_clear()

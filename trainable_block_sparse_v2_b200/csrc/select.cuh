@@ -293,7 +293,8 @@ IV2_DEV int cta_count(int local_count, int* red /* >= 2 * NT/32 ints */, int par
     return total;
 }
 
-// exclusive prefix over threads (in thread order) of `v`; returns the prefix, *total gets the sum
+// exclusive prefix over threads (in thread order) of `v`; returns the prefix, *total gets the sum.  Threads may
+// still read scan_smem when others return: the caller synchronises before scan_smem is written again.
 template <int NT>
 IV2_DEV int cta_exclusive_scan(int v, int* scan_smem /* NT/32 + 1 ints */, int* total)
 {
@@ -313,7 +314,6 @@ IV2_DEV int cta_exclusive_scan(int v, int* scan_smem /* NT/32 + 1 ints */, int* 
         if (i < w) wbase += s;
         tot += s;
     }
-    __syncthreads();
     *total = tot;
     return wbase + incl - v;
 }
@@ -422,7 +422,7 @@ IV2_DEV int cta_select_topk(const float* S, int c, int init, int local, int topk
             const int y = __shfl_up_sync(0xffffffffu, incl, o);
             if (lane >= o) incl += y;
         }
-        __syncthreads();  // hist reads done before red is reused
+        // red's last readers (the candidate count above) all passed the barrier after the histogram
         if (lane == 31) sm.red[warp] = incl;
         __syncthreads();
         int wbase = 0;
