@@ -1081,7 +1081,7 @@ def run_ours(args):
                               "algorithmic_bytes": win_bytes, "achieved_gbs": win_bytes / t_win / 1e9,
                               "frac_of_" + peak_kind: win_bytes / t_win / 1e9 / peaks["hbm_gbs"],
                               "note": "the draft model's sliding-window decode attention (last 2048 keys), "
-                                      "4 sequences per call, split + merge kernels"},
+                                      "4 sequences per call, in the decode step's cluster kernel"},
         }
         del db
         torch.cuda.empty_cache()
@@ -1128,7 +1128,7 @@ def run_ours(args):
                 "ms_per_step": bt / args.prefill_steps * 1e3, "steps": args.prefill_steps,
                 "algorithmic_tflop_per_step": bflops / 1e12, "achieved_tflops": bach,
                 "tc_frac_of_" + peak_kind: bach / peaks["bf16_tflops"],
-                "kernels": "zero, prep, scan, fill (block lists), dq (mma.sync), dkdv (mma.sync, fp32 atomics)",
+                "kernels": "zero, prep, scan, fill (block lists), bwd_dq_tc and bwd_dkdv_tc (tcgen05/TMEM, TMA)",
             }
             line["gpu_launches"] += args.prefill_steps * 6
         del pb

@@ -197,8 +197,11 @@ def test_selection_explicit_q_ctx_and_early_blocks(oracle):
 # step 3: attention (fed the oracle's selection, so it is compared on identical block sets)
 # ---------------------------------------------------------------------------------------------------
 
-@pytest.mark.parametrize("G,d,dense_len", [(2, 64, 0), (16, 128, 700), (1, 128, 0), (8, 64, 2000)])
+@pytest.mark.parametrize("G,d,dense_len", [(2, 64, 0), (16, 128, 700), (1, 128, 0), (8, 64, 2000), (16, 64, 300),
+                                         (4, 128, 0), (8, 128, 500), (4, 64, 0)])
 def test_sparse_prefill_attention(oracle, G, d, dense_len):
+    """Every tile shape of the tensor-core kernel (128 / G tokens x G heads; G = 1 runs on mma.sync), a ragged
+    last tile, dense rows before dense_len."""
     T = 1500
     w = prefill_case(T, 2 * G, 2, d, topk=5, dense_len=dense_len, seed=500 + G, n_needles=2)
     nk_cap = oracle.num_kernels(T)

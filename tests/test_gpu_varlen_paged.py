@@ -39,7 +39,8 @@ def _bf16(rng, shape):
 VARLEN_CASES = {
     # name: (Hq, Hkv, d, [(T_b, L_b)], topk, dense_len)
     "tensor_core": (32, 2, 128, [(1500, 1500), (700, 2100), (1, 900), (0, 300), (64, 64), (20, 31)], 8, 300),
-    "mma_sync": (4, 2, 64, [(1100, 1100), (333, 1800), (1, 64)], 6, 0),
+    "tensor_core_d64": (4, 2, 64, [(1100, 1100), (333, 1800), (1, 64)], 6, 0),
+    "mma_sync": (2, 2, 128, [(1100, 1100), (333, 1800), (1, 64)], 6, 0),
     "scan_rows": (32, 2, 128, [(5, 4000), (16, 2500), (1, 70)], 8, 0),
 }
 
@@ -126,7 +127,7 @@ def _paged(rng, K, V, lens, num_pages, max_pages):
     return kp, vp, table
 
 
-@pytest.mark.parametrize("Hq,Hkv,d", [(32, 2, 128), (4, 2, 64)])
+@pytest.mark.parametrize("Hq,Hkv,d", [(32, 2, 128), (4, 2, 64), (2, 2, 128)])
 def test_paged_cache_equals_contiguous_cache(oracle, Hq, Hkv, d):
     rng = np.random.default_rng(2500 + d)
     lens = np.array([5000, 130, 9000], np.int32)  # context lengths after the append below

@@ -2,18 +2,19 @@
 //
 // Same definition as attn.cu (MiniCPM4 technical details, InfLLM v2 overview: only the selected context
 // blocks take part in attention; "Model architecture: InfLLM v2" item 2: the query heads of one GQA group
-// share the block set).  Specialised for 16 query heads per KV group and head_dim 128.
+// share the block set).  Instantiated for G = 2, 4, 8 or 16 query heads per KV group and head_dim d = 64 or
+// 128 (not G = 2 with d = 128, whose token bitmaps and rings exceed shared memory).
 //
-// One CTA owns a 128-row tile = 8 consecutive query tokens x the 16 heads of one KV group, and walks the
+// One CTA owns a 128-row tile = 128 / G consecutive query tokens x the G heads of one KV group, and walks the
 // ascending union of those tokens' selected blocks two blocks (128 keys) at a time (a token attends to a
 // block only when it selected it; other rows of the tile are masked for that block).  Per step:
-//   S[128 x 128] = Q[128 x 128] . K^T       tcgen05.mma kind::f16 with A (Q) in TMEM and B (K) K-major in
+//   S[128 x 128] = Q[128 x d] . K^T         tcgen05.mma kind::f16 with A (Q) in TMEM and B (K) K-major in
 //                                            128B-swizzled smem, fp32 accumulator in TMEM (two S buffers)
 //   P            = online softmax of S       four warps, one TMEM lane (= one query row) per thread; P goes
 //                                            back to TMEM as bf16 pairs over its own S buffer; the output
 //                                            is rescaled only when a row's max grows by more than 2^8 (exact:
 //                                            O and the row sum share the reference max)
-//   O[128 x 128] += P[128 x 128] . V         A (P) in TMEM, B (V) MN-major in smem, O in TMEM
+//   O[128 x d] += P[128 x 128] . V           A (P) in TMEM, B (V) MN-major in smem, O in TMEM
 // Keeping Q and P in TMEM leaves shared memory to the K/V stream, and 128-key steps halve the number of
 // MMA instructions and pipeline hand-offs per key.
 // Warp roles: warps 0 and 10 issue TMA loads (Q once and K per step; V per step) into 3-deep rings, one
@@ -34,28 +35,34 @@ __device__ int g_tc_error = 0;
 
 namespace {
 
-constexpr int kTok = 8;           // tokens per tile
-constexpr int kG = 16;            // heads per KV group
-constexpr int kD = 128;           // head dim
 constexpr int kThreads = 352;     // 11 warps
 constexpr int kMaxBlk = 4096;     // context blocks (256K keys)
 constexpr int kWords = kMaxBlk / 32;
 constexpr int kStepKeys = 128;       // two 64-key blocks per pipeline step
-constexpr uint32_t kTmemCols = 512;  // O [0,128), S0 [128,256), S1 [256,384), Q [384,448); P(step) overwrites
+constexpr uint32_t kTmemCols = 512;  // O [0,d), S0 [128,256), S1 [256,384), Q [384,384+d/2); P(step) overwrites
                                      // the first 64 columns of its own S buffer
 constexpr uint32_t kColS = 128, kColQ = 384;
+constexpr int kRing = 3;             // ring depth, in steps of 128 keys
 
 // dynamic shared memory layout (base aligned to 1024 B).  K and V stream through separate rings so each
 // can be refilled as soon as its own MMA has consumed it; Q is staged once in the last V slot (it is
-// copied into TMEM before that slot is first filled).
-constexpr int kRing = 3;                     // ring depth, in steps of 128 keys
-constexpr int kSlot = 32768;                 // one step of K or V: two d-halves x 128 key rows x 128 B
-constexpr int kKOff = 0;
-constexpr int kVOff = kKOff + kRing * kSlot;
-constexpr int kQOff = kVOff + (kRing - 1) * kSlot;  // 2 atoms x 128 rows x 128 B, aliases V slot kRing-1
-constexpr int kBitsOff = kVOff + kRing * kSlot;     // [kTok][kWords] uint32
-constexpr int kListOff = kBitsOff + kTok * kWords * 4;  // uint16 block ids
-constexpr int kSmemBytes = kListOff + kMaxBlk * 2 + 1024;  // + alignment slack
+// copied into TMEM before that slot is first filled).  A 128-B swizzle atom holds 64 dims of 128 rows.
+template <int G, int D>
+struct TcShape {
+    static constexpr int kTok = 128 / G;                     // tokens per tile
+    static constexpr int kAtoms = D / 64;                    // 64-dim atoms of a row
+    static constexpr int kSlot = kAtoms * 16384;             // one step of K or V: atoms x 128 key rows x 128 B
+    static constexpr int kKOff = 0;
+    static constexpr int kVOff = kKOff + kRing * kSlot;
+    static constexpr int kQOff = kVOff + (kRing - 1) * kSlot;  // Q: atoms x 128 rows x 128 B, in V slot kRing-1
+    static constexpr int kBitsOff = kVOff + kRing * kSlot;     // [kTok][kWords] uint32
+    static constexpr int kListOff = kBitsOff + kTok * kWords * 4;  // uint16 block ids
+    // + alignment slack; at least 116 KB, so that two CTAs never share an SM: each allocates all 512 TMEM columns
+    static constexpr int kNeed = kListOff + kMaxBlk * 2 + 1024;
+    static constexpr int kSmemBytes = kNeed > 116 * 1024 ? kNeed : 116 * 1024;
+    static_assert(G * kTok == 128 && (D == 64 || D == 128), "128-row tiles of whole tokens, d 64 or 128");
+    static_assert(kSmemBytes <= 227 * 1024 - 4096, "dynamic + static shared memory of one CTA");
+};
 
 struct Bars {
     uint64_t q_full, q_tmem;
@@ -80,12 +87,16 @@ __device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity, volatil
 
 }  // namespace
 
+template <int G, int D>
 __global__ void __launch_bounds__(kThreads, 1)
 attn_tc_kernel(QueryRows qr, const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                const __grid_constant__ CUtensorMap tm_v, KvRows kr, const int32_t* __restrict__ idx,
                const int32_t* __restrict__ cnt, MethodConsts mc, int dense_all, __nv_bfloat16* __restrict__ out,
                float* __restrict__ lse)
 {
+    using Sh = TcShape<G, D>;
+    constexpr int kTok = Sh::kTok, kSlot = Sh::kSlot, kKOff = Sh::kKOff, kVOff = Sh::kVOff, kQOff = Sh::kQOff;
+    constexpr int kBitsOff = Sh::kBitsOff, kListOff = Sh::kListOff;
     pdl_launch_dependents();
     pdl_wait();
     extern __shared__ unsigned char smem_raw[];
@@ -195,10 +206,11 @@ attn_tc_kernel(QueryRows qr, const __grid_constant__ CUtensorMap tm_q, const __g
         if (warp == 0 && lane == 0) {
             tc::prefetch_tensormap(&tm_q);
             tc::prefetch_tensormap(&tm_k);
-            tc::mbar_arrive_expect_tx(&bars.q_full, 2 * 128 * 128);
+            tc::mbar_arrive_expect_tx(&bars.q_full, kSlot);
             const int zq = (int)q_row(qr, b, t0);  // rows past this sequence are masked (or zero-filled)
-            tc::tma_load_3d(smem + kQOff, &tm_q, 0, g * kG, zq, &bars.q_full);
-            tc::tma_load_3d(smem + kQOff + 16384, &tm_q, 64, g * kG, zq, &bars.q_full);
+#pragma unroll
+            for (int a = 0; a < Sh::kAtoms; ++a)
+                tc::tma_load_3d(smem + kQOff + a * 16384, &tm_q, 64 * a, g * G, zq, &bars.q_full);
             for (int p = 0; p < NP; ++p) {
                 const int s = p % kRing, k = p / kRing;
                 if (k >= 1 && !wait_bar(&bars.k_empty[s], (k - 1) & 1, err)) break;
@@ -206,12 +218,13 @@ attn_tc_kernel(QueryRows qr, const __grid_constant__ CUtensorMap tm_q, const __g
                 tc::mbar_arrive_expect_tx(&bars.k_full[s], kSlot);
 #pragma unroll
                 for (int i = 0; i < 2; ++i) {
-                    // key rows [64 i, 64 i + 64) of the step, d halves in two atoms of 128 rows; an unmapped
+                    // key rows [64 i, 64 i + 64) of the step, each 64-dim atom of 128 rows apart; an unmapped
                     // page starts a block before row 0, which the tensor map fills with zeros
                     const long zr = kv_block_row(kr, b, (int)list[min(2 * p + i, U - 1)]);
                     const int z = zr >= 0 ? (int)zr : -kBlock;
-                    tc::tma_load_3d(st + i * 8192, &tm_k, 0, g, z, &bars.k_full[s]);
-                    tc::tma_load_3d(st + 16384 + i * 8192, &tm_k, 64, g, z, &bars.k_full[s]);
+#pragma unroll
+                    for (int a = 0; a < Sh::kAtoms; ++a)
+                        tc::tma_load_3d(st + a * 16384 + i * 8192, &tm_k, 64 * a, g, z, &bars.k_full[s]);
                 }
             }
         } else if (warp == 10 && lane == 0) {
@@ -227,8 +240,9 @@ attn_tc_kernel(QueryRows qr, const __grid_constant__ CUtensorMap tm_q, const __g
                 for (int i = 0; i < 2; ++i) {
                     const long zr = kv_block_row(kr, b, (int)list[min(2 * p + i, U - 1)]);
                     const int z = zr >= 0 ? (int)zr : -kBlock;
-                    tc::tma_load_3d(st + i * 8192, &tm_v, 0, g, z, &bars.v_full[s]);
-                    tc::tma_load_3d(st + 16384 + i * 8192, &tm_v, 64, g, z, &bars.v_full[s]);
+#pragma unroll
+                    for (int a = 0; a < Sh::kAtoms; ++a)
+                        tc::tma_load_3d(st + a * 16384 + i * 8192, &tm_v, 64 * a, g, z, &bars.v_full[s]);
                 }
             }
         }
@@ -237,7 +251,7 @@ attn_tc_kernel(QueryRows qr, const __grid_constant__ CUtensorMap tm_q, const __g
         if (lane == 0 && wait_bar(&bars.q_tmem, 0, err)) {
             tc::tc_fence_after();
             constexpr uint32_t idesc_s = tc::idesc_bf16(128, kStepKeys, false);
-            constexpr uint32_t idesc_o = tc::idesc_bf16(128, kD, true);
+            constexpr uint32_t idesc_o = tc::idesc_bf16(128, D, true);
             for (int p = 0; p <= NP; ++p) {
                 if (p < NP) {
                     // S(p) = Q . [K_a ; K_b]^T into S buffer p&1 (in-order after PV(p-2), which read P(p-2) there)
@@ -247,7 +261,7 @@ attn_tc_kernel(QueryRows qr, const __grid_constant__ CUtensorMap tm_q, const __g
                     const uint32_t d_s = tmem + kColS + kStepKeys * sb;
                     const uint32_t kbase = sK + s * kSlot;
 #pragma unroll
-                    for (int ks = 0; ks < kD / 16; ++ks) {
+                    for (int ks = 0; ks < D / 16; ++ks) {
                         const uint32_t koff = (ks >> 2) * 16384 + (ks & 3) * 32;
                         tc::mma_bf16_ts(d_s, tmem + kColQ + 8 * ks, tc::desc_kmajor_sw128(kbase + koff), idesc_s,
                                         ks > 0);
@@ -277,8 +291,8 @@ attn_tc_kernel(QueryRows qr, const __grid_constant__ CUtensorMap tm_q, const __g
         // (keys 0..63), half 1 its second (keys 64..127); they exchange row maxima and sums in shared memory
         // under a named barrier of their own, and every barrier is reached by both on every step
         const int q4 = warp & 3, half = (warp - 2) >> 2;
-        const int r = q4 * 32 + lane;  // row = token * 16 + head
-        const int tt = r >> 4, hh = r & 15;
+        const int r = q4 * 32 + lane;  // row = token * G + head
+        const int tt = r / G, hh = r % G;
         const int t = t0 + tt;
         const bool valid = t < Tb;
         const int n = valid ? query_ctx(qr, b, t) : 0;
@@ -288,9 +302,9 @@ attn_tc_kernel(QueryRows qr, const __grid_constant__ CUtensorMap tm_q, const __g
         float m_ref = neg_inf(), l = 0.f;
         bool ok = wait_bar(&bars.q_full, 0, err);
         if (half == 0) {
-            // this row of Q (swizzled smem from TMA) -> TMEM columns [kColQ, kColQ + 64) as bf16 pairs
+            // this row of Q (swizzled smem from TMA) -> TMEM columns [kColQ, kColQ + d / 2) as bf16 pairs
 #pragma unroll
-            for (int a = 0; a < 2; ++a) {
+            for (int a = 0; a < Sh::kAtoms; ++a) {
                 uint32_t w[32];
                 const unsigned char* qrow = smem + kQOff + a * 16384 + r * 128;
 #pragma unroll
@@ -364,13 +378,13 @@ attn_tc_kernel(QueryRows qr, const __grid_constant__ CUtensorMap tm_q, const __g
                 ok = __all_sync(0xffffffffu, ok);
                 if (ok) {
 #pragma unroll 1
-                    for (int c4 = 0; c4 < 2; ++c4) {
+                    for (int c4 = 0; c4 < D / 64; ++c4) {  // this half's d / 2 columns of O
                         uint32_t o[32];
-                        tc::tmem_ld32(lane_addr + 64 * half + 32 * c4, o);
+                        tc::tmem_ld32(lane_addr + (D / 2) * half + 32 * c4, o);
                         tc::tmem_wait_ld();
 #pragma unroll
                         for (int j = 0; j < 32; ++j) o[j] = __float_as_uint(__uint_as_float(o[j]) * alpha);
-                        tc::tmem_st32(lane_addr + 64 * half + 32 * c4, o);
+                        tc::tmem_st32(lane_addr + (D / 2) * half + 32 * c4, o);
                     }
                     tc::tmem_wait_st();
                 }
@@ -414,11 +428,11 @@ attn_tc_kernel(QueryRows qr, const __grid_constant__ CUtensorMap tm_q, const __g
         if (ok) {
             tc::tc_fence_after();
             const float inv = lt > 0.f ? 1.f / lt : 0.f;
-            __nv_bfloat16* orow = out + ((size_t)q_row(qr, b, valid ? t : 0) * qr.Hq + g * kG + hh) * kD + 64 * half;
+            __nv_bfloat16* orow = out + ((size_t)q_row(qr, b, valid ? t : 0) * qr.Hq + g * G + hh) * D + (D / 2) * half;
 #pragma unroll 1
-            for (int c4 = 0; c4 < 2; ++c4) {
+            for (int c4 = 0; c4 < D / 64; ++c4) {
                 uint32_t o[32];
-                tc::tmem_ld32(lane_addr + 64 * half + 32 * c4, o);
+                tc::tmem_ld32(lane_addr + (D / 2) * half + 32 * c4, o);
                 tc::tmem_wait_ld();
                 if (valid) {
 #pragma unroll
@@ -433,7 +447,7 @@ attn_tc_kernel(QueryRows qr, const __grid_constant__ CUtensorMap tm_q, const __g
                 }
             }
             if (valid && lse && half == 0)
-                lse[(size_t)q_row(qr, b, t) * qr.Hq + g * kG + hh] = lt > 0.f ? (m_ref + __log2f(lt)) * kLn2 : neg_inf();
+                lse[(size_t)q_row(qr, b, t) * qr.Hq + g * G + hh] = lt > 0.f ? (m_ref + __log2f(lt)) * kLn2 : neg_inf();
         }
     }
     tc::tc_fence_before();
@@ -445,9 +459,36 @@ attn_tc_kernel(QueryRows qr, const __grid_constant__ CUtensorMap tm_q, const __g
 }
 
 // ---------------------------------------------------------------- host
+namespace {
+
+template <int G, int D>
+cudaError_t attn_tc_launch(const QueryRows& qr, const void* k, const void* v, const KvRows& kr, const int32_t* idx,
+                           const int32_t* cnt, const MethodConsts& mc, bool dense_all, void* out, float* lse,
+                           cudaStream_t s)
+{
+    using Sh = TcShape<G, D>;
+    CUtensorMap tq, tk, tv;
+    const uint64_t row = (uint64_t)D * 2;
+    if (!make_tma_map_bf16(&tq, qr.q, D, qr.Hq, (uint64_t)qr.q_rows, row, row * qr.Hq, G, Sh::kTok) ||
+        !make_tma_map_bf16(&tk, k, D, qr.Hkv, (uint64_t)kr.rows, row, row * qr.Hkv, 1, kBlock) ||
+        !make_tma_map_bf16(&tv, v, D, qr.Hkv, (uint64_t)kr.rows, row, row * qr.Hkv, 1, kBlock))
+        return cudaErrorNotSupported;
+    auto kfn = attn_tc_kernel<G, D>;
+    cudaError_t e = ensure_smem(kfn, Sh::kSmemBytes);
+    if (e != cudaSuccess) return e;
+    const dim3 grid((qr.T + Sh::kTok - 1) / Sh::kTok, qr.B * qr.Hkv);
+    return launch_pdl(kfn, grid, dim3(kThreads), (size_t)Sh::kSmemBytes, s, qr, tq, tk, tv, kr, idx, cnt, mc,
+                      dense_all ? 1 : 0, static_cast<__nv_bfloat16*>(out), lse);
+}
+
+}  // namespace
+
 bool attn_tc_supported(const QueryRows& qr)
 {
-    return qr.D == kD && qr.Hq / qr.Hkv == kG && (qr.max_ctx - 1) / kBlock + 1 <= kMaxBlk;
+    if (qr.Hkv <= 0 || qr.Hq % qr.Hkv != 0 || (qr.max_ctx - 1) / kBlock + 1 > kMaxBlk) return false;
+    const int G = qr.Hq / qr.Hkv;
+    if (qr.D == 64) return G == 2 || G == 4 || G == 8 || G == 16;
+    return qr.D == 128 && (G == 4 || G == 8 || G == 16);
 }
 
 cudaError_t launch_attn_rows_tc(const QueryRows& qr, const void* k, const void* v, const KvRows& kr,
@@ -455,17 +496,17 @@ cudaError_t launch_attn_rows_tc(const QueryRows& qr, const void* k, const void* 
                                 void* out, float* lse, cudaStream_t s)
 {
     if (!attn_tc_supported(qr)) return cudaErrorNotSupported;
-    CUtensorMap tq, tk, tv;
-    const uint64_t row = (uint64_t)kD * 2;
-    if (!make_tma_map_bf16(&tq, qr.q, kD, qr.Hq, (uint64_t)qr.q_rows, row, row * qr.Hq, kG, kTok) ||
-        !make_tma_map_bf16(&tk, k, kD, qr.Hkv, (uint64_t)kr.rows, row, row * qr.Hkv, 1, kBlock) ||
-        !make_tma_map_bf16(&tv, v, kD, qr.Hkv, (uint64_t)kr.rows, row, row * qr.Hkv, 1, kBlock))
-        return cudaErrorNotSupported;
-    cudaError_t e = ensure_smem(attn_tc_kernel, kSmemBytes);
-    if (e != cudaSuccess) return e;
-    const dim3 grid((qr.T + kTok - 1) / kTok, qr.B * qr.Hkv);
-    return launch_pdl(attn_tc_kernel, grid, dim3(kThreads), (size_t)kSmemBytes, s, qr, tq, tk, tv, kr, idx, cnt,
-                      mc, dense_all ? 1 : 0, static_cast<__nv_bfloat16*>(out), lse);
+#define IV2_TC(GG, DD)                                                                                           \
+    if (qr.Hq / qr.Hkv == GG && qr.D == DD) return attn_tc_launch<GG, DD>(qr, k, v, kr, idx, cnt, mc, dense_all, out, lse, s)
+    IV2_TC(16, 128);
+    IV2_TC(8, 128);
+    IV2_TC(4, 128);
+    IV2_TC(16, 64);
+    IV2_TC(8, 64);
+    IV2_TC(4, 64);
+    IV2_TC(2, 64);
+#undef IV2_TC
+    return cudaErrorNotSupported;
 }
 
 int tc_error_flag_read_and_clear()
