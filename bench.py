@@ -39,14 +39,14 @@ UNIT = "tokens/s"
 PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 LENS_128K = (131072, 98304, 65536, 131072)
 HQ, HKV, D = 32, 2, 128
-# DRAM bytes (read + write) per call of the dominant C-ABI calls, each from one ncu capture of the kernels
-# as they stand (profiles/decode_128k_launches.md, profiles/decode_fused_128k.md); None where the kernel
-# changed after its capture
+# DRAM bytes (read + write) per call of the dominant C-ABI calls, each from one ncu capture of the kernel as
+# it stands (profiles/decode_fused_128k.md, profiles/prefill_32k.md); None where the kernels changed after
+# their capture (the two-call decode kernels took the paged / packed addressing since)
 NCU_TRAFFIC = {
-    "sparse_decode_step": 31_304_192,                   # decode_fused_kernel: 31.30 MB read, ~0 written
-    "sparse_attn_decode": 17_430_000 + 1_150_000,       # attn_split_kernel + attn_merge_kernel
-    "block_score_topk": 13_680_000 + 960_000,           # score_scan_kernel + score_select_kernel
-    "sparse_attn_prefill": 322_021_888 + 222_341_376,   # attn_tc_kernel (profiles/prefill_32k.md)
+    "sparse_decode_step": 31_308_928,                   # decode_fused_kernel: 31.31 MB read, ~2 KB written
+    "sparse_attn_decode": None,                         # attn_split_kernel + attn_merge_kernel
+    "block_score_topk": None,                           # score_scan_kernel + score_select_kernel
+    "sparse_attn_prefill": 321_901_824 + 226_391_808,   # attn_tc_kernel<16, 128>
 }
 KERNELS_PER_STEP = {"two_call": 5,  # kernel pool, score scan, select, split attention, merge
                     "fused": 2}     # kernel pool, fused decode step (scoring + top-k + attention)
