@@ -8,8 +8,8 @@ model lists, per warp role, the operations that role performs in program order:
     ("arrive", bar, n)          n arrivals
     ("arrive_tx", bar, n, tx)   n arrivals and tx expected transaction units
     ("tma", bar, tx, writes)    an asynchronous copy; on completion it writes `writes` and completes tx on bar
-    ("mma", reads, writes, lbl) a tensor-core op; ops run in issue order, each at some later time
-    ("commit", bar)             one arrival on bar once every earlier tensor-core op has run
+    ("mma", reads, writes, lbl) a tensor-core op; one role's ops run in its issue order, each at some later time
+    ("commit", bar)             one arrival on bar once every earlier tensor-core op of the same role has run
     ("read", buf, tag)          a synchronous read (ld.shared, tcgen05.ld + wait) expecting content `tag`
     ("write", buf, tag)         a synchronous write (st.shared, tcgen05.st + wait)
     ("nbar", id, n)             a named barrier over n roles
@@ -17,7 +17,8 @@ model lists, per warp role, the operations that role performs in program order:
 `reads` / `writes` are lists of (buffer, tag); a tag names the data a buffer must hold (for example
 ("S", 3): the scores of pipeline step 3).  The scheduler interleaves the roles and the asynchronous
 completions at random, with per-run skewed speeds so that some runs starve a role or the asynchronous units
-for long stretches.  It reports:
+for long stretches.  The tensor-core ops of different roles (two issuing threads) run in no fixed order
+relative to each other.  It reports:
 
 * a deadlock (no role can move and nothing asynchronous is pending);
 * a wait that returns on another phase than the one it means (the barrier ran two phases ahead of the waiter,
@@ -62,7 +63,7 @@ class PipelineModel:
         self.bufs: dict[str, _Buf] = {}
         self.roles: dict[str, dict] = {}
         self.copies: list = []
-        self.tc_queue: list = []
+        self.tc_queues: dict[str, list] = {}  # per issuing role, in its program order
         self.named: dict = {}
         self.released: dict = {}
 
@@ -113,9 +114,9 @@ class PipelineModel:
                 self._buf(name).pending_reads += 1
             for name, _ in op[2]:
                 self._buf(name).pending_writes += 1
-            self.tc_queue.append(op)
+            self.tc_queues.setdefault(who, []).append(op)
         elif kind == "commit":
-            self.tc_queue.append(op)
+            self.tc_queues.setdefault(who, []).append(op)
         elif kind == "read":
             buf = self._buf(op[1])
             if buf.pending_writes:
@@ -133,7 +134,8 @@ class PipelineModel:
 
     # ---- asynchronous completions ----
     def _complete_one(self):
-        kinds = (["copy"] if self.copies else []) + (["tc"] if self.tc_queue else [])
+        busy = [q for q in self.tc_queues.values() if q]
+        kinds = (["copy"] if self.copies else []) + (["tc"] if busy else [])
         kind = self.rng.choice(kinds)
         if len(kinds) == 2 and self.rng.random() < 0.5:
             kind = self.prefer
@@ -150,7 +152,7 @@ class PipelineModel:
                 raise ProtocolError(f"more transaction units completed on {bar} than expected")
             b.maybe_complete()
             return
-        op = self.tc_queue.pop(0)
+        op = self.rng.choice(busy).pop(0)
         if op[0] == "commit":
             b = self.bars[op[1]]
             b.arrived += 1
@@ -195,7 +197,7 @@ class PipelineModel:
                         runnable.append(name)
                 elif self._ready(name, op):
                     runnable.append(name)
-            pending = bool(self.copies or self.tc_queue)
+            pending = bool(self.copies) or any(self.tc_queues.values())
             if not runnable and not pending:
                 if all(st["done"] for st in self.roles.values()):
                     return

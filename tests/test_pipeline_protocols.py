@@ -15,28 +15,34 @@ RING = 3
 
 # --------------------------------------------------------------------------------------------------------------
 # attn_tc_kernel (csrc/attn_tc.cu): 128-row tile, U union blocks in NP = ceil(U / 2) steps of 128 keys.
-# Warp 0: Q once, then K per step (3-slot ring); warp 10: V per step (Q is staged in the last V slot);
-# warp 1: S(p) = Q K^T into S buffer p & 1, then O += P(p - 1) V; warps 2-9: softmax, two per TMEM lane
-# quarter, each on 64 keys, P written over the first 64 columns of its S buffer.
+# Warp 0: Q once (shared memory, the A operand of every S MMA), then K per step (3-slot ring); warp 10: V per
+# step (a VR-slot ring: 2 at d 128, 3 at d 64); warp 1: S(p) = Q K^T into S buffer p % 3, after PV(p - 3)
+# completed; warp 11: O += P(v) V; warps 2-9: softmax, two per TMEM lane quarter, each on 64 keys, P written
+# over the first 64 columns of its S buffer.  Warps 1 and 11 issue tensor-core ops independently: nothing
+# orders one's ops after the other's except the mbarriers.
 # --------------------------------------------------------------------------------------------------------------
-def attn_tc_model(m: PipelineModel, U: int, rescale_steps=(), parts: int = 2, mistake: str = ""):
+NS = 3
+
+
+def attn_tc_model(m: PipelineModel, U: int, rescale_steps=(), parts: int = 2, mistake: str = "", VR: int = 2):
     NP = (U + 1) // 2
     m.bar("q_full", 1)
-    m.bar("q_tmem", 128)
     for i in range(RING):
-        for n in ("k_full", "k_empty", "v_full", "v_empty"):
+        for n in ("k_full", "k_empty"):
             m.bar(f"{n}{i}", 1)
-    for i in range(2):
+    for i in range(VR):
+        for n in ("v_full", "v_empty"):
+            m.bar(f"{n}{i}", 1)
+    for i in range(NS):
         m.bar(f"s_full{i}", 1)
         m.bar(f"p_full{i}", 128 * parts)
         m.bar(f"o_done{i}", 1)
-    vq = f"V{RING - 1}"
     rd = 8 // parts  # 16-column chunks of S read per part
     wr = 4 // parts  # 16-column chunks of P written per part
 
     def k_producer():
         yield ("arrive_tx", "q_full", 1, 1)
-        yield ("tma", "q_full", 1, [(vq, "Q")])
+        yield ("tma", "q_full", 1, [("Q", "Q")])
         for p in range(NP):
             s, k = p % RING, p // RING
             if k >= 1 and mistake != "k producer skips k_empty":
@@ -46,49 +52,45 @@ def attn_tc_model(m: PipelineModel, U: int, rescale_steps=(), parts: int = 2, mi
 
     def v_producer():
         for p in range(NP):
-            s, k = p % RING, p // RING
-            if k >= 1:
+            s, k = p % VR, p // VR
+            if k >= 1 and mistake != "v producer skips v_empty":
                 yield ("wait", f"v_empty{s}", k - 1)
-            if p == RING - 1 and mistake != "V fill ignores q_tmem":
-                yield ("wait", "q_tmem", 0)
             yield ("arrive_tx", f"v_full{s}", 1, 1)
             yield ("tma", f"v_full{s}", 1, [(f"V{s}", ("V", p))])
 
-    def issuer():
-        yield ("wait", "q_tmem", 0)
-        for p in range(NP + 1):
-            if p < NP:
-                s, sb = p % RING, p & 1
-                yield ("wait", f"k_full{s}", p // RING)
-                yield ("mma", [(f"QT.q{q}", "Q") for q in range(4)] + [(f"K{s}", ("K", p))],
-                       [(f"S{sb}.q{q}.c{c}", ("S", p)) for q in range(4) for c in range(8)], f"S{p}")
-                yield ("commit", f"s_full{sb}")
-                yield ("commit", f"k_empty{s}")
-            if p >= 1:
-                v = p - 1
-                if mistake != "issuer skips p_full":
-                    yield ("wait", f"p_full{v & 1}", v >> 1)
-                yield ("wait", f"v_full{v % RING}", v // RING)
-                reads = [(f"S{v & 1}.q{q}.c{c}", ("P", v)) for q in range(4) for c in range(4)]
-                reads += [(f"V{v % RING}", ("V", v))]
-                if v > 0:
-                    reads += [(f"O.q{q}.h{k}", ("O", v - 1)) for q in range(4) for k in range(parts)]
-                yield ("mma", reads, [(f"O.q{q}.h{k}", ("O", v)) for q in range(4) for k in range(parts)], f"PV{v}")
-                yield ("commit", f"o_done{v & 1}")
-                yield ("commit", f"v_empty{v % RING}")
+    def s_issuer():
+        yield ("wait", "q_full", 0)
+        for p in range(NP):
+            s, sb = p % RING, p % NS
+            if p >= NS and mistake != "S issuer skips o_done":
+                yield ("wait", f"o_done{sb}", (p - NS) // NS)
+            yield ("wait", f"k_full{s}", p // RING)
+            yield ("mma", [("Q", "Q"), (f"K{s}", ("K", p))],
+                   [(f"S{sb}.q{q}.c{c}", ("S", p)) for q in range(4) for c in range(8)], f"S{p}")
+            yield ("commit", f"s_full{sb}")
+            yield ("commit", f"k_empty{s}")
+
+    def pv_issuer():
+        for v in range(NP):
+            pv, sv = v % NS, v % VR
+            if mistake != "PV issuer skips p_full":
+                yield ("wait", f"p_full{pv}", v // NS)
+            yield ("wait", f"v_full{sv}", v // VR)
+            reads = [(f"S{pv}.q{q}.c{c}", ("P", v)) for q in range(4) for c in range(4)]
+            reads += [(f"V{sv}", ("V", v))]
+            if v > 0:
+                reads += [(f"O.q{q}.h{k}", ("O", v - 1)) for q in range(4) for k in range(parts)]
+            yield ("mma", reads, [(f"O.q{q}.h{k}", ("O", v)) for q in range(4) for k in range(parts)], f"PV{v}")
+            yield ("commit", f"o_done{pv}")
+            yield ("commit", f"v_empty{sv}")
 
     def softmax(warp):
         q4, part = warp & 3, (warp - 2) >> 2
         nb = 1 + q4
-        yield ("wait", "q_full", 0)
-        if part == 0:
-            yield ("read", vq, "Q")
-            yield ("write", f"QT.q{q4}", "Q")
-            yield ("arrive", "q_tmem", 32)
         for p in range(NP):
-            sb = p & 1
+            sb = p % NS
             xm = p & 1 if mistake != "single-buffered max exchange" else 0
-            yield ("wait", f"s_full{sb}", p >> 1)
+            yield ("wait", f"s_full{sb}", p // NS)
             for c in range(rd * part, rd * part + rd):
                 yield ("read", f"S{sb}.q{q4}.c{c}", ("S", p))
             yield ("write", f"xm{xm}.q{q4}.h{part}", ("m", p))
@@ -98,7 +100,7 @@ def attn_tc_model(m: PipelineModel, U: int, rescale_steps=(), parts: int = 2, mi
                 yield ("read", f"xm{xm}.q{q4}.h{k}", ("m", p))
             if p in rescale_steps and p >= 1:  # every part of a quarter takes the same decision
                 if mistake != "rescale without o_done":
-                    yield ("wait", f"o_done{(p - 1) & 1}", (p - 1) >> 1)
+                    yield ("wait", f"o_done{(p - 1) % NS}", (p - 1) // NS)
                 yield ("read", f"O.q{q4}.h{part}", ("O", p - 1))
                 yield ("write", f"O.q{q4}.h{part}", ("O", p - 1))
             for c in range(wr * part, wr * part + wr):
@@ -111,12 +113,13 @@ def attn_tc_model(m: PipelineModel, U: int, rescale_steps=(), parts: int = 2, mi
         for k in range(parts):
             yield ("read", f"xm0.q{q4}.h{k}", ("l",))
         if NP > 0:
-            yield ("wait", f"o_done{(NP - 1) & 1}", (NP - 1) >> 1)
+            yield ("wait", f"o_done{(NP - 1) % NS}", (NP - 1) // NS)
             yield ("read", f"O.q{q4}.h{part}", ("O", NP - 1))
 
     m.role("k_producer", k_producer())
     m.role("v_producer", v_producer())
-    m.role("issuer", issuer())
+    m.role("s_issuer", s_issuer())
+    m.role("pv_issuer", pv_issuer())
     for w in range(2, 2 + 4 * parts):
         m.role(f"softmax{w}", softmax(w))
 
@@ -212,13 +215,14 @@ def _run(model, seeds, *args, **kw):
         m.run()
 
 
+@pytest.mark.parametrize("VR", [2, 3])
 @pytest.mark.parametrize("U", [1, 2, 3, 4, 5, 7, 12, 33])
-def test_attn_tc_protocol(U):
+def test_attn_tc_protocol(U, VR):
     for seed in range(40):
         NP = (U + 1) // 2
         rescale = {p for p in range(NP) if (seed * 7 + p) % 3 == 0}
         m = PipelineModel(seed)
-        attn_tc_model(m, U, rescale)
+        attn_tc_model(m, U, rescale, VR=VR)
         m.run()
 
 
@@ -236,7 +240,8 @@ def _caught(model, seeds, *args, **kw):
 
 
 @pytest.mark.parametrize("mistake,U", [
-    ("k producer skips k_empty", 9), ("V fill ignores q_tmem", 9), ("issuer skips p_full", 5),
+    ("k producer skips k_empty", 9), ("v producer skips v_empty", 9), ("S issuer skips o_done", 9),
+    ("PV issuer skips p_full", 5),
     ("single-buffered max exchange", 5), ("no barrier before P", 3), ("rescale without o_done", 5),
     ("no barrier before the sums", 5),
 ])

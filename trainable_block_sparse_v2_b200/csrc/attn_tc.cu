@@ -8,18 +8,20 @@
 // One CTA owns a 128-row tile = 128 / G consecutive query tokens x the G heads of one KV group, and walks the
 // ascending union of those tokens' selected blocks two blocks (128 keys) at a time (a token attends to a
 // block only when it selected it; other rows of the tile are masked for that block).  Per step:
-//   S[128 x 128] = Q[128 x d] . K^T         tcgen05.mma kind::f16 with A (Q) in TMEM and B (K) K-major in
-//                                            128B-swizzled smem, fp32 accumulator in TMEM (two S buffers)
+//   S[128 x 128] = Q[128 x d] . K^T         tcgen05.mma kind::f16, A (Q) and B (K) K-major in 128B-swizzled
+//                                            smem, fp32 accumulator in TMEM (three S buffers)
 //   P            = online softmax of S       four warps, one TMEM lane (= one query row) per thread; P goes
 //                                            back to TMEM as bf16 pairs over its own S buffer; the output
 //                                            is rescaled only when a row's max grows by more than 2^8 (exact:
 //                                            O and the row sum share the reference max)
 //   O[128 x d] += P[128 x 128] . V           A (P) in TMEM, B (V) MN-major in smem, O in TMEM
-// Keeping Q and P in TMEM leaves shared memory to the K/V stream, and 128-key steps halve the number of
-// MMA instructions and pipeline hand-offs per key.
-// Warp roles: warps 0 and 10 issue TMA loads (Q once and K per step; V per step) into 3-deep rings, one
-// lane each, warp 1 (one thread) issues the MMAs, warps 2-9 run the softmax and the epilogue, two warps per
-// TMEM lane quarter, each on one of the step's two blocks.
+// The step chain P(p) -> PV(p) -> S(p + 3) -> P(p + 3) spans three steps: with three S buffers the softmax
+// of step p overlaps the MMAs of steps p + 1 and p + 2, and 128-key steps halve the number of MMA
+// instructions and pipeline hand-offs per key.
+// Warp roles: warps 0 and 10 issue TMA loads (Q once and K per step; V per step) into rings, one lane each,
+// warp 1 (one thread) issues the S MMAs and warp 11 (one thread) the PV MMAs, so that a late P does not hold
+// back the next scores; warps 2-9 run the softmax and the epilogue, two warps per TMEM lane quarter, each on
+// one of the step's two blocks.
 // Producer/consumer hand-offs use mbarriers; MMA completion is signalled with tcgen05.commit.  Every wait
 // is bounded: after the limit the CTA records an error (g_tc_error), skips the rest of its work, frees its
 // TMEM and exits.
@@ -35,27 +37,30 @@ __device__ int g_tc_error = 0;
 
 namespace {
 
-constexpr int kThreads = 352;     // 11 warps
+constexpr int kThreads = 384;     // 12 warps
 constexpr int kMaxBlk = 4096;     // context blocks (256K keys)
 constexpr int kWords = kMaxBlk / 32;
 constexpr int kStepKeys = 128;       // two 64-key blocks per pipeline step
-constexpr uint32_t kTmemCols = 512;  // O [0,d), S0 [128,256), S1 [256,384), Q [384,384+d/2); P(step) overwrites
+constexpr uint32_t kTmemCols = 512;  // O [0,d), S buffers [128,256), [256,384), [384,512); P(step) overwrites
                                      // the first 64 columns of its own S buffer
-constexpr uint32_t kColS = 128, kColQ = 384;
-constexpr int kRing = 3;             // ring depth, in steps of 128 keys
+constexpr uint32_t kColS = 128;
+constexpr int kNS = 3;               // S buffers: the scores of step p + 2 are computed while P(p) is formed
+constexpr int kRing = 3;             // K ring depth, in steps of 128 keys
 
 // dynamic shared memory layout (base aligned to 1024 B).  K and V stream through separate rings so each
-// can be refilled as soon as its own MMA has consumed it; Q is staged once in the last V slot (it is
-// copied into TMEM before that slot is first filled).  A 128-B swizzle atom holds 64 dims of 128 rows.
+// can be refilled as soon as its own MMA has consumed it; Q stays in shared memory as the A operand of every
+// S MMA.  A 128-B swizzle atom holds 64 dims of 128 rows.  V is needed only once P of its step is formed, two
+// steps after its slot was freed, so at d 128 a 2-deep V ring leaves room for Q.
 template <int G, int D>
 struct TcShape {
     static constexpr int kTok = 128 / G;                     // tokens per tile
     static constexpr int kAtoms = D / 64;                    // 64-dim atoms of a row
     static constexpr int kSlot = kAtoms * 16384;             // one step of K or V: atoms x 128 key rows x 128 B
+    static constexpr int kVRing = D == 128 ? 2 : 3;          // V ring depth
     static constexpr int kKOff = 0;
     static constexpr int kVOff = kKOff + kRing * kSlot;
-    static constexpr int kQOff = kVOff + (kRing - 1) * kSlot;  // Q: atoms x 128 rows x 128 B, in V slot kRing-1
-    static constexpr int kBitsOff = kVOff + kRing * kSlot;     // [kTok][kWords] uint32
+    static constexpr int kQOff = kVOff + kVRing * kSlot;       // Q: atoms x 128 rows x 128 B
+    static constexpr int kBitsOff = kQOff + kSlot;             // [kTok][kWords] uint32
     static constexpr int kListOff = kBitsOff + kTok * kWords * 4;  // uint16 block ids
     // + alignment slack; at least 116 KB, so that two CTAs never share an SM: each allocates all 512 TMEM columns
     static constexpr int kNeed = kListOff + kMaxBlk * 2 + 1024;
@@ -65,9 +70,9 @@ struct TcShape {
 };
 
 struct Bars {
-    uint64_t q_full, q_tmem;
+    uint64_t q_full;
     uint64_t k_full[kRing], k_empty[kRing], v_full[kRing], v_empty[kRing];
-    uint64_t s_full[2], p_full[2], o_done[2];
+    uint64_t s_full[kNS], p_full[kNS], o_done[kNS];
     uint32_t tmem_base;
     int n_union;
     int err;
@@ -96,6 +101,7 @@ attn_tc_kernel(QueryRows qr, const __grid_constant__ CUtensorMap tm_q, const __g
 {
     using Sh = TcShape<G, D>;
     constexpr int kTok = Sh::kTok, kSlot = Sh::kSlot, kKOff = Sh::kKOff, kVOff = Sh::kVOff, kQOff = Sh::kQOff;
+    constexpr int kVRing = Sh::kVRing;
     constexpr int kBitsOff = Sh::kBitsOff, kListOff = Sh::kListOff;
     pdl_launch_dependents();
     pdl_wait();
@@ -171,14 +177,13 @@ attn_tc_kernel(QueryRows qr, const __grid_constant__ CUtensorMap tm_q, const __g
     }
     if (threadIdx.x == 0) {
         tc::mbar_init(&bars.q_full, 1);
-        tc::mbar_init(&bars.q_tmem, 128);
         for (int i = 0; i < kRing; ++i) {
             tc::mbar_init(&bars.k_full[i], 1);
             tc::mbar_init(&bars.k_empty[i], 1);
             tc::mbar_init(&bars.v_full[i], 1);
             tc::mbar_init(&bars.v_empty[i], 1);
         }
-        for (int i = 0; i < 2; ++i) {
+        for (int i = 0; i < kNS; ++i) {
             tc::mbar_init(&bars.s_full[i], 1);
             tc::mbar_init(&bars.p_full[i], 256);
             tc::mbar_init(&bars.o_done[i], 1);
@@ -230,10 +235,8 @@ attn_tc_kernel(QueryRows qr, const __grid_constant__ CUtensorMap tm_q, const __g
         } else if (warp == 10 && lane == 0) {
             tc::prefetch_tensormap(&tm_v);
             for (int p = 0; p < NP; ++p) {
-                const int s = p % kRing, k = p / kRing;
+                const int s = p % kVRing, k = p / kVRing;
                 if (k >= 1 && !wait_bar(&bars.v_empty[s], (k - 1) & 1, err)) break;
-                // the last slot holds Q until the softmax warps have copied it into TMEM
-                if (p == kRing - 1 && !wait_bar(&bars.q_tmem, 0, err)) break;
                 unsigned char* st = smem + kVOff + s * kSlot;
                 tc::mbar_arrive_expect_tx(&bars.v_full[s], kSlot);
 #pragma unroll
@@ -247,42 +250,47 @@ attn_tc_kernel(QueryRows qr, const __grid_constant__ CUtensorMap tm_q, const __g
             }
         }
     } else if (warp == 1) {
-        // ---------------- MMA issuer ----------------
-        if (lane == 0 && wait_bar(&bars.q_tmem, 0, err)) {
+        // ---------------- S issuer ----------------
+        // S(p) overwrites the buffer of P(p - 3): it waits until PV(p - 3), issued by warp 11, has completed
+        if (lane == 0 && wait_bar(&bars.q_full, 0, err)) {
             tc::tc_fence_after();
             constexpr uint32_t idesc_s = tc::idesc_bf16(128, kStepKeys, false);
+            const uint32_t sQ = tc::smem_u32(smem + kQOff);
+            for (int p = 0; p < NP; ++p) {
+                // S(p) = Q . [K_a ; K_b]^T into S buffer p % kNS, both operands K-major in shared memory
+                const int s = p % kRing, sb = p % kNS;
+                if (p >= kNS && !wait_bar(&bars.o_done[sb], ((p - kNS) / kNS) & 1, err)) break;
+                if (!wait_bar(&bars.k_full[s], (p / kRing) & 1, err)) break;
+                tc::tc_fence_after();
+                const uint32_t d_s = tmem + kColS + kStepKeys * sb;
+                const uint32_t kbase = sK + s * kSlot;
+#pragma unroll
+                for (int ks = 0; ks < D / 16; ++ks) {
+                    const uint32_t koff = (ks >> 2) * 16384 + (ks & 3) * 32;
+                    tc::mma_bf16_ss(d_s, tc::desc_kmajor_sw128(sQ + koff), tc::desc_kmajor_sw128(kbase + koff),
+                                    idesc_s, ks > 0);
+                }
+                tc::mma_commit(&bars.s_full[sb]);
+                tc::mma_commit(&bars.k_empty[s]);
+            }
+        }
+    } else if (warp == 11) {
+        // ---------------- PV issuer ----------------
+        if (lane == 0) {
             constexpr uint32_t idesc_o = tc::idesc_bf16(128, D, true);
-            for (int p = 0; p <= NP; ++p) {
-                if (p < NP) {
-                    // S(p) = Q . [K_a ; K_b]^T into S buffer p&1 (in-order after PV(p-2), which read P(p-2) there)
-                    const int s = p % kRing, sb = p & 1;
-                    if (!wait_bar(&bars.k_full[s], (p / kRing) & 1, err)) break;
-                    tc::tc_fence_after();
-                    const uint32_t d_s = tmem + kColS + kStepKeys * sb;
-                    const uint32_t kbase = sK + s * kSlot;
+            for (int v = 0; v < NP; ++v) {
+                // O += P(v) . [V_a ; V_b], P(v) in the first 64 columns of S buffer v % kNS
+                const int pv = v % kNS, sv = v % kVRing;
+                if (!wait_bar(&bars.p_full[pv], (v / kNS) & 1, err)) break;
+                if (!wait_bar(&bars.v_full[sv], (v / kVRing) & 1, err)) break;
+                tc::tc_fence_after();
+                const uint32_t vbase = sV + sv * kSlot;
 #pragma unroll
-                    for (int ks = 0; ks < D / 16; ++ks) {
-                        const uint32_t koff = (ks >> 2) * 16384 + (ks & 3) * 32;
-                        tc::mma_bf16_ts(d_s, tmem + kColQ + 8 * ks, tc::desc_kmajor_sw128(kbase + koff), idesc_s,
-                                        ks > 0);
-                    }
-                    tc::mma_commit(&bars.s_full[sb]);
-                    tc::mma_commit(&bars.k_empty[s]);
-                }
-                if (p >= 1) {
-                    // O += P(v) . [V_a ; V_b], P(v) in the first 64 columns of S buffer v&1
-                    const int v = p - 1, pv = v & 1;
-                    if (!wait_bar(&bars.p_full[pv], (v >> 1) & 1, err)) break;
-                    if (!wait_bar(&bars.v_full[v % kRing], (v / kRing) & 1, err)) break;
-                    tc::tc_fence_after();
-                    const uint32_t vbase = sV + (v % kRing) * kSlot;
-#pragma unroll
-                    for (int ks = 0; ks < kStepKeys / 16; ++ks)
-                        tc::mma_bf16_ts(tmem, tmem + kColS + kStepKeys * pv + 8 * ks,
-                                        tc::desc_mnmajor_sw128(vbase + ks * 2048, 16384), idesc_o, (v > 0 || ks > 0));
-                    tc::mma_commit(&bars.o_done[pv]);
-                    tc::mma_commit(&bars.v_empty[v % kRing]);
-                }
+                for (int ks = 0; ks < kStepKeys / 16; ++ks)
+                    tc::mma_bf16_ts(tmem, tmem + kColS + kStepKeys * pv + 8 * ks,
+                                    tc::desc_mnmajor_sw128(vbase + ks * 2048, 16384), idesc_o, (v > 0 || ks > 0));
+                tc::mma_commit(&bars.o_done[pv]);
+                tc::mma_commit(&bars.v_empty[sv]);
             }
         }
     } else if (warp >= 2 && warp <= 9) {
@@ -300,31 +308,10 @@ attn_tc_kernel(QueryRows qr, const __grid_constant__ CUtensorMap tm_q, const __g
         const uint32_t pair_bar = 1 + q4;
         const float sl2 = mc.scale * kLog2e;
         float m_ref = neg_inf(), l = 0.f;
-        bool ok = wait_bar(&bars.q_full, 0, err);
-        if (half == 0) {
-            // this row of Q (swizzled smem from TMA) -> TMEM columns [kColQ, kColQ + d / 2) as bf16 pairs
-#pragma unroll
-            for (int a = 0; a < Sh::kAtoms; ++a) {
-                uint32_t w[32];
-                const unsigned char* qrow = smem + kQOff + a * 16384 + r * 128;
-#pragma unroll
-                for (int c = 0; c < 8; ++c) {
-                    const uint4 v4 = *reinterpret_cast<const uint4*>(qrow + ((c ^ (r & 7)) << 4));
-                    w[4 * c] = v4.x;
-                    w[4 * c + 1] = v4.y;
-                    w[4 * c + 2] = v4.z;
-                    w[4 * c + 3] = v4.w;
-                }
-                tc::tmem_st32(lane_addr + kColQ + 32 * a, w);
-            }
-            tc::tmem_wait_st();
-            tc::tc_fence_before();
-            tc::mbar_arrive(&bars.q_tmem);
-        }
-        ok = __all_sync(0xffffffffu, ok);
+        bool ok = true;
         for (int p = 0; p < NP; ++p) {
-            const int sb = p & 1;
-            if (ok) ok = wait_bar(&bars.s_full[sb], (p >> 1) & 1, err);
+            const int sb = p % kNS;
+            if (ok) ok = wait_bar(&bars.s_full[sb], (p / kNS) & 1, err);
             ok = __all_sync(0xffffffffu, ok);
             if (ok) tc::tc_fence_after();
             // this half's block of the step, whether this row's token selected it, and its keys in it
@@ -374,7 +361,7 @@ attn_tc_kernel(QueryRows qr, const __grid_constant__ CUtensorMap tm_q, const __g
             const float alpha = (rescale && m_ref != neg_inf()) ? exp2_fast(m_ref - new_ref) : 1.f;
             if (ok && __any_sync(0xffffffffu, alpha != 1.f)) {
                 // every PV so far must have landed before this half of O is rewritten
-                if (p >= 1) ok = wait_bar(&bars.o_done[(p - 1) & 1], ((p - 1) >> 1) & 1, err) && ok;
+                if (p >= 1) ok = wait_bar(&bars.o_done[(p - 1) % kNS], ((p - 1) / kNS) & 1, err) && ok;
                 ok = __all_sync(0xffffffffu, ok);
                 if (ok) {
 #pragma unroll 1
@@ -423,7 +410,7 @@ attn_tc_kernel(QueryRows qr, const __grid_constant__ CUtensorMap tm_q, const __g
         tc::named_bar_sync(pair_bar, 64);
         const float lt = l + bars.xm[0][half ^ 1][r];
         ok = __all_sync(0xffffffffu, ok);
-        if (ok && NP > 0) ok = wait_bar(&bars.o_done[(NP - 1) & 1], ((NP - 1) >> 1) & 1, err);
+        if (ok && NP > 0) ok = wait_bar(&bars.o_done[(NP - 1) % kNS], ((NP - 1) / kNS) & 1, err);
         ok = __all_sync(0xffffffffu, ok);
         if (ok) {
             tc::tc_fence_after();
