@@ -79,6 +79,37 @@ struct Bars {
     float xm[2][2][128];  // [step parity][half][row]: the two softmax halves' partial maxima, then sums
 };
 
+// sm_100 paired fp32 arithmetic (two lanes of a 64-bit register pair per instruction, each rounded as the
+// scalar op) and the three-input maximum
+__device__ __forceinline__ unsigned long long f2(float lo, float hi)
+{
+    unsigned long long r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+    return r;
+}
+__device__ __forceinline__ void f2_split(unsigned long long v, float& lo, float& hi)
+{
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ unsigned long long fma2(unsigned long long a, unsigned long long b, unsigned long long c)
+{
+    unsigned long long d;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+    return d;
+}
+__device__ __forceinline__ unsigned long long add2(unsigned long long a, unsigned long long b)
+{
+    unsigned long long d;
+    asm("add.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+__device__ __forceinline__ float max3(float a, float b, float c)
+{
+    float d;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+    return d;
+}
+
 __device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity, volatile int* err)
 {
     for (uint32_t i = 0; i < (1u << 22); ++i) {
@@ -339,15 +370,16 @@ attn_tc_kernel(QueryRows qr, const __grid_constant__ CUtensorMap tm_q, const __g
 #pragma unroll
                     for (int j = 0; j < 64; ++j) x[j] = j < nv ? __uint_as_float(sv[j]) : neg_inf();
                 }
+                // the maximum of 64 in 32 three-input steps: 64 -> 22 -> 8 -> 3 -> 1
+                float m22[22];
+#pragma unroll
+                for (int i = 0; i < 21; ++i) m22[i] = max3(x[i], x[i + 21], x[i + 42]);
+                m22[21] = x[63];
                 float m8[8];
 #pragma unroll
-                for (int i = 0; i < 8; ++i) {
-                    float m = x[i];
-#pragma unroll
-                    for (int j = 1; j < 8; ++j) m = fmaxf(m, x[i + 8 * j]);
-                    m8[i] = m;
-                }
-                mx = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])), fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
+                for (int i = 0; i < 7; ++i) m8[i] = max3(m22[i], m22[i + 7], m22[i + 14]);
+                m8[7] = m22[21];
+                mx = max3(max3(m8[0], m8[1], m8[2]), max3(m8[3], m8[4], m8[5]), fmaxf(m8[6], m8[7]));
                 mx *= sl2;  // log2 units (-inf stays -inf)
             }
             // double-buffered by step parity: a half can be at most one step ahead of its partner here
@@ -385,15 +417,21 @@ attn_tc_kernel(QueryRows qr, const __grid_constant__ CUtensorMap tm_q, const __g
                     // 2^(sl2 s - m_ref) in one FFMA per key; a row that did not select the block (or has no
                     // finite reference yet) gets 2^-inf = 0
                     const float mneg = (sel && m_ref != neg_inf()) ? -m_ref : neg_inf();
-                    float ps[4] = {0.f, 0.f, 0.f, 0.f};
+                    // the exponents of a key pair in one paired FMA, the row sums in four paired accumulators
+                    const unsigned long long sl2x2 = f2(sl2, sl2), mnegx2 = f2(mneg, mneg);
+                    unsigned long long ps2[4] = {0ull, 0ull, 0ull, 0ull};
 #pragma unroll
                     for (int j2 = 0; j2 < 32; ++j2) {
-                        const float p0 = ex2_approx(fmaf(x[2 * j2], sl2, mneg));
-                        const float p1 = ex2_approx(fmaf(x[2 * j2 + 1], sl2, mneg));
-                        ps[j2 & 3] += p0 + p1;
+                        float e0, e1;
+                        f2_split(fma2(f2(x[2 * j2], x[2 * j2 + 1]), sl2x2, mnegx2), e0, e1);
+                        const float p0 = ex2_approx(e0), p1 = ex2_approx(e1);
+                        ps2[j2 & 3] = add2(ps2[j2 & 3], f2(p0, p1));
                         w[j2] = pack_bf16(p0, p1);
                     }
-                    l += (ps[0] + ps[1]) + (ps[2] + ps[3]);
+                    float s0, s1, s2, s3;
+                    f2_split(add2(ps2[0], ps2[1]), s0, s1);
+                    f2_split(add2(ps2[2], ps2[3]), s2, s3);
+                    l += (s0 + s1) + (s2 + s3);
                 } else {
 #pragma unroll
                     for (int j = 0; j < 32; ++j) w[j] = 0u;
