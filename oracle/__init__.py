@@ -18,6 +18,8 @@ Functions and the steps they follow (sources: the MiniCPM4 pages):
   * ``sparse_attention_backward`` -- gradients of that attention for a fixed selection (training; same
                               section, item 3: operators for training and inference; the derivative of
                               the forward's definition)
+  * ``kernel_pool_backward`` -- the gradient of the semantic kernels with respect to K: the transpose of the
+                              window mean (same section, item 3; the derivative of step 1's definition)
   * ``dense_attention``    -- plain causal GQA attention, written separately
   * ``window_attention``   -- the draft model's sliding-window attention (same bullet as the tree drafts)
 The pages' "efficient LogSumExp estimation" is not defined there (parity unpinned); ``Params.lse_stride`` selects
@@ -113,6 +115,8 @@ def _load():
         lib.orc_dense_attention.restype = i
         lib.orc_window_attention.argtypes = [P, i, i, i, i, i, P, P, i, P, i, ctypes.c_double, P, P]
         lib.orc_window_attention.restype = i
+        lib.orc_kernel_pool_backward.argtypes = [P, i, i, i, i, P, i, i, i, P]
+        lib.orc_kernel_pool_backward.restype = i
         lib.orc_round_bf16.argtypes = [ctypes.c_double]
         lib.orc_round_bf16.restype = ctypes.c_uint16
         lib.orc_num_threads.restype = i
@@ -163,6 +167,21 @@ def kernel_pool(K, old_len, new_len, kernel_size, kernel_stride, kern=None, nk_c
     if rc != 0:
         raise ValueError(f"orc_kernel_pool: bad arguments (rc={rc})")
     return kern
+
+
+def kernel_pool_backward(dkern, lens, Lcap, kernel_size=32, kernel_stride=16):
+    """dK ([B, Lcap, Hkv, d] fp64) for the kernel gradients dkern ([B, Hkv, nk_cap, d] fp32) of the kernels
+    j < nk(lens[b]): each kernel gives 1/kernel_size of its gradient to each key of its window."""
+    lib = _load()
+    dkern = _c(dkern, np.float32)
+    B, Hkv, nk_cap, d = dkern.shape
+    lens = _c(lens, np.int32)
+    dk = np.zeros((B, Lcap, Hkv, d), np.float64)
+    rc = lib.orc_kernel_pool_backward(_ptr(dkern), B, Lcap, Hkv, d, _ptr(lens), kernel_size, kernel_stride, nk_cap,
+                                      _ptr(dk))
+    if rc != 0:
+        raise ValueError(f"orc_kernel_pool_backward: bad arguments (rc={rc})")
+    return dk
 
 
 def block_score_topk(q, kern, q_ctx, params: Params, nb_max=None):

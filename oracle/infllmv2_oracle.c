@@ -32,6 +32,8 @@
  *   7. the gradients of step 5's attention with respect to q, K and V for a fixed selection (training)
  *        -- "Model architecture: InfLLM v2", item 3 (operators for training as well as inference); the
  *           derivative of step 5's definition, the pages give no formula.
+ *   8. the gradient of step 1 (the semantic kernels) with respect to K: the adjoint of the window mean,
+ *      the bf16 rounding taken as the identity -- same item 3; the derivative of step 1's definition.
  *
  * Every floating-point step is fp64; inputs are bf16 bit patterns widened exactly.  Rows are
  * independent, so the only parallelism is an OpenMP loop over (sequence, token, group) rows; there is
@@ -48,7 +50,8 @@
  * Parity pins (tests/test_oracle_pins.py): hand-worked two-block example, closed forms of the window
  * mean, special cases that reduce to library softmax attention / average pooling, and invariants; the
  * backward (item 7) against central differences of the forward, library autograd on the dense case,
- * the one-key closed form and the sum rules of the softmax Jacobian.
+ * the one-key closed form and the sum rules of the softmax Jacobian; the kernel backward (item 8) against
+ * the forward by the adjoint identity on keys whose window means are exact in bf16.
  * The pages' "efficient LogSumExp estimation" is not defined there (parity unpinned): params.lse_stride > 1
  * selects one reading of it, the LSE from every s-th visible kernel times s, pinned only to its special cases
  * (s = 1 is exact; the closed form on equal scores).
@@ -654,6 +657,39 @@ int orc_window_attention(const uint16_t* q, int B, int T, int Hq, int Hkv, int d
 {
     if (window < 1) return -1;
     return range_attention(q, B, T, Hq, Hkv, d, K, V, Lcap, q_ctx, window, scale, out, lse_out);
+}
+
+/* ----------------------------------------------------------------------------------------------- */
+/* step 8: gradient of the semantic kernels with respect to K                                       */
+/* ----------------------------------------------------------------------------------------------- */
+
+/*
+ * The transpose of step 1's window mean (its bf16 rounding taken as the identity): every kernel j in
+ * [0, nk(lens[b])) hands 1/ks of its gradient to each of the ks keys of its window,
+ *   dk[b, i, g, :] = sum_{j : j*kst <= i < j*kst + ks} dkern[b, g, j, :] / ks.
+ * dkern: [B, Hkv, nk_cap, d] fp32; dk: [B, Lcap, Hkv, d] fp64, overwritten (rows no kernel reads are 0).
+ * Returns 0, or -1 when a length exceeds Lcap or nk(lens[b]) exceeds nk_cap.
+ */
+int orc_kernel_pool_backward(const float* dkern, int B, int Lcap, int Hkv, int d, const int32_t* lens,
+                             int kernel_size, int kernel_stride, int nk_cap, double* dk)
+{
+    orc_params p;
+    memset(&p, 0, sizeof p);
+    p.kernel_size = kernel_size;
+    p.kernel_stride = kernel_stride;
+    for (int b = 0; b < B; ++b)
+        if (lens[b] < 0 || lens[b] > Lcap || nk_of(lens[b], &p) > nk_cap) return -1;
+    memset(dk, 0, sizeof(double) * (size_t)B * Lcap * Hkv * d);
+    for (int b = 0; b < B; ++b) {
+        const long nk = nk_of(lens[b], &p);
+        for (int g = 0; g < Hkv; ++g)
+            for (long j = 0; j < nk; ++j)
+                for (long i = j * kernel_stride; i < j * kernel_stride + kernel_size; ++i)
+                    for (int c = 0; c < d; ++c)
+                        dk[(((size_t)b * Lcap + i) * Hkv + g) * d + c] +=
+                            (double)dkern[(((size_t)b * Hkv + g) * nk_cap + j) * d + c] / kernel_size;
+    }
+    return 0;
 }
 
 int orc_num_threads(void)

@@ -612,3 +612,48 @@ def test_lse_estimate_closed_form_on_equal_scores(oracle, stride):
     for t in range(3):
         nk = oracle.num_kernels(int(qc[0, t]))
         assert np.allclose(r["lse"][0, t], math.log(stride * math.ceil(nk / stride)), rtol=0, atol=1e-12)
+
+
+# ------------------------------------------------------------------------------------------------
+# gradient of the semantic kernels with respect to K (the transpose of the window mean)
+# ------------------------------------------------------------------------------------------------
+
+def test_kernel_pool_backward_is_the_adjoint_of_the_forward(oracle):
+    """<backward(dkern), K> = <dkern, kernel_pool(K)> for every K and dkern: with K in {0, 1}, every window
+    mean s / 32 (s <= 32) is exact in bf16, so the forward oracle's rounding drops out.  Ragged lengths, one
+    below a window, one not on the 16-key grid; the gradient of kernels past nk(lens) must not reach K."""
+    rng = np.random.default_rng(70)
+    B, Lcap, Hkv, d = 3, 300, 2, 8
+    lens = np.array([300, 151, 20], np.int32)
+    Kf = rng.integers(0, 2, (B, Lcap, Hkv, d)).astype(np.float32)
+    K = bits(Kf)
+    nk_cap = oracle.num_kernels(Lcap)
+    kern = oracle.kernel_pool(K, [0] * B, lens, 32, 16, nk_cap=nk_cap)
+    dkern = rng.standard_normal((B, Hkv, nk_cap, d)).astype(np.float32)
+    dk = oracle.kernel_pool_backward(dkern, lens, Lcap)
+    for b in range(B):
+        nk = oracle.num_kernels(int(lens[b]))
+        lhs = np.sum(dk[b] * Kf[b].astype(np.float64))
+        rhs = np.sum(dkern[b, :, :nk].astype(np.float64) * f64(kern[b, :, :nk]))
+        assert lhs == pytest.approx(rhs, rel=1e-12, abs=1e-12)
+        assert not dk[b, int(lens[b]):].any()  # keys past the context get nothing
+    assert not dk[2].any()  # 20 keys: no complete window
+
+
+def test_kernel_pool_backward_one_window_and_mass(oracle):
+    """One kernel with gradient 1 spreads 1/32 over exactly its 32 keys; in general each kernel's gradient mass
+    reaches K whole (the column sums of the mean are 1)."""
+    B, Lcap, Hkv, d = 1, 128, 1, 4
+    nk_cap = oracle.num_kernels(Lcap)
+    dkern = np.zeros((B, Hkv, nk_cap, d), np.float32)
+    dkern[0, 0, 3, :] = 1.0
+    dk = oracle.kernel_pool_backward(dkern, [Lcap], Lcap)
+    want = np.zeros(Lcap)
+    want[48:80] = 1.0 / 32
+    assert np.array_equal(dk[0, :, 0, 2], want)
+    rng = np.random.default_rng(71)
+    dkern = rng.standard_normal((2, 2, nk_cap, 6)).astype(np.float32)
+    dk = oracle.kernel_pool_backward(dkern, [Lcap, 100], Lcap)
+    assert np.allclose(dk[0].sum(axis=0), dkern[0].astype(np.float64).sum(axis=1), rtol=0, atol=1e-12)
+    nk = oracle.num_kernels(100)
+    assert np.allclose(dk[1].sum(axis=0), dkern[1, :, :nk].astype(np.float64).sum(axis=1), rtol=0, atol=1e-12)
