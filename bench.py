@@ -632,6 +632,37 @@ class PrefillBench:
         return total, per
 
 
+def kernel_pool_backward_leg(peaks, peak_kind, reps=20):
+    """The gradient of the semantic kernels with respect to K over the 128K decode batch's shapes (4 sequences
+    of 131072 keys, 2 KV heads, d 128): dk (fp32, 537 MB) overwritten from the kernel gradients (fp32, 34 MB).
+    HBM-bound; the algorithmic bytes are that write and that read.  The 537 MB written per call exceeds L2, so
+    consecutive calls do not hit it; the time is the mean of `reps` calls between two CUDA events."""
+    import torch
+    from trainable_block_sparse_v2_b200 import binding
+    B, L = len(LENS_128K), max(LENS_128K)
+    nk_cap = nk(L)
+    dkern = torch.randn((B, HKV, nk_cap, D), dtype=torch.float32, device="cuda")
+    dk = torch.empty((B, L, HKV, D), dtype=torch.float32, device="cuda")
+    lens = torch.tensor([L] * B, dtype=torch.int32, device="cuda")
+    p = binding.Params()
+    for _ in range(3):
+        binding.infllmv2_kernel_pool_backward(dkern, lens, L, p, dk)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(reps):
+        binding.infllmv2_kernel_pool_backward(dkern, lens, L, p, dk)
+    e1.record()
+    e1.synchronize()
+    t = e0.elapsed_time(e1) / 1e3 / reps
+    nbytes = dk.numel() * 4 + B * HKV * nk(L) * D * 4
+    del dkern, dk
+    torch.cuda.empty_cache()
+    return {"workload": "dk of 4 x 131072 keys, 2 KV heads, d 128 (fp32) from their kernel gradients",
+            "us_per_call": t * 1e6, "algorithmic_bytes": nbytes, "achieved_gbs": nbytes / t / 1e9,
+            "frac_of_" + peak_kind: nbytes / t / 1e9 / peaks["hbm_gbs"], "timing": f"mean of {reps} calls"}
+
+
 class Decode32kBench:
     """Decode at a 32K context, batch 1 (32 / 2 heads, d 128, top-k 64): one step = the kernel pool of the new
     key + the fused decode step (scoring, top-k, attention), on a cache restored every step (the pool of the
@@ -1133,6 +1164,8 @@ def run_ours(args):
             line["gpu_launches"] += args.prefill_steps * 6
         del pb
         torch.cuda.empty_cache()
+        if not args.no_backward:
+            line["kernel_pool_backward"] = kernel_pool_backward_leg(peaks, peak_kind)
 
     if not args.no_decode32k:
         # batch-1 decode at 32K: launch-latency bound by nature (5.4 MB per step); reported, like the tree leg,

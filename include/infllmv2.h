@@ -151,6 +151,29 @@ int infllmv2_kernel_pool(const void* k, int batch, int lcap, int hkv, int head_d
                          int nk_cap, infllmv2_stream_t stream);
 
 /*
+ * Backward of step 1 (training: MiniCPM4 technical details, "Model architecture: InfLLM v2", item 3 -- the
+ * operators serve training as well as inference; the pages give no formula, so this is the derivative of step
+ * 1's definition, with the bf16 rounding of the kernels taken as the identity).  For a loss that depends on the
+ * kernels differentiably (the attention backward passes no gradient through them), the transpose of the
+ * window mean:
+ *   dk[b, i, g, :] (+)= sum_{j < nk(lens[b]), 16 j <= i < 16 j + 32} dkern[b, g, j, :] / 32,  i in [0, lens[b])
+ * i.e. each key of the 16-key chunk c gets (dkern[c - 1] + dkern[c]) / 32, a term only for a complete window.
+ * The pair is summed in fp32 with one rounding and scaled exactly, so with accumulate = 0 a normal result is
+ * the correctly rounded exact value.
+ *   dkern      [B, Hkv, nk_cap, d] fp32 (device, 16-byte aligned)
+ *   lens       [B] int32 (device): keys per sequence; values past lcap are clamped to it, kernels past nk_cap
+ *              are not read
+ *   max_len    host upper bound of lens[b] (sizes the grid): 0 <= max_len <= lcap, nk(max_len) <= nk_cap
+ *   dk         [B, Lcap, Hkv, d] fp32 (device, 16-byte aligned).  accumulate = 1 adds into rows [0, lens[b])
+ *              (e.g. onto infllmv2_sparse_attn_backward's dk), 0 overwrites them; rows past lens[b] untouched.
+ * B * Hkv <= 65535.  Returns INFLLMV2_OK, INFLLMV2_ERR_INVALID_ARG, INFLLMV2_ERR_UNSUPPORTED or
+ * INFLLMV2_ERR_CUDA.
+ */
+int infllmv2_kernel_pool_backward(const float* dkern, int batch, int lcap, int hkv, int head_dim, const int32_t* lens,
+                                  int max_len, const infllmv2_params* params, int nk_cap, float* dk, int accumulate,
+                                  infllmv2_stream_t stream);
+
+/*
  * Step 2 -- block scoring and top-k selection (same section, items 1-3).
  * For each query (b, t) and KV group g, with kernel scores z_h(j) = scale * q_h . kern_j over the visible
  * kernels and LSE_h = log sum_j exp z_h(j) (exact), the group score of block blk is

@@ -128,6 +128,21 @@ def test_attention_entry_points_reject_bad_arguments(lib):
     assert lib.infllmv2_kernel_pool(A16, 1, 4096, 2, 128, A4, A4, 4096, ctypes.byref(bad), A16, 255, None) == \
         UNSUPPORTED
     assert lib.infllmv2_kernel_pool(A16, 1, 4096, 2, 128, A4, A4, 4096, ctypes.byref(cp), A16, 10, None) == INVALID
+    # kernel pool backward: misaligned gradients, max_len past lcap, kernel cache too small, bad mode, d 96
+    nk = binding.num_kernels(4096)
+    assert lib.infllmv2_kernel_pool_backward(A16 + 4, 1, 4096, 2, 128, A4, 4096, ctypes.byref(cp), nk, A16, 0,
+                                             None) == INVALID
+    assert lib.infllmv2_kernel_pool_backward(A16, 1, 4096, 2, 128, A4, 4097, ctypes.byref(cp), nk + 1, A16, 0,
+                                             None) == INVALID
+    assert lib.infllmv2_kernel_pool_backward(A16, 1, 4096, 2, 128, A4, 4096, ctypes.byref(cp), nk - 1, A16, 0,
+                                             None) == INVALID
+    assert lib.infllmv2_kernel_pool_backward(A16, 1, 4096, 2, 128, A4, 4096, ctypes.byref(cp), nk, A16, 2,
+                                             None) == INVALID
+    assert lib.infllmv2_kernel_pool_backward(A16, 1, 4096, 2, 96, A4, 4096, ctypes.byref(cp), nk, A16, 0,
+                                             None) == UNSUPPORTED
+    assert lib.infllmv2_kernel_pool_backward(A16, 1, 4096, 2, 128, A4, 4096, ctypes.byref(bad), nk, A16, 0,
+                                             None) == UNSUPPORTED
+    assert lib.infllmv2_kernel_pool_backward(A16, 1, 4096, 2, 128, A4, 0, ctypes.byref(cp), nk, A16, 0, None) == OK
     # window decode: window 0
     assert lib.infllmv2_window_attn_decode(A16, 1, 32, 2, 128, A16, A16, 4096, A4, 4096, 0, ctypes.c_float(0.0),
                                            A16, None, WS, 1 << 30, None) == INVALID

@@ -211,3 +211,53 @@ def test_backward_32k_prefill_full_size(oracle):
     lhs = float((dv64 * V.double()).sum())
     rhs = float((DO.double() * out.double()).sum())
     assert abs(lhs - rhs) <= 2e-3 * abs(rhs) + 1.0
+
+
+# ------------------------------------------------------------------------------------------------
+# gradient of the semantic kernels with respect to K (the transpose of the window mean)
+# ------------------------------------------------------------------------------------------------
+
+@pytest.mark.parametrize("d", [64, 128])
+def test_kernel_pool_backward_matches_oracle(oracle, d):
+    """Ragged lengths (below one window, off the 16-key grid, at the cache capacity, 0), two KV heads.
+    Overwrite: bit-exact with the oracle's fp64 value rounded to fp32 (one fp32 sum of two terms, an exact
+    power-of-two scale); rows past each length keep their bytes.  Accumulate: within one fp32 rounding of
+    dk0 + oracle."""
+    rng = np.random.default_rng(800 + d)
+    lens = np.array([5000, 31, 1043, 6000, 0], np.int32)
+    B, Lcap, Hkv = len(lens), 6000, 2
+    nk_cap = binding.num_kernels(Lcap)
+    dkern = rng.standard_normal((B, Hkv, nk_cap, d)).astype(np.float32)
+    ref = oracle.kernel_pool_backward(dkern, lens, Lcap)
+    dk0 = rng.standard_normal((B, Lcap, Hkv, d)).astype(np.float32)
+    p = binding.Params()
+    dkern_d, lens_d = torch.from_numpy(dkern).cuda(), dev_i32(lens)
+    dk = torch.from_numpy(dk0).cuda()
+    binding.infllmv2_kernel_pool_backward(dkern_d, lens_d, int(lens.max()), p, dk, accumulate=False)
+    got = dk.cpu().numpy()
+    for b in range(B):
+        n = int(lens[b])
+        assert np.array_equal(got[b, :n], ref[b, :n].astype(np.float32)), f"sequence {b}: rows [0, {n})"
+        assert np.array_equal(got[b, n:], dk0[b, n:]), f"sequence {b}: rows past the length were written"
+    dk = torch.from_numpy(dk0).cuda()
+    binding.infllmv2_kernel_pool_backward(dkern_d, lens_d, int(lens.max()), p, dk, accumulate=True)
+    got = dk.cpu().numpy().astype(np.float64)
+    want = dk0.astype(np.float64) + ref
+    for b in range(B):
+        n = int(lens[b])
+        tol = 2.0 ** -23 * (np.abs(dk0[b, :n]).astype(np.float64) + np.abs(ref[b, :n])) * 2
+        assert np.all(np.abs(got[b, :n] - want[b, :n]) <= tol + 1e-30), f"sequence {b} (accumulate)"
+        assert np.array_equal(got[b, n:], dk0[b, n:].astype(np.float64))
+
+
+def test_kernel_pool_backward_full_128k(oracle):
+    """One 128K sequence (2 KV heads, d 128), the size of the decode workload's longest rows: every row
+    bit-exact with the oracle rounded to fp32."""
+    rng = np.random.default_rng(810)
+    L, Hkv, d = 131072, 2, 128
+    nk_cap = binding.num_kernels(L)
+    dkern = rng.standard_normal((1, Hkv, nk_cap, d)).astype(np.float32)
+    ref = oracle.kernel_pool_backward(dkern, [L], L).astype(np.float32)
+    dk = torch.empty((1, L, Hkv, d), dtype=torch.float32, device="cuda")
+    binding.infllmv2_kernel_pool_backward(torch.from_numpy(dkern).cuda(), dev_i32([L]), L, binding.Params(), dk)
+    assert np.array_equal(dk.cpu().numpy(), ref)

@@ -75,6 +75,7 @@ _SIGS = {
     "infllmv2_workspace_size": ([_PP, _I, _I, _I, _I, _I, _I], _SZ),
     "infllmv2_kernel_pool": ([_P, _I, _I, _I, _I, _P, _P, _I, _PP, _P, _I, _P], _I),
     "infllmv2_kv_append": ([_P, _P, _I, _I, _I, _P, _P, _P, _I, _P], _I),
+    "infllmv2_kernel_pool_backward": ([_P, _I, _I, _I, _I, _P, _I, _PP, _I, _P, _I, _P], _I),
     "infllmv2_block_score_topk": ([_P, _I, _I, _I, _I, _I, _P, _P, _I, _P, _I, _PP, _P, _P, _P, _SZ, _P], _I),
     "infllmv2_sparse_attn_prefill": ([_P, _I, _I, _I, _I, _I, _P, _P, _I, _P, _P, _I, _P, _P, _PP, _P, _P, _P,
                                       _SZ, _P], _I),
@@ -245,6 +246,23 @@ def infllmv2_kernel_pool(k, old_lens, new_lens, max_new_keys, params: Params, ke
     st = load().infllmv2_kernel_pool(_ptr(k), B, Lcap, Hkv, d, _ptr(old_lens), _ptr(new_lens), int(max_new_keys),
                                      ctypes.byref(cp), _ptr(kern), kern.shape[2], _stream(stream))
     _check("infllmv2_kernel_pool", st)
+
+
+def infllmv2_kernel_pool_backward(dkern, lens, max_len, params: Params, dk, accumulate=False, stream=None):
+    """dk[b, i, g] (+)= sum over the complete windows j that contain key i of dkern[b, g, j] / 32, for
+    i < lens[b] (the gradient of the semantic kernels with respect to K)"""
+    _need(dkern, torch.float32, "dkern", 4)
+    B, Hkv, nk_cap, d = dkern.shape
+    _need(dk, torch.float32, "dk", 4)
+    if (dk.shape[0], dk.shape[2], dk.shape[3]) != (B, Hkv, d):
+        raise ValueError(f"dk: expected shape ({B}, Lcap, {Hkv}, {d}), got {tuple(dk.shape)}")
+    _int32(lens, "lens", B)
+    _devices("infllmv2_kernel_pool_backward", dkern, dk, lens)
+    cp = params.c()
+    st = load().infllmv2_kernel_pool_backward(_ptr(dkern), B, dk.shape[1], Hkv, d, _ptr(lens), int(max_len),
+                                              ctypes.byref(cp), nk_cap, _ptr(dk), 1 if accumulate else 0,
+                                              _stream(stream))
+    _check("infllmv2_kernel_pool_backward", st)
 
 
 def infllmv2_kv_append(k_new, v_new, pos, k_cache, v_cache, stream=None):

@@ -324,6 +324,24 @@ int infllmv2_kernel_pool(const void* k, int batch, int lcap, int hkv, int head_d
                                             max_new_keys, kern, nk_cap, (cudaStream_t)stream));
 }
 
+int infllmv2_kernel_pool_backward(const float* dkern, int batch, int lcap, int hkv, int head_dim, const int32_t* lens,
+                                  int max_len, const infllmv2_params* params, int nk_cap, float* dk, int accumulate,
+                                  infllmv2_stream_t stream)
+{
+    IV2_TRY(check_params(params));
+    IV2_TRY(check_heads(batch, 1, hkv, hkv, head_dim));
+    IV2_TRY(check_ptr16(dkern));
+    IV2_TRY(check_ptr16(dk));
+    IV2_TRY(check_ptr4(lens));
+    if (lcap < 1 || max_len < 0 || max_len > lcap || nk_cap < 1 || (accumulate != 0 && accumulate != 1))
+        return INFLLMV2_ERR_INVALID_ARG;
+    if (nk_cap < nk_of(max_len)) return INFLLMV2_ERR_INVALID_ARG;
+    if ((long)batch * hkv > 65535) return INFLLMV2_ERR_UNSUPPORTED;
+    if (max_len == 0) return INFLLMV2_OK;
+    return launched(iv2::launch_kernel_pool_backward(dkern, batch, lcap, hkv, head_dim, lens, max_len, nk_cap, dk,
+                                                     accumulate != 0, (cudaStream_t)stream));
+}
+
 int infllmv2_kv_append(const void* k_new, const void* v_new, int batch, int hkv, int head_dim, const int32_t* pos,
                        void* k_cache, void* v_cache, int lcap, infllmv2_stream_t stream)
 {

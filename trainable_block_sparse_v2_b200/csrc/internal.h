@@ -173,6 +173,9 @@ int attn_split_max_blocks(int max_ctx, int kmax, int dense_len, bool dense_all, 
 cudaError_t launch_kernel_pool(const void* k, int B, const KvRows& kr, int Hkv, int D, const int32_t* old_lens,
                                const int32_t* new_lens, int max_new_keys, void* kern, int nk_cap, cudaStream_t s);
 
+cudaError_t launch_kernel_pool_backward(const float* dkern, int B, int Lcap, int Hkv, int D, const int32_t* lens,
+                                        int max_len, int nk_cap, float* dk, bool accumulate, cudaStream_t s);
+
 cudaError_t launch_kv_append(const void* k_new, const void* v_new, int B, int Hkv, int D, const int32_t* pos,
                              void* k_cache, void* v_cache, const KvRows& kr, cudaStream_t s);
 

@@ -119,6 +119,63 @@ cudaError_t launch_kernel_pool(const void* k, int B, const KvRows& kr, int Hkv, 
 }
 
 // ---------------------------------------------------------------------------------------------------
+// Gradient of the semantic kernels with respect to K (training; MiniCPM4 technical details, "Model
+// architecture: InfLLM v2", item 3 -- the derivative of step 1's definition, the bf16 rounding of the kernels
+// taken as the identity): the transpose of the window mean.  With windows of 32 keys at stride 16, the keys of
+// the 16-key chunk c lie in exactly the windows c - 1 and c, so every key of the chunk receives
+//   dk = (dkern[c - 1] + dkern[c]) / 32         (a term only for a window j in [0, nk(len)))
+// fp32: the pair is summed with one rounding and the power-of-two scale is exact, so a normal result is the
+// correctly rounded value of the exact one.  One CTA writes one chunk of one (sequence, KV head): 16 rows of
+// d fp32 in 16-byte stores; the two kernel rows it reads are shared by all of them through L1.  Lengths are
+// clamped to Lcap and the kernel index to nk_cap, so no device-side value can move an access out of bounds.
+// ---------------------------------------------------------------------------------------------------
+template <int D>
+__global__ void __launch_bounds__(128) kernel_pool_bwd_kernel(const float4* __restrict__ dkern,
+                                                             const int32_t* __restrict__ lens, int Lcap, int Hkv,
+                                                             int nk_cap, float4* __restrict__ dk, int accumulate)
+{
+    pdl_launch_dependents();
+    pdl_wait();
+    constexpr int F = D / 4;  // float4 per row
+    const int c = blockIdx.x;
+    const int bg = blockIdx.y, b = bg / Hkv, g = bg % Hkv;
+    const int len = min(lens[b], Lcap);
+    const int i0 = c * kKernelStride;
+    if (i0 >= len) return;
+    const int nk = min(len >= kKernelSize ? (len - kKernelSize) / kKernelStride + 1 : 0, nk_cap);
+    const bool has_a = c >= 1 && c - 1 < nk, has_b = c < nk;
+    const float4* row_a = dkern + ((size_t)bg * nk_cap + (has_a ? c - 1 : 0)) * F;
+    const float4* row_b = dkern + ((size_t)bg * nk_cap + (has_b ? c : 0)) * F;
+    const int rows = min(kKernelStride, len - i0);
+    constexpr float kInv = 1.f / kKernelSize;
+    for (int e = threadIdx.x; e < rows * F; e += blockDim.x) {
+        const int row = e / F, f = e % F;
+        const float4 za = has_a ? row_a[f] : make_float4(0.f, 0.f, 0.f, 0.f);
+        const float4 zb = has_b ? row_b[f] : make_float4(0.f, 0.f, 0.f, 0.f);
+        float4 v = make_float4((za.x + zb.x) * kInv, (za.y + zb.y) * kInv, (za.z + zb.z) * kInv, (za.w + zb.w) * kInv);
+        float4* dst = dk + (((size_t)b * Lcap + i0 + row) * Hkv + g) * F + f;
+        if (accumulate) {
+            const float4 o = *dst;
+            v = make_float4(o.x + v.x, o.y + v.y, o.z + v.z, o.w + v.w);
+        }
+        *dst = v;
+    }
+}
+
+cudaError_t launch_kernel_pool_backward(const float* dkern, int B, int Lcap, int Hkv, int D, const int32_t* lens,
+                                        int max_len, int nk_cap, float* dk, bool accumulate, cudaStream_t s)
+{
+    const dim3 grid((max_len + kKernelStride - 1) / kKernelStride, B * Hkv);
+    const auto* dkp = reinterpret_cast<const float4*>(dkern);
+    auto* dkq = reinterpret_cast<float4*>(dk);
+    if (D == 128)
+        return launch_pdl(kernel_pool_bwd_kernel<128>, grid, dim3(128), 0, s, dkp, lens, Lcap, Hkv, nk_cap, dkq,
+                          accumulate ? 1 : 0);
+    return launch_pdl(kernel_pool_bwd_kernel<64>, grid, dim3(128), 0, s, dkp, lens, Lcap, Hkv, nk_cap, dkq,
+                      accumulate ? 1 : 0);
+}
+
+// ---------------------------------------------------------------------------------------------------
 // Cache maintenance of a decode step (the pages have no counterpart): one new key and value row per
 // sequence into the caches, k_cache[b, pos[b], :, :] = k_new[b, :, :] (v likewise).  16-byte copies; a
 // position outside [0, Lcap) writes nothing.  With a paged cache the row is that of position pos[b] through
