@@ -46,7 +46,7 @@ NCU_TRAFFIC = {
     "sparse_decode_step": 31_308_928,                   # decode_fused_kernel: 31.31 MB read, ~2 KB written
     "sparse_attn_decode": None,                         # attn_split_kernel + attn_merge_kernel
     "block_score_topk": None,                           # score_scan_kernel + score_select_kernel
-    "sparse_attn_prefill": None,                        # attn_tc_kernel<16, 128>
+    "sparse_attn_prefill": 322_111_488 + 229_101_312,   # attn_tc_kernel<16, 128>
 }
 KERNELS_PER_STEP = {"two_call": 5,  # kernel pool, score scan, select, split attention, merge
                     "fused": 2}     # kernel pool, fused decode step (scoring + top-k + attention)
