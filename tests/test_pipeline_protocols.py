@@ -271,18 +271,21 @@ def test_checker_reports_a_deadlock_and_a_wrong_phase():
 
 # --------------------------------------------------------------------------------------------------------------
 # bwd_dq_tc_kernel (csrc/attn_bwd_tc.cu): one 128-row tile over U union blocks.  Warp 0: Q and dO once, K per
-# step (3-slot ring); warp 10: V per step; warp 1: S(p) = Q K^T and dP(p) = dO V^T into buffers p & 1, then
-# dQ += dS(p - 1) K; warps 2-9: dS, two per lane quarter (half 0: keys 0-31, half 1: keys 32-63); dS goes
+# step (3-slot ring); warp 10: V per step; warp 1: S(p) = Q K^T into buffer p & 1 once dQ(p - 2) is done; warp
+# 11: dP(p) = dO V^T into buffer p & 1 once dS(p - 2) was signalled; warp 12: dQ += dS(p) K (the three issuers'
+# ops unordered relative to each other; K(p) freed by S(p)'s and dQ(p)'s commits); warps 2-9: dS, two per lane
+# quarter (half 0: keys 0-31, half 1: keys 32-63); dS goes
 # back over the first 32 columns of its S buffer after both halves' loads (named barrier per quarter).
 # --------------------------------------------------------------------------------------------------------------
 def bwd_dq_model(m: PipelineModel, U: int, mistake: str = ""):
     m.bar("qd_full", 1)
     m.bar("qd_tmem", 128)
     for i in range(RING):
-        for n in ("k_full", "k_empty", "v_full", "v_empty"):
+        for n in ("k_full", "v_full", "v_empty"):
             m.bar(f"{n}{i}", 1)
+        m.bar(f"k_empty{i}", 1 if mistake == "k_empty waits for one issuer" else 2)
     for i in range(2):
-        m.bar(f"s_full{i}", 1)
+        m.bar(f"s_full{i}", 2)
         m.bar(f"ds_full{i}", 256)
         m.bar(f"dq_done{i}", 1)
 
@@ -305,29 +308,41 @@ def bwd_dq_model(m: PipelineModel, U: int, mistake: str = ""):
             yield ("arrive_tx", f"v_full{s}", 1, 1)
             yield ("tma", f"v_full{s}", 1, [(f"V{s}", ("V", p))])
 
-    def issuer():
+    def s_issuer():
         yield ("wait", "qd_tmem", 0)
-        for p in range(U + 1):
-            if p < U:
-                s, sb = p % RING, p & 1
-                yield ("wait", f"k_full{s}", p // RING)
-                yield ("wait", f"v_full{s}", p // RING)
-                yield ("mma", [(f"QT.q{q}", "Q") for q in range(4)] + [(f"K{s}", ("K", p))],
-                       [(f"S{sb}.q{q}.{c}", ("S", p)) for q in range(4) for c in ("a", "b", "hi")], f"S{p}")
-                yield ("mma", [(f"dOT.q{q}", "dO") for q in range(4)] + [(f"V{s}", ("V", p))],
-                       [(f"DP{sb}.q{q}.{c}", ("DP", p)) for q in range(4) for c in ("lo", "hi")], f"DP{p}")
-                yield ("commit", f"s_full{sb}")
-                yield ("commit", f"v_empty{s}")
-            if p >= 1:
-                v = p - 1
-                db, s = v & 1, v % RING
-                if mistake != "issuer skips ds_full":
-                    yield ("wait", f"ds_full{db}", v >> 1)
-                reads = [(f"S{db}.q{q}.{c}", ("dS", v)) for q in range(4) for c in ("a", "b")]
-                reads += [(f"K{s}", ("K", v))] + ([("dQ", ("dQ", v - 1))] if v > 0 else [])
-                yield ("mma", reads, [("dQ", ("dQ", v))], f"dQ{v}")
-                yield ("commit", f"dq_done{db}")
-                yield ("commit", f"k_empty{s}")
+        for p in range(U):
+            s, sb = p % RING, p & 1
+            if p >= 2 and mistake != "S issuer skips dq_done":
+                yield ("wait", f"dq_done{sb}", (p - 2) >> 1)
+            yield ("wait", f"k_full{s}", p // RING)
+            yield ("mma", [(f"QT.q{q}", "Q") for q in range(4)] + [(f"K{s}", ("K", p))],
+                   [(f"S{sb}.q{q}.{c}", ("S", p)) for q in range(4) for c in ("a", "b", "hi")], f"S{p}")
+            yield ("commit", f"s_full{sb}")
+            yield ("commit", f"k_empty{s}")
+
+    def dp_issuer():
+        yield ("wait", "qd_tmem", 0)
+        for p in range(U):
+            s, sb = p % RING, p & 1
+            if p >= 2 and mistake != "dP issuer skips ds_full":
+                yield ("wait", f"ds_full{sb}", (p - 2) >> 1)
+            yield ("wait", f"v_full{s}", p // RING)
+            yield ("mma", [(f"dOT.q{q}", "dO") for q in range(4)] + [(f"V{s}", ("V", p))],
+                   [(f"DP{sb}.q{q}.{c}", ("DP", p)) for q in range(4) for c in ("lo", "hi")], f"DP{p}")
+            yield ("commit", f"s_full{sb}")
+            yield ("commit", f"v_empty{s}")
+
+    def dq_issuer():
+        for v in range(U):
+            db, s = v & 1, v % RING
+            if mistake != "issuer skips ds_full":
+                yield ("wait", f"ds_full{db}", v >> 1)
+            yield ("wait", f"k_full{s}", v // RING)
+            reads = [(f"S{db}.q{q}.{c}", ("dS", v)) for q in range(4) for c in ("a", "b")]
+            reads += [(f"K{s}", ("K", v))] + ([("dQ", ("dQ", v - 1))] if v > 0 else [])
+            yield ("mma", reads, [("dQ", ("dQ", v))], f"dQ{v}")
+            yield ("commit", f"dq_done{db}")
+            yield ("commit", f"k_empty{s}")
 
     def ds_warp(w):
         q4, half = w & 3, (w - 2) >> 2
@@ -359,7 +374,9 @@ def bwd_dq_model(m: PipelineModel, U: int, mistake: str = ""):
 
     m.role("warp0", warp0())
     m.role("warp10", warp10())
-    m.role("issuer", issuer())
+    m.role("s_issuer", s_issuer())
+    m.role("dp_issuer", dp_issuer())
+    m.role("dq_issuer", dq_issuer())
     for w in range(2, 10):
         m.role(f"ds{w}", ds_warp(w))
 
@@ -471,7 +488,8 @@ def test_bwd_dkdv_protocol(items):
 
 
 @pytest.mark.parametrize("mistake", ["K producer skips k_empty", "issuer skips ds_full", "no pair barrier",
-                                     "no final dq_done wait"])
+                                     "no final dq_done wait", "S issuer skips dq_done", "dP issuer skips ds_full",
+                                     "k_empty waits for one issuer"])
 def test_bwd_dq_planted_mistakes_are_caught(mistake):
     assert _caught(bwd_dq_model, range(300), 7, mistake=mistake), mistake
 

@@ -17,7 +17,8 @@
 // S and dP are double-buffered, so the products of step p + 1 run while the warps form dS of step p.  No
 // online softmax is needed: the forward's lse normalises every step directly.
 // Warp roles: warp 0 loads Q and dO once and K per step, warp 10 loads V per step (TMA, one lane each, 3-deep
-// rings), warp 1 (one thread) issues the MMAs, warps 2-9 form dS and write dq.  Every wait is bounded: after
+// rings), warps 1, 11 and 12 (one thread each) issue the S, dP and dQ MMAs (one thread issues a tcgen05.mma
+// every ~107 cycles; three keep the tensor pipe fed), warps 2-9 form dS and write dq.  Every wait is bounded: after
 // the limit the CTA records an error (g_bwd_tc_error), skips the rest of its work, frees its TMEM and exits.
 #include "common.cuh"
 #include "internal.h"
@@ -32,7 +33,7 @@ namespace {
 constexpr int kTok = 8;         // tokens per tile
 constexpr int kG = 16;          // heads per KV group
 constexpr int kD = 128;         // head dim
-constexpr int kThreads = 352;   // 11 warps
+constexpr int kThreads = 416;   // 13 warps
 constexpr int kMaxBlk = 4096;   // context blocks (256K keys)
 constexpr int kWords = kMaxBlk / 32;
 constexpr int kRing = 3;
@@ -151,12 +152,12 @@ bwd_dq_tc_kernel(QueryRows qr, const __grid_constant__ CUtensorMap tm_q, const _
         tc::mbar_init(&bars.qd_tmem, 128);
         for (int i = 0; i < kRing; ++i) {
             tc::mbar_init(&bars.k_full[i], 1);
-            tc::mbar_init(&bars.k_empty[i], 1);
+            tc::mbar_init(&bars.k_empty[i], 2);  // K(p) is read by S(p) and dQ(p): one commit from each issuer
             tc::mbar_init(&bars.v_full[i], 1);
             tc::mbar_init(&bars.v_empty[i], 1);
         }
         for (int i = 0; i < 2; ++i) {
-            tc::mbar_init(&bars.s_full[i], 1);
+            tc::mbar_init(&bars.s_full[i], 2);  // S(p) and dP(p) both landed: one commit from each issuer
             tc::mbar_init(&bars.ds_full[i], 256);
             tc::mbar_init(&bars.dq_done[i], 1);
         }
@@ -209,48 +210,51 @@ bwd_dq_tc_kernel(QueryRows qr, const __grid_constant__ CUtensorMap tm_q, const _
                 tc::tma_load_3d(st + 8192, &tm_v, 64, g, z, &bars.v_full[s]);
             }
         }
-    } else if (warp == 1) {
-        // ---------------- MMA issuer ----------------
+    } else if (warp == 1 || warp == 11) {
+        // ---------------- S issuer (warp 1) and dP issuer (warp 11) ----------------
+        // S(p) and dP(p) go to buffers p & 1.  S(p) overwrites dS(p - 2), so it waits until dQ(p - 2) has
+        // completed; dP(p) overwrites dP(p - 2), which the dS warps loaded before they signalled dS(p - 2)
+        const bool is_s = warp == 1;
         if (lane == 0 && wait_bar(&bars.qd_tmem, 0, err)) {
             tc::tc_fence_after();
             constexpr uint32_t idesc_s = tc::idesc_bf16(128, kBlock, false);
-            constexpr uint32_t idesc_q = tc::idesc_bf16(128, kD, true);
-            for (int p = 0; p <= U; ++p) {
-                if (p < U) {
-                    // S(p) = Q . K^T and dP(p) = dO . V^T into buffers p & 1 (in order after dQ(p - 2), which
-                    // read dS(p - 2) from S buffer p & 1; the warps loaded dP(p - 2) before dS(p - 2) was ready)
-                    const int s = p % kRing, sb = p & 1;
-                    if (!wait_bar(&bars.k_full[s], (p / kRing) & 1, err)) break;
-                    if (!wait_bar(&bars.v_full[s], (p / kRing) & 1, err)) break;
-                    tc::tc_fence_after();
-                    const uint32_t kb = sK + s * kSlot, vb = sV + s * kSlot;
+            for (int p = 0; p < U; ++p) {
+                const int s = p % kRing, sb = p & 1;
+                if (p >= 2 && !wait_bar(is_s ? &bars.dq_done[sb] : &bars.ds_full[sb], ((p - 2) >> 1) & 1, err))
+                    break;
+                if (!wait_bar(is_s ? &bars.k_full[s] : &bars.v_full[s], (p / kRing) & 1, err)) break;
+                tc::tc_fence_after();
+                const uint32_t ob = (is_s ? sK : sV) + s * kSlot;
+                const uint32_t d_t = tmem + (is_s ? kColS : kColDP) + kBlock * sb;
+                const uint32_t a_t = tmem + (is_s ? kColQ : kColDO);
 #pragma unroll
-                    for (int ks = 0; ks < kD / 16; ++ks) {
-                        const uint32_t off = (ks >> 2) * 8192 + (ks & 3) * 32;
-                        tc::mma_bf16_ts(tmem + kColS + kBlock * sb, tmem + kColQ + 8 * ks,
-                                        tc::desc_kmajor_sw128(kb + off), idesc_s, ks > 0);
-                        tc::mma_bf16_ts(tmem + kColDP + kBlock * sb, tmem + kColDO + 8 * ks,
-                                        tc::desc_kmajor_sw128(vb + off), idesc_s, ks > 0);
-                    }
-                    tc::mma_commit(&bars.s_full[sb]);
-                    tc::mma_commit(&bars.v_empty[s]);
+                for (int ks = 0; ks < kD / 16; ++ks) {
+                    const uint32_t off = (ks >> 2) * 8192 + (ks & 3) * 32;
+                    tc::mma_bf16_ts(d_t, a_t + 8 * ks, tc::desc_kmajor_sw128(ob + off), idesc_s, ks > 0);
                 }
-                if (p >= 1) {
-                    // dQ += dS(v) . K(v), dS(v) in the first 32 columns of S buffer v & 1
-                    const int v = p - 1, db = v & 1, s = v % kRing;
-                    if (!wait_bar(&bars.ds_full[db], (v >> 1) & 1, err)) break;
-                    tc::tc_fence_after();
-                    const uint32_t kb = sK + s * kSlot;
-#pragma unroll
-                    for (int ks = 0; ks < kBlock / 16; ++ks)
-                        tc::mma_bf16_ts(tmem, tmem + kColS + kBlock * db + 8 * ks,
-                                        tc::desc_mnmajor_sw128(kb + ks * 2048, 8192), idesc_q, (v > 0 || ks > 0));
-                    tc::mma_commit(&bars.dq_done[db]);
-                    tc::mma_commit(&bars.k_empty[s]);
-                }
+                tc::mma_commit(&bars.s_full[sb]);
+                tc::mma_commit(is_s ? &bars.k_empty[s] : &bars.v_empty[s]);
             }
         }
-    } else {
+    } else if (warp == 12) {
+        // ---------------- dQ issuer: dQ += dS(v) . K(v), dS(v) in the first 32 columns of S buffer v & 1 ----------
+        if (lane == 0) {
+            constexpr uint32_t idesc_q = tc::idesc_bf16(128, kD, true);
+            for (int v = 0; v < U; ++v) {
+                const int db = v & 1, s = v % kRing;
+                if (!wait_bar(&bars.ds_full[db], (v >> 1) & 1, err)) break;
+                if (!wait_bar(&bars.k_full[s], (v / kRing) & 1, err)) break;  // landed before S(v): no wait
+                tc::tc_fence_after();
+                const uint32_t kb = sK + s * kSlot;
+#pragma unroll
+                for (int ks = 0; ks < kBlock / 16; ++ks)
+                    tc::mma_bf16_ts(tmem, tmem + kColS + kBlock * db + 8 * ks,
+                                    tc::desc_mnmajor_sw128(kb + ks * 2048, 8192), idesc_q, (v > 0 || ks > 0));
+                tc::mma_commit(&bars.dq_done[db]);
+                tc::mma_commit(&bars.k_empty[s]);
+            }
+        }
+    } else if (warp >= 2 && warp <= 9) {
         // ---------------- dS and dq: one TMEM lane (query row) per thread, 32 keys of each step ----------------
         // warps w and w + 4 (2 <= w <= 5) share the lane quarter w & 3: half 0 takes keys 0..31 of the block,
         // half 1 keys 32..63; they meet at a named barrier of their own on every step before dS overwrites S
