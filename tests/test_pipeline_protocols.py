@@ -384,8 +384,9 @@ def bwd_dq_model(m: PipelineModel, U: int, mistake: str = ""):
 # --------------------------------------------------------------------------------------------------------------
 # bwd_dkdv_tc_kernel (csrc/attn_bwd_tc.cu): work items (one 64-key block and up to 256 of its listed tokens),
 # each in 8-token tiles.  Warp 0: the item's K and V, then per tile the token ids (shared memory) and the Q / dO
-# rows (TMA, 2 buffers); warp 1: S, dP per tile into buffers tile & 1 (one tile ahead), then dV^T += dO^T P and
-# dK^T += Q^T dS; warps 2-5: P and dS into shared-memory tiles (one row per thread), and after each item the
+# rows (TMA, 2 buffers); warp 1: S, dP per tile into buffers tile & 1; warp 6: dV^T += dO^T P and dK^T += Q^T dS
+# (the two issuers' ops unordered relative to each other; a Q / dO buffer is freed by both issuers' commits, K / V
+# by warp 1's); warps 2-5: P and dS into shared-memory tiles (one row per thread), and after each item the
 # flush of dV^T / dK^T from TMEM.
 # --------------------------------------------------------------------------------------------------------------
 def bwd_dkdv_model(m: PipelineModel, items, mistake: str = ""):
@@ -393,7 +394,7 @@ def bwd_dkdv_model(m: PipelineModel, items, mistake: str = ""):
     m.bar("kv_free", 1)
     for i in range(2):
         m.bar(f"qd_full{i}", 1)
-        m.bar(f"qd_free{i}", 1)
+        m.bar(f"qd_free{i}", 1 if mistake == "qd_free waits for one issuer" else 2)
         m.bar(f"s_full{i}", 1)
     m.bar("pd_full", 128)
     m.bar("pd_free", 1)
@@ -417,28 +418,31 @@ def bwd_dkdv_model(m: PipelineModel, items, mistake: str = ""):
                 yield ("tma", f"qd_full{qb}", 1, [(f"QdO{qb}", ("QdO", n_tile))])
                 n_tile += 1
 
-    def issuer():
+    def s_issuer():
         n_tile = 0
-
-        def issue_s(ctr, n_item):
-            b = ctr & 1
-            yield ("mma", [(f"QdO{b}", ("QdO", ctr)), ("KV", ("KV", n_item))],
-                   [(f"S{b}.q{q}", ("S", ctr)) for q in Q4] + [(f"DP{b}.q{q}", ("DP", ctr)) for q in Q4], f"S{ctr}")
-            yield ("commit", f"s_full{b}")
-
         for n_item, ntiles in enumerate(items):
             yield ("wait", "kv_full", n_item)
+            for i in range(ntiles):
+                ctr = n_tile + i
+                b = ctr & 1
+                # S buffer b held S(ctr - 2): QdO(ctr) is loaded only after both issuers freed buffer b for
+                # tile ctr - 2, and dVdK(ctr - 2) ran on P(ctr - 2), written after the warps read S(ctr - 2)
+                yield ("wait", f"qd_full{b}", ctr >> 1)
+                yield ("mma", [(f"QdO{b}", ("QdO", ctr)), ("KV", ("KV", n_item))],
+                       [(f"S{b}.q{q}", ("S", ctr)) for q in Q4] + [(f"DP{b}.q{q}", ("DP", ctr)) for q in Q4], f"S{ctr}")
+                yield ("commit", f"s_full{b}")
+                yield ("commit", f"qd_free{b}")
+            n_tile += ntiles
+            yield ("commit", "kv_free")
+
+    def acc_issuer():
+        n_tile = 0
+        for n_item, ntiles in enumerate(items):
             if n_item >= 1 and mistake != "issuer skips acc_free":
                 yield ("wait", "acc_free", n_item - 1)
-            tile0 = n_tile
-            if ntiles > 0:
-                yield ("wait", f"qd_full{tile0 & 1}", tile0 >> 1)
-                yield from issue_s(tile0, n_item)
             for i in range(ntiles):
-                ctr = tile0 + i
-                if i + 1 < ntiles:
-                    yield ("wait", f"qd_full{(ctr + 1) & 1}", (ctr + 1) >> 1)
-                    yield from issue_s(ctr + 1, n_item)
+                ctr = n_tile + i
+                yield ("wait", f"qd_full{ctr & 1}", ctr >> 1)
                 yield ("wait", "pd_full", ctr)
                 reads = [(f"QdO{ctr & 1}", ("QdO", ctr))] + [(f"P.q{q}", ("P", ctr)) for q in Q4]
                 if i > 0:
@@ -447,7 +451,6 @@ def bwd_dkdv_model(m: PipelineModel, items, mistake: str = ""):
                 yield ("commit", "pd_free")
                 yield ("commit", f"qd_free{ctr & 1}")
             n_tile += ntiles
-            yield ("commit", "kv_free")
             yield ("commit", "acc_done")
 
     def warps(q4):
@@ -472,7 +475,8 @@ def bwd_dkdv_model(m: PipelineModel, items, mistake: str = ""):
             yield ("arrive", "acc_free", 32)
 
     m.role("producer", producer())
-    m.role("issuer", issuer())
+    m.role("s_issuer", s_issuer())
+    m.role("acc_issuer", acc_issuer())
     for q4 in Q4:
         m.role(f"warp{2 + q4}", warps(q4))
 
@@ -495,7 +499,7 @@ def test_bwd_dq_planted_mistakes_are_caught(mistake):
 
 
 @pytest.mark.parametrize("mistake", ["producer skips kv_free", "producer skips qd_free", "issuer skips acc_free",
-                                     "warps skip pd_free", "warps skip acc_done"])
+                                     "warps skip pd_free", "warps skip acc_done", "qd_free waits for one issuer"])
 def test_bwd_dkdv_planted_mistakes_are_caught(mistake):
     # acc_free matters only where empty items let the issuer commit acc_done twice without a P tile between
     assert _caught(bwd_dkdv_model, range(300), [3, 0, 0, 2, 4], mistake=mistake), mistake

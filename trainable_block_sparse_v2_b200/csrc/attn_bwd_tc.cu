@@ -402,11 +402,13 @@ cudaError_t launch_bwd_dq_tc(const QueryRows& qr, const void* k, const void* v, 
 //   P, dS                      rows in TMEM -> bf16 tiles in smem (four warps, one row per thread)
 //   dV^T [128 dims x 64 keys] += dO^T . P           A (dO) MN-major, B (P) MN-major, in TMEM
 //   dK^T [128 dims x 64 keys] += Q^T . dS           the same with Q and dS
-// S and dP are double-buffered, so tile i + 1's products run while the warps form tile i's P and dS.  A
-// work item's sums go to dk / dv by fp32 atomics (one TMEM lane = one head dimension per thread).
+// S and dP are double-buffered, so tile i + 1's products run while the warps form tile i's P and dS.  Warp 1
+// issues S and dP, warp 6 the dV / dK sums (one thread issues a tcgen05.mma every ~107 cycles; two keep the
+// tensor pipe busier).  A work item's sums go to dk / dv by fp32 atomics (one TMEM lane = one head dimension
+// per thread).
 namespace {
 
-constexpr int kKvThreads = 192;   // warp 0 TMA, warp 1 MMA, warps 2-5 P / dS and the flush
+constexpr int kKvThreads = 224;   // warp 0 TMA, warps 1 and 6 MMA, warps 2-5 P / dS and the flush
 constexpr int kKvItemTokens = 256;  // tokens per work item (the list builder's chunk)
 constexpr int kKvTile = 16384;    // one 64-key block of K or V
 constexpr int kKvQd = 32768;      // one 8-token tile of Q or dO: two d-halves x 128 rows x 128 B
@@ -452,7 +454,7 @@ bwd_dkdv_tc_kernel(QueryRows qr, const __grid_constant__ CUtensorMap tm_q1, cons
         tc::mbar_init(&bars.kv_free, 1);
         for (int i = 0; i < 2; ++i) {
             tc::mbar_init(&bars.qd_full[i], 1);
-            tc::mbar_init(&bars.qd_free[i], 1);
+            tc::mbar_init(&bars.qd_free[i], 2);  // Q / dO are read by both issuers' products
             tc::mbar_init(&bars.s_full[i], 1);
         }
         tc::mbar_init(&bars.pd_full, 128);
@@ -524,48 +526,56 @@ bwd_dkdv_tc_kernel(QueryRows qr, const __grid_constant__ CUtensorMap tm_q1, cons
             }
         }
     } else if (warp == 1) {
-        // ---------------- MMA issuer ----------------
+        // ---------------- S / dP issuer ----------------
+        // S, dP of tile ctr into buffers ctr & 1.  That buffer held tile ctr - 2, whose reads are ordered before
+        // this product: Q / dO of tile ctr land only after both issuers freed the buffer for tile ctr - 2, and
+        // warp 6 freed it after dV / dK of P(ctr - 2), which the warps wrote after reading S(ctr - 2)
         if (lane == 0) {
             constexpr uint32_t idesc_s = tc::idesc_bf16_ab(128, kBlock, false, false);
-            constexpr uint32_t idesc_t = tc::idesc_bf16_ab(128, kBlock, true, true);
             int n_item = 0, n_tile = 0;
             bool ok = true;
-            auto issue_s = [&](int tile_ctr) {  // S, dP of the tile with global counter tile_ctr
-                const int qb = tile_ctr & 1, sb = tile_ctr & 1;
-                const uint32_t qa = sbase + kKvQOff + qb * 2 * kKvQd, da = qa + kKvQd;
-#pragma unroll
-                for (int ks = 0; ks < kD / 16; ++ks) {
-                    const uint32_t off = (ks >> 2) * 16384 + (ks & 3) * 32;
-                    const uint32_t boff = (ks >> 2) * 8192 + (ks & 3) * 32;
-                    tc::mma_bf16_ss(tmem + kKvColS + kBlock * sb, tc::desc_kmajor_sw128(qa + off),
-                                    tc::desc_kmajor_sw128(sbase + kKvKOff + boff), idesc_s, ks > 0);
-                    tc::mma_bf16_ss(tmem + kKvColDP + kBlock * sb, tc::desc_kmajor_sw128(da + off),
-                                    tc::desc_kmajor_sw128(sbase + kKvVOff + boff), idesc_s, ks > 0);
-                }
-                tc::mma_commit(&bars.s_full[sb]);
-            };
             for (int item = blockIdx.x; item < n_items && ok; item += gridDim.x, ++n_item) {
                 const int l = item_list[item], start = item_start[item];
                 const int ntok = min(min(kKvItemTokens, counts[l] - start), cap - offsets[l] - start);
                 const int ntiles = ntok > 0 ? (ntok + kTok - 1) / kTok : 0;
                 if (!(ok = wait_bar(&bars.kv_full, n_item & 1, err))) break;
+                for (int i = 0; i < ntiles; ++i) {
+                    const int ctr = n_tile + i, sb = ctr & 1;
+                    if (!(ok = wait_bar(&bars.qd_full[sb], (ctr >> 1) & 1, err))) break;
+                    tc::tc_fence_after();
+                    const uint32_t qa = sbase + kKvQOff + sb * 2 * kKvQd, da = qa + kKvQd;
+#pragma unroll
+                    for (int ks = 0; ks < kD / 16; ++ks) {
+                        const uint32_t off = (ks >> 2) * 16384 + (ks & 3) * 32;
+                        const uint32_t boff = (ks >> 2) * 8192 + (ks & 3) * 32;
+                        tc::mma_bf16_ss(tmem + kKvColS + kBlock * sb, tc::desc_kmajor_sw128(qa + off),
+                                        tc::desc_kmajor_sw128(sbase + kKvKOff + boff), idesc_s, ks > 0);
+                        tc::mma_bf16_ss(tmem + kKvColDP + kBlock * sb, tc::desc_kmajor_sw128(da + off),
+                                        tc::desc_kmajor_sw128(sbase + kKvVOff + boff), idesc_s, ks > 0);
+                    }
+                    tc::mma_commit(&bars.s_full[sb]);
+                    tc::mma_commit(&bars.qd_free[sb]);
+                }
+                if (!ok) break;
+                n_tile += ntiles;
+                tc::mma_commit(&bars.kv_free);  // only S and dP read the item's K and V
+            }
+        }
+    } else if (warp == 6) {
+        // ---------------- dV / dK issuer: dV^T += dO^T P, dK^T += Q^T dS per tile ----------------
+        if (lane == 0) {
+            constexpr uint32_t idesc_t = tc::idesc_bf16_ab(128, kBlock, true, true);
+            int n_item = 0, n_tile = 0;
+            bool ok = true;
+            for (int item = blockIdx.x; item < n_items && ok; item += gridDim.x, ++n_item) {
+                const int l = item_list[item], start = item_start[item];
+                const int ntok = min(min(kKvItemTokens, counts[l] - start), cap - offsets[l] - start);
+                const int ntiles = ntok > 0 ? (ntok + kTok - 1) / kTok : 0;
                 // the flush of the previous item's sums must be done before this item's first accumulation
                 if (n_item >= 1 && !(ok = wait_bar(&bars.acc_free, (n_item - 1) & 1, err))) break;
-                tc::tc_fence_after();
-                const int tile0 = n_tile;
-                if (ntiles > 0) {
-                    if (!(ok = wait_bar(&bars.qd_full[tile0 & 1], (tile0 >> 1) & 1, err))) break;
-                    tc::tc_fence_after();
-                    issue_s(tile0);
-                }
                 for (int i = 0; i < ntiles; ++i) {
-                    const int ctr = tile0 + i;
-                    if (i + 1 < ntiles) {
-                        // tile i + 1's products into the other S / dP buffers, read back by the warps for tile i - 1
-                        if (!(ok = wait_bar(&bars.qd_full[(ctr + 1) & 1], ((ctr + 1) >> 1) & 1, err))) break;
-                        tc::tc_fence_after();
-                        issue_s(ctr + 1);
-                    }
+                    const int ctr = n_tile + i;
+                    if (!(ok = wait_bar(&bars.qd_full[ctr & 1], (ctr >> 1) & 1, err))) break;
                     if (!(ok = wait_bar(&bars.pd_full, ctr & 1, err))) break;
                     tc::tc_fence_after();
                     const uint32_t qa = sbase + kKvQOff + (ctr & 1) * 2 * kKvQd, da = qa + kKvQd;
@@ -583,11 +593,10 @@ bwd_dkdv_tc_kernel(QueryRows qr, const __grid_constant__ CUtensorMap tm_q1, cons
                 }
                 if (!ok) break;
                 n_tile += ntiles;
-                tc::mma_commit(&bars.kv_free);
                 tc::mma_commit(&bars.acc_done);
             }
         }
-    } else {
+    } else if (warp >= 2 && warp <= 5) {
         // ---------------- P, dS (one query row per thread) and the flush (one head dimension per thread) ----------
         const int q4 = warp & 3;
         const int r = q4 * 32 + lane;  // tile row = token slot * 16 + head; in the flush: head dimension
