@@ -48,8 +48,9 @@ NCU_TRAFFIC = {
     "block_score_topk": None,                           # score_scan_kernel + score_select_kernel
     "sparse_attn_prefill": 322_111_488 + 229_101_312,   # attn_tc_kernel<16, 128>
 }
-KERNELS_PER_STEP = {"two_call": 5,  # kernel pool, score scan, select, split attention, merge
-                    "fused": 2}     # kernel pool, fused decode step (scoring + top-k + attention)
+KERNELS_PER_STEP = {"two_call": 5,    # kernel pool, score scan, select, split attention, merge
+                    "fused": 2,       # kernel pool, fused decode step (scoring + top-k + attention)
+                    "fused_pool": 1}  # the fused decode step pooling the new key's kernel itself
 
 
 def load_peaks():
@@ -134,7 +135,7 @@ def decode_step_bytes(lens, kmax=67):
 
 
 class DecodeBench:
-    def __init__(self, layers=8, steps_cycle=256, two_call=False):
+    def __init__(self, layers=8, steps_cycle=256, two_call=False, pooled=False):
         import torch
         from trainable_block_sparse_v2_b200 import binding
         from trainable_block_sparse_v2_b200.workloads import decode_128k_ragged
@@ -142,6 +143,7 @@ class DecodeBench:
         self.torch, self.b = torch, binding
         self.NL, self.S = layers, steps_cycle
         self.two_call = two_call
+        self.pooled = pooled and not two_call
         w = decode_128k_ragged(steps=steps_cycle)
         self.w = w
         self.p = binding.Params(**w.params)
@@ -199,14 +201,38 @@ class DecodeBench:
                                            self.lens[pos], self.max_ctx, self.p, self.idx, self.cnt, self.out, None,
                                            stream)
 
+    def fused_pool(self, layer, pos, stream=None):
+        self.b.infllmv2_sparse_decode_step_pool(self.q_of(layer, pos), self.kern[layer], self.k[layer], self.v[layer],
+                                                self.lens[pos], self.max_ctx, self.p, self.idx, self.cnt, self.out,
+                                                None, stream)
+
     def step_eager(self, s, stream=None):
         layer, pos = self._coords(s)
+        if self.pooled:
+            self.fused_pool(layer, pos, stream)
+            return
         self.pool(layer, pos, stream)
         if self.two_call:
             self.score(layer, pos, stream)
             self.attend(layer, pos, stream)
         else:
             self.fused(layer, pos, stream)
+
+    def decode_calls(self, q, layer, pos, out):
+        """the step's C-ABI calls after the new rows are in the caches, for a query and output of the caller's"""
+        if self.pooled:
+            self.b.infllmv2_sparse_decode_step_pool(q, self.kern[layer], self.k[layer], self.v[layer], self.lens[pos],
+                                                    self.max_ctx, self.p, self.idx, self.cnt, out, None)
+            return
+        self.b.infllmv2_kernel_pool(self.k[layer], self.old[pos], self.lens[pos], 1, self.p, self.kern[layer])
+        if self.two_call:
+            self.b.infllmv2_block_score_topk(q, None, self.lens[pos], self.max_ctx, self.kern[layer], self.p,
+                                             self.idx, self.cnt, self.ws)
+            self.b.infllmv2_sparse_attn_decode(q, self.k[layer], self.v[layer], self.lens[pos], self.max_ctx,
+                                               self.idx, self.cnt, self.p, out, None, self.ws)
+        else:
+            self.b.infllmv2_sparse_decode_step(q, self.kern[layer], self.k[layer], self.v[layer], self.lens[pos],
+                                               self.max_ctx, self.p, self.idx, self.cnt, out, None)
 
     def _capture(self, key, steps):
         """one CUDA graph of the given consecutive steps (warmed outside capture first)"""
@@ -269,8 +295,8 @@ class DecodeBench:
         and position) captured in one CUDA graph, replayed between two CUDA events on the current stream, so
         that neither host launch overhead nor the graph prologue is counted"""
         torch = self.torch
-        names = ["kernel_pool", "block_score_topk", "sparse_attn_decode", "sparse_decode_step"]
-        fns = [self.pool, self.score, self.attend, self.fused]
+        names = ["kernel_pool", "block_score_topk", "sparse_attn_decode", "sparse_decode_step", "sparse_decode_step_pool"]
+        fns = [self.pool, self.score, self.attend, self.fused, self.fused_pool]
         for s in range(warmup):
             self.step_eager(s)
         torch.cuda.synchronize()
@@ -365,16 +391,7 @@ class DecodeBench:
             layer, pos = self._coords(s)
             stage.copy_(host[pos], non_blocking=True)
             self.b.infllmv2_kv_append(k_new, v_new, self.old[pos], self.k[layer], self.v[layer])
-            self.b.infllmv2_kernel_pool(self.k[layer], self.old[pos], self.lens[pos], 1, self.p, self.kern[layer])
-            if self.two_call:
-                self.b.infllmv2_block_score_topk(q_dev, None, self.lens[pos], self.max_ctx, self.kern[layer], self.p,
-                                                 self.idx, self.cnt, self.ws)
-                self.b.infllmv2_sparse_attn_decode(q_dev, self.k[layer], self.v[layer], self.lens[pos], self.max_ctx,
-                                                   self.idx, self.cnt, self.p, self.out, None, self.ws)
-            else:
-                self.b.infllmv2_sparse_decode_step(q_dev, self.kern[layer], self.k[layer], self.v[layer],
-                                                   self.lens[pos], self.max_ctx, self.p, self.idx, self.cnt, self.out,
-                                                   None)
+            self.decode_calls(q_dev, layer, pos, self.out)
             out_host.copy_(self.out, non_blocking=True)
 
         # double-buffered staging for the overlapped form: step i's input copy and step i-1's read-back run on a
@@ -389,16 +406,7 @@ class DecodeBench:
             q2 = st[:nq].view(B, 1, HQ, D)
             kn, vn = st[nq:nq + nkv].view(B, HKV, D), st[nq + nkv:].view(B, HKV, D)
             self.b.infllmv2_kv_append(kn, vn, self.old[pos], self.k[layer], self.v[layer])
-            self.b.infllmv2_kernel_pool(self.k[layer], self.old[pos], self.lens[pos], 1, self.p, self.kern[layer])
-            if self.two_call:
-                self.b.infllmv2_block_score_topk(q2, None, self.lens[pos], self.max_ctx, self.kern[layer], self.p,
-                                                 self.idx, self.cnt, self.ws)
-                self.b.infllmv2_sparse_attn_decode(q2, self.k[layer], self.v[layer], self.lens[pos], self.max_ctx,
-                                                   self.idx, self.cnt, self.p, out2[buf], None, self.ws)
-            else:
-                self.b.infllmv2_sparse_decode_step(q2, self.kern[layer], self.k[layer], self.v[layer],
-                                                   self.lens[pos], self.max_ctx, self.p, self.idx, self.cnt,
-                                                   out2[buf], None)
+            self.decode_calls(q2, layer, pos, out2[buf])
 
         def overlapped(s0):
             """the NL steps of one position (captured): copies on copy_stream, kernels on the capture stream"""
@@ -504,16 +512,7 @@ class DecodeBench:
                 q2 = st[:nq].view(B, 1, HQ, D)
                 kn, vn = st[nq:nq + nkv].view(B, HKV, D), st[nq + nkv:].view(B, HKV, D)
                 self.b.infllmv2_kv_append(kn, vn, self.old[pos], self.k[layer], self.v[layer])
-                self.b.infllmv2_kernel_pool(self.k[layer], self.old[pos], self.lens[pos], 1, self.p, self.kern[layer])
-                if self.two_call:
-                    self.b.infllmv2_block_score_topk(q2, None, self.lens[pos], self.max_ctx, self.kern[layer], self.p,
-                                                     self.idx, self.cnt, self.ws)
-                    self.b.infllmv2_sparse_attn_decode(q2, self.k[layer], self.v[layer], self.lens[pos], self.max_ctx,
-                                                       self.idx, self.cnt, self.p, out[i], None, self.ws)
-                else:
-                    self.b.infllmv2_sparse_decode_step(q2, self.kern[layer], self.k[layer], self.v[layer],
-                                                       self.lens[pos], self.max_ctx, self.p, self.idx, self.cnt,
-                                                       out[i], None)
+                self.decode_calls(q2, layer, pos, out[i])
             out_host.copy_(out, non_blocking=True)
 
         lo = (warmup + NL - 1) // NL * NL
@@ -736,8 +735,8 @@ def kernel_pool_backward_leg(peaks, peak_kind, reps=20):
 
 
 class Decode32kBench:
-    """Decode at a 32K context, batch 1 (32 / 2 heads, d 128, top-k 64): one step = the kernel pool of the new
-    key + the fused decode step (scoring, top-k, attention), on a cache restored every step (the pool of the
+    """Decode at a 32K context, batch 1 (32 / 2 heads, d 128, top-k 64): one step = the fused decode step that
+    pools the new key's kernel, scores, selects and attends in one launch, on a cache restored every step (the pool of the
     step's window rewrites the same kernel).  Its working set (~5.4 MB) fits in L2, so L2 is flushed before
     every timed step; the time is the median of the steps."""
 
@@ -763,9 +762,8 @@ class Decode32kBench:
         self.l2_flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
 
     def step(self):
-        self.b.infllmv2_kernel_pool(self.k, self.old, self.lens, 1, self.p, self.kern)
-        self.b.infllmv2_sparse_decode_step(self.q, self.kern, self.k, self.v, self.lens, self.L, self.p, self.idx,
-                                           self.cnt, self.out, None)
+        self.b.infllmv2_sparse_decode_step_pool(self.q, self.kern, self.k, self.v, self.lens, self.L, self.p, self.idx,
+                                                self.cnt, self.out, None)
 
     def run(self, warmup, steps):
         """median seconds per step, each step timed alone after an L2 flush"""
@@ -1117,7 +1115,8 @@ def run_ours(args):
 
     if not args.no_decode:
         two_call = args.decode_path == "two_call"
-        db = DecodeBench(layers=args.layers, two_call=two_call)
+        pooled = args.decode_path == "fused_pool"
+        db = DecodeBench(layers=args.layers, two_call=two_call, pooled=pooled)
         # timed region: exactly K decode steps (graph replays), barrier + synchronize on both sides
         barrier(ws)
         with ClockSampler(torch.cuda.current_device()) as clk:
@@ -1128,7 +1127,7 @@ def run_ours(args):
 
         per = db.per_call_times(8, min(args.steps, 256)) if args.per_call else {
             "kernel_pool": float("nan"), "block_score_topk": float("nan"), "sparse_attn_decode": float("nan"),
-            "sparse_decode_step": float("nan")}
+            "sparse_decode_step": float("nan"), "sparse_decode_step_pool": float("nan")}
         lens_mid = [n + 128 for n in LENS_128K]
         scan_b, kv_b, step_b = decode_step_bytes(lens_mid)
         if two_call:
@@ -1136,8 +1135,9 @@ def run_ours(args):
             dom = max(("block_score_topk", "sparse_attn_decode"), key=lambda k: per[k] if per[k] == per[k] else -1.0)
             dom_bytes = {"block_score_topk": scan_b, "sparse_attn_decode": kv_b}[dom]
         else:
-            # the fused scoring + top-k + attention launch carries the whole step's traffic
-            dom = "sparse_decode_step"
+            # the fused scoring + top-k + attention launch carries the whole step's traffic (with pooling: plus the
+            # new key's 32-key window once per 16 steps, ~4 KB per sequence and step on average, not counted)
+            dom = "sparse_decode_step_pool" if pooled else "sparse_decode_step"
             dom_bytes = scan_b + kv_b
         achieved = dom_bytes / per[dom] / 1e9
         # the draft model's sliding-window attention on the same caches (next-row measurement)
@@ -1170,6 +1170,9 @@ def run_ours(args):
                              "before its layer returns",
                        "step": ("one decode step of one layer for 4 sequences: kernel_pool + block_score_topk + "
                                 "sparse_attn_decode, replayed as a CUDA graph" if two_call else
+                                "one decode step of one layer for 4 sequences: sparse_decode_step_pool (the new key's "
+                                "kernel pooled, scoring, top-k and sparse attention in one cluster kernel), replayed "
+                                "as a CUDA graph" if pooled else
                                 "one decode step of one layer for 4 sequences: kernel_pool + sparse_decode_step "
                                 "(scoring, top-k and sparse attention in one cluster kernel), replayed as a CUDA graph")},
             "hbm": {"algorithmic_bytes_per_step": step_b, "achieved_gbs_per_gpu": step_b / (t / args.steps) / 1e9,
@@ -1268,7 +1271,7 @@ def run_ours(args):
                 "steps": 1000, "timing": "median of 1000 steps, L2 flushed before each",
                 "algorithmic_bytes": b32, "achieved_gbs": b32 / t32 / 1e9,
                 "frac_of_" + peak_kind: b32 / t32 / 1e9 / peaks["hbm_gbs"],
-                "note": "one step = kernel_pool of the new key + sparse_decode_step, batch 1",
+                "note": "one step = sparse_decode_step_pool (the new key's kernel pooled in the same launch), batch 1",
             }
         else:
             line["decode_32k"] = {"workload": "decode_32k", "error": err or "no time"}
@@ -1404,8 +1407,9 @@ def main():
     ap.add_argument("--warmup", type=int, default=64)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--layers", type=int, default=8)
-    ap.add_argument("--decode-path", choices=["two_call", "fused"], default="fused",
-                    help="decode step as block_score_topk + sparse_attn_decode, or the one-launch sparse_decode_step")
+    ap.add_argument("--decode-path", choices=["two_call", "fused", "fused_pool"], default="fused_pool",
+                    help="decode step as kernel_pool + block_score_topk + sparse_attn_decode, kernel_pool + "
+                         "sparse_decode_step, or the one-launch sparse_decode_step_pool")
     ap.add_argument("--prefill-steps", type=int, default=3)
     ap.add_argument("--no-prefill", action="store_true")
     ap.add_argument("--no-backward", action="store_true", help="skip the prefill gradient pass")

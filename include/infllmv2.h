@@ -238,6 +238,19 @@ int infllmv2_sparse_decode_step(const void* q, int batch, int hq, int hkv, int h
                                 infllmv2_stream_t stream);
 
 /*
+ * Steps 1 + 2 + 3b of one decode step in a single launch: infllmv2_kernel_pool of each sequence's last key
+ * (old = n - 1, new = n keys, n = ctx_lens[b]) followed by infllmv2_sparse_decode_step, with the same results
+ * (the kernel the last key completes, if it completes one, is written to kern bit for bit as the pooling call
+ * writes it).  The CTA that scans that kernel's block pools it, from the 32 keys of its window in k, and uses it
+ * in its scan.  Arguments as infllmv2_sparse_decode_step; kern is read and written, and must hold every kernel
+ * of the first n - 1 keys.  q [B, 1, Hq, d].
+ */
+int infllmv2_sparse_decode_step_pool(const void* q, int batch, int hq, int hkv, int head_dim, void* kern, int nk_cap,
+                                const void* k, const void* v, int lcap, const int32_t* ctx_lens, int max_ctx,
+                                const infllmv2_params* params, int32_t* idx, int32_t* cnt, void* out, float* lse,
+                                infllmv2_stream_t stream);
+
+/*
  * Paged key/value cache (serving; the pages give no cache layout -- the CPM.cu runtime of the QbitAI
  * article, section "CPM.cu", manages static device memory, and a pool of fixed-size pages is that idea for
  * many sequences of unknown length).  One page holds one context block, 64 positions, so a selected block

@@ -368,6 +368,45 @@ FUSED_LENS_14 = [20000, 8192, 8193, 30, 4500, 65, 70000]
 FUSED_LENS_26 = [20000, 8192, 8193, 30, 4500, 65, 70000, 9000, 12345, 64 * 130 + 1, 40000, 8300, 98304]
 
 
+# lengths whose last key completes a kernel window ((n - 32) % 16 == 0: 20000, 8192, 70000, 32, 48, 9008, 98304) and
+# lengths whose last key completes none
+POOL_LENS = FUSED_LENS_14 + [32, 48, 9008, 31, 98304]
+
+
+@pytest.mark.parametrize("G,d,lens", [(16, 128, POOL_LENS), (2, 64, POOL_LENS), (8, 128, FUSED_LENS_26)])
+def test_fused_decode_step_pool_equals_pool_then_step(oracle, G, d, lens):
+    """infllmv2_sparse_decode_step_pool against infllmv2_kernel_pool (old = n - 1, new = n) followed by
+    infllmv2_sparse_decode_step on the same cache: the kernel cache and idx, cnt, out, lse bit for bit; the pooled
+    cache also bit for bit against the oracle's pool over all n keys.  Dense and sparse rows, windows completed
+    by the last key or not, 16- and 8-CTA clusters."""
+    w = decode_case(lens, 2 * G, 2, d, topk=16, dense_len=8192, seed=670 + G + len(lens), n_needles=8)
+    B = len(lens)
+    nk_cap = oracle.num_kernels(max(lens))
+    p = bparams(w.params)
+    K, V, q = dev(w.k), dev(w.v), dev(w.q)
+    prev = [n - 1 for n in lens]
+    kern_a = gpu_pool(w.k, [0] * B, prev, max(prev), nk_cap)
+    kern_b = kern_a.clone()
+    L = dev_i32(lens)
+    binding.infllmv2_kernel_pool(K, dev_i32(prev), L, 1, p, kern_a)
+
+    def outputs():
+        return (torch.full((B, 1, 2, p.kmax), -7, dtype=torch.int32, device="cuda"),
+                torch.full((B, 1, 2), -7, dtype=torch.int32, device="cuda"),
+                torch.empty((B, 1, 2 * G, d), dtype=torch.bfloat16, device="cuda"),
+                torch.empty((B, 1, 2 * G), dtype=torch.float32, device="cuda"))
+    a, bb = outputs(), outputs()
+    binding.infllmv2_sparse_decode_step(q, kern_a, K, V, L, max(lens), p, *a)
+    binding.infllmv2_sparse_decode_step_pool(q, kern_b, K, V, L, max(lens), p, *bb)
+    torch.cuda.synchronize()
+    assert binding.infllmv2_device_status() == 0
+    assert torch.equal(kern_a, kern_b), "kernel cache"
+    for x, y, name in zip(a, bb, ("idx", "cnt", "out", "lse")):
+        assert torch.equal(x, y) or (x.dtype.is_floating_point and torch.equal(x.nan_to_num(), y.nan_to_num())), name
+    kern_o = oracle.kernel_pool(w.k, [0] * B, lens, 32, 16, nk_cap=nk_cap)
+    assert np.array_equal(host_u16(kern_b), kern_o)
+
+
 @pytest.mark.parametrize("G,d,lens,membership,topk", [(16, 128, FUSED_LENS_14, 0, 16), (2, 64, FUSED_LENS_14, 0, 16),
                                                       (8, 128, FUSED_LENS_14, 1, 16), (16, 128, FUSED_LENS_26, 0, 16),
                                                       (4, 64, FUSED_LENS_26, 1, 16), (16, 128, FUSED_LENS_14, 0, 1200)])

@@ -82,6 +82,7 @@ _SIGS = {
     "infllmv2_sparse_attn_decode": ([_P, _I, _I, _I, _I, _P, _P, _I, _P, _I, _P, _P, _PP, _P, _P, _P, _SZ, _P], _I),
     "infllmv2_sparse_attn_decode_noalloc": ([_P, _I, _I, _I, _I, _P, _P, _I, _P, _I, _P, _P, _PP, _P, _P, _P], _I),
     "infllmv2_sparse_decode_step": ([_P, _I, _I, _I, _I, _P, _I, _P, _P, _I, _P, _I, _PP, _P, _P, _P, _P, _P], _I),
+    "infllmv2_sparse_decode_step_pool": ([_P, _I, _I, _I, _I, _P, _I, _P, _P, _I, _P, _I, _PP, _P, _P, _P, _P, _P], _I),
     "infllmv2_sparse_attn_tree_verify": ([_P, _I, _I, _I, _I, _I, _P, _P, _I, _P, _I, _P, _P, _P, _P, _P, _PP, _P,
                                           _P, _P, _SZ, _P], _I),
     "infllmv2_dense_attn_prefill": ([_P, _I, _I, _I, _I, _I, _P, _P, _I, _P, _P, _I, _F, _P, _P, _P, _SZ, _P], _I),
@@ -365,6 +366,21 @@ def infllmv2_sparse_decode_step(q, kern, k, v, ctx_lens, max_ctx, params: Params
                                             _ptr(ctx_lens), int(max_ctx), ctypes.byref(cp), _ptr(idx), _ptr(cnt),
                                             _ptr(out), _ptr(lse), _stream(stream))
     _check("infllmv2_sparse_decode_step", st)
+
+
+def infllmv2_sparse_decode_step_pool(q, kern, k, v, ctx_lens, max_ctx, params: Params, idx, cnt, out, lse=None,
+                                     stream=None):
+    """The kernel pool of each sequence's last key, then scoring, top-k and sparse attention, in one launch
+    (infllmv2_kernel_pool of old = n - 1, new = n followed by infllmv2_sparse_decode_step)"""
+    B, Hq, d, Lcap, Hkv = _decode_args("infllmv2_sparse_decode_step_pool", q, k, v, ctx_lens, out, lse, idx, cnt,
+                                       params, kern=kern)
+    if _checking():
+        _check_rows("infllmv2_sparse_decode_step_pool", B, 1, None, ctx_lens, True, Lcap, max_ctx)
+    cp = params.c()
+    st = load().infllmv2_sparse_decode_step_pool(_ptr(q), B, Hq, Hkv, d, _ptr(kern), kern.shape[2], _ptr(k), _ptr(v),
+                                                 Lcap, _ptr(ctx_lens), int(max_ctx), ctypes.byref(cp), _ptr(idx),
+                                                 _ptr(cnt), _ptr(out), _ptr(lse), _stream(stream))
+    _check("infllmv2_sparse_decode_step_pool", st)
 
 
 def infllmv2_sparse_attn_decode_noalloc(q, k, v, ctx_lens, max_ctx, idx, cnt, params: Params, out, lse=None,

@@ -454,6 +454,33 @@ int infllmv2_sparse_decode_step(const void* q, int batch, int hq, int hkv, int h
                                              (cudaStream_t)stream));
 }
 
+int infllmv2_sparse_decode_step_pool(const void* q, int batch, int hq, int hkv, int head_dim, void* kern, int nk_cap,
+                                const void* k, const void* v, int lcap, const int32_t* ctx_lens, int max_ctx,
+                                const infllmv2_params* params, int32_t* idx, int32_t* cnt, void* out, float* lse,
+                                infllmv2_stream_t stream)
+{
+    IV2_TRY(check_params(params));
+    if (params->lse_stride > 1) return INFLLMV2_ERR_UNSUPPORTED;  // the estimate is built for prefill scoring only
+    IV2_TRY(check_heads(batch, 1, hq, hkv, head_dim));
+    IV2_TRY(check_ptr16(q));
+    IV2_TRY(check_ptr16(kern));
+    IV2_TRY(check_ptr16(k));
+    IV2_TRY(check_ptr16(v));
+    IV2_TRY(check_ptr16(out));
+    IV2_TRY(check_ptr4(ctx_lens));
+    IV2_TRY(check_ptr4(idx));
+    IV2_TRY(check_ptr4(cnt));
+    IV2_TRY(check_opt4(lse));
+    IV2_TRY(check_ctx(max_ctx, lcap));
+    if (nk_cap < 1 || nk_cap < nk_of(max_ctx)) return INFLLMV2_ERR_INVALID_ARG;
+    if (batch * hkv > 65535) return INFLLMV2_ERR_UNSUPPORTED;
+    const MethodConsts mc = consts_of(params, head_dim);
+    const QueryRows qr = rows_of(q, batch, 1, hq, hkv, head_dim, nullptr, ctx_lens, 0, max_ctx);
+    if (!iv2::decode_fused_supported(qr, mc)) return INFLLMV2_ERR_UNSUPPORTED;
+    return launched(iv2::launch_decode_fused(qr, kern, nk_cap, mc, k, v, iv2::kv_contiguous(batch, lcap), idx, cnt, out, lse,
+                                             (cudaStream_t)stream, true));
+}
+
 int infllmv2_sparse_attn_tree_verify(const void* q, int batch, int n_draft, int hq, int hkv, int head_dim,
                                      const void* k, const void* v, int lcap, const int32_t* prefix_lens, int max_ctx,
                                      const void* k_draft, const void* v_draft, const uint32_t* tree_mask,

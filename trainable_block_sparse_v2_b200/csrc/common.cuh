@@ -43,6 +43,17 @@ IV2_DEV uint32_t pack_bf16(float lo, float hi)
     return *reinterpret_cast<uint32_t*>(&v);
 }
 
+// fp64 -> bf16, round to nearest even, in one correctly rounded step: round to odd into fp32 first (fp32 has
+// at least two more significand bits than bf16, so the second rounding equals a direct one; Boldo and
+// Melquiond, IEEE Trans. Computers 57(4), 2008).  The semantic kernels are rounded through it.
+IV2_DEV uint16_t f64_to_bf16_rne(double x)
+{
+    float f = __double2float_rz(x);                 // truncate toward zero into fp32
+    if ((double)f != x) f = __uint_as_float(__float_as_uint(f) | 1u);  // inexact: make the last bit odd
+    __nv_bfloat16 h = __float2bfloat16_rn(f);
+    return *reinterpret_cast<uint16_t*>(&h);
+}
+
 IV2_DEV float bf16_lo(uint32_t v) { return __uint_as_float(v << 16); }
 IV2_DEV float bf16_hi(uint32_t v) { return __uint_as_float(v & 0xffff0000u); }
 

@@ -172,9 +172,10 @@ IV2_DEV void scan_tile(const unsigned char* rows, int row0, int nvalid, const ui
 template <int D, int CL, int E>
 __global__ void __launch_bounds__(kFThreads, 2)
 decode_fused_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_constant__ CUtensorMap tmap_v,
-                    QueryRows qr, const __nv_bfloat16* __restrict__ kern, int nk_cap, MethodConsts mc, KvRows kr,
+                    QueryRows qr, __nv_bfloat16* __restrict__ kern, int nk_cap, MethodConsts mc, KvRows kr,
                     int32_t* __restrict__ idx, int32_t* __restrict__ cnt, __nv_bfloat16* __restrict__ out,
-                    float* __restrict__ lse_out, unsigned first_wait_limit)
+                    float* __restrict__ lse_out, unsigned first_wait_limit, const __nv_bfloat16* __restrict__ kraw,
+                    int pool_new)
 {
     using L = FLayout<D>;
     extern __shared__ unsigned char smem_raw[];
@@ -182,6 +183,7 @@ decode_fused_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_con
     __shared__ uint64_t full[kFStages];
     __shared__ uint64_t never;  // testing only: a barrier no thread or copy arrives on
     __shared__ int cta_err;  // set by a wait that ran out: the CTA's other waits then give up early
+    __shared__ __nv_bfloat16 new_kern[128];  // the kernel completed by the row's last key (pool_new)
     __shared__ float part_m[16], part_s[16], lse2[16], halo_out[16];
     __shared__ __align__(16) float lse_slot[kFMaxCL][16][2];  // (max, sum) partials pushed by every CTA
 
@@ -226,6 +228,30 @@ decode_fused_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_con
     const int nown = max(b1 - b0, 0);
     // a context past the launch's max_ctx would overrun the per-CTA tables: flag it, attend to nothing
     const bool bad = !dense && (bpc > kFMaxBpc || nb > kFThreads * E);
+    // pool_new: the kernel completed by the row's last key (when it completes one) is pooled here by the CTA that
+    // owns its block, with kernel_pool_kernel's arithmetic (two 16-key halves summed in row order in fp64, scaled
+    // by 1/32, rounded once): its scan stage is patched with it and it is stored to the cache after the scan
+    const int j_new = (pool_new && n >= kKernelSize && (n - kKernelSize) % kKernelStride == 0 && n <= qr.max_ctx)
+                          ? (n - kKernelSize) / kKernelStride : -1;
+    const bool own_new = j_new >= 0 && j_new < nk_cap && j_new / kKernelsPerBlock >= b0 &&
+                         j_new / kKernelsPerBlock < b1;
+    if (own_new && tid < D) {
+        double half[2];
+#pragma unroll
+        for (int hh = 0; hh < 2; ++hh) {
+            const long r0 = kv_pos_row(kr, b, (j_new + hh) * kKernelStride);  // 16 consecutive rows
+            double acc = 0.0;
+            if (r0 >= 0) {
+                const __nv_bfloat16* src = kraw + (r0 * qr.Hkv + g) * D + tid;
+#pragma unroll
+                for (int r = 0; r < kKernelStride; ++r)
+                    acc += (double)__bfloat162float(src[(size_t)r * qr.Hkv * D]);
+            }
+            half[hh] = acc;
+        }
+        const uint16_t bits = f64_to_bf16_rne((half[0] + half[1]) * (1.0 / kKernelSize));
+        new_kern[tid] = *reinterpret_cast<const __nv_bfloat16*>(&bits);
+    }
     const bool sparse = !dense && !bad;
     const __nv_bfloat16* qrow = static_cast<const __nv_bfloat16*>(qr.q) + ((size_t)bt * qr.Hq + g * G) * D;
     int32_t* idx_row = idx ? idx + (size_t)row * mc.kmax : nullptr;  // null: no block list is written
@@ -287,6 +313,14 @@ decode_fused_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_con
             phase_bits ^= 1u << st;
             const int sc = b0 + i * kFChunkBlocks, se = min(sc + kFChunkBlocks, b1);
             const int nblk = se - sc;
+            if (own_new && j_new >= sc * kKernelsPerBlock && j_new < se * kKernelsPerBlock) {
+                // the stage holds the cache's old row j_new: replace it with the pooled kernel
+                __nv_bfloat16* prow = reinterpret_cast<__nv_bfloat16*>(smem + (size_t)st * L::kChunkBytes) +
+                                      (size_t)(j_new - sc * kKernelsPerBlock) * D;
+                if (tid < D) prow[tid] = new_kern[tid];
+                tc::fence_proxy_async_smem();  // before the next copy into this stage
+                __syncthreads();
+            }
             const int nvalid = max(min(se * kKernelsPerBlock, nkv) - sc * kKernelsPerBlock, 0);  // rows staged
             const unsigned char* rows = smem + (size_t)st * L::kChunkBytes;
             // this warp's tiles: warp and warp + 8 of the stage's 16 (4 kernel rows per block, 8 per tile)
@@ -639,6 +673,8 @@ decode_fused_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_con
                 lse_out[(size_t)bt * qr.Hq + g * G + h] = Lsum > 0.f ? (M + __log2f(Lsum)) * kLn2 : neg_inf();
         }
     }
+    // the pooled kernel goes to the cache (this CTA's copies of it have all landed; no other CTA reads it)
+    if (own_new && tid < D) kern[(((size_t)b * qr.Hkv + g) * nk_cap + j_new) * D + tid] = new_kern[tid];
     // a wait that ran out (or a context past the launch's tables): the results of this row are not the method's
     if (failed) atomicOr(&g_fused_error, 1);
 }
@@ -649,7 +685,7 @@ namespace {
 template <int D, int CL, int E>
 cudaError_t fused_launch(const CUtensorMap& tk, const CUtensorMap& tv, const QueryRows& qr, const void* kern,
                          int nk_cap, const MethodConsts& mc, const KvRows& kr, int32_t* idx, int32_t* cnt, void* out,
-                         float* lse, cudaStream_t s)
+                         float* lse, const void* kraw, bool pool_new, cudaStream_t s)
 {
     auto kfn = decode_fused_kernel<D, CL, E>;
     cudaError_t e = ensure_smem(kfn, FLayout<D>::kBytes);
@@ -660,8 +696,9 @@ cudaError_t fused_launch(const CUtensorMap& tk, const CUtensorMap& tv, const Que
     }
     const int rows = qr.B * qr.T * qr.Hkv;
     return launch_pdl_cluster(kfn, dim3(CL, rows), dim3(kFThreads), CL, FLayout<D>::kBytes, s, tk, tv, qr,
-                              static_cast<const __nv_bfloat16*>(kern), nk_cap, mc, kr, idx, cnt,
-                              static_cast<__nv_bfloat16*>(out), lse, g_first_wait_limit.load(std::memory_order_relaxed));
+                              static_cast<__nv_bfloat16*>(const_cast<void*>(kern)), nk_cap, mc, kr, idx, cnt,
+                              static_cast<__nv_bfloat16*>(out), lse, g_first_wait_limit.load(std::memory_order_relaxed),
+                              static_cast<const __nv_bfloat16*>(kraw), pool_new ? 1 : 0);
 }
 
 // 16-CTA clusters of this kernel the device keeps resident at once (0 when 16 is not schedulable).  Cached per
@@ -701,16 +738,16 @@ int resident_clusters16()
 template <int D, int E>
 cudaError_t fused_dispatch_cl(const CUtensorMap& tk, const CUtensorMap& tv, const QueryRows& qr, const void* kern,
                               int nk_cap, const MethodConsts& mc, int nb_max, const KvRows& kr, int32_t* idx, int32_t* cnt,
-                              void* out, float* lse, cudaStream_t s)
+                              void* out, float* lse, const void* kraw, bool pool_new, cudaStream_t s)
 {
     const int rows = qr.B * qr.T * qr.Hkv;
     const bool need16 = nb_max > 8 * kFMaxBpc || mc.kmax > 8 * kFListCap;
     const int r16 = resident_clusters16<D, E>();
     if (need16 || (r16 > 0 && rows <= r16)) {
         if (r16 <= 0) return cudaErrorNotSupported;
-        return fused_launch<D, 16, E>(tk, tv, qr, kern, nk_cap, mc, kr, idx, cnt, out, lse, s);
+        return fused_launch<D, 16, E>(tk, tv, qr, kern, nk_cap, mc, kr, idx, cnt, out, lse, kraw, pool_new, s);
     }
-    return fused_launch<D, 8, E>(tk, tv, qr, kern, nk_cap, mc, kr, idx, cnt, out, lse, s);
+    return fused_launch<D, 8, E>(tk, tv, qr, kern, nk_cap, mc, kr, idx, cnt, out, lse, kraw, pool_new, s);
 }
 
 }  // namespace
@@ -724,7 +761,7 @@ bool decode_fused_supported(const QueryRows& qr, const MethodConsts& mc)
 
 cudaError_t launch_decode_fused(const QueryRows& qr, const void* kern, int nk_cap, const MethodConsts& mc,
                                 const void* k, const void* v, const KvRows& kr, int32_t* idx, int32_t* cnt, void* out,
-                                float* lse, cudaStream_t s)
+                                float* lse, cudaStream_t s, bool pool_new)
 {
     const int nb_max = (qr.max_ctx - 1) / kBlock + 1;
     if (!decode_fused_supported(qr, mc)) return cudaErrorNotSupported;
@@ -736,7 +773,7 @@ cudaError_t launch_decode_fused(const QueryRows& qr, const void* kern, int nk_ca
         return cudaErrorNotSupported;
     // the leader's top-k keeps E = ceil(nb_max / 256) blocks per thread
 #define IV2_FUSED(DD, EE) \
-    fused_dispatch_cl<DD, EE>(tk, tv, qr, kern, nk_cap, mc, nb_max, kr, idx, cnt, out, lse, s)
+    fused_dispatch_cl<DD, EE>(tk, tv, qr, kern, nk_cap, mc, nb_max, kr, idx, cnt, out, lse, k, pool_new, s)
     if (qr.D == 128) {
         if (nb_max <= 1024) return IV2_FUSED(128, 4);
         if (nb_max <= 2048) return IV2_FUSED(128, 8);

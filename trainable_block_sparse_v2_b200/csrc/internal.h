@@ -205,9 +205,11 @@ int tc_error_flag_read_and_clear();
 // one decode step (scoring, top-k, sparse attention) in a single cluster kernel; cudaErrorNotSupported when
 // the shape is outside what it handles
 bool decode_fused_supported(const QueryRows& qr, const MethodConsts& mc);
+// pool_new: first pool, into kern, the kernel completed by each row's last key (kernel_pool of old = n - 1,
+// new = n, done by the CTA that owns it)
 cudaError_t launch_decode_fused(const QueryRows& qr, const void* kern, int nk_cap, const MethodConsts& mc,
                                 const void* k, const void* v, const KvRows& kr, int32_t* idx, int32_t* cnt, void* out,
-                                float* lse, cudaStream_t s);
+                                float* lse, cudaStream_t s, bool pool_new = false);
 int fused_error_flag_read_and_clear();
 int fused_set_first_wait_limit(unsigned polls);  // testing only
 

@@ -27,15 +27,6 @@ namespace iv2 {
 constexpr int kPoolKernelsPerCta = 32;
 constexpr int kPoolThreads = 256;
 
-// fp64 -> bf16, round to nearest even, in one correctly rounded step (round-to-odd into fp32 first).
-IV2_DEV uint16_t f64_to_bf16_rne(double x)
-{
-    float f = __double2float_rz(x);                 // truncate toward zero into fp32
-    if ((double)f != x) f = __uint_as_float(__float_as_uint(f) | 1u);  // inexact: make the last bit odd
-    __nv_bfloat16 h = __float2bfloat16_rn(f);
-    return *reinterpret_cast<uint16_t*>(&h);
-}
-
 template <int D>
 __global__ void __launch_bounds__(kPoolThreads) kernel_pool_kernel(const __nv_bfloat16* __restrict__ k, KvRows kr,
                                                                    int Hkv, const int32_t* __restrict__ old_lens,
