@@ -463,17 +463,16 @@ decode_fused_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_con
         if (rank == 0 && tid == 0) cnt[row] = 0;
     } else {
         CtaSelectSmem& sel = *reinterpret_cast<CtaSelectSmem*>(smem + L::kSelWs);
-        int32_t* list_all = reinterpret_cast<int32_t*>(smem + L::kSelList);
+        // this CTA's entries rank, rank + CL, ... straight from the select's emit (no pass over the whole list)
         const int total = cta_select_topk<kFThreads, E>(S, c, mc.init_blocks, mc.local_blocks, mc.topk, mc.kmax,
                                                         rank == 0 ? idx_row : nullptr, rank == 0 ? cnt + row : nullptr,
-                                                        sel, list_all);
+                                                        sel, [&](int pos, int blk) {
+                                                            if (pos % CL == rank) {
+                                                                my_list[pos / CL] = blk;
+                                                                my_row[pos / CL] = first_row(blk);
+                                                            }
+                                                        });
         count = min(total, mc.kmax);
-        __syncthreads();
-        for (int i = tid; rank + CL * i < count; i += kFThreads) {
-            const int blk = list_all[rank + CL * i];
-            my_list[i] = blk;
-            my_row[i] = first_row(blk);
-        }
     }
     __syncthreads();
     // region A held generic-proxy data (scores, select scratch): order it before the TMA writes

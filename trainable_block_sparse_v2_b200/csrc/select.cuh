@@ -348,11 +348,15 @@ IV2_DEV int bucket_of(uint32_t key, uint32_t kmin, float bucket_scale)
     return min((int)((float)(key - kmin) * bucket_scale), kBuckets - 1);
 }
 
-// Returns the number of chosen blocks (every thread); when idx_sm is given the list is also written there;
-// idx_out / cnt_out may be null (the list then only goes to idx_sm).
-template <int NT, int E>
+// Returns the number of chosen blocks (every thread); on_entry(pos, block) is called, by the thread that owns
+// the block, for every list entry pos < kmax; idx_out / cnt_out may be null (the list then only goes to on_entry).
+struct NoListEntry {
+    IV2_DEV void operator()(int, int) const {}
+};
+
+template <int NT, int E, typename OnEntry = NoListEntry>
 IV2_DEV int cta_select_topk(const float* S, int c, int init, int local, int topk, int kmax, int32_t* idx_out,
-                            int32_t* cnt_out, CtaSelectSmem& sm, int32_t* idx_sm = nullptr)
+                            int32_t* cnt_out, CtaSelectSmem& sm, OnEntry on_entry = OnEntry())
 {
     constexpr int NW = NT / 32;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -361,12 +365,33 @@ IV2_DEV int cta_select_topk(const float* S, int c, int init, int local, int topk
     uint32_t key[E];
     int ncand_local = 0;
     uint32_t lo = 0xffffffffu, hi = 0u;
+    // the thread's E scores: with E a multiple of 4 and the whole range inside the row, E / 4 16-byte loads
+    // (consecutive threads start 16 E bytes apart: no bank conflict, where E scalar loads conflict 4 ways)
+    float sv[E];
+    if constexpr (E % 4 == 0) {
+        if (b0 + E <= nb) {
+#pragma unroll
+            for (int e4 = 0; e4 < E / 4; ++e4) {
+                const float4 v = reinterpret_cast<const float4*>(S + b0)[e4];
+                sv[4 * e4] = v.x;
+                sv[4 * e4 + 1] = v.y;
+                sv[4 * e4 + 2] = v.z;
+                sv[4 * e4 + 3] = v.w;
+            }
+        } else {
+#pragma unroll
+            for (int e = 0; e < E; ++e) sv[e] = b0 + e < nb ? S[b0 + e] : neg_inf();
+        }
+    } else {
+#pragma unroll
+        for (int e = 0; e < E; ++e) sv[e] = b0 + e < nb ? S[b0 + e] : neg_inf();
+    }
 #pragma unroll
     for (int e = 0; e < E; ++e) {
         const int b = b0 + e;
         key[e] = 0u;
         if (b < nb && !is_forced(b, c, init, local)) {
-            const float s = S[b];
+            const float s = sv[e];
             if (s != neg_inf()) key[e] = float_key(s);
         }
         if (key[e] != 0u) {
@@ -538,7 +563,7 @@ IV2_DEV int cta_select_topk(const float* S, int c, int init, int local, int topk
         if (chosen[e]) {
             if (pos < kmax) {
                 if (idx_out) idx_out[pos] = b0 + e;
-                if (idx_sm) idx_sm[pos] = b0 + e;
+                on_entry(pos, b0 + e);
             }
             ++pos;
         }
