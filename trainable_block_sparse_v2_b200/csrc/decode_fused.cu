@@ -50,14 +50,14 @@ constexpr int kFMaxBpc = 192;                           // context blocks per CT
 constexpr int kFBmaxPitch = kFMaxBpc + 1;               // odd pitch: the 8 head rows of a warp hit 8 banks
 constexpr int kFMaxCL = 16;
 constexpr int kFListCap = 192;                          // block-list entries per CTA
-constexpr int kFMaxKmax = 2048;                         // block-list length a CTA stages
+constexpr int kFMaxKmax = 2048;                         // longest block list (kmax) the step takes
 
 constexpr int cmax(int a, int b) { return a > b ? a : b; }
 constexpr int round_up(int a, int m) { return (a + m - 1) / m * m; }
 
 template <int D>
 struct FLayout {
-    // region A: scan ring | S, select scratch, whole list | attention ring | warp partials
+    // region A: scan ring | S, select scratch | attention ring | warp partials
     static constexpr int kChunkBytes = kFChunkRows * D * 2;
     static constexpr int kScanRing = kFStages * kChunkBytes;
     static constexpr int kBoxBytes = kBlock * 64 * 2;          // one TMA box: 64 keys x 64 dims
@@ -66,8 +66,7 @@ struct FLayout {
     static constexpr int kAttnRing = kFStages * kStageBytes;
     static constexpr int kS = 0;                               // S of every block of the row
     static constexpr int kSelWs = kFMaxCL * kFMaxBpc * 4 + 16;  // bucket-select scratch (S may overhang 3)
-    static constexpr int kSelList = round_up(kSelWs + (int)sizeof(CtaSelectSmem), 16);  // the whole list
-    static constexpr int kSelEnd = kSelList + kFMaxKmax * 4;
+    static constexpr int kSelEnd = kSelWs + (int)sizeof(CtaSelectSmem);
     static constexpr int kWo = 0;                              // [warp][16][kWoPitch] scaled warp outputs
     static constexpr int kWoPitch = D + 8;                     // floats; the 8 head rows a warp stores at once
                                                                // start 8 banks apart (conflict-free float2)
