@@ -44,7 +44,7 @@ HQ, HKV, D = 32, 2, 128
 # their capture (the two-call decode kernels took the paged / packed addressing since)
 NCU_TRAFFIC = {
     "sparse_decode_step": 31_308_928,                   # decode_fused_kernel: 31.31 MB read, ~2 KB written
-    "sparse_decode_step_pool": 31_313_408,              # the same kernel pooling the new key's kernel
+    "sparse_decode_step_pool": 31_319_552,              # the same kernel pooling the new key's kernel
     "sparse_attn_decode": None,                         # attn_split_kernel + attn_merge_kernel
     "block_score_topk": None,                           # score_scan_kernel + score_select_kernel
     "sparse_attn_prefill": 322_111_488 + 229_101_312,   # attn_tc_kernel<16, 128>
