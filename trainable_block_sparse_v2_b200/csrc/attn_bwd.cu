@@ -16,6 +16,9 @@
 //  4. fill      one warp per row: writes the token into the list of every block it attends (the order
 //               inside a list follows the atomics, so the fp32 sums of dk / dv are equal up to rounding
 //               order from run to run);
+//  4b. order    one CTA: the work items sorted by the first token of their chunk (a counting sort over
+//               token buckets), so that the items the persistent dk / dv CTAs run at the same time gather
+//               neighbouring tokens, whose Q and dO rows then come from L2 instead of DRAM;
 //  5. dq        one warp per row, the forward's walk over the row's blocks in 32-key halves, double-
 //               buffered (mma.sync m16n8k16 with the G <= 16 heads of the group as MMA rows):
 //               S = Q K^T, P = 2^(S log2e - lse log2e), dP = dO V^T, dS = P (dP - Dsum), dQ += dS K;
@@ -38,6 +41,7 @@ constexpr int kDqWarps = 2;       // rows per CTA of the dq kernel: 64 KB of sta
 constexpr int kDkvThreads = 128;  // 4 warps x 16 keys of one 64-key block
 constexpr int kItemTokens = 256;  // tokens per dkdv work item
 constexpr int kScanThreads = 1024;
+constexpr int kOrderBuckets = 4096;  // token buckets of the work-item sort
 
 size_t round256(size_t x) { return (x + 255) / 256 * 256; }
 
@@ -51,7 +55,7 @@ int bwd_max_per_row(int max_ctx, int kmax, int dense_len, bool dense_all)
 }
 
 struct BwdWsLayout {
-    size_t dsum, counts, offsets, cursor, nitems, item_list, item_start, tokens, end;
+    size_t dsum, counts, offsets, cursor, nitems, item_list, item_start, order_list, order_start, tokens, end;
     int nl, nb, cap, max_items;
 };
 
@@ -71,6 +75,8 @@ BwdWsLayout bwd_layout(int B, int T, int Hq, int Hkv, int max_ctx, int kmax, int
     w.nitems = o;     o += 256;
     w.item_list = o;  o += round256((size_t)w.max_items * 4);
     w.item_start = o; o += round256((size_t)w.max_items * 4);
+    w.order_list = o; o += round256((size_t)w.max_items * 4);
+    w.order_start = o; o += round256((size_t)w.max_items * 4);
     w.tokens = o;     o += round256((size_t)w.cap * 4);
     w.end = o;
     return w;
@@ -248,6 +254,77 @@ __global__ void __launch_bounds__(kBwdRowWarps * 32) bwd_fill_kernel(QueryRows q
         if (blk < 0 || blk >= nb) continue;
         const int pos = atomicAdd(&cl[blk], 1);
         if (pos < cap) tokens[pos] = r.t;
+    }
+}
+
+// ---------------------------------------------------------------------------------------------------
+// 4b. order: a counting sort of the work items by (batch, first token of the chunk) >> shift, stable up to
+// the order of the shared-memory atomics (any order of the items gives the same sums up to rounding order)
+__global__ void __launch_bounds__(kScanThreads) bwd_order_kernel(const int* __restrict__ nitems,
+                                                                 const int* __restrict__ item_list,
+                                                                 const int* __restrict__ item_start,
+                                                                 const int* __restrict__ offsets,
+                                                                 const int* __restrict__ tokens, int cap,
+                                                                 int lists_per_batch, int T, int shift,
+                                                                 int* __restrict__ order_list,
+                                                                 int* __restrict__ order_start)
+{
+    pdl_launch_dependents();
+    pdl_wait();
+    __shared__ int hist[kOrderBuckets];
+    __shared__ int wsum[32];
+    const int n = *nitems;
+    for (int i = threadIdx.x; i < kOrderBuckets; i += kScanThreads) hist[i] = 0;
+    __syncthreads();
+    // the bucket of item i; the token read is clamped into the list array, and the bucket into the histogram
+    // (a list entry past cap was never written: its value only orders the items)
+    auto bucket = [&](int i) {
+        const int l = item_list[i];
+        const long at = max(0L, min((long)offsets[l] + item_start[i], (long)cap - 1));
+        const long key = (long)(l / lists_per_batch) * T + (cap > 0 ? tokens[at] : 0);
+        return (int)max(0L, min(key >> shift, (long)kOrderBuckets - 1));
+    };
+    for (int i = threadIdx.x; i < n; i += kScanThreads) atomicAdd(&hist[bucket(i)], 1);
+    __syncthreads();
+    // exclusive scan of the buckets, kOrderBuckets / kScanThreads consecutive ones per thread
+    constexpr int kPer = kOrderBuckets / kScanThreads;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    int c[kPer], tot = 0;
+#pragma unroll
+    for (int j = 0; j < kPer; ++j) {
+        c[j] = hist[kPer * threadIdx.x + j];
+        tot += c[j];
+    }
+    int incl = tot;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += y;
+    }
+    if (lane == 31) wsum[warp] = incl;
+    __syncthreads();
+    if (warp == 0) {
+        const int a = wsum[lane];
+        int ia = a;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int y = __shfl_up_sync(0xffffffffu, ia, o);
+            if (lane >= o) ia += y;
+        }
+        wsum[lane] = ia - a;
+    }
+    __syncthreads();
+    int ex = wsum[warp] + incl - tot;
+#pragma unroll
+    for (int j = 0; j < kPer; ++j) {
+        hist[kPer * threadIdx.x + j] = ex;  // each thread rewrites only its own buckets
+        ex += c[j];
+    }
+    __syncthreads();
+    for (int i = threadIdx.x; i < n; i += kScanThreads) {
+        const int slot = atomicAdd(&hist[bucket(i)], 1);
+        order_list[slot] = item_list[i];
+        order_start[slot] = item_start[i];
     }
 }
 
@@ -612,6 +689,8 @@ cudaError_t bwd_impl(const QueryRows& qr, const void* k, const void* v, int Lcap
     int* nitems = reinterpret_cast<int*>(base + w.nitems);
     int* item_list = reinterpret_cast<int*>(base + w.item_list);
     int* item_start = reinterpret_cast<int*>(base + w.item_start);
+    int* order_list = reinterpret_cast<int*>(base + w.order_list);
+    int* order_start = reinterpret_cast<int*>(base + w.order_start);
     int* tokens = reinterpret_cast<int*>(base + w.tokens);
     const int dense_flag = dense_all ? 1 : 0;
     const long rows = (long)qr.B * qr.T * qr.Hkv;
@@ -634,6 +713,13 @@ cudaError_t bwd_impl(const QueryRows& qr, const void* k, const void* v, int Lcap
     e = launch_pdl(bwd_fill_kernel, dim3(row_grid), dim3(kBwdRowWarps * 32), 0, s, qr, idx, cnt, mc, dense_flag, w.nb,
                    cursor, tokens, w.cap);
     if (e != cudaSuccess) return e;
+    int shift = 0;
+    while (((long)qr.B * qr.T >> shift) >= kOrderBuckets) ++shift;
+    e = launch_pdl(bwd_order_kernel, dim3(1), dim3(kScanThreads), 0, s, static_cast<const int*>(nitems),
+                   static_cast<const int*>(item_list), static_cast<const int*>(item_start),
+                   static_cast<const int*>(offsets), static_cast<const int*>(tokens), w.cap, qr.Hkv * w.nb, qr.T,
+                   shift, order_list, order_start);
+    if (e != cudaSuccess) return e;
     e = cudaErrorNotSupported;
     if (D == 128 && bwd_dq_tc_supported(qr))
         e = launch_bwd_dq_tc(qr, k, v, Lcap, idx, cnt, mc, dense_all, lse, dsum, dout, dq, s);
@@ -648,8 +734,8 @@ cudaError_t bwd_impl(const QueryRows& qr, const void* k, const void* v, int Lcap
     }
     if (e != cudaSuccess) return e;
     if (D == 128 && bwd_dkdv_tc_supported(qr)) {
-        e = launch_bwd_dkdv_tc(qr, k, v, Lcap, mc, w.nb, lse, dsum, dout, counts, offsets, tokens, nitems, item_list,
-                               item_start, w.cap, w.max_items, dk, dv, s);
+        e = launch_bwd_dkdv_tc(qr, k, v, Lcap, mc, w.nb, lse, dsum, dout, counts, offsets, tokens, nitems, order_list,
+                               order_start, w.cap, w.max_items, dk, dv, s);
         if (e != cudaErrorNotSupported) return e;
     }
     e = ensure_smem(bwd_dkdv_kernel<D>, DkvSmem<D>::kBytes);
@@ -662,7 +748,7 @@ cudaError_t bwd_impl(const QueryRows& qr, const void* k, const void* v, int Lcap
                       static_cast<const float*>(dsum), static_cast<const __nv_bfloat16*>(dout),
                       static_cast<const int*>(counts), static_cast<const int*>(offsets),
                       static_cast<const int*>(tokens), static_cast<const int*>(nitems),
-                      static_cast<const int*>(item_list), static_cast<const int*>(item_start), w.cap, dk, dv);
+                      static_cast<const int*>(order_list), static_cast<const int*>(order_start), w.cap, dk, dv);
 }
 
 }  // namespace
