@@ -24,7 +24,9 @@ relative to each other.  It reports:
 * a wait that returns on another phase than the one it means (the barrier ran two phases ahead of the waiter,
   or the waiter is two phases ahead of the barrier);
 * a buffer read while a write to it is pending, or read holding other data than the reader expects;
-* a buffer overwritten while a tensor-core read or a copy into it is pending.
+* a buffer overwritten while a tensor-core read or a copy into it is pending;
+* the CTA ending (every role done: TMEM freed, shared memory released) while a tensor-core op, a commit or a
+  copy is still in flight.
 """
 from __future__ import annotations
 
@@ -180,6 +182,10 @@ class PipelineModel:
             st["op"] = next(st["gen"], None)
             st["done"] = st["op"] is None
         for _ in range(max_steps):
+            if all(st["done"] for st in self.roles.values()) and (self.copies or any(self.tc_queues.values())):
+                inflight = {n: len(q) for n, q in self.tc_queues.items() if q}
+                raise ProtocolError(f"the CTA ends with tensor-core ops {inflight} and {len(self.copies)} copies in "
+                                    "flight")
             runnable = []
             for name, st in self.roles.items():
                 if st["done"]:

@@ -13,6 +13,16 @@ from pipeline_model import PipelineModel, ProtocolError
 RING = 3
 
 
+def drained(m: PipelineModel, name: str, ops, skip: bool = False):
+    """an issuing role's ops, then its drain: a commit on a barrier of its own and the wait for it, after which
+    none of its tensor-core ops is in flight (the kernels drain every issuer before the CTA frees its TMEM)"""
+    m.bar(f"drain.{name}", 1)
+    yield from ops
+    if not skip:
+        yield ("commit", f"drain.{name}")
+        yield ("wait", f"drain.{name}", 0)
+
+
 # --------------------------------------------------------------------------------------------------------------
 # attn_tc_kernel (csrc/attn_tc.cu): 128-row tile, U union blocks in NP = ceil(U / 2) steps of 128 keys.
 # Warp 0: Q once (shared memory, the A operand of every S MMA), then K per step (3-slot ring); warp 10: V per
@@ -118,8 +128,8 @@ def attn_tc_model(m: PipelineModel, U: int, rescale_steps=(), parts: int = 2, mi
 
     m.role("k_producer", k_producer())
     m.role("v_producer", v_producer())
-    m.role("s_issuer", s_issuer())
-    m.role("pv_issuer", pv_issuer())
+    m.role("s_issuer", drained(m, "s_issuer", s_issuer()))
+    m.role("pv_issuer", drained(m, "pv_issuer", pv_issuer(), skip=mistake == "PV issuer skips its drain"))
     for w in range(2, 2 + 4 * parts):
         m.role(f"softmax{w}", softmax(w))
 
@@ -202,7 +212,7 @@ def score_tc_model(m: PipelineModel, ntiles: int, mistake: str = "", parts: int 
                 yield ("read", f"Ssm.t{ts}.s{q}.p{h}", "S")
 
     m.role("producer", producer())
-    m.role("issuer", issuer())
+    m.role("issuer", drained(m, "issuer", issuer()))
     for w in range(2, 2 + nreaders):
         m.role(f"reader{w}", reader(w))
 
@@ -243,7 +253,7 @@ def _caught(model, seeds, *args, **kw):
     ("k producer skips k_empty", 9), ("v producer skips v_empty", 9), ("S issuer skips o_done", 9),
     ("PV issuer skips p_full", 5),
     ("single-buffered max exchange", 5), ("no barrier before P", 3), ("rescale without o_done", 5),
-    ("no barrier before the sums", 5),
+    ("no barrier before the sums", 5), ("PV issuer skips its drain", 5),
 ])
 def test_attn_tc_planted_mistakes_are_caught(mistake, U):
     NP = (U + 1) // 2
@@ -374,9 +384,9 @@ def bwd_dq_model(m: PipelineModel, U: int, mistake: str = ""):
 
     m.role("warp0", warp0())
     m.role("warp10", warp10())
-    m.role("s_issuer", s_issuer())
-    m.role("dp_issuer", dp_issuer())
-    m.role("dq_issuer", dq_issuer())
+    m.role("s_issuer", drained(m, "s_issuer", s_issuer()))
+    m.role("dp_issuer", drained(m, "dp_issuer", dp_issuer()))
+    m.role("dq_issuer", drained(m, "dq_issuer", dq_issuer(), skip=mistake == "dQ issuer skips its drain"))
     for w in range(2, 10):
         m.role(f"ds{w}", ds_warp(w))
 
@@ -475,8 +485,8 @@ def bwd_dkdv_model(m: PipelineModel, items, mistake: str = ""):
             yield ("arrive", "acc_free", 32)
 
     m.role("producer", producer())
-    m.role("s_issuer", s_issuer())
-    m.role("acc_issuer", acc_issuer())
+    m.role("s_issuer", drained(m, "s_issuer", s_issuer(), skip=mistake == "S issuer skips its drain"))
+    m.role("acc_issuer", drained(m, "acc_issuer", acc_issuer()))
     for q4 in Q4:
         m.role(f"warp{2 + q4}", warps(q4))
 
@@ -493,13 +503,14 @@ def test_bwd_dkdv_protocol(items):
 
 @pytest.mark.parametrize("mistake", ["K producer skips k_empty", "issuer skips ds_full", "no pair barrier",
                                      "no final dq_done wait", "S issuer skips dq_done", "dP issuer skips ds_full",
-                                     "k_empty waits for one issuer"])
+                                     "k_empty waits for one issuer", "dQ issuer skips its drain"])
 def test_bwd_dq_planted_mistakes_are_caught(mistake):
     assert _caught(bwd_dq_model, range(300), 7, mistake=mistake), mistake
 
 
 @pytest.mark.parametrize("mistake", ["producer skips kv_free", "producer skips qd_free", "issuer skips acc_free",
-                                     "warps skip pd_free", "warps skip acc_done", "qd_free waits for one issuer"])
+                                     "warps skip pd_free", "warps skip acc_done", "qd_free waits for one issuer",
+                                     "S issuer skips its drain"])
 def test_bwd_dkdv_planted_mistakes_are_caught(mistake):
     # acc_free matters only where empty items let the issuer commit acc_done twice without a P tile between
     assert _caught(bwd_dkdv_model, range(300), [3, 0, 0, 2, 4], mistake=mistake), mistake

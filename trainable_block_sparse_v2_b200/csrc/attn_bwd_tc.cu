@@ -53,6 +53,7 @@ struct Bars {
     uint64_t qd_full, qd_tmem;
     uint64_t k_full[kRing], k_empty[kRing], v_full[kRing], v_empty[kRing];
     uint64_t s_full[2], ds_full[2], dq_done[2];
+    uint64_t drain[3];  // the S, dP and dQ issuers' last MMAs
     uint32_t tmem_base;
     int n_union;
     int err;
@@ -161,6 +162,7 @@ bwd_dq_tc_kernel(QueryRows qr, const __grid_constant__ CUtensorMap tm_q, const _
             tc::mbar_init(&bars.ds_full[i], 256);
             tc::mbar_init(&bars.dq_done[i], 1);
         }
+        for (int i = 0; i < 3; ++i) tc::mbar_init(&bars.drain[i], 1);
         tc::fence_barrier_init();
     }
     if (warp == 1) {
@@ -236,6 +238,7 @@ bwd_dq_tc_kernel(QueryRows qr, const __grid_constant__ CUtensorMap tm_q, const _
                 tc::mma_commit(is_s ? &bars.k_empty[s] : &bars.v_empty[s]);
             }
         }
+        if (lane == 0) tc::mma_drain(&bars.drain[is_s ? 0 : 1]);
     } else if (warp == 12) {
         // ---------------- dQ issuer: dQ += dS(v) . K(v), dS(v) in the first 32 columns of S buffer v & 1 ----------
         if (lane == 0) {
@@ -253,6 +256,7 @@ bwd_dq_tc_kernel(QueryRows qr, const __grid_constant__ CUtensorMap tm_q, const _
                 tc::mma_commit(&bars.dq_done[db]);
                 tc::mma_commit(&bars.k_empty[s]);
             }
+            tc::mma_drain(&bars.drain[2]);
         }
     } else if (warp >= 2 && warp <= 9) {
         // ---------------- dS and dq: one TMEM lane (query row) per thread, 32 keys of each step ----------------
@@ -424,6 +428,7 @@ constexpr uint32_t kKvCols = 512, kKvColS = 0, kKvColDP = 128, kKvColDV = 256, k
 
 struct KvBars {
     uint64_t kv_full, kv_free, qd_full[2], qd_free[2], s_full[2], pd_full, pd_free, acc_done, acc_free;
+    uint64_t drain[2];  // the S / dP and dV / dK issuers' last MMAs
     uint32_t tmem_base;
     int err;
 };
@@ -461,6 +466,8 @@ bwd_dkdv_tc_kernel(QueryRows qr, const __grid_constant__ CUtensorMap tm_q1, cons
         tc::mbar_init(&bars.pd_free, 1);
         tc::mbar_init(&bars.acc_done, 1);
         tc::mbar_init(&bars.acc_free, 128);
+        tc::mbar_init(&bars.drain[0], 1);
+        tc::mbar_init(&bars.drain[1], 1);
         tc::fence_barrier_init();
     }
     if (warp == 1) {
@@ -560,6 +567,7 @@ bwd_dkdv_tc_kernel(QueryRows qr, const __grid_constant__ CUtensorMap tm_q1, cons
                 n_tile += ntiles;
                 tc::mma_commit(&bars.kv_free);  // only S and dP read the item's K and V
             }
+            tc::mma_drain(&bars.drain[0]);
         }
     } else if (warp == 6) {
         // ---------------- dV / dK issuer: dV^T += dO^T P, dK^T += Q^T dS per tile ----------------
@@ -595,6 +603,7 @@ bwd_dkdv_tc_kernel(QueryRows qr, const __grid_constant__ CUtensorMap tm_q1, cons
                 n_tile += ntiles;
                 tc::mma_commit(&bars.acc_done);
             }
+            tc::mma_drain(&bars.drain[1]);
         }
     } else if (warp >= 2 && warp <= 5) {
         // ---------------- P, dS (one query row per thread) and the flush (one head dimension per thread) ----------

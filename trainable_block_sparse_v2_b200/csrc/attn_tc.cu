@@ -73,6 +73,7 @@ struct Bars {
     uint64_t q_full;
     uint64_t k_full[kRing], k_empty[kRing], v_full[kRing], v_empty[kRing];
     uint64_t s_full[kNS], p_full[kNS], o_done[kNS];
+    uint64_t drain[2];  // the S and PV issuers' last MMAs
     uint32_t tmem_base;
     int n_union;
     int err;
@@ -219,6 +220,8 @@ attn_tc_kernel(QueryRows qr, const __grid_constant__ CUtensorMap tm_q, const __g
             tc::mbar_init(&bars.p_full[i], 256);
             tc::mbar_init(&bars.o_done[i], 1);
         }
+        tc::mbar_init(&bars.drain[0], 1);
+        tc::mbar_init(&bars.drain[1], 1);
         tc::fence_barrier_init();
     }
     if (warp == 1) {
@@ -305,6 +308,7 @@ attn_tc_kernel(QueryRows qr, const __grid_constant__ CUtensorMap tm_q, const __g
                 tc::mma_commit(&bars.k_empty[s]);
             }
         }
+        if (lane == 0) tc::mma_drain(&bars.drain[0]);
     } else if (warp == 11) {
         // ---------------- PV issuer ----------------
         if (lane == 0) {
@@ -323,6 +327,7 @@ attn_tc_kernel(QueryRows qr, const __grid_constant__ CUtensorMap tm_q, const __g
                 tc::mma_commit(&bars.o_done[pv]);
                 tc::mma_commit(&bars.v_empty[sv]);
             }
+            tc::mma_drain(&bars.drain[1]);
         }
     } else if (warp >= 2 && warp <= 9) {
         // ---------------- softmax + epilogue: one TMEM lane (query row) per thread, one block of each step ----

@@ -63,6 +63,7 @@ struct SBars {
     uint64_t q_full, q_tmem;
     uint64_t k_full[kSRing], k_empty[kSRing];
     uint64_t s_full[2], s_empty[2];  // per tile (A, B): accumulator ready / read back
+    uint64_t drain;                  // the issuer's last MMAs
     uint32_t tmem_base;
     int err;
 };
@@ -146,6 +147,7 @@ score_tc_kernel(QueryRows qr, const __grid_constant__ CUtensorMap tm_q, const __
             tc::mbar_init(&bars.s_full[i], 1);
             tc::mbar_init(&bars.s_empty[i], kSEpiThreads);
         }
+        tc::mbar_init(&bars.drain, 1);
         tc::fence_barrier_init();
     }
     if (warp == 1) {
@@ -215,6 +217,7 @@ score_tc_kernel(QueryRows qr, const __grid_constant__ CUtensorMap tm_q, const __
                 tc::mma_commit(&bars.k_empty[s]);
             }
         }
+        if (lane == 0) tc::mma_drain(&bars.drain);
     } else {
         // ---------------- TMEM readers: lane r of both tiles per thread, 32 columns per warp ----------------
         const int q4 = warp & 3, part = (warp - 2) >> 2;

@@ -145,6 +145,15 @@ IV2_DEV void mma_commit(uint64_t* bar)
                  : "memory");
 }
 
+// after an issuing thread's last tcgen05.mma: wait (bounded) until every MMA it issued has completed, on a
+// barrier of its own used once, so that the CTA frees its TMEM and exits with no MMA in flight, also when one
+// of its waits ran out and the loops stopped early
+IV2_DEV void mma_drain(uint64_t* bar)
+{
+    mma_commit(bar);
+    (void)mbar_wait(bar, 0, 1u << 22);
+}
+
 // 32 consecutive 32-bit columns of this thread's TMEM lane (lane quarter = warp % 4)
 IV2_DEV void tmem_ld32(uint32_t taddr, uint32_t (&r)[32])
 {
