@@ -1,4 +1,5 @@
-"""The bounded-wait error path of the fused decode step, driven without a fault.
+"""The bounded-wait error paths of the fused decode step and of the tensor-core prefill attention, driven
+without a fault.
 
 infllmv2_test_set_first_wait_limit makes the first kernel-cache wait of every CTA poll a barrier that nothing
 arrives on, so it gives up after a few polls while that stage's copy is still in flight -- what a wait whose
@@ -57,3 +58,49 @@ def test_fused_decode_wait_that_runs_out_is_reported_and_the_next_call_is_clean(
     assert binding.infllmv2_device_status() == 0
     for a, b in zip(ref, again):
         assert torch.equal(a, b) or (a.dtype.is_floating_point and torch.equal(a.nan_to_num(), b.nan_to_num()))
+
+
+def test_prefill_attention_wait_that_runs_out_is_reported_and_the_next_call_is_clean():
+    """The same limit on the tensor-core prefill attention: the first wait of every CTA's score-MMA issuer runs
+    out, the CTA's roles stop, its producers wait for their copies and its issuers for their MMAs, and the
+    next call with the normal waits gives exactly the earlier results."""
+    from trainable_block_sparse_v2_b200.build import build
+    from trainable_block_sparse_v2_b200.workloads import prefill_case
+    build()
+    lib = binding.load()
+    T = 1500
+    w = prefill_case(T, 32, 2, 128, topk=5, dense_len=300, seed=1716, n_needles=2)  # 16 heads per group
+    p = bparams(w.params)
+    q, K, V = dev(w.q), dev(w.k), dev(w.v)
+    L = dev_i32(w.ctx_lens)
+    nk_cap = binding.num_kernels(T)
+    kern = torch.zeros((1, 2, nk_cap, 128), dtype=torch.bfloat16, device="cuda")
+    binding.infllmv2_kernel_pool(K, dev_i32(np.zeros(1)), L, T, p, kern)
+    idx = torch.empty((1, T, 2, p.kmax), dtype=torch.int32, device="cuda")
+    cnt = torch.empty((1, T, 2), dtype=torch.int32, device="cuda")
+    ws = binding.workspace(p, 1, T, T, 32, 2, 128)
+    binding.infllmv2_block_score_topk(q, None, L, T, kern, p, idx, cnt, ws)
+    torch.cuda.synchronize()
+
+    def attend():
+        out = torch.full((1, T, 32, 128), float("nan"), dtype=torch.bfloat16, device="cuda")
+        lse = torch.full((1, T, 32), float("nan"), dtype=torch.float32, device="cuda")
+        binding.infllmv2_sparse_attn_prefill(q, K, V, None, L, T, idx, cnt, p, out, lse)
+        torch.cuda.synchronize()
+        return out, lse
+
+    assert binding.infllmv2_device_status() == 0
+    ref = attend()
+    assert binding.infllmv2_device_status() == 0
+    assert not torch.isnan(ref[0]).any()
+    assert lib.infllmv2_test_set_first_wait_limit(64) == 0
+    try:
+        attend()  # must return: every wait is bounded
+        assert binding.infllmv2_device_status() == TIMEOUT
+        assert binding.infllmv2_device_status() == 0
+    finally:
+        assert lib.infllmv2_test_set_first_wait_limit(0) == 0
+    again = attend()
+    assert binding.infllmv2_device_status() == 0
+    for a, b in zip(ref, again):
+        assert torch.equal(a, b)

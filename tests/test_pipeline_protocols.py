@@ -59,6 +59,10 @@ def attn_tc_model(m: PipelineModel, U: int, rescale_steps=(), parts: int = 2, mi
                 yield ("wait", f"k_empty{s}", k - 1)
             yield ("arrive_tx", f"k_full{s}", 1, 1)
             yield ("tma", f"k_full{s}", 1, [(f"K{s}", ("K", p))])
+        # the producer's drain before the CTA ends: every copy it issued has landed
+        yield ("wait", "q_full", 0)
+        for s in range(min(RING, NP)):
+            yield ("wait", f"k_full{s}", (NP - 1 - s) // RING)
 
     def v_producer():
         for p in range(NP):
@@ -67,6 +71,8 @@ def attn_tc_model(m: PipelineModel, U: int, rescale_steps=(), parts: int = 2, mi
                 yield ("wait", f"v_empty{s}", k - 1)
             yield ("arrive_tx", f"v_full{s}", 1, 1)
             yield ("tma", f"v_full{s}", 1, [(f"V{s}", ("V", p))])
+        for s in range(min(VR, NP)):
+            yield ("wait", f"v_full{s}", (NP - 1 - s) // VR)
 
     def s_issuer():
         yield ("wait", "q_full", 0)

@@ -23,8 +23,9 @@
 // back the next scores; warps 2-9 run the softmax and the epilogue, two warps per TMEM lane quarter, each on
 // one of the step's two blocks.
 // Producer/consumer hand-offs use mbarriers; MMA completion is signalled with tcgen05.commit.  Every wait
-// is bounded: after the limit the CTA records an error (g_tc_error), skips the rest of its work, frees its
-// TMEM and exits.
+// is bounded: after the limit the CTA records an error (g_tc_error) and skips the rest of its work; each
+// producer then waits (bounded) for the copies it issued and each MMA issuer for its MMAs, and the CTA frees
+// its TMEM and exits with nothing in flight.
 #include <mutex>
 
 #include "common.cuh"
@@ -74,6 +75,7 @@ struct Bars {
     uint64_t k_full[kRing], k_empty[kRing], v_full[kRing], v_empty[kRing];
     uint64_t s_full[kNS], p_full[kNS], o_done[kNS];
     uint64_t drain[2];  // the S and PV issuers' last MMAs
+    uint64_t never;     // nothing arrives on it: the wait a test drives to run out
     uint32_t tmem_base;
     int n_union;
     int err;
@@ -111,9 +113,10 @@ __device__ __forceinline__ float max3(float a, float b, float c)
     return d;
 }
 
-__device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity, volatile int* err)
+__device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity, volatile int* err,
+                                         uint32_t limit = 1u << 22)
 {
-    for (uint32_t i = 0; i < (1u << 22); ++i) {
+    for (uint32_t i = 0; i < limit; ++i) {
         if (tc::mbar_try_wait(bar, parity)) return true;
         if ((i & 255u) == 255u && *err) return false;
     }
@@ -129,7 +132,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 attn_tc_kernel(QueryRows qr, const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                const __grid_constant__ CUtensorMap tm_v, KvRows kr, const int32_t* __restrict__ idx,
                const int32_t* __restrict__ cnt, MethodConsts mc, int dense_all, __nv_bfloat16* __restrict__ out,
-               float* __restrict__ lse)
+               float* __restrict__ lse, unsigned test_wait_limit)
 {
     using Sh = TcShape<G, D>;
     constexpr int kTok = Sh::kTok, kSlot = Sh::kSlot, kKOff = Sh::kKOff, kVOff = Sh::kVOff, kQOff = Sh::kQOff;
@@ -222,6 +225,7 @@ attn_tc_kernel(QueryRows qr, const __grid_constant__ CUtensorMap tm_q, const __g
         }
         tc::mbar_init(&bars.drain[0], 1);
         tc::mbar_init(&bars.drain[1], 1);
+        tc::mbar_init(&bars.never, 1);
         tc::fence_barrier_init();
     }
     if (warp == 1) {
@@ -250,7 +254,8 @@ attn_tc_kernel(QueryRows qr, const __grid_constant__ CUtensorMap tm_q, const __g
 #pragma unroll
             for (int a = 0; a < Sh::kAtoms; ++a)
                 tc::tma_load_3d(smem + kQOff + a * 16384, &tm_q, 64 * a, g * G, zq, &bars.q_full);
-            for (int p = 0; p < NP; ++p) {
+            int issued = 0;  // steps whose K copies are in flight or landed
+            for (int p = 0; p < NP; ++p, ++issued) {
                 const int s = p % kRing, k = p / kRing;
                 if (k >= 1 && !wait_bar(&bars.k_empty[s], (k - 1) & 1, err)) break;
                 unsigned char* st = smem + kKOff + s * kSlot;
@@ -266,9 +271,15 @@ attn_tc_kernel(QueryRows qr, const __grid_constant__ CUtensorMap tm_q, const __g
                         tc::tma_load_3d(st + a * 16384 + i * 8192, &tm_k, 64 * a, g, z, &bars.k_full[s]);
                 }
             }
+            // every copy this lane issued has landed before the CTA ends (on the normal path each one was
+            // waited for already); after a wait ran out, the rest of the CTA no longer waits for them
+            (void)tc::mbar_wait(&bars.q_full, 0, 1u << 22);
+            for (int s = 0; s < kRing && s < issued; ++s)  // stage s last took step s + kRing ((issued-1-s)/kRing)
+                (void)tc::mbar_wait(&bars.k_full[s], ((issued - 1 - s) / kRing) & 1, 1u << 22);
         } else if (warp == 10 && lane == 0) {
             tc::prefetch_tensormap(&tm_v);
-            for (int p = 0; p < NP; ++p) {
+            int issued = 0;
+            for (int p = 0; p < NP; ++p, ++issued) {
                 const int s = p % kVRing, k = p / kVRing;
                 if (k >= 1 && !wait_bar(&bars.v_empty[s], (k - 1) & 1, err)) break;
                 unsigned char* st = smem + kVOff + s * kSlot;
@@ -282,11 +293,15 @@ attn_tc_kernel(QueryRows qr, const __grid_constant__ CUtensorMap tm_q, const __g
                         tc::tma_load_3d(st + a * 16384 + i * 8192, &tm_v, 64 * a, g, z, &bars.v_full[s]);
                 }
             }
+            for (int s = 0; s < kVRing && s < issued; ++s)
+                (void)tc::mbar_wait(&bars.v_full[s], ((issued - 1 - s) / kVRing) & 1, 1u << 22);
         }
     } else if (warp == 1) {
         // ---------------- S issuer ----------------
-        // S(p) overwrites the buffer of P(p - 3): it waits until PV(p - 3), issued by warp 11, has completed
-        if (lane == 0 && wait_bar(&bars.q_full, 0, err)) {
+        // S(p) overwrites the buffer of P(p - 3): it waits until PV(p - 3), issued by warp 11, has completed.
+        // With a test limit, the first wait polls a barrier nothing arrives on instead of Q's
+        if (lane == 0 && (test_wait_limit ? wait_bar(&bars.never, 0, err, test_wait_limit)
+                                          : wait_bar(&bars.q_full, 0, err))) {
             tc::tc_fence_after();
             constexpr uint32_t idesc_s = tc::idesc_bf16(128, kStepKeys, false);
             const uint32_t sQ = tc::smem_u32(smem + kQOff);
@@ -508,7 +523,7 @@ cudaError_t attn_tc_launch(const QueryRows& qr, const void* k, const void* v, co
     if (e != cudaSuccess) return e;
     const dim3 grid((qr.T + Sh::kTok - 1) / Sh::kTok, qr.B * qr.Hkv);
     return launch_pdl(kfn, grid, dim3(kThreads), (size_t)Sh::kSmemBytes, s, qr, tq, tk, tv, kr, idx, cnt, mc,
-                      dense_all ? 1 : 0, static_cast<__nv_bfloat16*>(out), lse);
+                      dense_all ? 1 : 0, static_cast<__nv_bfloat16*>(out), lse, test_first_wait_limit());
 }
 
 }  // namespace

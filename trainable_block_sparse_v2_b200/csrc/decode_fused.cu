@@ -790,6 +790,8 @@ int fused_set_first_wait_limit(unsigned polls)
     return 0;
 }
 
+unsigned test_first_wait_limit() { return g_first_wait_limit.load(std::memory_order_relaxed); }
+
 int fused_error_flag_read_and_clear()
 {
     int h = 0;

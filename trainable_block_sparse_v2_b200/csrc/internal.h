@@ -212,6 +212,7 @@ cudaError_t launch_decode_fused(const QueryRows& qr, const void* kern, int nk_ca
                                 float* lse, cudaStream_t s, bool pool_new = false);
 int fused_error_flag_read_and_clear();
 int fused_set_first_wait_limit(unsigned polls);  // testing only
+unsigned test_first_wait_limit();                // the value set (0: the normal waits)
 
 // attention split over the selected blocks across CTAs, merged by LSE (decode and tree verification)
 cudaError_t launch_attn_split(const QueryRows& qr, const void* k, const void* v, const KvRows& kr, const int32_t* idx,
