@@ -106,11 +106,12 @@ int infllmv2_device_status(void);
  * limit.  That drives the bounded-wait error path without a fault: the step's CTAs issue no further copy,
  * wait (bounded) for the copies in flight, still reach every cluster barrier, and infllmv2_device_status then
  * returns INFLLMV2_ERR_TIMEOUT; the step's outputs are not the method's.  The same limit applies to the
- * first wait of the thread that issues the score MMAs in every CTA of the tensor-core prefill attention
- * (infllmv2_sparse_attn_prefill, its paged and packed forms, on the tcgen05 path).  Its CTAs then stop their
- * loops; each producer waits (bounded) for the copies it issued, and each MMA issuer for its MMAs.  The CTAs
- * free their TMEM and exit, and infllmv2_device_status returns INFLLMV2_ERR_TIMEOUT.  polls = 0 restores the
- * normal waits.  The limit is process-wide and becomes a launch argument of every such kernel launched after
+ * first wait of the MMA-issuing thread in every CTA of the tensor-core prefill kernels: the attention
+ * (infllmv2_sparse_attn_prefill, its paged and packed forms) and the scoring with top-k
+ * (infllmv2_block_score_topk and its packed form), on their tcgen05 paths.  Their CTAs then stop their loops;
+ * each producer waits (bounded) for the copies it issued, and each MMA issuer for its MMAs.  The CTAs free
+ * their TMEM and exit, and infllmv2_device_status returns INFLLMV2_ERR_TIMEOUT; idx / cnt or the attention
+ * outputs of that call are not the method's.  polls = 0 restores the normal waits.  The limit is process-wide and becomes a launch argument of every such kernel launched after
  * this returns (a CUDA graph captured before keeps the value it captured).  Returns INFLLMV2_OK.
  */
 int infllmv2_test_set_first_wait_limit(unsigned polls);

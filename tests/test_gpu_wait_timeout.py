@@ -104,3 +104,45 @@ def test_prefill_attention_wait_that_runs_out_is_reported_and_the_next_call_is_c
     assert binding.infllmv2_device_status() == 0
     for a, b in zip(ref, again):
         assert torch.equal(a, b)
+
+
+def test_prefill_scoring_wait_that_runs_out_is_reported_and_the_next_call_is_clean():
+    """The same limit on the tensor-core prefill scoring (16 heads per group, d 128): its MMA issuer's first wait
+    runs out, the readers stop and still meet at their named barriers, the producer waits for its copies, and
+    the next call selects exactly the earlier blocks."""
+    from trainable_block_sparse_v2_b200.build import build
+    from trainable_block_sparse_v2_b200.workloads import prefill_case
+    build()
+    lib = binding.load()
+    T = 1500
+    w = prefill_case(T, 32, 2, 128, topk=5, dense_len=300, seed=1717, n_needles=2)
+    p = bparams(w.params)
+    q, K = dev(w.q), dev(w.k)
+    L = dev_i32(w.ctx_lens)
+    nk_cap = binding.num_kernels(T)
+    kern = torch.zeros((1, 2, nk_cap, 128), dtype=torch.bfloat16, device="cuda")
+    binding.infllmv2_kernel_pool(K, dev_i32(np.zeros(1)), L, T, p, kern)
+    ws = binding.workspace(p, 1, T, T, 32, 2, 128)
+
+    def select():
+        idx = torch.full((1, T, 2, p.kmax), -7, dtype=torch.int32, device="cuda")
+        cnt = torch.full((1, T, 2), -7, dtype=torch.int32, device="cuda")
+        binding.infllmv2_block_score_topk(q, None, L, T, kern, p, idx, cnt, ws)
+        torch.cuda.synchronize()
+        return idx, cnt
+
+    assert binding.infllmv2_device_status() == 0
+    ref = select()
+    assert binding.infllmv2_device_status() == 0
+    assert bool((ref[1] > 0).all())
+    assert lib.infllmv2_test_set_first_wait_limit(64) == 0
+    try:
+        select()  # must return: every wait is bounded
+        assert binding.infllmv2_device_status() == TIMEOUT
+        assert binding.infllmv2_device_status() == 0
+    finally:
+        assert lib.infllmv2_test_set_first_wait_limit(0) == 0
+    again = select()
+    assert binding.infllmv2_device_status() == 0
+    for a, b in zip(ref, again):
+        assert torch.equal(a, b)

@@ -170,6 +170,10 @@ def score_tc_model(m: PipelineModel, ntiles: int, mistake: str = "", parts: int 
                 yield ("wait", f"k_empty{s}", k - 1)
             yield ("arrive_tx", f"k_full{s}", 1, 1)
             yield ("tma", f"k_full{s}", 1, [(f"kern{s}", ("kern", q))])
+        # the producer's drain before the CTA ends: every copy it issued has landed
+        yield ("wait", "q_full", 0)
+        for s in range(min(RING, nq)):
+            yield ("wait", f"k_full{s}", (nq - 1 - s) // RING)
 
     def issuer():
         yield ("wait", "q_tmem", 0)

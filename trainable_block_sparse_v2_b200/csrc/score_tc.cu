@@ -64,13 +64,14 @@ struct SBars {
     uint64_t k_full[kSRing], k_empty[kSRing];
     uint64_t s_full[2], s_empty[2];  // per tile (A, B): accumulator ready / read back
     uint64_t drain;                  // the issuer's last MMAs
+    uint64_t never;                  // nothing arrives on it: the wait a test drives to run out
     uint32_t tmem_base;
     int err;
 };
 
-__device__ __forceinline__ bool swait(uint64_t* bar, uint32_t parity, volatile int* err)
+__device__ __forceinline__ bool swait(uint64_t* bar, uint32_t parity, volatile int* err, uint32_t limit = 1u << 22)
 {
-    for (uint32_t i = 0; i < (1u << 22); ++i) {
+    for (uint32_t i = 0; i < limit; ++i) {
         if (tc::mbar_try_wait(bar, parity)) return true;
         if ((i & 255u) == 255u && *err) return false;
     }
@@ -92,7 +93,7 @@ template <int KW>
 __global__ void __launch_bounds__(kSThreads, 1)
 score_tc_kernel(QueryRows qr, const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_kern,
                 const __grid_constant__ CUtensorMap tm_kern_s, int nk_cap, MethodConsts mc, int nb_max,
-                int32_t* __restrict__ idx, int32_t* __restrict__ cnt)
+                int32_t* __restrict__ idx, int32_t* __restrict__ cnt, unsigned test_wait_limit)
 {
     pdl_launch_dependents();
     pdl_wait();
@@ -148,6 +149,7 @@ score_tc_kernel(QueryRows qr, const __grid_constant__ CUtensorMap tm_q, const __
             tc::mbar_init(&bars.s_empty[i], kSEpiThreads);
         }
         tc::mbar_init(&bars.drain, 1);
+        tc::mbar_init(&bars.never, 1);
         tc::fence_barrier_init();
     }
     if (warp == 1) {
@@ -174,7 +176,8 @@ score_tc_kernel(QueryRows qr, const __grid_constant__ CUtensorMap tm_q, const __
                 tc::tma_load_3d(smem + kSQOff + 32768 * tile + 16384, &tm_q, 64, g * kSG, zq, &bars.q_full);
             }
             const int zk = b * qr.Hkv + g;
-            for (int q = 0; q < nq; ++q) {
+            int issued = 0;  // stages whose copies are in flight or landed
+            for (int q = 0; q < nq; ++q, ++issued) {
                 const int s = q % kSRing, k = q / kSRing;
                 if (k >= 1 && !swait(&bars.k_empty[s], (k - 1) & 1, err)) break;
                 unsigned char* st = smem + s * kSSlot;
@@ -185,10 +188,16 @@ score_tc_kernel(QueryRows qr, const __grid_constant__ CUtensorMap tm_q, const __
                 tc::tma_load_3d(st, map, 0, row0, zk, &bars.k_full[s]);
                 tc::tma_load_3d(st + 16384, map, 64, row0, zk, &bars.k_full[s]);
             }
+            // every copy this lane issued has landed before the CTA ends (on the normal path each one was
+            // waited for already); after a wait ran out, the rest of the CTA no longer waits for them
+            (void)tc::mbar_wait(&bars.q_full, 0, 1u << 22);
+            for (int s = 0; s < kSRing && s < issued; ++s)
+                (void)tc::mbar_wait(&bars.k_full[s], ((issued - 1 - s) / kSRing) & 1, 1u << 22);
         }
     } else if (warp == 1) {
         // ---------------- MMA issuer: S_A(q), S_B(q) = Q_A, Q_B . K(q)^T ----------------
-        if (lane == 0 && swait(&bars.q_tmem, 0, err)) {
+        // (with a test limit, the first wait polls a barrier nothing arrives on instead)
+        if (lane == 0 && (test_wait_limit ? swait(&bars.never, 0, err, test_wait_limit) : swait(&bars.q_tmem, 0, err))) {
             tc::tc_fence_after();
             constexpr uint32_t idesc = tc::idesc_bf16(128, 128, false);
             const uint32_t sbase = tc::smem_u32(smem);
@@ -406,7 +415,7 @@ static cudaError_t score_tc_launch(const CUtensorMap& tq, const CUtensorMap& tk,
     if (e != cudaSuccess) return e;
     const dim3 grid((qr.T + kSTok - 1) / kSTok, qr.B * qr.Hkv);
     return launch_pdl(score_tc_kernel<KW>, grid, dim3(kSThreads), (size_t)lay.bytes, s, qr, tq, tk, tks, nk_cap, mc,
-                      nb_max, idx, cnt);
+                      nb_max, idx, cnt, test_first_wait_limit());
 }
 
 cudaError_t launch_score_tc(const QueryRows& qr, const void* kern, int nk_cap, const MethodConsts& mc, int nb_max,
