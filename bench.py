@@ -43,11 +43,11 @@ HQ, HKV, D = 32, 2, 128
 # it stands (profiles/decode_fused_128k.md, profiles/prefill_32k.md); None where the kernels changed after
 # their capture (the two-call decode kernels took the paged / packed addressing since)
 NCU_TRAFFIC = {
-    "sparse_decode_step": 31_308_928,                   # decode_fused_kernel: 31.31 MB read, ~2 KB written
-    "sparse_decode_step_pool": 31_319_552,              # the same kernel pooling the new key's kernel
+    "sparse_decode_step": None,                         # decode_fused_kernel without pooling: not captured at this build
+    "sparse_decode_step_pool": 31_319_552,              # decode_fused_kernel pooling the new key's kernel
     "sparse_attn_decode": None,                         # attn_split_kernel + attn_merge_kernel
     "block_score_topk": None,                           # score_scan_kernel + score_select_kernel
-    "sparse_attn_prefill": 322_111_488 + 229_101_312,   # attn_tc_kernel<16, 128>
+    "sparse_attn_prefill": None,                        # attn_tc_kernel<16, 128>: changed since its capture
 }
 KERNELS_PER_STEP = {"two_call": 5,    # kernel pool, score scan, select, split attention, merge
                     "fused": 2,       # kernel pool, fused decode step (scoring + top-k + attention)
