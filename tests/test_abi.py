@@ -200,3 +200,11 @@ def test_noalloc_decode_refuses_what_the_workspace_decode_refuses(lib):
     assert both(binding.Params(topk=64), lse=A4 + 2) == (INVALID, INVALID)
     assert both(binding.Params(topk=64), batch=1 << 15, hkv=4) == (UNSUPPORTED, UNSUPPORTED)
     assert both(binding.Params(block_size=32)) == (UNSUPPORTED, UNSUPPORTED)
+
+
+def test_test_wait_limit_is_set_on_the_host(lib):
+    """infllmv2_test_set_first_wait_limit only stores the value that later launches take as an argument: it makes
+    no CUDA call, returns INFLLMV2_OK, and 0 restores the normal waits (the GPU side is in
+    tests/test_gpu_wait_timeout.py)."""
+    assert lib.infllmv2_test_set_first_wait_limit(64) == OK
+    assert lib.infllmv2_test_set_first_wait_limit(0) == OK
